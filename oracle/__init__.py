@@ -1,0 +1,171 @@
+"""fp64 CPU oracle for the weight-quantized matrix-vector product (qmv).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` leg of ``bench.py`` may import this
+package.  The CUDA library never loads it and shares no code with it.
+
+The arithmetic lives in ``qmv_oracle.c`` (plain C, fp64); this module only
+compiles it with gcc and marshals numpy arrays through ctypes.  Calls release
+the GIL, so a thread pool over row ranges runs them in parallel
+(``threads`` argument).
+
+Page citations for each function are in the C file: the MLX
+``quantized_nax.h`` source page (pack geometry, LSB-first codes,
+``w = scale * q + bias``), the wh-iron kernel-op coverage audit (Track 1 formats:
+E2M1, E4M3, E8M0, MXFP4, NVFP4, MXFP8) and the MLX pull request adding
+``affine_qmv_fast_rows`` (fp32-widened sum(x)).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "qmv_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F32, F16, BF16 = 0, 1, 2
+MXFP4, NVFP4, MXFP8 = 0, 1, 2
+DTYPE_CODES = {"f32": F32, "f16": F16, "bf16": BF16}
+FP_MODES = {"mxfp4": MXFP4, "nvfp4": NVFP4, "mxfp8": MXFP8}
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` next to its source with gcc (no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+             "-ffp-contract=off", _SRC, "-o", _LIB, "-lm"])
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        ll, i, p, d, f, u = (ctypes.c_longlong, ctypes.c_int, ctypes.c_void_p,
+                             ctypes.c_double, ctypes.c_float, ctypes.c_uint32)
+        L.oracle_f16_value.argtypes = [u]; L.oracle_f16_value.restype = d
+        L.oracle_bf16_value.argtypes = [u]; L.oracle_bf16_value.restype = d
+        L.oracle_pack_factor.argtypes = [i]; L.oracle_pack_factor.restype = i
+        L.oracle_bytes_per_pack.argtypes = [i]; L.oracle_bytes_per_pack.restype = i
+        L.oracle_row_bytes.argtypes = [ll, i]; L.oracle_row_bytes.restype = ll
+        L.oracle_affine_code.argtypes = [p, ll, i]; L.oracle_affine_code.restype = u
+        L.oracle_e2m1.argtypes = [u]; L.oracle_e2m1.restype = d
+        L.oracle_e4m3.argtypes = [u]; L.oracle_e4m3.restype = d
+        L.oracle_e8m0.argtypes = [u]; L.oracle_e8m0.restype = d
+        L.oracle_round_f32_sum.argtypes = [d, d]; L.oracle_round_f32_sum.restype = f
+        L.oracle_dequant_affine_f32.argtypes = [p, p, p, p, ll, ll, i, i, i, ll, ll]
+        L.oracle_dequant_affine_f32.restype = None
+        L.oracle_dequant_fp_f32.argtypes = [p, p, f, p, ll, ll, i, ll, ll]
+        L.oracle_dequant_fp_f32.restype = None
+        L.oracle_qmv_affine.argtypes = [p, p, p, p, p, p, ll, ll, ll, i, i, i, ll, ll]
+        L.oracle_qmv_affine.restype = None
+        L.oracle_qmv_fp.argtypes = [p, p, p, f, p, p, ll, ll, ll, i, i, ll, ll]
+        L.oracle_qmv_fp.restype = None
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return a.ctypes.data
+
+
+def _ranges(rows, threads):
+    """Split a row list/range into contiguous (n0, n1) runs, then into chunks."""
+    rows = list(rows)
+    runs, start = [], None
+    for i, r in enumerate(rows):
+        if start is None:
+            start, prev = r, r
+        elif r == prev + 1:
+            prev = r
+        else:
+            runs.append((start, prev + 1)); start, prev = r, r
+    if start is not None:
+        runs.append((start, prev + 1))
+    out = []
+    for a, b in runs:
+        step = max(1, (b - a + threads - 1) // threads)
+        out += [(s, min(b, s + step)) for s in range(a, b, step)]
+    return out
+
+
+def _run(fn, ranges, threads):
+    if threads <= 1 or len(ranges) <= 1:
+        for a, b in ranges:
+            fn(a, b)
+        return
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(lambda r: fn(*r), ranges))
+
+
+# ---- scalar codecs (pinned in tests/test_oracle_pins.py) -------------------
+def f16_value(h): return lib().oracle_f16_value(int(h))
+def bf16_value(h): return lib().oracle_bf16_value(int(h))
+def pack_factor(bits): return lib().oracle_pack_factor(bits)
+def bytes_per_pack(bits): return lib().oracle_bytes_per_pack(bits)
+def row_bytes(K, bits): return lib().oracle_row_bytes(K, bits)
+def e2m1(c): return lib().oracle_e2m1(int(c))
+def e4m3(c): return lib().oracle_e4m3(int(c))
+def e8m0(e): return lib().oracle_e8m0(int(e))
+def round_f32_sum(a, b): return lib().oracle_round_f32_sum(float(a), float(b))
+
+
+def affine_codes(row: np.ndarray, K: int, bits: int) -> np.ndarray:
+    """All K codes of one packed row (uint8 array)."""
+    row = np.ascontiguousarray(row, dtype=np.uint8)
+    L = lib()
+    return np.array([L.oracle_affine_code(_ptr(row), k, bits) for k in range(K)], dtype=np.uint32)
+
+
+# ---- dequantization (fp32 out) ----------------------------------------------
+def dequant_affine_f32(w, scales, biases, N, K, bits, group, dtype, rows=None, threads=1):
+    out = np.zeros((N, K), dtype=np.float32)
+    L = lib()
+    fn = lambda a, b: L.oracle_dequant_affine_f32(_ptr(w), _ptr(scales), _ptr(biases), _ptr(out),
+                                                  N, K, bits, group, DTYPE_CODES[dtype], a, b)
+    _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
+    return out
+
+
+def dequant_fp_f32(w, scales, global_scale, N, K, mode, rows=None, threads=1):
+    out = np.zeros((N, K), dtype=np.float32)
+    L = lib()
+    g = float(global_scale) if global_scale is not None else 1.0
+    fn = lambda a, b: L.oracle_dequant_fp_f32(_ptr(w), _ptr(scales), g, _ptr(out), N, K,
+                                              FP_MODES[mode], a, b)
+    _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
+    return out
+
+
+# ---- the product --------------------------------------------------------------
+def qmv_affine(x, w, scales, biases, M, N, K, bits, group, dtype, rows=None, threads=1):
+    """Return (y, absdot), both float64 [M, N]; rows not requested stay NaN."""
+    y = np.full((M, N), np.nan); a = np.full((M, N), np.nan)
+    L = lib()
+    fn = lambda r0, r1: L.oracle_qmv_affine(_ptr(x), _ptr(w), _ptr(scales), _ptr(biases), _ptr(y),
+                                            _ptr(a), M, N, K, bits, group, DTYPE_CODES[dtype], r0, r1)
+    _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
+    return y, a
+
+
+def qmv_fp(x, w, scales, global_scale, M, N, K, mode, dtype, rows=None, threads=1):
+    y = np.full((M, N), np.nan); a = np.full((M, N), np.nan)
+    L = lib()
+    g = float(global_scale) if global_scale is not None else 1.0
+    fn = lambda r0, r1: L.oracle_qmv_fp(_ptr(x), _ptr(w), _ptr(scales), g, _ptr(y), _ptr(a),
+                                        M, N, K, FP_MODES[mode], DTYPE_CODES[dtype], r0, r1)
+    _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
+    return y, a

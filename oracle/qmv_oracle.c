@@ -1,0 +1,244 @@
+/*
+ * qmv_oracle.c -- plain, slow fp64 CPU oracle for the weight-quantized
+ * matrix-vector product  y[m,n] = sum_k x[m,k] * dequant(W)[n,k].
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * load this file: it is used by tests/, by __graft_entry__.smoke() and by the
+ * cpu_baseline / reference leg of bench.py, nowhere else.  It shares no code,
+ * header, table or constant with the CUDA library: every decoder below is
+ * written from the format definitions on the pages it cites.
+ *
+ * Sources (page title, section):
+ *  - MLX "quantized_nax.h" (mlx 1.0.0 source page), functions get_pack_factor,
+ *    get_bytes_per_pack, qdot, dequantize: affine pack geometry, LSB-first
+ *    code order inside a pack, and w = scale * q + bias.
+ *  - "wh-iron kernel-op coverage audit", section "Quantization precision
+ *    coverage", Track 1 table and the E2M1 / E4M3 / E8M0 codec notes:
+ *    MXFP4 = E2M1 x E8M0 per 32, NVFP4 = E2M1 x E4M3 per 16 x FP32 global,
+ *    MXFP8 = E4M3 x E8M0 per 32; E4M3 has 3 mantissa bits, exponent bias 7,
+ *    max 448 and an explicit NaN code.
+ *  - MLX pull request "affine_qmv_fast_rows / fp_qmv_fast_rows", description:
+ *    the sum(x) bias term is formed from values widened before accumulation.
+ *    The oracle has no such issue: it evaluates every product and sum in fp64.
+ *
+ * Every function is a direct statement of a definition; there is no blocking,
+ * fusion or reordering.  Parity status of each function is listed in the
+ * tests that pin it (tests/test_oracle_pins.py); every exported function here
+ * is pinned there, none is "parity unpinned".
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#include <stddef.h>
+
+/* dtype codes used on the oracle's own ctypes boundary */
+enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2 };
+/* FP weight modes */
+enum { OR_MXFP4 = 0, OR_NVFP4 = 1, OR_MXFP8 = 2 };
+
+/* ---------------------------------------------------------------------------
+ * Element types of x, y, scales and biases, widened exactly to fp64.
+ * binary16 and bfloat16 are decoded from their IEEE-style field definitions.
+ * ------------------------------------------------------------------------- */
+double oracle_f16_value(uint32_t h) {
+    uint32_t s = (h >> 15) & 1u, e = (h >> 10) & 31u, m = h & 1023u;
+    double v;
+    if (e == 0) v = ldexp((double)m, -24);                 /* subnormal: m * 2^-24 */
+    else if (e == 31) v = (m == 0) ? INFINITY : NAN;
+    else v = ldexp(1.0 + (double)m / 1024.0, (int)e - 15);
+    return s ? -v : v;
+}
+
+double oracle_bf16_value(uint32_t h) {
+    uint32_t s = (h >> 15) & 1u, e = (h >> 7) & 255u, m = h & 127u;
+    double v;
+    if (e == 0) v = ldexp((double)m, -133);                /* subnormal: m * 2^-133 */
+    else if (e == 255) v = (m == 0) ? INFINITY : NAN;
+    else v = ldexp(1.0 + (double)m / 128.0, (int)e - 127);
+    return s ? -v : v;
+}
+
+static double load_elem(const void* p, size_t i, int dtype) {
+    if (dtype == OR_F32) { float f; memcpy(&f, (const char*)p + 4 * i, 4); return (double)f; }
+    uint16_t h; memcpy(&h, (const char*)p + 2 * i, 2);
+    return dtype == OR_F16 ? oracle_f16_value(h) : oracle_bf16_value(h);
+}
+
+/* ---------------------------------------------------------------------------
+ * Affine pack geometry (MLX quantized_nax.h, get_pack_factor /
+ * get_bytes_per_pack with an 8-bit word): 3- and 5-bit codes come 8 to a pack
+ * of 3 or 5 bytes, 6-bit codes 4 to a pack of 3 bytes, and 2/4/8-bit codes
+ * 8/bits to a single byte.
+ * ------------------------------------------------------------------------- */
+int oracle_pack_factor(int bits) {
+    if (bits == 3 || bits == 5) return 8;
+    if (bits == 6) return 4;
+    return 8 / bits;
+}
+
+int oracle_bytes_per_pack(int bits) {
+    if ((bits & (bits - 1)) == 0) return 1;
+    return bits == 5 ? 5 : 3;
+}
+
+/* Row byte length K_w = K * bytes_per_pack / pack_factor (= K * bits / 8). */
+long long oracle_row_bytes(long long K, int bits) {
+    return K * oracle_bytes_per_pack(bits) / oracle_pack_factor(bits);
+}
+
+/* Code i of a packed row.  Inside a pack the codes are read least significant
+ * bit first: with the pack's bytes taken as one little-endian integer, code j
+ * of the pack occupies bits [bits*j, bits*j + bits).  This single reading is
+ * what the masks of MLX's qdot / dequantize select for every width. */
+uint32_t oracle_affine_code(const uint8_t* row, long long i, int bits) {
+    int pf = oracle_pack_factor(bits), bpp = oracle_bytes_per_pack(bits);
+    long long p = i / pf;
+    int j = (int)(i % pf);
+    uint64_t v = 0;
+    for (int b = 0; b < bpp; ++b) v |= (uint64_t)row[p * bpp + b] << (8 * b);
+    return (uint32_t)((v >> (bits * j)) & ((1u << bits) - 1u));
+}
+
+/* ---------------------------------------------------------------------------
+ * Micro-float codecs (wh-iron audit, Track 1 and the codec notes).
+ * ------------------------------------------------------------------------- */
+/* E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit, no inf/NaN. */
+double oracle_e2m1(uint32_t c) {
+    uint32_t s = (c >> 3) & 1u, e = (c >> 1) & 3u, m = c & 1u;
+    double v = (e == 0) ? 0.5 * (double)m : ldexp(1.0 + 0.5 * (double)m, (int)e - 1);
+    return s ? -v : v;
+}
+
+/* E4M3 (OCP "FN" flavour): sign, 4 exponent bits (bias 7), 3 mantissa bits;
+ * exponent field 0 is subnormal; S.1111.111 is NaN; no infinities. */
+double oracle_e4m3(uint32_t c) {
+    uint32_t s = (c >> 7) & 1u, e = (c >> 3) & 15u, m = c & 7u;
+    double v;
+    if ((c & 0x7Fu) == 0x7Fu) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, (int)e - 7);
+    return s ? -v : v;
+}
+
+/* E8M0: an unsigned power-of-two exponent byte, 2^(e - 127); 0xFF is NaN. */
+double oracle_e8m0(uint32_t e) {
+    if ((e & 0xFFu) == 0xFFu) return NAN;
+    return ldexp(1.0, (int)(e & 0xFFu) - 127);
+}
+
+/* ---------------------------------------------------------------------------
+ * One correctly rounded fp32 value of the exact sum a + b (a, b exact fp64).
+ * The fp64 sum is first rounded to odd (TwoSum gives its exact error), which
+ * makes the following fp64 -> fp32 conversion a single correct rounding
+ * (53 >= 24 + 2 bits).  Used for the dequantized fp32 weight
+ * round_f32(scale * q + bias).
+ * ------------------------------------------------------------------------- */
+float oracle_round_f32_sum(double a, double b) {
+    double s = a + b;
+    double bb = s - a;
+    double err = (a - (s - bb)) + (b - bb);            /* exact: a + b = s + err */
+    if (err != 0.0 && isfinite(s)) {
+        uint64_t u; memcpy(&u, &s, 8);
+        if ((u & 1u) == 0) {                               /* even: step toward err */
+            s = nextafter(s, err > 0 ? INFINITY : -INFINITY);
+        }
+    }
+    return (float)s;
+}
+
+/* Exact dequantized affine weight (fp64) of element (n, k). */
+static double affine_w(const uint8_t* w, const void* scales, const void* biases,
+                       long long n, long long k, long long K, int bits, int group, int dtype) {
+    const uint8_t* row = w + n * oracle_row_bytes(K, bits);
+    long long gi = n * (K / group) + k / group;
+    double s = load_elem(scales, (size_t)gi, dtype);
+    double b = load_elem(biases, (size_t)gi, dtype);
+    return s * (double)oracle_affine_code(row, k, bits) + b;
+}
+
+/* fp32 dequantized affine weights, out[n*K + k] = round_f32(scale*q + bias),
+ * rows [n0, n1). */
+void oracle_dequant_affine_f32(const uint8_t* w, const void* scales, const void* biases,
+                               float* out, long long N, long long K, int bits, int group,
+                               int dtype, long long n0, long long n1) {
+    (void)N;
+    for (long long n = n0; n < n1; ++n) {
+        const uint8_t* row = w + n * oracle_row_bytes(K, bits);
+        for (long long k = 0; k < K; ++k) {
+            long long gi = n * (K / group) + k / group;
+            double s = load_elem(scales, (size_t)gi, dtype);
+            double b = load_elem(biases, (size_t)gi, dtype);
+            double sq = s * (double)oracle_affine_code(row, k, bits); /* exact: <= 32 bits */
+            out[n * K + k] = oracle_round_f32_sum(sq, b);
+        }
+    }
+}
+
+/* Block size along K and per-element width of each FP mode. */
+static int fp_block(int mode) { return mode == OR_NVFP4 ? 16 : 32; }
+static int fp_bits(int mode) { return mode == OR_MXFP8 ? 8 : 4; }
+
+/* Exact dequantized FP weight (fp64) of element (n, k).  Codes are 4-bit
+ * (two per byte, even k in the low nibble) or one byte each; one scale byte
+ * per block; NVFP4 multiplies by the tensor-wide fp32 global scale. */
+static double fp_w(const uint8_t* w, const uint8_t* scales, double global,
+                   long long n, long long k, long long K, int mode) {
+    int bits = fp_bits(mode), blk = fp_block(mode);
+    const uint8_t* row = w + n * (K * bits / 8);
+    uint32_t code = (bits == 8) ? row[k] : ((row[k / 2] >> (4 * (k % 2))) & 0xFu);
+    uint32_t sc = scales[n * (K / blk) + k / blk];
+    double e = (bits == 8) ? oracle_e4m3(code) : oracle_e2m1(code);
+    if (mode == OR_NVFP4) return e * oracle_e4m3(sc) * global;
+    return e * oracle_e8m0(sc);
+}
+
+/* fp32 dequantized FP weights; every product is exact in fp64 (at most 30
+ * significant bits), so the cast is the one rounding. */
+void oracle_dequant_fp_f32(const uint8_t* w, const uint8_t* scales, float global,
+                           float* out, long long N, long long K, int mode,
+                           long long n0, long long n1) {
+    (void)N;
+    for (long long n = n0; n < n1; ++n)
+        for (long long k = 0; k < K; ++k)
+            out[n * K + k] = (float)fp_w(w, scales, (double)global, n, k, K, mode);
+}
+
+/* ---------------------------------------------------------------------------
+ * The product itself: y[m*N + n] = sum_k x[m,k] * w_hat[n,k] in fp64, plus
+ * absdot[m*N + n] = sum_k |x[m,k] * w_hat[n,k]| (the size of the terms, used
+ * by the tests' cancellation-aware tolerance).  Rows [n0, n1) only, so the
+ * caller can sample rows or split them over threads.
+ * ------------------------------------------------------------------------- */
+void oracle_qmv_affine(const void* x, const uint8_t* w, const void* scales, const void* biases,
+                       double* y, double* absdot, long long M, long long N, long long K,
+                       int bits, int group, int dtype, long long n0, long long n1) {
+    for (long long n = n0; n < n1; ++n)
+        for (long long m = 0; m < M; ++m) {
+            double acc = 0.0, aacc = 0.0;
+            for (long long k = 0; k < K; ++k) {
+                double t = load_elem(x, (size_t)(m * K + k), dtype) *
+                           affine_w(w, scales, biases, n, k, K, bits, group, dtype);
+                acc += t;
+                aacc += fabs(t);
+            }
+            y[m * N + n] = acc;
+            if (absdot) absdot[m * N + n] = aacc;
+        }
+}
+
+void oracle_qmv_fp(const void* x, const uint8_t* w, const uint8_t* scales, float global,
+                   double* y, double* absdot, long long M, long long N, long long K,
+                   int mode, int dtype, long long n0, long long n1) {
+    for (long long n = n0; n < n1; ++n)
+        for (long long m = 0; m < M; ++m) {
+            double acc = 0.0, aacc = 0.0;
+            for (long long k = 0; k < K; ++k) {
+                double t = load_elem(x, (size_t)(m * K + k), dtype) *
+                           fp_w(w, scales, (double)global, n, k, K, mode);
+                acc += t;
+                aacc += fabs(t);
+            }
+            y[m * N + n] = acc;
+            if (absdot) absdot[m * N + n] = aacc;
+        }
+}

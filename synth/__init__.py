@@ -1,0 +1,100 @@
+"""Seeded synthetic inputs for the qmv tests and benchmark.
+
+This module is shared by the oracle side and the CUDA side, so it holds none
+of the method's arithmetic: it draws random numbers, rounds them to the storage
+dtype with a plain cast, and returns raw bytes.  Packed weights are uniform
+random BYTES, which makes every code of every width uniform over its full range
+(2/3/4/5/6/8-bit affine codes and the 16 E2M1 codes alike); E4M3 codes are
+drawn from the 254 non-NaN byte values.  Nothing here unpacks, decodes or
+multiplies anything.
+
+Distributions (from the workload descriptions the tests and bench cover):
+  affine:  x ~ N(0, 1), scales ~ U(0.005, 0.02), biases ~ N(0, 0.01), all
+           rounded to the dtype; the precision case draws x ~ U(1e-4, 1e-3) and
+           uses the symmetric zero point bias = -scale * (2^bits - 1) / 2 that a
+           min/max quantizer gives for zero-mean weights.
+  FP:      E8M0 block exponents ~ U{118..130}; NVFP4 block scales are positive,
+           non-zero, non-NaN E4M3 bytes (0x01..0x7E); NVFP4 global ~ U(0.5, 2).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+_TORCH = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
+
+
+def rng(seed: int) -> np.random.Generator:
+    """Counter-based generator (Philox) so any seed is reproducible anywhere."""
+    return np.random.Generator(np.random.Philox(seed))
+
+
+def to_storage(values: np.ndarray, dtype: str) -> np.ndarray:
+    """Round float values to ``dtype`` (a plain cast) and return the raw storage:
+    float32 for f32, uint16 bit patterns for f16 / bf16."""
+    t = torch.from_numpy(np.ascontiguousarray(values, dtype=np.float32)).to(_TORCH[dtype])
+    if dtype == "f32":
+        return t.numpy().copy()
+    return t.view(torch.int16).numpy().view(np.uint16).copy()
+
+
+def storage_to_float(raw: np.ndarray, dtype: str) -> np.ndarray:
+    """Raw storage back to float32 values (a plain widening cast)."""
+    if dtype == "f32":
+        return raw.astype(np.float32)
+    t = torch.from_numpy(raw.view(np.int16).copy()).view(_TORCH[dtype])
+    return t.to(torch.float32).numpy()
+
+
+def random_bytes(g: np.random.Generator, shape) -> np.ndarray:
+    return g.integers(0, 256, size=shape, dtype=np.uint8)
+
+
+def affine_case(M, N, K, bits, group, dtype, seed, batch=1, precision=False):
+    """One affine problem.  Shapes: x [batch, M, K], w [batch, N, K*bits/8] u8,
+    scales / biases [batch, N, K/group]; x, scales and biases are raw storage
+    of ``dtype``."""
+    g = rng(seed)
+    if precision:
+        x = g.uniform(1e-4, 1e-3, size=(batch, M, K))
+    else:
+        x = g.standard_normal(size=(batch, M, K))
+    w = random_bytes(g, (batch, N, K * bits // 8))
+    s = g.uniform(0.005, 0.02, size=(batch, N, K // group))
+    s_raw = to_storage(s, dtype)
+    if precision:
+        b = -storage_to_float(s_raw, dtype).astype(np.float64) * ((2 ** bits - 1) / 2.0)
+    else:
+        b = g.normal(0.0, 0.01, size=(batch, N, K // group))
+    return {
+        "x": to_storage(x, dtype), "w": w, "scales": s_raw, "biases": to_storage(b, dtype),
+        "M": M, "N": N, "K": K, "bits": bits, "group": group, "dtype": dtype, "batch": batch,
+    }
+
+
+FP_BLOCK = {"mxfp4": 32, "nvfp4": 16, "mxfp8": 32}
+FP_BITS = {"mxfp4": 4, "nvfp4": 4, "mxfp8": 8}
+_E4M3_NON_NAN = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+
+
+def fp_case(M, N, K, mode, dtype, seed, batch=1):
+    """One block-scaled FP problem.  w [batch, N, K*bits/8] u8 codes, scales
+    [batch, N, K/block] u8, global (NVFP4 only) a float32 scalar."""
+    g = rng(seed)
+    x = g.standard_normal(size=(batch, M, K))
+    bits, blk = FP_BITS[mode], FP_BLOCK[mode]
+    if bits == 4:
+        w = random_bytes(g, (batch, N, K // 2))
+    else:
+        w = _E4M3_NON_NAN[g.integers(0, len(_E4M3_NON_NAN), size=(batch, N, K))]
+    if mode == "nvfp4":
+        sc = g.integers(0x01, 0x7F, size=(batch, N, K // blk), dtype=np.uint8)
+        glob = np.float32(g.uniform(0.5, 2.0))
+    else:
+        sc = g.integers(118, 131, size=(batch, N, K // blk), dtype=np.uint8)
+        glob = None
+    return {
+        "x": to_storage(x, dtype), "w": np.ascontiguousarray(w, dtype=np.uint8), "scales": sc,
+        "global": glob, "M": M, "N": N, "K": K, "mode": mode, "dtype": dtype, "batch": batch,
+    }

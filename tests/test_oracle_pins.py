@@ -1,0 +1,379 @@
+"""Pins of the fp64 oracle to things other than itself (CPU only).
+
+Each test ties one oracle function to a value printed on the pages, a hand-worked
+example, a library routine, a closed form, an invariant or exact rational brute
+force, so that a dropped term, wrong sign, wrong index or transposed operand in
+the oracle fails at least one of them:
+
+  codecs           E2M1 hand table (all 16 codes), E4M3 all 256 bytes vs torch's
+                   float8_e4m3fn + spot values, E8M0 spot values, binary16 /
+                   bfloat16 decoders vs numpy / torch for every bit pattern;
+  affine unpack    pack geometry, hand-packed rows for every width, and the
+                   single-bit bijection invariant of the LSB-first reading;
+  dequantization   min/max quantize -> pack -> dequantize round trip; fp32
+                   rounding vs exact rationals (round-to-odd sum);
+  product          exact Fraction brute force on tiny shapes (affine and FP),
+                   the all-zero-code closed form, x = e_k selects a column;
+  sum(x)           the emulated low-precision sum(x) mutant fails the test
+                   tolerance on the precision case, the widened sum passes.
+"""
+from __future__ import annotations
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from qmv_tol import check
+
+GOLD = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _read_pairs(name):
+    rows = []
+    for line in open(os.path.join(GOLD, name)):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        a, b = line.split()
+        rows.append((int(a, 0), float(b)))
+    return rows
+
+
+def _same(a, b):
+    if math.isnan(b):
+        return math.isnan(a)
+    return a == b and math.copysign(1.0, a) == math.copysign(1.0, b)
+
+
+# ---------------------------------------------------------------- codecs ----
+def test_e2m1_hand_table():
+    rows = _read_pairs("e2m1_values.txt")
+    assert len(rows) == 16
+    for c, v in rows:
+        assert _same(oracle.e2m1(c), v), (c, oracle.e2m1(c), v)
+
+
+def test_e4m3_all_bytes_vs_torch():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for c in range(256):
+        assert _same(oracle.e4m3(c), float(ref[c])), (hex(c), oracle.e4m3(c), ref[c])
+
+
+def test_e4m3_spot_values():
+    for c, v in _read_pairs("e4m3_spot.txt"):
+        assert _same(oracle.e4m3(c), v), (hex(c), oracle.e4m3(c), v)
+
+
+def test_e8m0_spot_values():
+    for e, v in _read_pairs("e8m0_spot.txt"):
+        assert _same(oracle.e8m0(e), v), (e, oracle.e8m0(e), v)
+
+
+def test_e8m0_vs_torch_if_available():
+    if not hasattr(torch, "float8_e8m0fnu"):
+        pytest.skip("torch has no float8_e8m0fnu")
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    for e in range(256):
+        assert _same(oracle.e8m0(e), float(ref[e])), (e, oracle.e8m0(e), ref[e])
+
+
+def test_f16_decoder_every_pattern():
+    pats = np.arange(65536, dtype=np.uint32)
+    ref = pats.astype(np.uint16).view(np.float16).astype(np.float64)
+    got = np.array([oracle.f16_value(int(p)) for p in pats])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    m = ~np.isnan(ref)
+    assert np.array_equal(got[m], ref[m])
+    assert np.array_equal(np.signbit(got[m]), np.signbit(ref[m]))
+
+
+def test_bf16_decoder_every_pattern():
+    pats = torch.arange(65536, dtype=torch.int32).to(torch.int16)
+    ref = pats.view(torch.bfloat16).to(torch.float64).numpy()
+    got = np.array([oracle.bf16_value(p & 0xFFFF) for p in range(65536)])
+    got = got[np.arange(65536).astype(np.int16).astype(np.int64) & 0xFFFF]
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    m = ~np.isnan(ref)
+    assert np.array_equal(got[m], ref[m])
+
+
+# --------------------------------------------------------- affine unpack ----
+def test_pack_geometry():
+    # get_pack_factor / get_bytes_per_pack with an 8-bit word (MLX quantized_nax.h)
+    expect = {2: (4, 1), 3: (8, 3), 4: (2, 1), 5: (8, 5), 6: (4, 3), 8: (1, 1)}
+    for bits, (pf, bpp) in expect.items():
+        assert oracle.pack_factor(bits) == pf
+        assert oracle.bytes_per_pack(bits) == bpp
+        for K in (32, 64, 128, 512, 2560, 4096):
+            assert oracle.row_bytes(K, bits) * 8 == K * bits
+
+
+def _golden_packs():
+    out = []
+    for line in open(os.path.join(GOLD, "affine_packs.txt")):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        b, codes, by = (s.strip() for s in line.split("|"))
+        out.append((int(b), [int(c) for c in codes.split()], bytes.fromhex(by.replace(" ", ""))))
+    return out
+
+
+@pytest.mark.parametrize("bits,codes,packed", _golden_packs())
+def test_affine_hand_packed_rows(bits, codes, packed):
+    row = np.frombuffer(packed, dtype=np.uint8)
+    assert len(codes) * bits == 8 * len(packed)
+    got = oracle.affine_codes(row, len(codes), bits)
+    assert list(got) == codes
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+def test_affine_single_bit_bijection(bits):
+    """Setting bit t of an all-zero row (bits counted LSB-first through the
+    bytes) must set exactly code t // bits to 2^(t % bits)."""
+    nbytes = 15 if bits in (3, 5) else 6           # whole packs
+    K = nbytes * 8 // bits
+    for t in range(nbytes * 8):
+        row = np.zeros(nbytes, dtype=np.uint8)
+        row[t // 8] = 1 << (t % 8)
+        got = oracle.affine_codes(row, K, bits)
+        want = np.zeros(K, dtype=np.uint32)
+        want[t // bits] = 1 << (t % bits)
+        assert np.array_equal(got, want), (bits, t, got, want)
+
+
+# ------------------------------------------------------------ helpers -------
+def _py_pack(codes, bits):
+    """Test-side packer: a plain LSB-first bit stream writer."""
+    v = 0
+    for i, c in enumerate(codes):
+        assert 0 <= c < (1 << bits)
+        v |= int(c) << (bits * i)
+    n = len(codes) * bits // 8
+    return np.frombuffer(v.to_bytes(n, "little"), dtype=np.uint8).copy()
+
+
+def _py_codes(row, K, bits):
+    v = int.from_bytes(bytes(row), "little")
+    return [(v >> (bits * i)) & ((1 << bits) - 1) for i in range(K)]
+
+
+def _val(raw, dtype):
+    """Exact values of raw storage via library casts (numpy / torch)."""
+    return synth.storage_to_float(np.asarray(raw), dtype).astype(np.float64)
+
+
+def _f32_round(fr: Fraction) -> float:
+    """Correctly rounded (nearest, ties to even) float32 of an exact rational."""
+    f = np.float32(float(fr))
+    cands = [f, np.nextafter(f, np.float32(np.inf)), np.nextafter(f, np.float32(-np.inf))]
+    best = None
+    for c in cands:
+        if not np.isfinite(c):
+            continue
+        d = abs(Fraction(float(c)) - fr)
+        key = (d, int(np.float32(c).view(np.uint32)) & 1)
+        if best is None or key < best[0]:
+            best = (key, c)
+    return float(best[1])
+
+
+# ---------------------------------------------------------- dequant pins ----
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_minmax_roundtrip(bits, dtype):
+    """Host min/max quantizer (scale = (max - min) / (2^b - 1), bias = min,
+    q = round((w - bias) / scale)), test-side packer, then the oracle's
+    dequantization: |w - w_hat| <= scale / 2 (+ dtype rounding of scale/bias)
+    and the codes come back exactly from w_hat."""
+    g = np.random.default_rng(bits)
+    N, K, group = 3, 128, 32
+    w = g.standard_normal((N, K))
+    qmax = (1 << bits) - 1
+    codes = np.zeros((N, K), dtype=np.int64)
+    s_vals = np.zeros((N, K // group)); b_vals = np.zeros((N, K // group))
+    for n in range(N):
+        for j in range(K // group):
+            blk = w[n, j * group:(j + 1) * group]
+            lo, hi = blk.min(), blk.max()
+            s_vals[n, j], b_vals[n, j] = (hi - lo) / qmax, lo
+    s_raw = synth.to_storage(s_vals, dtype); b_raw = synth.to_storage(b_vals, dtype)
+    s_q, b_q = _val(s_raw, dtype), _val(b_raw, dtype)
+    for n in range(N):
+        for k in range(K):
+            j = k // group
+            codes[n, k] = min(qmax, max(0, round((w[n, k] - b_q[n, j]) / s_q[n, j])))
+    packed = np.stack([_py_pack(codes[n], bits) for n in range(N)])
+    w_hat = oracle.dequant_affine_f32(packed, s_raw, b_raw, N, K, bits, group, dtype)
+    for n in range(N):
+        for k in range(K):
+            j = k // group
+            # exact dequant of the stored code, rounded once to fp32
+            assert w_hat[n, k] == _f32_round(Fraction(s_q[n, j]) * int(codes[n, k]) + Fraction(b_q[n, j]))
+            back = round((float(w_hat[n, k]) - b_q[n, j]) / s_q[n, j])
+            assert back == codes[n, k]
+    err = np.abs(w - w_hat.astype(np.float64))
+    tol = np.repeat(s_q, group, axis=1) * 0.5 + np.abs(w) * 2.0 ** -7 + 1e-6
+    # bf16 rounding of the min/max moves the grid a little; clamped ends may add one step
+    tol += np.repeat(s_q, group, axis=1) * (1.0 if dtype == "bf16" else 1e-6)
+    assert (err <= tol).all()
+
+
+def test_round_f32_sum_exact():
+    g = np.random.default_rng(7)
+    cases = []
+    for _ in range(2000):
+        a = float(np.float32(g.standard_normal()) * np.float32(g.integers(0, 256)))
+        b = float(np.float32(g.standard_normal() * 10.0 ** g.integers(-30, 4)))
+        cases.append((a, b))
+    # adversarial: the fp64 sum rounds to an exact fp32 tie
+    one = 1.0
+    cases += [(one + 2.0 ** -24, 2.0 ** -80), (one + 2.0 ** -24, -2.0 ** -80),
+              (one + 3 * 2.0 ** -24, 2.0 ** -79), (-(one + 2.0 ** -24), -2.0 ** -80)]
+    for a, b in cases:
+        want = _f32_round(Fraction(a) + Fraction(b))
+        got = oracle.round_f32_sum(a, b)
+        assert got == want, (a, b, got, want)
+
+
+@pytest.mark.parametrize("mode", ["mxfp4", "nvfp4", "mxfp8"])
+def test_fp_dequant_exact(mode):
+    c = synth.fp_case(1, 4, 64, mode, "bf16", seed=11)
+    w, sc = c["w"][0], c["scales"][0]
+    glob = c["global"]
+    out = oracle.dequant_fp_f32(w, sc, glob, 4, 64, mode)
+    e2m1 = {cc: v for cc, v in _read_pairs("e2m1_values.txt")}
+    e4 = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    blk = synth.FP_BLOCK[mode]
+    for n in range(4):
+        for k in range(64):
+            if mode == "mxfp8":
+                e = Fraction(float(e4[w[n, k]]))
+            else:
+                e = Fraction(e2m1[(int(w[n, k // 2]) >> (4 * (k % 2))) & 0xF])
+            s = int(sc[n, k // blk])
+            if mode == "nvfp4":
+                want = _f32_round(e * Fraction(float(e4[s])) * Fraction(float(glob)))
+            else:
+                want = _f32_round(e * Fraction(2) ** (s - 127))
+            assert out[n, k] == want, (mode, n, k, out[n, k], want)
+
+
+# ---------------------------------------------------------- product pins ----
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("group", [32, 64])
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+def test_affine_dot_exact_bruteforce(bits, group, dtype):
+    M, N, K = 2, 3, 2 * group
+    c = synth.affine_case(M, N, K, bits, group, dtype, seed=bits * 100 + group)
+    x, w, s, b = c["x"][0], c["w"][0], c["scales"][0], c["biases"][0]
+    y, absdot = oracle.qmv_affine(x, w, s, b, M, N, K, bits, group, dtype)
+    xv, sv, bv = _val(x, dtype), _val(s, dtype), _val(b, dtype)
+    for n in range(N):
+        codes = _py_codes(w[n], K, bits)
+        for m in range(M):
+            acc = Fraction(0); aacc = Fraction(0)
+            for k in range(K):
+                j = k // group
+                t = Fraction(xv[m, k]) * (Fraction(sv[n, j]) * codes[k] + Fraction(bv[n, j]))
+                acc += t; aacc += abs(t)
+            assert abs(Fraction(y[m, n]) - acc) <= aacc * Fraction(2) ** -40
+            assert abs(Fraction(absdot[m, n]) - aacc) <= aacc * Fraction(2) ** -40
+
+
+@pytest.mark.parametrize("mode", ["mxfp4", "nvfp4", "mxfp8"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_fp_dot_exact_bruteforce(mode, dtype):
+    M, N, K = 2, 3, 64
+    c = synth.fp_case(M, N, K, mode, dtype, seed=5)
+    x, w, sc, glob = c["x"][0], c["w"][0], c["scales"][0], c["global"]
+    y, absdot = oracle.qmv_fp(x, w, sc, glob, M, N, K, mode, dtype)
+    xv = _val(x, dtype)
+    e2m1 = {cc: v for cc, v in _read_pairs("e2m1_values.txt")}
+    e4 = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    blk = synth.FP_BLOCK[mode]
+    for n in range(N):
+        for m in range(M):
+            acc = Fraction(0)
+            for k in range(K):
+                if mode == "mxfp8":
+                    e = Fraction(float(e4[w[n, k]]))
+                else:
+                    e = Fraction(e2m1[(int(w[n, k // 2]) >> (4 * (k % 2))) & 0xF])
+                s = int(sc[n, k // blk])
+                scale = (Fraction(float(e4[s])) * Fraction(float(glob))) if mode == "nvfp4" \
+                    else Fraction(2) ** (s - 127)
+                acc += Fraction(xv[m, k]) * e * scale
+            assert abs(Fraction(y[m, n]) - acc) <= Fraction(absdot[m, n]) * Fraction(2) ** -40
+
+
+@pytest.mark.parametrize("bits", [3, 4, 6])
+def test_all_zero_codes_closed_form(bits):
+    """q = 0 everywhere: y[m, n] = sum_groups bias[n, g] * sum_{k in g} x[m, k]."""
+    M, N, K, group = 2, 4, 256, 64
+    c = synth.affine_case(M, N, K, bits, group, "bf16", seed=3)
+    w = np.zeros_like(c["w"][0])
+    y, _ = oracle.qmv_affine(c["x"][0], w, c["scales"][0], c["biases"][0], M, N, K, bits, group, "bf16")
+    xv, bv = _val(c["x"][0], "bf16"), _val(c["biases"][0], "bf16")
+    for m in range(M):
+        for n in range(N):
+            want = sum(Fraction(bv[n, j]) * sum(Fraction(v) for v in xv[m, j * group:(j + 1) * group])
+                       for j in range(K // group))
+            assert abs(Fraction(y[m, n]) - want) <= abs(want) * Fraction(2) ** -48 + Fraction(2) ** -200
+
+
+@pytest.mark.parametrize("bits", [2, 5, 8])
+def test_unit_x_selects_column(bits):
+    """x = e_k: y[0, n] = scale[n, k/g] * q[n, k] + bias[n, k/g] (codes from the
+    test-side reader, values from library casts)."""
+    N, K, group = 5, 128, 32
+    c = synth.affine_case(1, N, K, bits, group, "f32", seed=9)
+    for k in (0, 1, 37, 127):
+        x = np.zeros((1, K), dtype=np.float32); x[0, k] = 1.0
+        y, _ = oracle.qmv_affine(x, c["w"][0], c["scales"][0], c["biases"][0], 1, N, K, bits, group, "f32")
+        for n in range(N):
+            q = _py_codes(c["w"][0][n], K, bits)[k]
+            want = float(c["scales"][0][n, k // group]) * q + float(c["biases"][0][n, k // group])
+            assert y[0, n] == want
+
+
+# ------------------------------------------------------------ sum(x) pin ----
+def _emulate_kernel_bf16(case, widened):
+    """fp32 emulation of a qmv whose bias term uses sum(x) per group, either
+    widened per element (correct) or formed as bf16 sums of 4 consecutive x
+    before widening (the low-precision variant MLX's fix removed)."""
+    K, g = case["K"], case["group"]
+    x = _val(case["x"][0], "bf16").astype(np.float32)[0]
+    w = case["w"][0]
+    N = w.shape[0]
+    bits = case["bits"]
+    s = _val(case["scales"][0], "bf16").astype(np.float32)
+    b = _val(case["biases"][0], "bf16").astype(np.float32)
+    codes = np.array([_py_codes(w[n], K, bits) for n in range(N)], dtype=np.float32)
+    ng = K // g
+    xq = (codes * x[None, :]).reshape(N, ng, g).astype(np.float64).sum(-1).astype(np.float32)
+    if widened:
+        sx = x.reshape(ng, g).astype(np.float32).sum(-1, dtype=np.float32)
+    else:
+        xt = torch.from_numpy(x.reshape(ng, g // 4, 4)).to(torch.bfloat16)
+        four = ((xt[..., 0] + xt[..., 1]) + xt[..., 2]) + xt[..., 3]      # rounded in bf16
+        sx = four.to(torch.float32).sum(-1).numpy()
+    y = (s * xq + b * sx[None, :]).sum(-1, dtype=np.float32)
+    return torch.from_numpy(y).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def test_low_precision_sum_x_fails_tolerance():
+    case = synth.affine_case(1, 512, 2560, 4, 64, "bf16", seed=2, precision=True)
+    y_ref, absdot = oracle.qmv_affine(case["x"][0], case["w"][0], case["scales"][0], case["biases"][0],
+                                      1, 512, 2560, 4, 64, "bf16", threads=8)
+    ok_good, _ = check(_emulate_kernel_bf16(case, True)[None, :], y_ref, absdot, "bf16")
+    ok_bad, _ = check(_emulate_kernel_bf16(case, False)[None, :], y_ref, absdot, "bf16")
+    assert ok_good.all()
+    assert (~ok_bad).sum() >= 10, int((~ok_bad).sum())
