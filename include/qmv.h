@@ -1,0 +1,165 @@
+/*
+ * qmv.h -- C ABI of libqmv.so: the weight-quantized matrix-vector product on
+ * NVIDIA B200 (sm_100a).
+ *
+ *     y[m, n] = sum_k x[m, k] * dequant(W)[n, k]      0 <= m < M <= 8
+ *
+ * The operation and its formats are the ones defined on these pages:
+ *  - MLX "quantized_nax.h" (mlx 1.0.0 source page): affine group quantization,
+ *    w = scale * q + bias per group of `group_size` codes along K; pack geometry
+ *    in get_pack_factor / get_bytes_per_pack (3- and 5-bit codes 8 to a pack of
+ *    3 / 5 bytes, 6-bit codes 4 to a pack of 3 bytes, 2/4/8-bit codes 8/bits to
+ *    a byte); codes read least significant bit first inside a pack (qdot,
+ *    dequantize); scales and biases stored [N, K / group_size] in the dtype of x.
+ *  - wh-iron "kernel-op coverage audit", section "Quantization precision
+ *    coverage", Track 1 table: MXFP4 (E2M1 codes, E8M0 scale per 32),
+ *    NVFP4 (E2M1 codes, E4M3 scale per 16, FP32 global scale), MXFP8 (E4M3
+ *    codes, E8M0 scale per 32); 4-bit codes two to a byte, low nibble first.
+ *  - MLX pull request "affine_qmv_fast_rows / fp_qmv_fast_rows": the user call
+ *    (packed w, scales, biases, bits, group size / mode, NVFP4 global scale),
+ *    output sizes N that are not a multiple of the row tile, and the bias term
+ *    built from a sum(x) widened to fp32 element by element.
+ *
+ * Conventions shared by every entry point
+ *  - All array pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or keeps them.  Layouts are row-major and dense:
+ *      x        [M, K]          dtype
+ *      w_packed [N, K*bits/8]   bytes (affine); [N, K/2] (FP4); [N, K] (FP8)
+ *      scales   [N, K/group]    dtype (affine);  uint8 [N, K/block] (FP modes)
+ *      biases   [N, K/group]    dtype (affine only)
+ *      y        [M, N]          dtype
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *    asynchronous on that stream: it validates its arguments on the host, then
+ *    enqueues kernels; it never synchronizes.  Kernels are launched with
+ *    programmatic dependent launch, so they may start while the previous kernel
+ *    in the stream drains; they read no input before that kernel has finished.
+ *  - Calls are thread-safe for distinct streams.
+ *  - Return value: QMV_OK, or a negative qmv_status.  Argument errors are
+ *    detected before any launch (nothing is enqueued).  QMV_ECUDA means a launch
+ *    failed; qmv_last_cuda_error() gives the cudaError_t of the last such
+ *    failure on the calling thread.
+ *  - M == 0 or N == 0 is a no-op returning QMV_OK; K == 0 writes y = 0.
+ */
+#ifndef QMV_H
+#define QMV_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { QMV_F32 = 0, QMV_F16 = 1, QMV_BF16 = 2 } qmv_dtype;
+
+typedef enum { QMV_MXFP4 = 0, QMV_NVFP4 = 1, QMV_MXFP8_E4M3 = 2 } qmv_fp_mode;
+
+typedef enum {
+    QMV_OK = 0,
+    QMV_EINVAL = -1,        /* bad size, null pointer, K not a multiple of the group/block */
+    QMV_EUNSUPPORTED = -2,  /* bits, group_size, mode or dtype outside the supported set */
+    QMV_EALIGN = -3,        /* a pointer is not aligned to its element (w_packed: 4 bytes) */
+    QMV_ECUDA = -4          /* a CUDA launch or device query failed */
+} qmv_status;
+
+#define QMV_MAX_M 8
+
+/*
+ * qmv_affine -- affine group-quantized qmv.
+ *   x, y      dtype elements, [M, K] and [M, N]
+ *   w_packed  [N, K*bits/8] bytes; each row is a stream of packs as described
+ *             above (4 bytes alignment required; 16 bytes enables the wide-load
+ *             path when K is a multiple of its chunk)
+ *   scales,   [N, K/group_size] dtype elements
+ *   biases
+ *   bits in {2,3,4,5,6,8}; group_size in {32,64,128}; K % group_size == 0;
+ *   1 <= M <= 8 (0 allowed as a no-op); dtype a qmv_dtype.
+ * Each output is  sum over groups g of  scale[n,g] * sum_{k in g} x[m,k]*q[n,k]
+ *                                     + bias[n,g]  * sum_{k in g} x[m,k],
+ * accumulated in fp32 (sum(x) widened per element) and rounded once to dtype.
+ */
+int qmv_affine(const void* x, const void* w_packed, const void* scales, const void* biases,
+               void* y, int M, int N, int K, int bits, int group_size, int dtype,
+               void* stream);
+
+/*
+ * qmv_affine_batched -- `batch` independent affine problems in one launch
+ * (MLX quantized_nax.h, adjust_matrix_offsets: one batch index per grid z).
+ * w_packed, scales, biases and y are contiguous [batch, ...] stacks of the
+ * single-problem layouts.  x_batched = 1: x is [batch, M, K]; 0: one x [M, K]
+ * shared by every batch entry.  1 <= batch <= 65535.
+ */
+int qmv_affine_batched(const void* x, const void* w_packed, const void* scales,
+                       const void* biases, void* y, int M, int N, int K, int bits,
+                       int group_size, int dtype, int batch, int x_batched, void* stream);
+
+/*
+ * qmv_fp -- block-scaled FP qmv.
+ *   mode QMV_MXFP4:      w_packed [N, K/2] E2M1 codes (low nibble = even k),
+ *                        scales [N, K/32] E8M0 bytes; K % 32 == 0
+ *   mode QMV_NVFP4:      w_packed [N, K/2] E2M1 codes, scales [N, K/16] E4M3 bytes,
+ *                        global_scale: DEVICE pointer to one float (required);
+ *                        K % 16 == 0 (K % 32 == 0 for this implementation)
+ *   mode QMV_MXFP8_E4M3: w_packed [N, K] E4M3 codes, scales [N, K/32] E8M0 bytes;
+ *                        K % 32 == 0
+ *   global_scale must be NULL for the MX modes.
+ * Output: sum over blocks of  scale_blk * sum_{k in blk} x[m,k] * elem[n,k]
+ * (times the global scale for NVFP4), fp32 accumulation, one rounding to dtype.
+ * NaN codes (E4M3 0x7F/0xFF, E8M0 0xFF) propagate as NaN.
+ */
+int qmv_fp(const void* x, const void* w_packed, const void* scales, const float* global_scale,
+           void* y, int M, int N, int K, int mode, int dtype, void* stream);
+
+/* qmv_fp_batched -- batched form of qmv_fp; layouts as in qmv_affine_batched.
+ * For NVFP4 global_scale points to `batch` floats (one per weight tensor). */
+int qmv_fp_batched(const void* x, const void* w_packed, const void* scales,
+                   const float* global_scale, void* y, int M, int N, int K, int mode,
+                   int dtype, int batch, int x_batched, void* stream);
+
+/*
+ * qmv_dequant_affine_f32 -- check kernel: w_out[n*K + k] = fp32 value of
+ * scale * q + bias, computed with one rounding (fmaf) from the stored dtype
+ * scale / bias.  Uses the same device decoders as qmv_affine.  w_out is a
+ * caller-owned device buffer of N*K floats.
+ */
+int qmv_dequant_affine_f32(const void* w_packed, const void* scales, const void* biases,
+                           float* w_out, int N, int K, int bits, int group_size, int dtype,
+                           void* stream);
+
+/*
+ * qmv_dequant_fp_f32 -- check kernel: w_out[n*K + k] = elem * scale (MX), or
+ * (elem * e4m3_scale) * global (NVFP4, one rounding), in fp32.
+ */
+int qmv_dequant_fp_f32(const void* w_packed, const void* scales, const float* global_scale,
+                       float* w_out, int N, int K, int mode, void* stream);
+
+/* Human-readable text of a qmv_status. */
+const char* qmv_status_string(int status);
+
+/* cudaError_t of the last QMV_ECUDA returned on this thread (0 if none). */
+int qmv_last_cuda_error(void);
+
+/*
+ * qmv_describe_plan -- the launch the picker would choose for these sizes,
+ * written as text into buf (at most buflen bytes, NUL-terminated).  `family`
+ * is 0 for affine (bits, group_size used) or 1 + qmv_fp_mode.  Host-only; no
+ * CUDA call except a cached device-property query.  Returns QMV_OK or an
+ * argument error.
+ */
+int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size, int dtype,
+                      int w_align16, char* buf, int buflen);
+
+/*
+ * qmv_force_config -- benchmarking / testing knob: pin the launch shape used
+ * by every later call in this process.  path: 1 = wide-load chunks, 0 = 4-byte
+ * chunks, -1 = automatic; rows_per_warp in {1,2,4} or -1; warps_k (warps that
+ * split K inside a block) in {1,..,8} or -1; warps_rows in {1,..,8} or -1.
+ * Unsupported combinations fall back to automatic for that field.  Not
+ * thread-safe with concurrent calls; meant for single-threaded harnesses.
+ */
+void qmv_force_config(int path, int rows_per_warp, int warps_k, int warps_rows);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QMV_H */

@@ -1,0 +1,149 @@
+"""C ABI checks that need no GPU: the library loads, exports every function
+include/qmv.h declares, and rejects bad arguments on the host with the status
+the header documents (no kernel is launched for any of these calls)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import weight_quantized_matrix_b200 as q
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+EINVAL, EUNSUP, EALIGN = -1, -2, -3
+
+
+def _declared():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(qmv_\w+)\s*\(", src, flags=re.M))
+    return sorted(names)
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    for must in ("qmv_affine", "qmv_fp", "qmv_affine_batched", "qmv_fp_batched",
+                 "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_status_string"):
+        assert must in names
+
+
+@pytest.mark.parametrize("name", _declared())
+def test_library_exports(name):
+    lib = ctypes.CDLL(q.LIB_PATH)
+    assert hasattr(lib, name), name
+
+
+L = q.lib()
+FAKE = 1 << 20          # an aligned fake address: validation rejects before any use
+
+
+def aff(**kw):
+    a = dict(x=FAKE, w=FAKE, s=FAKE, b=FAKE, y=FAKE, M=1, N=8, K=128, bits=4, g=64, dt=2, st=None)
+    a.update(kw)
+    return L.qmv_affine(a["x"], a["w"], a["s"], a["b"], a["y"], a["M"], a["N"], a["K"], a["bits"], a["g"],
+                        a["dt"], a["st"])
+
+
+def fp(**kw):
+    a = dict(x=FAKE, w=FAKE, s=FAKE, gs=None, y=FAKE, M=1, N=8, K=128, mode=0, dt=2, st=None)
+    a.update(kw)
+    return L.qmv_fp(a["x"], a["w"], a["s"], a["gs"], a["y"], a["M"], a["N"], a["K"], a["mode"], a["dt"], a["st"])
+
+
+@pytest.mark.parametrize("bits", [0, 1, 7, 9, 16])
+def test_bad_bits(bits):
+    assert aff(bits=bits) == EUNSUP
+
+
+@pytest.mark.parametrize("g", [0, 16, 48, 256])
+def test_bad_group(g):
+    assert aff(g=g) == EUNSUP
+
+
+def test_k_not_multiple_of_group():
+    assert aff(K=96, g=64) == EINVAL
+
+
+def test_negative_sizes():
+    assert aff(M=-1) == EINVAL
+    assert aff(N=-1) == EINVAL
+    assert aff(K=-64) == EINVAL
+
+
+def test_m_above_max():
+    assert aff(M=9) == EUNSUP
+
+
+def test_bad_dtype():
+    assert aff(dt=3) == EUNSUP
+    assert fp(dt=-1) == EUNSUP
+
+
+def test_null_pointers():
+    for k in ("x", "w", "s", "b", "y"):
+        assert aff(**{k: None}) == EINVAL, k
+
+
+def test_misaligned_pointers():
+    assert aff(w=FAKE + 2) == EALIGN          # w_packed needs 4 bytes
+    assert aff(x=FAKE + 1) == EALIGN          # bf16 elements
+    assert aff(s=FAKE + 1) == EALIGN
+    assert aff(y=FAKE + 1, dt=0) == EALIGN
+
+
+def test_empty_is_noop_without_launch():
+    assert aff(M=0) == 0
+    assert aff(N=0) == 0
+    assert aff(M=0, x=None, w=None, s=None, b=None) == 0
+
+
+def test_fp_validation():
+    assert fp(mode=3) == EUNSUP
+    assert fp(mode=1, gs=None) == EINVAL           # NVFP4 needs the global scale
+    assert fp(mode=0, gs=FAKE) == EINVAL           # MX modes take none
+    assert fp(mode=0, K=48) == EINVAL
+    assert fp(mode=2, K=40) == EINVAL
+    assert fp(mode=1, gs=FAKE, K=40) == EINVAL     # not a multiple of the 16 block
+    assert fp(mode=1, gs=FAKE, K=48) == EUNSUP     # 16-code tail block not implemented
+    assert fp(mode=1, gs=FAKE + 2) == EALIGN
+
+
+def test_batched_validation():
+    assert L.qmv_affine_batched(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 128, 4, 64, 2, 0, 1, None) == EINVAL
+    assert L.qmv_affine_batched(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 128, 4, 64, 2, 70000, 1, None) == EINVAL
+    assert L.qmv_affine_batched(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 128, 4, 64, 2, 2, 3, None) == EINVAL
+    assert L.qmv_fp_batched(FAKE, FAKE, FAKE, None, FAKE, 1, 8, 128, 0, 2, 0, 1, None) == EINVAL
+
+
+def test_dequant_validation():
+    assert L.qmv_dequant_affine_f32(FAKE, FAKE, FAKE, FAKE, 8, 128, 7, 64, 2, None) == EUNSUP
+    assert L.qmv_dequant_affine_f32(FAKE, FAKE, FAKE, FAKE, 8, 100, 4, 64, 2, None) == EINVAL
+    assert L.qmv_dequant_affine_f32(FAKE, FAKE, FAKE, FAKE + 4, 8, 128, 4, 64, 2, None) == EALIGN
+    assert L.qmv_dequant_affine_f32(FAKE, FAKE, FAKE, FAKE, 0, 128, 4, 64, 2, None) == 0
+    assert L.qmv_dequant_fp_f32(FAKE, FAKE, None, FAKE, 8, 128, 1, None) == EINVAL
+
+
+def test_status_strings():
+    for st in (0, -1, -2, -3, -4):
+        assert q.qmv_status_string(st)
+    assert q.qmv_status_string(-99) == "unknown status"
+
+
+def test_python_binding_raises():
+    with pytest.raises(q.QmvError) as e:
+        q.qmv_affine(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 128, 7, 64, "bf16", stream=0)
+    assert e.value.status == EUNSUP
+
+
+def test_plan_no_n_cliff():
+    """Any N gets a plan from the same kernel (no N % 8 generic fallback)."""
+    for n in (1, 3, 5, 7, 8, 9, 12, 17, 4095, 4096, 4097):
+        s = q.qmv_describe_plan("affine", 1, n, 2560, bits=8, group_size=64)
+        assert "path=wide" in s, (n, s)
+    assert "path=narrow" in q.qmv_describe_plan("affine", 1, 64, 96, bits=3, group_size=32)
+    assert "path=narrow" in q.qmv_describe_plan("affine", 1, 64, 4096, bits=3, group_size=32, w_align16=False)

@@ -1,0 +1,358 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on the
+same seeded host bytes.  Every test here needs a B200 and is marked ``gpu``.
+
+Bars (see qmv_tol.py): dequantized weights bit-exact; f16 / bf16 outputs within
+1 ulp of the fp64 oracle (or 1e-5 * sum|x*w| where the sum cancels); f32 outputs
+within 1e-5 * sum|x*w|.  Workloads: every shape the workload list names, at
+full size (oracle on sampled rows) and at small sizes (oracle on every row),
+plus ragged N and K, batches, M = 1..8, empty and degenerate cases.
+"""
+from __future__ import annotations
+
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import (THREADS, compare, dev, oracle_affine, oracle_fp, require_cuda, run_affine, run_fp,
+                      sample_rows, to_f64, y_buffer)
+
+pytestmark = pytest.mark.gpu
+
+BITS = [2, 3, 4, 5, 6, 8]
+GROUPS = [32, 64, 128]
+DTYPES = ["f32", "f16", "bf16"]
+MODES = ["mxfp4", "nvfp4", "mxfp8"]
+
+
+@pytest.fixture(scope="module")
+def q():
+    return require_cuda()
+
+
+@pytest.fixture(autouse=True)
+def _auto_config(q):
+    q.qmv_force_config()
+    yield
+    q.qmv_force_config()
+
+
+def _seed(*parts):
+    return zlib.crc32("/".join(str(p) for p in parts).encode()) & 0x7FFFFFFF
+
+
+# ------------------------------------------------------------- native code --
+def test_native_library_is_what_runs(q):
+    c = synth.affine_case(1, 8, 64, 4, 64, "bf16", seed=1)
+    run_affine(q, c)
+    maps = open("/proc/self/maps").read()
+    assert q.LIB_PATH in maps
+
+
+# ------------------------------------------------------- dequant bit-exact --
+def _bits_equal(a, b):
+    a = np.asarray(a, np.float32); b = np.asarray(b, np.float32)
+    nan = np.isnan(a) & np.isnan(b)
+    return bool(np.all(nan | (a.view(np.uint32) == b.view(np.uint32))))
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("group", GROUPS)
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_dequant_affine_bit_exact(q, bits, group, dtype):
+    N, K = 37, 384
+    c = synth.affine_case(1, N, K, bits, group, dtype, seed=_seed("dqa", bits, group, dtype))
+    out = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    q.qmv_dequant_affine_f32(dev(c["w"]), dev(c["scales"]), dev(c["biases"]), out, N, K, bits, group, dtype)
+    torch.cuda.synchronize()
+    ref = oracle.dequant_affine_f32(c["w"][0], c["scales"][0], c["biases"][0], N, K, bits, group, dtype)
+    assert _bits_equal(out.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_dequant_fp_bit_exact_all_codes(q, mode):
+    """Every code byte and every scale byte (NaN encodings included)."""
+    bits, blk = synth.FP_BITS[mode], synth.FP_BLOCK[mode]
+    N, K = 256, 512
+    w = np.tile(np.arange(256, dtype=np.uint8), N * K * bits // 8 // 256 + 1)[: N * K * bits // 8]
+    w = np.ascontiguousarray(np.random.default_rng(3).permutation(w).reshape(N, K * bits // 8))
+    sc = (np.arange(N * (K // blk)) % 256).astype(np.uint8).reshape(N, K // blk)
+    g = np.float32(1.3) if mode == "nvfp4" else None
+    out = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    gd = torch.tensor([g], device="cuda") if g is not None else None
+    q.qmv_dequant_fp_f32(dev(w), dev(sc), gd, out, N, K, mode)
+    torch.cuda.synchronize()
+    ref = oracle.dequant_fp_f32(w, sc, g, N, K, mode)
+    assert _bits_equal(out.cpu().numpy(), ref)
+
+
+# ---------------------------------------------------- the small workload ----
+def test_small_config_4bit(q):
+    """M=1, N=256, K=512, 4-bit g64 bf16, seed 0 (every row checked)."""
+    c = synth.affine_case(1, 256, 512, 4, 64, "bf16", seed=0)
+    y = run_affine(q, c)[0]
+    ref, ad = oracle_affine(c)
+    compare(y, ref, ad, "bf16", what="small 4-bit")
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("group", GROUPS)
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_affine_grid(q, bits, group, dtype, M):
+    N, K = 67, 512
+    c = synth.affine_case(M, N, K, bits, group, dtype, seed=_seed("grid", bits, group, dtype, M))
+    y = run_affine(q, c)[0]
+    ref, ad = oracle_affine(c)
+    compare(y, ref, ad, dtype, what=f"b{bits} g{group} {dtype} M{M}")
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("M", [1, 2, 5])
+def test_affine_narrow_path_ragged_k(q, bits, M):
+    """K a multiple of the group but not of the wide chunk -> 4-byte chunks."""
+    N, K, group = 45, 480, 32
+    c = synth.affine_case(M, N, K, bits, group, "bf16", seed=_seed("narrow", bits, M))
+    y = run_affine(q, c)[0]
+    ref, ad = oracle_affine(c)
+    compare(y, ref, ad, "bf16", what=f"narrow b{bits}")
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_affine_misaligned_w_uses_narrow_path(q, bits):
+    N, K, group = 33, 1024, 64
+    c = synth.affine_case(2, N, K, bits, group, "f16", seed=_seed("mis", bits))
+    y = run_affine(q, c, w_offset=4)[0]
+    ref, ad = oracle_affine(c)
+    compare(y, ref, ad, "f16", what=f"misaligned b{bits}")
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("N", [1, 3, 5, 12, 17])
+def test_fast_rows_output_sizes(q, bits, N):
+    """The MLX fast_rows test sizes: K=2560, group 64, with batched weights."""
+    c = synth.affine_case(1, N, 2560, bits, 64, "bf16", seed=_seed("rows", bits, N), batch=2)
+    y = run_affine(q, c)
+    for b in range(2):
+        ref, ad = oracle_affine(c, b=b)
+        compare(y[b], ref, ad, "bf16", what=f"rows b{bits} N{N} batch{b}")
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("N", [1, 3, 5, 7, 8, 9, 12, 17])
+def test_fp_output_sizes(q, mode, dtype, N):
+    """The MLX fp fast_rows test sizes, all three modes and dtypes, batched."""
+    c = synth.fp_case(1, N, 1024, mode, dtype, seed=_seed("fprows", mode, dtype, N), batch=2)
+    y = run_fp(q, c)
+    for b in range(2):
+        ref, ad = oracle_fp(c, b=b)
+        compare(y[b], ref, ad, dtype, what=f"{mode} {dtype} N{N} b{b}")
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("shape", [(5, 1024, 2), (12, 4096, 1)])
+@pytest.mark.parametrize("x_batched", [True, False])
+def test_fp_workload_shapes(q, mode, shape, x_batched):
+    """Block-scaled FP workload shapes: (N=5, K=1024, batch=2 weights) and
+    (N=12, K=4096), bf16 x; x either batched or shared."""
+    N, K, B = shape
+    c = synth.fp_case(1, N, K, mode, "bf16", seed=_seed("fpw", mode, N), batch=B)
+    y = run_fp(q, c, x_batched=x_batched)
+    for b in range(B):
+        ref, ad = oracle_fp(c, b=b, x_batched=x_batched)
+        compare(y[b], ref, ad, "bf16", what=f"{mode} N{N} K{K} b{b}")
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("M", [2, 4, 8])
+def test_fp_multi_m(q, mode, M):
+    c = synth.fp_case(M, 77, 2048, mode, "bf16", seed=_seed("fpm", mode, M))
+    y = run_fp(q, c)[0]
+    ref, ad = oracle_fp(c)
+    compare(y, ref, ad, "bf16", what=f"{mode} M{M}")
+
+
+def test_fp_nan_codes_propagate(q):
+    c = synth.fp_case(1, 4, 64, "mxfp8", "bf16", seed=4)
+    c["w"][0, 2, 5] = 0x7F           # NaN element in row 2
+    c["scales"][0, 3, 1] = 0xFF      # NaN block scale in row 3
+    y = run_fp(q, c)[0]
+    ref, ad = oracle_fp(c)
+    assert np.isnan(y[0, 2]) and np.isnan(y[0, 3])
+    compare(y, ref, ad, "bf16", what="nan")
+
+
+# ------------------------------------------------------- tail invariant ----
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("n", [1, 3, 5, 12, 17])
+def test_tail_rows_bitwise_prefix(q, bits, n):
+    """N = n equals, bit for bit, the first n rows of the same weights padded
+    to a whole row tile (same launch shape), as the MLX fast_rows tests check."""
+    q.qmv_force_config(1, 4, 1, 4)            # row tile = 16
+    K, group = 2560, 64
+    pad = 16 * ((n + 15) // 16)
+    big = synth.affine_case(1, pad, K, bits, group, "bf16", seed=_seed("tail", bits, n))
+    small = dict(big, N=n, w=big["w"][:, :n].copy(), scales=big["scales"][:, :n].copy(),
+                 biases=big["biases"][:, :n].copy())
+    yb = run_affine(q, big)[0]
+    ys = run_affine(q, small)[0]
+    assert np.array_equal(ys, yb[:, :n])
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_fp_tail_rows_bitwise_prefix(q, mode):
+    q.qmv_force_config(1, 2, 1, 4)            # row tile = 8
+    big = synth.fp_case(1, 24, 4096, mode, "bf16", seed=_seed("fptail", mode))
+    for n in (1, 5, 9, 17):
+        small = dict(big, N=n, w=big["w"][:, :n].copy(), scales=big["scales"][:, :n].copy())
+        assert np.array_equal(run_fp(q, small)[0], run_fp(q, big)[0][:, :n])
+
+
+# --------------------------------------------------------- precision case ---
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6])
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_precision_case_sum_x(q, bits, dtype):
+    """x ~ U(1e-4, 1e-3), symmetric zero point: the bias term dominates and a
+    low-precision sum(x) would fail (see the mutant pin); every row checked."""
+    c = synth.affine_case(1, 4096, 2560, bits, 64, dtype, seed=_seed("prec", bits, dtype), precision=True)
+    y = run_affine(q, c)[0]
+    ref, ad = oracle_affine(c)
+    compare(y, ref, ad, dtype, what=f"precision b{bits} {dtype}")
+
+
+# -------------------------------------------------- full-size workloads ----
+@pytest.mark.parametrize("bits", [2, 3, 5, 6])
+@pytest.mark.parametrize("group", GROUPS)
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("M", [1, 4])
+def test_sweep_full_size(q, bits, group, dtype, M):
+    """Affine sweep at N = K = 4096 (oracle on sampled rows)."""
+    c = synth.affine_case(M, 4096, 4096, bits, group, dtype, seed=_seed("sweep", bits, group, dtype, M))
+    y = run_affine(q, c)[0]
+    rows = sample_rows(4096)
+    ref, ad = oracle_affine(c, rows=rows)
+    compare(y, ref, ad, dtype, rows=rows, what=f"sweep b{bits} g{group} {dtype} M{M}")
+
+
+LAYER = [("qkv", 6144, 4096), ("o", 4096, 4096), ("gate_up", 28672, 4096), ("down", 4096, 14336)]
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_decode_layer_chain(q, M):
+    """7B-class decode layer, 4-bit g64 bf16, the four projections chained:
+    each input is the previous output truncated to the next K (oracle fed the
+    GPU's actual input, sampled rows)."""
+    x = synth.affine_case(M, 1, 4096, 4, 64, "bf16", seed=_seed("layer_x", M))["x"]
+    for i, (name, N, K) in enumerate(LAYER):
+        c = synth.affine_case(M, N, K, 4, 64, "bf16", seed=_seed("layer", name, M))
+        c["x"] = np.ascontiguousarray(x[:, :, :K])
+        y = run_affine(q, c)[0]
+        rows = sample_rows(N, 32)
+        ref, ad = oracle_affine(c, rows=rows)
+        compare(y, ref, ad, "bf16", rows=rows, what=f"layer {name} M{M}")
+        # next input: this output (bf16 storage), truncated; rescaled to unit
+        # RMS on the host so the chain stays in range (parity-only variant)
+        yv = y.astype(np.float32)
+        yv = yv / np.sqrt(np.mean(yv ** 2, axis=-1, keepdims=True) + 1e-30)
+        x = synth.to_storage(yv[None], "bf16")
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_bandwidth_probe_16384(q, M):
+    c = synth.affine_case(M, 16384, 16384, 4, 64, "bf16", seed=_seed("probe", M))
+    y = run_affine(q, c)[0]
+    rows = sample_rows(16384, 24)
+    ref, ad = oracle_affine(c, rows=rows)
+    compare(y, ref, ad, "bf16", rows=rows, what=f"probe M{M}")
+
+
+# ------------------------------------------------------------ the chain ----
+@pytest.mark.parametrize("N", [1, 3, 4, 5, 12, 17, 4096])
+def test_chained_calls_8bit(q, N):
+    """64 dependent calls, 8-bit g64 bf16, K=2560: call t reads the previous
+    output zero-padded (N < K) or truncated (N >= K) to K.  Each call is checked
+    against the oracle fed the GPU's actual input, while that input is finite."""
+    K, T = 2560, 64
+    c = synth.affine_case(1, N, K, 8, 64, "bf16", seed=_seed("chain", N))
+    L = max(N, K)
+    w, s, b = dev(c["w"]), dev(c["scales"]), dev(c["biases"])
+    x0 = torch.zeros(L, dtype=torch.bfloat16, device="cuda")
+    x0[:K] = torch.from_numpy(c["x"][0, 0].view(np.int16)).view(torch.bfloat16).cuda()
+    bufs = [torch.zeros(L, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    rows = sample_rows(N, 24)
+    checked = 0
+    for t in range(T):
+        xin = x0 if t == 0 else bufs[(t - 1) % 2]
+        yout = bufs[t % 2]
+        q.qmv_affine(xin, w, s, b, yout, 1, N, K, 8, 64, "bf16")
+        torch.cuda.synchronize()
+        xh = xin[:K].cpu().view(torch.int16).numpy().view(np.uint16).reshape(1, K)
+        if not np.isfinite(xin[:K].float().cpu().numpy()).all():
+            break
+        if t % 8 == 0 or N < 4096:
+            cc = dict(c, x=xh[None])
+            ref, ad = oracle_affine(cc, rows=rows)
+            compare(to_f64(yout[:N]).reshape(1, N), ref, ad, "bf16", rows=rows, what=f"chain N{N} t{t}")
+            checked += 1
+    assert checked >= 2
+
+
+# ------------------------------------------------------- batches & edges ----
+@pytest.mark.parametrize("x_batched", [True, False])
+@pytest.mark.parametrize("bits", [3, 4])
+def test_affine_batched(q, x_batched, bits):
+    c = synth.affine_case(2, 300, 1024, bits, 64, "bf16", seed=_seed("batch", bits, x_batched), batch=3)
+    y = run_affine(q, c, x_batched=x_batched)
+    for b in range(3):
+        ref, ad = oracle_affine(c, b=b, x_batched=x_batched)
+        compare(y[b], ref, ad, "bf16", what=f"batch {b}")
+
+
+def test_k_zero_writes_zeros(q):
+    y = torch.full((2, 5), 7.0, dtype=torch.bfloat16, device="cuda")
+    dummy = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    q.qmv_affine(dummy, dummy, dummy, dummy, y, 2, 5, 0, 4, 64, "bf16")
+    torch.cuda.synchronize()
+    assert (y.float() == 0).all()
+
+
+def test_empty_m_or_n_leaves_y(q):
+    y = torch.full((4,), 7.0, dtype=torch.bfloat16, device="cuda")
+    q.qmv_affine(None, None, None, None, y, 0, 4, 64, 4, 64, "bf16")
+    q.qmv_affine(None, None, None, None, y, 1, 0, 64, 4, 64, "bf16")
+    torch.cuda.synchronize()
+    assert (y.float() == 7).all()
+
+
+@pytest.mark.parametrize("cfg", [(1, 1, 1, 1), (1, 2, 1, 4), (1, 4, 1, 2), (1, 1, 8, 1), (1, 1, 3, 2),
+                                 (0, 1, 1, 4), (0, 1, 4, 2), (1, 2, 2, 4)])
+@pytest.mark.parametrize("bits", [3, 4, 8])
+def test_forced_launch_shapes(q, cfg, bits):
+    """Every launch shape the picker can choose gives the same (tolerance) answer."""
+    q.qmv_force_config(*cfg)
+    c = synth.affine_case(2, 131, 2048, bits, 64, "bf16", seed=_seed("forced", cfg, bits))
+    y = run_affine(q, c)[0]
+    ref, ad = oracle_affine(c)
+    compare(y, ref, ad, "bf16", what=f"forced {cfg} b{bits}")
+
+
+@pytest.mark.parametrize("M", [5, 8])
+def test_x_tiles_when_x_exceeds_shared_memory(q, M):
+    """M * K large enough that x is staged in several K tiles."""
+    c = synth.affine_case(M, 96, 16384, 4, 128, "f32", seed=_seed("tiles", M))
+    y = run_affine(q, c)[0]
+    ref, ad = oracle_affine(c)
+    compare(y, ref, ad, "f32", what=f"tiles M{M}")
+
+
+def test_non_default_stream(q):
+    c = synth.affine_case(1, 100, 1024, 5, 32, "bf16", seed=77)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        y = run_affine(q, c, stream=s)[0]
+    ref, ad = oracle_affine(c)
+    compare(y, ref, ad, "bf16", what="stream")

@@ -1,0 +1,156 @@
+"""Python binding of libqmv.so (include/qmv.h): the weight-quantized
+matrix-vector product on B200.
+
+Argument marshalling only.  Every function takes device buffers as torch
+tensors (or raw integer device addresses), passes their pointers and sizes to
+the C ABI of the same name, and raises :class:`QmvError` on a non-zero status.
+All compute happens in the CUDA kernels of libqmv.so; there is no fallback: if
+the library has not been built, importing this package raises ImportError.
+
+The stream defaults to torch's current CUDA stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "QmvError", "qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
+    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_status_string", "qmv_last_cuda_error",
+    "qmv_describe_plan", "qmv_force_config", "DTYPES", "FP_MODES", "LIB_PATH", "lib",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libqmv.so")
+
+DTYPES = {"f32": 0, "f16": 1, "bf16": 2}
+FP_MODES = {"mxfp4": 0, "nvfp4": 1, "mxfp8": 2}
+STATUS = {0: "QMV_OK", -1: "QMV_EINVAL", -2: "QMV_EUNSUPPORTED", -3: "QMV_EALIGN", -4: "QMV_ECUDA"}
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libqmv.so not found at {LIB_PATH}; build it with "
+        "`python -m weight_quantized_matrix_b200.build_lib` (needs nvcc)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_p, _i, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong
+_lib.qmv_affine.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
+_lib.qmv_affine_batched.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p]
+_lib.qmv_fp.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
+_lib.qmv_fp_batched.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p]
+_lib.qmv_dequant_affine_f32.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
+_lib.qmv_dequant_fp_f32.argtypes = [_p, _p, _p, _p, _i, _i, _i, _p]
+_lib.qmv_status_string.argtypes = [_i]
+_lib.qmv_status_string.restype = ctypes.c_char_p
+_lib.qmv_last_cuda_error.argtypes = []
+_lib.qmv_describe_plan.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, ctypes.c_char_p, _i]
+_lib.qmv_force_config.argtypes = [_i, _i, _i, _i]
+_lib.qmv_force_config.restype = None
+for _f in ("qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
+           "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_last_cuda_error", "qmv_describe_plan"):
+    getattr(_lib, _f).restype = _i
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+class QmvError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        name = STATUS.get(status, str(status))
+        msg = f"{what}: {name} ({_lib.qmv_status_string(status).decode()})"
+        if status == -4:
+            msg += f", cudaError {_lib.qmv_last_cuda_error()}"
+        super().__init__(msg)
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    if isinstance(a, int):
+        return a
+    return a.data_ptr()
+
+
+def _dtype(d):
+    if isinstance(d, int):
+        return d
+    if isinstance(d, str):
+        return DTYPES[d]
+    import torch
+    return {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}[d]
+
+
+def _mode(m):
+    return m if isinstance(m, int) else FP_MODES[m]
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(st, what):
+    if st != 0:
+        raise QmvError(st, what)
+
+
+def qmv_affine(x, w_packed, scales, biases, y, M, N, K, bits, group_size, dtype, stream=None):
+    _check(_lib.qmv_affine(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(biases), _ptr(y), M, N, K,
+                           bits, group_size, _dtype(dtype), _stream(stream)), "qmv_affine")
+
+
+def qmv_affine_batched(x, w_packed, scales, biases, y, M, N, K, bits, group_size, dtype, batch,
+                       x_batched=True, stream=None):
+    _check(_lib.qmv_affine_batched(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(biases), _ptr(y), M, N, K,
+                                   bits, group_size, _dtype(dtype), batch, int(bool(x_batched)),
+                                   _stream(stream)), "qmv_affine_batched")
+
+
+def qmv_fp(x, w_packed, scales, global_scale, y, M, N, K, mode, dtype, stream=None):
+    _check(_lib.qmv_fp(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(global_scale), _ptr(y), M, N, K,
+                       _mode(mode), _dtype(dtype), _stream(stream)), "qmv_fp")
+
+
+def qmv_fp_batched(x, w_packed, scales, global_scale, y, M, N, K, mode, dtype, batch, x_batched=True,
+                   stream=None):
+    _check(_lib.qmv_fp_batched(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(global_scale), _ptr(y), M, N,
+                               K, _mode(mode), _dtype(dtype), batch, int(bool(x_batched)),
+                               _stream(stream)), "qmv_fp_batched")
+
+
+def qmv_dequant_affine_f32(w_packed, scales, biases, w_out, N, K, bits, group_size, dtype, stream=None):
+    _check(_lib.qmv_dequant_affine_f32(_ptr(w_packed), _ptr(scales), _ptr(biases), _ptr(w_out), N, K,
+                                       bits, group_size, _dtype(dtype), _stream(stream)),
+           "qmv_dequant_affine_f32")
+
+
+def qmv_dequant_fp_f32(w_packed, scales, global_scale, w_out, N, K, mode, stream=None):
+    _check(_lib.qmv_dequant_fp_f32(_ptr(w_packed), _ptr(scales), _ptr(global_scale), _ptr(w_out), N, K,
+                                   _mode(mode), _stream(stream)), "qmv_dequant_fp_f32")
+
+
+def qmv_status_string(status: int) -> str:
+    return _lib.qmv_status_string(status).decode()
+
+
+def qmv_last_cuda_error() -> int:
+    return _lib.qmv_last_cuda_error()
+
+
+def qmv_describe_plan(family, M, N, K, bits=4, group_size=64, dtype="bf16", w_align16=True) -> str:
+    """Text of the launch the picker chooses; family 'affine' or an FP mode name."""
+    fam = 0 if family == "affine" else 1 + _mode(family)
+    buf = ctypes.create_string_buffer(256)
+    _check(_lib.qmv_describe_plan(fam, M, N, K, bits, group_size, _dtype(dtype), int(w_align16), buf, 256),
+           "qmv_describe_plan")
+    return buf.value.decode()
+
+
+def qmv_force_config(path=-1, rows_per_warp=-1, warps_k=-1, warps_rows=-1):
+    _lib.qmv_force_config(path, rows_per_warp, warps_k, warps_rows)

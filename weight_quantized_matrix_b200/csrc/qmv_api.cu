@@ -1,0 +1,360 @@
+// qmv_api.cu -- the C ABI of libqmv.so (declared in include/qmv.h): argument
+// validation, the size-based kernel picker and the launches.
+//
+// The picker replaces the pages' three-way choice (MLX: qmv_fast when the
+// input is aligned and N % 8 == 0, qmv_fast_rows when aligned and N % 8 != 0,
+// a generic kernel otherwise -- MLX pull request "affine_qmv_fast_rows")
+// with one kernel template whose launch shape is chosen from the sizes:
+//   * path:   wide 16-byte chunk loads when K is a multiple of the wide chunk
+//             and w_packed is 16-byte aligned, else 4-byte chunks (any K that
+//             is a multiple of the group);
+//   * rows:   rows per warp R (x reuse) grows with N; any N works (tail rows
+//             are clamped and not stored), so there is no N % 8 cliff;
+//   * split-K inside the block: for narrow N the K chunks of a row are spread
+//             over up to 8 warps (wk) so one row still uses many threads;
+//   * x tile: the K range staged in shared memory at a time.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qmv.h"
+#include "qmv_launch.cuh"
+
+namespace {
+
+thread_local int g_last_cuda = 0;
+
+struct Forced { int path = -1, R = -1, wk = -1, wr = -1; };
+Forced g_forced;
+
+struct DevInfo { int sms = 0; int ok = 0; };
+DevInfo g_dev[64];
+std::mutex g_dev_mu;
+
+int device_sms() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!g_dev[dev].ok) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+            cudaGetLastError();
+            return 148;
+        }
+        g_dev[dev].sms = sms;
+        g_dev[dev].ok = 1;
+    }
+    return g_dev[dev].sms;
+}
+
+int elem_bytes(int dtype) { return dtype == QMV_F32 ? 4 : 2; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Per-format facts the picker needs (mirrors qmv::Fmt).
+struct FmtInfo {
+    int fam, bits, wide_units;
+};
+
+FmtInfo fmt_info(int fam, int bits) {
+    int b = fam == qmv::FAM_AFFINE ? bits : (fam == qmv::FAM_MXFP8 ? 8 : 4);
+    int wu = b == 2 ? 4 : b == 3 ? 4 : b == 4 ? 2 : b == 5 ? 4 : b == 6 ? 2 : 1;
+    return {fam, b, wu};
+}
+
+struct Plan {
+    int maxm, R, wide, wk, wr, tile_iters, C;
+    size_t smem;
+    dim3 grid, block;
+};
+
+int rows_per_warp_cap(int bits, int maxm) {
+    if (maxm <= 2) return (bits == 3 || bits == 5 || bits == 6) ? 2 : 4;
+    return 2;
+}
+
+// Choose the launch shape.  Returns QMV_OK or an error (sizes too large).
+int make_plan(int fam, int M, int N, int K, int bits, int dtype, bool w16, int batch, Plan* pl) {
+    const FmtInfo fi = fmt_info(fam, bits);
+    const bool aff = fam == qmv::FAM_AFFINE;
+    int maxm = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
+    const int c_wide = 32 * fi.wide_units;
+    bool wide = w16 && (K % c_wide == 0);
+    if (g_forced.path == 0) wide = false;
+    if (g_forced.path == 1 && w16 && (K % c_wide == 0)) wide = true;
+    const int U = wide ? fi.wide_units : 1;
+    const int C = 32 * U;
+    const int NC = K / C;
+    const int sms = device_sms();
+
+    int R = 1, wk = 1, wr = 1;
+    if (N <= 64) {
+        // narrow N: one row per warp, the row's chunks spread over the block
+        R = 1;
+        wr = 1;
+        wk = (NC + 31) / 32;
+        wk = wk < 1 ? 1 : (wk > 8 ? 8 : wk);
+        if (N * wk < 2 * sms && NC >= 64 * wk) {  // still few threads: more warps per row
+            while (wk < 8 && NC >= 32 * (wk + 1)) ++wk;
+        }
+    } else {
+        const int rcap = wide ? rows_per_warp_cap(fi.bits, maxm) : 1;
+        R = N >= 1024 ? rcap : (N >= 256 ? (rcap < 2 ? rcap : 2) : 1);
+        const long long warps = ((long long)N + R - 1) / R * batch;
+        wk = 1;
+        while (wk < 8 && warps * wk < (long long)sms * 8 && NC >= 64 * wk) wk *= 2;
+        wr = wk >= 8 ? 1 : 8 / wk;
+        if (wr > 4 && wk == 1) wr = 4;
+    }
+    if (g_forced.R > 0) R = g_forced.R;
+    if (g_forced.wk > 0) wk = g_forced.wk;
+    if (g_forced.wr > 0) wr = g_forced.wr;
+    if (!qmv::shape_instantiated(maxm, R, wide)) R = 1;
+    if (wk < 1) wk = 1;
+    if (wk > 8) wk = 8;
+    if (wr < 1) wr = 1;
+    while (wk * wr > 8) --wr;
+    if (wr < 1) wr = 1;
+
+    // x tile: shrink the k-warps until one iteration of x fits the budget
+    const size_t budget = 96 * 1024;
+    auto per_iter_of = [&](int wk_) {
+        return (size_t)maxm * C * 32 * wk_ * 4 + (aff ? (size_t)maxm * U * 32 * wk_ * 4 : 0);
+    };
+    while (wk > 1 && per_iter_of(wk) > budget) --wk;
+    const int KT = 32 * wk;
+    const size_t per_iter = per_iter_of(wk);
+    const size_t red = (size_t)wk * wr * R * maxm * 4;
+    long long iters_needed = ((long long)NC + KT - 1) / KT;
+    if (iters_needed < 1) iters_needed = 1;
+    long long ti = (long long)((budget > red ? budget - red : 0) / per_iter);
+    if (ti < 1) ti = 1;
+    if (ti > iters_needed) ti = iters_needed;
+    const size_t smem = per_iter * ti + red;
+    if (smem > (size_t)qmv::kMaxSmem) return QMV_EUNSUPPORTED;
+
+    const long long rows_per_block = (long long)wr * R;
+    const long long gx = ((long long)N + rows_per_block - 1) / rows_per_block;
+    if (gx > 0x7FFFFFFFLL) return QMV_EINVAL;
+
+    pl->maxm = maxm; pl->R = R; pl->wide = wide; pl->wk = wk; pl->wr = wr;
+    pl->tile_iters = (int)ti; pl->C = C; pl->smem = smem;
+    pl->grid = dim3((unsigned)gx, 1, (unsigned)batch);
+    pl->block = dim3(32 * wk * wr, 1, 1);
+    return QMV_OK;
+}
+
+int finish(cudaError_t e) {
+    if (e == cudaSuccess) return QMV_OK;
+    g_last_cuda = (int)e;
+    cudaGetLastError();  // clear the sticky-free launch error state
+    return QMV_ECUDA;
+}
+
+bool pdl_enabled() {
+    static int v = -1;
+    if (v < 0) {
+        const char* s = getenv("QMV_PDL");
+        v = (s && s[0] == '0') ? 0 : 1;
+    }
+    return v == 1;
+}
+
+int check_common(const void* x, const void* w, const void* s, void* y, int M, int N, int K, int dtype) {
+    if (M < 0 || N < 0 || K < 0) return QMV_EINVAL;
+    if (M > QMV_MAX_M) return QMV_EUNSUPPORTED;
+    if (dtype != QMV_F32 && dtype != QMV_F16 && dtype != QMV_BF16) return QMV_EUNSUPPORTED;
+    if (M == 0 || N == 0) return QMV_OK;
+    if (!y || (K > 0 && (!x || !w || !s))) return QMV_EINVAL;
+    const size_t eb = elem_bytes(dtype);
+    if (!aligned(y, eb) || (x && !aligned(x, eb))) return QMV_EALIGN;
+    if (w && !aligned(w, 4)) return QMV_EALIGN;
+    return QMV_OK;
+}
+
+int run(int fam, const void* x, const void* w, const void* scales, const void* biases,
+        const float* gscale, void* y, int M, int N, int K, int bits, int G, int dtype, int batch,
+        int x_batched, void* stream) {
+    const long long row_bytes = (long long)K * (fam == qmv::FAM_AFFINE ? bits : (fam == qmv::FAM_MXFP8 ? 8 : 4)) / 8;
+    Plan pl;
+    const bool w16 = aligned(w, 16);
+    int st = make_plan(fam, M, N, K, bits, dtype, w16, batch, &pl);
+    if (st != QMV_OK) return st;
+    qmv::Params p;
+    p.x = x; p.w = static_cast<const uint8_t*>(w); p.scales = scales; p.biases = biases;
+    p.gscale = gscale; p.y = y;
+    p.M = M; p.N = N; p.K = K; p.G = G;
+    p.wk = pl.wk; p.wr = pl.wr; p.tile_iters = pl.tile_iters;
+    const size_t eb = elem_bytes(dtype);
+    p.x_vec = (aligned(x, 16) && ((size_t)K * eb) % 16 == 0) ? 1 : 0;
+    p.x_bs = x_batched ? (long long)M * K : 0;
+    p.w_bs = (long long)N * row_bytes;
+    p.s_bs = (long long)N * (K / G);
+    p.y_bs = (long long)M * N;
+    p.w_row = row_bytes;
+    qmv::Launch L{pl.grid, pl.block, pl.smem, static_cast<cudaStream_t>(stream), pdl_enabled()};
+    cudaError_t e;
+    if (fam == qmv::FAM_AFFINE) {
+        switch (bits) {
+            case 2: e = qmv::launch_affine_b2(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
+            case 3: e = qmv::launch_affine_b3(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
+            case 4: e = qmv::launch_affine_b4(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
+            case 5: e = qmv::launch_affine_b5(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
+            case 6: e = qmv::launch_affine_b6(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
+            case 8: e = qmv::launch_affine_b8(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
+            default: return QMV_EUNSUPPORTED;
+        }
+    } else {
+        e = qmv::launch_fp(fam, dtype, pl.maxm, pl.R, pl.wide, p, L);
+    }
+    return finish(e);
+}
+
+int check_affine(int bits, int group) {
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 5 && bits != 6 && bits != 8) return QMV_EUNSUPPORTED;
+    if (group != 32 && group != 64 && group != 128) return QMV_EUNSUPPORTED;
+    return QMV_OK;
+}
+
+int fp_family(int mode) {
+    return mode == QMV_MXFP4 ? qmv::FAM_MXFP4 : mode == QMV_NVFP4 ? qmv::FAM_NVFP4
+         : mode == QMV_MXFP8_E4M3 ? qmv::FAM_MXFP8 : -1;
+}
+
+int check_fp(int mode, int K, const float* gscale) {
+    int fam = fp_family(mode);
+    if (fam < 0) return QMV_EUNSUPPORTED;
+    if (mode == QMV_NVFP4) {
+        if (K % 16 != 0) return QMV_EINVAL;
+        if (K % 32 != 0) return QMV_EUNSUPPORTED;   // 16-code tail blocks not implemented
+        if (!gscale) return QMV_EINVAL;
+        if (!aligned(gscale, 4)) return QMV_EALIGN;
+    } else {
+        if (K % 32 != 0) return QMV_EINVAL;
+        if (gscale) return QMV_EINVAL;
+    }
+    return QMV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qmv_affine_batched(const void* x, const void* w_packed, const void* scales, const void* biases,
+                       void* y, int M, int N, int K, int bits, int group_size, int dtype, int batch,
+                       int x_batched, void* stream) {
+    int st = check_affine(bits, group_size);
+    if (st != QMV_OK) return st;
+    if (batch < 1 || batch > 65535 || (x_batched != 0 && x_batched != 1)) return QMV_EINVAL;
+    if (K % group_size != 0) return QMV_EINVAL;
+    st = check_common(x, w_packed, scales, y, M, N, K, dtype);
+    if (st != QMV_OK || M == 0 || N == 0) return st;
+    if (K > 0 && !biases) return QMV_EINVAL;
+    const size_t eb = elem_bytes(dtype);
+    if (K > 0 && (!aligned(scales, eb) || !aligned(biases, eb))) return QMV_EALIGN;
+    return run(qmv::FAM_AFFINE, x, w_packed, scales, biases, nullptr, y, M, N, K, bits, group_size,
+               dtype, batch, x_batched, stream);
+}
+
+int qmv_affine(const void* x, const void* w_packed, const void* scales, const void* biases, void* y,
+               int M, int N, int K, int bits, int group_size, int dtype, void* stream) {
+    return qmv_affine_batched(x, w_packed, scales, biases, y, M, N, K, bits, group_size, dtype, 1, 1,
+                              stream);
+}
+
+int qmv_fp_batched(const void* x, const void* w_packed, const void* scales, const float* global_scale,
+                   void* y, int M, int N, int K, int mode, int dtype, int batch, int x_batched,
+                   void* stream) {
+    int st = check_fp(mode, K, global_scale);
+    if (st != QMV_OK) return st;
+    if (batch < 1 || batch > 65535 || (x_batched != 0 && x_batched != 1)) return QMV_EINVAL;
+    st = check_common(x, w_packed, scales, y, M, N, K, dtype);
+    if (st != QMV_OK || M == 0 || N == 0) return st;
+    const int fam = fp_family(mode);
+    const int G = mode == QMV_NVFP4 ? 16 : 32;
+    return run(fam, x, w_packed, scales, nullptr, global_scale, y, M, N, K, 0, G, dtype, batch,
+               x_batched, stream);
+}
+
+int qmv_fp(const void* x, const void* w_packed, const void* scales, const float* global_scale, void* y,
+           int M, int N, int K, int mode, int dtype, void* stream) {
+    return qmv_fp_batched(x, w_packed, scales, global_scale, y, M, N, K, mode, dtype, 1, 1, stream);
+}
+
+int qmv_dequant_affine_f32(const void* w_packed, const void* scales, const void* biases, float* w_out,
+                           int N, int K, int bits, int group_size, int dtype, void* stream) {
+    int st = check_affine(bits, group_size);
+    if (st != QMV_OK) return st;
+    if (dtype != QMV_F32 && dtype != QMV_F16 && dtype != QMV_BF16) return QMV_EUNSUPPORTED;
+    if (N < 0 || K < 0 || K % group_size != 0) return QMV_EINVAL;
+    if (N == 0 || K == 0) return QMV_OK;
+    if (!w_packed || !scales || !biases || !w_out) return QMV_EINVAL;
+    const size_t eb = elem_bytes(dtype);
+    if (!aligned(w_packed, 4) || !aligned(scales, eb) || !aligned(biases, eb) || !aligned(w_out, 16))
+        return QMV_EALIGN;
+    return finish(qmv::launch_dequant(qmv::FAM_AFFINE, bits, dtype, static_cast<const uint8_t*>(w_packed),
+                                      scales, biases, nullptr, w_out, N, K, group_size,
+                                      (long long)K * bits / 8, static_cast<cudaStream_t>(stream)));
+}
+
+int qmv_dequant_fp_f32(const void* w_packed, const void* scales, const float* global_scale, float* w_out,
+                       int N, int K, int mode, void* stream) {
+    int st = check_fp(mode, K, global_scale);
+    if (st != QMV_OK) return st;
+    if (N < 0 || K < 0) return QMV_EINVAL;
+    if (N == 0 || K == 0) return QMV_OK;
+    if (!w_packed || !scales || !w_out) return QMV_EINVAL;
+    if (!aligned(w_packed, 4) || !aligned(w_out, 16)) return QMV_EALIGN;
+    const int fam = fp_family(mode);
+    const int bits = fam == qmv::FAM_MXFP8 ? 8 : 4;
+    return finish(qmv::launch_dequant(fam, bits, 0, static_cast<const uint8_t*>(w_packed), scales, nullptr,
+                                      global_scale, w_out, N, K, mode == QMV_NVFP4 ? 16 : 32,
+                                      (long long)K * bits / 8, static_cast<cudaStream_t>(stream)));
+}
+
+const char* qmv_status_string(int status) {
+    switch (status) {
+        case QMV_OK: return "ok";
+        case QMV_EINVAL: return "invalid argument";
+        case QMV_EUNSUPPORTED: return "unsupported bits, group size, mode, dtype or size";
+        case QMV_EALIGN: return "misaligned pointer";
+        case QMV_ECUDA: return "CUDA launch error";
+        default: return "unknown status";
+    }
+}
+
+int qmv_last_cuda_error(void) { return g_last_cuda; }
+
+int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size, int dtype, int w_align16,
+                      char* buf, int buflen) {
+    if (!buf || buflen <= 0) return QMV_EINVAL;
+    if (M < 1 || M > QMV_MAX_M || N < 1 || K < 0) return QMV_EINVAL;
+    int fam;
+    if (family == 0) {
+        if (check_affine(bits, group_size) != QMV_OK) return QMV_EUNSUPPORTED;
+        fam = qmv::FAM_AFFINE;
+    } else {
+        fam = fp_family(family - 1);
+        if (fam < 0) return QMV_EUNSUPPORTED;
+        bits = 0;
+    }
+    Plan pl;
+    int st = make_plan(fam, M, N, K, bits, dtype, w_align16 != 0, 1, &pl);
+    if (st != QMV_OK) return st;
+    snprintf(buf, (size_t)buflen,
+             "path=%s chunk=%d maxm=%d rows_per_warp=%d warps_k=%d warps_rows=%d tile_iters=%d "
+             "grid=%u block=%u smem=%zu",
+             pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr, pl.tile_iters,
+             pl.grid.x, pl.block.x, pl.smem);
+    return QMV_OK;
+}
+
+void qmv_force_config(int path, int rows_per_warp, int warps_k, int warps_rows) {
+    g_forced.path = path;
+    g_forced.R = rows_per_warp;
+    g_forced.wk = warps_k;
+    g_forced.wr = warps_rows;
+}
+
+}  // extern "C"

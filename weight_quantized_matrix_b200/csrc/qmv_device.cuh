@@ -1,0 +1,536 @@
+// qmv_device.cuh -- device code of the weight-quantized matrix-vector product
+// for sm_100a: per-format decoders, the warp-per-row-block qmv kernel and the
+// dequantization check kernel.
+//
+// Formats (see include/qmv.h for the page citations):
+//   affine  2/3/4/5/6/8-bit codes, LSB-first bit stream per row (MLX
+//           quantized_nax.h, get_pack_factor / get_bytes_per_pack, qdot),
+//           w = scale * q + bias per group of G codes;
+//   MXFP4 / NVFP4 / MXFP8: E2M1 or E4M3 elements with E8M0 (per 32) or E4M3
+//           (per 16, times an FP32 global) block scales (wh-iron audit, Track 1).
+//
+// Work decomposition (B200-first, not the pages' Metal layout):
+//   * The K axis of a row is cut into CHUNKS of C codes (C a multiple of 32).
+//     A chunk is U "units" of 32 codes; a unit of b-bit codes is exactly b
+//     32-bit words, so every unit has the same bit layout.  The wide path loads
+//     a chunk with 16-byte vector loads (C chosen so a chunk is a whole number
+//     of 16-byte vectors); the narrow path uses 4-byte loads and C = 32.
+//   * A block has wr x wk warps.  Warp (wr, wk) owns R consecutive rows; its 32
+//     lanes together with the other wk warps ("k-threads", kt = 32*wk + lane)
+//     take the chunks of those rows round-robin, so small N still spreads one
+//     row over up to 256 threads (split-K inside the block), and large N keeps
+//     wk = 1 with R rows sharing every x load.
+//   * x is staged per block in shared memory, widened to fp32 and PRE-SCALED
+//     per code position: a code whose field sits at bit p of the word it is
+//     masked from is used unshifted (value c * 2^p), so its x is stored as
+//     x * 2^-p (exact: a power-of-two scale).  This is the x pre-scaling of
+//     MLX's load_vector, re-derived for 32-bit words.  The integer field is
+//     turned into a float without an int->float conversion: OR-ing it into the
+//     mantissa of 2^23 and subtracting 2^23 is exact for fields below bit 23.
+//   * Affine groups: each lane keeps fp32 partials sum(x~ * c 2^p) per
+//     segment (the part of a group inside one chunk), then adds
+//     scale * partial + bias * sum(x), where sum(x) of the segment is formed in
+//     the staging pass from x values widened to fp32 one by one (the precision
+//     fix of the MLX pull request).
+//   * Products and partial sums use Blackwell's packed fp32x2 FMA/ADD.
+//   * Reduction: lane partials -> warp butterfly shuffle -> (wk > 1) shared
+//     memory across the k-warps -> one rounding to the output dtype.
+//   * Rows past N in the last block read the last valid row and are not stored
+//     (the row-tail rule of the MLX fast_rows kernels).
+//   * The kernel waits on the previous grid (griddepcontrol.wait) before its
+//     first global read, so it may be launched with programmatic dependent
+//     launch; it lets dependents launch once its main loop is done.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace qmv {
+
+enum Family { FAM_AFFINE = 0, FAM_MXFP4 = 1, FAM_NVFP4 = 2, FAM_MXFP8 = 3 };
+
+struct Params {
+    const void* x;          // [batch?][M][K] dtype
+    const uint8_t* w;       // [batch][N][row bytes]
+    const void* scales;     // [batch][N][K/G] (dtype for affine, u8 for FP)
+    const void* biases;     // [batch][N][K/G] dtype (affine)
+    const float* gscale;    // NVFP4: [batch] floats
+    void* y;                // [batch][M][N] dtype
+    int M, N, K, G;         // G: group (affine) or block (FP) size
+    int wk, wr;             // warps along K, warps along rows
+    int tile_iters;         // x tile = 32*wk*tile_iters chunks
+    int x_vec;              // 1: x rows are 16-byte aligned (vector staging loads)
+    long long x_bs;         // x batch stride in elements (0 = shared x)
+    long long w_bs;         // w batch stride in bytes
+    long long s_bs;         // scales/biases batch stride in elements
+    long long y_bs;         // y batch stride in elements
+    long long w_row;        // bytes per packed row
+};
+
+// ---------------------------------------------------------------- dtypes ---
+template <class T> struct DT;
+template <> struct DT<float> {
+    static __device__ __forceinline__ float ld(const void* p, long long i) {
+        return __ldg(reinterpret_cast<const float*>(p) + i);
+    }
+    static __device__ __forceinline__ void st(void* p, long long i, float v) {
+        reinterpret_cast<float*>(p)[i] = v;
+    }
+};
+template <> struct DT<__half> {
+    static __device__ __forceinline__ float ld(const void* p, long long i) {
+        return __half2float(reinterpret_cast<const __half*>(p)[i]);
+    }
+    static __device__ __forceinline__ void st(void* p, long long i, float v) {
+        reinterpret_cast<__half*>(p)[i] = __float2half_rn(v);
+    }
+};
+template <> struct DT<__nv_bfloat16> {
+    static __device__ __forceinline__ float ld(const void* p, long long i) {
+        return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+    }
+    static __device__ __forceinline__ void st(void* p, long long i, float v) {
+        reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+    }
+};
+
+// Widen 8 consecutive dtype elements loaded as one 16-byte vector.
+template <class T> __device__ __forceinline__ void widen8(const uint4& v, float* o);
+template <> __device__ __forceinline__ void widen8<__half>(const uint4& v, float* o) {
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { float2 f = __half22float2(h[i]); o[2 * i] = f.x; o[2 * i + 1] = f.y; }
+}
+template <> __device__ __forceinline__ void widen8<__nv_bfloat16>(const uint4& v, float* o) {
+    const uint32_t* u = reinterpret_cast<const uint32_t*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        o[2 * i] = __uint_as_float(u[i] << 16);
+        o[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+    }
+}
+
+// ------------------------------------------------------- packed fp32 math --
+// Blackwell fp32x2 instructions: two independent IEEE fp32 operations per
+// issue slot (round to nearest even, no contraction across the pair).
+__device__ __forceinline__ unsigned long long pk(float a, float b) {
+    return (unsigned long long)__float_as_uint(a) | ((unsigned long long)__float_as_uint(b) << 32);
+}
+__device__ __forceinline__ float lo(unsigned long long v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float hi(unsigned long long v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// ------------------------------------------------- grid dependency control --
+__device__ __forceinline__ void grid_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// -------------------------------------------------- affine field extraction --
+// Field j (0..31) of a 32-code unit of B-bit codes held in B 32-bit words
+// (little-endian, LSB-first stream): starts at bit o = B*j of the unit.
+//   * r + B <= 23       : mask in place, value c * 2^r          (p = r)
+//   * 23 < r + B <= 32  : mask the word shifted right by 9     (p = r - 9)
+//   * r + B > 32        : funnel-shift the word pair to bit 0  (p = 0)
+// In every case the masked field lies below bit 23, so OR-ing it into the
+// mantissa of 2^23 and subtracting 2^23 yields c * 2^p exactly.
+__host__ __device__ constexpr int field_p(int B, int j) {
+    return ((B * j) % 32 + B > 32) ? 0
+         : ((B * j) % 32 + B <= 23) ? (B * j) % 32
+         : (B * j) % 32 - 9;
+}
+
+template <int B, int J>
+__device__ __forceinline__ uint32_t field_bits(const uint32_t* w) {
+    constexpr int o = B * J, wi = o / 32, r = o % 32;
+    constexpr uint32_t m = (1u << B) - 1u;
+    if constexpr (r + B > 32) {
+        return __funnelshift_r(w[wi], w[wi + 1], r) & m;
+    } else if constexpr (r + B <= 23) {
+        return w[wi] & (m << r);
+    } else {
+        return (w[wi] >> 9) & (m << (r - 9));
+    }
+}
+
+__device__ __forceinline__ unsigned long long magic_pair(uint32_t a, uint32_t b) {
+    // {a, b} fields (< 2^23) -> {a, b} as exact floats
+    const unsigned long long m = pk(-8388608.0f, -8388608.0f);
+    return add2(((unsigned long long)(a | 0x4B000000u)) | ((unsigned long long)(b | 0x4B000000u) << 32), m);
+}
+
+// ------------------------------------------------------- FP element decode --
+// E2M1 nibble -> float: the 3 magnitude bits placed at fp32 bits 22..24 form
+// a number equal to the E2M1 magnitude times 2^-126 (the subnormal code lands
+// on an fp32 subnormal of the same ratio); the sign goes to bit 31.  One exact
+// multiply by 2^126 restores the value (wh-iron audit: bit-pattern decode
+// followed by an exact power-of-two multiply).
+__device__ __forceinline__ uint32_t e2m1_pattern(uint32_t nib) {
+    return ((nib & 7u) << 22) | ((nib & 8u) << 28);
+}
+__device__ __forceinline__ float e2m1_value(uint32_t nib) {
+    return __uint_as_float(e2m1_pattern(nib)) * 0x1p126f;
+}
+// E4M3 byte -> float: exponent+mantissa bits at fp32 bits 20..26, times 2^120;
+// S.1111.111 is NaN.
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+    c &= 0xFFu;
+    float v = __uint_as_float(((c & 0x7Fu) << 20) | ((c & 0x80u) << 24)) * 0x1p120f;
+    return ((c & 0x7Fu) == 0x7Fu) ? __uint_as_float(0x7FC00000u) : v;
+}
+// E8M0 byte -> 2^(e-127); e = 0 is the fp32 subnormal 2^-127; 0xFF is NaN.
+__device__ __forceinline__ float e8m0_value(uint32_t e) {
+    e &= 0xFFu;
+    return e == 0xFFu ? __uint_as_float(0x7FC00000u)
+         : e == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(e << 23);
+}
+
+// ----------------------------------------------------------- format traits --
+template <int FAM, int BITS> struct Fmt {
+    static constexpr int kBits = (FAM == FAM_AFFINE) ? BITS : (FAM == FAM_MXFP8 ? 8 : 4);
+    static constexpr int kUnitWords = kBits;                 // words per 32 codes
+    // Units per chunk on the wide path: the smallest whole number of units
+    // whose byte size is a multiple of 16 (and at least 32 bytes for 2/4-bit).
+    static constexpr int kWideUnits =
+        kBits == 2 ? 4 : kBits == 3 ? 4 : kBits == 4 ? 2 : kBits == 5 ? 4 : kBits == 6 ? 2 : 1;
+};
+
+// ------------------------------------------------------------ the kernel ----
+// Shared memory layout (floats):
+//   xs : [MAXM][tile_iters][C/4][KT] float4   pre-scaled x of the tile
+//   sx : [MAXM][tile_iters][U][KT]            affine: sum(x) per unit-run
+//   red: [wk][wr*R*MAXM]                       cross-warp partials
+// KT = 32*wk.  Chunk c of the tile belongs to k-thread c % KT, iteration c / KT.
+template <int FAM, int BITS, class T, int MAXM, int R, bool WIDE>
+__global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
+    using F = Fmt<FAM, BITS>;
+    constexpr int B = F::kBits;
+    constexpr int UW = F::kUnitWords;
+    constexpr int U = WIDE ? F::kWideUnits : 1;
+    constexpr int C = 32 * U;
+    constexpr int CW = UW * U;
+    constexpr bool AFF = (FAM == FAM_AFFINE);
+
+    extern __shared__ float4 smem4[];
+    const int KT = 32 * p.wk;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wkid = warp % p.wk, wrid = warp / p.wk;
+    const int kt = wkid * 32 + lane;
+    const int bz = blockIdx.z;
+    const int row0 = (blockIdx.x * p.wr + wrid) * R;
+    const int NC = p.K / C;
+    const int TI = p.tile_iters;
+    const int TC = KT * TI;
+    const int G = p.G;
+    const int KG = p.K / G;
+
+    float4* xs = smem4;                                                  // [MAXM][TI][C/4][KT]
+    float* sx = reinterpret_cast<float*>(xs + (size_t)MAXM * TI * (C / 4) * KT);  // [MAXM][TI][U][KT]
+    float* red = sx + (AFF ? (size_t)MAXM * TI * U * KT : 0);            // [wk][wr*R*MAXM]
+
+    const uint8_t* W = p.w + bz * p.w_bs;
+    const char* Xb = reinterpret_cast<const char*>(p.x) + bz * p.x_bs * (long long)sizeof(T);
+    const long long sb = bz * p.s_bs;
+
+    int rowc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) rowc[r] = min(row0 + r, p.N - 1);
+
+    float acc[R][MAXM];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) acc[r][m] = 0.f;
+
+    grid_wait();   // inputs may come from the previous kernel in the stream
+
+    for (int t0 = 0; t0 < NC; t0 += TC) {
+        const int tcn = min(TC, NC - t0);          // chunks in this tile
+        __syncthreads();
+        // ---- stage x: one work item = (m, chunk, unit) = 32 codes ----------
+        {
+            const int items = MAXM * tcn * U;
+            for (int it = threadIdx.x; it < items; it += blockDim.x) {
+                const int u = it % U;
+                const int cc = (it / U) % tcn;
+                const int m = it / (U * tcn);
+                const int i = cc / KT, ktt = cc % KT;
+                float v[32];
+                if (m < p.M) {
+                    const long long k0 = (long long)(t0 + cc) * C + u * 32;
+                    const T* xr = reinterpret_cast<const T*>(Xb) + (long long)m * p.K + k0;
+                    if constexpr (sizeof(T) == 2) {
+                        if (p.x_vec) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                uint4 vv = __ldg(reinterpret_cast<const uint4*>(xr) + q);
+                                widen8<T>(vv, v + 8 * q);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = DT<T>::ld(xr, j);
+                        }
+                    } else {
+                        if (p.x_vec) {
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                float4 f = __ldg(reinterpret_cast<const float4*>(xr) + q);
+                                v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = DT<T>::ld(xr, j);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = 0.f;
+                }
+                if constexpr (AFF) {
+                    float s = 0.f;                      // sum(x), widened per element
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) s += v[j];
+                    sx[(((size_t)m * TI + i) * U + u) * KT + ktt] = s;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(v[j], __uint_as_float((127u - field_p(B, j)) << 23));
+                }
+                float4* dst = xs + (((size_t)m * TI + i) * (C / 4) + u * 8) * KT + ktt;
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    dst[(size_t)q * KT] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            }
+        }
+        __syncthreads();
+
+        // ---- main loop over this k-thread's chunks of the tile --------------
+        for (int i = 0; i < TI; ++i) {
+            const int cc = i * KT + kt;
+            if (cc >= tcn) break;
+            const int c = t0 + cc;
+            // load the chunk of every row
+            uint32_t wv[R][CW];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const uint8_t* src = W + (long long)rowc[r] * p.w_row + (long long)c * (C * B / 8);
+                if constexpr (WIDE) {
+#pragma unroll
+                    for (int q = 0; q < CW / 4; ++q) {
+                        uint4 t = __ldg(reinterpret_cast<const uint4*>(src) + q);
+                        wv[r][4 * q] = t.x; wv[r][4 * q + 1] = t.y; wv[r][4 * q + 2] = t.z; wv[r][4 * q + 3] = t.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < CW; ++q) wv[r][q] = __ldg(reinterpret_cast<const uint32_t*>(src) + q);
+                }
+            }
+            // per-unit scale (affine: scale + bias of the unit's group;
+            // MX: one block scale; NV: two block scales per unit)
+            float sc[R][U][2], bi[R][U];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const long long k0 = (long long)c * C + u * 32;
+                    const long long rb = (long long)rowc[r] * KG;
+                    if constexpr (AFF) {
+                        const long long gi = sb + rb + k0 / G;
+                        sc[r][u][0] = DT<T>::ld(p.scales, gi);
+                        bi[r][u] = DT<T>::ld(p.biases, gi);
+                    } else if constexpr (FAM == FAM_NVFP4) {
+                        const uint8_t* s8 = reinterpret_cast<const uint8_t*>(p.scales) + sb + rb + k0 / 16;
+                        sc[r][u][0] = e4m3_value(__ldg(s8));
+                        sc[r][u][1] = e4m3_value(__ldg(s8 + 1));
+                    } else {
+                        const uint8_t* s8 = reinterpret_cast<const uint8_t*>(p.scales) + sb + rb + k0 / 32;
+                        sc[r][u][0] = e8m0_value(__ldg(s8));
+                    }
+                }
+
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                unsigned long long part[R][MAXM][2];      // NV: one per 16-code block
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+#pragma unroll
+                    for (int m = 0; m < MAXM; ++m) { part[r][m][0] = 0ull; part[r][m][1] = 0ull; }
+                const float4* xu = xs + ((size_t)i * (C / 4) + u * 8) * KT + kt;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {              // 4 codes per step
+                    float4 xv[MAXM];
+#pragma unroll
+                    for (int m = 0; m < MAXM; ++m) xv[m] = xu[((size_t)m * TI * (C / 4) + q) * KT];
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        const uint32_t* wu = &wv[r][u * UW];
+                        unsigned long long d0, d1;         // codes 4q..4q+3 as two float pairs
+                        if constexpr (AFF) {
+                            // unrolled field plan (compile-time per q)
+                            uint32_t f0, f1, f2, f3;
+                            switch (q) {
+#define QMV_F4(QQ) case QQ: f0 = field_bits<B, 4 * QQ>(wu); f1 = field_bits<B, 4 * QQ + 1>(wu); \
+                   f2 = field_bits<B, 4 * QQ + 2>(wu); f3 = field_bits<B, 4 * QQ + 3>(wu); break;
+                                QMV_F4(0) QMV_F4(1) QMV_F4(2) QMV_F4(3) QMV_F4(4) QMV_F4(5) QMV_F4(6) QMV_F4(7)
+#undef QMV_F4
+                                default: f0 = f1 = f2 = f3 = 0;
+                            }
+                            d0 = magic_pair(f0, f1);
+                            d1 = magic_pair(f2, f3);
+                        } else if constexpr (B == 4) {
+                            const uint32_t wd = wu[q >> 1] >> (16 * (q & 1));
+                            const unsigned long long s126 = pk(0x1p126f, 0x1p126f);
+                            d0 = mul2(pk(__uint_as_float(e2m1_pattern(wd)), __uint_as_float(e2m1_pattern(wd >> 4))), s126);
+                            d1 = mul2(pk(__uint_as_float(e2m1_pattern(wd >> 8)), __uint_as_float(e2m1_pattern(wd >> 12))), s126);
+                        } else {
+                            const uint32_t wd = wu[q];
+                            d0 = pk(e4m3_value(wd), e4m3_value(wd >> 8));
+                            d1 = pk(e4m3_value(wd >> 16), e4m3_value(wd >> 24));
+                        }
+                        constexpr int blk = 0;
+                        const int h = (FAM == FAM_NVFP4) ? (q >> 2) : blk;   // 16-code block within the unit
+#pragma unroll
+                        for (int m = 0; m < MAXM; ++m) {
+                            unsigned long long a = part[r][m][h];
+                            a = fma2(pk(xv[m].x, xv[m].y), d0, a);
+                            a = fma2(pk(xv[m].z, xv[m].w), d1, a);
+                            part[r][m][h] = a;
+                        }
+                    }
+                }
+                // epilogue of the unit
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+#pragma unroll
+                    for (int m = 0; m < MAXM; ++m) {
+                        if constexpr (AFF) {
+                            const float s = sx[(((size_t)m * TI + i) * U + u) * KT + kt];
+                            const float pr = lo(part[r][m][0]) + hi(part[r][m][0]);
+                            acc[r][m] = fmaf(sc[r][u][0], pr, fmaf(bi[r][u], s, acc[r][m]));
+                        } else if constexpr (FAM == FAM_NVFP4) {
+                            acc[r][m] = fmaf(sc[r][u][0], lo(part[r][m][0]) + hi(part[r][m][0]), acc[r][m]);
+                            acc[r][m] = fmaf(sc[r][u][1], lo(part[r][m][1]) + hi(part[r][m][1]), acc[r][m]);
+                        } else {
+                            acc[r][m] = fmaf(sc[r][u][0], lo(part[r][m][0]) + hi(part[r][m][0]), acc[r][m]);
+                        }
+                    }
+            }
+        }
+    }
+
+    grid_launch_dependents();
+
+    // ---- reduction: warp butterfly, then across the k-warps -----------------
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) {
+            float v = acc[r][m];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+            acc[r][m] = v;
+        }
+    float gs = 1.f;
+    if constexpr (FAM == FAM_NVFP4) gs = __ldg(p.gscale + bz);
+    T* Y = reinterpret_cast<T*>(p.y) + bz * p.y_bs;
+    const int RM = R * MAXM;
+    if (p.wk == 1) {
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m)
+                if (lane == r * MAXM + m && row0 + r < p.N && m < p.M)
+                    DT<T>::st(Y, (long long)m * p.N + row0 + r, acc[r][m] * gs);
+    } else {
+        if (lane == 0) {
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int m = 0; m < MAXM; ++m) red[(wkid * p.wr + wrid) * RM + r * MAXM + m] = acc[r][m];
+        }
+        __syncthreads();
+        const int tot = p.wr * RM;
+        for (int t = threadIdx.x; t < tot; t += blockDim.x) {
+            float v = 0.f;
+            for (int k = 0; k < p.wk; ++k) v += red[k * tot + t];
+            const int wr_ = t / RM, rm = t % RM, r = rm / MAXM, m = rm % MAXM;
+            const int row = (blockIdx.x * p.wr + wr_) * R + r;
+            if (row < p.N && m < p.M) DT<T>::st(Y, (long long)m * p.N + row, v * gs);
+        }
+    }
+}
+
+// ------------------------------------------------- dequantization check ----
+// One thread per 32-code unit of one row; writes 32 fp32 weights.
+//   affine: fmaf(scale, c, bias) with c = (c * 2^p) * 2^-p (exact)
+//   MX:     elem * e8m0 (exact in fp32)
+//   NV:     (elem * e4m3) * global (the first product exact, one rounding)
+template <int FAM, int BITS, class T>
+__global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict__ w,
+                                                      const void* scales, const void* biases,
+                                                      const float* gscale, float* __restrict__ out,
+                                                      int N, int K, int G, long long w_row) {
+    using F = Fmt<FAM, BITS>;
+    constexpr int B = F::kBits;
+    const long long units = (long long)N * (K / 32);
+    grid_wait();
+    for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < units;
+         t += (long long)gridDim.x * blockDim.x) {
+        const long long n = t / (K / 32);
+        const int u = (int)(t % (K / 32));
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(w + n * w_row + (long long)u * 4 * B);
+        uint32_t wv[B];
+#pragma unroll
+        for (int q = 0; q < B; ++q) wv[q] = __ldg(src + q);
+        float o[32];
+        const long long k0 = (long long)u * 32;
+        if constexpr (FAM == FAM_AFFINE) {
+            const long long gi = n * (K / G) + k0 / G;
+            const float s = DT<T>::ld(scales, gi), b = DT<T>::ld(biases, gi);
+#define QMV_D4(QQ) { unsigned long long d0 = magic_pair(field_bits<B, 4 * QQ>(wv), field_bits<B, 4 * QQ + 1>(wv)); \
+                     unsigned long long d1 = magic_pair(field_bits<B, 4 * QQ + 2>(wv), field_bits<B, 4 * QQ + 3>(wv)); \
+                     float c[4] = {lo(d0), hi(d0), lo(d1), hi(d1)}; \
+                     _Pragma("unroll") for (int e = 0; e < 4; ++e) { \
+                         const float q_ = __fmul_rn(c[e], __uint_as_float((127u - field_p(B, 4 * QQ + e)) << 23)); \
+                         o[4 * QQ + e] = fmaf(s, q_, b); } }
+            QMV_D4(0) QMV_D4(1) QMV_D4(2) QMV_D4(3) QMV_D4(4) QMV_D4(5) QMV_D4(6) QMV_D4(7)
+#undef QMV_D4
+        } else if constexpr (B == 4) {
+            const uint8_t* s8 = reinterpret_cast<const uint8_t*>(scales) + n * (K / G);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float e = e2m1_value(wv[j / 8] >> (4 * (j % 8)));
+                if constexpr (FAM == FAM_NVFP4) {
+                    o[j] = __fmul_rn(__fmul_rn(e, e4m3_value(__ldg(s8 + (k0 + j) / 16))), __ldg(gscale));
+                } else {
+                    o[j] = __fmul_rn(e, e8m0_value(__ldg(s8 + (k0 + j) / 32)));
+                }
+            }
+        } else {
+            const uint8_t* s8 = reinterpret_cast<const uint8_t*>(scales) + n * (K / G);
+            const float s = e8m0_value(__ldg(s8 + k0 / 32));
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __fmul_rn(e4m3_value(wv[j / 4] >> (8 * (j % 4))), s);
+        }
+        float4* dst = reinterpret_cast<float4*>(out + n * (long long)K + k0);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    }
+}
+
+}  // namespace qmv

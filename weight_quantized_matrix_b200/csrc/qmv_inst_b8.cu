@@ -1,0 +1,14 @@
+// qmv_inst_b8.cu -- affine 8-bit qmv kernels (all dtypes and launch shapes).
+#include "qmv_launch.cuh"
+
+namespace qmv {
+
+cudaError_t launch_affine_b8(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L) {
+#define FAM_ FAM_AFFINE
+#define BITS_ 8
+    QMV_DISPATCH_DTYPE()
+#undef FAM_
+#undef BITS_
+}
+
+}  // namespace qmv

@@ -1,0 +1,94 @@
+// qmv_launch.cuh -- host-side launch helpers shared by the instantiation units
+// and the C ABI.  Each instantiation unit (qmv_inst_*.cu) compiles one family
+// of kernels and exposes one dispatcher declared here.
+#pragma once
+
+#include <atomic>
+#include <cuda_runtime.h>
+#include "qmv_device.cuh"
+
+namespace qmv {
+
+// Launch shape chosen by the picker (qmv_api.cu).
+struct Launch {
+    dim3 grid, block;
+    size_t smem;
+    cudaStream_t stream;
+    bool pdl;        // programmatic dependent launch
+};
+
+// Largest dynamic shared memory any kernel here asks for; set once per
+// (kernel, device) before the first launch.
+constexpr int kMaxSmem = 200 * 1024;
+
+template <class Kern>
+inline cudaError_t launch_kernel(Kern kern, std::atomic<unsigned>& configured, const Launch& L,
+                                 const Params& p) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned bit = 1u << (dev & 31);
+    if (!(configured.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = L.grid;
+    cfg.blockDim = L.block;
+    cfg.dynamicSmemBytes = L.smem;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = L.pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+// dtype: 0 f32, 1 f16, 2 bf16.  Returns cudaErrorInvalidValue for a
+// (maxm, R, wide) combination that is not instantiated.
+cudaError_t launch_affine_b2(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_affine_b3(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_affine_b4(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_affine_b5(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_affine_b6(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_affine_b8(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_fp(int fam, int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+
+cudaError_t launch_dequant(int fam, int bits, int dtype, const uint8_t* w, const void* scales,
+                           const void* biases, const float* gscale, float* out, int N, int K, int G,
+                           long long w_row, cudaStream_t s);
+
+// Which (maxm, R, wide) shapes exist.
+inline bool shape_instantiated(int maxm, int R, bool wide) {
+    if (!wide) return R == 1 && (maxm == 1 || maxm == 2 || maxm == 4 || maxm == 8);
+    if (maxm == 1 || maxm == 2) return R == 1 || R == 2 || R == 4;
+    if (maxm == 4 || maxm == 8) return R == 1 || R == 2;
+    return false;
+}
+
+}  // namespace qmv
+
+// Dispatch body shared by the instantiation units: FAM/BITS fixed, switch on
+// dtype and shape.
+#define QMV_SHAPE(T_, MAXM_, R_, WIDE_)                                                      \
+    if (maxm == MAXM_ && R == R_ && wide == WIDE_) {                                         \
+        static std::atomic<unsigned> cfg_{0};                                                \
+        return launch_kernel(qmv_kernel<FAM_, BITS_, T_, MAXM_, R_, WIDE_>, cfg_, L, p);     \
+    }
+#define QMV_ALL_SHAPES(T_)                                                                   \
+    QMV_SHAPE(T_, 1, 1, true) QMV_SHAPE(T_, 1, 2, true) QMV_SHAPE(T_, 1, 4, true)            \
+    QMV_SHAPE(T_, 2, 1, true) QMV_SHAPE(T_, 2, 2, true) QMV_SHAPE(T_, 2, 4, true)            \
+    QMV_SHAPE(T_, 4, 1, true) QMV_SHAPE(T_, 4, 2, true)                                      \
+    QMV_SHAPE(T_, 8, 1, true) QMV_SHAPE(T_, 8, 2, true)                                      \
+    QMV_SHAPE(T_, 1, 1, false) QMV_SHAPE(T_, 2, 1, false) QMV_SHAPE(T_, 4, 1, false)         \
+    QMV_SHAPE(T_, 8, 1, false)
+#define QMV_DISPATCH_DTYPE()                                                                 \
+    switch (dtype) {                                                                         \
+        case 0: { QMV_ALL_SHAPES(float) break; }                                             \
+        case 1: { QMV_ALL_SHAPES(__half) break; }                                            \
+        case 2: { QMV_ALL_SHAPES(__nv_bfloat16) break; }                                     \
+        default: break;                                                                      \
+    }                                                                                        \
+    return cudaErrorInvalidValue;
