@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Benchmark of the weight-quantized matrix-vector product on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload chain8|layer|probe]
+
+Prints ONE JSON line (rank 0).  Metric: qmv microseconds per call and achieved
+HBM GB/s.  Workloads (synthetic, seeded; see the design doc for the recipes):
+
+  chain8 (default)  affine 8-bit, group 64, bf16, M=1, K=2560, output sizes
+                    N in {1, 4, 3, 5, 12, 17, 4096}; for each N a chain of 64
+                    dependent calls in which call t reads the previous output
+                    zero-padded (N < K) or truncated (N >= K) to K.  One step =
+                    all seven chains = 448 calls.
+  layer             7B-class decode layer, affine 4-bit g64 bf16: QKV 6144x4096,
+                    O 4096x4096, gate+up 28672x4096, down 4096x14336, run once at
+                    M=1 and once at M=8 (8 calls per step).
+  probe             bandwidth probe, affine 4-bit g64 bf16, N=K=16384, M=1.
+
+Timing: W untimed warm-up steps, then K steps; each step is bracketed by CUDA
+events on the launching stream; L2 is flushed (a 512 MB buffer is written)
+before every step, outside the events, and within a step the weights rotate
+through copies totalling more than twice the L2 so calls read from HBM.  The
+timed region is bracketed by a barrier and a device synchronize; multi-GPU runs
+are N independent replicas (the path has no exchange step) and report the max
+over ranks.  nvidia-smi clocks are sampled during the timed region.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+this operation there is) on a bounded sample of the same workload, on the host
+cores, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+CHAIN_NS = [1, 4, 3, 5, 12, 17, 4096]
+CHAIN_K, CHAIN_BITS, CHAIN_G, CHAIN_CALLS = 2560, 8, 64, 64
+LAYER = [("qkv", 6144, 4096), ("o", 4096, 4096), ("gate_up", 28672, 4096), ("down", 4096, 14336)]
+METRIC = "qmv µs/call and achieved HBM GB/s (% of B200 peak) per format/bits/shape"
+
+
+def affine_bytes(M, N, K, bits, g, eb=2):
+    """Algorithmic bytes of one call: packed W + scales + biases + x + y."""
+    return N * K * bits // 8 + 2 * N * (K // g) * eb + M * K * eb + M * N * eb
+
+
+# ------------------------------------------------------------------ peaks --
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "weight_quantized_matrix_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel_key):
+    """dram bytes per launch from the committed ncu summary, only while the
+    kernel sources are unchanged since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+    except ValueError:
+        return None
+    e = d.get(kernel_key)
+    if not e or e.get("src_sha") != source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------- clocks --
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [r.split(", ") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            if len(r) < 9:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip() == "Active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# -------------------------------------------------------------- workloads --
+class Chain8:
+    """The chained 8-bit qmv workload (one step = 7 chains x 64 calls)."""
+    name = "chained affine 8-bit g64 bf16 qmv, M=1, K=2560, N in {1,4,3,5,12,17,4096}, 64 calls per N"
+
+    def __init__(self, q, torch, dev):
+        self.q, self.torch = q, torch
+        self.sets = []
+        for N in CHAIN_NS:
+            c = synth.affine_case(1, N, CHAIN_K, CHAIN_BITS, CHAIN_G, "bf16", seed=1000 + N)
+            per = affine_bytes(1, N, CHAIN_K, CHAIN_BITS, CHAIN_G) - CHAIN_K * 2 - N * 2
+            copies = int(min(CHAIN_CALLS, max(1, np.ceil(2 * L2_BYTES / per))))
+            ws = []
+            for i in range(copies):
+                ws.append(tuple(torch.from_numpy(np.ascontiguousarray(a).view(np.uint8).reshape(-1)).to(dev)
+                                for a in (c["w"], c["scales"], c["biases"])))
+            Lb = max(N, CHAIN_K)
+            x0_host = torch.zeros(Lb, dtype=torch.bfloat16).pin_memory()
+            x0_host[:CHAIN_K] = torch.from_numpy(c["x"][0, 0].view(np.int16)).view(torch.bfloat16)
+            x0 = x0_host.to(dev)
+            bufs = [torch.zeros(Lb, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+            y_host = torch.empty(N, dtype=torch.bfloat16).pin_memory()
+            self.sets.append(dict(N=N, ws=ws, x0=x0, x0_host=x0_host, bufs=bufs, y_host=y_host))
+        self.calls_per_step = CHAIN_CALLS * len(CHAIN_NS)
+        self.kernel_key = {}
+
+    def groups(self):
+        return [(f"N={s['N']}", s) for s in self.sets]
+
+    def graph_variants(self, s):
+        return 1          # the weight rotation is inside the chain
+
+    def run_group(self, s, e2e=False):
+        q, N = self.q, s["N"]
+        if e2e:
+            s["x0"].copy_(s["x0_host"], non_blocking=True)
+        bufs, ws = s["bufs"], s["ws"]
+        for t in range(CHAIN_CALLS):
+            xin = s["x0"] if t == 0 else bufs[(t - 1) % 2]
+            w, sc, bi = ws[t % len(ws)]
+            q.qmv_affine(xin, w, sc, bi, bufs[t % 2], 1, N, CHAIN_K, CHAIN_BITS, CHAIN_G, "bf16")
+        if e2e:
+            s["y_host"].copy_(bufs[(CHAIN_CALLS - 1) % 2][:N], non_blocking=True)
+        return CHAIN_CALLS
+
+    def group_bytes(self, s):
+        return affine_bytes(1, s["N"], CHAIN_K, CHAIN_BITS, CHAIN_G) * CHAIN_CALLS
+
+    def group_plan(self, s):
+        return self.q.qmv_describe_plan("affine", 1, s["N"], CHAIN_K, CHAIN_BITS, CHAIN_G, "bf16")
+
+    def h2d_d2h(self):
+        return (sum(CHAIN_K * 2 for _ in self.sets) + sum(max(s["N"], CHAIN_K) * 2 - CHAIN_K * 2 for s in self.sets),
+                sum(s["N"] * 2 for s in self.sets))
+
+    def config(self):
+        return {"workload": self.name, "bits": 8, "group": 64, "dtype": "bf16", "M": 1, "K": CHAIN_K,
+                "N": CHAIN_NS, "calls_per_N": CHAIN_CALLS, "calls_per_step": self.calls_per_step,
+                "chain": "x_{t+1} = y_t zero-padded (N<K) / truncated (N>=K) to K",
+                "l2": "flushed before every step (512 MB write); weights rotate through copies > 2x L2"}
+
+
+class Layer:
+    """7B-class decode layer, 4-bit g64 bf16, the four projections at M=1 and M=8."""
+    name = "7B-class decode layer, affine 4-bit g64 bf16, QKV/O/gate+up/down at M=1 and M=8"
+
+    def __init__(self, q, torch, dev):
+        self.q, self.torch = q, torch
+        self.sets = []
+        for M in (1, 8):
+            for name, N, K in LAYER:
+                c = synth.affine_case(M, N, K, 4, 64, "bf16", seed=2000 + N + K + M)
+                per = affine_bytes(M, N, K, 4, 64)
+                copies = int(max(1, min(8, np.ceil(2 * L2_BYTES / per))))
+                ws = [tuple(torch.from_numpy(np.ascontiguousarray(a).view(np.uint8).reshape(-1)).to(dev)
+                            for a in (c["w"], c["scales"], c["biases"])) for _ in range(copies)]
+                x_host = torch.from_numpy(c["x"][0].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+                x = x_host.to(dev)
+                y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+                y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+                self.sets.append(dict(name=name, M=M, N=N, K=K, ws=ws, x=x, x_host=x_host, y=y, y_host=y_host, it=0))
+        self.calls_per_step = len(self.sets)
+
+    def groups(self):
+        return [(f"{s['name']} M={s['M']}", s) for s in self.sets]
+
+    def graph_variants(self, s):
+        return len(s["ws"])   # one graph per weight copy; step k replays copy k
+
+    def run_group(self, s, e2e=False):
+        if e2e:
+            s["x"].copy_(s["x_host"], non_blocking=True)
+        w, sc, bi = s["ws"][s["it"] % len(s["ws"])]
+        s["it"] += 1
+        self.q.qmv_affine(s["x"], w, sc, bi, s["y"], s["M"], s["N"], s["K"], 4, 64, "bf16")
+        if e2e:
+            s["y_host"].copy_(s["y"], non_blocking=True)
+        return 1
+
+    def group_bytes(self, s):
+        return affine_bytes(s["M"], s["N"], s["K"], 4, 64)
+
+    def group_plan(self, s):
+        return self.q.qmv_describe_plan("affine", s["M"], s["N"], s["K"], 4, 64, "bf16")
+
+    def h2d_d2h(self):
+        return (sum(s["M"] * s["K"] * 2 for s in self.sets), sum(s["M"] * s["N"] * 2 for s in self.sets))
+
+    def config(self):
+        return {"workload": self.name, "bits": 4, "group": 64, "dtype": "bf16", "M": [1, 8],
+                "shapes_NxK": [[n, k] for _, n, k in LAYER], "calls_per_step": self.calls_per_step,
+                "l2": "flushed before every step (512 MB write); weights rotate through copies > 2x L2"}
+
+
+class Probe(Layer):
+    name = "bandwidth probe, affine 4-bit g64 bf16, N=K=16384, M=1"
+
+    def __init__(self, q, torch, dev):
+        self.q, self.torch = q, torch
+        c = synth.affine_case(1, 16384, 16384, 4, 64, "bf16", seed=3000)
+        ws = [tuple(torch.from_numpy(np.ascontiguousarray(a).view(np.uint8).reshape(-1)).to(dev)
+                    for a in (c["w"], c["scales"], c["biases"])) for _ in range(3)]
+        x_host = torch.from_numpy(c["x"][0].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+        self.sets = [dict(name="probe", M=1, N=16384, K=16384, ws=ws, x=x_host.to(dev), x_host=x_host,
+                          y=torch.empty((1, 16384), dtype=torch.bfloat16, device=dev),
+                          y_host=torch.empty((1, 16384), dtype=torch.bfloat16).pin_memory(), it=0)]
+        self.calls_per_step = 1
+
+    def config(self):
+        return {"workload": self.name, "bits": 4, "group": 64, "dtype": "bf16", "M": 1, "N": 16384, "K": 16384,
+                "calls_per_step": 1, "l2": "flushed before every step (512 MB write); 3 weight copies rotate"}
+
+
+WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe}
+
+
+# ---------------------------------------------------------------- our arm --
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: a CUDA device is required for --impl ours")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    import weight_quantized_matrix_b200 as q   # fails loudly if libqmv.so is missing
+
+    wl = WORKLOADS[args.workload](q, torch, dev)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    groups = wl.groups()
+    W = max(3, args.warmup)
+
+    with torch.cuda.stream(stream):
+        # eager warm-up through the public API (also sets kernel attributes)
+        for _ in range(W):
+            for _, s in groups:
+                wl.run_group(s)
+        torch.cuda.synchronize()
+        # one CUDA graph per group and weight copy: the chain's 64 dependent
+        # launches (with their programmatic-dependent-launch edges) replay
+        # without host overhead
+        graphs = []
+        for _, s in groups:
+            gs = []
+            for _ in range(wl.graph_variants(s)):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    wl.run_group(s)
+                gs.append(g)
+            graphs.append(gs)
+        for k in range(W):
+            for gs in graphs:
+                gs[k % len(gs)].replay()
+        torch.cuda.synchronize()
+
+        def timed(e2e):
+            ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in groups] for _ in range(args.steps)]
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            clk = ClockSampler(local_rank)
+            if not e2e:
+                clk.start()
+            t0 = time.perf_counter()
+            for k in range(args.steps):
+                flush.fill_(k & 0xFF)                   # L2 flush, outside the events
+                for gi, (_, s) in enumerate(groups):
+                    ev[k][gi][0].record(stream)
+                    if e2e:
+                        wl.run_group(s, e2e=True)       # public API, host copies included
+                    else:
+                        gs = graphs[gi]
+                        gs[k % len(gs)].replay()
+                    ev[k][gi][1].record(stream)
+            torch.cuda.synchronize()
+            wall = time.perf_counter() - t0
+            clocks = clk.stop() if not e2e else None
+            if world > 1:
+                dist.barrier()
+            per_group = np.array([[a.elapsed_time(b) for (a, b) in ev[k]] for k in range(args.steps)])  # ms
+            return per_group, wall, clocks
+
+        per_group, wall, clocks = timed(False)
+        per_group_e2e, _, _ = timed(True)
+        del graphs
+
+    step_ms = per_group.sum(axis=1)           # device time of each step
+    step_ms_e2e = per_group_e2e.sum(axis=1)
+    tot_ms = float(step_ms.sum())
+    tot_ms_e2e = float(step_ms_e2e.sum())
+    if world > 1:
+        t = torch.tensor([tot_ms, tot_ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms, tot_ms_e2e = float(t[0]), float(t[1])
+    calls = wl.calls_per_step * args.steps * world
+    us_per_call = tot_ms * 1e3 / calls
+    us_per_call_e2e = tot_ms_e2e * 1e3 / calls
+
+    # per-shape results and the dominant kernel (largest share of device time)
+    shapes, by_kernel = [], {}
+    peak, peak_kind = peaks()
+    for gi, (label, s) in enumerate(groups):
+        ms = float(per_group[:, gi].mean())
+        n = wl.calls_per_step // len(groups) if isinstance(wl, Chain8) else 1
+        b = wl.group_bytes(s)
+        plan = wl.group_plan(s)
+        gbs = b / (ms * 1e-3) / 1e9
+        shapes.append({"shape": label, "us_per_call": round(ms * 1e3 / n, 3), "GB_s": round(gbs, 1),
+                       "frac_of_hbm": round(gbs / peak, 4), "plan": plan})
+        k = by_kernel.setdefault(plan, {"ms": 0.0, "launches": 0, "bytes": 0})
+        k["ms"] += ms; k["launches"] += n; k["bytes"] += b
+    dom_plan, dom = max(by_kernel.items(), key=lambda kv: kv[1]["ms"])
+    achieved = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
+    traffic = traffic_for(dom_plan)
+    h2d, d2h = wl.h2d_d2h()
+    out = {
+        "metric": METRIC, "value": round(us_per_call, 4), "unit": "us/call", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(tot_ms / args.steps, 4),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in/out, fp32 accumulate",
+        "data": "synthetic (seeded)", "config": dict(wl.config(), parallelism=f"replicas x{world}"),
+        "e2e": {"value": round(us_per_call_e2e, 4), "unit": "us/call", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": wl.calls_per_step * args.steps,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
+                     "kernel": dom_plan, "kernel_share": round(dom["ms"] / sum(v["ms"] for v in by_kernel.values()), 3),
+                     "bytes_per_launch": dom["bytes"] // max(1, dom["launches"]),
+                     "avg_launch_us": round(dom["ms"] * 1e3 / max(1, dom["launches"]), 3)},
+        "clocks": clocks, "shapes": shapes, "wall_s_timed": round(wall, 3),
+    }
+    if rank == 0:
+        out["cpu_baseline"] = cpu_baseline(args.workload)
+        print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------- oracle (CPU) baseline --
+def _oracle_sample(workload, budget_s=12.0):
+    """Time the oracle, as it stands, on a bounded sample of the workload and
+    scale to microseconds per call of the full workload."""
+    import oracle
+    threads = os.cpu_count() or 1
+    t_by = {}
+    if workload == "chain8":
+        spec = [(1, N, CHAIN_K, CHAIN_BITS, CHAIN_G, CHAIN_CALLS) for N in CHAIN_NS]
+    elif workload == "layer":
+        spec = [(M, N, K, 4, 64, 1) for M in (1, 8) for _, N, K in LAYER]
+    else:
+        spec = [(1, 16384, 16384, 4, 64, 1)]
+    per_shape_budget = budget_s / len(spec)
+    sample = []
+    total_us = 0.0
+    for (M, N, K, bits, g, calls) in spec:
+        c = synth.affine_case(M, N, K, bits, g, "bf16", seed=7)
+        args = (c["x"][0], c["w"][0], c["scales"][0], c["biases"][0], M, N, K, bits, g, "bf16")
+        rows_all = list(range(N))
+        # grow the row sample until the budget for this shape is used
+        nrows = min(N, 64)
+        t0 = time.perf_counter()
+        oracle.qmv_affine(*args, rows=rows_all[:nrows], threads=threads)
+        dt = time.perf_counter() - t0
+        while nrows < N and dt < per_shape_budget / 4:
+            nrows = min(N, nrows * 4)
+            t0 = time.perf_counter()
+            oracle.qmv_affine(*args, rows=rows_all[:nrows], threads=threads)
+            dt = time.perf_counter() - t0
+        us_call = dt * 1e6 * (N / nrows)
+        total_us += us_call * calls
+        sample.append(f"M={M} N={N} K={K}: {nrows}/{N} rows, {dt:.3f}s")
+    ncalls = sum(s[-1] for s in spec)
+    return total_us / ncalls, threads, "; ".join(sample)
+
+
+def cpu_baseline(workload):
+    v, cores, sample = _oracle_sample(workload)
+    return {"value": round(v, 2), "unit": "us/call", "cores": cores, "kind": "oracle",
+            "sample": "fp64 C oracle over row samples of every shape, scaled to full calls: " + sample}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl = {"chain8": Chain8, "layer": Layer, "probe": Probe}[args.workload]
+    vals = []
+    for _ in range(max(1, args.warmup) if False else 0):
+        pass
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, cores, sample = _oracle_sample(args.workload, budget_s=6.0)
+        vals.append(v)
+    v = float(np.mean(vals))
+    cfg = {"workload": wl.name}
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "us/call", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)", "config": cfg,
+        "ms_per_step": round((time.perf_counter() - t0) * 1e3 / max(1, args.steps), 2),
+        "cpu_baseline": {"value": round(v, 2), "unit": "us/call", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(v, 2), "unit": "us/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="chain8")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
