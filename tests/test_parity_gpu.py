@@ -333,7 +333,8 @@ def test_empty_m_or_n_leaves_y(q):
 
 
 @pytest.mark.parametrize("cfg", [(1, 1, 1, 1), (1, 2, 1, 4), (1, 4, 1, 2), (1, 1, 8, 1), (1, 1, 3, 2),
-                                 (0, 1, 1, 4), (0, 1, 4, 2), (1, 2, 2, 4)])
+                                 (0, 1, 1, 4), (0, 1, 4, 2), (1, 2, 2, 4), (2, -1, -1, 8), (2, 2, -1, 4),
+                                 (2, 4, -1, 2)])
 @pytest.mark.parametrize("bits", [3, 4, 8])
 def test_forced_launch_shapes(q, cfg, bits):
     """Every launch shape the picker can choose gives the same (tolerance) answer."""

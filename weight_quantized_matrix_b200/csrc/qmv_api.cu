@@ -64,10 +64,17 @@ FmtInfo fmt_info(int fam, int bits) {
 }
 
 struct Plan {
-    int maxm, R, wide, wk, wr, tile_iters, C;
+    int maxm, R, wide, stream, wk, wr, tile_iters, C;
     size_t smem;
     dim3 grid, block;
 };
+
+// Rows per warp of the streaming kernel: enough rows to share each x load,
+// few enough that the ring stage and the chunk registers stay small.
+int stream_rows(int bits, int maxm) {
+    if (maxm <= 2) return (bits == 3 || bits == 5 || bits == 6) ? 2 : 4;
+    return (bits == 5 || maxm == 8) ? 1 : 2;
+}
 
 int rows_per_warp_cap(int bits, int maxm) {
     if (maxm <= 2) return (bits == 3 || bits == 5 || bits == 6) ? 2 : 4;
@@ -82,6 +89,30 @@ int make_plan(int fam, int M, int N, int K, int bits, int dtype, bool w16, int b
     const int c_wide = 32 * fi.wide_units;
     bool wide = w16 && (K % c_wide == 0);
     if (g_forced.path == 0) wide = false;
+
+    // ---- streaming kernel (large N, wide chunks, x fits in shared memory) ----
+    if (wide && K > 0 && g_forced.path == 2) {
+        const int U = fi.wide_units, C = 32 * U, CB = C * fi.bits / 8;
+        const int NC = K / C, I = (NC + 31) / 32;
+        int Rs = stream_rows(fi.bits, maxm);
+        if (g_forced.R > 0 && qmv::stream_instantiated(maxm, g_forced.R)) Rs = g_forced.R;
+        const size_t xs = (size_t)maxm * I * C * 32 * 4;
+        const size_t sxb = aff ? (size_t)maxm * I * U * 32 * 4 : 0;
+        const size_t ring_w = (size_t)qmv::kStreamStages * Rs * CB * 32;
+        const size_t avail = (size_t)qmv::kMaxSmem > xs + sxb ? (size_t)qmv::kMaxSmem - xs - sxb : 0;
+        int NW = (int)(avail / ring_w);
+        if (NW > 8) NW = 8;
+        if (g_forced.wr > 0 && g_forced.wr <= NW) NW = g_forced.wr;
+        if (NW >= 2 || (g_forced.path == 2 && NW >= 1)) {
+            const long long nrb = ((long long)N + Rs - 1) / Rs;
+            const long long gx = (nrb + NW - 1) / NW;
+            pl->maxm = maxm; pl->R = Rs; pl->wide = 1; pl->stream = 1; pl->wk = 1; pl->wr = NW;
+            pl->tile_iters = I; pl->C = C; pl->smem = xs + sxb + NW * ring_w;
+            pl->grid = dim3((unsigned)gx, 1, (unsigned)batch);
+            pl->block = dim3(32 * NW, 1, 1);
+            return QMV_OK;
+        }
+    }
     if (g_forced.path == 1 && w16 && (K % c_wide == 0)) wide = true;
     const int U = wide ? fi.wide_units : 1;
     const int C = 32 * U;
@@ -138,7 +169,7 @@ int make_plan(int fam, int M, int N, int K, int bits, int dtype, bool w16, int b
     const long long gx = ((long long)N + rows_per_block - 1) / rows_per_block;
     if (gx > 0x7FFFFFFFLL) return QMV_EINVAL;
 
-    pl->maxm = maxm; pl->R = R; pl->wide = wide; pl->wk = wk; pl->wr = wr;
+    pl->maxm = maxm; pl->R = R; pl->wide = wide; pl->stream = 0; pl->wk = wk; pl->wr = wr;
     pl->tile_iters = (int)ti; pl->C = C; pl->smem = smem;
     pl->grid = dim3((unsigned)gx, 1, (unsigned)batch);
     pl->block = dim3(32 * wk * wr, 1, 1);
@@ -195,6 +226,11 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     p.w_row = row_bytes;
     qmv::Launch L{pl.grid, pl.block, pl.smem, static_cast<cudaStream_t>(stream), pdl_enabled()};
     cudaError_t e;
+    if (pl.stream) {
+        e = fam == qmv::FAM_AFFINE ? qmv::launch_stream_affine(bits, dtype, pl.maxm, pl.R, p, L)
+                                   : qmv::launch_stream_fp(fam, dtype, pl.maxm, pl.R, p, L);
+        return finish(e);
+    }
     if (fam == qmv::FAM_AFFINE) {
         switch (bits) {
             case 2: e = qmv::launch_affine_b2(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
@@ -345,7 +381,7 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
     snprintf(buf, (size_t)buflen,
              "path=%s chunk=%d maxm=%d rows_per_warp=%d warps_k=%d warps_rows=%d tile_iters=%d "
              "grid=%u block=%u smem=%zu",
-             pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr, pl.tile_iters,
+             pl.stream ? "stream" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr, pl.tile_iters,
              pl.grid.x, pl.block.x, pl.smem);
     return QMV_OK;
 }

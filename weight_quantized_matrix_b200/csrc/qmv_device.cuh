@@ -212,20 +212,203 @@ template <int FAM, int BITS> struct Fmt {
         kBits == 2 ? 4 : kBits == 3 ? 4 : kBits == 4 ? 2 : kBits == 5 ? 4 : kBits == 6 ? 2 : 1;
 };
 
-// ------------------------------------------------------------ the kernel ----
+// ------------------------------------------------------- shared pieces -----
+// x staging: one work item = (m, chunk, unit) = 32 consecutive x values of
+// row m; writes the fp32 (pre-scaled for affine) values to
+// xs[((m*TI + i)*(C/4) + u*8 + q)*KT + kt] and, for affine, the unit's
+// sum(x) -- accumulated from values widened to fp32 one by one -- to
+// sx[((m*TI + i)*U + u)*KT + kt], where chunk cc of the tile is owned by
+// k-thread cc % KT at iteration cc / KT.
+template <int FAM, int B, class T, int MAXM, int U>
+__device__ __forceinline__ void stage_x(const Params& p, const char* Xb, float4* xs, float* sx, int t0,
+                                        int tcn, int KT, int TI) {
+    constexpr int C = 32 * U;
+    constexpr bool AFF = (FAM == FAM_AFFINE);
+    const int items = MAXM * tcn * U;
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+        const int u = it % U;
+        const int cc = (it / U) % tcn;
+        const int m = it / (U * tcn);
+        const int i = cc / KT, ktt = cc % KT;
+        float v[32];
+        if (m < p.M) {
+            const long long k0 = (long long)(t0 + cc) * C + u * 32;
+            const T* xr = reinterpret_cast<const T*>(Xb) + (long long)m * p.K + k0;
+            if constexpr (sizeof(T) == 2) {
+                if (p.x_vec) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 vv = __ldg(reinterpret_cast<const uint4*>(xr) + q);
+                        widen8<T>(vv, v + 8 * q);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = DT<T>::ld(xr, j);
+                }
+            } else {
+                if (p.x_vec) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float4 f = __ldg(reinterpret_cast<const float4*>(xr) + q);
+                        v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = DT<T>::ld(xr, j);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        }
+        if constexpr (AFF) {
+            float s = 0.f;                      // sum(x), widened per element
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s += v[j];
+            sx[(((size_t)m * TI + i) * U + u) * KT + ktt] = s;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(v[j], __uint_as_float((127u - field_p(B, j)) << 23));
+        }
+        float4* dst = xs + (((size_t)m * TI + i) * (C / 4) + u * 8) * KT + ktt;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            dst[(size_t)q * KT] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+}
+
+// Per-unit scales of chunk c for R rows (affine: scale + bias of the unit's
+// group; MX: one block scale; NV: two block scales per unit).
+template <int FAM, class T, int R, int U>
+__device__ __forceinline__ void load_scales(const Params& p, const int (&rowc)[R], int c, long long sb,
+                                            float (&sc)[R][U][2], float (&bi)[R][U]) {
+    constexpr int C = 32 * U;
+    const int G = p.G;
+    const long long KG = p.K / G;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long k0 = (long long)c * C + u * 32;
+            const long long rb = (long long)rowc[r] * KG;
+            if constexpr (FAM == FAM_AFFINE) {
+                const long long gi = sb + rb + k0 / G;
+                sc[r][u][0] = DT<T>::ld(p.scales, gi);
+                bi[r][u] = DT<T>::ld(p.biases, gi);
+            } else if constexpr (FAM == FAM_NVFP4) {
+                const uint8_t* s8 = reinterpret_cast<const uint8_t*>(p.scales) + sb + rb + k0 / 16;
+                sc[r][u][0] = e4m3_value(__ldg(s8));
+                sc[r][u][1] = e4m3_value(__ldg(s8 + 1));
+                bi[r][u] = 0.f;
+            } else {
+                const uint8_t* s8 = reinterpret_cast<const uint8_t*>(p.scales) + sb + rb + k0 / 32;
+                sc[r][u][0] = e8m0_value(__ldg(s8));
+                sc[r][u][1] = 0.f;
+                bi[r][u] = 0.f;
+            }
+        }
+}
+
+// Dot products of one chunk (U units of 32 codes) for R rows and MAXM x rows.
+//   wv    chunk words of each row (registers)
+//   xb    &xs[(i*(C/4))*KT + kt]; x row m, unit u, step q at xb[m*xm + (u*8+q)*KT]
+//   sxb   &sx[(i*U)*KT + kt];     x row m, unit u        at sxb[m*sxm + u*KT]
+template <int FAM, int B, int MAXM, int R, int U>
+__device__ __forceinline__ void compute_chunk(const uint32_t (&wv)[R][B * U], const float (&sc)[R][U][2],
+                                              const float (&bi)[R][U], const float4* xb, size_t xm,
+                                              const float* sxb, size_t sxm, int KT, float (&acc)[R][MAXM]) {
+    constexpr int UW = B;
+    constexpr bool AFF = (FAM == FAM_AFFINE);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        unsigned long long part[R][MAXM][2];      // NV: one per 16-code block
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m) { part[r][m][0] = 0ull; part[r][m][1] = 0ull; }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {              // 4 codes per step
+            float4 xv[MAXM];
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m) xv[m] = xb[(size_t)m * xm + (size_t)(u * 8 + q) * KT];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const uint32_t* wu = &wv[r][u * UW];
+                unsigned long long d0, d1;         // codes 4q..4q+3 as two float pairs
+                if constexpr (AFF) {
+                    uint32_t f0, f1, f2, f3;
+                    switch (q) {
+#define QMV_F4(QQ) case QQ: f0 = field_bits<B, 4 * QQ>(wu); f1 = field_bits<B, 4 * QQ + 1>(wu); \
+                   f2 = field_bits<B, 4 * QQ + 2>(wu); f3 = field_bits<B, 4 * QQ + 3>(wu); break;
+                        QMV_F4(0) QMV_F4(1) QMV_F4(2) QMV_F4(3) QMV_F4(4) QMV_F4(5) QMV_F4(6) QMV_F4(7)
+#undef QMV_F4
+                        default: f0 = f1 = f2 = f3 = 0;
+                    }
+                    d0 = magic_pair(f0, f1);
+                    d1 = magic_pair(f2, f3);
+                } else if constexpr (B == 4) {
+                    const uint32_t wd = wu[q >> 1] >> (16 * (q & 1));
+                    const unsigned long long s126 = pk(0x1p126f, 0x1p126f);
+                    d0 = mul2(pk(__uint_as_float(e2m1_pattern(wd)), __uint_as_float(e2m1_pattern(wd >> 4))), s126);
+                    d1 = mul2(pk(__uint_as_float(e2m1_pattern(wd >> 8)), __uint_as_float(e2m1_pattern(wd >> 12))), s126);
+                } else {
+                    const uint32_t wd = wu[q];
+                    d0 = pk(e4m3_value(wd), e4m3_value(wd >> 8));
+                    d1 = pk(e4m3_value(wd >> 16), e4m3_value(wd >> 24));
+                }
+                const int h = (FAM == FAM_NVFP4) ? (q >> 2) : 0;   // 16-code block within the unit
+#pragma unroll
+                for (int m = 0; m < MAXM; ++m) {
+                    unsigned long long a = part[r][m][h];
+                    a = fma2(pk(xv[m].x, xv[m].y), d0, a);
+                    a = fma2(pk(xv[m].z, xv[m].w), d1, a);
+                    part[r][m][h] = a;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m) {
+                if constexpr (AFF) {
+                    const float s = sxb[(size_t)m * sxm + (size_t)u * KT];
+                    const float pr = lo(part[r][m][0]) + hi(part[r][m][0]);
+                    acc[r][m] = fmaf(sc[r][u][0], pr, fmaf(bi[r][u], s, acc[r][m]));
+                } else if constexpr (FAM == FAM_NVFP4) {
+                    acc[r][m] = fmaf(sc[r][u][0], lo(part[r][m][0]) + hi(part[r][m][0]), acc[r][m]);
+                    acc[r][m] = fmaf(sc[r][u][1], lo(part[r][m][1]) + hi(part[r][m][1]), acc[r][m]);
+                } else {
+                    acc[r][m] = fmaf(sc[r][u][0], lo(part[r][m][0]) + hi(part[r][m][0]), acc[r][m]);
+                }
+            }
+    }
+}
+
+template <int R, int MAXM>
+__device__ __forceinline__ void warp_allreduce(float (&acc)[R][MAXM]) {
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) {
+            float v = acc[r][m];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+            acc[r][m] = v;
+        }
+}
+
+// ------------------------------------------------ kernel 1: narrow / general --
 // Shared memory layout (floats):
 //   xs : [MAXM][tile_iters][C/4][KT] float4   pre-scaled x of the tile
-//   sx : [MAXM][tile_iters][U][KT]            affine: sum(x) per unit-run
+//   sx : [MAXM][tile_iters][U][KT]            affine: sum(x) per unit
 //   red: [wk][wr*R*MAXM]                       cross-warp partials
 // KT = 32*wk.  Chunk c of the tile belongs to k-thread c % KT, iteration c / KT.
 template <int FAM, int BITS, class T, int MAXM, int R, bool WIDE>
 __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
     using F = Fmt<FAM, BITS>;
     constexpr int B = F::kBits;
-    constexpr int UW = F::kUnitWords;
     constexpr int U = WIDE ? F::kWideUnits : 1;
     constexpr int C = 32 * U;
-    constexpr int CW = UW * U;
+    constexpr int CW = B * U;
     constexpr bool AFF = (FAM == FAM_AFFINE);
 
     extern __shared__ float4 smem4[];
@@ -238,12 +421,10 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
     const int NC = p.K / C;
     const int TI = p.tile_iters;
     const int TC = KT * TI;
-    const int G = p.G;
-    const int KG = p.K / G;
 
-    float4* xs = smem4;                                                  // [MAXM][TI][C/4][KT]
-    float* sx = reinterpret_cast<float*>(xs + (size_t)MAXM * TI * (C / 4) * KT);  // [MAXM][TI][U][KT]
-    float* red = sx + (AFF ? (size_t)MAXM * TI * U * KT : 0);            // [wk][wr*R*MAXM]
+    float4* xs = smem4;
+    float* sx = reinterpret_cast<float*>(xs + (size_t)MAXM * TI * (C / 4) * KT);
+    float* red = sx + (AFF ? (size_t)MAXM * TI * U * KT : 0);
 
     const uint8_t* W = p.w + bz * p.w_bs;
     const char* Xb = reinterpret_cast<const char*>(p.x) + bz * p.x_bs * (long long)sizeof(T);
@@ -259,192 +440,51 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
 #pragma unroll
         for (int m = 0; m < MAXM; ++m) acc[r][m] = 0.f;
 
+    uint32_t wv[R][CW];
+    float sc[R][U][2], bi[R][U];
+    auto load_chunk = [&](int c) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const uint8_t* src = W + (long long)rowc[r] * p.w_row + (long long)c * (C * B / 8);
+            if constexpr (WIDE) {
+#pragma unroll
+                for (int q = 0; q < CW / 4; ++q) {
+                    uint4 t = __ldg(reinterpret_cast<const uint4*>(src) + q);
+                    wv[r][4 * q] = t.x; wv[r][4 * q + 1] = t.y; wv[r][4 * q + 2] = t.z; wv[r][4 * q + 3] = t.w;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < CW; ++q) wv[r][q] = __ldg(reinterpret_cast<const uint32_t*>(src) + q);
+            }
+        }
+        load_scales<FAM, T, R, U>(p, rowc, c, sb, sc, bi);
+    };
+
     grid_wait();   // inputs may come from the previous kernel in the stream
 
     for (int t0 = 0; t0 < NC; t0 += TC) {
         const int tcn = min(TC, NC - t0);          // chunks in this tile
         __syncthreads();
-        // ---- stage x: one work item = (m, chunk, unit) = 32 codes ----------
-        {
-            const int items = MAXM * tcn * U;
-            for (int it = threadIdx.x; it < items; it += blockDim.x) {
-                const int u = it % U;
-                const int cc = (it / U) % tcn;
-                const int m = it / (U * tcn);
-                const int i = cc / KT, ktt = cc % KT;
-                float v[32];
-                if (m < p.M) {
-                    const long long k0 = (long long)(t0 + cc) * C + u * 32;
-                    const T* xr = reinterpret_cast<const T*>(Xb) + (long long)m * p.K + k0;
-                    if constexpr (sizeof(T) == 2) {
-                        if (p.x_vec) {
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                uint4 vv = __ldg(reinterpret_cast<const uint4*>(xr) + q);
-                                widen8<T>(vv, v + 8 * q);
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] = DT<T>::ld(xr, j);
-                        }
-                    } else {
-                        if (p.x_vec) {
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                float4 f = __ldg(reinterpret_cast<const float4*>(xr) + q);
-                                v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] = DT<T>::ld(xr, j);
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = 0.f;
-                }
-                if constexpr (AFF) {
-                    float s = 0.f;                      // sum(x), widened per element
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) s += v[j];
-                    sx[(((size_t)m * TI + i) * U + u) * KT + ktt] = s;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(v[j], __uint_as_float((127u - field_p(B, j)) << 23));
-                }
-                float4* dst = xs + (((size_t)m * TI + i) * (C / 4) + u * 8) * KT + ktt;
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    dst[(size_t)q * KT] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-            }
-        }
+        // the first chunk's weights are independent of x: issue them before
+        // staging x so both latencies overlap
+        bool have = kt < tcn;
+        if (have) load_chunk(t0 + kt);
+        stage_x<FAM, B, T, MAXM, U>(p, Xb, xs, sx, t0, tcn, KT, TI);
         __syncthreads();
-
-        // ---- main loop over this k-thread's chunks of the tile --------------
-        for (int i = 0; i < TI; ++i) {
+        for (int i = 0; have;) {
+            compute_chunk<FAM, B, MAXM, R, U>(wv, sc, bi, xs + (size_t)i * (C / 4) * KT + kt,
+                                              (size_t)TI * (C / 4) * KT, sx + (size_t)i * U * KT + kt,
+                                              (size_t)TI * U * KT, KT, acc);
+            ++i;
             const int cc = i * KT + kt;
-            if (cc >= tcn) break;
-            const int c = t0 + cc;
-            // load the chunk of every row
-            uint32_t wv[R][CW];
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const uint8_t* src = W + (long long)rowc[r] * p.w_row + (long long)c * (C * B / 8);
-                if constexpr (WIDE) {
-#pragma unroll
-                    for (int q = 0; q < CW / 4; ++q) {
-                        uint4 t = __ldg(reinterpret_cast<const uint4*>(src) + q);
-                        wv[r][4 * q] = t.x; wv[r][4 * q + 1] = t.y; wv[r][4 * q + 2] = t.z; wv[r][4 * q + 3] = t.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < CW; ++q) wv[r][q] = __ldg(reinterpret_cast<const uint32_t*>(src) + q);
-                }
-            }
-            // per-unit scale (affine: scale + bias of the unit's group;
-            // MX: one block scale; NV: two block scales per unit)
-            float sc[R][U][2], bi[R][U];
-#pragma unroll
-            for (int r = 0; r < R; ++r)
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const long long k0 = (long long)c * C + u * 32;
-                    const long long rb = (long long)rowc[r] * KG;
-                    if constexpr (AFF) {
-                        const long long gi = sb + rb + k0 / G;
-                        sc[r][u][0] = DT<T>::ld(p.scales, gi);
-                        bi[r][u] = DT<T>::ld(p.biases, gi);
-                    } else if constexpr (FAM == FAM_NVFP4) {
-                        const uint8_t* s8 = reinterpret_cast<const uint8_t*>(p.scales) + sb + rb + k0 / 16;
-                        sc[r][u][0] = e4m3_value(__ldg(s8));
-                        sc[r][u][1] = e4m3_value(__ldg(s8 + 1));
-                    } else {
-                        const uint8_t* s8 = reinterpret_cast<const uint8_t*>(p.scales) + sb + rb + k0 / 32;
-                        sc[r][u][0] = e8m0_value(__ldg(s8));
-                    }
-                }
-
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                unsigned long long part[R][MAXM][2];      // NV: one per 16-code block
-#pragma unroll
-                for (int r = 0; r < R; ++r)
-#pragma unroll
-                    for (int m = 0; m < MAXM; ++m) { part[r][m][0] = 0ull; part[r][m][1] = 0ull; }
-                const float4* xu = xs + ((size_t)i * (C / 4) + u * 8) * KT + kt;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {              // 4 codes per step
-                    float4 xv[MAXM];
-#pragma unroll
-                    for (int m = 0; m < MAXM; ++m) xv[m] = xu[((size_t)m * TI * (C / 4) + q) * KT];
-#pragma unroll
-                    for (int r = 0; r < R; ++r) {
-                        const uint32_t* wu = &wv[r][u * UW];
-                        unsigned long long d0, d1;         // codes 4q..4q+3 as two float pairs
-                        if constexpr (AFF) {
-                            // unrolled field plan (compile-time per q)
-                            uint32_t f0, f1, f2, f3;
-                            switch (q) {
-#define QMV_F4(QQ) case QQ: f0 = field_bits<B, 4 * QQ>(wu); f1 = field_bits<B, 4 * QQ + 1>(wu); \
-                   f2 = field_bits<B, 4 * QQ + 2>(wu); f3 = field_bits<B, 4 * QQ + 3>(wu); break;
-                                QMV_F4(0) QMV_F4(1) QMV_F4(2) QMV_F4(3) QMV_F4(4) QMV_F4(5) QMV_F4(6) QMV_F4(7)
-#undef QMV_F4
-                                default: f0 = f1 = f2 = f3 = 0;
-                            }
-                            d0 = magic_pair(f0, f1);
-                            d1 = magic_pair(f2, f3);
-                        } else if constexpr (B == 4) {
-                            const uint32_t wd = wu[q >> 1] >> (16 * (q & 1));
-                            const unsigned long long s126 = pk(0x1p126f, 0x1p126f);
-                            d0 = mul2(pk(__uint_as_float(e2m1_pattern(wd)), __uint_as_float(e2m1_pattern(wd >> 4))), s126);
-                            d1 = mul2(pk(__uint_as_float(e2m1_pattern(wd >> 8)), __uint_as_float(e2m1_pattern(wd >> 12))), s126);
-                        } else {
-                            const uint32_t wd = wu[q];
-                            d0 = pk(e4m3_value(wd), e4m3_value(wd >> 8));
-                            d1 = pk(e4m3_value(wd >> 16), e4m3_value(wd >> 24));
-                        }
-                        constexpr int blk = 0;
-                        const int h = (FAM == FAM_NVFP4) ? (q >> 2) : blk;   // 16-code block within the unit
-#pragma unroll
-                        for (int m = 0; m < MAXM; ++m) {
-                            unsigned long long a = part[r][m][h];
-                            a = fma2(pk(xv[m].x, xv[m].y), d0, a);
-                            a = fma2(pk(xv[m].z, xv[m].w), d1, a);
-                            part[r][m][h] = a;
-                        }
-                    }
-                }
-                // epilogue of the unit
-#pragma unroll
-                for (int r = 0; r < R; ++r)
-#pragma unroll
-                    for (int m = 0; m < MAXM; ++m) {
-                        if constexpr (AFF) {
-                            const float s = sx[(((size_t)m * TI + i) * U + u) * KT + kt];
-                            const float pr = lo(part[r][m][0]) + hi(part[r][m][0]);
-                            acc[r][m] = fmaf(sc[r][u][0], pr, fmaf(bi[r][u], s, acc[r][m]));
-                        } else if constexpr (FAM == FAM_NVFP4) {
-                            acc[r][m] = fmaf(sc[r][u][0], lo(part[r][m][0]) + hi(part[r][m][0]), acc[r][m]);
-                            acc[r][m] = fmaf(sc[r][u][1], lo(part[r][m][1]) + hi(part[r][m][1]), acc[r][m]);
-                        } else {
-                            acc[r][m] = fmaf(sc[r][u][0], lo(part[r][m][0]) + hi(part[r][m][0]), acc[r][m]);
-                        }
-                    }
-            }
+            have = i < TI && cc < tcn;
+            if (have) load_chunk(t0 + cc);
         }
     }
 
     grid_launch_dependents();
 
-    // ---- reduction: warp butterfly, then across the k-warps -----------------
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int m = 0; m < MAXM; ++m) {
-            float v = acc[r][m];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-            acc[r][m] = v;
-        }
+    warp_allreduce<R, MAXM>(acc);
     float gs = 1.f;
     if constexpr (FAM == FAM_NVFP4) gs = __ldg(p.gscale + bz);
     T* Y = reinterpret_cast<T*>(p.y) + bz * p.y_bs;
@@ -473,6 +513,169 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
             if (row < p.N && m < p.M) DT<T>::st(Y, (long long)m * p.N + row, v * gs);
         }
     }
+}
+
+// ------------------------------------------ kernel 2: streaming, large N ----
+// Persistent blocks (about one wave); x is staged once per block.  Each warp
+// walks its own row blocks of R rows; its 32 lanes take the wide chunks of
+// those rows round-robin (chunk c = lane + 32*i).  Weights reach shared
+// memory through a per-warp ring of S stages filled with cp.async (16-byte
+// copies, L1 bypassed): while the warp computes iteration it, the copies for
+// iterations it+1 .. it+S-1 are in flight, so the bytes in flight are held in
+// shared memory, not registers.  Every lane consumes only the bytes it copied
+// itself, so cp.async.wait_group alone orders the data (a hardware wait on the
+// thread's own copies; nothing spins).  Scales are loaded one iteration ahead.
+//
+// Shared memory:  xs [MAXM][I][C/4][32] float4, sx [MAXM][I][U][32] float,
+//                 ring [warps][S][R][CW/4][32] uint4        (I = ceil(NC/32))
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N_>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N_) : "memory"); }
+
+template <int FAM, int BITS, class T, int MAXM, int R, int S>
+__global__ void __launch_bounds__(256) qmv_stream_kernel(const Params p) {
+    using F = Fmt<FAM, BITS>;
+    constexpr int B = F::kBits;
+    constexpr int U = F::kWideUnits;
+    constexpr int C = 32 * U;
+    constexpr int CW = B * U;
+    constexpr int CV = CW / 4;               // 16-byte vectors per chunk
+    constexpr bool AFF = (FAM == FAM_AFFINE);
+
+    extern __shared__ float4 smem4[];
+    const int NW = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bz = blockIdx.z;
+    const int NC = p.K / C;
+    const int I = (NC + 31) / 32;
+
+    float4* xs = smem4;
+    float* sx = reinterpret_cast<float*>(xs + (size_t)MAXM * I * (C / 4) * 32);
+    uint4* ring = reinterpret_cast<uint4*>(sx + (AFF ? (size_t)MAXM * I * U * 32 : 0));
+    uint4* my = ring + (size_t)warp * S * R * CV * 32;
+
+    const uint8_t* W = p.w + bz * p.w_bs;
+    const char* Xb = reinterpret_cast<const char*>(p.x) + bz * p.x_bs * (long long)sizeof(T);
+    const long long sb = bz * p.s_bs;
+
+    const int nrb = (p.N + R - 1) / R;
+    const int gw = blockIdx.x * NW + warp, GW = gridDim.x * NW;
+    const int my_rb = gw < nrb ? (nrb - gw + GW - 1) / GW : 0;
+    const int total = my_rb * I;
+
+    // A position in this warp's iteration sequence: row block j (global row
+    // block gw + j*GW), chunk iteration i (chunk lane + 32*i), ring slot s.
+    struct Pos { int i, j, s; };
+    auto advance = [&](Pos& q) {
+        if (++q.i == I) { q.i = 0; ++q.j; }
+        if (++q.s == S) q.s = 0;
+    };
+    auto rows_of = [&](const Pos& q, int (&rowc)[R]) {
+        const long long rb = (long long)gw + (long long)q.j * GW;
+#pragma unroll
+        for (int r = 0; r < R; ++r) rowc[r] = (int)min(rb * R + r, (long long)p.N - 1);
+    };
+    auto issue = [&](const Pos& q) {
+        const int c = lane + 32 * q.i;
+        if (c < NC) {
+            int rowc[R];
+            rows_of(q, rowc);
+            uint4* dst = my + (size_t)q.s * R * CV * 32 + lane;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const uint4* src = reinterpret_cast<const uint4*>(W + (long long)rowc[r] * p.w_row +
+                                                                  (long long)c * (C * B / 8));
+#pragma unroll
+                for (int q2 = 0; q2 < CV; ++q2) cp_async16(dst + (size_t)(r * CV + q2) * 32, src + q2);
+            }
+        }
+    };
+
+    grid_wait();
+    Pos pi = {0, 0, 0};                             // next iteration to issue
+    int n_issued = 0;
+#pragma unroll
+    for (int s = 0; s < S - 1; ++s) {
+        if (n_issued < total) issue(pi);
+        cp_async_commit();
+        advance(pi); ++n_issued;
+    }
+    stage_x<FAM, B, T, MAXM, U>(p, Xb, xs, sx, 0, NC, 32, I);
+    __syncthreads();
+
+    float acc[R][MAXM];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) acc[r][m] = 0.f;
+
+    float sc[R][U][2], bi[R][U], nsc[R][U][2], nbi[R][U];
+    Pos pc = {0, 0, 0};                             // iteration being computed
+    Pos pn = {0, 0, 0};                             // iteration whose scales are in nsc
+    if (total > 0 && lane < NC) {
+        int rowc[R];
+        rows_of(pn, rowc);
+        load_scales<FAM, T, R, U>(p, rowc, lane, sb, nsc, nbi);
+    }
+    float gs = 1.f;
+    if constexpr (FAM == FAM_NVFP4) gs = __ldg(p.gscale + bz);
+    T* Y = reinterpret_cast<T*>(p.y) + bz * p.y_bs;
+
+    for (int it = 0; it < total; ++it) {
+        if (n_issued < total) issue(pi);
+        cp_async_commit();
+        advance(pi); ++n_issued;
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int u = 0; u < U; ++u) { sc[r][u][0] = nsc[r][u][0]; sc[r][u][1] = nsc[r][u][1]; bi[r][u] = nbi[r][u]; }
+        advance(pn);
+        if (it + 1 < total) {                       // scales one iteration ahead
+            const int c1 = lane + 32 * pn.i;
+            if (c1 < NC) {
+                int rowc[R];
+                rows_of(pn, rowc);
+                load_scales<FAM, T, R, U>(p, rowc, c1, sb, nsc, nbi);
+            }
+        }
+        cp_async_wait<S - 1>();                     // this lane's copies for iteration it landed
+        const int i = pc.i;
+        const int c = lane + 32 * i;
+        if (c < NC) {
+            uint32_t wv[R][CW];
+            const uint4* src = my + (size_t)pc.s * R * CV * 32 + lane;
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int q = 0; q < CV; ++q) {
+                    const uint4 t = src[(size_t)(r * CV + q) * 32];
+                    wv[r][4 * q] = t.x; wv[r][4 * q + 1] = t.y; wv[r][4 * q + 2] = t.z; wv[r][4 * q + 3] = t.w;
+                }
+            compute_chunk<FAM, B, MAXM, R, U>(wv, sc, bi, xs + (size_t)i * (C / 4) * 32 + lane,
+                                              (size_t)I * (C / 4) * 32, sx + (size_t)i * U * 32 + lane,
+                                              (size_t)I * U * 32, 32, acc);
+        }
+        if (i == I - 1) {                           // row block done: reduce and store
+            warp_allreduce<R, MAXM>(acc);
+            const long long rb = (long long)gw + (long long)pc.j * GW;
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int m = 0; m < MAXM; ++m) {
+                    const long long row = rb * R + r;
+                    if (lane == r * MAXM + m && row < p.N && m < p.M)
+                        DT<T>::st(Y, (long long)m * p.N + row, acc[r][m] * gs);
+                    acc[r][m] = 0.f;
+                }
+        }
+        advance(pc);
+    }
+    cp_async_wait<0>();
+    grid_launch_dependents();
 }
 
 // ------------------------------------------------- dequantization check ----
