@@ -150,11 +150,12 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
 
 /*
  * qmv_force_config -- benchmarking / testing knob: pin the launch shape used
- * by every later call in this process.  path: 2 = persistent streaming kernel
- * (wide chunks through a shared-memory ring), 1 = wide-load chunks, 0 = 4-byte
- * chunks, -1 = automatic; rows_per_warp in {1,2,4} or -1; warps_k (warps that
- * split K inside a block) in {1,..,8} or -1; warps_rows in {1,..,8} or -1 (for
- * the streaming kernel: warps per block).
+ * by every later call in this process.  path: 3 = tensor-core kernel (affine
+ * formats; falls back to automatic where its size rules do not hold),
+ * 1 = CUDA-core kernel with wide (16-byte) chunk loads, 0 = CUDA-core kernel
+ * with 4-byte chunks, -1 = automatic; rows_per_warp in {1,2,4} or -1 (CUDA-core
+ * kernel); warps_k (warps that split K inside a block) in {1,..,8} or -1;
+ * warps_rows in {1,..,8} or -1.
  * Unsupported combinations fall back to automatic for that field.  Not
  * thread-safe with concurrent calls; meant for single-threaded harnesses.
  */

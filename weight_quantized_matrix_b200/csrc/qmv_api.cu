@@ -20,6 +20,7 @@
 
 #include "../../include/qmv.h"
 #include "qmv_launch.cuh"
+#include "qmv_tc_plan.cuh"
 
 namespace {
 
@@ -64,25 +65,90 @@ FmtInfo fmt_info(int fam, int bits) {
 }
 
 struct Plan {
-    int maxm, R, wide, stream, wk, wr, tile_iters, C;
+    int maxm, R, wide, tc, npass, wk, wr, tile_iters, C;
     size_t smem;
     dim3 grid, block;
 };
-
-// Rows per warp of the streaming kernel: enough rows to share each x load,
-// few enough that the ring stage and the chunk registers stay small.
-int stream_rows(int bits, int maxm) {
-    if (maxm <= 2) return (bits == 3 || bits == 5 || bits == 6) ? 2 : 4;
-    return (bits == 5 || maxm == 8) ? 1 : 2;
-}
 
 int rows_per_warp_cap(int bits, int maxm) {
     if (maxm <= 2) return (bits == 3 || bits == 5 || bits == 6) ? 2 : 4;
     return 2;
 }
 
+// ---- tensor-core launch shape --------------------------------------------------
+// Which path wins, measured on B200 (bf16 x): 6-bit codes have no field
+// pairing (one mask per code), so the CUDA cores win there; with several x rows
+// the tensor cores win (the CUDA cores would need M FMAs per code); with one x
+// row they win only once the matrix is large enough to hide their longer
+// pipeline (about 48 MB of packed weights).
+bool tc_preferred(int M, int N, int K, int bits) {
+    if (N < 64 || bits == 6) return false;
+    if (M >= 2) return true;
+    if (bits == 8) return false;
+    const double wbytes = (double)N * K * bits / 8.0;
+    return wbytes >= 48.0 * 1024 * 1024;
+}
+
+template <int B> int tc_np() { return qmv::tc_make_plan<B, false>().np; }
+int tc_np_of(int bits) {
+    switch (bits) {
+        case 2: return tc_np<2>(); case 3: return tc_np<3>(); case 4: return tc_np<4>();
+        case 5: return tc_np<5>(); case 6: return tc_np<6>(); case 8: return tc_np<8>();
+        default: return 0;
+    }
+}
+int tc_unit_bytes(int bits) { return (bits == 2 || bits == 4 || bits == 8) ? 16 : 4 * bits; }
+
+struct TcShape { int npass, wk, wr, tsb, sb; long long gx; size_t smem; };
+
+bool tc_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, TcShape* ts) {
+    const int ub = tc_unit_bytes(bits);
+    const int uc = ub * 8 / bits;
+    const int SB = 4 * uc;
+    if (K % SB != 0) return false;
+    if (ub == 16 && !w16) return false;
+    if (bits == 2 && G < 64) return false;          // a 64-code unit would span two groups
+    const int segsz = G < SB ? G : SB;
+    const int ngs = SB / segsz;
+    const int cols = M * ngs;
+    const int npass = cols <= 8 ? 1 : cols <= 16 ? 2 : cols <= 32 ? 4 : 0;
+    if (npass == 0) return false;
+    const int nsplit = dtype == QMV_BF16 ? 1 : dtype == QMV_F16 ? 2 : 3;
+    const int np = tc_np_of(bits);
+    const int nsbk = K / SB;
+    const long long tiles = ((long long)N + 15) / 16;
+    const int sms = device_sms();
+    // about 8 warps per SM: split K over k-warps only when the 16-row tiles
+    // alone cannot fill the GPU (measured best on B200 for 4..28K rows)
+    const long long target = (long long)sms * 8;
+    long long wk = 1;
+    while (wk < 8 && tiles * wk < target) wk *= 2;
+    if (wk > nsbk) wk = nsbk;
+    if (wk < 1) wk = 1;
+    long long wr = 8 / wk;
+    if (wr > tiles) wr = tiles;
+    if (wr < 1) wr = 1;
+    if (g_forced.wk > 0) wk = g_forced.wk > 8 ? 8 : g_forced.wk;
+    if (g_forced.wr > 0) wr = g_forced.wr;
+    while (wk * wr > 8) --wr;
+    const size_t red = (size_t)wk * wr * 16 * 8 * npass * 4;
+    // per super-block of x tile: bf16 planes (x rows + zero row), sum(x) and
+    // sum(x~) per segment, two per-unit sums
+    const size_t per_sb = (size_t)nsplit * (M + 1) * 4 * np * 4 + (size_t)M * ngs * 4 * 2 + (size_t)M * 4 * 2 * 4;
+    const size_t fixed = (size_t)nsplit * (M + 1) * 16 + red;
+    const size_t budget = 160 * 1024;
+    long long tsb = budget > fixed ? (long long)((budget - fixed) / per_sb) : 0;
+    if (tsb > nsbk) tsb = nsbk;
+    if (tsb < 1) return false;
+    ts->npass = npass; ts->wk = (int)wk; ts->wr = (int)wr; ts->tsb = (int)tsb; ts->sb = SB;
+    ts->gx = (tiles + wr - 1) / wr;
+    ts->smem = (size_t)nsplit * (M + 1) * ((size_t)tsb * 4 * np + 4) * 4 + (size_t)M * tsb * ngs * 4 * 2 +
+               (size_t)M * tsb * 4 * 2 * 4 + red;
+    return ts->gx <= 0x7FFFFFFFLL && ts->smem <= (size_t)qmv::kMaxSmem;
+}
+
 // Choose the launch shape.  Returns QMV_OK or an error (sizes too large).
-int make_plan(int fam, int M, int N, int K, int bits, int dtype, bool w16, int batch, Plan* pl) {
+int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, bool w16, int batch, Plan* pl) {
     const FmtInfo fi = fmt_info(fam, bits);
     const bool aff = fam == qmv::FAM_AFFINE;
     int maxm = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
@@ -90,29 +156,19 @@ int make_plan(int fam, int M, int N, int K, int bits, int dtype, bool w16, int b
     bool wide = w16 && (K % c_wide == 0);
     if (g_forced.path == 0) wide = false;
 
-    // ---- streaming kernel (large N, wide chunks, x fits in shared memory) ----
-    if (wide && K > 0 && g_forced.path == 2) {
-        const int U = fi.wide_units, C = 32 * U, CB = C * fi.bits / 8;
-        const int NC = K / C, I = (NC + 31) / 32;
-        int Rs = stream_rows(fi.bits, maxm);
-        if (g_forced.R > 0 && qmv::stream_instantiated(maxm, g_forced.R)) Rs = g_forced.R;
-        const size_t xs = (size_t)maxm * I * C * 32 * 4;
-        const size_t sxb = aff ? (size_t)maxm * I * U * 32 * 4 : 0;
-        const size_t ring_w = (size_t)qmv::kStreamStages * Rs * CB * 32;
-        const size_t avail = (size_t)qmv::kMaxSmem > xs + sxb ? (size_t)qmv::kMaxSmem - xs - sxb : 0;
-        int NW = (int)(avail / ring_w);
-        if (NW > 8) NW = 8;
-        if (g_forced.wr > 0 && g_forced.wr <= NW) NW = g_forced.wr;
-        if (NW >= 2 || (g_forced.path == 2 && NW >= 1)) {
-            const long long nrb = ((long long)N + Rs - 1) / Rs;
-            const long long gx = (nrb + NW - 1) / NW;
-            pl->maxm = maxm; pl->R = Rs; pl->wide = 1; pl->stream = 1; pl->wk = 1; pl->wr = NW;
-            pl->tile_iters = I; pl->C = C; pl->smem = xs + sxb + NW * ring_w;
-            pl->grid = dim3((unsigned)gx, 1, (unsigned)batch);
-            pl->block = dim3(32 * NW, 1, 1);
+    // ---- tensor-core kernel (affine, enough rows to fill the GPU) -------------
+    if (aff && K > 0 && g_forced.path != 0 && g_forced.path != 1 &&
+        (g_forced.path == 3 || tc_preferred(M, N, K, bits))) {
+        TcShape ts;
+        if (tc_shape(M, N, K, bits, G_of_plan, dtype, w16, &ts)) {
+            pl->maxm = maxm; pl->R = 1; pl->wide = 1; pl->tc = 1; pl->npass = ts.npass;
+            pl->wk = ts.wk; pl->wr = ts.wr; pl->tile_iters = ts.tsb; pl->C = ts.sb; pl->smem = ts.smem;
+            pl->grid = dim3((unsigned)ts.gx, 1, (unsigned)batch);
+            pl->block = dim3(32 * ts.wk * ts.wr, 1, 1);
             return QMV_OK;
         }
     }
+
     if (g_forced.path == 1 && w16 && (K % c_wide == 0)) wide = true;
     const int U = wide ? fi.wide_units : 1;
     const int C = 32 * U;
@@ -169,7 +225,7 @@ int make_plan(int fam, int M, int N, int K, int bits, int dtype, bool w16, int b
     const long long gx = ((long long)N + rows_per_block - 1) / rows_per_block;
     if (gx > 0x7FFFFFFFLL) return QMV_EINVAL;
 
-    pl->maxm = maxm; pl->R = R; pl->wide = wide; pl->stream = 0; pl->wk = wk; pl->wr = wr;
+    pl->maxm = maxm; pl->R = R; pl->wide = wide; pl->tc = 0; pl->npass = 0; pl->wk = wk; pl->wr = wr;
     pl->tile_iters = (int)ti; pl->C = C; pl->smem = smem;
     pl->grid = dim3((unsigned)gx, 1, (unsigned)batch);
     pl->block = dim3(32 * wk * wr, 1, 1);
@@ -210,7 +266,7 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     const long long row_bytes = (long long)K * (fam == qmv::FAM_AFFINE ? bits : (fam == qmv::FAM_MXFP8 ? 8 : 4)) / 8;
     Plan pl;
     const bool w16 = aligned(w, 16);
-    int st = make_plan(fam, M, N, K, bits, dtype, w16, batch, &pl);
+    int st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl);
     if (st != QMV_OK) return st;
     qmv::Params p;
     p.x = x; p.w = static_cast<const uint8_t*>(w); p.scales = scales; p.biases = biases;
@@ -226,10 +282,9 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     p.w_row = row_bytes;
     qmv::Launch L{pl.grid, pl.block, pl.smem, static_cast<cudaStream_t>(stream), pdl_enabled()};
     cudaError_t e;
-    if (pl.stream) {
-        e = fam == qmv::FAM_AFFINE ? qmv::launch_stream_affine(bits, dtype, pl.maxm, pl.R, p, L)
-                                   : qmv::launch_stream_fp(fam, dtype, pl.maxm, pl.R, p, L);
-        return finish(e);
+    if (pl.tc) {
+        p.tile_iters = pl.tile_iters;
+        return finish(qmv::launch_tc_affine(bits, dtype, pl.npass, p, L));
     }
     if (fam == qmv::FAM_AFFINE) {
         switch (bits) {
@@ -376,12 +431,12 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
         bits = 0;
     }
     Plan pl;
-    int st = make_plan(fam, M, N, K, bits, dtype, w_align16 != 0, 1, &pl);
+    int st = make_plan(fam, M, N, K, bits, fam == qmv::FAM_AFFINE ? group_size : (family == 2 ? 16 : 32), dtype, w_align16 != 0, 1, &pl);
     if (st != QMV_OK) return st;
     snprintf(buf, (size_t)buflen,
              "path=%s chunk=%d maxm=%d rows_per_warp=%d warps_k=%d warps_rows=%d tile_iters=%d "
              "grid=%u block=%u smem=%zu",
-             pl.stream ? "stream" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr, pl.tile_iters,
+             pl.tc ? "tc" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr, pl.tile_iters,
              pl.grid.x, pl.block.x, pl.smem);
     return QMV_OK;
 }

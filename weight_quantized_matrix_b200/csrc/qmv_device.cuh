@@ -113,29 +113,13 @@ template <> __device__ __forceinline__ void widen8<__nv_bfloat16>(const uint4& v
 }
 
 // ------------------------------------------------------- packed fp32 math --
-// Blackwell fp32x2 instructions: two independent IEEE fp32 operations per
-// issue slot (round to nearest even, no contraction across the pair).
-__device__ __forceinline__ unsigned long long pk(float a, float b) {
-    return (unsigned long long)__float_as_uint(a) | ((unsigned long long)__float_as_uint(b) << 32);
-}
-__device__ __forceinline__ float lo(unsigned long long v) { return __uint_as_float((uint32_t)v); }
-__device__ __forceinline__ float hi(unsigned long long v) { return __uint_as_float((uint32_t)(v >> 32)); }
-__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
-                                                   unsigned long long c) {
-    unsigned long long d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
-    unsigned long long d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
-    unsigned long long d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
+// Blackwell fp32x2 instructions through the compiler's builtins (so constant
+// operands stay in registers or immediates instead of being re-materialised
+// around inline asm): two independent IEEE fp32 operations per issue slot,
+// round to nearest even.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 
 // ------------------------------------------------- grid dependency control --
 __device__ __forceinline__ void grid_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -170,10 +154,10 @@ __device__ __forceinline__ uint32_t field_bits(const uint32_t* w) {
     }
 }
 
-__device__ __forceinline__ unsigned long long magic_pair(uint32_t a, uint32_t b) {
+__device__ __forceinline__ float2 magic_pair(uint32_t a, uint32_t b) {
     // {a, b} fields (< 2^23) -> {a, b} as exact floats
-    const unsigned long long m = pk(-8388608.0f, -8388608.0f);
-    return add2(((unsigned long long)(a | 0x4B000000u)) | ((unsigned long long)(b | 0x4B000000u) << 32), m);
+    return add2(make_float2(__uint_as_float(a | 0x4B000000u), __uint_as_float(b | 0x4B000000u)),
+                make_float2(-8388608.0f, -8388608.0f));
 }
 
 // ------------------------------------------------------- FP element decode --
@@ -320,11 +304,11 @@ __device__ __forceinline__ void compute_chunk(const uint32_t (&wv)[R][B * U], co
     constexpr bool AFF = (FAM == FAM_AFFINE);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-        unsigned long long part[R][MAXM][2];      // NV: one per 16-code block
+        float2 part[R][MAXM][2];                  // NV: one per 16-code block
 #pragma unroll
         for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int m = 0; m < MAXM; ++m) { part[r][m][0] = 0ull; part[r][m][1] = 0ull; }
+            for (int m = 0; m < MAXM; ++m) { part[r][m][0] = make_float2(0.f, 0.f); part[r][m][1] = make_float2(0.f, 0.f); }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {              // 4 codes per step
             float4 xv[MAXM];
@@ -333,7 +317,7 @@ __device__ __forceinline__ void compute_chunk(const uint32_t (&wv)[R][B * U], co
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 const uint32_t* wu = &wv[r][u * UW];
-                unsigned long long d0, d1;         // codes 4q..4q+3 as two float pairs
+                float2 d0, d1;                     // codes 4q..4q+3 as two float pairs
                 if constexpr (AFF) {
                     uint32_t f0, f1, f2, f3;
                     switch (q) {
@@ -347,20 +331,20 @@ __device__ __forceinline__ void compute_chunk(const uint32_t (&wv)[R][B * U], co
                     d1 = magic_pair(f2, f3);
                 } else if constexpr (B == 4) {
                     const uint32_t wd = wu[q >> 1] >> (16 * (q & 1));
-                    const unsigned long long s126 = pk(0x1p126f, 0x1p126f);
-                    d0 = mul2(pk(__uint_as_float(e2m1_pattern(wd)), __uint_as_float(e2m1_pattern(wd >> 4))), s126);
-                    d1 = mul2(pk(__uint_as_float(e2m1_pattern(wd >> 8)), __uint_as_float(e2m1_pattern(wd >> 12))), s126);
+                    const float2 s126 = make_float2(0x1p126f, 0x1p126f);
+                    d0 = mul2(make_float2(__uint_as_float(e2m1_pattern(wd)), __uint_as_float(e2m1_pattern(wd >> 4))), s126);
+                    d1 = mul2(make_float2(__uint_as_float(e2m1_pattern(wd >> 8)), __uint_as_float(e2m1_pattern(wd >> 12))), s126);
                 } else {
                     const uint32_t wd = wu[q];
-                    d0 = pk(e4m3_value(wd), e4m3_value(wd >> 8));
-                    d1 = pk(e4m3_value(wd >> 16), e4m3_value(wd >> 24));
+                    d0 = make_float2(e4m3_value(wd), e4m3_value(wd >> 8));
+                    d1 = make_float2(e4m3_value(wd >> 16), e4m3_value(wd >> 24));
                 }
                 const int h = (FAM == FAM_NVFP4) ? (q >> 2) : 0;   // 16-code block within the unit
 #pragma unroll
                 for (int m = 0; m < MAXM; ++m) {
-                    unsigned long long a = part[r][m][h];
-                    a = fma2(pk(xv[m].x, xv[m].y), d0, a);
-                    a = fma2(pk(xv[m].z, xv[m].w), d1, a);
+                    float2 a = part[r][m][h];
+                    a = fma2(make_float2(xv[m].x, xv[m].y), d0, a);
+                    a = fma2(make_float2(xv[m].z, xv[m].w), d1, a);
                     part[r][m][h] = a;
                 }
             }
@@ -371,13 +355,13 @@ __device__ __forceinline__ void compute_chunk(const uint32_t (&wv)[R][B * U], co
             for (int m = 0; m < MAXM; ++m) {
                 if constexpr (AFF) {
                     const float s = sxb[(size_t)m * sxm + (size_t)u * KT];
-                    const float pr = lo(part[r][m][0]) + hi(part[r][m][0]);
+                    const float pr = part[r][m][0].x + part[r][m][0].y;
                     acc[r][m] = fmaf(sc[r][u][0], pr, fmaf(bi[r][u], s, acc[r][m]));
                 } else if constexpr (FAM == FAM_NVFP4) {
-                    acc[r][m] = fmaf(sc[r][u][0], lo(part[r][m][0]) + hi(part[r][m][0]), acc[r][m]);
-                    acc[r][m] = fmaf(sc[r][u][1], lo(part[r][m][1]) + hi(part[r][m][1]), acc[r][m]);
+                    acc[r][m] = fmaf(sc[r][u][0], part[r][m][0].x + part[r][m][0].y, acc[r][m]);
+                    acc[r][m] = fmaf(sc[r][u][1], part[r][m][1].x + part[r][m][1].y, acc[r][m]);
                 } else {
-                    acc[r][m] = fmaf(sc[r][u][0], lo(part[r][m][0]) + hi(part[r][m][0]), acc[r][m]);
+                    acc[r][m] = fmaf(sc[r][u][0], part[r][m][0].x + part[r][m][0].y, acc[r][m]);
                 }
             }
     }
@@ -515,169 +499,6 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
     }
 }
 
-// ------------------------------------------ kernel 2: streaming, large N ----
-// Persistent blocks (about one wave); x is staged once per block.  Each warp
-// walks its own row blocks of R rows; its 32 lanes take the wide chunks of
-// those rows round-robin (chunk c = lane + 32*i).  Weights reach shared
-// memory through a per-warp ring of S stages filled with cp.async (16-byte
-// copies, L1 bypassed): while the warp computes iteration it, the copies for
-// iterations it+1 .. it+S-1 are in flight, so the bytes in flight are held in
-// shared memory, not registers.  Every lane consumes only the bytes it copied
-// itself, so cp.async.wait_group alone orders the data (a hardware wait on the
-// thread's own copies; nothing spins).  Scales are loaded one iteration ahead.
-//
-// Shared memory:  xs [MAXM][I][C/4][32] float4, sx [MAXM][I][U][32] float,
-//                 ring [warps][S][R][CW/4][32] uint4        (I = ceil(NC/32))
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N_>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N_) : "memory"); }
-
-template <int FAM, int BITS, class T, int MAXM, int R, int S>
-__global__ void __launch_bounds__(256) qmv_stream_kernel(const Params p) {
-    using F = Fmt<FAM, BITS>;
-    constexpr int B = F::kBits;
-    constexpr int U = F::kWideUnits;
-    constexpr int C = 32 * U;
-    constexpr int CW = B * U;
-    constexpr int CV = CW / 4;               // 16-byte vectors per chunk
-    constexpr bool AFF = (FAM == FAM_AFFINE);
-
-    extern __shared__ float4 smem4[];
-    const int NW = blockDim.x >> 5;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bz = blockIdx.z;
-    const int NC = p.K / C;
-    const int I = (NC + 31) / 32;
-
-    float4* xs = smem4;
-    float* sx = reinterpret_cast<float*>(xs + (size_t)MAXM * I * (C / 4) * 32);
-    uint4* ring = reinterpret_cast<uint4*>(sx + (AFF ? (size_t)MAXM * I * U * 32 : 0));
-    uint4* my = ring + (size_t)warp * S * R * CV * 32;
-
-    const uint8_t* W = p.w + bz * p.w_bs;
-    const char* Xb = reinterpret_cast<const char*>(p.x) + bz * p.x_bs * (long long)sizeof(T);
-    const long long sb = bz * p.s_bs;
-
-    const int nrb = (p.N + R - 1) / R;
-    const int gw = blockIdx.x * NW + warp, GW = gridDim.x * NW;
-    const int my_rb = gw < nrb ? (nrb - gw + GW - 1) / GW : 0;
-    const int total = my_rb * I;
-
-    // A position in this warp's iteration sequence: row block j (global row
-    // block gw + j*GW), chunk iteration i (chunk lane + 32*i), ring slot s.
-    struct Pos { int i, j, s; };
-    auto advance = [&](Pos& q) {
-        if (++q.i == I) { q.i = 0; ++q.j; }
-        if (++q.s == S) q.s = 0;
-    };
-    auto rows_of = [&](const Pos& q, int (&rowc)[R]) {
-        const long long rb = (long long)gw + (long long)q.j * GW;
-#pragma unroll
-        for (int r = 0; r < R; ++r) rowc[r] = (int)min(rb * R + r, (long long)p.N - 1);
-    };
-    auto issue = [&](const Pos& q) {
-        const int c = lane + 32 * q.i;
-        if (c < NC) {
-            int rowc[R];
-            rows_of(q, rowc);
-            uint4* dst = my + (size_t)q.s * R * CV * 32 + lane;
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const uint4* src = reinterpret_cast<const uint4*>(W + (long long)rowc[r] * p.w_row +
-                                                                  (long long)c * (C * B / 8));
-#pragma unroll
-                for (int q2 = 0; q2 < CV; ++q2) cp_async16(dst + (size_t)(r * CV + q2) * 32, src + q2);
-            }
-        }
-    };
-
-    grid_wait();
-    Pos pi = {0, 0, 0};                             // next iteration to issue
-    int n_issued = 0;
-#pragma unroll
-    for (int s = 0; s < S - 1; ++s) {
-        if (n_issued < total) issue(pi);
-        cp_async_commit();
-        advance(pi); ++n_issued;
-    }
-    stage_x<FAM, B, T, MAXM, U>(p, Xb, xs, sx, 0, NC, 32, I);
-    __syncthreads();
-
-    float acc[R][MAXM];
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int m = 0; m < MAXM; ++m) acc[r][m] = 0.f;
-
-    float sc[R][U][2], bi[R][U], nsc[R][U][2], nbi[R][U];
-    Pos pc = {0, 0, 0};                             // iteration being computed
-    Pos pn = {0, 0, 0};                             // iteration whose scales are in nsc
-    if (total > 0 && lane < NC) {
-        int rowc[R];
-        rows_of(pn, rowc);
-        load_scales<FAM, T, R, U>(p, rowc, lane, sb, nsc, nbi);
-    }
-    float gs = 1.f;
-    if constexpr (FAM == FAM_NVFP4) gs = __ldg(p.gscale + bz);
-    T* Y = reinterpret_cast<T*>(p.y) + bz * p.y_bs;
-
-    for (int it = 0; it < total; ++it) {
-        if (n_issued < total) issue(pi);
-        cp_async_commit();
-        advance(pi); ++n_issued;
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int u = 0; u < U; ++u) { sc[r][u][0] = nsc[r][u][0]; sc[r][u][1] = nsc[r][u][1]; bi[r][u] = nbi[r][u]; }
-        advance(pn);
-        if (it + 1 < total) {                       // scales one iteration ahead
-            const int c1 = lane + 32 * pn.i;
-            if (c1 < NC) {
-                int rowc[R];
-                rows_of(pn, rowc);
-                load_scales<FAM, T, R, U>(p, rowc, c1, sb, nsc, nbi);
-            }
-        }
-        cp_async_wait<S - 1>();                     // this lane's copies for iteration it landed
-        const int i = pc.i;
-        const int c = lane + 32 * i;
-        if (c < NC) {
-            uint32_t wv[R][CW];
-            const uint4* src = my + (size_t)pc.s * R * CV * 32 + lane;
-#pragma unroll
-            for (int r = 0; r < R; ++r)
-#pragma unroll
-                for (int q = 0; q < CV; ++q) {
-                    const uint4 t = src[(size_t)(r * CV + q) * 32];
-                    wv[r][4 * q] = t.x; wv[r][4 * q + 1] = t.y; wv[r][4 * q + 2] = t.z; wv[r][4 * q + 3] = t.w;
-                }
-            compute_chunk<FAM, B, MAXM, R, U>(wv, sc, bi, xs + (size_t)i * (C / 4) * 32 + lane,
-                                              (size_t)I * (C / 4) * 32, sx + (size_t)i * U * 32 + lane,
-                                              (size_t)I * U * 32, 32, acc);
-        }
-        if (i == I - 1) {                           // row block done: reduce and store
-            warp_allreduce<R, MAXM>(acc);
-            const long long rb = (long long)gw + (long long)pc.j * GW;
-#pragma unroll
-            for (int r = 0; r < R; ++r)
-#pragma unroll
-                for (int m = 0; m < MAXM; ++m) {
-                    const long long row = rb * R + r;
-                    if (lane == r * MAXM + m && row < p.N && m < p.M)
-                        DT<T>::st(Y, (long long)m * p.N + row, acc[r][m] * gs);
-                    acc[r][m] = 0.f;
-                }
-        }
-        advance(pc);
-    }
-    cp_async_wait<0>();
-    grid_launch_dependents();
-}
-
 // ------------------------------------------------- dequantization check ----
 // One thread per 32-code unit of one row; writes 32 fp32 weights.
 //   affine: fmaf(scale, c, bias) with c = (c * 2^p) * 2^-p (exact)
@@ -705,9 +526,9 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
         if constexpr (FAM == FAM_AFFINE) {
             const long long gi = n * (K / G) + k0 / G;
             const float s = DT<T>::ld(scales, gi), b = DT<T>::ld(biases, gi);
-#define QMV_D4(QQ) { unsigned long long d0 = magic_pair(field_bits<B, 4 * QQ>(wv), field_bits<B, 4 * QQ + 1>(wv)); \
-                     unsigned long long d1 = magic_pair(field_bits<B, 4 * QQ + 2>(wv), field_bits<B, 4 * QQ + 3>(wv)); \
-                     float c[4] = {lo(d0), hi(d0), lo(d1), hi(d1)}; \
+#define QMV_D4(QQ) { float2 d0 = magic_pair(field_bits<B, 4 * QQ>(wv), field_bits<B, 4 * QQ + 1>(wv)); \
+                     float2 d1 = magic_pair(field_bits<B, 4 * QQ + 2>(wv), field_bits<B, 4 * QQ + 3>(wv)); \
+                     float c[4] = {d0.x, d0.y, d1.x, d1.y}; \
                      _Pragma("unroll") for (int e = 0; e < 4; ++e) { \
                          const float q_ = __fmul_rn(c[e], __uint_as_float((127u - field_p(B, 4 * QQ + e)) << 23)); \
                          o[4 * QQ + e] = fmaf(s, q_, b); } }

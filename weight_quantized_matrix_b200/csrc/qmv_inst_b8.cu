@@ -11,12 +11,4 @@ cudaError_t launch_affine_b8(int dtype, int maxm, int R, bool wide, const Params
 #undef BITS_
 }
 
-cudaError_t launch_stream_affine_b8(int dtype, int maxm, int R, const Params& p, const Launch& L) {
-#define FAM_ FAM_AFFINE
-#define BITS_ 8
-    QMV_STREAM_DISPATCH_DTYPE()
-#undef FAM_
-#undef BITS_
-}
-
 }  // namespace qmv

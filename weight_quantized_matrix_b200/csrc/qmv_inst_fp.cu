@@ -26,37 +26,6 @@ static cudaError_t launch_mxfp8(int dtype, int maxm, int R, bool wide, const Par
 #undef BITS_
 }
 
-static cudaError_t stream_mxfp4(int dtype, int maxm, int R, const Params& p, const Launch& L) {
-#define FAM_ FAM_MXFP4
-#define BITS_ 4
-    QMV_STREAM_DISPATCH_DTYPE()
-#undef FAM_
-#undef BITS_
-}
-static cudaError_t stream_nvfp4(int dtype, int maxm, int R, const Params& p, const Launch& L) {
-#define FAM_ FAM_NVFP4
-#define BITS_ 4
-    QMV_STREAM_DISPATCH_DTYPE()
-#undef FAM_
-#undef BITS_
-}
-static cudaError_t stream_mxfp8(int dtype, int maxm, int R, const Params& p, const Launch& L) {
-#define FAM_ FAM_MXFP8
-#define BITS_ 8
-    QMV_STREAM_DISPATCH_DTYPE()
-#undef FAM_
-#undef BITS_
-}
-
-cudaError_t launch_stream_fp(int fam, int dtype, int maxm, int R, const Params& p, const Launch& L) {
-    switch (fam) {
-        case FAM_MXFP4: return stream_mxfp4(dtype, maxm, R, p, L);
-        case FAM_NVFP4: return stream_nvfp4(dtype, maxm, R, p, L);
-        case FAM_MXFP8: return stream_mxfp8(dtype, maxm, R, p, L);
-        default: return cudaErrorInvalidValue;
-    }
-}
-
 cudaError_t launch_fp(int fam, int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L) {
     switch (fam) {
         case FAM_MXFP4: return launch_mxfp4(dtype, maxm, R, wide, p, L);

@@ -1,0 +1,12 @@
+// qmv_inst_tc_b4.cu -- tensor-core affine 4-bit qmv kernels (all dtypes).
+#include "qmv_launch.cuh"
+
+namespace qmv {
+
+cudaError_t launch_tc_affine_b4(int dtype, int npass, const Params& p, const Launch& L) {
+#define BITS_ 4
+    QMV_TC_DISPATCH_DTYPE()
+#undef BITS_
+}
+
+}  // namespace qmv

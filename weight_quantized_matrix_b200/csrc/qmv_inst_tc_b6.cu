@@ -1,0 +1,12 @@
+// qmv_inst_tc_b6.cu -- tensor-core affine 6-bit qmv kernels (all dtypes).
+#include "qmv_launch.cuh"
+
+namespace qmv {
+
+cudaError_t launch_tc_affine_b6(int dtype, int npass, const Params& p, const Launch& L) {
+#define BITS_ 6
+    QMV_TC_DISPATCH_DTYPE()
+#undef BITS_
+}
+
+}  // namespace qmv

@@ -6,6 +6,7 @@
 #include <atomic>
 #include <cuda_runtime.h>
 #include "qmv_device.cuh"
+#include "qmv_tc.cuh"
 
 namespace qmv {
 
@@ -46,32 +47,6 @@ inline cudaError_t launch_kernel(Kern kern, std::atomic<unsigned>& configured, c
     return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
-// Persistent streaming kernels: L.grid.x is an upper bound (enough blocks for
-// every row block); it is capped to the number of blocks that are resident at
-// once (occupancy x SMs), so the blocks stay resident and stage x once.
-template <class Kern>
-inline cudaError_t launch_stream_kernel(Kern kern, std::atomic<unsigned>& configured, Launch L,
-                                        const Params& p) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    const unsigned bit = 1u << (dev & 31);
-    if (!(configured.load(std::memory_order_acquire) & bit)) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
-        if (e != cudaSuccess) return e;
-        configured.fetch_or(bit, std::memory_order_acq_rel);
-    }
-    int per_sm = 0, sms = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, (int)L.block.x, L.smem);
-    if (e != cudaSuccess) return e;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    const unsigned cap = (unsigned)per_sm * (unsigned)sms;
-    if (L.grid.x > cap) L.grid.x = cap;
-    return launch_kernel(kern, configured, L, p);
-}
-
 // dtype: 0 f32, 1 f16, 2 bf16.  Returns cudaErrorInvalidValue for a
 // (maxm, R, wide) combination that is not instantiated.
 cudaError_t launch_affine_b2(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
@@ -82,15 +57,10 @@ cudaError_t launch_affine_b6(int dtype, int maxm, int R, bool wide, const Params
 cudaError_t launch_affine_b8(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
 cudaError_t launch_fp(int fam, int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
 
-// Streaming kernels (qmv_stream_kernel, S = kStreamStages ring stages).
-constexpr int kStreamStages = 4;
-cudaError_t launch_stream_affine(int bits, int dtype, int maxm, int R, const Params& p, const Launch& L);
-cudaError_t launch_stream_fp(int fam, int dtype, int maxm, int R, const Params& p, const Launch& L);
-inline bool stream_instantiated(int maxm, int R) {
-    if (maxm == 1 || maxm == 2) return R == 2 || R == 4;
-    if (maxm == 4 || maxm == 8) return R == 1 || R == 2;
-    return false;
-}
+// Tensor-core kernels (qmv_tc_kernel): npass in {1, 2, 4}.
+cudaError_t launch_tc_affine(int bits, int dtype, int npass, const Params& p, const Launch& L);
+
+
 
 cudaError_t launch_dequant(int fam, int bits, int dtype, const uint8_t* w, const void* scales,
                            const void* biases, const float* gscale, float* out, int N, int K, int G,
@@ -120,20 +90,17 @@ inline bool shape_instantiated(int maxm, int R, bool wide) {
     QMV_SHAPE(T_, 8, 1, true) QMV_SHAPE(T_, 8, 2, true)                                      \
     QMV_SHAPE(T_, 1, 1, false) QMV_SHAPE(T_, 2, 1, false) QMV_SHAPE(T_, 4, 1, false)         \
     QMV_SHAPE(T_, 8, 1, false)
-#define QMV_STREAM_SHAPE(T_, MAXM_, R_)                                                      \
-    if (maxm == MAXM_ && R == R_) {                                                          \
+#define QMV_TC_SHAPE(T_, NPASS_)                                                             \
+    if (npass == NPASS_) {                                                                   \
         static std::atomic<unsigned> cfg_{0};                                                \
-        return launch_stream_kernel(qmv_stream_kernel<FAM_, BITS_, T_, MAXM_, R_, kStreamStages>, cfg_, L, p); \
+        return launch_kernel(qmv_tc_kernel<BITS_, T_, NPASS_, QMV_TC_PD(BITS_)>, cfg_, L, p); \
     }
-#define QMV_STREAM_ALL(T_)                                                                   \
-    QMV_STREAM_SHAPE(T_, 1, 2) QMV_STREAM_SHAPE(T_, 1, 4) QMV_STREAM_SHAPE(T_, 2, 2)          \
-    QMV_STREAM_SHAPE(T_, 2, 4) QMV_STREAM_SHAPE(T_, 4, 1) QMV_STREAM_SHAPE(T_, 4, 2)          \
-    QMV_STREAM_SHAPE(T_, 8, 1) QMV_STREAM_SHAPE(T_, 8, 2)
-#define QMV_STREAM_DISPATCH_DTYPE()                                                          \
+#define QMV_TC_PD(B_) (((B_) == 5 || (B_) == 6) ? 2 : 4)
+#define QMV_TC_DISPATCH_DTYPE()                                                              \
     switch (dtype) {                                                                         \
-        case 0: { QMV_STREAM_ALL(float) break; }                                             \
-        case 1: { QMV_STREAM_ALL(__half) break; }                                            \
-        case 2: { QMV_STREAM_ALL(__nv_bfloat16) break; }                                     \
+        case 0: { QMV_TC_SHAPE(float, 1) QMV_TC_SHAPE(float, 2) QMV_TC_SHAPE(float, 4) break; }                 \
+        case 1: { QMV_TC_SHAPE(__half, 1) QMV_TC_SHAPE(__half, 2) QMV_TC_SHAPE(__half, 4) break; }              \
+        case 2: { QMV_TC_SHAPE(__nv_bfloat16, 1) QMV_TC_SHAPE(__nv_bfloat16, 2) QMV_TC_SHAPE(__nv_bfloat16, 4) break; } \
         default: break;                                                                      \
     }                                                                                        \
     return cudaErrorInvalidValue;
