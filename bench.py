@@ -5,7 +5,7 @@
                     [--workload chain8|layer|probe]
 
 Prints ONE JSON line (rank 0).  Metric: qmv microseconds per call and achieved
-HBM GB/s.  Workloads (synthetic, seeded; see the design doc for the recipes):
+HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
 
   chain8 (default)  affine 8-bit, group 64, bf16, M=1, K=2560, output sizes
                     N in {1, 4, 3, 5, 12, 17, 4096}; for each N a chain of 64
@@ -18,12 +18,14 @@ HBM GB/s.  Workloads (synthetic, seeded; see the design doc for the recipes):
   probe             bandwidth probe, affine 4-bit g64 bf16, N=K=16384, M=1.
 
 Timing: W untimed warm-up steps, then K steps; each step is bracketed by CUDA
-events on the launching stream; L2 is flushed (a 512 MB buffer is written)
-before every step, outside the events, and within a step the weights rotate
+events on the launching stream; L2 is flushed before every step, outside the
+events (a 512 MB buffer is written, then a 256 MB buffer is read so that no
+dirty line's write-back falls inside the timed region), and within a step the weights rotate
 through copies totalling more than twice the L2 so calls read from HBM.  The
 timed region is bracketed by a barrier and a device synchronize; multi-GPU runs
 are N independent replicas (the path has no exchange step) and report the max
-over ranks.  nvidia-smi clocks are sampled during the timed region.
+over ranks.  nvidia-smi clocks are sampled (20 ms) from the graph warm-up through
+the timed region.
 
 --impl reference times the fp64 CPU oracle (the only other implementation of
 this operation there is) on a bounded sample of the same workload, on the host
@@ -93,7 +95,10 @@ def traffic_for(kernel_key):
 
 # ----------------------------------------------------------------- clocks --
 class ClockSampler:
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples (20 ms period) taken while the GPU is under load: it
+    is started before the warm-up replays and stopped after the timed steps,
+    so the window covers the timed region with load on both sides."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -109,13 +114,16 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "20"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while time.time() - t0 < 3.0 and os.path.getsize(self.path) == 0:
+                time.sleep(0.01)
         except (OSError, ValueError):
             self.proc = None
 
     def stop(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -123,18 +131,26 @@ class ClockSampler:
             self.proc.kill()
         rows = [r.split(", ") for r in open(self.path).read().strip().splitlines() if r.strip()]
         os.unlink(self.path)
-        sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+        rows = [r for r in rows if len(r) >= 10]
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        mx = [num(r[3]) for r in rows if num(r[3]) is not None]
+        pw = [num(r[4]) for r in rows if num(r[4]) is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = set()
         for r in rows:
-            if len(r) < 9:
-                continue
-            for n, v in zip(names, r[5:9]):
+            for n, v in zip(names, r[6:10]):
                 if v.strip() == "Active":
                     reasons.add(n)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(rows)}
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(pw) if pw else None,
+                "window": "warm-up replays + timed steps (continuous load), 20 ms period"}
 
 
 # -------------------------------------------------------------- workloads --
@@ -196,7 +212,7 @@ class Chain8:
         return {"workload": self.name, "bits": 8, "group": 64, "dtype": "bf16", "M": 1, "K": CHAIN_K,
                 "N": CHAIN_NS, "calls_per_N": CHAIN_CALLS, "calls_per_step": self.calls_per_step,
                 "chain": "x_{t+1} = y_t zero-padded (N<K) / truncated (N>=K) to K",
-                "l2": "flushed before every step (512 MB write); weights rotate through copies > 2x L2"}
+                "l2": "flushed before every step (512 MB write + 256 MB read); weights rotate through copies > 2x L2"}
 
 
 class Layer:
@@ -248,7 +264,7 @@ class Layer:
     def config(self):
         return {"workload": self.name, "bits": 4, "group": 64, "dtype": "bf16", "M": [1, 8],
                 "shapes_NxK": [[n, k] for _, n, k in LAYER], "calls_per_step": self.calls_per_step,
-                "l2": "flushed before every step (512 MB write); weights rotate through copies > 2x L2"}
+                "l2": "flushed before every step (512 MB write + 256 MB read); weights rotate through copies > 2x L2"}
 
 
 class Probe(Layer):
@@ -267,7 +283,7 @@ class Probe(Layer):
 
     def config(self):
         return {"workload": self.name, "bits": 4, "group": 64, "dtype": "bf16", "M": 1, "N": 16384, "K": 16384,
-                "calls_per_step": 1, "l2": "flushed before every step (512 MB write); 3 weight copies rotate"}
+                "calls_per_step": 1, "l2": "flushed before every step (512 MB write + 256 MB read); 3 weight copies rotate"}
 
 
 WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe}
@@ -286,6 +302,10 @@ def run_ours(args, rank, world, local_rank):
     wl = WORKLOADS[args.workload](q, torch, dev)
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    # after the write pass, a read pass over another buffer larger than the L2
+    # evicts the dirty lines, so their write-back is not charged to the timed
+    # kernels; the L2 then holds only unrelated clean lines
+    flush_rd = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
     groups = wl.groups()
     W = max(3, args.warmup)
 
@@ -307,9 +327,16 @@ def run_ours(args, rank, world, local_rank):
                     wl.run_group(s)
                 gs.append(g)
             graphs.append(gs)
-        for k in range(W):
+        clk = ClockSampler(local_rank)
+        clk.start()
+        t_load = time.perf_counter()
+        k = 0
+        while k < W or time.perf_counter() - t_load < 0.3:     # warm-up replays, >= 0.3 s of load
             for gs in graphs:
                 gs[k % len(gs)].replay()
+            k += 1
+            if k % 16 == 0:
+                torch.cuda.synchronize()
         torch.cuda.synchronize()
 
         def timed(e2e):
@@ -318,12 +345,10 @@ def run_ours(args, rank, world, local_rank):
             if world > 1:
                 dist.barrier()
             torch.cuda.synchronize()
-            clk = ClockSampler(local_rank)
-            if not e2e:
-                clk.start()
             t0 = time.perf_counter()
             for k in range(args.steps):
                 flush.fill_(k & 0xFF)                   # L2 flush, outside the events
+                flush_rd.max()
                 for gi, (_, s) in enumerate(groups):
                     ev[k][gi][0].record(stream)
                     if e2e:
@@ -364,10 +389,11 @@ def run_ours(args, rank, world, local_rank):
         n = wl.calls_per_step // len(groups) if isinstance(wl, Chain8) else 1
         b = wl.group_bytes(s)
         plan = wl.group_plan(s)
+        kern = " ".join(w for w in plan.split() if w.split("=")[0] in ("path", "chunk", "maxm", "rows_per_warp"))
         gbs = b / (ms * 1e-3) / 1e9
         shapes.append({"shape": label, "us_per_call": round(ms * 1e3 / n, 3), "GB_s": round(gbs, 1),
                        "frac_of_hbm": round(gbs / peak, 4), "plan": plan})
-        k = by_kernel.setdefault(plan, {"ms": 0.0, "launches": 0, "bytes": 0})
+        k = by_kernel.setdefault(kern, {"ms": 0.0, "launches": 0, "bytes": 0})
         k["ms"] += ms; k["launches"] += n; k["bytes"] += b
     dom_plan, dom = max(by_kernel.items(), key=lambda kv: kv[1]["ms"])
     achieved = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
@@ -394,11 +420,11 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ------------------------------------------------- oracle (CPU) baseline --
-def _oracle_sample(workload, budget_s=12.0):
+def _oracle_sample(workload, budget_s=12.0, threads=None):
     """Time the oracle, as it stands, on a bounded sample of the workload and
     scale to microseconds per call of the full workload."""
     import oracle
-    threads = os.cpu_count() or 1
+    threads = threads or os.cpu_count() or 1
     t_by = {}
     if workload == "chain8":
         spec = [(1, N, CHAIN_K, CHAIN_BITS, CHAIN_G, CHAIN_CALLS) for N in CHAIN_NS]
@@ -431,28 +457,34 @@ def _oracle_sample(workload, budget_s=12.0):
 
 
 def cpu_baseline(workload):
-    v, cores, sample = _oracle_sample(workload)
+    v, cores, sample = _oracle_sample(workload, budget_s=12.0)
+    v1, _, sample1 = _oracle_sample(workload, budget_s=4.0, threads=1)
     return {"value": round(v, 2), "unit": "us/call", "cores": cores, "kind": "oracle",
-            "sample": "fp64 C oracle over row samples of every shape, scaled to full calls: " + sample}
+            "sample": "fp64 C oracle over row samples of every shape, scaled to full calls: " + sample,
+            "value_1thread": round(v1, 2), "sample_1thread": sample1}
 
 
 def run_reference(args, rank, world):
+    """The oracle on the host cores, rank 0 only.  Each step is one bounded
+    sample of the workload; the per-step budget keeps the whole run near a
+    minute whatever --steps is."""
     if rank != 0:
         return
-    wl = {"chain8": Chain8, "layer": Layer, "probe": Probe}[args.workload]
+    wl = WORKLOADS[args.workload]
+    budget = max(0.2, min(6.0, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        _oracle_sample(args.workload, budget_s=budget)
     vals = []
-    for _ in range(max(1, args.warmup) if False else 0):
-        pass
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        v, cores, sample = _oracle_sample(args.workload, budget_s=6.0)
+        v, cores, sample = _oracle_sample(args.workload, budget_s=budget)
         vals.append(v)
     v = float(np.mean(vals))
-    cfg = {"workload": wl.name}
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "us/call", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)", "config": cfg,
+        "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
+        "config": {"workload": wl.name},
         "ms_per_step": round((time.perf_counter() - t0) * 1e3 / max(1, args.steps), 2),
         "cpu_baseline": {"value": round(v, 2), "unit": "us/call", "cores": cores, "kind": "oracle",
                          "sample": sample},
@@ -463,7 +495,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="chain8")
