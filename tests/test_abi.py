@@ -149,3 +149,15 @@ def test_plan_no_n_cliff():
     assert "path=narrow" in q.qmv_describe_plan("affine", 1, 64, 4096, bits=4, group_size=32, w_align16=False)
     # 3-bit tensor-core units are 12 bytes: 4-byte alignment is enough
     assert "path=tc" in q.qmv_describe_plan("affine", 4, 64, 4096, bits=3, group_size=32, w_align16=False)
+
+
+def test_fast_extension_forwards_status():
+    """The CPython entry points are the in-tree extension over the same
+    library and return the C ABI's status unchanged."""
+    assert os.path.dirname(q._fast.__file__) == os.path.dirname(q.LIB_PATH.rsplit("/lib/", 1)[0] + "/")
+    assert q._fast.affine(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 128, 7, 64, 2, 1, 1, 0) == EUNSUP
+    assert q._fast.affine(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 96, 4, 64, 2, 1, 1, 0) == EINVAL
+    assert q._fast.fp(FAKE, FAKE, FAKE, None, FAKE, 1, 8, 128, 1, 2, 1, 1, 0) == EINVAL
+    assert q._fast.affine(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 128, 4, 64, 2, 1, 1, 0) == 0
+    with pytest.raises(TypeError):
+        q._fast.affine(FAKE)

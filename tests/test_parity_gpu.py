@@ -413,6 +413,89 @@ def test_tensor_core_x_tiles(q):
     compare(y, ref, ad, "f32", what="tc tiles")
 
 
+# ------------------------------------------ tensor cores + bulk-copy ring ----
+@pytest.fixture
+def ring(q):
+    """Force the bulk-ring kernel; afterwards no bounded wait may have expired."""
+    q.qmv_device_fault(clear=True)
+    yield
+    torch.cuda.synchronize()
+    assert q.qmv_device_fault(clear=True) == 0
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("group", GROUPS)
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_bulk_ring_path_grid(q, ring, bits, group, dtype, M):
+    """The bulk-ring kernel on every width / group / dtype (2-bit with group
+    32 falls back: a 64-code unit would span two groups)."""
+    q.qmv_force_config(4, -1, -1, -1)
+    N, K = 100, 1024
+    plan = q.qmv_describe_plan("affine", M, N, K, bits, group, dtype)
+    assert ("path=tcb" in plan) == (not (bits == 2 and group == 32)), plan
+    c = synth.affine_case(M, N, K, bits, group, dtype, seed=_seed("tcb", bits, group, dtype, M))
+    y = run_affine(q, c)[0]
+    ref, ad = oracle_affine(c)
+    compare(y, ref, ad, dtype, what=f"tcb b{bits} g{group} {dtype} M{M}")
+
+
+@pytest.mark.parametrize("cfg", [(4, -1, 1, 1), (4, -1, 8, 1), (4, -1, 1, 8), (4, -1, 2, 4), (4, -1, 4, 2),
+                                 (4, -1, 3, 2)])
+@pytest.mark.parametrize("bits", [2, 3, 5, 8])
+def test_bulk_ring_block_shapes(q, ring, cfg, bits):
+    q.qmv_force_config(*cfg)
+    c = synth.affine_case(2, 333, 2048, bits, 64, "bf16", seed=_seed("tcbshape", cfg, bits), batch=2)
+    assert "path=tcb" in q.qmv_describe_plan("affine", 2, 333, 2048, bits, 64, "bf16")
+    y = run_affine(q, c)
+    for b in range(2):
+        ref, ad = oracle_affine(c, b=b)
+        compare(y[b], ref, ad, "bf16", what=f"tcb shape {cfg} b{bits} batch{b}")
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+@pytest.mark.parametrize("M", [1, 3])
+def test_bulk_ring_persistent_row_blocks(q, ring, bits, M):
+    """More row blocks than SMs: each block walks several row blocks and the
+    ring runs across their boundaries; K = 5760 leaves a ragged last stage."""
+    q.qmv_force_config(4, -1, 8, 1)
+    N, K = 16 * 148 * 2 + 37, 5760
+    c = synth.affine_case(M, N, K, bits, 64, "bf16", seed=_seed("tcbpers", bits, M))
+    plan = q.qmv_describe_plan("affine", M, N, K, bits, 64, "bf16")
+    assert "path=tcb" in plan and "grid=148 " in plan, plan
+    y = run_affine(q, c)[0]
+    rows = sorted(set(sample_rows(N, 96)) | {0, 15, 16, N - 38, N - 37, N - 1})
+    ref, ad = oracle_affine(c, rows=rows)
+    compare(y[:, rows], ref[:, rows], ad[:, rows], "bf16", what=f"tcb persistent b{bits} M{M}")
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_bulk_ring_tail_rows_bitwise_prefix(q, ring, bits):
+    q.qmv_force_config(4, -1, 2, 1)            # 16-row tiles, K over 2 warps
+    K = 2560
+    big = synth.affine_case(1, 48, K, bits, 64, "bf16", seed=_seed("tcbtail", bits))
+    yb = run_affine(q, big)[0]
+    for n in (1, 5, 17, 33):
+        small = dict(big, N=n, w=big["w"][:, :n].copy(), scales=big["scales"][:, :n].copy(),
+                     biases=big["biases"][:, :n].copy())
+        assert np.array_equal(run_affine(q, small)[0], yb[:, :n])
+
+
+@pytest.mark.parametrize("N", [80, 16 * 148 + 5])
+def test_bulk_ring_x_tiles(q, ring, N):
+    """M=8, f32 x, K large enough that x is staged in several K tiles (and,
+    with more row blocks than SMs, staged again for every row block)."""
+    q.qmv_force_config(4, -1, 8, 1)
+    K = 16384
+    plan = q.qmv_describe_plan("affine", 8, N, K, 4, 32, "f32")
+    assert "path=tcb" in plan and "tile_iters=128" not in plan, plan
+    c = synth.affine_case(8, N, K, 4, 32, "f32", seed=_seed("tcbtile", N))
+    y = run_affine(q, c)[0]
+    rows = list(range(N)) if N <= 80 else sorted(set(sample_rows(N, 48)) | {N - 1})
+    ref, ad = oracle_affine(c, rows=rows)
+    compare(y[:, rows], ref[:, rows], ad[:, rows], "f32", what="tcb tiles")
+
+
 @pytest.mark.parametrize("bits", [3, 4, 8])
 def test_cuda_core_path_grid(q, bits):
     """The CUDA-core kernel (wide and narrow chunks) stays covered."""

@@ -4,6 +4,8 @@ matrix-vector product on B200.
 Argument marshalling only.  Every function takes device buffers as torch
 tensors (or raw integer device addresses), passes their pointers and sizes to
 the C ABI of the same name, and raises :class:`QmvError` on a non-zero status.
+The per-call entry points go through the CPython extension ``_qmv_fast``
+(csrc/qmv_py.c), the rest through ctypes.
 All compute happens in the CUDA kernels of libqmv.so; there is no fallback: if
 the library has not been built, importing this package raises ImportError.
 
@@ -33,6 +35,12 @@ if not os.path.exists(LIB_PATH):
         "`python -m weight_quantized_matrix_b200.build_lib` (needs nvcc)")
 
 _lib = ctypes.CDLL(LIB_PATH)
+try:
+    from . import _qmv_fast as _fast      # per-call entry points (CPython extension over libqmv.so)
+except ImportError as _e:
+    raise ImportError(
+        "the _qmv_fast extension is missing; build it with "
+        "`python -m weight_quantized_matrix_b200.build_lib` (needs gcc)") from _e
 _p, _i, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong
 _lib.qmv_affine.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
 _lib.qmv_affine_batched.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p]
@@ -44,10 +52,12 @@ _lib.qmv_status_string.argtypes = [_i]
 _lib.qmv_status_string.restype = ctypes.c_char_p
 _lib.qmv_last_cuda_error.argtypes = []
 _lib.qmv_describe_plan.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, ctypes.c_char_p, _i]
+_lib.qmv_device_fault.argtypes = [ctypes.POINTER(ctypes.c_uint), _i]
 _lib.qmv_force_config.argtypes = [_i, _i, _i, _i]
 _lib.qmv_force_config.restype = None
 for _f in ("qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
-           "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_last_cuda_error", "qmv_describe_plan"):
+           "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_last_cuda_error", "qmv_describe_plan",
+           "qmv_device_fault"):
     getattr(_lib, _f).restype = _i
 
 
@@ -86,10 +96,20 @@ def _mode(m):
     return m if isinstance(m, int) else FP_MODES[m]
 
 
+_raw_stream = None
+
+
 def _stream(s):
+    global _raw_stream
     if s is None:
-        import torch
-        return torch.cuda.current_stream().cuda_stream
+        if _raw_stream is None:
+            import torch
+            c = torch._C
+            if hasattr(c, "_cuda_getCurrentRawStream") and hasattr(c, "_cuda_getDevice"):
+                _raw_stream = lambda: c._cuda_getCurrentRawStream(c._cuda_getDevice())  # noqa: E731
+            else:
+                _raw_stream = lambda: torch.cuda.current_stream().cuda_stream  # noqa: E731
+        return _raw_stream()
     if isinstance(s, int):
         return s
     return s.cuda_stream
@@ -101,27 +121,30 @@ def _check(st, what):
 
 
 def qmv_affine(x, w_packed, scales, biases, y, M, N, K, bits, group_size, dtype, stream=None):
-    _check(_lib.qmv_affine(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(biases), _ptr(y), M, N, K,
-                           bits, group_size, _dtype(dtype), _stream(stream)), "qmv_affine")
+    st = _fast.affine(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(biases), _ptr(y), M, N, K, bits, group_size,
+                      _dtype(dtype), 1, 1, _stream(stream))
+    if st:
+        raise QmvError(st, "qmv_affine")
 
 
 def qmv_affine_batched(x, w_packed, scales, biases, y, M, N, K, bits, group_size, dtype, batch,
                        x_batched=True, stream=None):
-    _check(_lib.qmv_affine_batched(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(biases), _ptr(y), M, N, K,
-                                   bits, group_size, _dtype(dtype), batch, int(bool(x_batched)),
-                                   _stream(stream)), "qmv_affine_batched")
+    _check(_fast.affine(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(biases), _ptr(y), M, N, K, bits,
+                        group_size, _dtype(dtype), batch, int(bool(x_batched)), _stream(stream)),
+           "qmv_affine_batched")
 
 
 def qmv_fp(x, w_packed, scales, global_scale, y, M, N, K, mode, dtype, stream=None):
-    _check(_lib.qmv_fp(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(global_scale), _ptr(y), M, N, K,
-                       _mode(mode), _dtype(dtype), _stream(stream)), "qmv_fp")
+    st = _fast.fp(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(global_scale), _ptr(y), M, N, K, _mode(mode),
+                  _dtype(dtype), 1, 1, _stream(stream))
+    if st:
+        raise QmvError(st, "qmv_fp")
 
 
 def qmv_fp_batched(x, w_packed, scales, global_scale, y, M, N, K, mode, dtype, batch, x_batched=True,
                    stream=None):
-    _check(_lib.qmv_fp_batched(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(global_scale), _ptr(y), M, N,
-                               K, _mode(mode), _dtype(dtype), batch, int(bool(x_batched)),
-                               _stream(stream)), "qmv_fp_batched")
+    _check(_fast.fp(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(global_scale), _ptr(y), M, N, K, _mode(mode),
+                    _dtype(dtype), batch, int(bool(x_batched)), _stream(stream)), "qmv_fp_batched")
 
 
 def qmv_dequant_affine_f32(w_packed, scales, biases, w_out, N, K, bits, group_size, dtype, stream=None):
@@ -150,6 +173,14 @@ def qmv_describe_plan(family, M, N, K, bits=4, group_size=64, dtype="bf16", w_al
     _check(_lib.qmv_describe_plan(fam, M, N, K, bits, group_size, _dtype(dtype), int(w_align16), buf, 256),
            "qmv_describe_plan")
     return buf.value.decode()
+
+
+def qmv_device_fault(clear=False) -> int:
+    """Fault word of the current device (nonzero: a bounded wait in a kernel
+    expired and that call's output is undefined); synchronous."""
+    code = ctypes.c_uint(0)
+    _check(_lib.qmv_device_fault(ctypes.byref(code), int(bool(clear))), "qmv_device_fault")
+    return code.value
 
 
 def qmv_force_config(path=-1, rows_per_warp=-1, warps_k=-1, warps_rows=-1):

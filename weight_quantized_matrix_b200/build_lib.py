@@ -4,7 +4,8 @@
 
 Each kernel family compiles in its own nvcc process (in parallel); the objects
 are linked into ``weight_quantized_matrix_b200/lib/libqmv.so`` with the CUDA
-runtime linked statically, so the library needs only the NVIDIA driver.
+runtime linked statically, so the library needs only the NVIDIA driver.  The
+CPython extension ``_qmv_fast`` (csrc/qmv_py.c, gcc) is linked against it.
 """
 from __future__ import annotations
 
@@ -34,6 +35,32 @@ def nvcc() -> str:
     return path
 
 
+def _ext_path() -> str:
+    import sysconfig
+    return os.path.join(HERE, "_qmv_fast" + sysconfig.get_config_var("EXT_SUFFIX"))
+
+
+def build_ext() -> str:
+    """The CPython extension _qmv_fast (per-call entry points, linked to libqmv.so)."""
+    import sysconfig
+    src = os.path.join(CSRC, "qmv_py.c")
+    out = _ext_path()
+    if (os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src)
+            and os.path.getmtime(out) >= os.path.getmtime(LIB)):
+        return out
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if not cc:
+        raise RuntimeError("gcc not found: needed to build the _qmv_fast extension")
+    cmd = [cc, "-O2", "-shared", "-fPIC", "-Wall", "-I", sysconfig.get_paths()["include"],
+           "-I", os.path.join(ROOT, "include"), src, "-L", LIBDIR, "-lqmv", "-Wl,-rpath,$ORIGIN/lib",
+           "-o", out + ".tmp"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"building _qmv_fast failed:\n{r.stdout}\n{r.stderr}")
+    os.replace(out + ".tmp", out)
+    return out
+
+
 def _deps():
     return (glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
             + [os.path.join(ROOT, "include", "qmv.h")])
@@ -48,6 +75,7 @@ def up_to_date() -> bool:
 
 def build(force: bool = False, jobs: int | None = None, verbose: bool = False) -> str:
     if not force and up_to_date():
+        build_ext()
         return LIB
     os.makedirs(OBJ, exist_ok=True)
     os.makedirs(LIBDIR, exist_ok=True)
@@ -73,6 +101,7 @@ def build(force: bool = False, jobs: int | None = None, verbose: bool = False) -
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
+    build_ext()
     return LIB
 
 

@@ -29,7 +29,7 @@ thread_local int g_last_cuda = 0;
 struct Forced { int path = -1, R = -1, wk = -1, wr = -1; };
 Forced g_forced;
 
-struct DevInfo { int sms = 0; int ok = 0; };
+struct DevInfo { int sms = 0; int ok = 0; unsigned* fault = nullptr; };
 DevInfo g_dev[64];
 std::mutex g_dev_mu;
 
@@ -51,6 +51,29 @@ int device_sms() {
 
 int elem_bytes(int dtype) { return dtype == QMV_F32 ? 4 : 2; }
 
+}  // namespace
+
+// Fault word of the bulk-ring kernels: a bounded wait that expired ORs its
+// code in (1: consumer, full stage; 2: producer, empty stage; 4: producer,
+// own copies).  Zero at module load; read and cleared by qmv_device_fault.
+__device__ unsigned g_qmv_fault;
+
+namespace {
+
+// Device address of g_qmv_fault on the current device (looked up once per
+// device); nullptr if the lookup fails.
+unsigned* fault_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) { cudaGetLastError(); return nullptr; }
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!g_dev[dev].fault) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_qmv_fault) != cudaSuccess) { cudaGetLastError(); return nullptr; }
+        g_dev[dev].fault = static_cast<unsigned*>(a);
+    }
+    return g_dev[dev].fault;
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Per-format facts the picker needs (mirrors qmv::Fmt).
@@ -65,7 +88,8 @@ FmtInfo fmt_info(int fam, int bits) {
 }
 
 struct Plan {
-    int maxm, R, wide, tc, npass, wk, wr, tile_iters, C;
+    int maxm, R, wide, tc, npass, wk, wr, tile_iters, C;   // tc: 0 CUDA cores, 1 tensor cores, 2 + bulk ring
+    int sps = 0, pitch = 0;
     size_t smem;
     dim3 grid, block;
 };
@@ -147,6 +171,66 @@ bool tc_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, TcShape
     return ts->gx <= 0x7FFFFFFFLL && ts->smem <= (size_t)qmv::kMaxSmem;
 }
 
+// ---- bulk-ring tensor-core launch shape ----------------------------------------
+// Row blocks of 16*wr rows are spread over a persistent grid of one block per
+// SM, wk consumer warps split K.  wr = 2, wk = 4 measured best or within a few
+// percent of best on B200 for 4K..28K rows (M = 1..8).  A ring stage holds
+// about 32 KB; the x tile takes what shared memory is left.
+struct TcbShape { int npass, wk, wr, tsb, sps, pitch; long long gx; size_t smem; };
+
+bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, TcbShape* ts) {
+    const int ub = tc_unit_bytes(bits);
+    const int uc = ub * 8 / bits;
+    const int SB = 4 * uc;
+    if (K % SB != 0 || !w16) return false;
+    if (((long long)K * bits / 8) % 16 != 0) return false;     // bulk copies: 16-byte rows
+    if (bits == 2 && G < 64) return false;
+    const int segsz = G < SB ? G : SB;
+    const int ngs = SB / segsz;
+    const int cols = M * ngs;
+    const int npass = cols <= 8 ? 1 : cols <= 16 ? 2 : cols <= 32 ? 4 : 0;
+    if (npass == 0) return false;
+    const int nsplit = dtype == QMV_BF16 ? 1 : dtype == QMV_F16 ? 2 : 3;
+    const int np = tc_np_of(bits);
+    const int nsbk = K / SB;
+    const int sms = device_sms();
+    int wr = 2;
+    int wk = 4;
+    if (g_forced.wr > 0) wr = g_forced.wr > 8 ? 8 : g_forced.wr;
+    if (g_forced.wk > 0) wk = g_forced.wk > 8 ? 8 : g_forced.wk;
+    while (wk * wr > 8) --wk;
+    if (wk > nsbk) wk = nsbk;
+    if (wk < 1) wk = 1;
+    const int rows = 16 * wr;
+    int sps = 32768 / (rows * 4 * ub);
+    sps = sps / wk * wk;
+    if (sps < wk) sps = wk;
+    if (sps > nsbk) sps = nsbk;
+    auto pitch_of = [&](int s) { return ((s * 4 * ub + 127) / 128) * 128 + (ub == 16 ? 64 : 16); };
+    const int ncw = wk * wr;
+    const size_t red = (size_t)ncw * 16 * 8 * npass * 4;
+    const size_t per_sb = (size_t)nsplit * M * 4 * np * 4 + (size_t)M * ngs * 4 * 2 + (size_t)M * 4 * 2 * 4;
+    long long tsb = 0;
+    size_t fixed = 0;
+    for (;;) {
+        fixed = 128 + (size_t)qmv::kTcbStages * rows * pitch_of(sps) + red + (size_t)nsplit * (M * 4 + 4 * np + 4) * 4;
+        tsb = fixed < (size_t)qmv::kMaxSmem ? (long long)(((size_t)qmv::kMaxSmem - fixed) / per_sb) : 0;
+        if (tsb >= nsbk) { tsb = nsbk; break; }
+        tsb = tsb / sps * sps;
+        if (tsb >= sps) break;
+        if (sps <= 1) return false;
+        sps = sps > wk ? (sps / 2 / wk) * wk : sps / 2;
+        if (sps < 1) sps = 1;
+    }
+    const long long nrb = ((long long)N + rows - 1) / rows;
+    ts->npass = npass; ts->wk = wk; ts->wr = wr; ts->tsb = (int)tsb; ts->sps = sps; ts->pitch = pitch_of(sps);
+    ts->gx = nrb < sms ? nrb : sms;
+    const size_t plane = (size_t)M * ((size_t)tsb * 4 * np + 4) + 4 * np + 4;
+    ts->smem = 128 + (size_t)qmv::kTcbStages * rows * ts->pitch + (size_t)nsplit * plane * 4 +
+               (size_t)M * tsb * ngs * 4 * 2 + (size_t)M * tsb * 4 * 2 * 4 + red;
+    return ts->smem <= (size_t)qmv::kMaxSmem;
+}
+
 // Choose the launch shape.  Returns QMV_OK or an error (sizes too large).
 int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, bool w16, int batch, Plan* pl) {
     const FmtInfo fi = fmt_info(fam, bits);
@@ -155,6 +239,20 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     const int c_wide = 32 * fi.wide_units;
     bool wide = w16 && (K % c_wide == 0);
     if (g_forced.path == 0) wide = false;
+
+    // ---- tensor-core kernel with the bulk-copy weight ring --------------------
+    // (measured: wins over the register-prefetch kernel once M >= 2)
+    if (aff && K > 0 && (g_forced.path == 4 || (g_forced.path < 0 && M >= 2 && tc_preferred(M, N, K, bits)))) {
+        TcbShape ts;
+        if (tcb_shape(M, N, K, bits, G_of_plan, dtype, w16, &ts)) {
+            pl->maxm = maxm; pl->R = 1; pl->wide = 1; pl->tc = 2; pl->npass = ts.npass;
+            pl->wk = ts.wk; pl->wr = ts.wr; pl->tile_iters = ts.tsb; pl->sps = ts.sps; pl->pitch = ts.pitch;
+            pl->C = 4 * tc_unit_bytes(bits) * 8 / bits; pl->smem = ts.smem;
+            pl->grid = dim3((unsigned)ts.gx, 1, (unsigned)batch);
+            pl->block = dim3(32 * (ts.wk * ts.wr + 1), 1, 1);
+            return QMV_OK;
+        }
+    }
 
     // ---- tensor-core kernel (affine, enough rows to fill the GPU) -------------
     if (aff && K > 0 && g_forced.path != 0 && g_forced.path != 1 &&
@@ -282,10 +380,13 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     p.w_row = row_bytes;
     qmv::Launch L{pl.grid, pl.block, pl.smem, static_cast<cudaStream_t>(stream), pdl_enabled()};
     cudaError_t e;
-    if (pl.tc) {
-        p.tile_iters = pl.tile_iters;
-        return finish(qmv::launch_tc_affine(bits, dtype, pl.npass, p, L));
+    p.sps = pl.sps; p.pitch = pl.pitch; p.fault = nullptr;
+    if (pl.tc == 2) {
+        p.fault = fault_word();
+        if (!p.fault) return QMV_ECUDA;
+        return finish(qmv::launch_tcb_affine(bits, dtype, pl.npass, p, L));
     }
+    if (pl.tc) return finish(qmv::launch_tc_affine(bits, dtype, pl.npass, p, L));
     if (fam == qmv::FAM_AFFINE) {
         switch (bits) {
             case 2: e = qmv::launch_affine_b2(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
@@ -435,10 +536,22 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
     if (st != QMV_OK) return st;
     snprintf(buf, (size_t)buflen,
              "path=%s chunk=%d maxm=%d rows_per_warp=%d warps_k=%d warps_rows=%d tile_iters=%d "
-             "grid=%u block=%u smem=%zu",
-             pl.tc ? "tc" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr, pl.tile_iters,
-             pl.grid.x, pl.block.x, pl.smem);
+             "grid=%u block=%u smem=%zu stage_sb=%d",
+             pl.tc == 2 ? "tcb" : pl.tc ? "tc" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr,
+             pl.tile_iters, pl.grid.x, pl.block.x, pl.smem, pl.sps);
     return QMV_OK;
+}
+
+int qmv_device_fault(unsigned int* code, int clear) {
+    if (!code) return QMV_EINVAL;
+    *code = 0;
+    if (!fault_word()) return QMV_ECUDA;
+    cudaError_t e = cudaMemcpyFromSymbol(code, g_qmv_fault, sizeof(unsigned));
+    if (e == cudaSuccess && clear) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_qmv_fault, &zero, sizeof(unsigned));
+    }
+    return finish(e);
 }
 
 void qmv_force_config(int path, int rows_per_warp, int warps_k, int warps_rows) {

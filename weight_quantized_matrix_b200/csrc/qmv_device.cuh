@@ -67,6 +67,9 @@ struct Params {
     long long s_bs;         // scales/biases batch stride in elements
     long long y_bs;         // y batch stride in elements
     long long w_row;        // bytes per packed row
+    int sps;                // bulk-ring kernel: super-blocks per ring stage
+    int pitch;              // bulk-ring kernel: bytes per ring row
+    unsigned* fault;        // bulk-ring kernel: device fault word (bounded waits that expired)
 };
 
 // ---------------------------------------------------------------- dtypes ---

@@ -1,0 +1,13 @@
+// qmv_inst_tcb_b6.cu -- tensor-core affine 6-bit qmv kernels with the bulk-copy
+// weight ring (all dtypes).
+#include "qmv_launch.cuh"
+
+namespace qmv {
+
+cudaError_t launch_tcb_affine_b6(int dtype, int npass, const Params& p, const Launch& L) {
+#define BITS_ 6
+    QMV_TCB_DISPATCH_DTYPE()
+#undef BITS_
+}
+
+}  // namespace qmv

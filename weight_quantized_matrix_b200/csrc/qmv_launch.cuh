@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include "qmv_device.cuh"
 #include "qmv_tc.cuh"
+#include "qmv_tcb.cuh"
 
 namespace qmv {
 
@@ -59,6 +60,9 @@ cudaError_t launch_fp(int fam, int dtype, int maxm, int R, bool wide, const Para
 
 // Tensor-core kernels (qmv_tc_kernel): npass in {1, 2, 4}.
 cudaError_t launch_tc_affine(int bits, int dtype, int npass, const Params& p, const Launch& L);
+// Tensor-core kernels with the bulk-copy weight ring (qmv_tcb_kernel).
+cudaError_t launch_tcb_affine(int bits, int dtype, int npass, const Params& p, const Launch& L);
+constexpr int kTcbStages = 4;
 
 
 
@@ -95,6 +99,19 @@ inline bool shape_instantiated(int maxm, int R, bool wide) {
         static std::atomic<unsigned> cfg_{0};                                                \
         return launch_kernel(qmv_tc_kernel<BITS_, T_, NPASS_, QMV_TC_PD(BITS_)>, cfg_, L, p); \
     }
+#define QMV_TCB_SHAPE(T_, NPASS_)                                                            \
+    if (npass == NPASS_) {                                                                   \
+        static std::atomic<unsigned> cfg_{0};                                                \
+        return launch_kernel(qmv_tcb_kernel<BITS_, T_, NPASS_, kTcbStages>, cfg_, L, p);     \
+    }
+#define QMV_TCB_DISPATCH_DTYPE()                                                             \
+    switch (dtype) {                                                                         \
+        case 0: { QMV_TCB_SHAPE(float, 1) QMV_TCB_SHAPE(float, 2) QMV_TCB_SHAPE(float, 4) break; }                 \
+        case 1: { QMV_TCB_SHAPE(__half, 1) QMV_TCB_SHAPE(__half, 2) QMV_TCB_SHAPE(__half, 4) break; }              \
+        case 2: { QMV_TCB_SHAPE(__nv_bfloat16, 1) QMV_TCB_SHAPE(__nv_bfloat16, 2) QMV_TCB_SHAPE(__nv_bfloat16, 4) break; } \
+        default: break;                                                                      \
+    }                                                                                        \
+    return cudaErrorInvalidValue;
 #define QMV_TC_PD(B_) (((B_) == 5 || (B_) == 6) ? 2 : 4)
 #define QMV_TC_DISPATCH_DTYPE()                                                              \
     switch (dtype) {                                                                         \
