@@ -40,12 +40,12 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def run_affine(q, c, w_offset=0, x_batched=True, stream=None):
+def run_affine(q, c, w_offset=0, x_batched=True, stream=None, s_offset=0):
     B, M, N, K = c["batch"], c["M"], c["N"], c["K"]
     x = c["x"] if x_batched else c["x"][:1]
     y = y_buffer(B, M, N, c["dtype"])
-    args = (dev(x), dev(c["w"], w_offset), dev(c["scales"]), dev(c["biases"]), y, M, N, K, c["bits"],
-            c["group"], c["dtype"])
+    args = (dev(x), dev(c["w"], w_offset), dev(c["scales"], s_offset), dev(c["biases"], s_offset), y, M, N, K,
+            c["bits"], c["group"], c["dtype"])
     if B == 1 and x_batched:
         q.qmv_affine(*args, stream=stream)
     else:

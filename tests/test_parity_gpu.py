@@ -481,6 +481,23 @@ def test_bulk_ring_tail_rows_bitwise_prefix(q, ring, bits):
         assert np.array_equal(run_affine(q, small)[0], yb[:, :n])
 
 
+@pytest.mark.parametrize("bits,group,M", [(4, 64, 1), (4, 32, 8), (3, 128, 2), (8, 128, 1), (5, 64, 3)])
+def test_bulk_ring_scales_in_or_out_of_ring(q, ring, bits, group, M):
+    """Scales and biases ride in the ring when 16-byte aligned and read from
+    global memory otherwise: the two give bitwise equal outputs."""
+    q.qmv_force_config(4, -1, -1, -1)
+    N, K = 300, 4096
+    plan = q.qmv_describe_plan("affine", M, N, K, bits, group, "bf16")
+    assert "path=tcb" in plan and "scale_ring=1" in plan, plan
+    c = synth.affine_case(M, N, K, bits, group, "bf16", seed=_seed("tcbscale", bits, group, M), batch=2)
+    y_in = run_affine(q, c)
+    y_out = run_affine(q, c, s_offset=2)
+    assert np.array_equal(y_in, y_out)
+    for b in range(2):
+        ref, ad = oracle_affine(c, b=b)
+        compare(y_in[b], ref, ad, "bf16", what=f"tcb scales b{bits} g{group} M{M} batch{b}")
+
+
 @pytest.mark.parametrize("N", [80, 16 * 148 + 5])
 def test_bulk_ring_x_tiles(q, ring, N):
     """M=8, f32 x, K large enough that x is staged in several K tiles (and,

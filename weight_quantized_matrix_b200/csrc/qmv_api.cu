@@ -18,6 +18,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "../../include/qmv.h"
 #include "qmv_launch.cuh"
 #include "qmv_tc_plan.cuh"
@@ -89,7 +91,7 @@ FmtInfo fmt_info(int fam, int bits) {
 
 struct Plan {
     int maxm, R, wide, tc, npass, wk, wr, tile_iters, C;   // tc: 0 CUDA cores, 1 tensor cores, 2 + bulk ring
-    int sps = 0, pitch = 0;
+    int sps = 0, pitch = 0, spb = 1, sring = 0, soff = 0, boff = 0, sbw = 0;
     size_t smem;
     dim3 grid, block;
 };
@@ -173,12 +175,11 @@ bool tc_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, TcShape
 
 // ---- bulk-ring tensor-core launch shape ----------------------------------------
 // Row blocks of 16*wr rows are spread over a persistent grid of one block per
-// SM, wk consumer warps split K.  wr = 2, wk = 4 measured best or within a few
-// percent of best on B200 for 4K..28K rows (M = 1..8).  A ring stage holds
-// about 32 KB; the x tile takes what shared memory is left.
-struct TcbShape { int npass, wk, wr, tsb, sps, pitch; long long gx; size_t smem; };
+// SM, wk = 8 / wr consumer warps split K.  A ring stage holds about 32 KB;
+// the x tile takes what shared memory is left.
+struct TcbShape { int npass, spb, wk, wr, tsb, sps, pitch, sring, soff, boff, sbw; long long gx; size_t smem; };
 
-bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, TcbShape* ts) {
+bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s16, TcbShape* ts) {
     const int ub = tc_unit_bytes(bits);
     const int uc = ub * 8 / bits;
     const int SB = 4 * uc;
@@ -190,49 +191,80 @@ bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, TcbSha
     const int cols = M * ngs;
     const int npass = cols <= 8 ? 1 : cols <= 16 ? 2 : cols <= 32 ? 4 : 0;
     if (npass == 0) return false;
+    int spb = 8 * npass / cols;
+    spb = spb >= 8 ? 8 : spb >= 4 ? 4 : spb >= 2 ? 2 : 1;
     const int nsplit = dtype == QMV_BF16 ? 1 : dtype == QMV_F16 ? 2 : 3;
+    const int es = elem_bytes(dtype);
     const int np = tc_np_of(bits);
     const int nsbk = K / SB;
     const int sms = device_sms();
-    int wr = 2;
-    int wk = 4;
+    // rows per block: one x row -> 32 (2-bit: 64); several x rows -> 64 rows
+    // once that still gives ~96+ row blocks, else 32, else 16 (measured on B200)
+    int wr = M == 1 ? (bits == 2 ? 4 : 2) : (N >= 6144 ? 4 : N >= 2048 ? 2 : 1);
+    int wk = 8 / wr;
     if (g_forced.wr > 0) wr = g_forced.wr > 8 ? 8 : g_forced.wr;
     if (g_forced.wk > 0) wk = g_forced.wk > 8 ? 8 : g_forced.wk;
     while (wk * wr > 8) --wk;
     if (wk > nsbk) wk = nsbk;
     if (wk < 1) wk = 1;
     const int rows = 16 * wr;
+    // stage size: a multiple of one batch of every k-warp (SPB * wk super-blocks)
+    // and of the super-blocks one group spans (G / SB when G > SB)
+    const int gq = G > SB ? G / SB : 1;
+    auto quantum_of = [&](int b) { int qv = b * wk; while (qv % gq) qv *= 2; return qv; };
+    // a ring stage of one quantum must leave room for the x tile: fewer
+    // super-blocks per batch (fewer slot columns used) where it would not
+    while (spb > 1 && (size_t)qmv::kTcbStages * rows * quantum_of(spb) * 4 * ub > 144 * 1024) spb /= 2;
+    const int quantum = quantum_of(spb);
+    // scale bytes of s super-blocks (G <= SB: s * SB / G groups; else s / (G / SB))
     int sps = 32768 / (rows * 4 * ub);
-    sps = sps / wk * wk;
-    if (sps < wk) sps = wk;
-    if (sps > nsbk) sps = nsbk;
-    auto pitch_of = [&](int s) { return ((s * 4 * ub + 127) / 128) * 128 + (ub == 16 ? 64 : 16); };
+    sps = sps / quantum * quantum;
+    if (sps < quantum) sps = quantum;
+    if (sps > nsbk) sps = (nsbk + quantum - 1) / quantum * quantum;
+    // stage layout: ROWS packed rows, pitch bytes apart, then (scales in the
+    // ring) a scale tile and a bias tile of ROWS x sbw bytes, filled by tensor
+    // copies whose column start must sit on 16 bytes and whose box is <= 256
+    auto layout = [&](int s, int* sring, int* sbw, int* stage) {
+        const int box0 = G <= SB ? s * (SB / G) : s / (G / SB);
+        *sbw = box0 * es;
+        *sring = (s16 && ((long long)(K / G) * es) % 16 == 0 && *sbw % 16 == 0 && box0 <= 256 && rows <= 256) ? 1 : 0;
+        const int wpart = (s * 4 * ub + 15) / 16 * 16;
+        const int pad = ub == 16 ? 64 : 16;           // pitch mod 128 (bank spread of the unit loads)
+        const int pitch = wpart + ((pad - wpart % 128) % 128 + 128) % 128;
+        *stage = rows * pitch + (*sring ? 2 * rows * *sbw : 0);
+        return pitch;
+    };
     const int ncw = wk * wr;
     const size_t red = (size_t)ncw * 16 * 8 * npass * 4;
     const size_t per_sb = (size_t)nsplit * M * 4 * np * 4 + (size_t)M * ngs * 4 * 2 + (size_t)M * 4 * 2 * 4;
     long long tsb = 0;
-    size_t fixed = 0;
+    int sring = 0, sbw = 0, stage = 0, pitch = 0;
     for (;;) {
-        fixed = 128 + (size_t)qmv::kTcbStages * rows * pitch_of(sps) + red + (size_t)nsplit * (M * 4 + 4 * np + 4) * 4;
+        pitch = layout(sps, &sring, &sbw, &stage);
+        // 128 bytes of barriers + 128 of alignment slack for the ring
+        const size_t fixed = 256 + (size_t)qmv::kTcbStages * stage + red + (size_t)nsplit * (M * 4 + 4 * np + 4) * 4;
         tsb = fixed < (size_t)qmv::kMaxSmem ? (long long)(((size_t)qmv::kMaxSmem - fixed) / per_sb) : 0;
         if (tsb >= nsbk) { tsb = nsbk; break; }
         tsb = tsb / sps * sps;
         if (tsb >= sps) break;
-        if (sps <= 1) return false;
-        sps = sps > wk ? (sps / 2 / wk) * wk : sps / 2;
-        if (sps < 1) sps = 1;
+        if (sps <= quantum) return false;
+        sps = (sps / 2) / quantum * quantum;
+        if (sps < quantum) sps = quantum;
     }
     const long long nrb = ((long long)N + rows - 1) / rows;
-    ts->npass = npass; ts->wk = wk; ts->wr = wr; ts->tsb = (int)tsb; ts->sps = sps; ts->pitch = pitch_of(sps);
+    ts->npass = npass; ts->spb = spb; ts->wk = wk; ts->wr = wr; ts->tsb = (int)tsb; ts->sps = sps;
+    ts->pitch = pitch; ts->sring = sring; ts->sbw = sbw;
+    ts->soff = rows * pitch; ts->boff = rows * pitch + rows * sbw;
     ts->gx = nrb < sms ? nrb : sms;
     const size_t plane = (size_t)M * ((size_t)tsb * 4 * np + 4) + 4 * np + 4;
-    ts->smem = 128 + (size_t)qmv::kTcbStages * rows * ts->pitch + (size_t)nsplit * plane * 4 +
+    ts->smem = 256 + (size_t)qmv::kTcbStages * stage + (size_t)nsplit * plane * 4 +
                (size_t)M * tsb * ngs * 4 * 2 + (size_t)M * tsb * 4 * 2 * 4 + red;
     return ts->smem <= (size_t)qmv::kMaxSmem;
 }
 
 // Choose the launch shape.  Returns QMV_OK or an error (sizes too large).
-int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, bool w16, int batch, Plan* pl) {
+int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, bool w16, int batch, Plan* pl,
+              bool s16 = true) {
     const FmtInfo fi = fmt_info(fam, bits);
     const bool aff = fam == qmv::FAM_AFFINE;
     int maxm = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
@@ -241,12 +273,16 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     if (g_forced.path == 0) wide = false;
 
     // ---- tensor-core kernel with the bulk-copy weight ring --------------------
-    // (measured: wins over the register-prefetch kernel once M >= 2)
-    if (aff && K > 0 && (g_forced.path == 4 || (g_forced.path < 0 && M >= 2 && tc_preferred(M, N, K, bits)))) {
+    // (measured on B200: the fastest path once M >= 2, and for large 2-bit
+    // matrices at M = 1)
+    // (6-bit codes do not pair: the ring kernel wins there only at M = 8)
+    const bool ring_pick = M >= 2 ? (N >= 64 && (bits != 6 || M >= 8)) : (bits == 2 && tc_preferred(M, N, K, bits));
+    if (aff && K > 0 && (g_forced.path == 4 || (g_forced.path < 0 && ring_pick))) {
         TcbShape ts;
-        if (tcb_shape(M, N, K, bits, G_of_plan, dtype, w16, &ts)) {
+        if (tcb_shape(M, N, K, bits, G_of_plan, dtype, w16, s16, &ts)) {
             pl->maxm = maxm; pl->R = 1; pl->wide = 1; pl->tc = 2; pl->npass = ts.npass;
             pl->wk = ts.wk; pl->wr = ts.wr; pl->tile_iters = ts.tsb; pl->sps = ts.sps; pl->pitch = ts.pitch;
+            pl->spb = ts.spb; pl->sring = ts.sring; pl->soff = ts.soff; pl->boff = ts.boff; pl->sbw = ts.sbw;
             pl->C = 4 * tc_unit_bytes(bits) * 8 / bits; pl->smem = ts.smem;
             pl->grid = dim3((unsigned)ts.gx, 1, (unsigned)batch);
             pl->block = dim3(32 * (ts.wk * ts.wr + 1), 1, 1);
@@ -358,15 +394,59 @@ int check_common(const void* x, const void* w, const void* s, void* y, int M, in
     return QMV_OK;
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// [batch][N][K/G] scales (or biases) as a 3-D tensor map with box
+// {box0 groups, rows, 1}; out-of-range elements read as zero.
+bool encode_scale_map(CUtensorMap* m, const void* base, int dtype, long long KG, int N, int batch, int box0,
+                      int rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const CUtensorMapDataType dt = dtype == QMV_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : dtype == QMV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint64_t es = (cuuint64_t)elem_bytes(dtype);
+    const cuuint64_t dims[3] = {(cuuint64_t)KG, (cuuint64_t)N, (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)KG * es, (cuuint64_t)KG * es * (cuuint64_t)N};
+    const cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 int run(int fam, const void* x, const void* w, const void* scales, const void* biases,
         const float* gscale, void* y, int M, int N, int K, int bits, int G, int dtype, int batch,
         int x_batched, void* stream) {
     const long long row_bytes = (long long)K * (fam == qmv::FAM_AFFINE ? bits : (fam == qmv::FAM_MXFP8 ? 8 : 4)) / 8;
     Plan pl;
     const bool w16 = aligned(w, 16);
-    int st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl);
+    const bool s16 = fam == qmv::FAM_AFFINE && aligned(scales, 16) && aligned(biases, 16);
+    int st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, s16);
     if (st != QMV_OK) return st;
     qmv::Params p;
+    if (pl.tc == 2 && pl.sring) {
+        const int box0 = pl.sbw / elem_bytes(dtype), rows = 16 * pl.wr;
+        if (!encode_scale_map(&p.smap, scales, dtype, K / G, N, batch, box0, rows) ||
+            !encode_scale_map(&p.bmap, biases, dtype, K / G, N, batch, box0, rows)) {
+            st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, false);   // scales from global memory
+            if (st != QMV_OK) return st;
+        }
+    }
     p.x = x; p.w = static_cast<const uint8_t*>(w); p.scales = scales; p.biases = biases;
     p.gscale = gscale; p.y = y;
     p.M = M; p.N = N; p.K = K; p.G = G;
@@ -381,10 +461,13 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     qmv::Launch L{pl.grid, pl.block, pl.smem, static_cast<cudaStream_t>(stream), pdl_enabled()};
     cudaError_t e;
     p.sps = pl.sps; p.pitch = pl.pitch; p.fault = nullptr;
+    p.sring = pl.sring; p.soff = pl.soff; p.boff = pl.boff; p.sbw = pl.sbw;
+    p.kf32 = 0x4B000000u;
+    p.kbf16 = 0x43004300u;
     if (pl.tc == 2) {
         p.fault = fault_word();
         if (!p.fault) return QMV_ECUDA;
-        return finish(qmv::launch_tcb_affine(bits, dtype, pl.npass, p, L));
+        return finish(qmv::launch_tcb_affine(bits, dtype, pl.npass, pl.spb, p, L));
     }
     if (pl.tc) return finish(qmv::launch_tc_affine(bits, dtype, pl.npass, p, L));
     if (fam == qmv::FAM_AFFINE) {
@@ -536,9 +619,9 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
     if (st != QMV_OK) return st;
     snprintf(buf, (size_t)buflen,
              "path=%s chunk=%d maxm=%d rows_per_warp=%d warps_k=%d warps_rows=%d tile_iters=%d "
-             "grid=%u block=%u smem=%zu stage_sb=%d",
+             "grid=%u block=%u smem=%zu stage_sb=%d batch_sb=%d scale_ring=%d",
              pl.tc == 2 ? "tcb" : pl.tc ? "tc" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr,
-             pl.tile_iters, pl.grid.x, pl.block.x, pl.smem, pl.sps);
+             pl.tile_iters, pl.grid.x, pl.block.x, pl.smem, pl.sps, pl.spb, pl.sring);
     return QMV_OK;
 }
 

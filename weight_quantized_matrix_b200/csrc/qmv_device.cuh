@@ -42,6 +42,7 @@
 //     launch; it lets dependents launch once its main loop is done.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -70,6 +71,15 @@ struct Params {
     int sps;                // bulk-ring kernel: super-blocks per ring stage
     int pitch;              // bulk-ring kernel: bytes per ring row
     unsigned* fault;        // bulk-ring kernel: device fault word (bounded waits that expired)
+    int sring;              // bulk-ring kernel: 1 = scales / biases travel in the ring (tensor copies)
+    int soff, boff;         // bulk-ring kernel: byte offsets of the scale / bias tiles in a ring stage
+    int sbw;                // bulk-ring kernel: bytes per row of those tiles
+    CUtensorMap smap, bmap; // bulk-ring kernel: scales / biases as [batch][N][K/G] tensors
+    // Exponent patterns OR-ed into decoded fields, passed in so that kernels
+    // hold them in registers: then mask-and-OR is one three-input logic op
+    // (with both operands immediate it would take two).
+    unsigned kf32;          // 0x4B000000: fp32 2^23
+    unsigned kbf16;         // 0x43004300: bf16 pair {128, 128}
 };
 
 // ---------------------------------------------------------------- dtypes ---
@@ -155,6 +165,33 @@ __device__ __forceinline__ uint32_t field_bits(const uint32_t* w) {
     } else {
         return (w[wi] >> 9) & (m << (r - 9));
     }
+}
+
+// (a & MASK) | c as one three-input logic op.
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(MASK), "r"(c));
+    return d;
+}
+
+// field_bits OR-ed with kf32 (the fp32 pattern of 2^23) in the same op.
+template <int B, int J>
+__device__ __forceinline__ uint32_t field_magic(const uint32_t* w, uint32_t kf32) {
+    constexpr int o = B * J, wi = o / 32, r = o % 32;
+    constexpr uint32_t m = (1u << B) - 1u;
+    if constexpr (r + B > 32) {
+        return and_or<m>(__funnelshift_r(w[wi], w[wi + 1], r), kf32);
+    } else if constexpr (r + B <= 23) {
+        return and_or<(m << r)>(w[wi], kf32);
+    } else {
+        return and_or<(m << (r - 9))>(w[wi] >> 9, kf32);
+    }
+}
+
+// {a, b}: fields already OR-ed into 2^23 -> their values as exact floats.
+__device__ __forceinline__ float2 magic_pair_ored(uint32_t a, uint32_t b) {
+    return add2(make_float2(__uint_as_float(a), __uint_as_float(b)), make_float2(-8388608.0f, -8388608.0f));
 }
 
 __device__ __forceinline__ float2 magic_pair(uint32_t a, uint32_t b) {
@@ -302,7 +339,8 @@ __device__ __forceinline__ void load_scales(const Params& p, const int (&rowc)[R
 template <int FAM, int B, int MAXM, int R, int U>
 __device__ __forceinline__ void compute_chunk(const uint32_t (&wv)[R][B * U], const float (&sc)[R][U][2],
                                               const float (&bi)[R][U], const float4* xb, size_t xm,
-                                              const float* sxb, size_t sxm, int KT, float (&acc)[R][MAXM]) {
+                                              const float* sxb, size_t sxm, int KT, float (&acc)[R][MAXM],
+                                              uint32_t kf32) {
     constexpr int UW = B;
     constexpr bool AFF = (FAM == FAM_AFFINE);
 #pragma unroll
@@ -324,14 +362,14 @@ __device__ __forceinline__ void compute_chunk(const uint32_t (&wv)[R][B * U], co
                 if constexpr (AFF) {
                     uint32_t f0, f1, f2, f3;
                     switch (q) {
-#define QMV_F4(QQ) case QQ: f0 = field_bits<B, 4 * QQ>(wu); f1 = field_bits<B, 4 * QQ + 1>(wu); \
-                   f2 = field_bits<B, 4 * QQ + 2>(wu); f3 = field_bits<B, 4 * QQ + 3>(wu); break;
+#define QMV_F4(QQ) case QQ: f0 = field_magic<B, 4 * QQ>(wu, kf32); f1 = field_magic<B, 4 * QQ + 1>(wu, kf32); \
+                   f2 = field_magic<B, 4 * QQ + 2>(wu, kf32); f3 = field_magic<B, 4 * QQ + 3>(wu, kf32); break;
                         QMV_F4(0) QMV_F4(1) QMV_F4(2) QMV_F4(3) QMV_F4(4) QMV_F4(5) QMV_F4(6) QMV_F4(7)
 #undef QMV_F4
-                        default: f0 = f1 = f2 = f3 = 0;
+                        default: f0 = f1 = f2 = f3 = kf32;
                     }
-                    d0 = magic_pair(f0, f1);
-                    d1 = magic_pair(f2, f3);
+                    d0 = magic_pair_ored(f0, f1);
+                    d1 = magic_pair_ored(f2, f3);
                 } else if constexpr (B == 4) {
                     const uint32_t wd = wu[q >> 1] >> (16 * (q & 1));
                     const float2 s126 = make_float2(0x1p126f, 0x1p126f);
@@ -447,6 +485,7 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
         load_scales<FAM, T, R, U>(p, rowc, c, sb, sc, bi);
     };
 
+    const uint32_t kf32 = p.kf32;
     grid_wait();   // inputs may come from the previous kernel in the stream
 
     for (int t0 = 0; t0 < NC; t0 += TC) {
@@ -461,7 +500,7 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
         for (int i = 0; have;) {
             compute_chunk<FAM, B, MAXM, R, U>(wv, sc, bi, xs + (size_t)i * (C / 4) * KT + kt,
                                               (size_t)TI * (C / 4) * KT, sx + (size_t)i * U * KT + kt,
-                                              (size_t)TI * U * KT, KT, acc);
+                                              (size_t)TI * U * KT, KT, acc, kf32);
             ++i;
             const int cc = i * KT + kt;
             have = i < TI && cc < tcn;

@@ -60,8 +60,9 @@ cudaError_t launch_fp(int fam, int dtype, int maxm, int R, bool wide, const Para
 
 // Tensor-core kernels (qmv_tc_kernel): npass in {1, 2, 4}.
 cudaError_t launch_tc_affine(int bits, int dtype, int npass, const Params& p, const Launch& L);
-// Tensor-core kernels with the bulk-copy weight ring (qmv_tcb_kernel).
-cudaError_t launch_tcb_affine(int bits, int dtype, int npass, const Params& p, const Launch& L);
+// Tensor-core kernels with the bulk-copy weight ring (qmv_tcb_kernel):
+// (npass, spb) in {(1,1), (1,2), (1,4), (1,8), (2,1), (4,1)}.
+cudaError_t launch_tcb_affine(int bits, int dtype, int npass, int spb, const Params& p, const Launch& L);
 constexpr int kTcbStages = 4;
 
 
@@ -99,16 +100,19 @@ inline bool shape_instantiated(int maxm, int R, bool wide) {
         static std::atomic<unsigned> cfg_{0};                                                \
         return launch_kernel(qmv_tc_kernel<BITS_, T_, NPASS_, QMV_TC_PD(BITS_)>, cfg_, L, p); \
     }
-#define QMV_TCB_SHAPE(T_, NPASS_)                                                            \
-    if (npass == NPASS_) {                                                                   \
+#define QMV_TCB_SHAPE(T_, NPASS_, SPB_)                                                      \
+    if (npass == NPASS_ && spb == SPB_) {                                                    \
         static std::atomic<unsigned> cfg_{0};                                                \
-        return launch_kernel(qmv_tcb_kernel<BITS_, T_, NPASS_, kTcbStages>, cfg_, L, p);     \
+        return launch_kernel(qmv_tcb_kernel<BITS_, T_, NPASS_, SPB_, kTcbStages>, cfg_, L, p); \
     }
+#define QMV_TCB_SHAPES(T_)                                                                   \
+    QMV_TCB_SHAPE(T_, 1, 1) QMV_TCB_SHAPE(T_, 1, 2) QMV_TCB_SHAPE(T_, 1, 4)                 \
+    QMV_TCB_SHAPE(T_, 1, 8) QMV_TCB_SHAPE(T_, 2, 1) QMV_TCB_SHAPE(T_, 4, 1)
 #define QMV_TCB_DISPATCH_DTYPE()                                                             \
     switch (dtype) {                                                                         \
-        case 0: { QMV_TCB_SHAPE(float, 1) QMV_TCB_SHAPE(float, 2) QMV_TCB_SHAPE(float, 4) break; }                 \
-        case 1: { QMV_TCB_SHAPE(__half, 1) QMV_TCB_SHAPE(__half, 2) QMV_TCB_SHAPE(__half, 4) break; }              \
-        case 2: { QMV_TCB_SHAPE(__nv_bfloat16, 1) QMV_TCB_SHAPE(__nv_bfloat16, 2) QMV_TCB_SHAPE(__nv_bfloat16, 4) break; } \
+        case 0: { QMV_TCB_SHAPES(float) break; }                                             \
+        case 1: { QMV_TCB_SHAPES(__half) break; }                                            \
+        case 2: { QMV_TCB_SHAPES(__nv_bfloat16) break; }                                     \
         default: break;                                                                      \
     }                                                                                        \
     return cudaErrorInvalidValue;

@@ -54,7 +54,7 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 // Pair p of a unit as bf16x2 {128 + low field * 2^slo, 128 + high field * 2^shi}
 // (an empty high half is 128 + 0; an empty pair is 0).
 template <int B, int p>
-__device__ __forceinline__ uint32_t tc_pair(const uint32_t (&w)[TcGeom<B>::NW]) {
+__device__ __forceinline__ uint32_t tc_pair(const uint32_t (&w)[TcGeom<B>::NW], uint32_t kbf16) {
     constexpr TcPlanData P = tc_make_plan<B, false>();
     if constexpr (P.lo[p] < 0) {
         return 0u;
@@ -73,7 +73,7 @@ __device__ __forceinline__ uint32_t tc_pair(const uint32_t (&w)[TcGeom<B>::NW]) 
         }
         constexpr uint32_t fm = (1u << fb) - 1u;
         constexpr uint32_t m = (fm << P.slo[p]) | (P.hi[p] >= 0 ? (fm << (16 + P.shi[p])) : 0u);
-        return (v & m) | 0x43004300u;
+        return and_or<m>(v, kbf16);      // kbf16 = 0x43004300, held in a register
     }
 }
 
@@ -86,14 +86,15 @@ __device__ __forceinline__ uint32_t bf16_bits(float v) {
 template <int B, int NPASS, int NSPLIT, int... S2>
 __device__ __forceinline__ void tc_steps(std::integer_sequence<int, S2...>, const uint32_t (&wg)[TcGeom<B>::NW],
                                          const uint32_t (&wh)[TcGeom<B>::NW], float (&D)[NPASS][4],
-                                         const uint32_t* __restrict__ xb, const int (&xoff)[NPASS], int plane) {
+                                         const uint32_t* __restrict__ xb, const int (&xoff)[NPASS], int plane,
+                                         uint32_t kbf16) {
     (
         [&] {
             constexpr int s = 2 * S2;
-            const uint32_t a0 = tc_pair<B, 2 * s>(wg), a2 = tc_pair<B, 2 * s + 1>(wg);
-            const uint32_t a1 = tc_pair<B, 2 * s>(wh), a3 = tc_pair<B, 2 * s + 1>(wh);
-            const uint32_t c0 = tc_pair<B, 2 * s + 2>(wg), c2 = tc_pair<B, 2 * s + 3>(wg);
-            const uint32_t c1 = tc_pair<B, 2 * s + 2>(wh), c3 = tc_pair<B, 2 * s + 3>(wh);
+            const uint32_t a0 = tc_pair<B, 2 * s>(wg, kbf16), a2 = tc_pair<B, 2 * s + 1>(wg, kbf16);
+            const uint32_t a1 = tc_pair<B, 2 * s>(wh, kbf16), a3 = tc_pair<B, 2 * s + 1>(wh, kbf16);
+            const uint32_t c0 = tc_pair<B, 2 * s + 2>(wg, kbf16), c2 = tc_pair<B, 2 * s + 3>(wg, kbf16);
+            const uint32_t c1 = tc_pair<B, 2 * s + 2>(wh, kbf16), c3 = tc_pair<B, 2 * s + 3>(wh, kbf16);
 #pragma unroll
             for (int pp = 0; pp < NPASS; ++pp)
 #pragma unroll
@@ -101,6 +102,32 @@ __device__ __forceinline__ void tc_steps(std::integer_sequence<int, S2...>, cons
                     const uint4 b = *reinterpret_cast<const uint4*>(xb + xoff[pp] + sp * plane + 2 * s);
                     mma_bf16_16816(D[pp], a0, a1, a2, a3, b.x, b.y);
                     mma_bf16_16816(D[pp], c0, c1, c2, c3, b.z, b.w);
+                }
+        }(),
+        ...);
+}
+
+// As tc_steps, with the two k-steps of each B load accumulated into separate
+// registers (D, E): two independent MMA dependency chains instead of one.
+template <int B, int NPASS, int NSPLIT, int... S2>
+__device__ __forceinline__ void tc_steps2(std::integer_sequence<int, S2...>, const uint32_t (&wg)[TcGeom<B>::NW],
+                                          const uint32_t (&wh)[TcGeom<B>::NW], float (&D)[NPASS][4],
+                                          float (&E)[NPASS][4], const uint32_t* __restrict__ xb,
+                                          const int (&xoff)[NPASS], int plane, uint32_t kbf16) {
+    (
+        [&] {
+            constexpr int s = 2 * S2;
+            const uint32_t a0 = tc_pair<B, 2 * s>(wg, kbf16), a2 = tc_pair<B, 2 * s + 1>(wg, kbf16);
+            const uint32_t a1 = tc_pair<B, 2 * s>(wh, kbf16), a3 = tc_pair<B, 2 * s + 1>(wh, kbf16);
+            const uint32_t c0 = tc_pair<B, 2 * s + 2>(wg, kbf16), c2 = tc_pair<B, 2 * s + 3>(wg, kbf16);
+            const uint32_t c1 = tc_pair<B, 2 * s + 2>(wh, kbf16), c3 = tc_pair<B, 2 * s + 3>(wh, kbf16);
+#pragma unroll
+            for (int pp = 0; pp < NPASS; ++pp)
+#pragma unroll
+                for (int sp = 0; sp < NSPLIT; ++sp) {
+                    const uint4 b = *reinterpret_cast<const uint4*>(xb + xoff[pp] + sp * plane + 2 * s);
+                    mma_bf16_16816(D[pp], a0, a1, a2, a3, b.x, b.y);
+                    mma_bf16_16816(E[pp], c0, c1, c2, c3, b.z, b.w);
                 }
         }(),
         ...);
@@ -208,6 +235,7 @@ __global__ void __launch_bounds__(256) qmv_tc_kernel(const Params p) {
         }
     };
 
+    const uint32_t kbf16 = p.kbf16;
     uint32_t wring[PD][2][NW];
     float sc[NPASS][4], bi[NPASS][4];
 
@@ -325,7 +353,7 @@ __global__ void __launch_bounds__(256) qmv_tc_kernel(const Params p) {
                     for (int pp = 0; pp < NPASS; ++pp)
                         xoff[pp] = (bsbi[pp] == bi_ ? brow[pp] : M) * xrow + ((sb - t0) * 4 + t) * NP;
                     tc_steps<B, NPASS, NSPLIT>(std::make_integer_sequence<int, NSTEP / 2>{}, wring[q][0], wring[q][1],
-                                               D, xs, xoff, plane);
+                                               D, xs, xoff, plane, kbf16);
                     if (sb + PD * wk < end) loadW(wring[q][0], wring[q][1], sb + PD * wk);
                     if (bi_ == SPB - 1 || sb + wk >= end) {
                         // epilogue of the batch: each slot's (super-block, group)

@@ -9,12 +9,17 @@
 //
 // Work: the grid is persistent over ROW BLOCKS of ROWS = 16*wr rows (block b
 // takes row blocks b, b + gridDim.x, ...).  A row block's packed rows are cut
-// along K into STAGES of S super-blocks; the producer copies stage after stage
-// (one bulk copy per row, issued by the producer's lanes) into the ring, across
-// row-block boundaries, while consumers compute.  Consumer warp (wrid, wkid)
-// owns row tile wrid (16 rows) and the super-blocks wkid, wkid + wk, ... of
-// every stage; the decode, the slot-column MMAs and the exact per-group fp32
-// epilogue are those of qmv_tc.cuh.
+// along K into ring STAGES of S super-blocks; the producer copies stage after
+// stage (per row: the packed bytes and, when their layout allows, the stage's
+// scales and biases; one bulk copy each, issued by the producer's lanes) into
+// the ring, across row-block boundaries, while consumers compute.  Consumer
+// warp (wrid, wkid) owns row tile wrid (16 rows) and the super-blocks wkid,
+// wkid + wk, ... of every stage, taken SPB at a time: one BATCH fills the 8*NPASS
+// slot columns of the MMAs (decode and slot columns as in qmv_tc.cuh) and
+// ends in one exact fp32 epilogue.  Everything a lane needs to place its x
+// fragments, scales and sums inside a batch is computed once per kernel, so a
+// full batch runs without per-super-block index arithmetic or predicates; only
+// the last, partial batch of a row takes the guarded path.
 //
 // Flow control: full[s] (one producer arrival + the copies' byte count) and
 // empty[s] (one arrival per consumer warp).  Every wait is bounded (about one
@@ -28,6 +33,8 @@
 // 128 for 12/20-byte units) so the 8 rows read by one load instruction fall in
 // distinct banks.
 #pragma once
+
+#include <type_traits>
 
 #include "qmv_tc.cuh"
 
@@ -84,28 +91,53 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
+// Tensor tile [box] of a 3-D tensor map -> this CTA's shared memory (128-byte
+// aligned destination), completion counted on `bar` in bytes (the full box,
+// out-of-range elements zero-filled).  No multicast.
+__device__ __forceinline__ void tensor_copy_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                               uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+        : "memory");
+}
 // Barrier over the consumer warps only (named barrier 1).
 __device__ __forceinline__ void consumer_sync(int nthreads) {
     asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
+// Scale / bias element of a ring row (x dtype), widened to fp32.
+template <class T> __device__ __forceinline__ float ring_scale(const unsigned char* row, int i);
+template <> __device__ __forceinline__ float ring_scale<float>(const unsigned char* row, int i) {
+    return reinterpret_cast<const float*>(row)[i];
+}
+template <> __device__ __forceinline__ float ring_scale<__half>(const unsigned char* row, int i) {
+    return __half2float(reinterpret_cast<const __half*>(row)[i]);
+}
+template <> __device__ __forceinline__ float ring_scale<__nv_bfloat16>(const unsigned char* row, int i) {
+    return __uint_as_float((uint32_t)reinterpret_cast<const unsigned short*>(row)[i] << 16);
+}
+
 // Shared memory (bytes, in order):
 //   bars  128            full[STAGES], empty[STAGES]
-//   ring  STAGES * ROWS * pitch
+//   ring  STAGES stages (128-byte aligned) of: ROWS packed rows (pitch bytes
+//         apart), then (p.sring) the scale tile at p.soff and the bias tile at
+//         p.boff, ROWS x p.sbw bytes each
 //   xs    NSPLIT * plane * 4    plane = M*xrow + 4*NP + 4 u32: the x rows of
 //                               the tile (bf16 pairs, fragment order), then one
 //                               super-block of zeros read by inactive lanes
-//   sx    M * NSEG floats        sum(x) per segment of the tile
-//   sxt   M * NSEG floats        sum(x~) per segment
-//   us    M * TU * 2 floats      per-unit sums
+//   sxx   M * NSEG float2      {sum(x), sum(x~)} per segment of the tile
+//   us    M * TU * 2 floats    per-unit sums
 //   red   NCW * 16 * 8*NPASS floats
-template <int B, class T, int NPASS, int STAGES>
-__global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const Params p) {
+template <int B, class T, int NPASS, int SPB, int STAGES>
+__global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const __grid_constant__ Params p) {
     using Gm = TcGeom<B>;
     constexpr TcPlanData P = tc_make_plan<B, false>();
     constexpr int NP = P.np, NSTEP = NP / 2;
     constexpr int NW = Gm::NW, UB = Gm::UNIT_BYTES, UC = Gm::UNIT_CODES, SB = Gm::SB;
     constexpr int NSPLIT = TcSplit<T>::n;
+    constexpr int ES = (int)sizeof(T);
     static_assert(2 * STAGES * 8 <= 128, "barrier area");
 
     extern __shared__ float4 smem4[];
@@ -118,24 +150,30 @@ __global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const Params p) {
     const int NSBK = p.K / SB;
     const int S = p.sps;
     const int pitch = p.pitch;
-    const int stage_bytes = ROWS * pitch;
+    const int sbw = p.sbw;
+    const bool sring = p.sring != 0;
+    const int stage_bytes = ROWS * pitch + (sring ? 2 * ROWS * sbw : 0);
     const int TSB = p.tile_iters;
     const int TU = TSB * 4;
-    const int segsz = min(p.G, SB);
-    const int NGS = SB / segsz;
     const int G = p.G;
+    const int segsz = min(G, SB);
+    const int NGS = SB / segsz;
     const long long KG = p.K / G;
     const int xrow = TU * NP + 4;
     const int plane = M * xrow + 4 * NP + 4;
     const int NSEG = TSB * NGS;
     const int bz = blockIdx.z;
+    // groups of a super-block: SB / G (G <= SB) or one per G / SB super-blocks
+    const int gmul = G < SB ? __ffs(SB / G) - 1 : 0;
+    const int gdiv = G > SB ? __ffs(G / SB) - 1 : 0;
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    unsigned char* ring = smem + 128;
+    // ring on a 128-byte boundary (tensor-copy destinations); the host adds
+    // 128 bytes of slack for this
+    unsigned char* ring = smem + 128 + ((128u - (smem_addr(smem) & 127u)) & 127u);
     uint32_t* xs = reinterpret_cast<uint32_t*>(ring + (size_t)STAGES * stage_bytes);
-    float* sx = reinterpret_cast<float*>(xs + (size_t)NSPLIT * plane);
-    float* sxt = sx + (size_t)M * NSEG;
-    float* us = sxt + (size_t)M * NSEG;
+    float2* sxx = reinterpret_cast<float2*>(xs + (size_t)NSPLIT * plane);
+    float* us = reinterpret_cast<float*>(sxx + (size_t)M * NSEG);
     float* red = us + (size_t)M * TU * 2;
     const uint32_t bar0 = smem_addr(bars);
     auto full = [&](int s) { return bar0 + 8u * (uint32_t)s; };
@@ -152,6 +190,7 @@ __global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const Params p) {
     grid_wait();
 
     const uint8_t* W = p.w + bz * p.w_bs;
+    const long long sb0 = bz * p.s_bs;
     const int nks = (NSBK + S - 1) / S;
 
     // ============================ producer warp ==============================
@@ -165,12 +204,23 @@ __global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const Params p) {
                 if (f > 0 && !mbar_wait(empty(slot), (uint32_t)((f - 1) & 1))) { ok = false; break; }
                 const int nsb = min(S, NSBK - ks * S);
                 const uint32_t rowb = (uint32_t)(nsb * 4 * UB);
-                if (lane == 0) mbar_arrive_expect_tx(full(slot), (uint32_t)ROWS * rowb);
+                const uint32_t st0 = ring0 + (uint32_t)(slot * stage_bytes);
+                if (lane == 0) {
+                    // packed rows (one bulk copy per row) + the stage's scale and
+                    // bias tiles (one tensor copy each: ROWS x sbw bytes, columns
+                    // past K / G and rows past N zero-filled)
+                    mbar_arrive_expect_tx(full(slot), (uint32_t)ROWS * (rowb + (sring ? 2u * (uint32_t)sbw : 0u)));
+                    if (sring) {
+                        const int g0 = ((ks * S) << gmul) >> gdiv;
+                        tensor_copy_3d(st0 + (uint32_t)p.soff, &p.smap, g0, rb * ROWS, bz, full(slot));
+                        tensor_copy_3d(st0 + (uint32_t)p.boff, &p.bmap, g0, rb * ROWS, bz, full(slot));
+                    }
+                }
                 __syncwarp();
                 for (int r = lane; r < ROWS; r += 32) {
                     const int row = min(rb * ROWS + r, p.N - 1);
-                    bulk_copy_g2s(ring0 + (uint32_t)(slot * stage_bytes + r * pitch),
-                                  W + (long long)row * p.w_row + (long long)ks * S * 4 * UB, rowb, full(slot));
+                    bulk_copy_g2s(st0 + (uint32_t)(r * pitch), W + (long long)row * p.w_row + (long long)ks * S * 4 * UB,
+                                  rowb, full(slot));
                 }
                 ++it;
             }
@@ -191,39 +241,52 @@ __global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const Params p) {
     const int g = lane >> 2, t = lane & 3;
     const int wkid = warp % wk, wrid = warp / wk;
     const T* X = reinterpret_cast<const T*>(p.x) + bz * p.x_bs;
-    const long long sb0 = bz * p.s_bs;
 
     // zero super-block of every plane (never overwritten by the x staging)
     for (int i = threadIdx.x; i < 4 * NP; i += nthr)
 #pragma unroll
         for (int sp = 0; sp < NSPLIT; ++sp) xs[(size_t)sp * plane + (size_t)M * xrow + i] = 0u;
 
+    // ---- per-lane slot geometry, fixed for the kernel ------------------------
+    // Slot column j of pass pp (j = 8 pp + column) is (super-block sbi of the
+    // batch, segment gs, x row m):  j = (sbi * NGS + gs) * M + m.
     const int per_sb = NGS * M;
-    const int SPB = max(1, (8 * NPASS) / per_sb);
     const int nslots = SPB * per_sb;
-    const int gmul = G < SB ? __ffs(SB / G) - 1 : 0;
-    const int gdiv = G > SB ? __ffs(G / SB) - 1 : 0;
-    const int useg = (t * UC) / segsz;
-    int bsbi[NPASS], brow[NPASS];
+    const int useg = (t * UC) / segsz;            // segment of this lane's unit
+    // B operand: the lane supplies x of slot column g; active in the batch's
+    // super-block bi iff that slot belongs to (bi, useg).  Offsets are relative
+    // to the batch's first super-block; xact multiplies the batch advance.
+    int xo[NPASS][SPB], xact[NPASS][SPB];
 #pragma unroll
     for (int pp = 0; pp < NPASS; ++pp) {
         const int j = 8 * pp + g;
         const int m = j % M, q = j / M, gs = q % NGS, sbi = q / NGS;
-        bsbi[pp] = (j < nslots && gs == useg) ? sbi : -1;
-        brow[pp] = m;
+#pragma unroll
+        for (int bi = 0; bi < SPB; ++bi) {
+            const bool a = j < nslots && gs == useg && sbi == bi;
+            xact[pp][bi] = a ? 1 : 0;
+            xo[pp][bi] = a ? m * xrow + (bi * wk * 4 + t) * NP : M * xrow + t * NP;
+        }
     }
-    int dsbi[NPASS][2], dgs[NPASS][2], dm[NPASS][2];
+    // D / Y elements: column 8 pp + 2 t + c, rows g (e = c) and g + 8 (e = 2 + c)
+    int dsb[NPASS][2];      // super-block of the slot within the batch (0 if unused)
+    int dseg[NPASS][2];     // sxx offset: m * NSEG + sbi * wk * NGS + gs
+    int dgrp[NPASS][2];     // super-block offset of the slot within the batch: sbi * wk
+    int dgs[NPASS][2];
 #pragma unroll
     for (int pp = 0; pp < NPASS; ++pp)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
             const int j = 8 * pp + 2 * t + c;
-            const int q = j / M;
-            dm[pp][c] = j % M;
-            dgs[pp][c] = q % NGS;
-            dsbi[pp][c] = j < nslots ? q / NGS : -1;
+            const int m = j % M, q = j / M;
+            const int gs = q % NGS, sbi = j < nslots ? q / NGS : 0;
+            dsb[pp][c] = j < nslots ? sbi : SPB;   // SPB: never present
+            dseg[pp][c] = (j < nslots ? m : 0) * NSEG + sbi * wk * NGS + gs;
+            dgrp[pp][c] = sbi * wk;
+            dgs[pp][c] = gs;
         }
 
+    const uint32_t kbf16 = p.kbf16;
     int it = 0;
     bool ok = true;
     bool x_whole = false;            // x of the whole K is staged (one tile)
@@ -237,11 +300,11 @@ __global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const Params p) {
         const T* big = reinterpret_cast<const T*>(p.biases) + sb0 + (long long)rg * KG;
         const T* bih = reinterpret_cast<const T*>(p.biases) + sb0 + (long long)rh * KG;
 
-        float D[NPASS][4], Y[NPASS][4], sc[NPASS][4], bi[NPASS][4];
+        float Y[NPASS][4];
 #pragma unroll
         for (int pp = 0; pp < NPASS; ++pp)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) { D[pp][e] = 0.f; Y[pp][e] = 0.f; sc[pp][e] = 0.f; bi[pp][e] = 0.f; }
+            for (int e = 0; e < 4; ++e) Y[pp][e] = 0.f;
 
         for (int t0 = 0; t0 < NSBK; t0 += TSB) {
             const int tn = min(TSB, NSBK - t0);
@@ -312,84 +375,104 @@ __global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const Params p) {
                     const float* ur = us + ((size_t)m * TU + (size_t)sg * upseg) * 2;
                     float a = 0.f, b = 0.f;
                     for (int q = 0; q < upseg; ++q) { a += ur[2 * q]; b += ur[2 * q + 1]; }
-                    sx[(size_t)m * NSEG + sg] = a;
-                    sxt[(size_t)m * NSEG + sg] = b;
+                    sxx[(size_t)m * NSEG + sg] = make_float2(a, b);
                 }
                 consumer_sync(nthr);
                 x_whole = (TSB >= NSBK);
             }
 
+            // ---- one batch: SPB super-blocks of this warp, then the epilogue ---
+            // FULL: all SPB super-blocks exist (no guards); otherwise nex of them.
+            auto run_batch = [&](auto full_c, int sbf, int nex, int sbase, const unsigned char* rowg,
+                                 const unsigned char* rowh, const unsigned char* tileg) {
+                constexpr bool FULL = decltype(full_c)::value;
+                float sc[NPASS][4], bs[NPASS][4];
+#pragma unroll
+                for (int pp = 0; pp < NPASS; ++pp)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const bool pres = FULL || dsb[pp][c] < nex;
+                        float s0 = 0.f, s1 = 0.f, b0 = 0.f, b1 = 0.f;
+                        if (sring) {
+                            const int gl = ((((sbf - sbase) + dgrp[pp][c]) << gmul) >> gdiv) + dgs[pp][c];
+                            if (pres) {
+                                s0 = ring_scale<T>(tileg + p.soff, gl); s1 = ring_scale<T>(tileg + p.soff + 8 * sbw, gl);
+                                b0 = ring_scale<T>(tileg + p.boff, gl); b1 = ring_scale<T>(tileg + p.boff + 8 * sbw, gl);
+                            }
+                        } else {
+                            const int gg = (((sbf + dgrp[pp][c]) << gmul) >> gdiv) + dgs[pp][c];
+                            if (pres) {
+                                s0 = DT<T>::ld(scg, gg); s1 = DT<T>::ld(sch, gg);
+                                b0 = DT<T>::ld(big, gg); b1 = DT<T>::ld(bih, gg);
+                            }
+                        }
+                        sc[pp][c] = s0; sc[pp][2 + c] = s1; bs[pp][c] = b0; bs[pp][2 + c] = b1;
+                    }
+                float D[NPASS][4], E[NPASS][4];     // two MMA chains (even / odd k-steps)
+#pragma unroll
+                for (int pp = 0; pp < NPASS; ++pp)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) { D[pp][e] = 0.f; E[pp][e] = 0.f; }
+                const int xadv = (sbf - t0) * 4 * NP;
+#pragma unroll
+                for (int bi = 0; bi < SPB; ++bi) {
+                    if (FULL || bi < nex) {
+                        const int uo = (sbf - sbase + bi * wk) * 4 * UB + t * UB;
+                        uint32_t wg[NW], wh[NW];
+                        if constexpr (UB == 16) {
+                            const uint4 a = *reinterpret_cast<const uint4*>(rowg + uo);
+                            const uint4 b = *reinterpret_cast<const uint4*>(rowh + uo);
+                            wg[0] = a.x; wg[1] = a.y; wg[2] = a.z; wg[3] = a.w;
+                            wh[0] = b.x; wh[1] = b.y; wh[2] = b.z; wh[3] = b.w;
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < NW; ++q) {
+                                wg[q] = reinterpret_cast<const uint32_t*>(rowg + uo)[q];
+                                wh[q] = reinterpret_cast<const uint32_t*>(rowh + uo)[q];
+                            }
+                        }
+                        int xoff[NPASS];
+#pragma unroll
+                        for (int pp = 0; pp < NPASS; ++pp) xoff[pp] = xo[pp][bi] + xact[pp][bi] * xadv;
+                        tc_steps2<B, NPASS, NSPLIT>(std::make_integer_sequence<int, NSTEP / 2>{}, wg, wh, D, E, xs,
+                                                    xoff, plane, kbf16);
+                    }
+                }
+                const int segadv = (sbf - t0) * NGS;
+#pragma unroll
+                for (int pp = 0; pp < NPASS; ++pp)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        float2 ab = make_float2(0.f, 0.f);
+                        if (FULL || dsb[pp][c] < nex) ab = sxx[dseg[pp][c] + segadv];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int e = 2 * h + c;
+                            Y[pp][e] = fmaf(sc[pp][e], fmaf(-128.f, ab.y, D[pp][e] + E[pp][e]),
+                                            fmaf(bs[pp][e], ab.x, Y[pp][e]));
+                        }
+                    }
+            };
+
             // ---- this warp's super-blocks of the tile, stage by stage -------
             const int end = t0 + tn;
-            int sb = t0 + wkid;
-            int bi_ = 0;
             for (int ks = t0 / S; ks * S < end; ++ks) {
                 const int slot = it % STAGES, f = it / STAGES;
                 if (ok && !mbar_wait(full(slot), (uint32_t)(f & 1))) {
                     ok = false;
                     if (lane == 0) atomicOr(p.fault, 1u);
                 }
-                const int send = min(end, (ks + 1) * S);
+                const int sbase = ks * S;
+                const int send = min(end, sbase + S);
                 if (ok) {
-                    const unsigned char* st = ring + (size_t)slot * stage_bytes + (size_t)(wrid * 16 + g) * pitch + t * UB;
-                    for (; sb < send; sb += wk) {
-                        uint32_t wg[NW], wh[NW];
-                        const unsigned char* u = st + (sb - ks * S) * 4 * UB;
-                        if constexpr (UB == 16) {
-                            const uint4 a = *reinterpret_cast<const uint4*>(u);
-                            const uint4 b = *reinterpret_cast<const uint4*>(u + 8 * pitch);
-                            wg[0] = a.x; wg[1] = a.y; wg[2] = a.z; wg[3] = a.w;
-                            wh[0] = b.x; wh[1] = b.y; wh[2] = b.z; wh[3] = b.w;
-                        } else {
-#pragma unroll
-                            for (int q = 0; q < NW; ++q) {
-                                wg[q] = reinterpret_cast<const uint32_t*>(u)[q];
-                                wh[q] = reinterpret_cast<const uint32_t*>(u + 8 * pitch)[q];
-                            }
-                        }
-                        if (bi_ == 0) {
-                            // new batch: scales / biases of its slots (used at batch end)
-#pragma unroll
-                            for (int pp = 0; pp < NPASS; ++pp)
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int c = e & 1;
-                                    const int sbs = sb + dsbi[pp][c] * wk;
-                                    sc[pp][e] = 0.f; bi[pp][e] = 0.f;
-                                    if (dsbi[pp][c] >= 0 && sbs < end) {
-                                        const int grp = ((sbs << gmul) >> gdiv) + dgs[pp][c];
-                                        sc[pp][e] = DT<T>::ld((e >> 1) ? sch : scg, grp);
-                                        bi[pp][e] = DT<T>::ld((e >> 1) ? bih : big, grp);
-                                    }
-                                }
-                        }
-                        int xoff[NPASS];
-#pragma unroll
-                        for (int pp = 0; pp < NPASS; ++pp)
-                            xoff[pp] = bsbi[pp] == bi_ ? brow[pp] * xrow + ((sb - t0) * 4 + t) * NP
-                                                       : M * xrow + t * NP;
-                        tc_steps<B, NPASS, NSPLIT>(std::make_integer_sequence<int, NSTEP / 2>{}, wg, wh, D, xs, xoff,
-                                                   plane);
-                        if (bi_ == SPB - 1 || sb + wk >= end) {
-                            const int sb_first = sb - bi_ * wk;
-#pragma unroll
-                            for (int pp = 0; pp < NPASS; ++pp)
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int c = e & 1;
-                                    float a = 0.f, b = 0.f;
-                                    if (dsbi[pp][c] >= 0 && dsbi[pp][c] <= bi_) {
-                                        const int sl = (sb_first + dsbi[pp][c] * wk - t0) * NGS + dgs[pp][c];
-                                        a = sx[(size_t)dm[pp][c] * NSEG + sl];
-                                        b = sxt[(size_t)dm[pp][c] * NSEG + sl];
-                                    }
-                                    Y[pp][e] = fmaf(sc[pp][e], fmaf(-128.f, b, D[pp][e]), fmaf(bi[pp][e], a, Y[pp][e]));
-                                    D[pp][e] = 0.f;
-                                }
-                            bi_ = 0;
-                        } else {
-                            ++bi_;
-                        }
+                    const unsigned char* rowg = ring + (size_t)slot * stage_bytes + (size_t)(wrid * 16 + g) * pitch;
+                    const unsigned char* rowh = rowg + 8 * pitch;
+                    // scale / bias tile rows of this lane: stage + offset + row * sbw
+                    const unsigned char* tileg = ring + (size_t)slot * stage_bytes + (size_t)(wrid * 16 + g) * sbw;
+                    for (int sbf = sbase + wkid; sbf < send; sbf += SPB * wk) {
+                        const int nex = (send - sbf + wk - 1) / wk;
+                        if (nex >= SPB) run_batch(std::true_type{}, sbf, SPB, sbase, rowg, rowh, tileg);
+                        else run_batch(std::false_type{}, sbf, nex, sbase, rowg, rowh, tileg);
                     }
                 }
                 __syncwarp();
