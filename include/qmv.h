@@ -32,7 +32,11 @@
  *    asynchronous on that stream: it validates its arguments on the host, then
  *    enqueues kernels; it never synchronizes.  Kernels are launched with
  *    programmatic dependent launch, so they may start while the previous kernel
- *    in the stream drains; they read no input before that kernel has finished.
+ *    in the stream drains.  They read x (and write y) only after that kernel
+ *    has finished, but they begin fetching the WEIGHTS (w_packed, scales,
+ *    biases) at once: the kernel launched immediately before the call on the
+ *    same stream must not write them.  (Weights written by an earlier kernel,
+ *    by a copy, or on another stream ordered by an event are fine.)
  *  - Calls are thread-safe for distinct streams.
  *  - Return value: QMV_OK, or a negative qmv_status.  Argument errors are
  *    detected before any launch (nothing is enqueued).  QMV_ECUDA means a launch

@@ -37,9 +37,10 @@
 //     memory across the k-warps -> one rounding to the output dtype.
 //   * Rows past N in the last block read the last valid row and are not stored
 //     (the row-tail rule of the MLX fast_rows kernels).
-//   * The kernel waits on the previous grid (griddepcontrol.wait) before its
-//     first global read, so it may be launched with programmatic dependent
-//     launch; it lets dependents launch once its main loop is done.
+//   * The kernel waits on the previous grid (griddepcontrol.wait) before it
+//     reads x, so it may be launched with programmatic dependent launch; the
+//     first weight chunk is fetched before that wait, and dependents are let
+//     launch right after it (they too wait before reading this grid's y).
 #pragma once
 
 #include <cuda.h>
@@ -486,15 +487,25 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
     };
 
     const uint32_t kf32 = p.kf32;
-    grid_wait();   // inputs may come from the previous kernel in the stream
+    // The first chunk's weights (packed codes, scales, biases) are loaded
+    // before waiting on the previous kernel in the stream: weights are not
+    // produced by it (a precondition of the C ABI), x and y may be.
+    bool have = kt < min(TC, NC);
+    if (have) load_chunk(kt);
+    // let the next kernel in the stream start its own weight fetch now; it
+    // still waits for this grid to complete before it reads x
+    grid_launch_dependents();
+    grid_wait();
 
     for (int t0 = 0; t0 < NC; t0 += TC) {
         const int tcn = min(TC, NC - t0);          // chunks in this tile
         __syncthreads();
-        // the first chunk's weights are independent of x: issue them before
-        // staging x so both latencies overlap
-        bool have = kt < tcn;
-        if (have) load_chunk(t0 + kt);
+        // the tile's first chunk of weights is independent of x: issue it
+        // before staging x so both latencies overlap
+        if (t0 > 0) {
+            have = kt < tcn;
+            if (have) load_chunk(t0 + kt);
+        }
         stage_x<FAM, B, T, MAXM, U>(p, Xb, xs, sx, t0, tcn, KT, TI);
         __syncthreads();
         for (int i = 0; have;) {
@@ -507,8 +518,6 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
             if (have) load_chunk(t0 + cc);
         }
     }
-
-    grid_launch_dependents();
 
     warp_allreduce<R, MAXM>(acc);
     float gs = 1.f;

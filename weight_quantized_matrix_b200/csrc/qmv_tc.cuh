@@ -239,17 +239,26 @@ __global__ void __launch_bounds__(256) qmv_tc_kernel(const Params p) {
     uint32_t wring[PD][2][NW];
     float sc[NPASS][4], bi[NPASS][4];
 
+    // The first super-blocks' weights are loaded before waiting on the
+    // previous kernel in the stream: weights are not produced by it (a
+    // precondition of the C ABI), x and y may be.
+#pragma unroll
+    for (int q = 0; q < PD; ++q)
+        if (wkid + q * wk < min(TSB, NSBK)) loadW(wring[q][0], wring[q][1], wkid + q * wk);
+    grid_launch_dependents();        // the next kernel may start fetching its weights
     grid_wait();
 
     for (int t0 = 0; t0 < NSBK; t0 += TSB) {
         const int tn = min(TSB, NSBK - t0);
         const int first = t0 + wkid, end = t0 + tn;
         __syncthreads();
-        // weights of the first super-blocks do not depend on x: issue them
-        // before staging x
+        // weights of the tile's first super-blocks do not depend on x: issue
+        // them before staging x
+        if (t0 > 0) {
 #pragma unroll
-        for (int q = 0; q < PD; ++q)
-            if (first + q * wk < end) loadW(wring[q][0], wring[q][1], first + q * wk);
+            for (int q = 0; q < PD; ++q)
+                if (first + q * wk < end) loadW(wring[q][0], wring[q][1], first + q * wk);
+        }
 
         // ---- stage x: fragment-ordered bf16 planes + per-unit sums ------------
         {
@@ -381,8 +390,6 @@ __global__ void __launch_bounds__(256) qmv_tc_kernel(const Params p) {
             }
         }
     }
-
-    grid_launch_dependents();
 
     // ---- reduce over slots of the same x row and over k-warps, store ---------
     float* myred = red + (size_t)(wrid * wk + wkid) * 16 * 8 * NPASS;

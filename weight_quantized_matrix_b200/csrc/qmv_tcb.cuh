@@ -187,7 +187,6 @@ __global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const __grid_constant__
         mbar_init_fence();
     }
     __syncthreads();
-    grid_wait();
 
     const uint8_t* W = p.w + bz * p.w_bs;
     const long long sb0 = bz * p.s_bs;
@@ -195,6 +194,7 @@ __global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const __grid_constant__
 
     // ============================ producer warp ==============================
     if (warp == NCW) {
+        grid_launch_dependents();    // the next kernel may start fetching its weights
         const uint32_t ring0 = smem_addr(ring);
         int it = 0;
         bool ok = true;
@@ -232,11 +232,13 @@ __global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const __grid_constant__
             if (!mbar_wait(full(s), (uint32_t)(last & 1))) code |= 4u;
         }
         if (code && lane == 0) atomicOr(p.fault, code);
-        grid_launch_dependents();
         return;
     }
 
     // ============================ consumer warps ============================
+    // The producer streams only weights and starts at once; the consumers
+    // read x and write y, which the previous kernel in the stream may own.
+    grid_wait();
     const int nthr = NCW * 32;
     const int g = lane >> 2, t = lane & 3;
     const int wkid = warp % wk, wrid = warp / wk;
@@ -480,8 +482,6 @@ __global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const __grid_constant__
                 ++it;
             }
         }
-
-        if (rb + (int)gridDim.x >= nrb) grid_launch_dependents();
 
         // ---- reduce over slots of the same x row and over k-warps, store -----
         float* myred = red + (size_t)warp * 16 * 8 * NPASS;
