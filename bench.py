@@ -17,15 +17,19 @@ HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
                     M=1 and once at M=8 (8 calls per step).
   probe             bandwidth probe, affine 4-bit g64 bf16, N=K=16384, M=1.
 
-Timing: W untimed warm-up steps, then K steps; each step is bracketed by CUDA
-events on the launching stream; L2 is flushed before every step, outside the
-events (a 512 MB buffer is written, then a 256 MB buffer is read so that no
-dirty line's write-back falls inside the timed region), and within a step the weights rotate
+Timing: W untimed warm-up steps, then K steps.  A step is ONE CUDA graph
+holding every call of the workload (dependent calls linked by programmatic
+dependent launch), as a decode step would run; it is bracketed by CUDA events
+on the launching stream.  L2 is flushed before every step, outside the events
+(a 512 MB buffer is written, then a 256 MB buffer is read so that no dirty
+line's write-back falls inside the timed region), and the weights rotate
 through copies totalling more than twice the L2 so calls read from HBM.  The
 timed region is bracketed by a barrier and a device synchronize; multi-GPU runs
 are N independent replicas (the path has no exchange step) and report the max
 over ranks.  nvidia-smi clocks are sampled (20 ms) from the graph warm-up through
-the timed region.
+the timed region.  The per-shape lines (and the roofline's dominant kernel)
+come from a second pass that replays each shape's own graph alone, L2 flushed,
+between a pair of CUDA events (one graph launch per shape included).
 
 --impl reference times the fp64 CPU oracle (the only other implementation of
 this operation there is) on a bounded sample of the same workload, on the host
@@ -185,7 +189,7 @@ class Chain8:
     def graph_variants(self, s):
         return 1          # the weight rotation is inside the chain
 
-    def run_group(self, s, e2e=False):
+    def run_group(self, s, e2e=False, v=0):
         q, N = self.q, s["N"]
         if e2e:
             s["x0"].copy_(s["x0_host"], non_blocking=True)
@@ -242,11 +246,10 @@ class Layer:
     def graph_variants(self, s):
         return len(s["ws"])   # one graph per weight copy; step k replays copy k
 
-    def run_group(self, s, e2e=False):
+    def run_group(self, s, e2e=False, v=0):
         if e2e:
             s["x"].copy_(s["x_host"], non_blocking=True)
-        w, sc, bi = s["ws"][s["it"] % len(s["ws"])]
-        s["it"] += 1
+        w, sc, bi = s["ws"][v % len(s["ws"])]      # weight copy v: copies rotate across steps
         self.q.qmv_affine(s["x"], w, sc, bi, s["y"], s["M"], s["N"], s["K"], 4, 64, "bf16")
         if e2e:
             s["y_host"].copy_(s["y"], non_blocking=True)
@@ -311,37 +314,45 @@ def run_ours(args, rank, world, local_rank):
 
     with torch.cuda.stream(stream):
         # eager warm-up through the public API (also sets kernel attributes)
-        for _ in range(W):
+        for k in range(W):
             for _, s in groups:
-                wl.run_group(s)
+                wl.run_group(s, v=k)
         torch.cuda.synchronize()
-        # one CUDA graph per group and weight copy: the chain's 64 dependent
-        # launches (with their programmatic-dependent-launch edges) replay
-        # without host overhead
-        graphs = []
+        # One CUDA graph per STEP (all groups, their dependent launches with
+        # programmatic-dependent-launch edges), one per weight-copy variant,
+        # as a decode step would run; and one graph per group for the
+        # per-shape breakdown.
+        nv = max(wl.graph_variants(s) for _, s in groups)
+        step_graphs = []
+        for v in range(nv):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _, s in groups:
+                    wl.run_group(s, v=v)
+            step_graphs.append(g)
+        group_graphs = []
         for _, s in groups:
             gs = []
-            for _ in range(wl.graph_variants(s)):
+            for v in range(wl.graph_variants(s)):
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=stream):
-                    wl.run_group(s)
+                    wl.run_group(s, v=v)
                 gs.append(g)
-            graphs.append(gs)
+            group_graphs.append(gs)
         clk = ClockSampler(local_rank)
         clk.start()
         t_load = time.perf_counter()
         k = 0
         while k < W or time.perf_counter() - t_load < 0.3:     # warm-up replays, >= 0.3 s of load
-            for gs in graphs:
-                gs[k % len(gs)].replay()
+            step_graphs[k % nv].replay()
             k += 1
             if k % 16 == 0:
                 torch.cuda.synchronize()
         torch.cuda.synchronize()
 
         def timed(e2e):
-            ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in groups] for _ in range(args.steps)]
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
             if world > 1:
                 dist.barrier()
             torch.cuda.synchronize()
@@ -349,28 +360,41 @@ def run_ours(args, rank, world, local_rank):
             for k in range(args.steps):
                 flush.fill_(k & 0xFF)                   # L2 flush, outside the events
                 flush_rd.max()
-                for gi, (_, s) in enumerate(groups):
-                    ev[k][gi][0].record(stream)
-                    if e2e:
-                        wl.run_group(s, e2e=True)       # public API, host copies included
-                    else:
-                        gs = graphs[gi]
-                        gs[k % len(gs)].replay()
-                    ev[k][gi][1].record(stream)
+                ev[k][0].record(stream)
+                if e2e:
+                    for _, s in groups:
+                        wl.run_group(s, e2e=True, v=k)  # public API, host copies included
+                else:
+                    step_graphs[k % nv].replay()
+                ev[k][1].record(stream)
             torch.cuda.synchronize()
             wall = time.perf_counter() - t0
             clocks = clk.stop() if not e2e else None
             if world > 1:
                 dist.barrier()
-            per_group = np.array([[a.elapsed_time(b) for (a, b) in ev[k]] for k in range(args.steps)])  # ms
-            return per_group, wall, clocks
+            return np.array([a.elapsed_time(b) for (a, b) in ev]), wall, clocks   # ms per step
 
-        per_group, wall, clocks = timed(False)
-        per_group_e2e, _, _ = timed(True)
-        del graphs
+        step_ms, wall, clocks = timed(False)
+        step_ms_e2e, _, _ = timed(True)
 
-    step_ms = per_group.sum(axis=1)           # device time of each step
-    step_ms_e2e = per_group_e2e.sum(axis=1)
+        # per-shape breakdown (not the headline): each group's own graph, L2
+        # flushed before every replay, timed alone between a pair of events
+        # (so it also carries one graph launch per group)
+        reps = max(8, nv)
+        per_group = []
+        for gi, (_, s) in enumerate(groups):
+            gs = group_graphs[gi]
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+            for r in range(reps):
+                flush.fill_(r & 0xFF)
+                flush_rd.max()
+                ev[r][0].record(stream)
+                gs[r % len(gs)].replay()
+                ev[r][1].record(stream)
+            torch.cuda.synchronize()
+            per_group.append(float(np.mean([a.elapsed_time(b) for a, b in ev])))   # ms per group replay
+        del step_graphs, group_graphs
+
     tot_ms = float(step_ms.sum())
     tot_ms_e2e = float(step_ms_e2e.sum())
     if world > 1:
@@ -385,7 +409,7 @@ def run_ours(args, rank, world, local_rank):
     shapes, by_kernel = [], {}
     peak, peak_kind = peaks()
     for gi, (label, s) in enumerate(groups):
-        ms = float(per_group[:, gi].mean())
+        ms = float(per_group[gi])
         n = wl.calls_per_step // len(groups) if isinstance(wl, Chain8) else 1
         b = wl.group_bytes(s)
         plan = wl.group_plan(s)

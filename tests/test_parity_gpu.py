@@ -513,6 +513,46 @@ def test_bulk_ring_x_tiles(q, ring, N):
     compare(y[:, rows], ref[:, rows], ad[:, rows], "f32", what="tcb tiles")
 
 
+# ----------------------------------------- few rows: the latency kernel ----
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("M", [1, 3, 8])
+@pytest.mark.parametrize("K", [480, 2560, 19200])
+def test_direct_path_grid(q, bits, dtype, M, K):
+    """N <= 64 rows: every width and dtype, one to two units per lane and
+    (K = 19200, 600 units) units dequantized after the wait."""
+    group = 32 if K == 480 else 64
+    N = 17
+    plan = q.qmv_describe_plan("affine", M, N, K, bits, group, dtype)
+    assert "path=direct" in plan, plan
+    c = synth.affine_case(M, N, K, bits, group, dtype, seed=_seed("direct", bits, dtype, M, K))
+    y = run_affine(q, c)[0]
+    ref, ad = oracle_affine(c)
+    compare(y, ref, ad, dtype, what=f"direct b{bits} {dtype} M{M} K{K}")
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("M", [1, 4])
+def test_direct_path_fp(q, mode, dtype, M):
+    q.qmv_force_config(5, -1, -1, -1)
+    c = synth.fp_case(M, 9, 2048, mode, dtype, seed=_seed("directfp", mode, dtype, M), batch=2)
+    y = run_fp(q, c)
+    for b in range(2):
+        ref, ad = oracle_fp(c, b=b)
+        compare(y[b], ref, ad, dtype, what=f"direct {mode} {dtype} M{M} batch{b}")
+
+
+@pytest.mark.parametrize("bits", [3, 8])
+def test_direct_path_misaligned_and_batched(q, bits):
+    """4-byte aligned weights (no 16-byte loads) and batch 2 with a shared x."""
+    c = synth.affine_case(2, 40, 2560, bits, 64, "bf16", seed=_seed("directmis", bits), batch=2)
+    y = run_affine(q, c, w_offset=4, x_batched=False)
+    for b in range(2):
+        ref, ad = oracle_affine(c, b=b, x_batched=False)
+        compare(y[b], ref, ad, "bf16", what=f"direct misaligned b{bits} batch{b}")
+
+
 @pytest.mark.parametrize("bits", [3, 4, 8])
 def test_cuda_core_path_grid(q, bits):
     """The CUDA-core kernel (wide and narrow chunks) stays covered."""

@@ -272,6 +272,22 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     bool wide = w16 && (K % c_wide == 0);
     if (g_forced.path == 0) wide = false;
 
+    // ---- few output rows: the latency kernel (weights dequantized before the
+    // grid-dependency wait, one block per row) --------------------------------
+    if (K > 0 && (g_forced.path == 5 || (g_forced.path < 0 && N <= 64))) {
+        const int units = K / 32;
+        int thr = ((units + 31) / 32) * 32;
+        if (thr > 256) thr = 256;
+        if (thr < 32) thr = 32;
+        const long long row_bytes = (long long)K * fi.bits / 8;
+        pl->maxm = maxm; pl->R = 1; pl->tc = 3; pl->npass = 0; pl->wk = thr / 32; pl->wr = 1;
+        pl->wide = (w16 && fi.bits % 4 == 0 && row_bytes % 16 == 0) ? 1 : 0;
+        pl->tile_iters = (units + thr - 1) / thr; pl->C = 32; pl->smem = (size_t)8 * maxm * 4;
+        pl->grid = dim3((unsigned)N, 1, (unsigned)batch);
+        pl->block = dim3((unsigned)thr, 1, 1);
+        return QMV_OK;
+    }
+
     // ---- tensor-core kernel with the bulk-copy weight ring --------------------
     // (measured on B200: the fastest path once M >= 2, and for large 2-bit
     // matrices at M = 1)
@@ -469,6 +485,7 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
         if (!p.fault) return QMV_ECUDA;
         return finish(qmv::launch_tcb_affine(bits, dtype, pl.npass, pl.spb, p, L));
     }
+    if (pl.tc == 3) return finish(qmv::launch_direct(fam, bits, dtype, pl.maxm, pl.wide != 0, p, L));
     if (pl.tc) return finish(qmv::launch_tc_affine(bits, dtype, pl.npass, p, L));
     if (fam == qmv::FAM_AFFINE) {
         switch (bits) {
@@ -620,7 +637,7 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
     snprintf(buf, (size_t)buflen,
              "path=%s chunk=%d maxm=%d rows_per_warp=%d warps_k=%d warps_rows=%d tile_iters=%d "
              "grid=%u block=%u smem=%zu stage_sb=%d batch_sb=%d scale_ring=%d",
-             pl.tc == 2 ? "tcb" : pl.tc ? "tc" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr,
+             pl.tc == 3 ? "direct" : pl.tc == 2 ? "tcb" : pl.tc ? "tc" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr,
              pl.tile_iters, pl.grid.x, pl.block.x, pl.smem, pl.sps, pl.spb, pl.sring);
     return QMV_OK;
 }

@@ -67,6 +67,10 @@ constexpr int kTcbStages = 4;
 
 
 
+// Few-rows latency kernels (qmv_direct_kernel): maxm in {1, 2, 4, 8}; wide =
+// 16-byte unit loads (4- and 8-bit codes, 16-byte aligned rows).
+cudaError_t launch_direct(int fam, int bits, int dtype, int maxm, bool wide, const Params& p, const Launch& L);
+
 cudaError_t launch_dequant(int fam, int bits, int dtype, const uint8_t* w, const void* scales,
                            const void* biases, const float* gscale, float* out, int N, int K, int G,
                            long long w_row, cudaStream_t s);
