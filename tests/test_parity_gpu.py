@@ -441,7 +441,7 @@ def test_bulk_ring_path_grid(q, ring, bits, group, dtype, M):
 
 
 @pytest.mark.parametrize("cfg", [(4, -1, 1, 1), (4, -1, 8, 1), (4, -1, 1, 8), (4, -1, 2, 4), (4, -1, 4, 2),
-                                 (4, -1, 3, 2)])
+                                 (4, -1, 3, 2), (4, -1, 6, 2), (4, -1, 4, 3), (4, -1, 12, 1), (4, -1, 3, 4)])
 @pytest.mark.parametrize("bits", [2, 3, 5, 8])
 def test_bulk_ring_block_shapes(q, ring, cfg, bits):
     q.qmv_force_config(*cfg)

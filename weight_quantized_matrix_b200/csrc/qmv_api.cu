@@ -198,13 +198,27 @@ bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s
     const int np = tc_np_of(bits);
     const int nsbk = K / SB;
     const int sms = device_sms();
-    // rows per block: one x row -> 32 (2-bit: 64); several x rows -> 64 rows
-    // once that still gives ~96+ row blocks, else 32, else 16 (measured on B200)
-    int wr = M == 1 ? (bits == 2 ? 4 : 2) : (N >= 6144 ? 4 : N >= 2048 ? 2 : 1);
-    int wk = 8 / wr;
-    if (g_forced.wr > 0) wr = g_forced.wr > 8 ? 8 : g_forced.wr;
-    if (g_forced.wk > 0) wk = g_forced.wk > 8 ? 8 : g_forced.wk;
-    while (wk * wr > 8) --wk;
+    // Consumer warps and rows per block (measured on B200).  One x row: 8
+    // consumer warps, 32-row blocks (2-bit: 64).  Several x rows: 12 consumer
+    // warps, wr in {2, 3, 4} (wk = 12 / wr) minimising (rounds of row blocks
+    // over the SMs) x (rows per block), i.e. the busiest SM's share.
+    int wr, wk;
+    if (M == 1) {
+        wr = bits == 2 ? 4 : 2;
+        wk = 8 / wr;
+    } else {
+        wr = 2;
+        long long best = -1;
+        for (int w = 2; w <= 4; ++w) {
+            const long long nrb = ((long long)N + 16 * w - 1) / (16 * w);
+            const long long cost = ((nrb + sms - 1) / sms) * w;
+            if (best < 0 || cost < best) { best = cost; wr = w; }
+        }
+        wk = 12 / wr;
+    }
+    if (g_forced.wr > 0) wr = g_forced.wr > 12 ? 12 : g_forced.wr;
+    if (g_forced.wk > 0) wk = g_forced.wk > 12 ? 12 : g_forced.wk;
+    while (wk * wr > 12) --wk;
     if (wk > nsbk) wk = nsbk;
     if (wk < 1) wk = 1;
     const int rows = 16 * wr;
@@ -483,7 +497,7 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     if (pl.tc == 2) {
         p.fault = fault_word();
         if (!p.fault) return QMV_ECUDA;
-        return finish(qmv::launch_tcb_affine(bits, dtype, pl.npass, pl.spb, p, L));
+        return finish(qmv::launch_tcb_affine(bits, dtype, pl.npass, pl.spb, pl.wk * pl.wr > 8, p, L));
     }
     if (pl.tc == 3) return finish(qmv::launch_direct(fam, bits, dtype, pl.maxm, pl.wide != 0, p, L));
     if (pl.tc) return finish(qmv::launch_tc_affine(bits, dtype, pl.npass, p, L));

@@ -61,8 +61,9 @@ cudaError_t launch_fp(int fam, int dtype, int maxm, int R, bool wide, const Para
 // Tensor-core kernels (qmv_tc_kernel): npass in {1, 2, 4}.
 cudaError_t launch_tc_affine(int bits, int dtype, int npass, const Params& p, const Launch& L);
 // Tensor-core kernels with the bulk-copy weight ring (qmv_tcb_kernel):
-// (npass, spb) in {(1,1), (1,2), (1,4), (1,8), (2,1), (4,1)}.
-cudaError_t launch_tcb_affine(int bits, int dtype, int npass, int spb, const Params& p, const Launch& L);
+// (npass, spb) in {(1,1), (1,2), (1,4), (1,8), (2,1), (4,1)}; w12: built for
+// 12 consumer warps (else 8).
+cudaError_t launch_tcb_affine(int bits, int dtype, int npass, int spb, bool w12, const Params& p, const Launch& L);
 constexpr int kTcbStages = 4;
 
 
@@ -106,8 +107,12 @@ inline bool shape_instantiated(int maxm, int R, bool wide) {
     }
 #define QMV_TCB_SHAPE(T_, NPASS_, SPB_)                                                      \
     if (npass == NPASS_ && spb == SPB_) {                                                    \
+        if (w12) {                                                                           \
+            static std::atomic<unsigned> cfg_{0};                                            \
+            return launch_kernel(qmv_tcb_kernel<BITS_, T_, NPASS_, SPB_, kTcbStages, 416>, cfg_, L, p); \
+        }                                                                                    \
         static std::atomic<unsigned> cfg_{0};                                                \
-        return launch_kernel(qmv_tcb_kernel<BITS_, T_, NPASS_, SPB_, kTcbStages>, cfg_, L, p); \
+        return launch_kernel(qmv_tcb_kernel<BITS_, T_, NPASS_, SPB_, kTcbStages, 288>, cfg_, L, p); \
     }
 #define QMV_TCB_SHAPES(T_)                                                                   \
     QMV_TCB_SHAPE(T_, 1, 1) QMV_TCB_SHAPE(T_, 1, 2) QMV_TCB_SHAPE(T_, 1, 4)                 \

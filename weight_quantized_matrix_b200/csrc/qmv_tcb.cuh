@@ -130,8 +130,10 @@ template <> __device__ __forceinline__ float ring_scale<__nv_bfloat16>(const uns
 //   sxx   M * NSEG float2      {sum(x), sum(x~)} per segment of the tile
 //   us    M * TU * 2 floats    per-unit sums
 //   red   NCW * 16 * 8*NPASS floats
-template <int B, class T, int NPASS, int SPB, int STAGES>
-__global__ void __launch_bounds__(288, 1) qmv_tcb_kernel(const __grid_constant__ Params p) {
+// MAXT: threads per block the kernel is compiled for (288 = 8 consumer warps
+// + producer, 416 = 12 + producer; the register budget follows).
+template <int B, class T, int NPASS, int SPB, int STAGES, int MAXT>
+__global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant__ Params p) {
     using Gm = TcGeom<B>;
     constexpr TcPlanData P = tc_make_plan<B, false>();
     constexpr int NP = P.np, NSTEP = NP / 2;
