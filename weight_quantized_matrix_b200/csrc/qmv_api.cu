@@ -96,9 +96,11 @@ struct Plan {
     dim3 grid, block;
 };
 
+// Rows per warp on the wide path (x reuse vs registers); measured on B200:
+// 4 rows win at M <= 2 for every width (5/6-bit included).
 int rows_per_warp_cap(int bits, int maxm) {
-    if (maxm <= 2) return (bits == 3 || bits == 5 || bits == 6) ? 2 : 4;
-    return 2;
+    (void)bits;
+    return maxm <= 2 ? 4 : 2;
 }
 
 // ---- tensor-core launch shape --------------------------------------------------
@@ -353,7 +355,10 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
         const int rcap = wide ? rows_per_warp_cap(fi.bits, maxm) : 1;
         R = N >= 1024 ? rcap : (N >= 256 ? (rcap < 2 ? rcap : 2) : 1);
         const long long warps = ((long long)N + R - 1) / R * batch;
-        wk = 1;
+        // k-warps: at least 2 for long rows (>= 256 chunks: more loads in
+        // flight per row; not for 6-bit, whose 12-word chunks already fill
+        // the registers), more while the GPU holds fewer than ~8 warps per SM
+        wk = (NC >= 256 && fi.bits != 6) ? 2 : 1;
         while (wk < 8 && warps * wk < (long long)sms * 8 && NC >= 64 * wk) wk *= 2;
         wr = wk >= 8 ? 1 : 8 / wk;
         if (wr > 4 && wk == 1) wr = 4;
