@@ -485,7 +485,7 @@ def test_bulk_ring_tail_rows_bitwise_prefix(q, ring, bits):
 def test_bulk_ring_scales_in_or_out_of_ring(q, ring, bits, group, M):
     """Scales and biases ride in the ring when 16-byte aligned and read from
     global memory otherwise: the two give bitwise equal outputs."""
-    q.qmv_force_config(4, -1, -1, -1)
+    q.qmv_force_config(4, -1, 4, 2)
     N, K = 300, 4096
     plan = q.qmv_describe_plan("affine", M, N, K, bits, group, "bf16")
     assert "path=tcb" in plan and "scale_ring=1" in plan, plan

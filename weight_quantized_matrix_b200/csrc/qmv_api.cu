@@ -109,10 +109,10 @@ int rows_per_warp_cap(int bits, int maxm) {
 // the tensor cores win (the CUDA cores would need M FMAs per code); with one x
 // row they win only once the matrix is large enough to hide their longer
 // pipeline (about 48 MB of packed weights).
-bool tc_preferred(int M, int N, int K, int bits) {
+bool tc_preferred(int M, int N, int K, int bits, int dtype) {
     if (N < 64 || bits == 6) return false;
     if (M >= 2) return true;
-    if (bits == 8) return false;
+    if (bits == 8 || dtype != QMV_BF16) return false;   // one x row in f16 / f32: the CUDA cores win
     const double wbytes = (double)N * K * bits / 8.0;
     return wbytes >= 48.0 * 1024 * 1024;
 }
@@ -204,9 +204,14 @@ bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s
     // consumer warps, 32-row blocks (2-bit: 64).  Several x rows: 12 consumer
     // warps, wr in {2, 3, 4} (wk = 12 / wr) minimising (rounds of row blocks
     // over the SMs) x (rows per block), i.e. the busiest SM's share.
+    // x of the whole K staged once per block needs about this much shared memory
+    const long long x_bytes = (long long)nsplit * M * (K / uc) * np * 4;
     int wr, wk;
-    if (M == 1) {
-        wr = bits == 2 ? 4 : 2;
+    if (M == 1 || (N >= 15360 && (M == 2 || x_bytes > 96 * 1024))) {
+        // one or two x rows over many rows, or x too large to stay staged
+        // across row blocks: 128-row blocks, K not split, as few row blocks
+        // per block as possible (5-bit: 64 rows, K over 2 warps)
+        wr = bits == 5 ? 4 : 8;
         wk = 8 / wr;
     } else {
         wr = 2;
@@ -237,16 +242,26 @@ bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s
     sps = sps / quantum * quantum;
     if (sps < quantum) sps = quantum;
     if (sps > nsbk) sps = (nsbk + quantum - 1) / quantum * quantum;
-    // stage layout: ROWS packed rows, pitch bytes apart, then (scales in the
-    // ring) a scale tile and a bias tile of ROWS x sbw bytes, filled by tensor
-    // copies whose column start must sit on 16 bytes and whose box is <= 256
+    if (rows > 256) return false;
+    // a scale tile row must be a whole number of 16 bytes to travel in the
+    // ring: grow a short stage to the next such multiple of the quantum
+    if (s16 && ((long long)(K / G) * es) % 16 == 0) {
+        auto sb_bytes = [&](int v) { return (G <= SB ? v * (SB / G) : v / (G / SB)) * es; };
+        int v = sps;
+        while (v < 4 * sps && v < nsbk && sb_bytes(v) % 16 != 0) v += quantum;
+        if (sb_bytes(v) % 16 == 0 && v * 4 * ub / 8 <= 256) sps = v;
+    }
+    while (sps > quantum && sps * 4 * ub / 8 > 256) sps -= quantum;
+    if (sps * 4 * ub / 8 > 256) return false;
+    // stage layout: ROWS packed rows of pitch = S * 4 * UB bytes, then (scales
+    // in the ring) a scale tile and a bias tile of ROWS x sbw bytes; each is
+    // one tensor copy, whose column start must sit on 16 bytes and whose box
+    // is at most 256 elements a side (the rows' box counts 8-byte elements)
     auto layout = [&](int s, int* sring, int* sbw, int* stage) {
         const int box0 = G <= SB ? s * (SB / G) : s / (G / SB);
         *sbw = box0 * es;
         *sring = (s16 && ((long long)(K / G) * es) % 16 == 0 && *sbw % 16 == 0 && box0 <= 256 && rows <= 256) ? 1 : 0;
-        const int wpart = (s * 4 * ub + 15) / 16 * 16;
-        const int pad = ub == 16 ? 64 : 16;           // pitch mod 128 (bank spread of the unit loads)
-        const int pitch = wpart + ((pad - wpart % 128) % 128 + 128) % 128;
+        const int pitch = s * 4 * ub;                 // dense rows, as the tensor copy lays them out
         *stage = rows * pitch + (*sring ? 2 * rows * *sbw : 0);
         return pitch;
     };
@@ -305,10 +320,10 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     }
 
     // ---- tensor-core kernel with the bulk-copy weight ring --------------------
-    // (measured on B200: the fastest path once M >= 2, and for large 2-bit
+    // (measured on B200: the fastest path once M >= 2, and for large 2/3/4/5-bit
     // matrices at M = 1)
     // (6-bit codes do not pair: the ring kernel wins there only at M = 8)
-    const bool ring_pick = M >= 2 ? (N >= 64 && (bits != 6 || M >= 8)) : (bits == 2 && tc_preferred(M, N, K, bits));
+    const bool ring_pick = M >= 2 ? (N >= 64 && (bits != 6 || M >= 8)) : tc_preferred(M, N, K, bits, dtype);
     if (aff && K > 0 && (g_forced.path == 4 || (g_forced.path < 0 && ring_pick))) {
         TcbShape ts;
         if (tcb_shape(M, N, K, bits, G_of_plan, dtype, w16, s16, &ts)) {
@@ -324,7 +339,7 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
 
     // ---- tensor-core kernel (affine, enough rows to fill the GPU) -------------
     if (aff && K > 0 && g_forced.path != 0 && g_forced.path != 1 &&
-        (g_forced.path == 3 || tc_preferred(M, N, K, bits))) {
+        (g_forced.path == 3 || tc_preferred(M, N, K, bits, dtype))) {
         TcShape ts;
         if (tc_shape(M, N, K, bits, G_of_plan, dtype, w16, &ts)) {
             pl->maxm = maxm; pl->R = 1; pl->wide = 1; pl->tc = 1; pl->npass = ts.npass;
@@ -445,6 +460,20 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
+// [batch][N][row bytes / 8] packed rows as a 3-D tensor map of 8-byte
+// elements with box {box0, rows, 1}; out-of-range elements read as zero.
+bool encode_rows_map(CUtensorMap* m, const void* base, long long row_bytes, int N, int batch, int box0, int rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)(row_bytes / 8), (cuuint64_t)N, (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)row_bytes * (cuuint64_t)N};
+    const cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // [batch][N][K/G] scales (or biases) as a 3-D tensor map with box
 // {box0 groups, rows, 1}; out-of-range elements read as zero.
 bool encode_scale_map(CUtensorMap* m, const void* base, int dtype, long long KG, int N, int batch, int box0,
@@ -478,9 +507,15 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
         const int box0 = pl.sbw / elem_bytes(dtype), rows = 16 * pl.wr;
         if (!encode_scale_map(&p.smap, scales, dtype, K / G, N, batch, box0, rows) ||
             !encode_scale_map(&p.bmap, biases, dtype, K / G, N, batch, box0, rows)) {
+            cudaGetLastError();
             st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, false);   // scales from global memory
             if (st != QMV_OK) return st;
         }
+    }
+    // the packed rows' tensor map, for the final plan
+    if (pl.tc == 2 && !encode_rows_map(&p.wmap, w, row_bytes, N, batch, pl.pitch / 8, 16 * pl.wr)) {
+        cudaGetLastError();
+        return QMV_ECUDA;
     }
     p.x = x; p.w = static_cast<const uint8_t*>(w); p.scales = scales; p.biases = biases;
     p.gscale = gscale; p.y = y;

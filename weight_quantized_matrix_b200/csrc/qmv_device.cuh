@@ -76,6 +76,7 @@ struct Params {
     int soff, boff;         // bulk-ring kernel: byte offsets of the scale / bias tiles in a ring stage
     int sbw;                // bulk-ring kernel: bytes per row of those tiles
     CUtensorMap smap, bmap; // bulk-ring kernel: scales / biases as [batch][N][K/G] tensors
+    CUtensorMap wmap;       // bulk-ring kernel: packed rows as [batch][N][row bytes / 8] u64
     // Exponent patterns OR-ed into decoded fields, passed in so that kernels
     // hold them in registers: then mask-and-OR is one three-input logic op
     // (with both operands immediate it would take two).

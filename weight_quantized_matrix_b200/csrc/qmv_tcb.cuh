@@ -10,9 +10,9 @@
 // Work: the grid is persistent over ROW BLOCKS of ROWS = 16*wr rows (block b
 // takes row blocks b, b + gridDim.x, ...).  A row block's packed rows are cut
 // along K into ring STAGES of S super-blocks; the producer copies stage after
-// stage (per row: the packed bytes and, when their layout allows, the stage's
-// scales and biases; one bulk copy each, issued by the producer's lanes) into
-// the ring, across row-block boundaries, while consumers compute.  Consumer
+// stage (the packed rows, and when their layout allows the stage's scales and
+// biases: one 3-D tensor copy each) into the ring, across row-block
+// boundaries, while consumers compute.  Consumer
 // warp (wrid, wkid) owns row tile wrid (16 rows) and the super-blocks wkid,
 // wkid + wk, ... of every stage, taken SPB at a time: one BATCH fills the 8*NPASS
 // slot columns of the MMAs (decode and slot columns as in qmv_tc.cuh) and
@@ -29,9 +29,9 @@
 // computing, keeps its barrier schedule so no warp waits on another forever,
 // and the producer waits (bounded) for every copy it issued before it exits.
 //
-// Ring rows are padded (pitch = 64 mod 128 bytes for 16-byte units, 16 mod
-// 128 for 12/20-byte units) so the 8 rows read by one load instruction fall in
-// distinct banks.
+// Ring rows are dense (pitch = the stage's S * 4 * UB bytes, as the tensor copy
+// lays them out); the two rows one load instruction touches per 8 lanes then
+// share banks, a 2-way conflict on the two unit loads per super-block.
 #pragma once
 
 #include <type_traits>
@@ -83,14 +83,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
         if (global_ns() - t0 > kWaitLimitNs) return false;
     }
 }
-// Global -> this CTA's shared memory, completion counted on `bar` in bytes.
-// dst, src 16-byte aligned; bytes a multiple of 16.
-__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
 // Tensor tile [box] of a 3-D tensor map -> this CTA's shared memory (128-byte
 // aligned destination), completion counted on `bar` in bytes (the full box,
 // out-of-range elements zero-filled).  No multicast.
@@ -122,8 +114,8 @@ template <> __device__ __forceinline__ float ring_scale<__nv_bfloat16>(const uns
 // Shared memory (bytes, in order):
 //   bars  128            full[STAGES], empty[STAGES]
 //   ring  STAGES stages (128-byte aligned) of: ROWS packed rows (pitch bytes
-//         apart), then (p.sring) the scale tile at p.soff and the bias tile at
-//         p.boff, ROWS x p.sbw bytes each
+//         each, dense), then (p.sring) the scale tile at p.soff and the bias
+//         tile at p.boff, ROWS x p.sbw bytes each
 //   xs    NSPLIT * plane * 4    plane = M*xrow + 4*NP + 4 u32: the x rows of
 //                               the tile (bf16 pairs, fragment order), then one
 //                               super-block of zeros read by inactive lanes
@@ -190,7 +182,6 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
     }
     __syncthreads();
 
-    const uint8_t* W = p.w + bz * p.w_bs;
     const long long sb0 = bz * p.s_bs;
     const int nks = (NSBK + S - 1) / S;
 
@@ -205,13 +196,14 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
                 const int slot = it % STAGES, f = it / STAGES;
                 if (f > 0 && !mbar_wait(empty(slot), (uint32_t)((f - 1) & 1))) { ok = false; break; }
                 const int nsb = min(S, NSBK - ks * S);
-                const uint32_t rowb = (uint32_t)(nsb * 4 * UB);
                 const uint32_t st0 = ring0 + (uint32_t)(slot * stage_bytes);
                 if (lane == 0) {
-                    // packed rows (one bulk copy per row) + the stage's scale and
-                    // bias tiles (one tensor copy each: ROWS x sbw bytes, columns
-                    // past K / G and rows past N zero-filled)
-                    mbar_arrive_expect_tx(full(slot), (uint32_t)ROWS * (rowb + (sring ? 2u * (uint32_t)sbw : 0u)));
+                    // one tensor copy each: the stage's packed rows (ROWS x pitch
+                    // bytes), scale tile and bias tile (ROWS x sbw bytes); rows
+                    // past N and columns past the row end are zero-filled and
+                    // count in full
+                    mbar_arrive_expect_tx(full(slot), (uint32_t)ROWS * ((uint32_t)pitch + (sring ? 2u * (uint32_t)sbw : 0u)));
+                    tensor_copy_3d(st0, &p.wmap, (ks * S * 4 * UB) / 8, rb * ROWS, bz, full(slot));
                     if (sring) {
                         const int g0 = ((ks * S) << gmul) >> gdiv;
                         tensor_copy_3d(st0 + (uint32_t)p.soff, &p.smap, g0, rb * ROWS, bz, full(slot));
@@ -219,11 +211,6 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
                     }
                 }
                 __syncwarp();
-                for (int r = lane; r < ROWS; r += 32) {
-                    const int row = min(rb * ROWS + r, p.N - 1);
-                    bulk_copy_g2s(st0 + (uint32_t)(r * pitch), W + (long long)row * p.w_row + (long long)ks * S * 4 * UB,
-                                  rowb, full(slot));
-                }
                 ++it;
             }
         }
