@@ -143,17 +143,18 @@ def test_python_binding_raises():
 def test_plan_no_n_cliff():
     """Any N gets a plan (no N % 8 generic fallback): N <= 64 the latency
     kernel, larger N the row-tiled kernels, whatever N % 8 is."""
-    for n in (1, 3, 5, 7, 8, 9, 12, 17, 64):
+    for n in (1, 3, 5, 7, 8, 9, 12, 17, 64, 65, 512):
         s = q.qmv_describe_plan("affine", 1, n, 2560, bits=8, group_size=64)
         assert "path=direct" in s, (n, s)
-    for n in (65, 4095, 4096, 4097):
+    for n in (513, 4095, 4096, 4097):
         s = q.qmv_describe_plan("affine", 1, n, 2560, bits=8, group_size=64)
         assert "path=wide" in s, (n, s)
     # few output rows: the latency kernel, for every format
     assert "path=direct" in q.qmv_describe_plan("affine", 1, 64, 96, bits=3, group_size=32)
     assert "path=direct" in q.qmv_describe_plan("affine", 1, 64, 4096, bits=4, group_size=32, w_align16=False)
     assert "path=direct" in q.qmv_describe_plan("mxfp4", 2, 12, 4096)
-    assert "path=direct" not in q.qmv_describe_plan("affine", 1, 65, 4096, bits=4, group_size=64)
+    assert "path=direct" not in q.qmv_describe_plan("affine", 1, 513, 4096, bits=4, group_size=64)
+    assert "path=direct" not in q.qmv_describe_plan("affine", 3, 65, 4096, bits=4, group_size=64)
     # 3-bit tensor-core units are 12 bytes: 4-byte alignment is enough
     assert "path=tc" in q.qmv_describe_plan("affine", 4, 100, 4096, bits=3, group_size=32, w_align16=False)
 

@@ -211,7 +211,9 @@ bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s
         // one or two x rows over many rows, or x too large to stay staged
         // across row blocks: 128-row blocks, K not split, as few row blocks
         // per block as possible (5-bit: 64 rows, K over 2 warps)
-        wr = bits == 5 ? 4 : 8;
+        // (one scale group per super-block, ngs = 1: only SPB slot columns of 8
+        // are live, so 64-row blocks with K over 2 warps measured faster too)
+        wr = (bits == 5 || ngs == 1) ? 4 : 8;
         wk = 8 / wr;
     } else {
         wr = 2;
@@ -305,7 +307,9 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
 
     // ---- few output rows: the latency kernel (weights dequantized before the
     // grid-dependency wait, one block per row) --------------------------------
-    if (K > 0 && (g_forced.path == 5 || (g_forced.path < 0 && N <= 64))) {
+    // (N <= 64 any M; up to 512 rows for one or two x rows: measured faster
+    // than the row-tiled kernels on B200 up to about 1.3 MB of weights)
+    if (K > 0 && (g_forced.path == 5 || (g_forced.path < 0 && (N <= 64 || (N <= 512 && M <= 2))))) {
         const int units = K / 32;
         int thr = ((units + 31) / 32) * 32;
         if (thr > 256) thr = 256;
