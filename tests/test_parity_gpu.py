@@ -441,7 +441,8 @@ def test_bulk_ring_path_grid(q, ring, bits, group, dtype, M):
 
 
 @pytest.mark.parametrize("cfg", [(4, -1, 1, 1), (4, -1, 8, 1), (4, -1, 1, 8), (4, -1, 2, 4), (4, -1, 4, 2),
-                                 (4, -1, 3, 2), (4, -1, 6, 2), (4, -1, 4, 3), (4, -1, 12, 1), (4, -1, 3, 4)])
+                                 (4, -1, 3, 2), (4, -1, 6, 2), (4, -1, 4, 3), (4, -1, 12, 1), (4, -1, 3, 4),
+                                 (4, -1, 2, 8), (4, -1, 4, 4), (4, -1, 16, 1)])
 @pytest.mark.parametrize("bits", [2, 3, 5, 8])
 def test_bulk_ring_block_shapes(q, ring, cfg, bits):
     q.qmv_force_config(*cfg)
@@ -511,6 +512,100 @@ def test_bulk_ring_x_tiles(q, ring, N):
     rows = list(range(N)) if N <= 80 else sorted(set(sample_rows(N, 48)) | {N - 1})
     ref, ad = oracle_affine(c, rows=rows)
     compare(y[:, rows], ref[:, rows], ad[:, rows], "f32", what="tcb tiles")
+
+
+# ------------------------------- CUDA cores + weight ring, one bf16 x row ----
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("group", GROUPS)
+@pytest.mark.parametrize("K", [1024, 5760])
+def test_fma_ring_path_grid(q, ring, bits, group, K):
+    """The CUDA-core ring kernel on every width and group (2-bit with group 32
+    falls back: a 64-code unit would span two groups); K = 5760 leaves an odd
+    number of super-blocks for most widths (a half-empty last step)."""
+    q.qmv_force_config(6, -1, -1, -1)
+    N = 100
+    sb = 512 // bits if bits in (2, 4, 8) else 128       # codes per super-block
+    if K % sb != 0:
+        pytest.skip("K not a whole number of super-blocks")
+    plan = q.qmv_describe_plan("affine", 1, N, K, bits, group, "bf16")
+    assert ("path=tcf" in plan) == (not (bits == 2 and group == 32)), plan
+    c = synth.affine_case(1, N, K, bits, group, "bf16", seed=_seed("tcf", bits, group, K))
+    y = run_affine(q, c)[0]
+    ref, ad = oracle_affine(c)
+    compare(y, ref, ad, "bf16", what=f"tcf b{bits} g{group} K{K}")
+
+
+@pytest.mark.parametrize("cfg", [(6, -1, 1, 8), (6, -1, 2, 4), (6, -1, 4, 2), (6, -1, 8, 1), (6, -1, 1, 12),
+                                 (6, -1, 3, 4), (6, -1, 6, 2), (6, -1, 12, 1), (6, -1, 2, 8), (6, -1, 4, 4),
+                                 (6, -1, 16, 1), (6, -1, 1, 16)])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+def test_fma_ring_block_shapes(q, ring, cfg, bits):
+    unit_bytes = 16 if bits in (2, 4, 8) else 4 * bits
+    if 2 * cfg[2] * 4 * unit_bytes > 2048:
+        pytest.skip("a stage of 2 * wk super-blocks exceeds one tensor-copy box (256 x 8 bytes)")
+    q.qmv_force_config(*cfg)
+    c = synth.affine_case(1, 333, 2048, bits, 64, "bf16", seed=_seed("tcfshape", cfg, bits), batch=2)
+    assert "path=tcf" in q.qmv_describe_plan("affine", 1, 333, 2048, bits, 64, "bf16")
+    y = run_affine(q, c)
+    for b in range(2):
+        ref, ad = oracle_affine(c, b=b)
+        compare(y[b], ref, ad, "bf16", what=f"tcf shape {cfg} b{bits} batch{b}")
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_fma_ring_persistent_row_blocks(q, ring, bits):
+    """More row blocks than SMs, a ragged last stage and a ragged last row block."""
+    q.qmv_force_config(6, -1, 8, 1)
+    N, K = 16 * 148 * 2 + 37, 5760
+    c = synth.affine_case(1, N, K, bits, 64, "bf16", seed=_seed("tcfpers", bits))
+    plan = q.qmv_describe_plan("affine", 1, N, K, bits, 64, "bf16")
+    assert "path=tcf" in plan and "grid=148 " in plan, plan
+    y = run_affine(q, c)[0]
+    rows = sorted(set(sample_rows(N, 96)) | {0, 15, 16, N - 38, N - 37, N - 1})
+    ref, ad = oracle_affine(c, rows=rows)
+    compare(y[:, rows], ref[:, rows], ad[:, rows], "bf16", what=f"tcf persistent b{bits}")
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_fma_ring_tail_rows_bitwise_prefix(q, ring, bits):
+    q.qmv_force_config(6, -1, 4, 2)
+    K = 2560
+    big = synth.affine_case(1, 48, K, bits, 64, "bf16", seed=_seed("tcftail", bits))
+    yb = run_affine(q, big)[0]
+    for n in (1, 5, 17, 33):
+        small = dict(big, N=n, w=big["w"][:, :n].copy(), scales=big["scales"][:, :n].copy(),
+                     biases=big["biases"][:, :n].copy())
+        assert np.array_equal(run_affine(q, small)[0], yb[:, :n])
+
+
+@pytest.mark.parametrize("bits,group", [(4, 64), (4, 32), (3, 128), (8, 128), (5, 64), (2, 128)])
+def test_fma_ring_scales_in_or_out_of_ring(q, ring, bits, group):
+    q.qmv_force_config(6, -1, 4, 2)
+    N, K = 300, 4096
+    plan = q.qmv_describe_plan("affine", 1, N, K, bits, group, "bf16")
+    assert "path=tcf" in plan and "scale_ring=1" in plan, plan
+    c = synth.affine_case(1, N, K, bits, group, "bf16", seed=_seed("tcfscale", bits, group), batch=2)
+    y_in = run_affine(q, c)
+    y_out = run_affine(q, c, s_offset=2)
+    assert np.array_equal(y_in, y_out)
+    for b in range(2):
+        ref, ad = oracle_affine(c, b=b)
+        compare(y_in[b], ref, ad, "bf16", what=f"tcf scales b{bits} g{group} batch{b}")
+
+
+@pytest.mark.parametrize("N", [80, 16 * 148 + 5])
+def test_fma_ring_x_tiles(q, ring, N):
+    """K large enough that x is staged in several K tiles (and again for every
+    row block when there are more row blocks than SMs)."""
+    q.qmv_force_config(6, -1, 8, 1)
+    K = 65536
+    plan = q.qmv_describe_plan("affine", 1, N, K, 4, 64, "bf16")
+    assert "path=tcf" in plan and "tile_iters=512" not in plan, plan
+    c = synth.affine_case(1, N, K, 4, 64, "bf16", seed=_seed("tcftile", N))
+    y = run_affine(q, c)[0]
+    rows = list(range(N)) if N <= 80 else sorted(set(sample_rows(N, 48)) | {N - 1})
+    ref, ad = oracle_affine(c, rows=rows)
+    compare(y[:, rows], ref[:, rows], ad[:, rows], "bf16", what="tcf tiles")
 
 
 # ----------------------------------------- few rows: the latency kernel ----

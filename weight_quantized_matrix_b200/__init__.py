@@ -32,15 +32,20 @@ STATUS = {0: "QMV_OK", -1: "QMV_EINVAL", -2: "QMV_EUNSUPPORTED", -3: "QMV_EALIGN
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"libqmv.so not found at {LIB_PATH}; build it with "
-        "`python -m weight_quantized_matrix_b200.build_lib` (needs nvcc)")
+        "`python weight_quantized_matrix_b200/build_lib.py` (needs nvcc)")
 
-_lib = ctypes.CDLL(LIB_PATH)
+try:
+    _lib = ctypes.CDLL(LIB_PATH)
+except OSError as _e:
+    raise ImportError(
+        f"libqmv.so at {LIB_PATH} does not load ({_e}); rebuild it with "
+        "`python weight_quantized_matrix_b200/build_lib.py --force`") from _e
 try:
     from . import _qmv_fast as _fast      # per-call entry points (CPython extension over libqmv.so)
 except ImportError as _e:
     raise ImportError(
         "the _qmv_fast extension is missing; build it with "
-        "`python -m weight_quantized_matrix_b200.build_lib` (needs gcc)") from _e
+        "`python weight_quantized_matrix_b200/build_lib.py` (needs gcc)") from _e
 _p, _i, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong
 _lib.qmv_affine.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
 _lib.qmv_affine_batched.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _p]

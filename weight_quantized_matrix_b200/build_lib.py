@@ -1,6 +1,8 @@
 """Build libqmv.so in-tree for sm_100a (B200).
 
-    python -m weight_quantized_matrix_b200.build_lib [--force]
+    python weight_quantized_matrix_b200/build_lib.py [--force]
+
+(run as a file: importing the package needs the library this builds)
 
 Each kernel family compiles in its own nvcc process (in parallel); the objects
 are linked into ``weight_quantized_matrix_b200/lib/libqmv.so`` with the CUDA

@@ -225,11 +225,20 @@ bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s
         }
         wk = 12 / wr;
     }
-    if (g_forced.wr > 0) wr = g_forced.wr > 12 ? 12 : g_forced.wr;
-    if (g_forced.wk > 0) wk = g_forced.wk > 12 ? 12 : g_forced.wk;
-    while (wk * wr > 12) --wk;
+    if (g_forced.wr > 0) wr = g_forced.wr > 16 ? 16 : g_forced.wr;
+    if (g_forced.wk > 0) wk = g_forced.wk > 16 ? 16 : g_forced.wk;
     if (wk > nsbk) wk = nsbk;
     if (wk < 1) wk = 1;
+    // a block is 8, 12 or 16 warps (16 only while npass <= 2): otherwise the
+    // largest wk <= the chosen one that divides such a count, and its wr
+    auto valid_ncw = [&](int n) { return n == 8 || n == 12 || (n == 16 && npass <= 2); };
+    if (!valid_ncw(wk * wr)) {
+        int bk = 0, bw = 0;
+        for (int k = wk; k >= 1 && bk == 0; --k)
+            for (int n = 8; n <= 16 && bk == 0; n += 4)
+                if (valid_ncw(n) && n % k == 0) { bk = k; bw = n / k; }
+        wk = bk; wr = bw;
+    }
     const int rows = 16 * wr;
     // stage size: a multiple of one batch of every k-warp (SPB * wk super-blocks)
     // and of the super-blocks one group spans (G / SB when G > SB)
@@ -295,6 +304,92 @@ bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s
     return ts->smem <= (size_t)qmv::kMaxSmem;
 }
 
+// ---- CUDA-core ring launch shape (one bf16 x row, qmv_tcf.cuh) ---------------
+// Same ring and stage layout as the tensor-core ring; a warp takes two
+// super-blocks per step, so a stage is a multiple of 2 * wk super-blocks.  The
+// x tile holds (NP + 4) words of x~ pairs and two sums per unit.
+bool tcf_shape(int N, int K, int bits, int G, bool w16, bool s16, TcbShape* ts) {
+    const int ub = tc_unit_bytes(bits);
+    const int uc = ub * 8 / bits;
+    const int SB = 4 * uc;
+    if (K % SB != 0 || !w16) return false;
+    if (((long long)K * bits / 8) % 16 != 0) return false;     // tensor copies: 16-byte rows
+    if (G < uc) return false;                                   // a unit lies in one group
+    const int es = 2;
+    const int nps = tc_np_of(bits) + 4;
+    const int nsbk = K / SB;
+    const int sms = device_sms();
+    // Block shape (measured on B200): the fewest rows on the busiest SM
+    // (rounds of row blocks over the SMs x rows per block), with at least 4
+    // steps of 2 super-blocks per warp and row block; ties go to 16 warps, then
+    // to fewer row blocks.  Units that are not 16 bytes (3/5/6-bit codes)
+    // split K over at most 2 warps.
+    const int steps = (nsbk + 1) / 2;
+    int wr = 8, wk = 1;
+    {
+        static const int cand[9][2] = {{16, 1}, {8, 2}, {4, 4}, {2, 8}, {1, 16}, {8, 1}, {4, 2}, {2, 4}, {1, 8}};
+        long long best = -1;
+        for (const auto& c : cand) {
+            const int k = c[0], r = c[1];
+            if (k > 1 && steps < 4 * k) continue;
+            if (ub != 16 && k > 2) continue;
+            const long long nrb_c = ((long long)N + 16 * r - 1) / (16 * r);
+            const long long cost = ((nrb_c + sms - 1) / sms) * 16 * r;
+            if (best < 0 || cost < best) { best = cost; wk = k; wr = r; }
+        }
+    }
+    if (g_forced.wr > 0) wr = g_forced.wr > 16 ? 16 : g_forced.wr;
+    if (g_forced.wk > 0) wk = g_forced.wk > 16 ? 16 : g_forced.wk;
+    const int ncw = wk * wr;
+    if (ncw != 8 && ncw != 12 && ncw != 16) return false;
+    const int rows = 16 * wr;
+    const int gq = G > SB ? G / SB : 1;
+    int quantum = 2 * wk;
+    while (quantum % gq) quantum *= 2;
+    int sps = 32768 / (rows * 4 * ub);
+    sps = sps / quantum * quantum;
+    if (sps < quantum) sps = quantum;
+    if (sps > nsbk) sps = (nsbk + quantum - 1) / quantum * quantum;
+    if (s16 && ((long long)(K / G) * es) % 16 == 0) {
+        auto sb_bytes = [&](int v) { return (G <= SB ? v * (SB / G) : v / (G / SB)) * es; };
+        int v = sps;
+        while (v < 4 * sps && v < nsbk && sb_bytes(v) % 16 != 0) v += quantum;
+        if (sb_bytes(v) % 16 == 0 && v * 4 * ub / 8 <= 256) sps = v;
+    }
+    while (sps > quantum && sps * 4 * ub / 8 > 256) sps -= quantum;
+    if (sps * 4 * ub / 8 > 256) return false;
+    auto layout = [&](int s, int* sring, int* sbw, int* stage) {
+        const int box0 = G <= SB ? s * (SB / G) : s / (G / SB);
+        *sbw = box0 * es;
+        *sring = (s16 && ((long long)(K / G) * es) % 16 == 0 && *sbw % 16 == 0 && box0 <= 256 && rows <= 256) ? 1 : 0;
+        const int pitch = s * 4 * ub;
+        *stage = rows * pitch + (*sring ? 2 * rows * *sbw : 0);
+        return pitch;
+    };
+    const size_t red = (size_t)(qmv::kTcbStages + 1) * ncw * 16 * 4;
+    const size_t per_sb = (size_t)4 * (nps * 4 + 8);
+    long long tsb = 0;
+    int sring = 0, sbw = 0, stage = 0, pitch = 0;
+    for (;;) {
+        pitch = layout(sps, &sring, &sbw, &stage);
+        const size_t fixed = 256 + (size_t)qmv::kTcbStages * stage + red;
+        tsb = fixed < (size_t)qmv::kMaxSmem ? (long long)(((size_t)qmv::kMaxSmem - fixed) / per_sb) : 0;
+        if (tsb >= nsbk) { tsb = nsbk; break; }
+        tsb = tsb / sps * sps;
+        if (tsb >= sps) break;
+        if (sps <= quantum) return false;
+        sps = (sps / 2) / quantum * quantum;
+        if (sps < quantum) sps = quantum;
+    }
+    const long long nrb = ((long long)N + rows - 1) / rows;
+    ts->npass = 0; ts->spb = 1; ts->wk = wk; ts->wr = wr; ts->tsb = (int)tsb; ts->sps = sps;
+    ts->pitch = pitch; ts->sring = sring; ts->sbw = sbw;
+    ts->soff = rows * pitch; ts->boff = rows * pitch + rows * sbw;
+    ts->gx = nrb < sms ? nrb : sms;
+    ts->smem = 256 + (size_t)qmv::kTcbStages * stage + (size_t)tsb * per_sb + red;
+    return ts->smem <= (size_t)qmv::kMaxSmem;
+}
+
 // Choose the launch shape.  Returns QMV_OK or an error (sizes too large).
 int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, bool w16, int batch, Plan* pl,
               bool s16 = true) {
@@ -323,6 +418,25 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
         return QMV_OK;
     }
 
+    // ---- one bf16 x row: CUDA cores with the weight ring ----------------------
+    // (measured on B200: the fastest path for one bf16 x row from about 16 MB
+    // of 2/3/4/5-bit weights; 6-bit codes do not pair and 8-bit codes take two
+    // fields each, where the register-streaming CUDA-core kernel wins)
+    const bool fma_ring_pick = M == 1 && dtype == QMV_BF16 && bits >= 2 && bits <= 5 &&
+                               (double)N * K * bits / 8.0 >= 16.0 * 1024 * 1024;
+    if (aff && K > 0 && M == 1 && dtype == QMV_BF16 && (g_forced.path == 6 || (g_forced.path < 0 && fma_ring_pick))) {
+        TcbShape ts;
+        if (tcf_shape(N, K, bits, G_of_plan, w16, s16, &ts)) {
+            pl->maxm = 1; pl->R = 1; pl->wide = 1; pl->tc = 4; pl->npass = 0;
+            pl->wk = ts.wk; pl->wr = ts.wr; pl->tile_iters = ts.tsb; pl->sps = ts.sps; pl->pitch = ts.pitch;
+            pl->spb = 1; pl->sring = ts.sring; pl->soff = ts.soff; pl->boff = ts.boff; pl->sbw = ts.sbw;
+            pl->C = 4 * tc_unit_bytes(bits) * 8 / bits; pl->smem = ts.smem;
+            pl->grid = dim3((unsigned)ts.gx, 1, (unsigned)batch);
+            pl->block = dim3(32 * ts.wk * ts.wr, 1, 1);
+            return QMV_OK;
+        }
+    }
+
     // ---- tensor-core kernel with the bulk-copy weight ring --------------------
     // (measured on B200: the fastest path once M >= 2, and for large 2/3/4/5-bit
     // matrices at M = 1)
@@ -336,7 +450,7 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
             pl->spb = ts.spb; pl->sring = ts.sring; pl->soff = ts.soff; pl->boff = ts.boff; pl->sbw = ts.sbw;
             pl->C = 4 * tc_unit_bytes(bits) * 8 / bits; pl->smem = ts.smem;
             pl->grid = dim3((unsigned)ts.gx, 1, (unsigned)batch);
-            pl->block = dim3(32 * (ts.wk * ts.wr + 1), 1, 1);
+            pl->block = dim3(32 * ts.wk * ts.wr, 1, 1);
             return QMV_OK;
         }
     }
@@ -507,7 +621,8 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     int st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, s16);
     if (st != QMV_OK) return st;
     qmv::Params p;
-    if (pl.tc == 2 && pl.sring) {
+    const bool ring = pl.tc == 2 || pl.tc == 4;        // the weight-ring kernels
+    if (ring && pl.sring) {
         const int box0 = pl.sbw / elem_bytes(dtype), rows = 16 * pl.wr;
         if (!encode_scale_map(&p.smap, scales, dtype, K / G, N, batch, box0, rows) ||
             !encode_scale_map(&p.bmap, biases, dtype, K / G, N, batch, box0, rows)) {
@@ -517,7 +632,7 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
         }
     }
     // the packed rows' tensor map, for the final plan
-    if (pl.tc == 2 && !encode_rows_map(&p.wmap, w, row_bytes, N, batch, pl.pitch / 8, 16 * pl.wr)) {
+    if (ring && !encode_rows_map(&p.wmap, w, row_bytes, N, batch, pl.pitch / 8, 16 * pl.wr)) {
         cudaGetLastError();
         return QMV_ECUDA;
     }
@@ -541,7 +656,12 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     if (pl.tc == 2) {
         p.fault = fault_word();
         if (!p.fault) return QMV_ECUDA;
-        return finish(qmv::launch_tcb_affine(bits, dtype, pl.npass, pl.spb, pl.wk * pl.wr > 8, p, L));
+        return finish(qmv::launch_tcb_affine(bits, dtype, pl.npass, pl.spb, pl.wk * pl.wr, p, L));
+    }
+    if (pl.tc == 4) {
+        p.fault = fault_word();
+        if (!p.fault) return QMV_ECUDA;
+        return finish(qmv::launch_tcf_affine(bits, pl.wk * pl.wr, p, L));
     }
     if (pl.tc == 3) return finish(qmv::launch_direct(fam, bits, dtype, pl.maxm, pl.wide != 0, p, L));
     if (pl.tc) return finish(qmv::launch_tc_affine(bits, dtype, pl.npass, p, L));
@@ -695,7 +815,7 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
     snprintf(buf, (size_t)buflen,
              "path=%s chunk=%d maxm=%d rows_per_warp=%d warps_k=%d warps_rows=%d tile_iters=%d "
              "grid=%u block=%u smem=%zu stage_sb=%d batch_sb=%d scale_ring=%d",
-             pl.tc == 3 ? "direct" : pl.tc == 2 ? "tcb" : pl.tc ? "tc" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr,
+             pl.tc == 4 ? "tcf" : pl.tc == 3 ? "direct" : pl.tc == 2 ? "tcb" : pl.tc ? "tc" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr,
              pl.tile_iters, pl.grid.x, pl.block.x, pl.smem, pl.sps, pl.spb, pl.sring);
     return QMV_OK;
 }

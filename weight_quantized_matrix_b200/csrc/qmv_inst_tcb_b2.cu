@@ -4,7 +4,7 @@
 
 namespace qmv {
 
-cudaError_t launch_tcb_affine_b2(int dtype, int npass, int spb, bool w12, const Params& p, const Launch& L) {
+cudaError_t launch_tcb_affine_b2(int dtype, int npass, int spb, int ncw, const Params& p, const Launch& L) {
 #define BITS_ 2
     QMV_TCB_DISPATCH_DTYPE()
 #undef BITS_

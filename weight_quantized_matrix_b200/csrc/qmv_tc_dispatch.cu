@@ -10,12 +10,12 @@ cudaError_t launch_tc_affine_b5(int, int, const Params&, const Launch&);
 cudaError_t launch_tc_affine_b6(int, int, const Params&, const Launch&);
 cudaError_t launch_tc_affine_b8(int, int, const Params&, const Launch&);
 
-cudaError_t launch_tcb_affine_b2(int, int, int, bool, const Params&, const Launch&);
-cudaError_t launch_tcb_affine_b3(int, int, int, bool, const Params&, const Launch&);
-cudaError_t launch_tcb_affine_b4(int, int, int, bool, const Params&, const Launch&);
-cudaError_t launch_tcb_affine_b5(int, int, int, bool, const Params&, const Launch&);
-cudaError_t launch_tcb_affine_b6(int, int, int, bool, const Params&, const Launch&);
-cudaError_t launch_tcb_affine_b8(int, int, int, bool, const Params&, const Launch&);
+cudaError_t launch_tcb_affine_b2(int, int, int, int, const Params&, const Launch&);
+cudaError_t launch_tcb_affine_b3(int, int, int, int, const Params&, const Launch&);
+cudaError_t launch_tcb_affine_b4(int, int, int, int, const Params&, const Launch&);
+cudaError_t launch_tcb_affine_b5(int, int, int, int, const Params&, const Launch&);
+cudaError_t launch_tcb_affine_b6(int, int, int, int, const Params&, const Launch&);
+cudaError_t launch_tcb_affine_b8(int, int, int, int, const Params&, const Launch&);
 
 cudaError_t launch_tc_affine(int bits, int dtype, int npass, const Params& p, const Launch& L) {
     switch (bits) {
@@ -29,14 +29,14 @@ cudaError_t launch_tc_affine(int bits, int dtype, int npass, const Params& p, co
     }
 }
 
-cudaError_t launch_tcb_affine(int bits, int dtype, int npass, int spb, bool w12, const Params& p, const Launch& L) {
+cudaError_t launch_tcb_affine(int bits, int dtype, int npass, int spb, int ncw, const Params& p, const Launch& L) {
     switch (bits) {
-        case 2: return launch_tcb_affine_b2(dtype, npass, spb, w12, p, L);
-        case 3: return launch_tcb_affine_b3(dtype, npass, spb, w12, p, L);
-        case 4: return launch_tcb_affine_b4(dtype, npass, spb, w12, p, L);
-        case 5: return launch_tcb_affine_b5(dtype, npass, spb, w12, p, L);
-        case 6: return launch_tcb_affine_b6(dtype, npass, spb, w12, p, L);
-        case 8: return launch_tcb_affine_b8(dtype, npass, spb, w12, p, L);
+        case 2: return launch_tcb_affine_b2(dtype, npass, spb, ncw, p, L);
+        case 3: return launch_tcb_affine_b3(dtype, npass, spb, ncw, p, L);
+        case 4: return launch_tcb_affine_b4(dtype, npass, spb, ncw, p, L);
+        case 5: return launch_tcb_affine_b5(dtype, npass, spb, ncw, p, L);
+        case 6: return launch_tcb_affine_b6(dtype, npass, spb, ncw, p, L);
+        case 8: return launch_tcb_affine_b8(dtype, npass, spb, ncw, p, L);
         default: return cudaErrorInvalidValue;
     }
 }
