@@ -156,9 +156,9 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
  * qmv_device_fault -- the fault word of the current device.  Kernels that
  * stream weights through a shared-memory ring wait on barriers with a bound
  * (about one second); a wait that expires ORs a nonzero code into this word
- * (1: a warp gave up waiting for a ring stage to arrive, 4: a block gave up
- * waiting, at exit, for the copies it issued) and the call that hit it leaves
- * y undefined.  Writes the word to *code and, if clear != 0,
+ * (1: a consumer warp gave up on a ring stage, 2: the producer warp gave up on
+ * a free stage, 4: the producer gave up waiting for its own copies) and the
+ * call that hit it leaves y undefined.  Writes the word to *code and, if clear != 0,
  * resets it to zero.  Synchronous: it waits for the device's pending work
  * (cudaMemcpyFromSymbol).  Returns QMV_OK, QMV_EINVAL (code NULL) or QMV_ECUDA.
  */
@@ -173,8 +173,9 @@ int qmv_device_fault(unsigned int* code, int clear);
  * hold), 1 = CUDA-core kernel with wide (16-byte) chunk loads, 0 = CUDA-core
  * kernel with 4-byte chunks, -1 = automatic; rows_per_warp in {1,2,4} or -1
  * (CUDA-core kernel); warps_k (warps that split K inside a block) and
- * warps_rows (16-row tiles per block) up to 16 each, or -1; the weight-ring
- * kernels run blocks of warps_k * warps_rows in {8, 12, 16} warps.
+ * warps_rows (16-row tiles per block) up to 12 each, or -1; the weight-ring
+ * kernels run warps_k * warps_rows in {8, 12} compute warps and a producer
+ * warp.
  * Unsupported combinations fall back to automatic for that field.  Not
  * thread-safe with concurrent calls; meant for single-threaded harnesses.
  */

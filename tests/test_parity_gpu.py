@@ -441,8 +441,7 @@ def test_bulk_ring_path_grid(q, ring, bits, group, dtype, M):
 
 
 @pytest.mark.parametrize("cfg", [(4, -1, 1, 1), (4, -1, 8, 1), (4, -1, 1, 8), (4, -1, 2, 4), (4, -1, 4, 2),
-                                 (4, -1, 3, 2), (4, -1, 6, 2), (4, -1, 4, 3), (4, -1, 12, 1), (4, -1, 3, 4),
-                                 (4, -1, 2, 8), (4, -1, 4, 4), (4, -1, 16, 1)])
+                                 (4, -1, 3, 2), (4, -1, 6, 2), (4, -1, 4, 3), (4, -1, 12, 1), (4, -1, 3, 4)])
 @pytest.mark.parametrize("bits", [2, 3, 5, 8])
 def test_bulk_ring_block_shapes(q, ring, cfg, bits):
     q.qmv_force_config(*cfg)
@@ -536,8 +535,7 @@ def test_fma_ring_path_grid(q, ring, bits, group, K):
 
 
 @pytest.mark.parametrize("cfg", [(6, -1, 1, 8), (6, -1, 2, 4), (6, -1, 4, 2), (6, -1, 8, 1), (6, -1, 1, 12),
-                                 (6, -1, 3, 4), (6, -1, 6, 2), (6, -1, 12, 1), (6, -1, 2, 8), (6, -1, 4, 4),
-                                 (6, -1, 16, 1), (6, -1, 1, 16)])
+                                 (6, -1, 3, 4), (6, -1, 6, 2), (6, -1, 12, 1), (6, -1, 2, 6), (6, -1, 4, 3)])
 @pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
 def test_fma_ring_block_shapes(q, ring, cfg, bits):
     unit_bytes = 16 if bits in (2, 4, 8) else 4 * bits

@@ -225,17 +225,17 @@ bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s
         }
         wk = 12 / wr;
     }
-    if (g_forced.wr > 0) wr = g_forced.wr > 16 ? 16 : g_forced.wr;
-    if (g_forced.wk > 0) wk = g_forced.wk > 16 ? 16 : g_forced.wk;
+    if (g_forced.wr > 0) wr = g_forced.wr > 12 ? 12 : g_forced.wr;
+    if (g_forced.wk > 0) wk = g_forced.wk > 12 ? 12 : g_forced.wk;
     if (wk > nsbk) wk = nsbk;
     if (wk < 1) wk = 1;
-    // a block is 8, 12 or 16 warps (16 only while npass <= 2): otherwise the
-    // largest wk <= the chosen one that divides such a count, and its wr
-    auto valid_ncw = [&](int n) { return n == 8 || n == 12 || (n == 16 && npass <= 2); };
+    // a block is 8 or 12 consumer warps: otherwise the largest wk <= the
+    // chosen one that divides such a count, and its wr
+    auto valid_ncw = [&](int n) { return n == 8 || n == 12; };
     if (!valid_ncw(wk * wr)) {
         int bk = 0, bw = 0;
         for (int k = wk; k >= 1 && bk == 0; --k)
-            for (int n = 8; n <= 16 && bk == 0; n += 4)
+            for (int n = 8; n <= 12 && bk == 0; n += 4)
                 if (valid_ncw(n) && n % k == 0) { bk = k; bw = n / k; }
         wk = bk; wr = bw;
     }
@@ -321,27 +321,27 @@ bool tcf_shape(int N, int K, int bits, int G, bool w16, bool s16, TcbShape* ts) 
     const int sms = device_sms();
     // Block shape (measured on B200): the fewest rows on the busiest SM
     // (rounds of row blocks over the SMs x rows per block), with at least 4
-    // steps of 2 super-blocks per warp and row block; ties go to 16 warps, then
-    // to fewer row blocks.  Units that are not 16 bytes (3/5/6-bit codes)
-    // split K over at most 2 warps.
+    // steps of 2 super-blocks per warp and row block; ties go to 8 compute
+    // warps, then to fewer row blocks.
     const int steps = (nsbk + 1) / 2;
     int wr = 8, wk = 1;
     {
-        static const int cand[9][2] = {{16, 1}, {8, 2}, {4, 4}, {2, 8}, {1, 16}, {8, 1}, {4, 2}, {2, 4}, {1, 8}};
+        static const int cand[10][2] = {{8, 1}, {4, 2}, {2, 4}, {1, 8},
+                                        {12, 1}, {6, 2}, {4, 3}, {3, 4}, {2, 6}, {1, 12}};
         long long best = -1;
         for (const auto& c : cand) {
             const int k = c[0], r = c[1];
             if (k > 1 && steps < 4 * k) continue;
-            if (ub != 16 && k > 2) continue;
             const long long nrb_c = ((long long)N + 16 * r - 1) / (16 * r);
             const long long cost = ((nrb_c + sms - 1) / sms) * 16 * r;
-            if (best < 0 || cost < best) { best = cost; wk = k; wr = r; }
+            const bool same_warps = (k * r) == (wk * wr);
+            if (best < 0 || cost < best || (cost == best && same_warps && r > wr)) { best = cost; wk = k; wr = r; }
         }
     }
-    if (g_forced.wr > 0) wr = g_forced.wr > 16 ? 16 : g_forced.wr;
-    if (g_forced.wk > 0) wk = g_forced.wk > 16 ? 16 : g_forced.wk;
+    if (g_forced.wr > 0) wr = g_forced.wr > 12 ? 12 : g_forced.wr;
+    if (g_forced.wk > 0) wk = g_forced.wk > 12 ? 12 : g_forced.wk;
     const int ncw = wk * wr;
-    if (ncw != 8 && ncw != 12 && ncw != 16) return false;
+    if (ncw != 8 && ncw != 12) return false;
     const int rows = 16 * wr;
     const int gq = G > SB ? G / SB : 1;
     int quantum = 2 * wk;
@@ -419,11 +419,11 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     }
 
     // ---- one bf16 x row: CUDA cores with the weight ring ----------------------
-    // (measured on B200: the fastest path for one bf16 x row from about 16 MB
-    // of 2/3/4/5-bit weights; 6-bit codes do not pair and 8-bit codes take two
-    // fields each, where the register-streaming CUDA-core kernel wins)
-    const bool fma_ring_pick = M == 1 && dtype == QMV_BF16 && bits >= 2 && bits <= 5 &&
-                               (double)N * K * bits / 8.0 >= 16.0 * 1024 * 1024;
+    // (measured on B200: the fastest path for one bf16 x row from about 10 MB
+    // of 2/3/4/5/6-bit weights; 8-bit codes take two fields each, and there
+    // the register-streaming CUDA-core kernel is as fast)
+    const bool fma_ring_pick = M == 1 && dtype == QMV_BF16 && bits >= 2 && bits <= 6 &&
+                               (double)N * K * bits / 8.0 >= 10.0 * 1024 * 1024;
     if (aff && K > 0 && M == 1 && dtype == QMV_BF16 && (g_forced.path == 6 || (g_forced.path < 0 && fma_ring_pick))) {
         TcbShape ts;
         if (tcf_shape(N, K, bits, G_of_plan, w16, s16, &ts)) {
@@ -432,7 +432,7 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
             pl->spb = 1; pl->sring = ts.sring; pl->soff = ts.soff; pl->boff = ts.boff; pl->sbw = ts.sbw;
             pl->C = 4 * tc_unit_bytes(bits) * 8 / bits; pl->smem = ts.smem;
             pl->grid = dim3((unsigned)ts.gx, 1, (unsigned)batch);
-            pl->block = dim3(32 * ts.wk * ts.wr, 1, 1);
+            pl->block = dim3(32 * (ts.wk * ts.wr + 1), 1, 1);
             return QMV_OK;
         }
     }
@@ -450,7 +450,7 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
             pl->spb = ts.spb; pl->sring = ts.sring; pl->soff = ts.soff; pl->boff = ts.boff; pl->sbw = ts.sbw;
             pl->C = 4 * tc_unit_bytes(bits) * 8 / bits; pl->smem = ts.smem;
             pl->grid = dim3((unsigned)ts.gx, 1, (unsigned)batch);
-            pl->block = dim3(32 * ts.wk * ts.wr, 1, 1);
+            pl->block = dim3(32 * (ts.wk * ts.wr + 1), 1, 1);       // + the producer warp
             return QMV_OK;
         }
     }

@@ -1,5 +1,5 @@
 // qmv_inst_tcf.cu -- CUDA-core affine qmv kernels with the weight ring, one
-// bf16 x row (every code width; 8, 12 or 16 warps per block).
+// bf16 x row (every code width; 8 or 12 compute warps and a producer warp).
 #include "qmv_launch.cuh"
 #include "qmv_tcf.cuh"
 
@@ -11,15 +11,11 @@ template <int B>
 cudaError_t tcf_b(int ncw, const Params& p, const Launch& L) {
     if (ncw == 8) {
         static std::atomic<unsigned> cfg_{0};
-        return launch_kernel(qmv_tcf_kernel<B, kTcbStages, 256>, cfg_, L, p);
+        return launch_kernel(qmv_tcf_kernel<B, kTcbStages, 288>, cfg_, L, p);
     }
     if (ncw == 12) {
         static std::atomic<unsigned> cfg_{0};
-        return launch_kernel(qmv_tcf_kernel<B, kTcbStages, 384>, cfg_, L, p);
-    }
-    if (ncw == 16) {
-        static std::atomic<unsigned> cfg_{0};
-        return launch_kernel(qmv_tcf_kernel<B, kTcbStages, 512>, cfg_, L, p);
+        return launch_kernel(qmv_tcf_kernel<B, kTcbStages, 416>, cfg_, L, p);
     }
     return cudaErrorInvalidValue;
 }

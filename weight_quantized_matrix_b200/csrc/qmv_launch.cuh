@@ -61,12 +61,12 @@ cudaError_t launch_fp(int fam, int dtype, int maxm, int R, bool wide, const Para
 // Tensor-core kernels (qmv_tc_kernel): npass in {1, 2, 4}.
 cudaError_t launch_tc_affine(int bits, int dtype, int npass, const Params& p, const Launch& L);
 // Tensor-core kernels with the bulk-copy weight ring (qmv_tcb_kernel):
-// (npass, spb) in {(1,1), (1,2), (1,4), (1,8), (2,1), (4,1)}; ncw = warps per
-// block in {8, 12, 16} (16 only for npass <= 2).
+// (npass, spb) in {(1,1), (1,2), (1,4), (1,8), (2,1), (4,1)}; ncw = consumer
+// warps per block in {8, 12} (plus the producer warp).
 cudaError_t launch_tcb_affine(int bits, int dtype, int npass, int spb, int ncw, const Params& p, const Launch& L);
 constexpr int kTcbStages = 4;
 // CUDA-core kernels with the weight ring, one bf16 x row (qmv_tcf_kernel):
-// ncw = warps per block in {8, 12, 16}.
+// ncw = compute warps per block in {8, 12} (plus the producer warp).
 cudaError_t launch_tcf_affine(int bits, int ncw, const Params& p, const Launch& L);
 
 
@@ -112,17 +112,11 @@ inline bool shape_instantiated(int maxm, int R, bool wide) {
     if (npass == NPASS_ && spb == SPB_) {                                                    \
         if (ncw == 8) {                                                                      \
             static std::atomic<unsigned> cfg_{0};                                            \
-            return launch_kernel(qmv_tcb_kernel<BITS_, T_, NPASS_, SPB_, kTcbStages, 256>, cfg_, L, p); \
+            return launch_kernel(qmv_tcb_kernel<BITS_, T_, NPASS_, SPB_, kTcbStages, 288>, cfg_, L, p); \
         }                                                                                    \
         if (ncw == 12) {                                                                     \
             static std::atomic<unsigned> cfg_{0};                                            \
-            return launch_kernel(qmv_tcb_kernel<BITS_, T_, NPASS_, SPB_, kTcbStages, 384>, cfg_, L, p); \
-        }                                                                                    \
-        if constexpr (NPASS_ <= 2) {                                                         \
-            if (ncw == 16) {                                                                 \
-                static std::atomic<unsigned> cfg_{0};                                        \
-                return launch_kernel(qmv_tcb_kernel<BITS_, T_, NPASS_, SPB_, kTcbStages, 512>, cfg_, L, p); \
-            }                                                                                \
+            return launch_kernel(qmv_tcb_kernel<BITS_, T_, NPASS_, SPB_, kTcbStages, 416>, cfg_, L, p); \
         }                                                                                    \
     }
 #define QMV_TCB_SHAPES(T_)                                                                   \

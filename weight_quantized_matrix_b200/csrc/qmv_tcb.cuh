@@ -1,38 +1,33 @@
 // qmv_tcb.cuh -- tensor-core affine qmv whose weights stream through a
 // shared-memory ring filled by the tensor-copy engine (cp.async.bulk.tensor)
-// under mbarrier flow control.  Every warp of the block computes; there is no
-// dedicated producer warp.
+// under mbarrier flow control: one producer warp, wr x wk consumer warps.
 //
 // Why: the register-prefetch kernel (qmv_tc.cuh) keeps only a few KB per SM in
 // flight, bounded by registers and occupancy, and stalls on load latency.  Here
 // the bytes in flight are STAGES ring stages per SM (tens of KB), independent
-// of the warps' registers.  Registers are allocated per SM sub-partition, so a
-// block of 8, 12 or 16 warps (2, 3 or 4 per sub-partition) gets up to 255, 168
-// or 128 registers a thread; a ninth, producer-only warp would cost a quarter
-// of that budget.
+// of the consumers' registers.
 //
 // Work: the grid is persistent over ROW BLOCKS of ROWS = 16*wr rows (block b
 // takes row blocks b, b + gridDim.x, ...).  A row block's packed rows are cut
-// along K into ring STAGES of S super-blocks; the block's stages form one
-// sequence across its row blocks.  Warp (wrid, wkid) owns row tile wrid (16
-// rows) and the super-blocks wkid, wkid + wk, ... of every stage, taken SPB at
-// a time: one BATCH fills the 8*NPASS slot columns of the MMAs (decode and slot
-// columns as in qmv_tc.cuh) and ends in one exact fp32 epilogue.  Everything a
-// lane needs to place its x fragments, scales and sums inside a batch is
-// computed once per kernel, so a full batch runs without per-super-block index
-// arithmetic or predicates; only the last, partial batch of a row takes the
-// guarded path.
+// along K into ring STAGES of S super-blocks; the producer copies stage after
+// stage (the packed rows, and when their layout allows the stage's scales and
+// biases: one 3-D tensor copy each) into the ring, across row-block
+// boundaries, while consumers compute.  Consumer warp (wrid, wkid) owns row
+// tile wrid (16 rows) and the super-blocks wkid, wkid + wk, ... of every
+// stage, taken SPB at a time: one BATCH fills the 8*NPASS slot columns of the
+// MMAs (decode and slot columns as in qmv_tc.cuh) and ends in one exact fp32
+// epilogue.  Everything a lane needs to place its x fragments, scales and sums
+// inside a batch is computed once per kernel, so a full batch runs without
+// per-super-block index arithmetic or predicates; only the last, partial
+// batch of a row takes the guarded path.
 //
-// Flow control: full[s] (one arrival with the copies' byte count) per ring
-// slot, and a shared arrival counter per slot.  Thread 0 issues the first
-// STAGES stages (weights only, before the grid-dependency wait).  A warp done
-// with a stage adds one to its slot's counter; the warp whose arrival completes
-// the count (every NCW-th) refills the slot with stage j + STAGES at once.
-// Every wait is bounded (about one second of %globaltimer); on expiry the
-// kernel ORs a code into the fault word p.fault (1: a warp gave up on a full
-// stage, 4: the block gave up waiting for its own copies at exit), stops
-// computing, keeps its arrival schedule so no warp waits on another forever,
-// and thread 0 waits (bounded) for every copy the block issued before exit.
+// Flow control: full[s] (one producer arrival + the copies' byte count) and
+// empty[s] (one arrival per consumer warp).  Every wait is bounded (about one
+// second of %globaltimer); on expiry the kernel ORs a code into the fault word
+// p.fault (1: a consumer gave up on a full stage, 2: the producer gave up on an
+// empty stage, 4: the producer gave up waiting for its own copies), stops
+// computing, keeps its barrier schedule so no warp waits on another forever,
+// and the producer waits (bounded) for every copy it issued before it exits.
 //
 // Ring rows are dense (pitch = the stage's S * 4 * UB bytes, as the tensor copy
 // lays them out); the two rows one load instruction touches per 8 lanes then
@@ -99,15 +94,17 @@ __device__ __forceinline__ void tensor_copy_3d(uint32_t dst, const CUtensorMap* 
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
         : "memory");
 }
-// Barrier over the block's warps (named barrier 1).
+// Barrier over the consumer warps only (named barrier 1).
 __device__ __forceinline__ void consumer_sync(int nthreads) {
     asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
-// Orders this thread's earlier generic-proxy shared-memory accesses (and those
-// it has observed) before its later async-proxy ones: a slot's readers before
-// the tensor copy that overwrites it.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+// Adds one to a shared arrival counter, ordered after this thread's (and,
+// through a preceding __syncwarp, its warp's) earlier shared-memory accesses
+// and before its later ones; returns the previous count.
+__device__ __forceinline__ unsigned arrive_count(unsigned* ctr) {
+    unsigned old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], 1;" : "=r"(old) : "r"(smem_addr(ctr)) : "memory");
+    return old;
 }
 
 // Scale / bias element of a ring row (x dtype), widened to fp32.
@@ -123,8 +120,7 @@ template <> __device__ __forceinline__ float ring_scale<__nv_bfloat16>(const uns
 }
 
 // Shared memory (bytes, in order):
-//   bars  128            full[STAGES] (8 bytes each), then the arrival
-//                        counters arrivals[STAGES] (4 bytes each) at byte 64
+//   bars  128            full[STAGES], empty[STAGES] (8 bytes each)
 //   ring  STAGES stages (128-byte aligned) of: ROWS packed rows (pitch bytes
 //         each, dense), then (p.sring) the scale tile at p.soff and the bias
 //         tile at p.boff, ROWS x p.sbw bytes each
@@ -134,8 +130,9 @@ template <> __device__ __forceinline__ float ring_scale<__nv_bfloat16>(const uns
 //   sxx   M * NSEG float2      {sum(x), sum(x~)} per segment of the tile
 //   us    M * TU * 2 floats    per-unit sums
 //   red   NCW * 16 * 8*NPASS floats
-// MAXT: threads per block the kernel is compiled for, 32 * (wk * wr) with
-// wk * wr in {8, 12, 16} (the register budget follows).
+// MAXT: threads per block the kernel is compiled for, 32 * (wk * wr + 1) with
+// wk * wr in {8, 12} consumer warps plus the producer warp (the register
+// budget follows).
 template <int B, class T, int NPASS, int SPB, int STAGES, int MAXT>
 __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant__ Params p) {
     using Gm = TcGeom<B>;
@@ -144,7 +141,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
     constexpr int NW = Gm::NW, UB = Gm::UNIT_BYTES, UC = Gm::UNIT_CODES, SB = Gm::SB;
     constexpr int NSPLIT = TcSplit<T>::n;
     constexpr int ES = (int)sizeof(T);
-    static_assert(8 * STAGES <= 64 && 4 * STAGES <= 64, "barrier area");
+    static_assert(2 * STAGES * 8 <= 128, "barrier area");
 
     extern __shared__ float4 smem4[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(smem4);
@@ -174,7 +171,6 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
     const int gdiv = G > SB ? __ffs(G / SB) - 1 : 0;
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    unsigned* arrivals = reinterpret_cast<unsigned*>(smem + 64);
     // ring on a 128-byte boundary (tensor-copy destinations); the host adds
     // 128 bytes of slack for this
     unsigned char* ring = smem + 128 + ((128u - (smem_addr(smem) & 127u)) & 127u);
@@ -184,11 +180,12 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
     float* red = us + (size_t)M * TU * 2;
     const uint32_t bar0 = smem_addr(bars);
     auto full = [&](int s) { return bar0 + 8u * (uint32_t)s; };
+    auto empty = [&](int s) { return bar0 + 8u * (uint32_t)(STAGES + s); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full(s), 1);
-            arrivals[s] = 0u;
+            mbar_init(empty(s), (uint32_t)NCW);
         }
         mbar_init_fence();
     }
@@ -197,32 +194,48 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
     const long long sb0 = bz * p.s_bs;
     const int nks = (NSBK + S - 1) / S;
     // this block's stages: j = (i-th row block of the block) * nks + K stage
-    const int total = blockIdx.x < nrb ? ((nrb - 1 - (int)blockIdx.x) / (int)gridDim.x + 1) * nks : 0;
-    const uint32_t ring0 = smem_addr(ring);
-    const uint32_t stage_tx = (uint32_t)ROWS * ((uint32_t)pitch + (sring ? 2u * (uint32_t)sbw : 0u));
-    // Stage j into its slot: one tensor copy each for the packed rows (ROWS x
-    // pitch bytes), the scale tile and the bias tile (ROWS x sbw bytes); rows
-    // past N and columns past the row end are zero-filled and count in full.
-    auto issue = [&](int j) {
-        const int slot = j % STAGES;
-        const int rb = (int)blockIdx.x + (j / nks) * (int)gridDim.x, ks = j % nks;
-        const uint32_t st0 = ring0 + (uint32_t)(slot * stage_bytes);
-        mbar_arrive_expect_tx(full(slot), stage_tx);
-        tensor_copy_3d(st0, &p.wmap, (ks * S * 4 * UB) / 8, rb * ROWS, bz, full(slot));
-        if (sring) {
-            const int g0 = ((ks * S) << gmul) >> gdiv;
-            tensor_copy_3d(st0 + (uint32_t)p.soff, &p.smap, g0, rb * ROWS, bz, full(slot));
-            tensor_copy_3d(st0 + (uint32_t)p.boff, &p.bmap, g0, rb * ROWS, bz, full(slot));
+    // ---- producer warp: streams weights only, so it starts at once ---------
+    // (written out here, not as a helper taking the tensor maps' addresses:
+    // that form measured up to 25 % slower on B200 for the whole kernel)
+    if (warp == NCW) {
+        grid_launch_dependents();    // the next kernel may start fetching its weights
+        const uint32_t ring0 = smem_addr(ring);
+        const uint32_t stage_tx = (uint32_t)ROWS * ((uint32_t)pitch + (sring ? 2u * (uint32_t)sbw : 0u));
+        int it = 0;
+        bool ok = true;
+        for (int rb = blockIdx.x; rb < nrb && ok; rb += gridDim.x) {
+            for (int ks = 0; ks < nks; ++ks) {
+                const int slot = it % STAGES, f = it / STAGES;
+                if (f > 0 && !mbar_wait(empty(slot), (uint32_t)((f - 1) & 1))) { ok = false; break; }
+                const uint32_t st0 = ring0 + (uint32_t)(slot * stage_bytes);
+                if (lane == 0) {
+                    // one tensor copy each: the stage's packed rows (ROWS x pitch
+                    // bytes), scale tile and bias tile (ROWS x sbw bytes); rows
+                    // past N and columns past the row end are zero-filled and
+                    // count in full
+                    mbar_arrive_expect_tx(full(slot), stage_tx);
+                    tensor_copy_3d(st0, &p.wmap, (ks * S * 4 * UB) / 8, rb * ROWS, bz, full(slot));
+                    if (sring) {
+                        const int g0 = ((ks * S) << gmul) >> gdiv;
+                        tensor_copy_3d(st0 + (uint32_t)p.soff, &p.smap, g0, rb * ROWS, bz, full(slot));
+                        tensor_copy_3d(st0 + (uint32_t)p.boff, &p.bmap, g0, rb * ROWS, bz, full(slot));
+                    }
+                }
+                __syncwarp();
+                ++it;
+            }
         }
-    };
+        unsigned code = ok ? 0u : 2u;
+        // wait for the copies this warp issued: the last fill of each slot
+        for (int s = 0; s < STAGES && s < it; ++s) {
+            const int last = (it - 1 - s) / STAGES;
+            if (!mbar_wait(full(s), (uint32_t)(last & 1))) code |= 4u;
+        }
+        if (code && lane == 0) atomicOr(p.fault, code);
+        return;
+    }
 
-    // the next kernel in the stream may launch and start fetching its weights
-    grid_launch_dependents();
-    // the first stages stream weights only: issued before the grid-dependency
-    // wait (x and y may belong to the previous kernel in the stream)
-    if (threadIdx.x == 0)
-        for (int j = 0; j < STAGES && j < total; ++j) issue(j);
-
+    // ---- consumer warps: x and y may belong to the previous kernel ---------
     grid_wait();
     const int nthr = NCW * 32;
     const int g = lane >> 2, t = lane & 3;
@@ -274,6 +287,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
         }
 
     const uint32_t kbf16 = p.kbf16;
+    const bool pairc = (M & 1) == 0;   // even M: both columns of a lane in one slot group
     int it = 0;
     bool ok = true;
     bool x_whole = false;            // x of the whole K is staged (one tile)
@@ -370,27 +384,35 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
 
             // ---- one batch: SPB super-blocks of this warp, then the epilogue ---
             // FULL: all SPB super-blocks exist (no guards); otherwise nex of them.
-            auto run_batch = [&](auto full_c, int sbf, int nex, int sbase, const unsigned char* rowg,
-                                 const unsigned char* rowh, const unsigned char* tileg) {
+            // RING: scales and biases from the stage's tiles (sp: scale row g,
+            // scale row g + 8, bias row g, bias row g + 8, each indexed by the
+            // group within the stage), else from global memory (indexed by the
+            // group within the row).  With an even M the two columns of a lane
+            // share their slot's group: its scales are loaded once.
+            auto run_batch = [&](auto full_c, auto ring_c, int sbf, int nex, int sbase, const unsigned char* rowg,
+                                 const unsigned char* rowh, const unsigned char* const (&sp)[4]) {
                 constexpr bool FULL = decltype(full_c)::value;
+                constexpr bool RING = decltype(ring_c)::value;
                 float sc[NPASS][4], bs[NPASS][4];
+                const int a0 = RING ? sbf - sbase : sbf;
 #pragma unroll
                 for (int pp = 0; pp < NPASS; ++pp)
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
+                        if (c == 1 && pairc) {
+                            sc[pp][1] = sc[pp][0]; sc[pp][3] = sc[pp][2]; bs[pp][1] = bs[pp][0]; bs[pp][3] = bs[pp][2];
+                            continue;
+                        }
                         const bool pres = FULL || dsb[pp][c] < nex;
+                        const int gi = (((a0 + dgrp[pp][c]) << gmul) >> gdiv) + dgs[pp][c];
                         float s0 = 0.f, s1 = 0.f, b0 = 0.f, b1 = 0.f;
-                        if (sring) {
-                            const int gl = ((((sbf - sbase) + dgrp[pp][c]) << gmul) >> gdiv) + dgs[pp][c];
-                            if (pres) {
-                                s0 = ring_scale<T>(tileg + p.soff, gl); s1 = ring_scale<T>(tileg + p.soff + 8 * sbw, gl);
-                                b0 = ring_scale<T>(tileg + p.boff, gl); b1 = ring_scale<T>(tileg + p.boff + 8 * sbw, gl);
-                            }
-                        } else {
-                            const int gg = (((sbf + dgrp[pp][c]) << gmul) >> gdiv) + dgs[pp][c];
-                            if (pres) {
-                                s0 = DT<T>::ld(scg, gg); s1 = DT<T>::ld(sch, gg);
-                                b0 = DT<T>::ld(big, gg); b1 = DT<T>::ld(bih, gg);
+                        if (pres) {
+                            if constexpr (RING) {
+                                s0 = ring_scale<T>(sp[0], gi); s1 = ring_scale<T>(sp[1], gi);
+                                b0 = ring_scale<T>(sp[2], gi); b1 = ring_scale<T>(sp[3], gi);
+                            } else {
+                                s0 = DT<T>::ld(scg, gi); s1 = DT<T>::ld(sch, gi);
+                                b0 = DT<T>::ld(big, gi); b1 = DT<T>::ld(bih, gi);
                             }
                         }
                         sc[pp][c] = s0; sc[pp][2 + c] = s1; bs[pp][c] = b0; bs[pp][2 + c] = b1;
@@ -456,23 +478,23 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
                     const unsigned char* rowh = rowg + 8 * pitch;
                     // scale / bias tile rows of this lane: stage + offset + row * sbw
                     const unsigned char* tileg = ring + (size_t)slot * stage_bytes + (size_t)(wrid * 16 + g) * sbw;
-                    for (int sbf = sbase + wkid; sbf < send; sbf += SPB * wk) {
-                        const int nex = (send - sbf + wk - 1) / wk;
-                        if (nex >= SPB) run_batch(std::true_type{}, sbf, SPB, sbase, rowg, rowh, tileg);
-                        else run_batch(std::false_type{}, sbf, nex, sbase, rowg, rowh, tileg);
-                    }
+                    const unsigned char* const sp[4] = {tileg + p.soff, tileg + p.soff + 8 * sbw, tileg + p.boff,
+                                                        tileg + p.boff + 8 * sbw};
+                    auto batches = [&](auto ring_c) {
+                        for (int sbf = sbase + wkid; sbf < send; sbf += SPB * wk) {
+                            if (sbf + (SPB - 1) * wk < send) {
+                                run_batch(std::true_type{}, ring_c, sbf, SPB, sbase, rowg, rowh, sp);
+                            } else {
+                                const int nex = (send - sbf + wk - 1) / wk;
+                                run_batch(std::false_type{}, ring_c, sbf, nex, sbase, rowg, rowh, sp);
+                            }
+                        }
+                    };
+                    if (sring) batches(std::true_type{});
+                    else batches(std::false_type{});
                 }
-                // done with the slot: the warp completing its count refills it
                 __syncwarp();
-                if (lane == 0) {
-                    __threadfence_block();
-                    // the slot's f-th fill is complete at arrival (f + 1) * NCW
-                    const unsigned before = atomicAdd(&arrivals[slot], 1u);
-                    if (before + 1u == (unsigned)((f + 1) * NCW) && it + STAGES < total) {
-                        fence_proxy_async_smem();
-                        issue(it + STAGES);
-                    }
-                }
+                if (lane == 0) mbar_arrive(empty(slot));
                 ++it;
             }
         }
@@ -498,17 +520,6 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
         consumer_sync(nthr);
     }
 
-    // Every warp has passed its last stage, so every refill has been issued.
-    // Without a fault each was awaited already; otherwise wait (bounded) for
-    // the last fill of each slot before the block's shared memory is released.
-    if (threadIdx.x == 0) {
-        unsigned code = 0u;
-        for (int s = 0; s < STAGES && s < total; ++s) {
-            const int last = (total - 1 - s) / STAGES;
-            if (!mbar_wait(full(s), (uint32_t)(last & 1))) code |= 4u;
-        }
-        if (code) atomicOr(p.fault, code);
-    }
 }
 
 }  // namespace qmv

@@ -1,7 +1,6 @@
 // qmv_tcf.cuh -- affine qmv for one bf16 x row on the CUDA cores, with the
-// weights streaming through the same shared-memory ring as qmv_tcb.cuh (tensor
-// copies, full barriers, arrival counters, refill by the warp that completes a
-// slot's count; thread 0 fills the first STAGES stages).
+// weights streaming through the same shared-memory ring as qmv_tcb.cuh (one
+// producer warp issuing tensor copies, full / empty barriers, bounded waits).
 //
 // Why: with one x row an m16n8k16 MMA uses one of its eight columns, and on
 // B200 the warp-level MMAs of that kernel, issued in order between the decode
@@ -55,14 +54,15 @@ __device__ __forceinline__ void tcf_unit(std::integer_sequence<int, Q...>, const
 }
 
 // Shared memory (bytes, in order):
-//   bars  128            full[STAGES], arrivals[STAGES] at byte 64, row-block
-//                        completion counters rdone[STAGES + 1] at byte 96
+//   bars  128            full[STAGES], empty[STAGES], row-block completion
+//                        counters rdone[STAGES + 1] at byte 96
 //   ring  STAGES stages (128-byte aligned): ROWS packed rows (pitch bytes
 //         each), then (p.sring) the scale tile at p.soff and the bias tile at
 //         p.boff, ROWS x p.sbw bytes each
 //   xs    TU * (NP + 4) u32     x~ pairs of the tile's units (bf16x2, plan order)
 //   us    TU * 2 floats         {sum(x), sum(x~)} per unit
 //   red   (STAGES + 1) * NCW * 16 floats   per-warp row sums, by row block
+// MAXT = 32 * (NCW + 1): NCW = wk * wr in {8, 12} compute warps + the producer.
 template <int B, int STAGES, int MAXT>
 __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant__ Params p) {
     using T = __nv_bfloat16;
@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
     constexpr TcPlanData P = tc_make_plan<B, false>();
     constexpr int NP = P.np, NPS = NP + 4;
     constexpr int NW = Gm::NW, UB = Gm::UNIT_BYTES, UC = Gm::UNIT_CODES, SB = Gm::SB;
-    static_assert(8 * STAGES <= 64 && 4 * STAGES <= 32 && 4 * (STAGES + 1) <= 32, "barrier area");
+    static_assert(2 * STAGES * 8 <= 96 && 4 * (STAGES + 1) <= 32, "barrier area");
 
     extern __shared__ float4 smem4[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(smem4);
@@ -94,7 +94,6 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
     const int gdiv = G > SB ? __ffs(G / SB) - 1 : 0;
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    unsigned* arrivals = reinterpret_cast<unsigned*>(smem + 64);
     unsigned* rdone = reinterpret_cast<unsigned*>(smem + 96);
     unsigned char* ring = smem + 128 + ((128u - (smem_addr(smem) & 127u)) & 127u);
     uint32_t* xs = reinterpret_cast<uint32_t*>(ring + (size_t)STAGES * stage_bytes);
@@ -102,11 +101,12 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
     float* red = reinterpret_cast<float*>(us + TU);
     const uint32_t bar0 = smem_addr(bars);
     auto full = [&](int s) { return bar0 + 8u * (uint32_t)s; };
+    auto empty = [&](int s) { return bar0 + 8u * (uint32_t)(STAGES + s); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full(s), 1);
-            arrivals[s] = 0u;
+            mbar_init(empty(s), (uint32_t)NCW);
         }
         for (int s = 0; s <= STAGES; ++s) rdone[s] = 0u;
         mbar_init_fence();
@@ -115,25 +115,38 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
 
     const long long sb0 = bz * p.s_bs;
     const int nks = (NSBK + S - 1) / S;
-    const int total = blockIdx.x < nrb ? ((nrb - 1 - (int)blockIdx.x) / (int)gridDim.x + 1) * nks : 0;
-    const uint32_t ring0 = smem_addr(ring);
-    const uint32_t stage_tx = (uint32_t)ROWS * ((uint32_t)pitch + (sring ? 2u * (uint32_t)sbw : 0u));
-    auto issue = [&](int j) {
-        const int slot = j % STAGES;
-        const int rb = (int)blockIdx.x + (j / nks) * (int)gridDim.x, ks = j % nks;
-        const uint32_t st0 = ring0 + (uint32_t)(slot * stage_bytes);
-        mbar_arrive_expect_tx(full(slot), stage_tx);
-        tensor_copy_3d(st0, &p.wmap, (ks * S * 4 * UB) / 8, rb * ROWS, bz, full(slot));
-        if (sring) {
-            const int g0 = ((ks * S) << gmul) >> gdiv;
-            tensor_copy_3d(st0 + (uint32_t)p.soff, &p.smap, g0, rb * ROWS, bz, full(slot));
-            tensor_copy_3d(st0 + (uint32_t)p.boff, &p.bmap, g0, rb * ROWS, bz, full(slot));
+    if (warp == NCW) {                               // the producer warp
+        grid_launch_dependents();
+        const uint32_t ring0 = smem_addr(ring);
+        const uint32_t stage_tx = (uint32_t)ROWS * ((uint32_t)pitch + (sring ? 2u * (uint32_t)sbw : 0u));
+        int it = 0;
+        bool ok = true;
+        for (int rb = blockIdx.x; rb < nrb && ok; rb += gridDim.x) {
+            for (int ks = 0; ks < nks; ++ks) {
+                const int slot = it % STAGES, f = it / STAGES;
+                if (f > 0 && !mbar_wait(empty(slot), (uint32_t)((f - 1) & 1))) { ok = false; break; }
+                const uint32_t st0 = ring0 + (uint32_t)(slot * stage_bytes);
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(full(slot), stage_tx);
+                    tensor_copy_3d(st0, &p.wmap, (ks * S * 4 * UB) / 8, rb * ROWS, bz, full(slot));
+                    if (sring) {
+                        const int g0 = ((ks * S) << gmul) >> gdiv;
+                        tensor_copy_3d(st0 + (uint32_t)p.soff, &p.smap, g0, rb * ROWS, bz, full(slot));
+                        tensor_copy_3d(st0 + (uint32_t)p.boff, &p.bmap, g0, rb * ROWS, bz, full(slot));
+                    }
+                }
+                __syncwarp();
+                ++it;
+            }
         }
-    };
-
-    grid_launch_dependents();
-    if (threadIdx.x == 0)
-        for (int j = 0; j < STAGES && j < total; ++j) issue(j);
+        unsigned code = ok ? 0u : 2u;
+        for (int s = 0; s < STAGES && s < it; ++s) {
+            const int last = (it - 1 - s) / STAGES;
+            if (!mbar_wait(full(s), (uint32_t)(last & 1))) code |= 4u;
+        }
+        if (code && lane == 0) atomicOr(p.fault, code);
+        return;
+    }
     grid_wait();
 
     const int nthr = NCW * 32;
@@ -265,17 +278,8 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
                         for (int j = wkid; j < nsteps; j += wk) step(std::false_type{}, j);
                     }
                 }
-                // done with the slot: the warp completing its count refills it
                 __syncwarp();
-                if (lane == 0) {
-                    __threadfence_block();
-                    // the slot's f-th fill is complete at arrival (f + 1) * NCW
-                    const unsigned before = atomicAdd(&arrivals[slot], 1u);
-                    if (before + 1u == (unsigned)((f + 1) * NCW) && it + STAGES < total) {
-                        fence_proxy_async_smem();
-                        issue(it + STAGES);
-                    }
-                }
+                if (lane == 0) mbar_arrive(empty(slot));
                 ++it;
             }
         }
@@ -298,13 +302,11 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
             __syncwarp();
             unsigned last = 0u;
             if (lane == 0) {
-                __threadfence_block();
-                const unsigned before = atomicAdd(&rdone[buf], 1u);
+                const unsigned before = arrive_count(&rdone[buf]);
                 last = before + 1u == (unsigned)((round + 1) * NCW) ? 1u : 0u;
             }
             last = __shfl_sync(0xFFFFFFFFu, last, 0);
             if (last) {
-                __threadfence_block();
                 for (int i = lane; i < ROWS; i += 32) {
                     const int w_ = i >> 4, r = i & 15;
                     float v = 0.f;
@@ -317,14 +319,6 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
         ++rbi;
     }
 
-    if (threadIdx.x == 0) {
-        unsigned code = 0u;
-        for (int s = 0; s < STAGES && s < total; ++s) {
-            const int last = (total - 1 - s) / STAGES;
-            if (!mbar_wait(full(s), (uint32_t)(last & 1))) code |= 4u;
-        }
-        if (code) atomicOr(p.fault, code);
-    }
 }
 
 }  // namespace qmv
