@@ -271,7 +271,10 @@ class Layer:
 
 
 class Probe(Layer):
+    """Sustained streaming: each step makes CALLS calls, one on each of CALLS
+    distinct weight copies (151 MB each, more than L2), back to back."""
     name = "bandwidth probe, affine 4-bit g64 bf16, N=K=16384, M=1"
+    CALLS = 3
 
     def __init__(self, q, torch, dev):
         self.q, self.torch = q, torch
@@ -282,11 +285,29 @@ class Probe(Layer):
         self.sets = [dict(name="probe", M=1, N=16384, K=16384, ws=ws, x=x_host.to(dev), x_host=x_host,
                           y=torch.empty((1, 16384), dtype=torch.bfloat16, device=dev),
                           y_host=torch.empty((1, 16384), dtype=torch.bfloat16).pin_memory(), it=0)]
-        self.calls_per_step = 1
+        self.calls_per_step = self.CALLS
+
+    def graph_variants(self, s):
+        return 1
+
+    def run_group(self, s, e2e=False, v=0):
+        if e2e:
+            s["x"].copy_(s["x_host"], non_blocking=True)
+        for c in range(self.CALLS):
+            w, sc, bi = s["ws"][c]
+            self.q.qmv_affine(s["x"], w, sc, bi, s["y"], 1, s["N"], s["K"], 4, 64, "bf16")
+        if e2e:
+            s["y_host"].copy_(s["y"], non_blocking=True)
+        return self.CALLS
+
+    def group_bytes(self, s):
+        return affine_bytes(1, s["N"], s["K"], 4, 64) * self.CALLS
 
     def config(self):
         return {"workload": self.name, "bits": 4, "group": 64, "dtype": "bf16", "M": 1, "N": 16384, "K": 16384,
-                "calls_per_step": 1, "l2": "flushed before every step (512 MB write + 256 MB read); 3 weight copies rotate"}
+                "calls_per_step": self.CALLS,
+                "l2": "flushed before every step (512 MB write + 256 MB read); each of the step's 3 calls reads "
+                      "its own 151 MB weight copy"}
 
 
 WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe}
@@ -410,7 +431,7 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_kind = peaks()
     for gi, (label, s) in enumerate(groups):
         ms = float(per_group[gi])
-        n = wl.calls_per_step // len(groups) if isinstance(wl, Chain8) else 1
+        n = wl.calls_per_step // len(groups)        # calls per group replay
         b = wl.group_bytes(s)
         plan = wl.group_plan(s)
         kern = " ".join(w for w in plan.split() if w.split("=")[0] in ("path", "chunk", "maxm", "rows_per_warp"))

@@ -500,6 +500,8 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
         }
 
         // ---- reduce over slots of the same x row and over k-warps, store -----
+        // (every consumer takes a share: a reduction done by the last warp
+        // alone measured up to 2x slower, it lands on the critical path)
         float* myred = red + (size_t)warp * 16 * 8 * NPASS;
 #pragma unroll
         for (int pp = 0; pp < NPASS; ++pp)

@@ -307,6 +307,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
             }
             last = __shfl_sync(0xFFFFFFFFu, last, 0);
             if (last) {
+                __syncwarp();                  // lane 0's acquire, for every lane
                 for (int i = lane; i < ROWS; i += 32) {
                     const int w_ = i >> 4, r = i & 15;
                     float v = 0.f;
