@@ -169,3 +169,20 @@ def test_fast_extension_forwards_status():
     assert q._fast.affine(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 128, 4, 64, 2, 1, 1, 0) == 0
     with pytest.raises(TypeError):
         q._fast.affine(FAKE)
+
+
+def test_build_module_loads_without_the_library(tmp_path):
+    """The build script runs on a fresh checkout, where libqmv.so does not
+    exist yet: loading it by path must not import the package (whose import
+    needs the library)."""
+    import subprocess
+    import sys
+    code = (
+        "import importlib.util, sys\n"
+        f"spec = importlib.util.spec_from_file_location('b', {str(ROOT)!r} + '/weight_quantized_matrix_b200/build_lib.py')\n"
+        "m = importlib.util.module_from_spec(spec); spec.loader.exec_module(m)\n"
+        "assert callable(m.build) and callable(m.build_ext)\n"
+        "assert 'weight_quantized_matrix_b200' not in sys.modules\n"
+    )
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=str(tmp_path))
+    assert r.returncode == 0, r.stderr
