@@ -71,6 +71,10 @@ def lib():
         L.oracle_qmv_affine.restype = None
         L.oracle_qmv_fp.argtypes = [p, p, p, f, p, p, ll, ll, ll, i, i, ll, ll]
         L.oracle_qmv_fp.restype = None
+        L.oracle_f32_to_bf16.argtypes = [f]; L.oracle_f32_to_bf16.restype = u
+        L.oracle_f32_to_f16.argtypes = [f]; L.oracle_f32_to_f16.restype = u
+        L.oracle_quantize_affine.argtypes = [p, p, p, p, ll, ll, i, i, i, ll, ll]
+        L.oracle_quantize_affine.restype = None
         _lib = L
     return _lib
 
@@ -121,6 +125,8 @@ def e2m1(c): return lib().oracle_e2m1(int(c))
 def e4m3(c): return lib().oracle_e4m3(int(c))
 def e8m0(e): return lib().oracle_e8m0(int(e))
 def round_f32_sum(a, b): return lib().oracle_round_f32_sum(float(a), float(b))
+def f32_to_bf16(v): return lib().oracle_f32_to_bf16(float(v))
+def f32_to_f16(v): return lib().oracle_f32_to_f16(float(v))
 
 
 def affine_codes(row: np.ndarray, K: int, bits: int) -> np.ndarray:
@@ -169,3 +175,21 @@ def qmv_fp(x, w, scales, global_scale, M, N, K, mode, dtype, rows=None, threads=
                                         M, N, K, FP_MODES[mode], DTYPE_CODES[dtype], r0, r1)
     _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
     return y, a
+
+
+# ---- affine quantizer -------------------------------------------------------
+def quantize_affine(w, N, K, bits, group, dtype, rows=None, threads=1):
+    """Quantize w ([N, K] elements of `dtype`, given as a numpy array of that
+    element's storage: float32, or uint16 bit patterns for f16 / bf16) into
+    (packed codes uint8 [N, row_bytes], scales, biases) with the storage of
+    `dtype`.  Rows outside `rows` stay zero."""
+    w = np.ascontiguousarray(w)
+    st = np.float32 if dtype == "f32" else np.uint16
+    wq = np.zeros((N, row_bytes(K, bits)), dtype=np.uint8)
+    sc = np.zeros((N, K // group), dtype=st)
+    bi = np.zeros((N, K // group), dtype=st)
+    L = lib()
+    fn = lambda a, b: L.oracle_quantize_affine(_ptr(w), _ptr(wq), _ptr(sc), _ptr(bi), N, K, bits, group,
+                                               DTYPE_CODES[dtype], a, b)
+    _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
+    return wq, sc, bi

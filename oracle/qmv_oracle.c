@@ -242,3 +242,105 @@ void oracle_qmv_fp(const void* x, const uint8_t* w, const uint8_t* scales, float
             if (absdot) absdot[m * N + n] = aacc;
         }
 }
+
+/* ---------------------------------------------------------------------------
+ * Rounding fp32 to the element types, to nearest, ties to even (IEEE 754
+ * roundTiesToEven), from the field definitions above.  Finite inputs.
+ * ------------------------------------------------------------------------- */
+/* bfloat16 keeps fp32's sign and exponent and the top 7 mantissa bits: the
+ * dropped low 16 bits decide the rounding (above half up, below down, exactly
+ * half to the even neighbour). */
+uint32_t oracle_f32_to_bf16(float f) {
+    uint32_t u; memcpy(&u, &f, 4);
+    uint32_t lo = u & 0xFFFFu, hi = u >> 16;
+    if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u))) hi += 1u;   /* a carry into the exponent is correct */
+    return hi & 0xFFFFu;
+}
+
+/* binary16: |v| >= 65520 rounds to infinity; below 2^-14 the value is an
+ * integer multiple of 2^-24 (subnormal); otherwise 1.m * 2^e with 10 mantissa
+ * bits.  Scaling by powers of two is exact in fp64, and nearbyint rounds ties
+ * to even under the default rounding mode. */
+uint32_t oracle_f32_to_f16(float f) {
+    double v = (double)f;
+    uint32_t s = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    if (a >= 65520.0) return s | 0x7C00u;
+    if (a < ldexp(1.0, -14)) {
+        double m = nearbyint(a * ldexp(1.0, 24));          /* 0..1024; 1024 encodes 2^-14 */
+        return s | (uint32_t)m;
+    }
+    int e;
+    double fr = frexp(a, &e);                              /* a = fr * 2^e, fr in [0.5, 1) */
+    e -= 1;                                                /* a = (2 fr) * 2^e, 2 fr in [1, 2) */
+    double m = nearbyint((2.0 * fr - 1.0) * 1024.0);
+    if (m == 1024.0) { m = 0.0; e += 1; }
+    return s | ((uint32_t)(e + 15) << 10) | (uint32_t)m;
+}
+
+/* ---------------------------------------------------------------------------
+ * Affine quantizer (wh-iron kernel-op coverage audit, the "quantized
+ * (affine_quantize / affine_dequantize)" row: quantize and dequantize for
+ * every width).  The pages name these kernels but do not state their
+ * arithmetic; this is the plainest reading consistent with w = scale*q + bias
+ * (MLX quantized_nax.h, dequantize): for each group of `group` consecutive
+ * weights of a row,
+ *     bias  = min(w),  scale = (max(w) - min(w)) / (2^bits - 1),
+ * both rounded to the element type, and
+ *     q = nearest integer, ties to even, to (w - bias_T) / scale_T,
+ * clamped to [0, 2^bits - 1] (q = 0 when scale_T is 0).  Every step that
+ * decides a code is one fp32 IEEE operation (subtract, divide, round), the
+ * precision the CUDA kernel takes the same decision in.  Codes are packed
+ * LSB first exactly as oracle_affine_code reads them.  Rows [n0, n1).
+ * ------------------------------------------------------------------------- */
+static float load_f32(const void* p, size_t i, int dtype) {
+    return (float)load_elem(p, i, dtype);                  /* exact: every T is an fp32 value */
+}
+
+static float store_round(void* p, size_t i, int dtype, float v) {
+    if (dtype == OR_F32) { memcpy((char*)p + 4 * i, &v, 4); return v; }
+    uint16_t h = (uint16_t)(dtype == OR_F16 ? oracle_f32_to_f16(v) : oracle_f32_to_bf16(v));
+    memcpy((char*)p + 2 * i, &h, 2);
+    return (float)(dtype == OR_F16 ? oracle_f16_value(h) : oracle_bf16_value(h));
+}
+
+static void put_code(uint8_t* row, long long i, int bits, uint32_t code) {
+    int pf = oracle_pack_factor(bits), bpp = oracle_bytes_per_pack(bits);
+    long long p = i / pf;
+    int j = (int)(i % pf);
+    uint64_t v = (uint64_t)code << (bits * j);
+    for (int b = 0; b < bpp; ++b) row[p * bpp + b] |= (uint8_t)(v >> (8 * b));
+}
+
+void oracle_quantize_affine(const void* w, uint8_t* wq, void* scales, void* biases, long long N,
+                            long long K, int bits, int group, int dtype, long long n0, long long n1) {
+    (void)N;
+    const int qmax = (1 << bits) - 1;
+    const long long rb = oracle_row_bytes(K, bits);
+    for (long long n = n0; n < n1; ++n) {
+        uint8_t* row = wq + n * rb;
+        memset(row, 0, (size_t)rb);
+        for (long long g0 = 0; g0 < K; g0 += group) {
+            float lo = load_f32(w, (size_t)(n * K + g0), dtype), hi = lo;
+            for (long long k = g0 + 1; k < g0 + group; ++k) {
+                float v = load_f32(w, (size_t)(n * K + k), dtype);
+                if (v < lo) lo = v;
+                if (v > hi) hi = v;
+            }
+            const float range = hi - lo;                    /* fp32 */
+            const float scale = range / (float)qmax;        /* fp32 */
+            const size_t gi = (size_t)(n * (K / group) + g0 / group);
+            const float sT = store_round(scales, gi, dtype, scale);
+            const float bT = store_round(biases, gi, dtype, lo);
+            for (long long k = g0; k < g0 + group; ++k) {
+                uint32_t q = 0;
+                if (sT != 0.0f) {
+                    const float d = (load_f32(w, (size_t)(n * K + k), dtype) - bT) / sT;   /* fp32, fp32 */
+                    const float r = rintf(d);
+                    q = r <= 0.0f ? 0u : r >= (float)qmax ? (uint32_t)qmax : (uint32_t)r;
+                }
+                put_code(row, k, bits, q);
+            }
+        }
+    }
+}

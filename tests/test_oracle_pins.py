@@ -15,7 +15,11 @@ the oracle fails at least one of them:
   product          exact Fraction brute force on tiny shapes (affine and FP),
                    the all-zero-code closed form, x = e_k selects a column;
   sum(x)           the emulated low-precision sum(x) mutant fails the test
-                   tolerance on the precision case, the widened sum passes.
+                   tolerance on the precision case, the widened sum passes;
+  quantizer        fp32 -> binary16 / bfloat16 rounding vs numpy / torch; codes
+                   of weights on an exact grid recovered bit for bit for every
+                   width (through the pinned unpack); a constant group; brute
+                   force nearest code in exact rationals.
 """
 from __future__ import annotations
 
@@ -377,3 +381,91 @@ def test_low_precision_sum_x_fails_tolerance():
     ok_bad, _ = check(_emulate_kernel_bf16(case, False)[None, :], y_ref, absdot, "bf16")
     assert ok_good.all()
     assert (~ok_bad).sum() >= 10, int((~ok_bad).sum())
+
+
+# ------------------------------------------------------------- quantizer ----
+def _f32_specials():
+    rng = np.random.default_rng(77)
+    v = np.concatenate([
+        rng.standard_normal(4000).astype(np.float32) * np.float32(3.0),
+        (rng.standard_normal(2000) * 1e-5).astype(np.float32),           # binary16 subnormal range
+        np.array([0.0, -0.0, 1.0, -1.0, 65504.0, 65519.0, 65520.0, 6e-8, 2.0 ** -24, 2.0 ** -25,
+                  1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8], dtype=np.float32),
+    ])
+    # exact ties of the binary16 / bfloat16 grids
+    base = rng.integers(0, 1 << 10, 500).astype(np.uint32)
+    ties16 = np.array([(1.0 + (b + 0.5) / 1024.0) for b in base], dtype=np.float32)
+    tiesbf = ((rng.integers(0x3F80, 0x4080, 500).astype(np.uint32) << 16) | 0x8000).view(np.float32)
+    return np.concatenate([v, ties16, tiesbf])
+
+
+def test_f32_to_f16_matches_numpy():
+    for v in _f32_specials():
+        assert oracle.f32_to_f16(v) == int(np.float32(v).astype(np.float16).view(np.uint16)), v
+
+
+def test_f32_to_bf16_matches_torch():
+    v = _f32_specials()
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    got = np.array([oracle.f32_to_bf16(x) for x in v], dtype=np.uint16)
+    assert np.array_equal(got, ref)
+
+
+def _bits_of(a, dtype):
+    if dtype == "f32":
+        return np.asarray(a, dtype=np.float32)
+    if dtype == "f16":
+        return np.asarray(a, dtype=np.float32).astype(np.float16).view(np.uint16)
+    return torch.from_numpy(np.asarray(a, dtype=np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_quantize_exact_grid_recovers_codes(bits, dtype):
+    """Weights bias + q * scale with scale a power of two, every code present in
+    each group: min = bias, max = bias + (2^b - 1) scale, so the quantizer must
+    return exactly that scale, that bias and the codes q (read back through the
+    pinned unpack)."""
+    rng = np.random.default_rng(bits * 10 + len(dtype))
+    qmax = (1 << bits) - 1
+    group, N = 64, 3
+    K = 4 * group
+    q = rng.integers(0, qmax + 1, (N, K))
+    q[:, ::group] = 0
+    q[:, 1::group] = qmax
+    scale, bias = 2.0 ** -3, -1.5
+    w = (bias + q * scale).astype(np.float32)
+    wq, sc, bi = oracle.quantize_affine(_bits_of(w, dtype), N, K, bits, group, dtype)
+    assert np.array_equal(sc, np.full_like(sc, _bits_of([scale], dtype)[0]))
+    assert np.array_equal(bi, np.full_like(bi, _bits_of([bias], dtype)[0]))
+    for n in range(N):
+        assert np.array_equal(oracle.affine_codes(wq[n], K, bits), q[n].astype(np.uint32))
+
+
+def test_quantize_constant_group():
+    w = np.full((1, 32), 0.7, dtype=np.float32)
+    wq, sc, bi = oracle.quantize_affine(w, 1, 32, 4, 32, "f32")
+    assert sc[0, 0] == 0.0 and bi[0, 0] == np.float32(0.7) and not wq.any()
+
+
+@pytest.mark.parametrize("bits", [3, 4, 8])
+def test_quantize_nearest_code_brute_force(bits):
+    """Each code is the nearest of the 2^b grid points bias_T + q scale_T to w
+    (exact rationals), except where the distance to two grid points is equal
+    within fp32 rounding of (w - bias_T) / scale_T."""
+    rng = np.random.default_rng(bits)
+    group, N, K = 32, 4, 64
+    w = (rng.standard_normal((N, K)) * 0.3).astype(np.float32)
+    wq, sc, bi = oracle.quantize_affine(w, N, K, bits, group, "f32")
+    qmax = (1 << bits) - 1
+    for n in range(N):
+        codes = oracle.affine_codes(wq[n], K, bits)
+        for k in range(K):
+            s = Fraction(float(sc[n, k // group])); b = Fraction(float(bi[n, k // group]))
+            x = Fraction(float(w[n, k]))
+            d = [abs(x - (b + s * c)) for c in range(qmax + 1)]
+            best = min(d)
+            got = d[int(codes[k])]
+            if got != best:
+                assert float(got - best) <= 1e-6 * float(s), (n, k, codes[k])
+            assert float(got) <= float(s) / 2 * (1 + 1e-6) or codes[k] in (0, qmax)
