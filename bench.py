@@ -2,7 +2,7 @@
 """Benchmark of the weight-quantized matrix-vector product on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload chain8|layer|probe]
+                    [--workload chain8|layer|probe|quantize]
 
 Prints ONE JSON line (rank 0).  Metric: qmv microseconds per call and achieved
 HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
@@ -15,7 +15,11 @@ HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
   layer             7B-class decode layer, affine 4-bit g64 bf16: QKV 6144x4096,
                     O 4096x4096, gate+up 28672x4096, down 4096x14336, run once at
                     M=1 and once at M=8 (8 calls per step).
-  probe             bandwidth probe, affine 4-bit g64 bf16, N=K=16384, M=1.
+  probe             bandwidth probe, affine 4-bit g64 bf16, N=K=16384, M=1:
+                    three back-to-back calls per step, each on its own weight copy.
+  quantize          the affine quantizer (qmv_quantize_affine) on a bf16
+                    16384 x 16384 matrix -> 4-bit g64 (one call per step; its
+                    metric is the quantizer's microseconds per call).
 
 Timing: W untimed warm-up steps, then K steps.  A step is ONE CUDA graph
 holding every call of the workload (dependent calls linked by programmatic
@@ -310,7 +314,55 @@ class Probe(Layer):
                       "its own 151 MB weight copy"}
 
 
-WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe}
+class Quantize(Layer):
+    """The affine quantizer on the bandwidth-probe matrix: bf16 w [16384,
+    16384] -> 4-bit g64 codes, scales, biases; two weight copies (537 MB each,
+    more than L2) alternate across steps."""
+    name = "affine quantizer, bf16 16384 x 16384 -> 4-bit g64"
+
+    def __init__(self, q, torch, dev):
+        self.q, self.torch = q, torch
+        N = K = 16384
+        g = torch.Generator(device="cpu").manual_seed(4000)
+        w_host = (torch.randn((N, K), generator=g) * 0.05).to(torch.bfloat16).pin_memory()
+        ws = [w_host.to(dev) for _ in range(2)]
+        self.sets = [dict(name="quantize", M=1, N=N, K=K, ws=ws, w_host=w_host,
+                          wq=torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                          sc=torch.empty((N, K // 64), dtype=torch.bfloat16, device=dev),
+                          bi=torch.empty((N, K // 64), dtype=torch.bfloat16, device=dev),
+                          sc_host=torch.empty((N, K // 64), dtype=torch.bfloat16).pin_memory(), it=0)]
+        self.calls_per_step = 1
+
+    def graph_variants(self, s):
+        return len(s["ws"])
+
+    def run_group(self, s, e2e=False, v=0):
+        w = s["ws"][v % len(s["ws"])]
+        if e2e:
+            w.copy_(s["w_host"], non_blocking=True)
+        self.q.qmv_quantize_affine(w, s["wq"], s["sc"], s["bi"], s["N"], s["K"], 4, 64, "bf16")
+        if e2e:
+            s["sc_host"].copy_(s["sc"], non_blocking=True)
+        return 1
+
+    def group_bytes(self, s):
+        N, K = s["N"], s["K"]
+        return N * K * 2 + N * K // 2 + 2 * N * (K // 64) * 2
+
+    def group_plan(self, s):
+        return "path=quantize chunk=64 maxm=0 rows_per_warp=0 bits=4 group=64 dtype=bf16"
+
+    def h2d_d2h(self):
+        s = self.sets[0]
+        return s["N"] * s["K"] * 2, s["N"] * (s["K"] // 64) * 2
+
+    def config(self):
+        return {"workload": self.name, "bits": 4, "group": 64, "dtype": "bf16", "N": 16384, "K": 16384,
+                "calls_per_step": 1, "bytes_per_call": "w read + codes, scales, biases written",
+                "l2": "flushed before every step (512 MB write + 256 MB read); 2 weight copies alternate"}
+
+
+WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe, "quantize": Quantize}
 
 
 # ---------------------------------------------------------------- our arm --
@@ -471,6 +523,8 @@ def _oracle_sample(workload, budget_s=12.0, threads=None):
     import oracle
     threads = threads or os.cpu_count() or 1
     t_by = {}
+    if workload == "quantize":
+        return _oracle_quantize_sample(budget_s, threads)
     if workload == "chain8":
         spec = [(1, N, CHAIN_K, CHAIN_BITS, CHAIN_G, CHAIN_CALLS) for N in CHAIN_NS]
     elif workload == "layer":
@@ -499,6 +553,25 @@ def _oracle_sample(workload, budget_s=12.0, threads=None):
         sample.append(f"M={M} N={N} K={K}: {nrows}/{N} rows, {dt:.3f}s")
     ncalls = sum(s[-1] for s in spec)
     return total_us / ncalls, threads, "; ".join(sample)
+
+
+def _oracle_quantize_sample(budget_s, threads):
+    """The oracle quantizer on a growing row sample of the 16384 x 16384 bf16
+    matrix, scaled to one full call."""
+    import oracle
+    N = K = 16384
+    rng = np.random.default_rng(9)
+    w = rng.standard_normal((N, K), dtype=np.float32).astype(np.float32) * np.float32(0.05)
+    wb = (w.view(np.uint32) >> 16).astype(np.uint16)                 # bf16 bit patterns (truncated sample data)
+    nrows = 16
+    while True:
+        t0 = time.perf_counter()
+        oracle.quantize_affine(np.ascontiguousarray(wb[:nrows]), nrows, K, 4, 64, "bf16", threads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s / 4 or nrows >= N:
+            break
+        nrows = min(N, nrows * 4)
+    return dt * 1e6 * (N / nrows), threads, f"N={N} K={K} 4-bit g64 bf16: {nrows}/{N} rows, {dt:.3f}s"
 
 
 def cpu_baseline(workload):

@@ -120,6 +120,29 @@ int qmv_fp_batched(const void* x, const void* w_packed, const void* scales,
                    int dtype, int batch, int x_batched, void* stream);
 
 /*
+ * qmv_quantize_affine -- affine quantizer (wh-iron kernel-op coverage audit,
+ * "quantized (affine_quantize / affine_dequantize)" row: quantize kernels for
+ * every width; the pages do not state their arithmetic, this is the plainest
+ * reading consistent with w = scale * q + bias, MLX quantized_nax.h).
+ *   w         [N, K] row-major in dtype (finite values)
+ *   w_packed  [N, K*bits/8] bytes out, the layout qmv_affine reads (LSB-first
+ *             packs: 2/4/8-bit 8/bits codes per byte, 3/5-bit 8 codes per 3/5
+ *             bytes, 6-bit 4 codes per 3 bytes)
+ *   scales, biases  [N, K/group_size] in dtype, out
+ * For each group of group_size consecutive weights of a row: bias = min,
+ * scale = (max - min) / (2^bits - 1), both rounded to dtype (to nearest, ties
+ * to even); q = rint((w - bias) / scale) in fp32 with the rounded values,
+ * clamped to [0, 2^bits - 1], and q = 0 when the rounded scale is 0.
+ * bits in {2,3,4,5,6,8}, group_size in {32,64,128}, K % group_size == 0.
+ * Alignment: w, scales, biases to their element size, w_packed to 4 bytes
+ * (QMV_EALIGN otherwise); 16-byte aligned rows of w are read 16 bytes at a
+ * time.  Asynchronous on `stream`; the caller owns every buffer.  Returns
+ * QMV_OK or a status as for qmv_affine.
+ */
+int qmv_quantize_affine(const void* w, void* w_packed, void* scales, void* biases, int N, int K,
+                        int bits, int group_size, int dtype, void* stream);
+
+/*
  * qmv_dequant_affine_f32 -- check kernel: w_out[n*K + k] = fp32 value of
  * scale * q + bias, computed with one rounding (fmaf) from the stored dtype
  * scale / bias.  Uses the same device decoders as qmv_affine.  w_out is a

@@ -186,3 +186,18 @@ def test_build_module_loads_without_the_library(tmp_path):
     )
     r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=str(tmp_path))
     assert r.returncode == 0, r.stderr
+
+
+def test_quantize_validation_before_any_launch():
+    """Argument errors of the quantizer come back as statuses before any CUDA
+    call (host-side checks; fake device pointers are never dereferenced)."""
+    F = FAKE
+    assert L.qmv_quantize_affine(F, F, F, F, 8, 128, 7, 64, 2, None) == EUNSUP       # bits
+    assert L.qmv_quantize_affine(F, F, F, F, 8, 128, 4, 48, 2, None) == EUNSUP       # group
+    assert L.qmv_quantize_affine(F, F, F, F, 8, 128, 4, 64, 5, None) == EUNSUP       # dtype
+    assert L.qmv_quantize_affine(F, F, F, F, 8, 100, 4, 64, 2, None) == EINVAL       # K % group
+    assert L.qmv_quantize_affine(F, F, F, F, -1, 128, 4, 64, 2, None) == EINVAL      # N < 0
+    assert L.qmv_quantize_affine(None, F, F, F, 8, 128, 4, 64, 2, None) == EINVAL    # null
+    assert L.qmv_quantize_affine(F + 1, F, F, F, 8, 128, 4, 64, 2, None) == EALIGN   # w alignment
+    assert L.qmv_quantize_affine(F, F + 2, F, F, 8, 128, 4, 64, 2, None) == EALIGN   # packed alignment
+    assert L.qmv_quantize_affine(F, F, F, F, 0, 128, 4, 64, 2, None) == 0            # empty: nothing to do

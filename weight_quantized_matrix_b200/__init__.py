@@ -18,7 +18,8 @@ import os
 
 __all__ = [
     "QmvError", "qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
-    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_status_string", "qmv_last_cuda_error",
+    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_status_string",
+    "qmv_last_cuda_error",
     "qmv_describe_plan", "qmv_force_config", "DTYPES", "FP_MODES", "LIB_PATH", "lib",
 ]
 
@@ -53,6 +54,7 @@ _lib.qmv_fp.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 _lib.qmv_fp_batched.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p]
 _lib.qmv_dequant_affine_f32.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 _lib.qmv_dequant_fp_f32.argtypes = [_p, _p, _p, _p, _i, _i, _i, _p]
+_lib.qmv_quantize_affine.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 _lib.qmv_status_string.argtypes = [_i]
 _lib.qmv_status_string.restype = ctypes.c_char_p
 _lib.qmv_last_cuda_error.argtypes = []
@@ -61,8 +63,8 @@ _lib.qmv_device_fault.argtypes = [ctypes.POINTER(ctypes.c_uint), _i]
 _lib.qmv_force_config.argtypes = [_i, _i, _i, _i]
 _lib.qmv_force_config.restype = None
 for _f in ("qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
-           "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_last_cuda_error", "qmv_describe_plan",
-           "qmv_device_fault"):
+           "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_last_cuda_error",
+           "qmv_describe_plan", "qmv_device_fault"):
     getattr(_lib, _f).restype = _i
 
 
@@ -161,6 +163,14 @@ def qmv_dequant_affine_f32(w_packed, scales, biases, w_out, N, K, bits, group_si
 def qmv_dequant_fp_f32(w_packed, scales, global_scale, w_out, N, K, mode, stream=None):
     _check(_lib.qmv_dequant_fp_f32(_ptr(w_packed), _ptr(scales), _ptr(global_scale), _ptr(w_out), N, K,
                                    _mode(mode), _stream(stream)), "qmv_dequant_fp_f32")
+
+
+def qmv_quantize_affine(w, w_packed, scales, biases, N, K, bits, group_size, dtype, stream=None):
+    """Affine quantizer (C ABI qmv_quantize_affine): w [N, K] in dtype ->
+    packed codes [N, K*bits/8] bytes, scales and biases [N, K/group_size] in
+    dtype, all caller-owned device buffers."""
+    _check(_lib.qmv_quantize_affine(_ptr(w), _ptr(w_packed), _ptr(scales), _ptr(biases), N, K, bits,
+                                    group_size, _dtype(dtype), _stream(stream)), "qmv_quantize_affine")
 
 
 def qmv_status_string(status: int) -> str:

@@ -783,6 +783,21 @@ int qmv_dequant_fp_f32(const void* w_packed, const void* scales, const float* gl
                                       (long long)K * bits / 8, static_cast<cudaStream_t>(stream)));
 }
 
+int qmv_quantize_affine(const void* w, void* w_packed, void* scales, void* biases, int N, int K, int bits,
+                        int group_size, int dtype, void* stream) {
+    int st = check_affine(bits, group_size);
+    if (st != QMV_OK) return st;
+    if (dtype != QMV_F32 && dtype != QMV_F16 && dtype != QMV_BF16) return QMV_EUNSUPPORTED;
+    if (N < 0 || K < 0 || K % group_size != 0) return QMV_EINVAL;
+    if (N == 0 || K == 0) return QMV_OK;
+    if (!w || !w_packed || !scales || !biases) return QMV_EINVAL;
+    const size_t eb = elem_bytes(dtype);
+    if (!aligned(w, eb) || !aligned(w_packed, 4) || !aligned(scales, eb) || !aligned(biases, eb)) return QMV_EALIGN;
+    const int vec = (aligned(w, 16) && ((size_t)K * eb) % 16 == 0) ? 1 : 0;
+    return finish(qmv::launch_quantize_affine(bits, dtype, w, w_packed, scales, biases, N, K, group_size, vec,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 const char* qmv_status_string(int status) {
     switch (status) {
         case QMV_OK: return "ok";

@@ -75,6 +75,11 @@ cudaError_t launch_tcf_affine(int bits, int ncw, const Params& p, const Launch& 
 // 16-byte unit loads (4- and 8-bit codes, 16-byte aligned rows).
 cudaError_t launch_direct(int fam, int bits, int dtype, int maxm, bool wide, const Params& p, const Launch& L);
 
+// Affine quantizer (qmv_quantize.cu): w [N, K] in dtype -> packed codes,
+// scales, biases; vec = 16-byte loads of w (aligned rows).
+cudaError_t launch_quantize_affine(int bits, int dtype, const void* w, void* wq, void* scales, void* biases,
+                                   int N, int K, int G, int vec, cudaStream_t st);
+
 cudaError_t launch_dequant(int fam, int bits, int dtype, const uint8_t* w, const void* scales,
                            const void* biases, const float* gscale, float* out, int N, int K, int G,
                            long long w_row, cudaStream_t s);
