@@ -131,8 +131,9 @@ int qmv_fp_batched(const void* x, const void* w_packed, const void* scales,
  *   scales, biases  [N, K/group_size] in dtype, out
  * For each group of group_size consecutive weights of a row: bias = min,
  * scale = (max - min) / (2^bits - 1), both rounded to dtype (to nearest, ties
- * to even); q = rint((w - bias) / scale) in fp32 with the rounded values,
- * clamped to [0, 2^bits - 1], and q = 0 when the rounded scale is 0.
+ * to even); inv = 1 / scale and q = rint((w - bias) * inv), in fp32 with the
+ * rounded values, clamped to [0, 2^bits - 1]; q = 0 when the rounded scale
+ * is 0.
  * bits in {2,3,4,5,6,8}, group_size in {32,64,128}, K % group_size == 0.
  * Alignment: w, scales, biases to their element size, w_packed to 4 bytes
  * (QMV_EALIGN otherwise); 16-byte aligned rows of w are read 16 bytes at a

@@ -286,11 +286,15 @@ uint32_t oracle_f32_to_f16(float f) {
  * (MLX quantized_nax.h, dequantize): for each group of `group` consecutive
  * weights of a row,
  *     bias  = min(w),  scale = (max(w) - min(w)) / (2^bits - 1),
- * both rounded to the element type, and
- *     q = nearest integer, ties to even, to (w - bias_T) / scale_T,
- * clamped to [0, 2^bits - 1] (q = 0 when scale_T is 0).  Every step that
- * decides a code is one fp32 IEEE operation (subtract, divide, round), the
- * precision the CUDA kernel takes the same decision in.  Codes are packed
+ * both rounded to the element type, inv = 1 / scale_T, and
+ *     q = nearest integer, ties to even, to (w - bias_T) * inv,
+ * clamped to [0, 2^bits - 1] (q = 0 when scale_T is 0, and when the
+ * quotient is NaN: a zero difference times the infinite reciprocal of a
+ * scale below 2^-128).  min and max are taken in element order with strict
+ * comparisons, so of +0 and -0 the first one met is kept.  Weights are
+ * finite.  Every step that decides a code is one fp32 IEEE operation (divide
+ * once per group, then subtract, multiply, round per weight), the precision
+ * the CUDA kernel takes the same decision in.  Codes are packed
  * LSB first exactly as oracle_affine_code reads them.  Rows [n0, n1).
  * ------------------------------------------------------------------------- */
 static float load_f32(const void* p, size_t i, int dtype) {
@@ -332,12 +336,14 @@ void oracle_quantize_affine(const void* w, uint8_t* wq, void* scales, void* bias
             const size_t gi = (size_t)(n * (K / group) + g0 / group);
             const float sT = store_round(scales, gi, dtype, scale);
             const float bT = store_round(biases, gi, dtype, lo);
+            const float inv = sT != 0.0f ? 1.0f / sT : 0.0f;   /* fp32 */
             for (long long k = g0; k < g0 + group; ++k) {
                 uint32_t q = 0;
                 if (sT != 0.0f) {
-                    const float d = (load_f32(w, (size_t)(n * K + k), dtype) - bT) / sT;   /* fp32, fp32 */
-                    const float r = rintf(d);
-                    q = r <= 0.0f ? 0u : r >= (float)qmax ? (uint32_t)qmax : (uint32_t)r;
+                    const float d = (load_f32(w, (size_t)(n * K + k), dtype) - bT) * inv;  /* fp32, fp32 */
+                    /* clamp, then round to nearest even; a NaN quotient (a zero
+                       difference times an infinite reciprocal) is code 0 */
+                    q = !(d > 0.0f) ? 0u : d >= (float)qmax ? (uint32_t)qmax : (uint32_t)rintf(d);
                 }
                 put_code(row, k, bits, q);
             }

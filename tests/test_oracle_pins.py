@@ -442,6 +442,28 @@ def test_quantize_exact_grid_recovers_codes(bits, dtype):
         assert np.array_equal(oracle.affine_codes(wq[n], K, bits), q[n].astype(np.uint32))
 
 
+def test_quantize_signed_zero_extremes_keep_the_first_met():
+    """min / max by strict comparisons in element order: of +0 and -0 the first
+    one met is the bias (or the maximum), whatever follows."""
+    w = np.zeros((2, 32), dtype=np.float32)
+    w[0, :] = np.arange(32) * 0.5
+    w[0, 3] = -0.0                       # +0 at 0 comes first: bias +0
+    w[1, :] = np.arange(32) * 0.5
+    w[1, 0] = -0.0                       # -0 first: bias -0
+    _, _, bi = oracle.quantize_affine(w, 2, 32, 4, 32, "f32")
+    assert np.signbit(bi[1, 0]) and not np.signbit(bi[0, 0])
+
+
+def test_quantize_infinite_reciprocal():
+    """A subnormal range: scale below 2^-128, 1 / scale = inf; the weight equal
+    to the bias (0 * inf = NaN) is code 0, every larger weight the top code."""
+    w = (np.arange(32, dtype=np.float32) * np.float32(1e-41)).reshape(1, 32)
+    wq, sc, bi = oracle.quantize_affine(w, 1, 32, 4, 32, "f32")
+    assert 0 < sc[0, 0] < 2.0 ** -128 and bi[0, 0] == 0.0
+    codes = oracle.affine_codes(wq[0], 32, 4)
+    assert codes[0] == 0 and (codes[1:] == 15).all()
+
+
 def test_quantize_constant_group():
     w = np.full((1, 32), 0.7, dtype=np.float32)
     wq, sc, bi = oracle.quantize_affine(w, 1, 32, 4, 32, "f32")
@@ -452,7 +474,7 @@ def test_quantize_constant_group():
 def test_quantize_nearest_code_brute_force(bits):
     """Each code is the nearest of the 2^b grid points bias_T + q scale_T to w
     (exact rationals), except where the distance to two grid points is equal
-    within fp32 rounding of (w - bias_T) / scale_T."""
+    within fp32 rounding of (w - bias_T) * (1 / scale_T)."""
     rng = np.random.default_rng(bits)
     group, N, K = 32, 4, 64
     w = (rng.standard_normal((N, K)) * 0.3).astype(np.float32)

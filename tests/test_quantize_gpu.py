@@ -1,7 +1,8 @@
 """GPU parity of the affine quantizer (qmv_quantize_affine) against the oracle.
 
 The packed codes, scales and biases are integers and bit patterns decided by
-the same fp32 operations on both sides (min / max, subtract, divide, round to
+the same fp32 operations on both sides (min / max, subtract, a reciprocal per
+group and a multiply per weight, round to
 nearest even, round to the element type), so every byte must match exactly.
 """
 from __future__ import annotations
@@ -80,16 +81,26 @@ def test_quantize_unaligned_rows_take_the_scalar_path(q, dtype):
 
 @pytest.mark.parametrize("dtype", DTYPES)
 def test_quantize_special_groups(q, dtype):
-    """Constant groups (scale 0, codes 0), groups of +0 / -0, a tiny range
-    (subnormal-sized scale), exact ties of the code grid."""
-    N, K, group, bits = 4, 256, 64, 4
+    """Constant groups (scale 0, codes 0), groups of +0 / -0 in both orders
+    and with a zero minimum or maximum, a tiny range, exact ties of the code
+    grid, a subnormal range whose scale has an infinite reciprocal."""
+    N, K, group, bits = 5, 256, 64, 4
     w = np.zeros((N, K), dtype=np.float32)
     w[0, :64] = 0.75                                   # constant
     w[0, 64:128] = np.where(np.arange(64) % 2 == 0, 0.0, -0.0)
+    w[0, 128:192] = np.where(np.arange(64) % 2 == 0, -0.0, 0.0)
+    w[0, 192:256] = -np.arange(64, dtype=np.float32) * 0.25     # max 0 first ...
+    w[0, 200] = -0.0                                          # ... then -0
     w[1, :64] = 1.0 + np.arange(64, dtype=np.float32) * np.float32(2.0 ** -20)    # tiny range
+    w[1, 64:128] = np.arange(64, dtype=np.float32) * 0.125     # min 0 first
+    w[1, 70] = -0.0
+    w[1, 128:192] = np.arange(64, dtype=np.float32) * 0.125
+    w[1, 128] = -0.0                                          # min -0 first, +0 later
+    w[1, 150] = 0.0
     w[2, :64] = np.arange(64, dtype=np.float32) % 31 * 0.5                       # ties: (w - 0) / 1.0
     rng = np.random.default_rng(5)
     w[3] = rng.standard_normal(K).astype(np.float32)
+    w[4, :64] = np.arange(64, dtype=np.float32) * np.float32(1e-41)              # subnormal range
     t = torch.from_numpy(w).to({"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[dtype])
     wb = t.view(torch.int32 if dtype == "f32" else torch.int16).numpy().view(STORAGE[dtype]).copy()
     got = _run(q, wb, N, K, bits, group, dtype)

@@ -793,7 +793,9 @@ int qmv_quantize_affine(const void* w, void* w_packed, void* scales, void* biase
     if (!w || !w_packed || !scales || !biases) return QMV_EINVAL;
     const size_t eb = elem_bytes(dtype);
     if (!aligned(w, eb) || !aligned(w_packed, 4) || !aligned(scales, eb) || !aligned(biases, eb)) return QMV_EALIGN;
-    const int vec = (aligned(w, 16) && ((size_t)K * eb) % 16 == 0) ? 1 : 0;
+    // 2: coalesced tiles (w and w_packed 16-byte aligned); 1: 16-byte loads of
+    // w per thread; 0: element loads
+    const int vec = (aligned(w, 16) && ((size_t)K * eb) % 16 == 0) ? (aligned(w_packed, 16) ? 2 : 1) : 0;
     return finish(qmv::launch_quantize_affine(bits, dtype, w, w_packed, scales, biases, N, K, group_size, vec,
                                               static_cast<cudaStream_t>(stream)));
 }
