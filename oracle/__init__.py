@@ -70,6 +70,8 @@ def lib():
         L.oracle_qmv_affine.argtypes = [p, p, p, p, p, p, ll, ll, ll, i, i, i, ll, ll]
         L.oracle_qmv_affine.restype = None
         L.oracle_qmv_fp.argtypes = [p, p, p, f, p, p, ll, ll, ll, i, i, ll, ll]
+        L.oracle_qvm_affine.argtypes = [p, p, p, p, p, p, ll, ll, ll, i, i, i, ll, ll]
+        L.oracle_qvm_affine.restype = None
         L.oracle_qmv_fp.restype = None
         L.oracle_f32_to_bf16.argtypes = [f]; L.oracle_f32_to_bf16.restype = u
         L.oracle_f32_to_f16.argtypes = [f]; L.oracle_f32_to_f16.restype = u
@@ -164,6 +166,18 @@ def qmv_affine(x, w, scales, biases, M, N, K, bits, group, dtype, rows=None, thr
     fn = lambda r0, r1: L.oracle_qmv_affine(_ptr(x), _ptr(w), _ptr(scales), _ptr(biases), _ptr(y),
                                             _ptr(a), M, N, K, bits, group, DTYPE_CODES[dtype], r0, r1)
     _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
+    return y, a
+
+
+def qvm_affine(x, w, scales, biases, M, N, K, bits, group, dtype, cols=None, threads=1):
+    """x [M, K] times W stored [K, N] (packed rows of N codes, scales and
+    biases [K, N / group]).  Return (y, absdot), both float64 [M, N]; columns
+    not requested stay NaN."""
+    y = np.full((M, N), np.nan); a = np.full((M, N), np.nan)
+    L = lib()
+    fn = lambda c0, c1: L.oracle_qvm_affine(_ptr(x), _ptr(w), _ptr(scales), _ptr(biases), _ptr(y),
+                                            _ptr(a), M, N, K, bits, group, DTYPE_CODES[dtype], c0, c1)
+    _run(fn, _ranges(range(N) if cols is None else cols, threads), threads)
     return y, a
 
 

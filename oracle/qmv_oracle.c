@@ -226,6 +226,33 @@ void oracle_qmv_affine(const void* x, const uint8_t* w, const void* scales, cons
         }
 }
 
+/* ---------------------------------------------------------------------------
+ * qvm: x times a weight matrix stored [K, N] (MLX quantized_nax.h, qouter,
+ * the outer-product accumulate result[j] += x * (scale * q_j + bias); the
+ * wh-iron audit's qvm family, "x.W with W [K, N]").  Row k of w packs the N
+ * codes of the output columns LSB first exactly like a qmv row, with scales
+ * and biases [K, N / group] grouped along N:
+ *     y[m, n] = sum_k x[m, k] * (scale[k, n/group] * q[k, n] + bias[k, n/group])
+ * Products and sum in fp64 as in oracle_qmv_affine.  Columns [n0, n1).
+ * ------------------------------------------------------------------------- */
+void oracle_qvm_affine(const void* x, const uint8_t* w, const void* scales, const void* biases,
+                       double* y, double* absdot, long long M, long long N, long long K,
+                       int bits, int group, int dtype, long long n0, long long n1) {
+    for (long long n = n0; n < n1; ++n)
+        for (long long m = 0; m < M; ++m) {
+            double acc = 0.0, aacc = 0.0;
+            for (long long k = 0; k < K; ++k) {
+                /* element (k, n): row k, position n of a row of N codes */
+                double t = load_elem(x, (size_t)(m * K + k), dtype) *
+                           affine_w(w, scales, biases, k, n, N, bits, group, dtype);
+                acc += t;
+                aacc += fabs(t);
+            }
+            y[m * N + n] = acc;
+            if (absdot) absdot[m * N + n] = aacc;
+        }
+}
+
 void oracle_qmv_fp(const void* x, const uint8_t* w, const uint8_t* scales, float global,
                    double* y, double* absdot, long long M, long long N, long long K,
                    int mode, int dtype, long long n0, long long n1) {

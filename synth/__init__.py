@@ -73,6 +73,26 @@ def affine_case(M, N, K, bits, group, dtype, seed, batch=1, precision=False):
     }
 
 
+def qvm_case(M, N, K, bits, group, dtype, seed, precision=False):
+    """One qvm problem (W stored [K, N], grouped along N).  x [M, K], w
+    [K, N*bits/8] u8, scales / biases [K, N/group]; x, scales and biases are
+    raw storage of ``dtype``.  Same value distributions as affine_case."""
+    g = rng(seed)
+    if precision:
+        x = g.uniform(1e-4, 1e-3, size=(M, K))
+    else:
+        x = g.standard_normal(size=(M, K))
+    w = random_bytes(g, (K, N * bits // 8))
+    s = g.uniform(0.005, 0.02, size=(K, N // group))
+    s_raw = to_storage(s, dtype)
+    if precision:
+        b = -storage_to_float(s_raw, dtype).astype(np.float64) * ((2 ** bits - 1) / 2.0)
+    else:
+        b = g.normal(0.0, 0.01, size=(K, N // group))
+    return {"x": to_storage(x, dtype), "w": w, "scales": s_raw, "biases": to_storage(b, dtype),
+            "M": M, "N": N, "K": K, "bits": bits, "group": group, "dtype": dtype}
+
+
 FP_BLOCK = {"mxfp4": 32, "nvfp4": 16, "mxfp8": 32}
 FP_BITS = {"mxfp4": 4, "nvfp4": 4, "mxfp8": 8}
 _E4M3_NON_NAN = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)

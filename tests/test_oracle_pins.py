@@ -348,6 +348,63 @@ def test_unit_x_selects_column(bits):
             assert y[0, n] == want
 
 
+# ------------------------------------------------------------- qvm pins ----
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_qvm_equals_qmv_of_the_transpose(bits, dtype):
+    """qvm over W stored [K, N] equals qmv over W^T stored [N, K].  The test
+    transposes the codes with its own bit-stream reader and writer.  qvm's
+    scales and biases are drawn constant over blocks of 32 rows, so W^T's
+    parameters fit qmv's [N, K/32] layout: p^T[n, kb] = p[32 kb, n / group].
+    Both sums run over k in order on the same fp64 terms: equal bit for bit."""
+    M, N, K, group = 2, 128, 96, 64
+    c = synth.qvm_case(M, N, K, bits, group, dtype, seed=bits)
+    sc = np.repeat(c["scales"][::32], 32, axis=0).copy()
+    bi = np.repeat(c["biases"][::32], 32, axis=0).copy()
+    y, a = oracle.qvm_affine(c["x"], c["w"], sc, bi, M, N, K, bits, group, dtype)
+    codes = np.array([_py_codes(c["w"][k], N, bits) for k in range(K)])      # [K, N]
+    wt = np.stack([_py_pack(codes[:, n], bits) for n in range(N)])          # [N, K*bits/8]
+    cols = np.arange(N) // group
+    sct = np.ascontiguousarray(sc[::32][:, cols].T)                          # [N, K/32]
+    bit = np.ascontiguousarray(bi[::32][:, cols].T)
+    yt, at = oracle.qmv_affine(c["x"], wt, sct, bit, M, N, K, bits, 32, dtype)
+    assert np.array_equal(y, yt) and np.array_equal(a, at)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 5, 8])
+def test_qvm_unit_x_selects_row(bits):
+    """x = e_k: y[0, n] = scale[k, n/g] * q[k, n] + bias[k, n/g] (codes from the
+    test-side reader, values from library casts)."""
+    N, K, group = 96, 40, 32
+    c = synth.qvm_case(1, N, K, bits, group, "f32", seed=11)
+    for k in (0, 1, 17, 39):
+        x = np.zeros((1, K), dtype=np.float32); x[0, k] = 1.0
+        y, _ = oracle.qvm_affine(x, c["w"], c["scales"], c["biases"], 1, N, K, bits, group, "f32")
+        q = _py_codes(c["w"][k], N, bits)
+        for n in range(N):
+            want = float(c["scales"][k, n // group]) * q[n] + float(c["biases"][k, n // group])
+            assert y[0, n] == want, (k, n)
+
+
+@pytest.mark.parametrize("bits", [3, 4, 6])
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_qvm_exact_bruteforce(bits, dtype):
+    """Random per-(k, group) scales and biases: y against exact rationals."""
+    M, N, K, group = 2, 64, 24, 32
+    c = synth.qvm_case(M, N, K, bits, group, dtype, seed=bits + 50)
+    y, absdot = oracle.qvm_affine(c["x"], c["w"], c["scales"], c["biases"], M, N, K, bits, group, dtype)
+    xv, sv, bv = _val(c["x"], dtype), _val(c["scales"], dtype), _val(c["biases"], dtype)
+    codes = [_py_codes(c["w"][k], N, bits) for k in range(K)]
+    for m in range(M):
+        for n in range(0, N, 7):
+            acc = Fraction(0); aacc = Fraction(0)
+            for k in range(K):
+                t = Fraction(xv[m, k]) * (Fraction(sv[k, n // group]) * codes[k][n] + Fraction(bv[k, n // group]))
+                acc += t; aacc += abs(t)
+            assert abs(Fraction(y[m, n]) - acc) <= aacc * Fraction(2) ** -40
+            assert abs(Fraction(absdot[m, n]) - aacc) <= aacc * Fraction(2) ** -40
+
+
 # ------------------------------------------------------------ sum(x) pin ----
 def _emulate_kernel_bf16(case, widened):
     """fp32 emulation of a qmv whose bias term uses sum(x) per group, either
