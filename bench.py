@@ -2,7 +2,7 @@
 """Benchmark of the weight-quantized matrix-vector product on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload chain8|layer|probe|quantize]
+                    [--workload chain8|layer|probe|quantize|qvm]
 
 Prints ONE JSON line (rank 0).  Metric: qmv microseconds per call and achieved
 HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
@@ -20,6 +20,9 @@ HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
   quantize          the affine quantizer (qmv_quantize_affine) on a bf16
                     16384 x 16384 matrix -> 4-bit g64 (one call per step; its
                     metric is the quantizer's microseconds per call).
+  qvm               x times W stored [K, N] (qmv_qvm_affine), affine 4-bit g64
+                    bf16, N=K=16384, M=1, with the K-split workspace: three
+                    back-to-back calls per step, each on its own weight copy.
 
 Timing: W untimed warm-up steps, then K steps.  A step is ONE CUDA graph
 holding every call of the workload (dependent calls linked by programmatic
@@ -362,7 +365,58 @@ class Quantize(Layer):
                 "l2": "flushed before every step (512 MB write + 256 MB read); 2 weight copies alternate"}
 
 
-WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe, "quantize": Quantize}
+class Qvm(Layer):
+    """qvm on the bandwidth-probe matrix stored [K, N]: x [1, 16384] times
+    4-bit g64 W [16384, 16384], bf16, with the K-split workspace; each step
+    makes CALLS calls, one on each of CALLS distinct weight copies (151 MB
+    each, more than L2), back to back."""
+    name = "qvm, affine 4-bit g64 bf16, W stored [K, N], N=K=16384, M=1"
+    CALLS = 3
+
+    def __init__(self, q, torch, dev):
+        self.q, self.torch = q, torch
+        N = K = 16384
+        c = synth.qvm_case(1, N, K, 4, 64, "bf16", seed=3100)
+        ws = [tuple(torch.from_numpy(np.ascontiguousarray(a).view(np.uint8).reshape(-1)).to(dev)
+                    for a in (c["w"], c["scales"], c["biases"])) for _ in range(self.CALLS)]
+        x_host = torch.from_numpy(c["x"].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+        self.sets = [dict(name="qvm", M=1, N=N, K=K, ws=ws, x=x_host.to(dev), x_host=x_host,
+                          work=torch.zeros(q.qmv_qvm_workspace_bytes(1, N), dtype=torch.uint8, device=dev),
+                          y=torch.empty((1, N), dtype=torch.bfloat16, device=dev),
+                          y_host=torch.empty((1, N), dtype=torch.bfloat16).pin_memory(), it=0)]
+        self.calls_per_step = self.CALLS
+
+    def graph_variants(self, s):
+        return 1
+
+    def run_group(self, s, e2e=False, v=0):
+        if e2e:
+            s["x"].copy_(s["x_host"], non_blocking=True)
+        for c in range(self.CALLS):
+            w, sc, bi = s["ws"][c]
+            self.q.qmv_qvm_affine(s["x"], w, sc, bi, s["y"], 1, s["N"], s["K"], 4, 64, "bf16", workspace=s["work"])
+        if e2e:
+            s["y_host"].copy_(s["y"], non_blocking=True)
+        return self.CALLS
+
+    def group_bytes(self, s):
+        return affine_bytes(1, s["N"], s["K"], 4, 64) * self.CALLS
+
+    def group_plan(self, s):
+        return "path=qvm chunk=32 maxm=1 rows_per_warp=0 bits=4 group=64 dtype=bf16"
+
+    def h2d_d2h(self):
+        s = self.sets[0]
+        return s["K"] * 2, s["N"] * 2
+
+    def config(self):
+        return {"workload": self.name, "bits": 4, "group": 64, "dtype": "bf16", "M": 1, "N": 16384, "K": 16384,
+                "calls_per_step": self.CALLS,
+                "l2": "flushed before every step (512 MB write + 256 MB read); each of the step's 3 calls reads "
+                      "its own 151 MB weight copy"}
+
+
+WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe, "quantize": Quantize, "qvm": Qvm}
 
 
 # ---------------------------------------------------------------- our arm --
@@ -525,6 +579,8 @@ def _oracle_sample(workload, budget_s=12.0, threads=None):
     t_by = {}
     if workload == "quantize":
         return _oracle_quantize_sample(budget_s, threads)
+    if workload == "qvm":
+        return _oracle_qvm_sample(budget_s, threads)
     if workload == "chain8":
         spec = [(1, N, CHAIN_K, CHAIN_BITS, CHAIN_G, CHAIN_CALLS) for N in CHAIN_NS]
     elif workload == "layer":
@@ -553,6 +609,24 @@ def _oracle_sample(workload, budget_s=12.0, threads=None):
         sample.append(f"M={M} N={N} K={K}: {nrows}/{N} rows, {dt:.3f}s")
     ncalls = sum(s[-1] for s in spec)
     return total_us / ncalls, threads, "; ".join(sample)
+
+
+def _oracle_qvm_sample(budget_s, threads):
+    """The oracle qvm on a growing column sample of the 16384 x 16384 4-bit
+    matrix, scaled to one full call."""
+    import oracle
+    N = K = 16384
+    c = synth.qvm_case(1, N, K, 4, 64, "bf16", seed=3100)
+    args = (c["x"], c["w"], c["scales"], c["biases"], 1, N, K, 4, 64, "bf16")
+    ncols = 16
+    while True:
+        t0 = time.perf_counter()
+        oracle.qvm_affine(*args, cols=range(ncols), threads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s / 4 or ncols >= N:
+            break
+        ncols = min(N, ncols * 4)
+    return dt * 1e6 * (N / ncols), threads, f"qvm N={N} K={K} 4-bit g64 bf16: {ncols}/{N} columns, {dt:.3f}s"
 
 
 def _oracle_quantize_sample(budget_s, threads):

@@ -47,6 +47,7 @@
 #ifndef QMV_H
 #define QMV_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -142,6 +143,41 @@ int qmv_fp_batched(const void* x, const void* w_packed, const void* scales,
  */
 int qmv_quantize_affine(const void* w, void* w_packed, void* scales, void* biases, int N, int K,
                         int bits, int group_size, int dtype, void* stream);
+
+/*
+ * qmv_qvm_affine -- qvm: x times an affine weight matrix stored [K, N]
+ * (MLX quantized_nax.h, qouter: result[j] += x * (scale * q_j + bias) over a
+ * packed row; the wh-iron audit's qvm family, "x.W with W [K, N]").
+ *   x         [M, K] dtype
+ *   w_packed  [K, N*bits/8] bytes: row k packs the codes of output columns
+ *             0..N-1 exactly like a qmv_affine row (LSB-first packs); 16-byte
+ *             aligned
+ *   scales,   [K, N/group_size] dtype (grouped along N)
+ *   biases
+ *   y         [M, N] dtype
+ *   workspace NULL, or a device buffer of qmv_qvm_workspace_bytes(M, N) bytes,
+ *             16-byte aligned, ALL ZERO before its first use (cudaMemset
+ *             once); every call returns it to zero.  With it, K is split over
+ *             several blocks whose fp32 partial sums meet there (the order of
+ *             that final fp32 sum varies between runs); without it, each 1024
+ *             columns are summed by a single block (few blocks for small N).
+ *             Calls that share a workspace must not overlap on the GPU (one
+ *             stream, or ordered by events).
+ *   bits in {2,3,4,5,6,8}; group_size in {32,64,128}; N % group_size == 0;
+ *   1 <= M <= 8 (0 allowed as a no-op); K >= 0 (K == 0 writes y = 0).
+ * y[m, n] = sum_k x[m,k] * (scale[k, n/group_size] * q[k,n] + bias[k, n/group_size]),
+ * accumulated in fp32 and rounded once to dtype.  Alignment: x, y, scales,
+ * biases to their element (QMV_EALIGN otherwise).  Asynchronous on `stream`;
+ * no programmatic dependent launch.  Returns QMV_OK or a status as for
+ * qmv_affine.
+ */
+int qmv_qvm_affine(const void* x, const void* w_packed, const void* scales, const void* biases,
+                   void* y, int M, int N, int K, int bits, int group_size, int dtype,
+                   void* workspace, void* stream);
+
+/* Bytes of the qmv_qvm_affine workspace for M x rows and N columns (0 for a
+ * negative size).  Host-only. */
+size_t qmv_qvm_workspace_bytes(int M, int N);
 
 /*
  * qmv_dequant_affine_f32 -- check kernel: w_out[n*K + k] = fp32 value of

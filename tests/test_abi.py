@@ -201,3 +201,33 @@ def test_quantize_validation_before_any_launch():
     assert L.qmv_quantize_affine(F + 1, F, F, F, 8, 128, 4, 64, 2, None) == EALIGN   # w alignment
     assert L.qmv_quantize_affine(F, F + 2, F, F, 8, 128, 4, 64, 2, None) == EALIGN   # packed alignment
     assert L.qmv_quantize_affine(F, F, F, F, 0, 128, 4, 64, 2, None) == 0            # empty: nothing to do
+
+
+def test_qvm_validation_before_any_launch():
+    """qvm argument errors come back as statuses before any CUDA call."""
+    F = FAKE
+
+    def qvm(x=F, w=F, s=F, b=F, y=F, M=1, N=128, K=64, bits=4, g=64, dt=2, ws=None):
+        return L.qmv_qvm_affine(x, w, s, b, y, M, N, K, bits, g, dt, ws, None)
+
+    assert qvm(bits=7) == EUNSUP
+    assert qvm(g=48) == EUNSUP
+    assert qvm(dt=5) == EUNSUP
+    assert qvm(N=96) == EINVAL                  # N % group
+    assert qvm(M=9) == EINVAL                   # M > 8
+    assert qvm(K=-1) == EINVAL
+    assert qvm(w=None) == EINVAL
+    assert qvm(y=None) == EINVAL
+    assert qvm(w=F + 4) == EALIGN               # w_packed needs 16 bytes
+    assert qvm(x=F + 1) == EALIGN
+    assert qvm(ws=F + 8) == EALIGN
+    assert qvm(M=0) == 0 and qvm(N=0) == 0      # empty: nothing to do
+
+
+def test_qvm_workspace_size():
+    """fp32 [M, N] partial sums (rounded to 256 bytes) plus one counter per
+    (1024-column tile, x row), also rounded to 256 bytes."""
+    assert q.qmv_qvm_workspace_bytes(1, 16384) == 65536 + 256
+    assert q.qmv_qvm_workspace_bytes(8, 4096) == 131072 + 256
+    assert q.qmv_qvm_workspace_bytes(3, 32) == 512 + 256
+    assert q.qmv_qvm_workspace_bytes(-1, 32) == 0

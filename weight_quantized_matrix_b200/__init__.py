@@ -18,7 +18,8 @@ import os
 
 __all__ = [
     "QmvError", "qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
-    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_status_string",
+    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_qvm_affine",
+    "qmv_qvm_workspace_bytes", "qmv_status_string",
     "qmv_last_cuda_error",
     "qmv_describe_plan", "qmv_force_config", "DTYPES", "FP_MODES", "LIB_PATH", "lib",
 ]
@@ -55,6 +56,9 @@ _lib.qmv_fp_batched.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, 
 _lib.qmv_dequant_affine_f32.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 _lib.qmv_dequant_fp_f32.argtypes = [_p, _p, _p, _p, _i, _i, _i, _p]
 _lib.qmv_quantize_affine.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
+_lib.qmv_qvm_affine.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p]
+_lib.qmv_qvm_workspace_bytes.argtypes = [_i, _i]
+_lib.qmv_qvm_workspace_bytes.restype = ctypes.c_size_t
 _lib.qmv_status_string.argtypes = [_i]
 _lib.qmv_status_string.restype = ctypes.c_char_p
 _lib.qmv_last_cuda_error.argtypes = []
@@ -63,7 +67,8 @@ _lib.qmv_device_fault.argtypes = [ctypes.POINTER(ctypes.c_uint), _i]
 _lib.qmv_force_config.argtypes = [_i, _i, _i, _i]
 _lib.qmv_force_config.restype = None
 for _f in ("qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
-           "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_last_cuda_error",
+           "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_qvm_affine",
+           "qmv_last_cuda_error",
            "qmv_describe_plan", "qmv_device_fault"):
     getattr(_lib, _f).restype = _i
 
@@ -171,6 +176,20 @@ def qmv_quantize_affine(w, w_packed, scales, biases, N, K, bits, group_size, dty
     dtype, all caller-owned device buffers."""
     _check(_lib.qmv_quantize_affine(_ptr(w), _ptr(w_packed), _ptr(scales), _ptr(biases), N, K, bits,
                                     group_size, _dtype(dtype), _stream(stream)), "qmv_quantize_affine")
+
+
+def qmv_qvm_affine(x, w_packed, scales, biases, y, M, N, K, bits, group_size, dtype, workspace=None,
+                   stream=None):
+    """qvm (C ABI qmv_qvm_affine): x [M, K] times W stored [K, N] (w_packed
+    [K, N*bits/8] bytes, scales / biases [K, N/group_size]) -> y [M, N].
+    workspace: None, or a zero-filled device buffer of
+    qmv_qvm_workspace_bytes(M, N) bytes that every call leaves zero."""
+    _check(_lib.qmv_qvm_affine(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(biases), _ptr(y), M, N, K, bits,
+                               group_size, _dtype(dtype), _ptr(workspace), _stream(stream)), "qmv_qvm_affine")
+
+
+def qmv_qvm_workspace_bytes(M, N) -> int:
+    return int(_lib.qmv_qvm_workspace_bytes(M, N))
 
 
 def qmv_status_string(status: int) -> str:

@@ -800,6 +800,28 @@ int qmv_quantize_affine(const void* w, void* w_packed, void* scales, void* biase
                                               static_cast<cudaStream_t>(stream)));
 }
 
+int qmv_qvm_affine(const void* x, const void* w_packed, const void* scales, const void* biases, void* y,
+                   int M, int N, int K, int bits, int group_size, int dtype, void* workspace, void* stream) {
+    int st = check_affine(bits, group_size);
+    if (st != QMV_OK) return st;
+    if (dtype != QMV_F32 && dtype != QMV_F16 && dtype != QMV_BF16) return QMV_EUNSUPPORTED;
+    if (M < 0 || M > QMV_MAX_M || N < 0 || K < 0 || N % group_size != 0) return QMV_EINVAL;
+    if (M == 0 || N == 0) return QMV_OK;
+    if (!y || (K > 0 && (!x || !w_packed || !scales || !biases))) return QMV_EINVAL;
+    const size_t eb = elem_bytes(dtype);
+    if (!aligned(y, eb) || (x && !aligned(x, eb)) || (scales && !aligned(scales, eb)) ||
+        (biases && !aligned(biases, eb)) || (w_packed && !aligned(w_packed, 16)) ||
+        (workspace && !aligned(workspace, 16)))
+        return QMV_EALIGN;
+    return finish(qmv::launch_qvm_affine(bits, dtype, x, w_packed, scales, biases, y, workspace, M, N, K,
+                                         group_size, static_cast<cudaStream_t>(stream)));
+}
+
+size_t qmv_qvm_workspace_bytes(int M, int N) {
+    if (M < 0 || N < 0) return 0;
+    return qmv::qvm_workspace_bytes(M, N);
+}
+
 const char* qmv_status_string(int status) {
     switch (status) {
         case QMV_OK: return "ok";

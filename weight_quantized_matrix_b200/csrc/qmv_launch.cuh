@@ -75,6 +75,12 @@ cudaError_t launch_tcf_affine(int bits, int ncw, const Params& p, const Launch& 
 // 16-byte unit loads (4- and 8-bit codes, 16-byte aligned rows).
 cudaError_t launch_direct(int fam, int bits, int dtype, int maxm, bool wide, const Params& p, const Launch& L);
 
+// qvm (qmv_qvm.cu): x [M, K] times W stored [K, N]; workspace may be null.
+size_t qvm_workspace_bytes(int M, int N);
+cudaError_t launch_qvm_affine(int bits, int dtype, const void* x, const void* w, const void* scales,
+                              const void* biases, void* y, void* workspace, int M, int N, int K, int G,
+                              cudaStream_t st);
+
 // Affine quantizer (qmv_quantize.cu): w [N, K] in dtype -> packed codes,
 // scales, biases; vec = 16-byte loads of w (aligned rows).
 cudaError_t launch_quantize_affine(int bits, int dtype, const void* w, void* wq, void* scales, void* biases,
