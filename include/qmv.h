@@ -180,6 +180,34 @@ int qmv_qvm_affine(const void* x, const void* w_packed, const void* scales, cons
 size_t qmv_qvm_workspace_bytes(int M, int N);
 
 /*
+ * qmv_qvm_affine_noalloc -- qmv_qvm_affine for callers that cannot allocate
+ * device memory.  The pages have no counterpart; this is a library addition.
+ * Some callers must not allocate at all: a plugin whose host framework owns
+ * every device byte through its own pool and forbids driver allocations, or a
+ * latency-critical decode loop that cannot afford the device synchronization
+ * that cudaMalloc / cudaFree may imply.  They cannot hand qmv_qvm_affine a
+ * workspace; this call uses a fixed scratch array of
+ * QMV_QVM_NOALLOC_SCRATCH_BYTES that the library holds on every GPU that
+ * loads it, until the process exits, and allocates nothing.
+ *   Arguments, layouts and result as qmv_qvm_affine without `workspace`.
+ *   Limit: qmv_qvm_workspace_bytes(M, N) <= QMV_QVM_NOALLOC_SCRATCH_BYTES
+ *   (M = 1 with N up to 261888, M = 8 with N up to 32736); larger sizes
+ *   return QMV_EUNSUPPORTED before any launch.
+ *   The first call on a device looks up the scratch's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.  Each call clears the part of the scratch it uses on `stream`,
+ *   then launches.  Every call, on every stream, shares the one array:
+ *   calls that overlap on the GPU race and give wrong results, so order them
+ *   (one stream, or events).
+ *   A failure of the address lookup or of the clearing returns QMV_ECUDA
+ *   without updating qmv_last_cuda_error; a failed kernel launch updates it.
+ */
+#define QMV_QVM_NOALLOC_SCRATCH_BYTES (1u << 20)
+int qmv_qvm_affine_noalloc(const void* x, const void* w_packed, const void* scales,
+                           const void* biases, void* y, int M, int N, int K, int bits,
+                           int group_size, int dtype, void* stream);
+
+/*
  * qmv_dequant_affine_f32 -- check kernel: w_out[n*K + k] = fp32 value of
  * scale * q + bias, computed with one rounding (fmaf) from the stored dtype
  * scale / bias.  Uses the same device decoders as qmv_affine.  w_out is a

@@ -19,7 +19,7 @@ import os
 __all__ = [
     "QmvError", "qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
     "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_qvm_affine",
-    "qmv_qvm_workspace_bytes", "qmv_status_string",
+    "qmv_qvm_workspace_bytes", "qmv_qvm_affine_noalloc", "qmv_status_string",
     "qmv_last_cuda_error",
     "qmv_describe_plan", "qmv_force_config", "DTYPES", "FP_MODES", "LIB_PATH", "lib",
 ]
@@ -186,6 +186,19 @@ def qmv_qvm_affine(x, w_packed, scales, biases, y, M, N, K, bits, group_size, dt
     qmv_qvm_workspace_bytes(M, N) bytes that every call leaves zero."""
     _check(_lib.qmv_qvm_affine(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(biases), _ptr(y), M, N, K, bits,
                                group_size, _dtype(dtype), _ptr(workspace), _stream(stream)), "qmv_qvm_affine")
+
+
+_lib.qmv_qvm_affine_noalloc.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
+_lib.qmv_qvm_affine_noalloc.restype = _i
+
+
+def qmv_qvm_affine_noalloc(x, w_packed, scales, biases, y, M, N, K, bits, group_size, dtype, stream=None):
+    """qvm for callers that cannot allocate device memory (C ABI
+    qmv_qvm_affine_noalloc): as qmv_qvm_affine, with the K-split scratch in a
+    fixed 1 MiB array the library holds; calls that overlap on the GPU race."""
+    _check(_lib.qmv_qvm_affine_noalloc(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(biases), _ptr(y), M, N, K,
+                                       bits, group_size, _dtype(dtype), _stream(stream)),
+           "qmv_qvm_affine_noalloc")
 
 
 def qmv_qvm_workspace_bytes(M, N) -> int:
