@@ -2,7 +2,7 @@
 """Benchmark of the weight-quantized matrix-vector product on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload chain8|layer|probe|quantize|qvm]
+                    [--workload chain8|layer|probe|quantize|qvm|qmm]
 
 Prints ONE JSON line (rank 0).  Metric: qmv microseconds per call and achieved
 HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
@@ -20,6 +20,8 @@ HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
   quantize          the affine quantizer (qmv_quantize_affine) on a bf16
                     16384 x 16384 matrix -> 4-bit g64 (one call per step; its
                     metric is the quantizer's microseconds per call).
+  qmm               small-M qmm (qmv_qmm_affine): the layer's four projections
+                    at M=32 (4 calls per step).
   qvm               x times W stored [K, N] (qmv_qvm_affine), affine 4-bit g64
                     bf16, N=K=16384, M=1, with the K-split workspace: three
                     back-to-back calls per step, each on its own weight copy.
@@ -365,6 +367,45 @@ class Quantize(Layer):
                 "l2": "flushed before every step (512 MB write + 256 MB read); 2 weight copies alternate"}
 
 
+class Qmm(Layer):
+    """Small-M qmm: the 7B-class layer's four projections (4-bit g64 bf16) at
+    M = 32 through qmv_qmm_affine (4 calls per step)."""
+    name = "small-M qmm, 7B-class layer projections, affine 4-bit g64 bf16, M=32"
+    M = 32
+
+    def __init__(self, q, torch, dev):
+        self.q, self.torch = q, torch
+        self.sets = []
+        for name, N, K in LAYER:
+            c = synth.affine_case(self.M, N, K, 4, 64, "bf16", seed=5000 + N + K)
+            per = affine_bytes(self.M, N, K, 4, 64)
+            copies = int(max(1, min(8, np.ceil(2 * L2_BYTES / per))))
+            ws = [tuple(torch.from_numpy(np.ascontiguousarray(a).view(np.uint8).reshape(-1)).to(dev)
+                        for a in (c["w"], c["scales"], c["biases"])) for _ in range(copies)]
+            x_host = torch.from_numpy(c["x"][0].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+            self.sets.append(dict(name=name, M=self.M, N=N, K=K, ws=ws, x=x_host.to(dev), x_host=x_host,
+                                  y=torch.empty((self.M, N), dtype=torch.bfloat16, device=dev),
+                                  y_host=torch.empty((self.M, N), dtype=torch.bfloat16).pin_memory(), it=0))
+        self.calls_per_step = len(self.sets)
+
+    def run_group(self, s, e2e=False, v=0):
+        if e2e:
+            s["x"].copy_(s["x_host"], non_blocking=True)
+        w, sc, bi = s["ws"][v % len(s["ws"])]
+        self.q.qmv_qmm_affine(s["x"], w, sc, bi, s["y"], s["M"], s["N"], s["K"], 4, 64, "bf16")
+        if e2e:
+            s["y_host"].copy_(s["y"], non_blocking=True)
+        return 1
+
+    def group_plan(self, s):
+        return "path=qmm " + self.q.qmv_describe_plan("affine", 8, s["N"], s["K"], 4, 64, "bf16")
+
+    def config(self):
+        return {"workload": self.name, "bits": 4, "group": 64, "dtype": "bf16", "M": self.M,
+                "shapes_NxK": [[n, k] for _, n, k in LAYER], "calls_per_step": self.calls_per_step,
+                "l2": "flushed before every step (512 MB write + 256 MB read); weights rotate through copies > 2x L2"}
+
+
 class Qvm(Layer):
     """qvm on the bandwidth-probe matrix stored [K, N]: x [1, 16384] times
     4-bit g64 W [16384, 16384], bf16, with the K-split workspace; each step
@@ -416,7 +457,7 @@ class Qvm(Layer):
                       "its own 151 MB weight copy"}
 
 
-WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe, "quantize": Quantize, "qvm": Qvm}
+WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe, "quantize": Quantize, "qvm": Qvm, "qmm": Qmm}
 
 
 # ---------------------------------------------------------------- our arm --
@@ -585,6 +626,8 @@ def _oracle_sample(workload, budget_s=12.0, threads=None):
         spec = [(1, N, CHAIN_K, CHAIN_BITS, CHAIN_G, CHAIN_CALLS) for N in CHAIN_NS]
     elif workload == "layer":
         spec = [(M, N, K, 4, 64, 1) for M in (1, 8) for _, N, K in LAYER]
+    elif workload == "qmm":
+        spec = [(32, N, K, 4, 64, 1) for _, N, K in LAYER]
     else:
         spec = [(1, 16384, 16384, 4, 64, 1)]
     per_shape_budget = budget_s / len(spec)

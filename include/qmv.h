@@ -145,6 +145,19 @@ int qmv_quantize_affine(const void* w, void* w_packed, void* scales, void* biase
                         int bits, int group_size, int dtype, void* stream);
 
 /*
+ * qmv_qmm_affine -- small-M quantized matmul, y = x * dequant(W)^T for up to
+ * QMV_QMM_MAX_M x rows (the qmm family of MLX quantized_nax.h and of the
+ * wh-iron audit, M-batched prefill).  Arguments and layouts as qmv_affine,
+ * with 1 <= M <= 64 (0 allowed as a no-op).  The rows run as chunks of
+ * QMV_MAX_M through the qmv_affine kernels, back to back on `stream` (a weight
+ * matrix that fits in L2 is read from HBM once); every argument is checked
+ * before the first launch.  Same accumulation and rounding as qmv_affine.
+ */
+#define QMV_QMM_MAX_M 64
+int qmv_qmm_affine(const void* x, const void* w_packed, const void* scales, const void* biases,
+                   void* y, int M, int N, int K, int bits, int group_size, int dtype, void* stream);
+
+/*
  * qmv_qvm_affine -- qvm: x times an affine weight matrix stored [K, N]
  * (MLX quantized_nax.h, qouter: result[j] += x * (scale * q_j + bias) over a
  * packed row; the wh-iron audit's qvm family, "x.W with W [K, N]").

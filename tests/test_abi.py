@@ -231,3 +231,18 @@ def test_qvm_workspace_size():
     assert q.qmv_qvm_workspace_bytes(8, 4096) == 131072 + 256
     assert q.qmv_qvm_workspace_bytes(3, 32) == 512 + 256
     assert q.qmv_qvm_workspace_bytes(-1, 32) == 0
+
+
+def test_qmm_validation_before_any_launch():
+    F = FAKE
+
+    def qmm(x=F, w=F, s=F, b=F, y=F, M=16, N=128, K=128, bits=4, g=64, dt=2):
+        return L.qmv_qmm_affine(x, w, s, b, y, M, N, K, bits, g, dt, None)
+
+    assert qmm(M=65) == EINVAL
+    assert qmm(M=-1) == EINVAL
+    assert qmm(bits=7) == EUNSUP
+    assert qmm(K=100) == EINVAL
+    assert qmm(b=None) == EINVAL
+    assert qmm(x=F + 1) == EALIGN
+    assert qmm(M=0) == 0 and qmm(N=0) == 0

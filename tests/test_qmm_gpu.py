@@ -1,0 +1,56 @@
+"""GPU parity of the small-M qmm (qmv_qmm_affine: up to 64 x rows, run as
+8-row chunks through the qmv kernels) against the oracle, element by element,
+within the qmv output tolerance.  Row counts cover one chunk plus a ragged
+remainder, several full chunks and the maximum of 64."""
+from __future__ import annotations
+
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import THREADS, TORCH_DT, dev, require_cuda, to_f64
+from qmv_tol import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    return require_cuda()
+
+
+def _run(q, c, M, N, K):
+    y = torch.full((M, N), float("nan"), dtype=TORCH_DT[c["dtype"]], device="cuda")
+    q.qmv_qmm_affine(dev(c["x"][0]), dev(c["w"][0]), dev(c["scales"][0]), dev(c["biases"][0]), y, M, N, K,
+                     c["bits"], c["group"], c["dtype"])
+    torch.cuda.synchronize()
+    return to_f64(y)
+
+
+@pytest.mark.parametrize("M", [9, 16, 23, 33, 64])
+@pytest.mark.parametrize("bits,group,dtype", [(4, 64, "bf16"), (3, 32, "f16"), (8, 128, "f32"), (6, 64, "bf16")])
+def test_qmm_rows(q, M, bits, group, dtype):
+    N, K = 1000, 1024
+    c = synth.affine_case(M, N, K, bits, group, dtype, seed=M * 10 + bits)
+    y = _run(q, c, M, N, K)
+    ref, ad = oracle.qmv_affine(c["x"][0], c["w"][0], c["scales"][0], c["biases"][0], M, N, K, bits, group, dtype,
+                                threads=THREADS)
+    assert_close(y, ref, ad, dtype, what=f"qmm M={M} b{bits} g{group} {dtype}")
+
+
+def test_qmm_layer_shape(q):
+    """The 7B down projection (4096 x 14336, 4-bit g64 bf16) at M = 32, sampled rows."""
+    M, N, K = 32, 4096, 14336
+    c = synth.affine_case(M, N, K, 4, 64, "bf16", seed=77)
+    y = _run(q, c, M, N, K)
+    rows = list(range(0, N, 97)) + [N - 1]
+    ref, ad = oracle.qmv_affine(c["x"][0], c["w"][0], c["scales"][0], c["biases"][0], M, N, K, 4, 64, "bf16",
+                                rows=rows, threads=THREADS)
+    assert_close(y[:, rows], ref[:, rows], ad[:, rows], "bf16", what="qmm 4096x14336 M=32")
+
+
+def test_qmm_rejects_more_than_64_rows(q):
+    e = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(Exception):
+        q.qmv_qmm_affine(e, e, e, e, e, 65, 64, 64, 4, 64, "bf16")

@@ -18,7 +18,7 @@ import os
 
 __all__ = [
     "QmvError", "qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
-    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_qvm_affine",
+    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_qmm_affine", "qmv_qvm_affine",
     "qmv_qvm_workspace_bytes", "qmv_qvm_affine_noalloc", "qmv_status_string",
     "qmv_last_cuda_error",
     "qmv_describe_plan", "qmv_force_config", "DTYPES", "FP_MODES", "LIB_PATH", "lib",
@@ -57,6 +57,8 @@ _lib.qmv_dequant_affine_f32.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 _lib.qmv_dequant_fp_f32.argtypes = [_p, _p, _p, _p, _i, _i, _i, _p]
 _lib.qmv_quantize_affine.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 _lib.qmv_qvm_affine.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p]
+_lib.qmv_qmm_affine.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
+_lib.qmv_qmm_affine.restype = _i
 _lib.qmv_qvm_workspace_bytes.argtypes = [_i, _i]
 _lib.qmv_qvm_workspace_bytes.restype = ctypes.c_size_t
 _lib.qmv_status_string.argtypes = [_i]
@@ -176,6 +178,13 @@ def qmv_quantize_affine(w, w_packed, scales, biases, N, K, bits, group_size, dty
     dtype, all caller-owned device buffers."""
     _check(_lib.qmv_quantize_affine(_ptr(w), _ptr(w_packed), _ptr(scales), _ptr(biases), N, K, bits,
                                     group_size, _dtype(dtype), _stream(stream)), "qmv_quantize_affine")
+
+
+def qmv_qmm_affine(x, w_packed, scales, biases, y, M, N, K, bits, group_size, dtype, stream=None):
+    """Small-M qmm (C ABI qmv_qmm_affine): qmv_affine's layouts with up to 64
+    x rows, run as chunks of 8 rows back to back on the stream."""
+    _check(_lib.qmv_qmm_affine(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(biases), _ptr(y), M, N, K, bits,
+                               group_size, _dtype(dtype), _stream(stream)), "qmv_qmm_affine")
 
 
 def qmv_qvm_affine(x, w_packed, scales, biases, y, M, N, K, bits, group_size, dtype, workspace=None,

@@ -800,6 +800,33 @@ int qmv_quantize_affine(const void* w, void* w_packed, void* scales, void* biase
                                               static_cast<cudaStream_t>(stream)));
 }
 
+int qmv_qmm_affine(const void* x, const void* w_packed, const void* scales, const void* biases, void* y,
+                   int M, int N, int K, int bits, int group_size, int dtype, void* stream) {
+    if (M < 0 || M > QMV_QMM_MAX_M) return QMV_EINVAL;
+    // every argument is checked once, on the first chunk: the later chunks
+    // differ only by whole-row offsets of x and y, which keep the alignment
+    const int m1 = M < QMV_MAX_M ? M : QMV_MAX_M;
+    int st = check_affine(bits, group_size);
+    if (st != QMV_OK) return st;
+    if (K % group_size != 0) return QMV_EINVAL;
+    st = check_common(x, w_packed, scales, y, m1, N, K, dtype);
+    if (st != QMV_OK || M == 0 || N == 0) return st;
+    if (K > 0 && !biases) return QMV_EINVAL;
+    const size_t eb = elem_bytes(dtype);
+    if (K > 0 && (!aligned(scales, eb) || !aligned(biases, eb))) return QMV_EALIGN;
+    // chunks of QMV_MAX_M x rows, back to back on the stream: a weight matrix
+    // that fits in L2 is read from HBM by the first chunk only
+    for (int m0 = 0; m0 < M; m0 += QMV_MAX_M) {
+        const int mc = M - m0 < QMV_MAX_M ? M - m0 : QMV_MAX_M;
+        const void* xc = x ? static_cast<const char*>(x) + (size_t)m0 * K * eb : nullptr;
+        void* yc = static_cast<char*>(y) + (size_t)m0 * N * eb;
+        st = run(qmv::FAM_AFFINE, xc, w_packed, scales, biases, nullptr, yc, mc, N, K, bits, group_size, dtype, 1,
+                 1, stream);
+        if (st != QMV_OK) return st;
+    }
+    return QMV_OK;
+}
+
 int qmv_qvm_affine(const void* x, const void* w_packed, const void* scales, const void* biases, void* y,
                    int M, int N, int K, int bits, int group_size, int dtype, void* workspace, void* stream) {
     int st = check_affine(bits, group_size);
