@@ -169,6 +169,27 @@ def qmv_affine(x, w, scales, biases, M, N, K, bits, group, dtype, rows=None, thr
     return y, a
 
 
+def qmv_affine_gather(x, w, scales, biases, ids, M, N, K, bits, group, dtype, n_experts, x_batched=True,
+                      threads=1):
+    """Expert-indexed qmv (wh-iron kernel-op coverage audit, "gather_qmv /
+    gather_qmm" row; DS4 moe.metal, kernel_mul_mv_id: the ids tensor selects
+    the routed expert of each slot).  Token t multiplies x[t] (or the shared
+    x) by matrix ids[t] of the stacks w [E, N, row bytes], scales / biases
+    [E, N, K/group], each product being qmv_affine above.  An id outside
+    [0, n_experts) has no matrix: that token's outputs are NaN.  Returns (y,
+    absdot), float64 [T, M, N]."""
+    T = len(ids)
+    y = np.full((T, M, N), np.nan); a = np.full((T, M, N), np.nan)
+    for t in range(T):
+        e = int(ids[t])
+        if not 0 <= e < n_experts:
+            continue
+        xt = np.ascontiguousarray(x[t] if x_batched else x)
+        y[t], a[t] = qmv_affine(xt, np.ascontiguousarray(w[e]), np.ascontiguousarray(scales[e]),
+                                np.ascontiguousarray(biases[e]), M, N, K, bits, group, dtype, threads=threads)
+    return y, a
+
+
 def qvm_affine(x, w, scales, biases, M, N, K, bits, group, dtype, cols=None, threads=1):
     """x [M, K] times W stored [K, N] (packed rows of N codes, scales and
     biases [K, N / group]).  Return (y, absdot), both float64 [M, N]; columns

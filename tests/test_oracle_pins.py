@@ -405,6 +405,47 @@ def test_qvm_exact_bruteforce(bits, dtype):
             assert abs(Fraction(absdot[m, n]) - aacc) <= aacc * Fraction(2) ** -40
 
 
+# ---------------------------------------------------------- gather pins ----
+def _expert_stack(E, N, K, bits, group, seed):
+    cs = [synth.affine_case(1, N, K, bits, group, "f32", seed=seed + e) for e in range(E)]
+    return (np.stack([c["w"][0] for c in cs]), np.stack([c["scales"][0] for c in cs]),
+            np.stack([c["biases"][0] for c in cs]))
+
+
+def test_gather_unit_x_selects_the_routed_expert():
+    """x[t] = e_k: y[t, 0, n] is element (n, k) of expert ids[t]'s weights
+    (codes from the test-side reader, values from library casts)."""
+    E, N, K, bits, group = 4, 6, 64, 4, 32
+    w, sc, bi = _expert_stack(E, N, K, bits, group, seed=40)
+    ids = np.array([2, 0, 2, 3], dtype=np.int32)
+    ks = [5, 17, 40, 63]
+    x = np.zeros((len(ids), 1, K), dtype=np.float32)
+    for t, k in enumerate(ks):
+        x[t, 0, k] = 1.0
+    y, _ = oracle.qmv_affine_gather(x, w, sc, bi, ids, 1, N, K, bits, group, "f32", E)
+    for t, (e, k) in enumerate(zip(ids, ks)):
+        for n in range(N):
+            q = _py_codes(w[e, n], K, bits)[k]
+            assert y[t, 0, n] == float(sc[e, n, k // group]) * q + float(bi[e, n, k // group])
+
+
+def test_gather_token_permutation_and_bad_id():
+    """Permuting the tokens (x rows with their ids) permutes the outputs; an
+    id outside the stack gives a NaN token and leaves the others unchanged."""
+    E, N, K, bits, group = 3, 5, 64, 3, 32
+    w, sc, bi = _expert_stack(E, N, K, bits, group, seed=60)
+    x = synth.affine_case(2, 1, K, bits, group, "f32", seed=61, batch=4)["x"]         # [4, 2, K]
+    ids = np.array([1, 2, 0, 1], dtype=np.int32)
+    y, _ = oracle.qmv_affine_gather(x, w, sc, bi, ids, 2, N, K, bits, group, "f32", E)
+    perm = np.array([3, 1, 0, 2])
+    yp, _ = oracle.qmv_affine_gather(np.ascontiguousarray(x[perm]), w, sc, bi, ids[perm], 2, N, K, bits, group,
+                                     "f32", E)
+    assert np.array_equal(yp, y[perm])
+    bad = ids.copy(); bad[2] = E
+    yb, _ = oracle.qmv_affine_gather(x, w, sc, bi, bad, 2, N, K, bits, group, "f32", E)
+    assert np.isnan(yb[2]).all() and np.array_equal(np.delete(yb, 2, 0), np.delete(y, 2, 0))
+
+
 # ------------------------------------------------------------ sum(x) pin ----
 def _emulate_kernel_bf16(case, widened):
     """fp32 emulation of a qmv whose bias term uses sum(x) per group, either
