@@ -2,7 +2,7 @@
 """Benchmark of the weight-quantized matrix-vector product on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload chain8|layer|probe|quantize|qvm|qmm]
+                    [--workload chain8|layer|probe|quantize|qvm|qmm|moe]
 
 Prints ONE JSON line (rank 0).  Metric: qmv microseconds per call and achieved
 HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
@@ -20,6 +20,8 @@ HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
   quantize          the affine quantizer (qmv_quantize_affine) on a bf16
                     16384 x 16384 matrix -> 4-bit g64 (one call per step; its
                     metric is the quantizer's microseconds per call).
+  moe               MoE decode (qmv_affine_gather): 16 tokens routed by device
+                    ids to one of 64 experts of 1536 x 2048 each (one call per step).
   qmm               small-M qmm (qmv_qmm_affine): the layer's four projections
                     at M=32 (4 calls per step).
   qvm               x times W stored [K, N] (qmv_qvm_affine), affine 4-bit g64
@@ -406,6 +408,57 @@ class Qmm(Layer):
                 "l2": "flushed before every step (512 MB write + 256 MB read); weights rotate through copies > 2x L2"}
 
 
+class Moe(Layer):
+    """MoE decode: 16 tokens, each routed (device-side ids) to one of 64
+    experts of 1536 x 2048, 4-bit g64 bf16, one qmv_affine_gather call per step.
+    Algorithmic bytes: the distinct experts' weights once, plus x and y."""
+    name = "MoE decode gather-qmv, 16 tokens over 64 experts of 1536x2048, affine 4-bit g64 bf16, M=1"
+    T, E, N, K = 16, 64, 1536, 2048
+
+    def __init__(self, q, torch, dev):
+        self.q, self.torch = q, torch
+        T, E, N, K = self.T, self.E, self.N, self.K
+        g = np.random.default_rng(6000)
+        rb = K * 4 // 8
+        w = torch.from_numpy(g.integers(0, 256, size=(E, N, rb), dtype=np.uint8)).to(dev)
+        sc = torch.from_numpy(synth.to_storage(g.uniform(0.005, 0.02, size=(E, N, K // 64)), "bf16").view(np.int16)).view(torch.bfloat16).to(dev)
+        bi = torch.from_numpy(synth.to_storage(g.normal(0.0, 0.01, size=(E, N, K // 64)), "bf16").view(np.int16)).view(torch.bfloat16).to(dev)
+        ids = g.integers(0, E, size=T).astype(np.int32)
+        self.distinct = len(set(ids.tolist()))
+        x_host = torch.from_numpy(synth.to_storage(g.standard_normal((T, 1, K)), "bf16").view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.sets = [dict(name="moe", M=1, N=N, K=K, w=w, sc=sc, bi=bi, ids=torch.from_numpy(ids).to(dev),
+                          x=x_host.to(dev), x_host=x_host, y=torch.empty((T, 1, N), dtype=torch.bfloat16, device=dev),
+                          y_host=torch.empty((T, 1, N), dtype=torch.bfloat16).pin_memory(), it=0)]
+        self.calls_per_step = 1
+
+    def graph_variants(self, s):
+        return 1
+
+    def run_group(self, s, e2e=False, v=0):
+        if e2e:
+            s["x"].copy_(s["x_host"], non_blocking=True)
+        self.q.qmv_affine_gather(s["x"], s["w"], s["sc"], s["bi"], s["ids"], s["y"], 1, self.N, self.K, 4, 64, "bf16",
+                                 self.T, self.E)
+        if e2e:
+            s["y_host"].copy_(s["y"], non_blocking=True)
+        return 1
+
+    def group_bytes(self, s):
+        N, K = self.N, self.K
+        return self.distinct * (N * K // 2 + 2 * N * (K // 64) * 2) + self.T * (K + N) * 2
+
+    def group_plan(self, s):
+        return "path=gather chunk=32 maxm=1 rows_per_warp=0 kernel=CUDA-core row-tiled bits=4 group=64 dtype=bf16"
+
+    def h2d_d2h(self):
+        return self.T * self.K * 2, self.T * self.N * 2
+
+    def config(self):
+        return {"workload": self.name, "bits": 4, "group": 64, "dtype": "bf16", "M": 1, "N": self.N, "K": self.K,
+                "tokens": self.T, "experts": self.E, "distinct_experts": self.distinct, "calls_per_step": 1,
+                "l2": "flushed before every step (512 MB write + 256 MB read)"}
+
+
 class Qvm(Layer):
     """qvm on the bandwidth-probe matrix stored [K, N]: x [1, 16384] times
     4-bit g64 W [16384, 16384], bf16, with the K-split workspace; each step
@@ -457,7 +510,7 @@ class Qvm(Layer):
                       "its own 151 MB weight copy"}
 
 
-WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe, "quantize": Quantize, "qvm": Qvm, "qmm": Qmm}
+WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe, "quantize": Quantize, "qvm": Qvm, "qmm": Qmm, "moe": Moe}
 
 
 # ---------------------------------------------------------------- our arm --
@@ -628,6 +681,8 @@ def _oracle_sample(workload, budget_s=12.0, threads=None):
         spec = [(M, N, K, 4, 64, 1) for M in (1, 8) for _, N, K in LAYER]
     elif workload == "qmm":
         spec = [(32, N, K, 4, 64, 1) for _, N, K in LAYER]
+    elif workload == "moe":
+        spec = [(1, 1536, 2048, 4, 64, 16)]
     else:
         spec = [(1, 16384, 16384, 4, 64, 1)]
     per_shape_budget = budget_s / len(spec)
@@ -650,7 +705,7 @@ def _oracle_sample(workload, budget_s=12.0, threads=None):
         us_call = dt * 1e6 * (N / nrows)
         total_us += us_call * calls
         sample.append(f"M={M} N={N} K={K}: {nrows}/{N} rows, {dt:.3f}s")
-    ncalls = sum(s[-1] for s in spec)
+    ncalls = 1 if workload == "moe" else sum(s[-1] for s in spec)     # moe: one call = all its tokens
     return total_us / ncalls, threads, "; ".join(sample)
 
 

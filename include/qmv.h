@@ -145,6 +145,30 @@ int qmv_quantize_affine(const void* w, void* w_packed, void* scales, void* biase
                         int bits, int group_size, int dtype, void* stream);
 
 /*
+ * qmv_affine_gather -- expert-indexed (MoE) qmv: for each token t,
+ *     y[t] = x[t] * dequant(W[expert_ids[t]])^T
+ * (wh-iron kernel-op coverage audit, "gather_qmv / gather_qmm" row; DS4
+ * moe.metal, kernel_mul_mv_id: an ids tensor selects each slot's routed expert
+ * on the device, with no per-expert dispatch from the host).
+ *   w_packed  [n_experts, N, K*bits/8] bytes, a stack of qmv_affine matrices
+ *   scales,   [n_experts, N, K/group_size] dtype
+ *   biases
+ *   expert_ids DEVICE int32 [n_tokens] (4-byte aligned), read on the GPU; an
+ *             id outside [0, n_experts) makes that token's y rows NaN (nothing
+ *             out of bounds is read)
+ *   x         [n_tokens, M, K] (x_batched = 1) or one [M, K] for every token
+ *   y         [n_tokens, M, N]
+ *   1 <= n_tokens <= 65535, n_experts >= 1; other arguments as qmv_affine.
+ * Runs on the CUDA-core kernels (row-tiled, or few-rows for small N), launched
+ * without programmatic dependent launch so that ids written by the previous
+ * kernel in the stream are complete.  Same accumulation and rounding as
+ * qmv_affine.
+ */
+int qmv_affine_gather(const void* x, const void* w_packed, const void* scales, const void* biases,
+                      const int* expert_ids, void* y, int M, int N, int K, int bits, int group_size,
+                      int dtype, int n_tokens, int n_experts, int x_batched, void* stream);
+
+/*
  * qmv_qmm_affine -- small-M quantized matmul, y = x * dequant(W)^T for up to
  * QMV_QMM_MAX_M x rows (the qmm family of MLX quantized_nax.h and of the
  * wh-iron audit, M-batched prefill).  Arguments and layouts as qmv_affine,

@@ -246,3 +246,18 @@ def test_qmm_validation_before_any_launch():
     assert qmm(b=None) == EINVAL
     assert qmm(x=F + 1) == EALIGN
     assert qmm(M=0) == 0 and qmm(N=0) == 0
+
+
+def test_gather_validation_before_any_launch():
+    F = FAKE
+
+    def g(x=F, w=F, s=F, b=F, ids=F, y=F, M=1, N=64, K=128, bits=4, gs=64, dt=2, T=4, E=8, xb=1):
+        return L.qmv_affine_gather(x, w, s, b, ids, y, M, N, K, bits, gs, dt, T, E, xb, None)
+
+    assert g(ids=None) == EINVAL
+    assert g(ids=F + 2) == EALIGN
+    assert g(T=0) == EINVAL and g(T=65536) == EINVAL
+    assert g(E=0) == EINVAL
+    assert g(xb=2) == EINVAL
+    assert g(bits=7) == EUNSUP
+    assert g(M=0) == 0

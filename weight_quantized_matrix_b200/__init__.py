@@ -18,7 +18,7 @@ import os
 
 __all__ = [
     "QmvError", "qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
-    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_qmm_affine", "qmv_qvm_affine",
+    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_affine_gather", "qmv_qmm_affine", "qmv_qvm_affine",
     "qmv_qvm_workspace_bytes", "qmv_qvm_affine_noalloc", "qmv_status_string",
     "qmv_last_cuda_error",
     "qmv_describe_plan", "qmv_force_config", "DTYPES", "FP_MODES", "LIB_PATH", "lib",
@@ -58,6 +58,8 @@ _lib.qmv_dequant_fp_f32.argtypes = [_p, _p, _p, _p, _i, _i, _i, _p]
 _lib.qmv_quantize_affine.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 _lib.qmv_qvm_affine.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p]
 _lib.qmv_qmm_affine.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
+_lib.qmv_affine_gather.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _p]
+_lib.qmv_affine_gather.restype = _i
 _lib.qmv_qmm_affine.restype = _i
 _lib.qmv_qvm_workspace_bytes.argtypes = [_i, _i]
 _lib.qmv_qvm_workspace_bytes.restype = ctypes.c_size_t
@@ -178,6 +180,16 @@ def qmv_quantize_affine(w, w_packed, scales, biases, N, K, bits, group_size, dty
     dtype, all caller-owned device buffers."""
     _check(_lib.qmv_quantize_affine(_ptr(w), _ptr(w_packed), _ptr(scales), _ptr(biases), N, K, bits,
                                     group_size, _dtype(dtype), _stream(stream)), "qmv_quantize_affine")
+
+
+def qmv_affine_gather(x, w_packed, scales, biases, expert_ids, y, M, N, K, bits, group_size, dtype, n_tokens,
+                      n_experts, x_batched=True, stream=None):
+    """Expert-indexed qmv (C ABI qmv_affine_gather): y[t] = x[t] times the
+    dequantized matrix expert_ids[t] of the stack; expert_ids is a device
+    int32 tensor."""
+    _check(_lib.qmv_affine_gather(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(biases), _ptr(expert_ids), _ptr(y),
+                                  M, N, K, bits, group_size, _dtype(dtype), n_tokens, n_experts,
+                                  1 if x_batched else 0, _stream(stream)), "qmv_affine_gather")
 
 
 def qmv_qmm_affine(x, w_packed, scales, biases, y, M, N, K, bits, group_size, dtype, stream=None):

@@ -392,7 +392,7 @@ bool tcf_shape(int N, int K, int bits, int G, bool w16, bool s16, TcbShape* ts) 
 
 // Choose the launch shape.  Returns QMV_OK or an error (sizes too large).
 int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, bool w16, int batch, Plan* pl,
-              bool s16 = true) {
+              bool s16 = true, bool gather = false) {
     const FmtInfo fi = fmt_info(fam, bits);
     const bool aff = fam == qmv::FAM_AFFINE;
     int maxm = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
@@ -424,7 +424,8 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     // the register-streaming CUDA-core kernel is as fast)
     const bool fma_ring_pick = M == 1 && dtype == QMV_BF16 && bits >= 2 && bits <= 6 &&
                                (double)N * K * bits / 8.0 >= 10.0 * 1024 * 1024;
-    if (aff && K > 0 && M == 1 && dtype == QMV_BF16 && (g_forced.path == 6 || (g_forced.path < 0 && fma_ring_pick))) {
+    if (!gather && aff && K > 0 && M == 1 && dtype == QMV_BF16 &&
+        (g_forced.path == 6 || (g_forced.path < 0 && fma_ring_pick))) {
         TcbShape ts;
         if (tcf_shape(N, K, bits, G_of_plan, w16, s16, &ts)) {
             pl->maxm = 1; pl->R = 1; pl->wide = 1; pl->tc = 4; pl->npass = 0;
@@ -442,7 +443,7 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     // matrices at M = 1)
     // (6-bit codes do not pair: the ring kernel wins there only at M = 8)
     const bool ring_pick = M >= 2 ? (N >= 64 && (bits != 6 || M >= 8)) : tc_preferred(M, N, K, bits, dtype);
-    if (aff && K > 0 && (g_forced.path == 4 || (g_forced.path < 0 && ring_pick))) {
+    if (!gather && aff && K > 0 && (g_forced.path == 4 || (g_forced.path < 0 && ring_pick))) {
         TcbShape ts;
         if (tcb_shape(M, N, K, bits, G_of_plan, dtype, w16, s16, &ts)) {
             pl->maxm = maxm; pl->R = 1; pl->wide = 1; pl->tc = 2; pl->npass = ts.npass;
@@ -456,7 +457,7 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     }
 
     // ---- tensor-core kernel (affine, enough rows to fill the GPU) -------------
-    if (aff && K > 0 && g_forced.path != 0 && g_forced.path != 1 &&
+    if (!gather && aff && K > 0 && g_forced.path != 0 && g_forced.path != 1 &&
         (g_forced.path == 3 || tc_preferred(M, N, K, bits, dtype))) {
         TcShape ts;
         if (tc_shape(M, N, K, bits, G_of_plan, dtype, w16, &ts)) {
@@ -613,12 +614,12 @@ bool encode_scale_map(CUtensorMap* m, const void* base, int dtype, long long KG,
 
 int run(int fam, const void* x, const void* w, const void* scales, const void* biases,
         const float* gscale, void* y, int M, int N, int K, int bits, int G, int dtype, int batch,
-        int x_batched, void* stream) {
+        int x_batched, void* stream, const int* ids = nullptr, int n_experts = 0) {
     const long long row_bytes = (long long)K * (fam == qmv::FAM_AFFINE ? bits : (fam == qmv::FAM_MXFP8 ? 8 : 4)) / 8;
     Plan pl;
     const bool w16 = aligned(w, 16);
     const bool s16 = fam == qmv::FAM_AFFINE && aligned(scales, 16) && aligned(biases, 16);
-    int st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, s16);
+    int st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, s16, ids != nullptr);
     if (st != QMV_OK) return st;
     qmv::Params p;
     const bool ring = pl.tc == 2 || pl.tc == 4;        // the weight-ring kernels
@@ -647,7 +648,11 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     p.s_bs = (long long)N * (K / G);
     p.y_bs = (long long)M * N;
     p.w_row = row_bytes;
-    qmv::Launch L{pl.grid, pl.block, pl.smem, static_cast<cudaStream_t>(stream), pdl_enabled()};
+    // gather reads ids (often written by the kernel just before) ahead of its
+    // grid-dependency wait: it launches without programmatic dependent launch
+    qmv::Launch L{pl.grid, pl.block, pl.smem, static_cast<cudaStream_t>(stream), pdl_enabled() && !ids};
+    p.ids = ids;
+    p.n_experts = n_experts;
     cudaError_t e;
     p.sps = pl.sps; p.pitch = pl.pitch; p.fault = nullptr;
     p.sring = pl.sring; p.soff = pl.soff; p.boff = pl.boff; p.sbw = pl.sbw;
@@ -798,6 +803,24 @@ int qmv_quantize_affine(const void* w, void* w_packed, void* scales, void* biase
     const int vec = (aligned(w, 16) && ((size_t)K * eb) % 16 == 0) ? (aligned(w_packed, 16) ? 2 : 1) : 0;
     return finish(qmv::launch_quantize_affine(bits, dtype, w, w_packed, scales, biases, N, K, group_size, vec,
                                               static_cast<cudaStream_t>(stream)));
+}
+
+int qmv_affine_gather(const void* x, const void* w_packed, const void* scales, const void* biases,
+                      const int* expert_ids, void* y, int M, int N, int K, int bits, int group_size, int dtype,
+                      int n_tokens, int n_experts, int x_batched, void* stream) {
+    int st = check_affine(bits, group_size);
+    if (st != QMV_OK) return st;
+    if (n_tokens < 1 || n_tokens > 65535 || n_experts < 1 || (x_batched != 0 && x_batched != 1))
+        return QMV_EINVAL;
+    if (K % group_size != 0) return QMV_EINVAL;
+    st = check_common(x, w_packed, scales, y, M, N, K, dtype);
+    if (st != QMV_OK || M == 0 || N == 0) return st;
+    if (!expert_ids || (K > 0 && !biases)) return QMV_EINVAL;
+    if (!aligned(expert_ids, 4)) return QMV_EALIGN;
+    const size_t eb = elem_bytes(dtype);
+    if (K > 0 && (!aligned(scales, eb) || !aligned(biases, eb))) return QMV_EALIGN;
+    return run(qmv::FAM_AFFINE, x, w_packed, scales, biases, nullptr, y, M, N, K, bits, group_size, dtype, n_tokens,
+               x_batched, stream, expert_ids, n_experts);
 }
 
 int qmv_qmm_affine(const void* x, const void* w_packed, const void* scales, const void* biases, void* y,

@@ -82,6 +82,11 @@ struct Params {
     // (with both operands immediate it would take two).
     unsigned kf32;          // 0x4B000000: fp32 2^23
     unsigned kbf16;         // 0x43004300: bf16 pair {128, 128}
+    // Gather (expert-indexed batches): batch entry z multiplies by weight
+    // matrix ids[z] of the stack (x and y stay entry z's); null: matrix z.
+    // Only the CUDA-core row-tiled and the few-rows kernels read it.
+    const int* ids;
+    int n_experts;
 };
 
 // ---------------------------------------------------------------- dtypes ---
@@ -445,6 +450,23 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
     const int kt = wkid * 32 + lane;
     const int bz = blockIdx.z;
     const int row0 = (blockIdx.x * p.wr + wrid) * R;
+    // gather: entry bz's weights are matrix ids[bz]; an id outside the stack
+    // has no weights, and this block's outputs of the entry become NaN
+    // (gather launches without programmatic dependent launch, so the ids
+    // written by the previous kernel are complete)
+    int be = bz;
+    if (p.ids) {
+        be = __ldg(p.ids + bz);
+        if (be < 0 || be >= p.n_experts) {
+            T* Yn = reinterpret_cast<T*>(p.y) + bz * p.y_bs;
+            const int rows = p.wr * R, r0 = blockIdx.x * rows;
+            for (int i = threadIdx.x; i < rows * p.M; i += blockDim.x) {
+                const int n = r0 + i / p.M, m = i % p.M;
+                if (n < p.N) DT<T>::st(Yn, (long long)m * p.N + n, __int_as_float(0x7FC00000));
+            }
+            return;
+        }
+    }
     const int NC = p.K / C;
     const int TI = p.tile_iters;
     const int TC = KT * TI;
@@ -453,9 +475,9 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
     float* sx = reinterpret_cast<float*>(xs + (size_t)MAXM * TI * (C / 4) * KT);
     float* red = sx + (AFF ? (size_t)MAXM * TI * U * KT : 0);
 
-    const uint8_t* W = p.w + bz * p.w_bs;
+    const uint8_t* W = p.w + be * p.w_bs;
     const char* Xb = reinterpret_cast<const char*>(p.x) + bz * p.x_bs * (long long)sizeof(T);
-    const long long sb = bz * p.s_bs;
+    const long long sb = be * p.s_bs;
 
     int rowc[R];
 #pragma unroll
@@ -522,7 +544,7 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
 
     warp_allreduce<R, MAXM>(acc);
     float gs = 1.f;
-    if constexpr (FAM == FAM_NVFP4) gs = __ldg(p.gscale + bz);
+    if constexpr (FAM == FAM_NVFP4) gs = __ldg(p.gscale + be);
     T* Y = reinterpret_cast<T*>(p.y) + bz * p.y_bs;
     const int RM = R * MAXM;
     if (p.wk == 1) {

@@ -124,8 +124,21 @@ __global__ void __launch_bounds__(256) qmv_direct_kernel(const Params p) {
     const int n = blockIdx.x, bz = blockIdx.z;
     const int units = p.K / 32;
     const int nthr = blockDim.x;
-    const uint8_t* row = p.w + bz * p.w_bs + (long long)n * p.w_row;
-    const long long srow = bz * p.s_bs + (long long)n * (p.K / p.G);
+    // gather: entry bz's weights are matrix ids[bz] (read before the grid
+    // wait: gather launches without programmatic dependent launch); an id
+    // outside the stack gives NaN outputs
+    int be = bz;
+    if (p.ids) {
+        be = __ldg(p.ids + bz);
+        if (be < 0 || be >= p.n_experts) {
+            if ((int)threadIdx.x < p.M)
+                DT<T>::st(reinterpret_cast<T*>(p.y) + bz * p.y_bs, (long long)threadIdx.x * p.N + n,
+                          __int_as_float(0x7FC00000));
+            return;
+        }
+    }
+    const uint8_t* row = p.w + be * p.w_bs + (long long)n * p.w_row;
+    const long long srow = be * p.s_bs + (long long)n * (p.K / p.G);
     const uint32_t kf32 = p.kf32;
 
     // the next kernel in the stream may launch and start fetching its own
@@ -174,7 +187,7 @@ __global__ void __launch_bounds__(256) qmv_direct_kernel(const Params p) {
         const int m = threadIdx.x;
         float v = 0.f;
         for (int k = 0; k < (nthr >> 5); ++k) v += red[k * MAXM + m];
-        if constexpr (FAM == FAM_NVFP4) v = v * __ldg(p.gscale + bz);
+        if constexpr (FAM == FAM_NVFP4) v = v * __ldg(p.gscale + be);
         DT<T>::st(reinterpret_cast<T*>(p.y) + bz * p.y_bs, (long long)m * p.N + n, v);
     }
 }
