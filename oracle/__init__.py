@@ -76,6 +76,10 @@ def lib():
         L.oracle_f32_to_bf16.argtypes = [f]; L.oracle_f32_to_bf16.restype = u
         L.oracle_f32_to_f16.argtypes = [f]; L.oracle_f32_to_f16.restype = u
         L.oracle_quantize_affine.argtypes = [p, p, p, p, ll, ll, i, i, i, ll, ll]
+        L.oracle_quantize_fp.argtypes = [p, p, p, f, ll, ll, i, i, ll, ll]
+        L.oracle_quantize_fp.restype = None
+        L.oracle_nearest_e2m1.argtypes = [d]; L.oracle_nearest_e2m1.restype = u
+        L.oracle_nearest_e4m3.argtypes = [d]; L.oracle_nearest_e4m3.restype = u
         L.oracle_quantize_affine.restype = None
         _lib = L
     return _lib
@@ -228,3 +232,23 @@ def quantize_affine(w, N, K, bits, group, dtype, rows=None, threads=1):
                                                DTYPE_CODES[dtype], a, b)
     _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
     return wq, sc, bi
+
+
+# ---- FP quantizer -----------------------------------------------------------
+def nearest_e2m1(a): return lib().oracle_nearest_e2m1(float(a))
+def nearest_e4m3(a): return lib().oracle_nearest_e4m3(float(a))
+
+
+def quantize_fp(w, N, K, mode, dtype, global_scale=1.0, rows=None, threads=1):
+    """Quantize w ([N, K] storage of `dtype`) to (codes uint8 [N, K/2] (FP4,
+    low nibble = even k) or [N, K] (FP8), scale bytes uint8 [N, K/block])."""
+    w = np.ascontiguousarray(w)
+    fp8 = mode == "mxfp8"
+    blk = 16 if mode == "nvfp4" else 32
+    wq = np.zeros((N, K if fp8 else K // 2), dtype=np.uint8)
+    sc = np.zeros((N, K // blk), dtype=np.uint8)
+    L = lib()
+    fn = lambda a, b: L.oracle_quantize_fp(_ptr(w), _ptr(wq), _ptr(sc), float(global_scale), N, K, FP_MODES[mode],
+                                           DTYPE_CODES[dtype], a, b)
+    _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
+    return wq, sc

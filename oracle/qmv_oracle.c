@@ -377,3 +377,94 @@ void oracle_quantize_affine(const void* w, uint8_t* wq, void* scales, void* bias
         }
     }
 }
+
+/* ---------------------------------------------------------------------------
+ * FP quantizer (wh-iron kernel-op coverage audit, "fp_quantized (fp4/fp8
+ * quant + dequant)" row: a per-group max scale and mantissa rounding, exact
+ * for fp8 normals and subnormals, saturating with no NaN or infinity; Track 1
+ * format table for the block sizes and scale types).  The pages give no
+ * formula for the scale; the reading here:
+ *   MXFP4 / MXFP8-E4M3, blocks of 32: the E8M0 byte is
+ *     clamp(floor(log2(amax)) - emax + 127, 0, 254)   (emax 2 for E2M1, 8 for
+ *     E4M3; byte 0 when amax is 0), and element d = w * 2^(127 - byte);
+ *   NVFP4, blocks of 16, FP32 global g > 0: the E4M3 scale is the nearest E4M3
+ *     to t = amax / (6 * g) (fp32 operations), and d = w / (scale * g) (fp32
+ *     operations; d = 0 when the scale is 0).
+ * Every code is the element whose value is nearest to |d| (exact distances),
+ * ties to the even code, saturating at the largest finite element; the sign
+ * bit is set for d < 0.  Codes are found by trying every element value, not
+ * by arithmetic on the bits.  Rows [n0, n1).
+ * ------------------------------------------------------------------------- */
+/* Nearest E2M1 magnitude code (0..7) to a >= 0, ties to even, saturating. */
+static uint32_t nearest_e2m1(double a) {
+    uint32_t best = 0;
+    double bd = INFINITY;
+    for (uint32_t c = 0; c < 8; ++c) {
+        double dd = fabs(oracle_e2m1(c) - a);
+        if (dd < bd || (dd == bd && (c & 1u) == 0)) { bd = dd; best = c; }
+    }
+    return best;
+}
+
+/* Nearest finite E4M3 magnitude code (0..126) to a >= 0, ties to even. */
+static uint32_t nearest_e4m3(double a) {
+    uint32_t best = 0;
+    double bd = INFINITY;
+    for (uint32_t c = 0; c < 127; ++c) {
+        double dd = fabs(oracle_e4m3(c) - a);
+        if (dd < bd || (dd == bd && (c & 1u) == 0)) { bd = dd; best = c; }
+    }
+    return best;
+}
+
+uint32_t oracle_nearest_e2m1(double a) { return nearest_e2m1(a); }
+uint32_t oracle_nearest_e4m3(double a) { return nearest_e4m3(a); }
+
+void oracle_quantize_fp(const void* w, uint8_t* wq, uint8_t* scales, float global, long long N, long long K,
+                        int mode, int dtype, long long n0, long long n1) {
+    (void)N;
+    const int fp8 = mode == OR_MXFP8, nv = mode == OR_NVFP4;
+    const int blk = nv ? 16 : 32;
+    const long long rb = fp8 ? K : K / 2;
+    for (long long n = n0; n < n1; ++n) {
+        uint8_t* row = wq + n * rb;
+        memset(row, 0, (size_t)rb);
+        for (long long b0 = 0; b0 < K; b0 += blk) {
+            float amax = 0.0f;
+            for (long long k = b0; k < b0 + blk; ++k) {
+                float a = fabsf(load_f32(w, (size_t)(n * K + k), dtype));
+                if (a > amax) amax = a;
+            }
+            const size_t si = (size_t)(n * (K / blk) + b0 / blk);
+            float sT = 0.0f;                 /* NVFP4 scale value */
+            double mul = 0.0;                /* MX: 2^(127 - byte) */
+            if (nv) {
+                const float t = amax / (6.0f * global);              /* fp32, fp32 */
+                const uint32_t sc = nearest_e4m3((double)t);
+                scales[si] = (uint8_t)sc;
+                sT = (float)oracle_e4m3(sc);
+            } else {
+                int byte = 0;
+                if (amax > 0.0f) {
+                    int e;
+                    frexp((double)amax, &e);                          /* amax = f * 2^e, f in [0.5, 1) */
+                    int x = (e - 1) - (fp8 ? 8 : 2) + 127;
+                    byte = x < 0 ? 0 : x > 254 ? 254 : x;
+                }
+                scales[si] = (uint8_t)byte;
+                mul = ldexp(1.0, 127 - byte);
+            }
+            for (long long k = b0; k < b0 + blk; ++k) {
+                const float v = load_f32(w, (size_t)(n * K + k), dtype);
+                double d;
+                if (nv) d = sT == 0.0f ? 0.0 : (double)(v / (sT * global));   /* fp32, fp32 */
+                else d = (double)v * mul;                                      /* exact */
+                uint32_t code;
+                if (fp8) code = nearest_e4m3(fabs(d)) | (d < 0 ? 0x80u : 0u);
+                else code = nearest_e2m1(fabs(d)) | (d < 0 ? 0x8u : 0u);
+                if (fp8) row[k] = (uint8_t)code;
+                else row[k / 2] |= (uint8_t)(code << (4 * (k % 2)));
+            }
+        }
+    }
+}

@@ -589,3 +589,99 @@ def test_quantize_nearest_code_brute_force(bits):
             if got != best:
                 assert float(got - best) <= 1e-6 * float(s), (n, k, codes[k])
             assert float(got) <= float(s) / 2 * (1 + 1e-6) or codes[k] in (0, qmax)
+
+
+# ------------------------------------------------------ FP quantizer pins ----
+@pytest.mark.parametrize("a,code", [(0.0, 0), (0.24, 0), (0.25, 0), (0.26, 1), (0.75, 2), (1.25, 2), (1.75, 4),
+                                    (2.5, 4), (3.5, 6), (4.9, 6), (5.0, 6), (5.1, 7), (6.0, 7), (7.0, 7), (1e9, 7)])
+def test_nearest_e2m1_hand_cases(a, code):
+    """E2M1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}: the midpoints go to the even
+    code, anything past 6 saturates to 6 (code 7)."""
+    assert oracle.nearest_e2m1(a) == code
+
+
+def test_nearest_e4m3_vs_torch_in_range():
+    """Inside the finite range torch's float8_e4m3fn conversion rounds to
+    nearest even exactly as the definition does; past 448 the quantizer
+    saturates (code 0x7E)."""
+    rng = np.random.default_rng(0)
+    a = np.concatenate([rng.uniform(0, 448, 4000), np.exp2(rng.uniform(-12, 8.8, 4000)),
+                        np.arange(0, 2 ** -6, 2 ** -10)]).astype(np.float32)
+    a = a[a <= 448]
+    want = torch.from_numpy(a).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.nearest_e4m3(float(v)) for v in a], dtype=np.uint8)
+    assert np.array_equal(got, want)
+    assert oracle.nearest_e4m3(449.0) == 0x7E and oracle.nearest_e4m3(1e30) == 0x7E
+
+
+def _fp_grid_weights(mode, N, K, rng):
+    """Weights that lie exactly on a block's element grid, with the block
+    maximum at the largest element, so the quantizer must return their codes."""
+    fp8 = mode == "mxfp8"
+    blk = 16 if mode == "nvfp4" else 32
+    vals = np.array([oracle.e4m3(c) for c in range(127)]) if fp8 else np.array([oracle.e2m1(c) for c in range(8)])
+    top = len(vals) - 1
+    codes = rng.integers(0, top + 1, size=(N, K))
+    codes[:, ::blk] = top                                   # every block reaches the top element
+    sign = rng.integers(0, 2, size=(N, K))
+    if mode == "nvfp4":
+        s_codes = rng.integers(8, 100, size=(N, K // blk))  # normal E4M3 scales
+        scale = np.array([[oracle.e4m3(c) for c in r] for r in s_codes])
+    else:
+        s_codes = rng.integers(120, 135, size=(N, K // blk))
+        scale = np.exp2(s_codes.astype(np.float64) - 127)
+    g = 0.5 if mode == "nvfp4" else 1.0                      # NVFP4: a non-unit global scale
+    w = vals[codes] * np.repeat(scale, blk, axis=1) * g * np.where(sign == 1, -1.0, 1.0)
+    return w.astype(np.float32), codes, sign, s_codes, g
+
+
+@pytest.mark.parametrize("mode", ["mxfp4", "mxfp8", "nvfp4"])
+def test_quantize_fp_recovers_grid_weights(mode):
+    """On-grid weights come back exactly (codes with their signs, scale
+    bytes): MX scale byte = floor(log2(amax)) - emax + 127; NVFP4 scale =
+    amax / (6 * global) with global 0.5."""
+    rng = np.random.default_rng(7)
+    N, K = 4, 128
+    w, codes, sign, s_codes, g = _fp_grid_weights(mode, N, K, rng)
+    wq, sc = oracle.quantize_fp(w, N, K, mode, "f32", global_scale=g)
+    assert np.array_equal(sc, s_codes.astype(np.uint8))
+    fp8 = mode == "mxfp8"
+    got = wq.astype(np.int64) if fp8 else np.stack([wq & 0xF, wq >> 4], axis=-1).reshape(N, K).astype(np.int64)
+    sbit = 0x80 if fp8 else 0x8
+    want = codes + sign * sbit
+    want[codes == 0] = 0                                    # +0 and -0 (not < 0) take code 0
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("mode", ["mxfp4", "mxfp8", "nvfp4"])
+def test_quantize_fp_dequant_error_bound(mode):
+    """Random weights: quantize, dequantize with the oracle's decoder; each
+    weight is within half an element step (times the block scale) of its
+    dequantized value, the step taken at the element's own magnitude, except
+    past the largest element, where it saturates."""
+    rng = np.random.default_rng(11)
+    N, K = 3, 256
+    w = (rng.standard_normal((N, K)) * 0.3).astype(np.float32)
+    g = 0.7
+    wq, sc = oracle.quantize_fp(w, N, K, mode, "f32", global_scale=g)
+    deq = oracle.dequant_fp_f32(wq, sc, g if mode == "nvfp4" else None, N, K, mode)
+    blk = 16 if mode == "nvfp4" else 32
+    if mode == "nvfp4":
+        bscale = np.array([[oracle.e4m3(int(c)) for c in r] for r in sc]) * np.float32(g)
+    else:
+        bscale = np.exp2(sc.astype(np.float64) - 127)
+    bs = np.repeat(bscale, blk, axis=1)
+    d = np.abs(w.astype(np.float64)) / bs
+    if mode == "mxfp8":
+        step = np.where(d < 2 ** -6, 2 ** -9, np.exp2(np.floor(np.log2(np.maximum(d, 2 ** -6))) - 3))
+    else:
+        step = np.where(d < 2, 0.5, np.where(d < 4, 1.0, 2.0))
+    err = np.abs(w.astype(np.float64) - deq.astype(np.float64))
+    top = 448.0 if mode == "mxfp8" else 6.0
+    # past the largest element (MX scales put the block maximum in [4, 8) or
+    # [256, 512) elements) the code saturates: the error is the excess
+    bound = np.where(d > top, (d - top) * bs, 0.5 * step * bs)
+    ulp = np.abs(deq.astype(np.float64)) * 2.0 ** -23      # the dequantized value is one fp32 rounding
+    assert (err <= bound * (1 + 1e-6) + ulp + 1e-30).all()
+    sat = d > top
+    assert (np.abs(np.abs(deq[sat]) - (top * bs)[sat]) <= ulp[sat]).all()
