@@ -390,13 +390,16 @@ void oracle_quantize_affine(const void* w, uint8_t* wq, void* scales, void* bias
  *   NVFP4, blocks of 16, FP32 global g > 0: the E4M3 scale is the nearest E4M3
  *     to t = amax / (6 * g) (fp32 operations), and d = w / (scale * g) (fp32
  *     operations; d = 0 when the scale is 0).
- * Every code is the element whose value is nearest to |d| (exact distances),
- * ties to the even code, saturating at the largest finite element; the sign
- * bit is set for d < 0.  Codes are found by trying every element value, not
+ * Every code is the element whose value is nearest to |d| (exact distances
+ * below the largest element), ties to the even code, and the largest finite
+ * element from there up (saturation); the sign bit is set for d < 0.  Codes are found by trying every element value, not
  * by arithmetic on the bits.  Rows [n0, n1).
  * ------------------------------------------------------------------------- */
-/* Nearest E2M1 magnitude code (0..7) to a >= 0, ties to even, saturating. */
+/* Nearest E2M1 magnitude code (0..7) to a >= 0, ties to even, saturating:
+ * from the largest element up the code is the largest (the distances of a
+ * huge a to the elements would round to the same fp64 value). */
 static uint32_t nearest_e2m1(double a) {
+    if (a >= oracle_e2m1(7)) return 7;
     uint32_t best = 0;
     double bd = INFINITY;
     for (uint32_t c = 0; c < 8; ++c) {
@@ -406,8 +409,10 @@ static uint32_t nearest_e2m1(double a) {
     return best;
 }
 
-/* Nearest finite E4M3 magnitude code (0..126) to a >= 0, ties to even. */
+/* Nearest finite E4M3 magnitude code (0..126) to a >= 0, ties to even,
+ * saturating at 448 as above. */
 static uint32_t nearest_e4m3(double a) {
+    if (a >= oracle_e4m3(126)) return 126;
     uint32_t best = 0;
     double bd = INFINITY;
     for (uint32_t c = 0; c < 127; ++c) {

@@ -593,7 +593,8 @@ def test_quantize_nearest_code_brute_force(bits):
 
 # ------------------------------------------------------ FP quantizer pins ----
 @pytest.mark.parametrize("a,code", [(0.0, 0), (0.24, 0), (0.25, 0), (0.26, 1), (0.75, 2), (1.25, 2), (1.75, 4),
-                                    (2.5, 4), (3.5, 6), (4.9, 6), (5.0, 6), (5.1, 7), (6.0, 7), (7.0, 7), (1e9, 7)])
+                                    (2.5, 4), (3.5, 6), (4.9, 6), (5.0, 6), (5.1, 7), (6.0, 7), (7.0, 7), (1e9, 7),
+                                    (6.7e35, 7), (1e300, 7)])
 def test_nearest_e2m1_hand_cases(a, code):
     """E2M1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}: the midpoints go to the even
     code, anything past 6 saturates to 6 (code 7)."""
@@ -612,6 +613,7 @@ def test_nearest_e4m3_vs_torch_in_range():
     got = np.array([oracle.nearest_e4m3(float(v)) for v in a], dtype=np.uint8)
     assert np.array_equal(got, want)
     assert oracle.nearest_e4m3(449.0) == 0x7E and oracle.nearest_e4m3(1e30) == 0x7E
+    assert oracle.nearest_e4m3(3e38 / 7) == 0x7E and oracle.nearest_e4m3(1e300) == 0x7E
 
 
 def _fp_grid_weights(mode, N, K, rng):
