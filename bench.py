@@ -2,7 +2,7 @@
 """Benchmark of the weight-quantized matrix-vector product on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload chain8|layer|probe|quantize|qvm|qmm|moe]
+                    [--workload chain8|layer|probe|quantize|quantize_fp|qvm|qmm|moe]
 
 Prints ONE JSON line (rank 0).  Metric: qmv microseconds per call and achieved
 HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
@@ -20,6 +20,8 @@ HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
   quantize          the affine quantizer (qmv_quantize_affine) on a bf16
                     16384 x 16384 matrix -> 4-bit g64 (one call per step; its
                     metric is the quantizer's microseconds per call).
+  quantize_fp       the FP quantizer (qmv_quantize_fp) on a bf16 16384 x 16384
+                    matrix -> NVFP4 (one call per step).
   moe               MoE decode (qmv_affine_gather): 16 tokens routed by device
                     ids to one of 64 experts of 1536 x 2048 each (one call per step).
   qmm               small-M qmm (qmv_qmm_affine): the layer's four projections
@@ -408,6 +410,50 @@ class Qmm(Layer):
                 "l2": "flushed before every step (512 MB write + 256 MB read); weights rotate through copies > 2x L2"}
 
 
+class QuantizeFp(Quantize):
+    """The block-scaled FP quantizer on the bandwidth-probe matrix: bf16 w
+    [16384, 16384] -> NVFP4 (E2M1 codes, E4M3 scale per 16, FP32 global)."""
+    name = "FP quantizer, bf16 16384 x 16384 -> NVFP4"
+
+    def __init__(self, q, torch, dev):
+        self.q, self.torch = q, torch
+        N = K = 16384
+        g = torch.Generator(device="cpu").manual_seed(4100)
+        w_host = (torch.randn((N, K), generator=g) * 0.05).to(torch.bfloat16).pin_memory()
+        ws = [w_host.to(dev) for _ in range(2)]
+        self.sets = [dict(name="quantize_fp", M=1, N=N, K=K, ws=ws, w_host=w_host,
+                          wq=torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                          sc=torch.empty((N, K // 16), dtype=torch.uint8, device=dev),
+                          gs=torch.tensor([0.05 * 4 / (6 * 448)], dtype=torch.float32, device=dev),
+                          sc_host=torch.empty((N, K // 16), dtype=torch.uint8).pin_memory(), it=0)]
+        self.calls_per_step = 1
+
+    def run_group(self, s, e2e=False, v=0):
+        w = s["ws"][v % len(s["ws"])]
+        if e2e:
+            w.copy_(s["w_host"], non_blocking=True)
+        self.q.qmv_quantize_fp(w, s["wq"], s["sc"], s["gs"], s["N"], s["K"], "nvfp4", "bf16")
+        if e2e:
+            s["sc_host"].copy_(s["sc"], non_blocking=True)
+        return 1
+
+    def group_bytes(self, s):
+        N, K = s["N"], s["K"]
+        return N * K * 2 + N * K // 2 + N * (K // 16)
+
+    def group_plan(self, s):
+        return "path=quantize_fp chunk=16 maxm=0 rows_per_warp=0 mode=nvfp4 dtype=bf16"
+
+    def h2d_d2h(self):
+        s = self.sets[0]
+        return s["N"] * s["K"] * 2, s["N"] * (s["K"] // 16)
+
+    def config(self):
+        return {"workload": self.name, "mode": "nvfp4", "dtype": "bf16", "N": 16384, "K": 16384,
+                "calls_per_step": 1, "bytes_per_call": "w read + codes and scale bytes written",
+                "l2": "flushed before every step (512 MB write + 256 MB read); 2 weight copies alternate"}
+
+
 class Moe(Layer):
     """MoE decode: 16 tokens, each routed (device-side ids) to one of 64
     experts of 1536 x 2048, 4-bit g64 bf16, one qmv_affine_gather call per step.
@@ -510,7 +556,8 @@ class Qvm(Layer):
                       "its own 151 MB weight copy"}
 
 
-WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe, "quantize": Quantize, "qvm": Qvm, "qmm": Qmm, "moe": Moe}
+WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe, "quantize": Quantize, "qvm": Qvm, "qmm": Qmm, "moe": Moe,
+             "quantize_fp": QuantizeFp}
 
 
 # ---------------------------------------------------------------- our arm --
@@ -675,6 +722,8 @@ def _oracle_sample(workload, budget_s=12.0, threads=None):
         return _oracle_quantize_sample(budget_s, threads)
     if workload == "qvm":
         return _oracle_qvm_sample(budget_s, threads)
+    if workload == "quantize_fp":
+        return _oracle_quantize_fp_sample(budget_s, threads)
     if workload == "chain8":
         spec = [(1, N, CHAIN_K, CHAIN_BITS, CHAIN_G, CHAIN_CALLS) for N in CHAIN_NS]
     elif workload == "layer":
@@ -707,6 +756,26 @@ def _oracle_sample(workload, budget_s=12.0, threads=None):
         sample.append(f"M={M} N={N} K={K}: {nrows}/{N} rows, {dt:.3f}s")
     ncalls = 1 if workload == "moe" else sum(s[-1] for s in spec)     # moe: one call = all its tokens
     return total_us / ncalls, threads, "; ".join(sample)
+
+
+def _oracle_quantize_fp_sample(budget_s, threads):
+    """The oracle FP quantizer (NVFP4) on a growing row sample of the 16384 x
+    16384 bf16 matrix, scaled to one full call."""
+    import oracle
+    N = K = 16384
+    rng = np.random.default_rng(9)
+    w = rng.standard_normal((N, K), dtype=np.float32).astype(np.float32) * np.float32(0.05)
+    wb = (w.view(np.uint32) >> 16).astype(np.uint16)
+    nrows = 16
+    while True:
+        t0 = time.perf_counter()
+        oracle.quantize_fp(np.ascontiguousarray(wb[:nrows]), nrows, K, "nvfp4", "bf16",
+                           global_scale=np.float32(0.05 * 4 / (6 * 448)), threads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s / 4 or nrows >= N:
+            break
+        nrows = min(N, nrows * 4)
+    return dt * 1e6 * (N / nrows), threads, f"NVFP4 N={N} K={K} bf16: {nrows}/{N} rows, {dt:.3f}s"
 
 
 def _oracle_qvm_sample(budget_s, threads):

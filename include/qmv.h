@@ -245,6 +245,31 @@ int qmv_qvm_affine_noalloc(const void* x, const void* w_packed, const void* scal
                            int group_size, int dtype, void* stream);
 
 /*
+ * qmv_quantize_fp -- block-scaled FP quantizer (wh-iron kernel-op coverage
+ * audit, "fp_quantized (fp4/fp8 quant + dequant)" row: a per-group max
+ * scale and mantissa rounding, saturating with no NaN or infinity; the pages
+ * give no formula for the scale, this is the reading used).
+ *   w        [N, K] row-major in dtype (finite values)
+ *   mode QMV_MXFP4:      w_packed [N, K/2] E2M1 codes (low nibble = even k),
+ *                        scales [N, K/32] E8M0 bytes; K % 32 == 0
+ *   mode QMV_MXFP8_E4M3: w_packed [N, K] E4M3 codes, scales [N, K/32] E8M0
+ *   mode QMV_NVFP4:      w_packed [N, K/2] E2M1 codes, scales [N, K/16] E4M3
+ *                        bytes, global_scale: DEVICE pointer to one float g
+ *                        (required, normal and > 0); K % 16 == 0
+ *   global_scale must be NULL for the MX modes.
+ * MX: E8M0 byte = clamp(floor(log2(amax)) - emax + 127, 0, 254) per block
+ * (emax 2 for E2M1, 8 for E4M3; 0 when amax is 0), element w * 2^(127 - byte).
+ * NVFP4: scale = nearest E4M3 to amax / (6 g), element w / (scale * g), both
+ * in fp32.  Each code is the nearest element, ties to the even code,
+ * saturating at the largest finite element (6 or 448); the sign bit is set
+ * for negative elements.  The output is the layout qmv_fp reads.  Alignment:
+ * w to its element (QMV_EALIGN otherwise); 16-byte aligned w and w_packed use
+ * vector loads and stores.  Asynchronous on `stream`; caller-owned buffers.
+ */
+int qmv_quantize_fp(const void* w, void* w_packed, void* scales, const float* global_scale, int N, int K,
+                    int mode, int dtype, void* stream);
+
+/*
  * qmv_dequant_affine_f32 -- check kernel: w_out[n*K + k] = fp32 value of
  * scale * q + bias, computed with one rounding (fmaf) from the stored dtype
  * scale / bias.  Uses the same device decoders as qmv_affine.  w_out is a

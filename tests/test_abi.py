@@ -261,3 +261,20 @@ def test_gather_validation_before_any_launch():
     assert g(xb=2) == EINVAL
     assert g(bits=7) == EUNSUP
     assert g(M=0) == 0
+
+
+def test_quantize_fp_validation_before_any_launch():
+    F = FAKE
+
+    def qf(w=F, wq=F, s=F, g=None, N=8, K=128, mode=0, dt=2):
+        return L.qmv_quantize_fp(w, wq, s, g, N, K, mode, dt, None)
+
+    assert qf(mode=5) == EUNSUP
+    assert qf(dt=7) == EUNSUP
+    assert qf(K=48) == EINVAL                   # MX blocks of 32
+    assert qf(mode=1, K=40, g=F) == EINVAL      # NVFP4 blocks of 16
+    assert qf(mode=1) == EINVAL                 # NVFP4 needs the global scale
+    assert qf(g=F) == EINVAL                    # MX takes none
+    assert qf(w=None) == EINVAL
+    assert qf(w=F + 1) == EALIGN
+    assert qf(N=0) == 0

@@ -18,7 +18,7 @@ import os
 
 __all__ = [
     "QmvError", "qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
-    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_affine_gather", "qmv_qmm_affine", "qmv_qvm_affine",
+    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_quantize_fp", "qmv_affine_gather", "qmv_qmm_affine", "qmv_qvm_affine",
     "qmv_qvm_workspace_bytes", "qmv_qvm_affine_noalloc", "qmv_status_string",
     "qmv_last_cuda_error",
     "qmv_describe_plan", "qmv_force_config", "DTYPES", "FP_MODES", "LIB_PATH", "lib",
@@ -59,6 +59,8 @@ _lib.qmv_quantize_affine.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
 _lib.qmv_qvm_affine.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p]
 _lib.qmv_qmm_affine.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
 _lib.qmv_affine_gather.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _p]
+_lib.qmv_quantize_fp.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _p]
+_lib.qmv_quantize_fp.restype = _i
 _lib.qmv_affine_gather.restype = _i
 _lib.qmv_qmm_affine.restype = _i
 _lib.qmv_qvm_workspace_bytes.argtypes = [_i, _i]
@@ -180,6 +182,14 @@ def qmv_quantize_affine(w, w_packed, scales, biases, N, K, bits, group_size, dty
     dtype, all caller-owned device buffers."""
     _check(_lib.qmv_quantize_affine(_ptr(w), _ptr(w_packed), _ptr(scales), _ptr(biases), N, K, bits,
                                     group_size, _dtype(dtype), _stream(stream)), "qmv_quantize_affine")
+
+
+def qmv_quantize_fp(w, w_packed, scales, global_scale, N, K, mode, dtype, stream=None):
+    """Block-scaled FP quantizer (C ABI qmv_quantize_fp): w [N, K] in dtype ->
+    codes and scale bytes in the layout qmv_fp reads; global_scale is a device
+    float tensor for NVFP4, None for the MX modes."""
+    _check(_lib.qmv_quantize_fp(_ptr(w), _ptr(w_packed), _ptr(scales), _ptr(global_scale), N, K, FP_MODES[mode],
+                                _dtype(dtype), _stream(stream)), "qmv_quantize_fp")
 
 
 def qmv_affine_gather(x, w_packed, scales, biases, expert_ids, y, M, N, K, bits, group_size, dtype, n_tokens,

@@ -805,6 +805,22 @@ int qmv_quantize_affine(const void* w, void* w_packed, void* scales, void* biase
                                               static_cast<cudaStream_t>(stream)));
 }
 
+int qmv_quantize_fp(const void* w, void* w_packed, void* scales, const float* global_scale, int N, int K,
+                    int mode, int dtype, void* stream) {
+    if (fp_family(mode) < 0) return QMV_EUNSUPPORTED;
+    if (dtype != QMV_F32 && dtype != QMV_F16 && dtype != QMV_BF16) return QMV_EUNSUPPORTED;
+    const int blk = mode == QMV_NVFP4 ? 16 : 32;
+    if (N < 0 || K < 0 || K % blk != 0) return QMV_EINVAL;
+    if ((mode == QMV_NVFP4) != (global_scale != nullptr)) return QMV_EINVAL;
+    if (N == 0 || K == 0) return QMV_OK;
+    if (!w || !w_packed || !scales) return QMV_EINVAL;
+    const size_t eb = elem_bytes(dtype);
+    if (!aligned(w, eb) || (global_scale && !aligned(global_scale, 4))) return QMV_EALIGN;
+    const bool vec = aligned(w, 16) && aligned(w_packed, mode == QMV_NVFP4 ? 8 : 16);
+    return finish(qmv::launch_quantize_fp(mode, dtype, w, w_packed, scales, global_scale, N, K, vec,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 int qmv_affine_gather(const void* x, const void* w_packed, const void* scales, const void* biases,
                       const int* expert_ids, void* y, int M, int N, int K, int bits, int group_size, int dtype,
                       int n_tokens, int n_experts, int x_batched, void* stream) {

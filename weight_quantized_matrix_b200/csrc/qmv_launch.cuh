@@ -81,6 +81,11 @@ cudaError_t launch_qvm_affine(int bits, int dtype, const void* x, const void* w,
                               const void* biases, void* y, void* workspace, int M, int N, int K, int G,
                               cudaStream_t st);
 
+// FP quantizer (qmv_quantize_fp.cu): mode 0 MXFP4, 1 NVFP4, 2 MXFP8-E4M3; vec =
+// 16-byte loads of w and vector stores of the codes (aligned buffers).
+cudaError_t launch_quantize_fp(int mode, int dtype, const void* w, void* wq, void* scales, const float* gscale,
+                               int N, int K, bool vec, cudaStream_t st);
+
 // Affine quantizer (qmv_quantize.cu): w [N, K] in dtype -> packed codes,
 // scales, biases; vec = 16-byte loads of w (aligned rows).
 cudaError_t launch_quantize_affine(int bits, int dtype, const void* w, void* wq, void* scales, void* biases,
