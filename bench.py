@@ -110,6 +110,19 @@ def traffic_for(kernel_key):
     return e.get("dram_bytes_per_launch")
 
 
+def max_over_ranks(values, world, device):
+    """Each value's maximum over all ranks (one all_reduce MAX); the values
+    themselves at world 1.  The timed totals of every rank go through it, so
+    a multi-GPU run reports the slowest replica."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 # ----------------------------------------------------------------- clocks --
 class ClockSampler:
     """nvidia-smi samples (20 ms period) taken while the GPU is under load: it
@@ -663,12 +676,7 @@ def run_ours(args, rank, world, local_rank):
             per_group.append(float(np.mean([a.elapsed_time(b) for a, b in ev])))   # ms per group replay
         del step_graphs, group_graphs
 
-    tot_ms = float(step_ms.sum())
-    tot_ms_e2e = float(step_ms_e2e.sum())
-    if world > 1:
-        t = torch.tensor([tot_ms, tot_ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        tot_ms, tot_ms_e2e = float(t[0]), float(t[1])
+    tot_ms, tot_ms_e2e = max_over_ranks([float(step_ms.sum()), float(step_ms_e2e.sum())], world, dev)
     calls = wl.calls_per_step * args.steps * world
     us_per_call = tot_ms * 1e3 / calls
     us_per_call_e2e = tot_ms_e2e * 1e3 / calls
