@@ -1,7 +1,7 @@
 """Shared pytest configuration: the ``gpu`` marker is registered in pytest.ini.
 
 GPU tests fail loudly (never skip) when CUDA or the compiled library is
-missing, so a run on a GPU machine can never pass on a fallback path.
+missing, so a GPU run can never pass on a fallback path.
 """
 import os
 import sys
