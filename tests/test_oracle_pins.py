@@ -498,8 +498,9 @@ def _f32_specials():
 
 
 def test_f32_to_f16_matches_numpy():
-    for v in _f32_specials():
-        assert oracle.f32_to_f16(v) == int(np.float32(v).astype(np.float16).view(np.uint16)), v
+    with np.errstate(over="ignore"):                 # values past the f16 range round to infinity
+        for v in _f32_specials():
+            assert oracle.f32_to_f16(v) == int(np.float32(v).astype(np.float16).view(np.uint16)), v
 
 
 def test_f32_to_bf16_matches_torch():
