@@ -278,3 +278,9 @@ def test_quantize_fp_validation_before_any_launch():
     assert qf(w=None) == EINVAL
     assert qf(w=F + 1) == EALIGN
     assert qf(N=0) == 0
+
+
+@pytest.mark.parametrize("name", _declared())
+def test_python_binding_has_every_entry_point(name):
+    """The binding exposes each C-ABI entry point under the same name."""
+    assert callable(getattr(q, name, None)), name
