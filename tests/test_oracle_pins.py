@@ -688,3 +688,51 @@ def test_quantize_fp_dequant_error_bound(mode):
     assert (err <= bound * (1 + 1e-6) + ulp + 1e-30).all()
     sat = d > top
     assert (np.abs(np.abs(deq[sat]) - (top * bs)[sat]) <= ulp[sat]).all()
+
+
+# ------------------------------------------------------------ SwiGLU pins ----
+def _swiglu_case(M, N, K, bits, group, seed):
+    cg = synth.affine_case(M, N, K, bits, group, "f32", seed=seed)
+    cu = synth.affine_case(M, N, K, bits, group, "f32", seed=seed + 1)
+    return cg["x"][0], (cg["w"][0], cg["scales"][0], cg["biases"][0]), (cu["w"][0], cu["scales"][0], cu["biases"][0])
+
+
+def test_swiglu_unit_x_closed_form():
+    """x = e_k: gate and up are single dequantized weights (test-side reader,
+    library casts), and mid = g * u / (1 + e^-g) by the math library."""
+    N, K, bits, group = 6, 64, 4, 32
+    _, (wg, sg, bg), (wu, su, bu) = _swiglu_case(1, N, K, bits, group, seed=70)
+    for k in (0, 33, 63):
+        x = np.zeros((1, K), dtype=np.float32); x[0, k] = 1.0
+        mid, g, u, _, _ = oracle.qmv_affine_swiglu(x, wg, sg, bg, wu, su, bu, 1, N, K, bits, group, "f32")
+        for n in range(N):
+            gv = float(sg[n, k // group]) * _py_codes(wg[n], K, bits)[k] + float(bg[n, k // group])
+            uv = float(su[n, k // group]) * _py_codes(wu[n], K, bits)[k] + float(bu[n, k // group])
+            assert g[0, n] == gv and u[0, n] == uv
+            assert math.isclose(mid[0, n], gv * uv / (1.0 + math.exp(-gv)), rel_tol=1e-15, abs_tol=1e-300)
+
+
+def test_swiglu_clamp_route_weight_and_limits():
+    """The clamp limits gate from above and up on both sides only when it is
+    above 1e-6; the route weight scales mid exactly; silu(g) -> g for large g
+    and -> 0 for very negative g."""
+    M, N, K, bits, group = 2, 8, 128, 4, 64
+    x, (wg, sg, bg), (wu, su, bu) = _swiglu_case(M, N, K, bits, group, seed=80)
+    args = (x, wg, sg, bg, wu, su, bu, M, N, K, bits, group, "f32")
+    m0, g, u, _, _ = oracle.qmv_affine_swiglu(*args)
+    m2, _, _, _, _ = oracle.qmv_affine_swiglu(*args, route_weight=2.0)
+    assert np.array_equal(m2, 2.0 * m0)
+    tiny, _, _, _, _ = oracle.qmv_affine_swiglu(*args, clamp=1e-7)          # at or below 1e-6: no clamp
+    assert np.array_equal(tiny, m0)
+    c = float(np.median(np.abs(np.concatenate([g.ravel(), u.ravel()]))))
+    mc, _, _, _, _ = oracle.qmv_affine_swiglu(*args, clamp=c)
+    gc, uc = np.minimum(g, c), np.clip(u, -c, c)
+    assert np.allclose(mc, gc * uc / (1.0 + np.exp(-gc)), rtol=1e-15, atol=0)
+    assert (np.abs(uc) <= c).all() and (gc <= c).all() and not np.array_equal(mc, m0)
+    # limits of silu on planted rows: scale every bias of the gate to +-40
+    big = np.full_like(bg, 40.0); neg = np.full_like(bg, -40.0)
+    zero_w = np.zeros_like(wg); ones = np.ones((M, K), dtype=np.float32) / K
+    mp, gp, up, _, _ = oracle.qmv_affine_swiglu(ones, zero_w, sg, big, wu, su, bu, M, N, K, bits, group, "f32")
+    assert np.allclose(mp, gp * up, rtol=1e-15)                               # silu(40) = 40 (1 - 4e-18)
+    mn, _, _, _, _ = oracle.qmv_affine_swiglu(ones, zero_w, sg, neg, wu, su, bu, M, N, K, bits, group, "f32")
+    assert (np.abs(mn) < 1e-15 * np.abs(up) + 1e-300).all()                   # silu(-40) = -40 e^-40
