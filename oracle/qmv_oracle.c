@@ -308,21 +308,22 @@ uint32_t oracle_f32_to_f16(float f) {
 /* ---------------------------------------------------------------------------
  * Affine quantizer (wh-iron kernel-op coverage audit, the "quantized
  * (affine_quantize / affine_dequantize)" row: quantize and dequantize for
- * every width).  The pages name these kernels but do not state their
- * arithmetic; this is the plainest reading consistent with w = scale*q + bias
- * (MLX quantized_nax.h, dequantize): for each group of `group` consecutive
- * weights of a row,
+ * every width; the audit's Track 2 describes the scheme as a min/max range
+ * mapped to a scale and a bias).  The pages name these kernels but do not
+ * state their arithmetic; this is the plainest reading consistent with the
+ * dequantization w = scale*q + bias (MLX quantized_nax.h, dequantize), whose
+ * inverse is the quotient (w - bias) / scale: for each group of `group`
+ * consecutive weights of a row,
  *     bias  = min(w),  scale = (max(w) - min(w)) / (2^bits - 1),
- * both rounded to the element type, inv = 1 / scale_T, and
- *     q = nearest integer, ties to even, to (w - bias_T) * inv,
- * clamped to [0, 2^bits - 1] (q = 0 when scale_T is 0, and when the
- * quotient is NaN: a zero difference times the infinite reciprocal of a
- * scale below 2^-128).  min and max are taken in element order with strict
- * comparisons, so of +0 and -0 the first one met is kept.  Weights are
- * finite.  Every step that decides a code is one fp32 IEEE operation (divide
- * once per group, then subtract, multiply, round per weight), the precision
- * the CUDA kernel takes the same decision in.  Codes are packed
- * LSB first exactly as oracle_affine_code reads them.  Rows [n0, n1).
+ * both rounded to the element type, and
+ *     q = nearest integer, ties to even, to (w - bias_T) / scale_T,
+ * the difference and the quotient each one fp32 IEEE operation (one correctly
+ * rounded division per weight), clamped to [0, 2^bits - 1].  q = 0 when
+ * scale_T is 0 and when the quotient is NaN (an infinite difference over an
+ * infinite scale, from a range beyond the fp32 maximum).  min and max are
+ * taken in element order with strict comparisons, so of +0 and -0 the first
+ * one met is kept.  Weights are finite.  Codes are packed LSB first exactly as
+ * oracle_affine_code reads them.  Rows [n0, n1).
  * ------------------------------------------------------------------------- */
 static float load_f32(const void* p, size_t i, int dtype) {
     return (float)load_elem(p, i, dtype);                  /* exact: every T is an fp32 value */
@@ -363,14 +364,13 @@ void oracle_quantize_affine(const void* w, uint8_t* wq, void* scales, void* bias
             const size_t gi = (size_t)(n * (K / group) + g0 / group);
             const float sT = store_round(scales, gi, dtype, scale);
             const float bT = store_round(biases, gi, dtype, lo);
-            const float inv = sT != 0.0f ? 1.0f / sT : 0.0f;   /* fp32 */
             for (long long k = g0; k < g0 + group; ++k) {
                 uint32_t q = 0;
                 if (sT != 0.0f) {
-                    const float d = (load_f32(w, (size_t)(n * K + k), dtype) - bT) * inv;  /* fp32, fp32 */
-                    /* clamp, then round to nearest even; a NaN quotient (a zero
-                       difference times an infinite reciprocal) is code 0 */
-                    q = !(d > 0.0f) ? 0u : d >= (float)qmax ? (uint32_t)qmax : (uint32_t)rintf(d);
+                    const float diff = load_f32(w, (size_t)(n * K + k), dtype) - bT;   /* fp32 */
+                    const float d = diff / sT;                                          /* fp32 */
+                    const float r = rintf(d);                      /* nearest, ties to even */
+                    q = !(r > 0.0f) ? 0u : r >= (float)qmax ? (uint32_t)qmax : (uint32_t)r;
                 }
                 put_code(row, k, bits, q);
             }

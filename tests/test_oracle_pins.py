@@ -471,14 +471,18 @@ def _emulate_kernel_bf16(case, widened):
     return torch.from_numpy(y).to(torch.bfloat16).to(torch.float64).numpy()
 
 
-def test_low_precision_sum_x_fails_tolerance():
-    case = synth.affine_case(1, 512, 2560, 4, 64, "bf16", seed=2, precision=True)
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6])
+def test_low_precision_sum_x_fails_tolerance(bits):
+    """The precision case at every width it names: sum(x) widened per element
+    passes every output without the floor clause; the bf16-pairwise sum(x)
+    mutant fails a majority of the outputs."""
+    case = synth.affine_case(1, 512, 2560, bits, 64, "bf16", seed=2, precision=True)
     y_ref, absdot = oracle.qmv_affine(case["x"][0], case["w"][0], case["scales"][0], case["biases"][0],
-                                      1, 512, 2560, 4, 64, "bf16", threads=8)
-    ok_good, _ = check(_emulate_kernel_bf16(case, True)[None, :], y_ref, absdot, "bf16")
+                                      1, 512, 2560, bits, 64, "bf16", threads=8)
+    ok_good, needed = check(_emulate_kernel_bf16(case, True)[None, :], y_ref, absdot, "bf16")
     ok_bad, _ = check(_emulate_kernel_bf16(case, False)[None, :], y_ref, absdot, "bf16")
-    assert ok_good.all()
-    assert (~ok_bad).sum() >= 10, int((~ok_bad).sum())
+    assert ok_good.all() and needed == 0
+    assert (~ok_bad).sum() > 256, int((~ok_bad).sum())
 
 
 # ------------------------------------------------------------- quantizer ----
@@ -553,14 +557,37 @@ def test_quantize_signed_zero_extremes_keep_the_first_met():
     assert np.signbit(bi[1, 0]) and not np.signbit(bi[0, 0])
 
 
-def test_quantize_infinite_reciprocal():
-    """A subnormal range: scale below 2^-128, 1 / scale = inf; the weight equal
-    to the bias (0 * inf = NaN) is code 0, every larger weight the top code."""
+def test_quantize_subnormal_range_takes_the_nearest_code():
+    """A range in the fp32 subnormals: scale below 2^-128 (its reciprocal would
+    overflow), yet the quotient (w - bias) / scale is an ordinary number and
+    every code is the nearest grid point (exact rationals)."""
     w = (np.arange(32, dtype=np.float32) * np.float32(1e-41)).reshape(1, 32)
     wq, sc, bi = oracle.quantize_affine(w, 1, 32, 4, 32, "f32")
     assert 0 < sc[0, 0] < 2.0 ** -128 and bi[0, 0] == 0.0
     codes = oracle.affine_codes(wq[0], 32, 4)
-    assert codes[0] == 0 and (codes[1:] == 15).all()
+    s = Fraction(float(sc[0, 0]))
+    for k in range(32):
+        d = [abs(Fraction(float(w[0, k])) - s * c) for c in range(16)]
+        assert d[int(codes[k])] == min(d), (k, codes[k])
+    assert codes[0] == 0 and codes[31] == 15
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_quantize_exact_half_quotients_round_to_even(dtype):
+    """Group min 0 and max 45 at 4 bits: scale 45 / 15 = 3 exactly.  The
+    weights 7.5 and 13.5 sit exactly halfway between grid points (quotients 2.5
+    and 4.5): the nearest-integer rule with ties to even gives codes 2 and 4.
+    (A reciprocal-times-difference reading would give 3 and 5 here: 1 / 3
+    rounds up in fp32, pushing both products just past the half.)"""
+    w = np.zeros((1, 32), dtype=np.float32)
+    w[0, 1] = 45.0
+    w[0, 2] = 7.5
+    w[0, 3] = 13.5
+    w[0, 4] = 10.5                      # quotient 3.5: ties to 4
+    wq, sc, bi = oracle.quantize_affine(_bits_of(w, dtype), 1, 32, 4, 32, dtype)
+    assert np.array_equal(sc, _bits_of([3.0], dtype).reshape(1, 1))
+    codes = oracle.affine_codes(wq[0], 32, 4)
+    assert list(codes[:5]) == [0, 15, 2, 4, 4]
 
 
 def test_quantize_constant_group():
@@ -573,7 +600,7 @@ def test_quantize_constant_group():
 def test_quantize_nearest_code_brute_force(bits):
     """Each code is the nearest of the 2^b grid points bias_T + q scale_T to w
     (exact rationals), except where the distance to two grid points is equal
-    within fp32 rounding of (w - bias_T) * (1 / scale_T)."""
+    within the fp32 rounding of the difference and the quotient."""
     rng = np.random.default_rng(bits)
     group, N, K = 32, 4, 64
     w = (rng.standard_normal((N, K)) * 0.3).astype(np.float32)
