@@ -132,9 +132,11 @@ int qmv_fp_batched(const void* x, const void* w_packed, const void* scales,
  *   scales, biases  [N, K/group_size] in dtype, out
  * For each group of group_size consecutive weights of a row: bias = min,
  * scale = (max - min) / (2^bits - 1), both rounded to dtype (to nearest, ties
- * to even); inv = 1 / scale and q = rint((w - bias) * inv), in fp32 with the
- * rounded values, clamped to [0, 2^bits - 1]; q = 0 when the rounded scale
- * is 0.
+ * to even); q = rint((w - bias) / scale), the difference and the quotient each
+ * one fp32 operation on the rounded values (ties to even), clamped to
+ * [0, 2^bits - 1]; q = 0 when the rounded scale is 0 or the quotient is NaN.
+ * (The kernel multiplies by one reciprocal per group and divides only where
+ * that could change a code: the codes are those of the division.)
  * bits in {2,3,4,5,6,8}, group_size in {32,64,128}, K % group_size == 0.
  * Alignment: w, scales, biases to their element size, w_packed to 4 bytes
  * (QMV_EALIGN otherwise); 16-byte aligned rows of w are read 16 bytes at a
@@ -167,6 +169,36 @@ int qmv_quantize_affine(const void* w, void* w_packed, void* scales, void* biase
 int qmv_affine_gather(const void* x, const void* w_packed, const void* scales, const void* biases,
                       const int* expert_ids, void* y, int M, int N, int K, int bits, int group_size,
                       int dtype, int n_tokens, int n_experts, int x_batched, void* stream);
+
+/*
+ * qmv_affine_swiglu -- decode gate + up projection fused with the SwiGLU
+ * activation (DS4 moe.metal: kernel_mul_mv_id_q4_K_pair_swiglu_f32, the
+ * paired gate / up matvec whose lanes derive the routed SwiGLU input, and
+ * kernel_dsv4_moe_swiglu_weight for the activation; wh-iron kernel-op
+ * coverage audit, "moe routed-expert decode fuse" row: the activation fused
+ * into the gate / up qmv epilogue).  For every x row m and output n:
+ *     g = sum_k x[m,k] * dequant(W_gate)[n,k],  u = same with W_up,
+ *     if clamp > 1e-6:  g = min(g, clamp),  u = min(max(u, -clamp), clamp),
+ *     mid[m, n] = g / (1 + exp(-g)) * u * route_weight[m],
+ * with g and u accumulated in fp32 exactly as qmv_affine does, the
+ * activation in fp32 and one rounding of mid to dtype.  gate and up are not
+ * written.
+ *   w_gate, s_gate, b_gate   the gate matrix, as qmv_affine's w_packed,
+ *   w_up, s_up, b_up         scales, biases (same N, K, bits, group_size)
+ *   route_weight  DEVICE pointer to M floats (one per x row, read after the
+ *                 previous kernel in the stream completes), or NULL for 1
+ *   mid           [M, N] dtype
+ *   clamp         >= 0 (QMV_EINVAL if negative or NaN); at or below 1e-6 no
+ *                 clamping
+ * Other arguments, alignment and errors as qmv_affine; both matrices take
+ * the wide-load path when both are 16-byte aligned.  Runs the row-tiled
+ * CUDA-core kernel over the 2N interleaved gate / up rows, so each warp holds
+ * both sums of its outputs.
+ */
+int qmv_affine_swiglu(const void* x, const void* w_gate, const void* s_gate, const void* b_gate,
+                      const void* w_up, const void* s_up, const void* b_up, const float* route_weight,
+                      void* mid, int M, int N, int K, int bits, int group_size, int dtype, float clamp,
+                      void* stream);
 
 /*
  * qmv_qmm_affine -- small-M quantized matmul, y = x * dequant(W)^T for up to
@@ -232,7 +264,9 @@ size_t qmv_qvm_workspace_bytes(int M, int N);
  *   return QMV_EUNSUPPORTED before any launch.
  *   The first call on a device looks up the scratch's device address (once per
  *   device, with that device current); make that first call before any stream
- *   capture.  Each call clears the part of the scratch it uses on `stream`,
+ *   capture.  The address is kept for the life of the process: calls after a
+ *   cudaDeviceReset() of that device are not supported (the module reloads
+ *   and the array may move).  Each call clears the part of the scratch it uses on `stream`,
  *   then launches.  Every call, on every stream, shares the one array:
  *   calls that overlap on the GPU race and give wrong results, so order them
  *   (one stream, or events).
@@ -326,8 +360,12 @@ int qmv_device_fault(unsigned int* code, int clear);
  * warps_rows (16-row tiles per block) up to 12 each, or -1; the weight-ring
  * kernels run warps_k * warps_rows in {8, 12} compute warps and a producer
  * warp.
- * Unsupported combinations fall back to automatic for that field.  Not
- * thread-safe with concurrent calls; meant for single-threaded harnesses.
+ * Unsupported combinations fall back to automatic for that field.
+ * NOT FOR PRODUCTION USE: this is process-wide state for the parity tests and
+ * the benchmark's sweeps; it is not thread-safe with concurrent calls and
+ * overrides the picker for every caller in the process.  (Likewise the
+ * environment variable QMV_PDL=0, read once per process, turns programmatic
+ * dependent launch off; it exists for A/B timing only.)
  */
 void qmv_force_config(int path, int rows_per_warp, int warps_k, int warps_rows);
 

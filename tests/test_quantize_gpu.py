@@ -1,9 +1,10 @@
 """GPU parity of the affine quantizer (qmv_quantize_affine) against the oracle.
 
-The packed codes, scales and biases are integers and bit patterns decided by
-the same fp32 operations on both sides (min / max, subtract, a reciprocal per
-group and a multiply per weight, round to
-nearest even, round to the element type), so every byte must match exactly.
+The packed codes, scales and biases are integers and bit patterns defined by
+fp32 operations (min / max, subtract, divide, round to nearest even, round to
+the element type).  The kernel reaches the same codes through a reciprocal per
+group with an exact-division fallback near every rounding edge, so every byte
+must match exactly.
 """
 from __future__ import annotations
 
@@ -83,7 +84,9 @@ def test_quantize_unaligned_rows_take_the_scalar_path(q, dtype):
 def test_quantize_special_groups(q, dtype):
     """Constant groups (scale 0, codes 0), groups of +0 / -0 in both orders
     and with a zero minimum or maximum, a tiny range, exact ties of the code
-    grid, a subnormal range whose scale has an infinite reciprocal."""
+    grid, a subnormal range whose scale has an infinite reciprocal, exact
+    half quotients (ties to even by the division), and (f32) a range past the
+    fp32 maximum (infinite scale: every code 0)."""
     N, K, group, bits = 5, 256, 64, 4
     w = np.zeros((N, K), dtype=np.float32)
     w[0, :64] = 0.75                                   # constant
@@ -101,6 +104,10 @@ def test_quantize_special_groups(q, dtype):
     rng = np.random.default_rng(5)
     w[3] = rng.standard_normal(K).astype(np.float32)
     w[4, :64] = np.arange(64, dtype=np.float32) * np.float32(1e-41)              # subnormal range
+    w[4, 64:128] = 0.0
+    w[4, 65], w[4, 66], w[4, 67], w[4, 68] = 45.0, 7.5, 13.5, 10.5               # scale 3: quotients 2.5, 4.5, 3.5
+    if dtype == "f32":
+        w[4, 128:192] = np.linspace(-3e38, 3e38, 64, dtype=np.float32)          # max - min overflows
     t = torch.from_numpy(w).to({"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[dtype])
     wb = t.view(torch.int32 if dtype == "f32" else torch.int16).numpy().view(STORAGE[dtype]).copy()
     got = _run(q, wb, N, K, bits, group, dtype)

@@ -5,17 +5,30 @@
 // coverage audit, "quantized (affine_quantize / affine_dequantize)" row) but
 // do not state their arithmetic.  The reading implemented here is the
 // plainest one consistent with w = scale * q + bias (MLX quantized_nax.h,
-// dequantize): per group of G consecutive weights of a row,
+// dequantize), whose inverse is the quotient (w - bias) / scale: per group of
+// G consecutive weights of a row,
 //     bias  = min(w),  scale = (max(w) - min(w)) / (2^B - 1),
-// both rounded to T (to nearest, ties to even), inv = 1 / scale_T, and
-//     q = rint((w - bias_T) * inv)  clamped to [0, 2^B - 1]
-// (q = 0 when scale_T is 0 and when the product is NaN), every step one fp32
-// IEEE operation (one division per group; a division per weight made the
-// kernel compute-bound).  min and max keep, of +0 and -0, the first met in
-// element order (what strict in-order comparisons give); weights are finite.  Codes are
-// packed LSB first: with a group starting on a pack boundary (G a multiple of
-// 32), code k of the group occupies bits [k B, k B + B) of the group's byte
-// stream read as little-endian words, for every width.
+// both rounded to T (to nearest, ties to even), and
+//     q = rint((w - bias_T) / scale_T)  clamped to [0, 2^B - 1]
+// with the difference and the quotient each one fp32 IEEE operation (q = 0
+// when scale_T is 0 or the quotient is NaN).  min and max keep, of +0 and -0,
+// the first met in element order (what strict in-order comparisons give);
+// weights are finite.  Codes are packed LSB first: with a group starting on a
+// pack boundary (G a multiple of 32), code k of the group occupies bits
+// [k B, k B + B) of the group's byte stream read as little-endian words, for
+// every width.
+//
+// The division per weight is exact but slow; the kernels get the same codes
+// from one reciprocal per group.  With inv = 1 / scale_T rounded to fp32 and t
+// the fp32 product (w - bias_T) * inv, t lies within 2.0001 * 2^-24 |Q| of the
+// exact quotient Q (two roundings, while inv and t are normal) and the
+// correctly rounded quotient d within 2^-24 |Q|, so |t - d| <= 3.0001 * 2^-24
+// |Q|.  When t is
+// farther than that from every half-integer, t and d round (and clamp) to the
+// same code.  The kernels test the clamped t against the conservative margin
+// (2^B - 1) * 2^-21 and redo a weight with the division when it is closer, or
+// when the reciprocal is not a normal number (a scale beyond 2^125 or below
+// 2^-125): the codes are those of the division, bit for bit.
 //
 // Two forms: quantize_affine_tiles (aligned buffers: a warp double-buffers 32
 // groups at a time through shared memory for coalesced loads and stores) and
@@ -48,14 +61,18 @@ template <> struct QT<__nv_bfloat16> {
     static __device__ __forceinline__ float rt(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 };
 
-// Code of v: (v - bias_T) * inv clamped to [0, QMAX] (a NaN product -- a zero
-// difference times the infinite reciprocal of a scale below 2^-128 -- clamps
-// to 0), then rounded to the nearest integer, ties to even, by adding 2^23: an
-// fp32 in [2^23, 2^24) has unit spacing, so the sum is 2^23 plus the rounded
-// value and its low bits are the code.  Two values per packed fp32x2 op.
+// Codes of v[0..E): (v - bias_T) * inv clamped to [0, QMAX], then rounded to
+// the nearest integer, ties to even, by adding 2^23: an fp32 in [2^23, 2^24)
+// has unit spacing, so the sum is 2^23 plus the rounded value and its low bits
+// are the code.  Two values per packed fp32x2 op.  Returns true when some
+// clamped product lies within QMAX * 2^-21 of a half-integer, where it might
+// round differently from the quotient (the caller redoes those with
+// exact_code).
 template <int QMAX, int E>
-__device__ __forceinline__ void quantize_codes(const float* v, float bT, float inv, uint32_t* q) {
+__device__ __forceinline__ bool quantize_codes(const float* v, float bT, float inv, uint32_t* q) {
     static_assert(E % 2 == 0, "pairs");
+    constexpr float EDGE = 0.5f - (float)QMAX * 4.76837158203125e-07f;      // 0.5 - QMAX * 2^-21
+    bool near = false;
 #pragma unroll
     for (int e = 0; e < E; e += 2) {
         const float2 d = mul2(add2(make_float2(v[e], v[e + 1]), make_float2(-bT, -bT)), make_float2(inv, inv));
@@ -63,7 +80,26 @@ __device__ __forceinline__ void quantize_codes(const float* v, float bT, float i
         const float2 r = add2(c, make_float2(8388608.0f, 8388608.0f));
         q[e] = __float_as_uint(r.x) & (uint32_t)QMAX;
         q[e + 1] = __float_as_uint(r.y) & (uint32_t)QMAX;
+        // c minus its rounded value (both exact): in [-0.5, 0.5]
+        const float2 f = add2(c, add2(make_float2(-r.x, -r.y), make_float2(8388608.0f, 8388608.0f)));
+        near |= (fabsf(f.x) >= EDGE) | (fabsf(f.y) >= EDGE);
     }
+    return near;
+}
+
+// The code by the defining division: rint(fl(fl(v - bias_T) / scale_T)),
+// clamped; 0 for a zero scale or a NaN quotient.
+template <int QMAX>
+__device__ __forceinline__ uint32_t exact_code(float v, float bT, float sT) {
+    if (sT == 0.0f) return 0u;
+    const float r = rintf(__fdiv_rn(__fsub_rn(v, bT), sT));
+    return !(r > 0.0f) ? 0u : r >= (float)QMAX ? (uint32_t)QMAX : (uint32_t)r;
+}
+
+// Whether the reciprocal fast path applies to a group: a zero scale (every
+// code 0, which the product with inv = 0 gives), or a normal reciprocal.
+__device__ __forceinline__ bool reciprocal_ok(float sT, float inv) {
+    return sT == 0.0f || (inv >= 2.350988701644575e-38f && inv <= 4.253529586511731e+37f);   // 2^-125, 2^125
 }
 
 // The 16 bytes at element k of a group as 16 / sizeof(T) fp32 values.
@@ -117,6 +153,7 @@ __global__ void __launch_bounds__(256) quantize_affine_kernel(const T* __restric
     DT<T>::st(biases, gi, lo);
     const float sT = QT<T>::rt(scale), bT = QT<T>::rt(lo);
     const float inv = sT != 0.0f ? __fdiv_rn(1.0f, sT) : 0.0f;
+    const bool fast = reciprocal_ok(sT, inv);
 
     // ---- pass 2: codes, packed LSB first into 32-bit words ------------------
     uint32_t* dst = wq + n * row_words + (long long)gj * (G * B / 32);
@@ -125,8 +162,8 @@ __global__ void __launch_bounds__(256) quantize_affine_kernel(const T* __restric
     auto put = [&](float v) {
         const float two[2] = {v, v};
         uint32_t qq[2];
-        quantize_codes<QMAX, 2>(two, bT, inv, qq);
-        const uint32_t q = qq[0];
+        const bool near = quantize_codes<QMAX, 2>(two, bT, inv, qq);
+        const uint32_t q = (near || !fast) ? exact_code<QMAX>(v, bT, sT) : qq[0];
         acc |= (uint64_t)q << nb;
         nb += B;
         if (nb >= 32) {
@@ -279,6 +316,7 @@ __global__ void __launch_bounds__(32) quantize_affine_tiles(const T* __restrict_
             DT<T>::st(biases, gi, lo);
             const float sT = QT<T>::rt(scale), bT = QT<T>::rt(lo);
             const float inv = sT != 0.0f ? __fdiv_rn(1.0f, sT) : 0.0f;
+            const bool fast = reciprocal_ok(sT, inv);
             uint32_t* mo = out + lane * S::OUT_STRIDE;
 #pragma unroll 1
             for (int blk = 0; blk < G / 32; ++blk) {
@@ -290,7 +328,11 @@ __global__ void __launch_bounds__(32) quantize_affine_tiles(const T* __restrict_
                     float v[E];
                     widen16<T>(my[blk * (32 / E) + cc], v);
                     uint32_t q[E];
-                    quantize_codes<QMAX, E>(v, bT, inv, q);
+                    const bool near = quantize_codes<QMAX, E>(v, bT, inv, q);
+                    if (near || !fast) {
+#pragma unroll 1
+                        for (int e = 0; e < E; ++e) q[e] = exact_code<QMAX>(v[e], bT, sT);
+                    }
 #pragma unroll
                     for (int e = 0; e < E; ++e) {
                         const int p = (cc * E + e) * B, wi = p >> 5, sh = p & 31;
