@@ -98,11 +98,12 @@ FP_BITS = {"mxfp4": 4, "nvfp4": 4, "mxfp8": 8}
 _E4M3_NON_NAN = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
 
 
-def fp_case(M, N, K, mode, dtype, seed, batch=1):
+def fp_case(M, N, K, mode, dtype, seed, batch=1, precision=False):
     """One block-scaled FP problem.  w [batch, N, K*bits/8] u8 codes, scales
-    [batch, N, K/block] u8, global (NVFP4 only) a float32 scalar."""
+    [batch, N, K/block] u8, global (NVFP4 only) a float32 scalar.  The
+    precision case draws x ~ U(1e-4, 1e-3) (all positive, as the affine one)."""
     g = rng(seed)
-    x = g.standard_normal(size=(batch, M, K))
+    x = g.uniform(1e-4, 1e-3, size=(batch, M, K)) if precision else g.standard_normal(size=(batch, M, K))
     bits, blk = FP_BITS[mode], FP_BLOCK[mode]
     if bits == 4:
         w = random_bytes(g, (batch, N, K // 2))

@@ -9,17 +9,19 @@
 //     codes for 3/5/6-bit).  The quad's four units form a SUPER-BLOCK of the
 //     row; a k16 step takes two code pairs of each thread's unit.  A code pair
 //     becomes one bf16x2 register with a single masked OR (qmv_tc_plan.cuh):
-//     {128 + c_lo 2^s_lo, 128 + c_hi 2^s_hi}.  The 128 offsets are not removed
-//     per pair: 128 * sum(x~) of each segment is subtracted once, in fp32, in
-//     the epilogue (x~ = the fragment-ordered x values, whose sum is formed
-//     while staging x).
+//     {128 + c_lo 2^s_lo, 128 + c_hi 2^s_hi}, and one bf16x2 subtraction
+//     removes both 128 offsets exactly ({c_lo 2^s_lo, c_hi 2^s_hi}).  (Left in
+//     and taken out of the fp32 sum as 128 * sum(x~), the offsets made the
+//     accumulator carry terms about 128 / c times the codes' own: with x all
+//     positive and a symmetric zero point that cancellation cost about
+//     2.6e-5 * sum|x * w| at 2 bits, above the f32 bar.)
 //   * B (16 x 8) is x, with its 8 columns used as SLOTS (super-block in the
 //     batch, segment, x row): the B value of k-slot k in slot column c is x~[k]
 //     when code k belongs to that super-block and segment, else 0 (inactive
 //     lanes read a zero row).  A segment is min(group, super-block) codes, so
 //     every D column is the partial dot product of one x row over one
 //     (super-block, group) pair, and the exact fp32 epilogue applies that
-//     group's scale and bias:   Y += scale * (D - 128 sum x~) + bias * sum x.
+//     group's scale and bias:   Y += scale * D + bias * sum x.
 //     Filling all 8 columns with several super-blocks ("batch") runs the
 //     epilogue once per batch; more slots than 8 use several MMAs per step.
 //   * x is staged per block per K tile in shared memory, permuted into
@@ -51,10 +53,19 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Pair p of a unit as bf16x2 {128 + low field * 2^slo, 128 + high field * 2^shi}
-// (an empty high half is 128 + 0; an empty pair is 0).
+// {a.lo - b.lo, a.hi - b.hi} on bf16x2 (round to nearest; exact here).
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Pair p of a unit as bf16x2 {128 + low field * 2^slo, 128 + high field *
+// 2^shi}: one masked OR, offsets kept (an empty high half is 128 + 0; an
+// empty pair is 0).  For kernels that take the offsets out of their own fp32
+// sums.
 template <int B, int p>
-__device__ __forceinline__ uint32_t tc_pair(const uint32_t (&w)[TcGeom<B>::NW], uint32_t kbf16) {
+__device__ __forceinline__ uint32_t tc_pair_offset(const uint32_t (&w)[TcGeom<B>::NW], uint32_t kbf16) {
     constexpr TcPlanData P = tc_make_plan<B, false>();
     if constexpr (P.lo[p] < 0) {
         return 0u;
@@ -74,6 +85,21 @@ __device__ __forceinline__ uint32_t tc_pair(const uint32_t (&w)[TcGeom<B>::NW], 
         constexpr uint32_t fm = (1u << fb) - 1u;
         constexpr uint32_t m = (fm << P.slo[p]) | (P.hi[p] >= 0 ? (fm << (16 + P.shi[p])) : 0u);
         return and_or<m>(v, kbf16);      // kbf16 = 0x43004300, held in a register
+    }
+}
+
+// Pair p of a unit as bf16x2 {low field * 2^slo, high field * 2^shi}: the
+// masked OR gives {128 + c_lo 2^slo, 128 + c_hi 2^shi} (fields below bit 7 of
+// the bf16 mantissa), and one bf16x2 subtraction of {128, 128} removes the
+// offsets exactly, so every product the MMA accumulates is an exact code
+// times x~ (an empty high half is 0; an empty pair is 0).
+template <int B, int p>
+__device__ __forceinline__ uint32_t tc_pair(const uint32_t (&w)[TcGeom<B>::NW], uint32_t kbf16) {
+    constexpr TcPlanData P = tc_make_plan<B, false>();
+    if constexpr (P.lo[p] < 0) {
+        return 0u;
+    } else {
+        return bf16x2_sub(tc_pair_offset<B, p>(w, kbf16), kbf16);
     }
 }
 
@@ -372,13 +398,12 @@ __global__ void __launch_bounds__(256) qmv_tc_kernel(const Params p) {
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const int c = e & 1;
-                                float a = 0.f, b = 0.f;
+                                float a = 0.f;
                                 if (dsbi[pp][c] >= 0 && dsbi[pp][c] <= bi_) {
                                     const int sl = (sb_first + dsbi[pp][c] * wk - t0) * NGS + dgs[pp][c];
                                     a = sx[(size_t)dm[pp][c] * NSEG + sl];
-                                    b = sxt[(size_t)dm[pp][c] * NSEG + sl];
                                 }
-                                Y[pp][e] = fmaf(sc[pp][e], fmaf(-128.f, b, D[pp][e]), fmaf(bi[pp][e], a, Y[pp][e]));
+                                Y[pp][e] = fmaf(sc[pp][e], D[pp][e], fmaf(bi[pp][e], a, Y[pp][e]));
                                 D[pp][e] = 0.f;
                             }
                         bi_ = 0;

@@ -457,8 +457,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             const int e = 2 * h + c;
-                            Y[pp][e] = fmaf(sc[pp][e], fmaf(-128.f, ab.y, D[pp][e] + E[pp][e]),
-                                            fmaf(bs[pp][e], ab.x, Y[pp][e]));
+                            Y[pp][e] = fmaf(sc[pp][e], D[pp][e] + E[pp][e], fmaf(bs[pp][e], ab.x, Y[pp][e]));
                         }
                     }
             };

@@ -13,6 +13,10 @@
 // x).  The 128 offsets are removed per unit in fp32, and the unit's group
 // scale and bias applied:
 //     y += scale * (sum_unit - 128 * sum(x~_unit)) + bias * sum(x_unit).
+// (The tensor-core kernels subtract the offsets before accumulating, one more
+// instruction per pair, because their f16 / f32 outputs are held to the fp32
+// bar; this kernel serves bf16 x and y only, where the offset's fp32
+// cancellation stays inside the output's 1-ulp bar, and it is issue-bound.)
 //
 // Lanes: a warp owns a 16-row tile; lane = (r4 = lane / 8, u8 = lane % 8)
 // takes rows r4, r4 + 4, r4 + 8, r4 + 12 and unit u8 of a STEP of two
@@ -48,8 +52,8 @@ __device__ __forceinline__ float fma_bf16_f32(uint32_t a, uint32_t b, float c) {
 template <int B, int... Q>
 __device__ __forceinline__ void tcf_unit(std::integer_sequence<int, Q...>, const uint32_t (&w)[TcGeom<B>::NW],
                                          const uint32_t* xq, uint32_t kbf16, float& lo, float& hi) {
-    ((lo = fma_bf16_f32<false>(tc_pair<B, Q>(w, kbf16), xq[Q], lo),
-      hi = fma_bf16_f32<true>(tc_pair<B, Q>(w, kbf16), xq[Q], hi)),
+    ((lo = fma_bf16_f32<false>(tc_pair_offset<B, Q>(w, kbf16), xq[Q], lo),
+      hi = fma_bf16_f32<true>(tc_pair_offset<B, Q>(w, kbf16), xq[Q], hi)),
      ...);
 }
 
