@@ -254,7 +254,7 @@ def quantize_fp(w, N, K, mode, dtype, global_scale=1.0, rows=None, threads=1):
     return wq, sc
 
 
-# ---- fused gate + up with SwiGLU (kernel not built yet) --------------------
+# ---- fused gate + up with SwiGLU ---------------------------------------------
 def qmv_affine_swiglu(x, w_gate, s_gate, b_gate, w_up, s_up, b_up, M, N, K, bits, group, dtype, clamp=0.0,
                       route_weight=1.0, threads=1):
     """Decode gate/up projection fused with the SwiGLU activation (DS4
@@ -262,13 +262,18 @@ def qmv_affine_swiglu(x, w_gate, s_gate, b_gate, w_up, s_up, b_up, M, N, K, bits
     mid = silu(clamp(gate)) * clamp(up) * route_weight; wh-iron audit, swiglu
     row).  gate = x W_gate^T and up = x W_up^T are qmv_affine products (fp64);
     when clamp > 1e-6 the gate is limited to <= clamp and up to [-clamp,
-    clamp]; silu(g) = g / (1 + exp(-g)).  All in fp64.  Returns (mid, gate,
-    up, absdot_gate, absdot_up), each float64 [M, N]."""
+    clamp]; silu(g) = g / (1 + exp(-g)).  All in fp64.  route_weight is one
+    number, or one per x row (the page's kernel reads one weight per routed
+    token).  Returns (mid, gate, up, absdot_gate, absdot_up), each float64
+    [M, N]."""
     g, ag = qmv_affine(x, w_gate, s_gate, b_gate, M, N, K, bits, group, dtype, threads=threads)
     u, au = qmv_affine(x, w_up, s_up, b_up, M, N, K, bits, group, dtype, threads=threads)
     gc, uc = g, u
     if clamp > 1e-6:
         gc = np.minimum(g, clamp)
         uc = np.clip(u, -clamp, clamp)
-    silu = gc / (1.0 + np.exp(-gc))
-    return silu * uc * float(route_weight), g, u, ag, au
+    with np.errstate(over="ignore"):             # exp(-g) -> inf for very negative g: silu -> -0
+        silu = gc / (1.0 + np.exp(-gc))
+    rw = np.asarray(route_weight, dtype=np.float64)
+    rw = rw.reshape(M, 1) if rw.ndim == 1 else rw
+    return silu * uc * rw, g, u, ag, au

@@ -169,6 +169,11 @@ def test_fast_extension_forwards_status():
     assert q._fast.affine(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 128, 4, 64, 2, 1, 1, 0) == 0
     with pytest.raises(TypeError):
         q._fast.affine(FAKE)
+    # sizes beyond a C int raise instead of being narrowed (2^32 + 8 would wrap to 8)
+    with pytest.raises(OverflowError):
+        q._fast.affine(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2 ** 32 + 8, 128, 4, 64, 2, 1, 1, 0)
+    with pytest.raises(OverflowError):
+        q._fast.fp(FAKE, FAKE, FAKE, None, FAKE, 1, 8, -(2 ** 31) - 1, 1, 2, 1, 1, 0)
 
 
 def test_build_module_loads_without_the_library(tmp_path):
@@ -278,6 +283,24 @@ def test_quantize_fp_validation_before_any_launch():
     assert qf(w=None) == EINVAL
     assert qf(w=F + 1) == EALIGN
     assert qf(N=0) == 0
+
+
+def test_swiglu_validation_before_any_launch():
+    F = FAKE
+
+    def sw(x=F, wg=F, sg=F, bg=F, wu=F, su=F, bu=F, rw=None, y=F, M=1, N=64, K=128, bits=4, gs=64, dt=2,
+           clamp=0.0):
+        return L.qmv_affine_swiglu(x, wg, sg, bg, wu, su, bu, rw, y, M, N, K, bits, gs, dt, ctypes.c_float(clamp),
+                                   None)
+
+    assert sw(bits=7) == EUNSUP and sw(gs=16) == EUNSUP
+    assert sw(K=100) == EINVAL
+    assert sw(clamp=-1.0) == EINVAL and sw(clamp=float("nan")) == EINVAL
+    assert sw(wu=None) == EINVAL and sw(bu=None) == EINVAL and sw(bg=None) == EINVAL
+    assert sw(wu=F + 2) == EALIGN and sw(su=F + 1) == EALIGN and sw(rw=F + 2) == EALIGN
+    assert sw(M=9) == EUNSUP
+    assert sw(M=-1) == EINVAL
+    assert sw(M=0) == 0 and sw(N=0) == 0
 
 
 @pytest.mark.parametrize("name", _declared())

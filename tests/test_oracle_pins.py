@@ -749,6 +749,8 @@ def test_swiglu_clamp_route_weight_and_limits():
     m0, g, u, _, _ = oracle.qmv_affine_swiglu(*args)
     m2, _, _, _, _ = oracle.qmv_affine_swiglu(*args, route_weight=2.0)
     assert np.array_equal(m2, 2.0 * m0)
+    rows, _, _, _, _ = oracle.qmv_affine_swiglu(*args, route_weight=np.array([0.5, 4.0]))   # one per x row
+    assert np.array_equal(rows[0], 0.5 * m0[0]) and np.array_equal(rows[1], 4.0 * m0[1])
     tiny, _, _, _, _ = oracle.qmv_affine_swiglu(*args, clamp=1e-7)          # at or below 1e-6: no clamp
     assert np.array_equal(tiny, m0)
     c = float(np.median(np.abs(np.concatenate([g.ravel(), u.ravel()]))))

@@ -18,7 +18,7 @@ import os
 
 __all__ = [
     "QmvError", "qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
-    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_quantize_fp", "qmv_affine_gather", "qmv_qmm_affine", "qmv_qvm_affine",
+    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_quantize_fp", "qmv_affine_gather", "qmv_affine_swiglu", "qmv_qmm_affine", "qmv_qvm_affine",
     "qmv_qvm_workspace_bytes", "qmv_qvm_affine_noalloc", "qmv_status_string",
     "qmv_last_cuda_error",
     "qmv_describe_plan", "qmv_force_config", "DTYPES", "FP_MODES", "LIB_PATH", "lib",
@@ -61,6 +61,8 @@ _lib.qmv_qmm_affine.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
 _lib.qmv_affine_gather.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _p]
 _lib.qmv_quantize_fp.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _p]
 _lib.qmv_quantize_fp.restype = _i
+_lib.qmv_affine_swiglu.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, ctypes.c_float, _p]
+_lib.qmv_affine_swiglu.restype = _i
 _lib.qmv_affine_gather.restype = _i
 _lib.qmv_qmm_affine.restype = _i
 _lib.qmv_qvm_workspace_bytes.argtypes = [_i, _i]
@@ -242,6 +244,15 @@ def qmv_status_string(status: int) -> str:
 
 def qmv_last_cuda_error() -> int:
     return _lib.qmv_last_cuda_error()
+
+
+def qmv_affine_swiglu(x, w_gate, s_gate, b_gate, w_up, s_up, b_up, route_weight, mid, M, N, K, bits, group_size,
+                      dtype, clamp=0.0, stream=None):
+    """Fused gate + up projection with SwiGLU: mid = silu(clamp(x W_gate^T)) *
+    clamp(x W_up^T) * route_weight (route_weight: device float32 [M] or None)."""
+    _check(_lib.qmv_affine_swiglu(_ptr(x), _ptr(w_gate), _ptr(s_gate), _ptr(b_gate), _ptr(w_up), _ptr(s_up),
+                                  _ptr(b_up), _ptr(route_weight), _ptr(mid), M, N, K, bits, group_size,
+                                  _dtype(dtype), ctypes.c_float(clamp), _stream(stream)), "qmv_affine_swiglu")
 
 
 def qmv_describe_plan(family, M, N, K, bits=4, group_size=64, dtype="bf16", w_align16=True) -> str:

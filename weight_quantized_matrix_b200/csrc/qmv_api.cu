@@ -392,7 +392,10 @@ bool tcf_shape(int N, int K, int bits, int G, bool w16, bool s16, TcbShape* ts) 
 
 // Choose the launch shape.  Returns QMV_OK or an error (sizes too large).
 int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, bool w16, int batch, Plan* pl,
-              bool s16 = true, bool gather = false) {
+              bool s16 = true, bool gather = false, bool pair = false) {
+    // pair (fused gate + up): N counts the 2N virtual rows; only the
+    // row-tiled CUDA-core kernel has the pair epilogue
+    if (pair) gather = true;
     const FmtInfo fi = fmt_info(fam, bits);
     const bool aff = fam == qmv::FAM_AFFINE;
     int maxm = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
@@ -404,7 +407,7 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     // grid-dependency wait, one block per row) --------------------------------
     // (N <= 64 any M; up to 512 rows for one or two x rows: measured faster
     // than the row-tiled kernels on B200 up to about 1.3 MB of weights)
-    if (K > 0 && (g_forced.path == 5 || (g_forced.path < 0 && (N <= 64 || (N <= 512 && M <= 2))))) {
+    if (!pair && K > 0 && (g_forced.path == 5 || (g_forced.path < 0 && (N <= 64 || (N <= 512 && M <= 2))))) {
         const int units = K / 32;
         int thr = ((units + 31) / 32) * 32;
         if (thr > 256) thr = 256;
@@ -500,7 +503,12 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     if (g_forced.R > 0) R = g_forced.R;
     if (g_forced.wk > 0) wk = g_forced.wk;
     if (g_forced.wr > 0) wr = g_forced.wr;
-    if (!qmv::shape_instantiated(maxm, R, wide)) R = 1;
+    if (pair) {
+        if (R < 2) R = 2;
+        if (!qmv::pair_shape_instantiated(maxm, R, wide)) R = 2;
+    } else if (!qmv::shape_instantiated(maxm, R, wide)) {
+        R = 1;
+    }
     if (wk < 1) wk = 1;
     if (wk > 8) wk = 8;
     if (wr < 1) wr = 1;
@@ -686,6 +694,34 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     return finish(e);
 }
 
+// The fused gate + up projection with SwiGLU: the row-tiled CUDA-core kernel
+// over the 2N interleaved rows of the pair.
+int run_pair(const void* x, const void* wg, const void* sg, const void* bg, const void* wu, const void* su,
+             const void* bu, const float* route_w, void* y, int M, int N, int K, int bits, int G, int dtype,
+             float clamp, void* stream) {
+    const long long row_bytes = (long long)K * bits / 8;
+    Plan pl;
+    const bool w16 = aligned(wg, 16) && aligned(wu, 16);
+    int st = make_plan(qmv::FAM_AFFINE, M, 2 * N, K, bits, G, dtype, w16, 1, &pl, false, true, true);
+    if (st != QMV_OK) return st;
+    qmv::Params p;
+    p.x = x; p.w = static_cast<const uint8_t*>(wg); p.scales = sg; p.biases = bg; p.gscale = nullptr; p.y = y;
+    p.w2 = static_cast<const uint8_t*>(wu); p.scales2 = su; p.biases2 = bu;
+    p.route_w = route_w; p.act_clamp = clamp;
+    p.M = M; p.N = N; p.K = K; p.G = G;
+    p.wk = pl.wk; p.wr = pl.wr; p.tile_iters = pl.tile_iters;
+    const size_t eb = elem_bytes(dtype);
+    p.x_vec = (aligned(x, 16) && ((size_t)K * eb) % 16 == 0) ? 1 : 0;
+    p.x_bs = 0; p.w_bs = 0; p.s_bs = 0; p.y_bs = 0;
+    p.w_row = row_bytes;
+    p.ids = nullptr; p.n_experts = 0;
+    p.sps = 0; p.pitch = 0; p.fault = nullptr; p.sring = 0; p.soff = 0; p.boff = 0; p.sbw = 0;
+    p.kf32 = 0x4B000000u;
+    p.kbf16 = 0x43004300u;
+    qmv::Launch L{pl.grid, pl.block, pl.smem, static_cast<cudaStream_t>(stream), pdl_enabled()};
+    return finish(qmv::launch_affine_pair(bits, dtype, pl.maxm, pl.R, pl.wide != 0, p, L));
+}
+
 int check_affine(int bits, int group) {
     if (bits != 2 && bits != 3 && bits != 4 && bits != 5 && bits != 6 && bits != 8) return QMV_EUNSUPPORTED;
     if (group != 32 && group != 64 && group != 128) return QMV_EUNSUPPORTED;
@@ -864,6 +900,26 @@ int qmv_qmm_affine(const void* x, const void* w_packed, const void* scales, cons
         if (st != QMV_OK) return st;
     }
     return QMV_OK;
+}
+
+int qmv_affine_swiglu(const void* x, const void* w_gate, const void* s_gate, const void* b_gate, const void* w_up,
+                      const void* s_up, const void* b_up, const float* route_weight, void* mid, int M, int N, int K,
+                      int bits, int group_size, int dtype, float clamp, void* stream) {
+    int st = check_affine(bits, group_size);
+    if (st != QMV_OK) return st;
+    if (K % group_size != 0) return QMV_EINVAL;
+    if (!(clamp >= 0.0f)) return QMV_EINVAL;                     // negative or NaN clamp
+    st = check_common(x, w_gate, s_gate, mid, M, N, K, dtype);
+    if (st != QMV_OK || M == 0 || N == 0) return st;
+    if (K > 0 && (!b_gate || !w_up || !s_up || !b_up)) return QMV_EINVAL;
+    const size_t eb = elem_bytes(dtype);
+    if (K > 0 && (!aligned(w_up, 4) || !aligned(s_gate, eb) || !aligned(b_gate, eb) || !aligned(s_up, eb) ||
+                  !aligned(b_up, eb)))
+        return QMV_EALIGN;
+    if (route_weight && !aligned(route_weight, 4)) return QMV_EALIGN;
+    if ((long long)N * 2 > 0x7FFFFFFFLL) return QMV_EINVAL;
+    return run_pair(x, w_gate, s_gate, b_gate, w_up, s_up, b_up, route_weight, mid, M, N, K, bits, group_size,
+                    dtype, clamp, stream);
 }
 
 int qmv_qvm_affine(const void* x, const void* w_packed, const void* scales, const void* biases, void* y,

@@ -87,6 +87,14 @@ struct Params {
     // Only the CUDA-core row-tiled and the few-rows kernels read it.
     const int* ids;
     int n_experts;
+    // Fused gate + up with SwiGLU (pair kernels only): w / scales / biases
+    // are the gate matrix, w2 / scales2 / biases2 the up matrix; output row n
+    // is silu(clamp(gate_n)) * clamp(up_n) * route_w[m] (see swiglu_act).
+    const uint8_t* w2;
+    const void* scales2;
+    const void* biases2;
+    const float* route_w;   // [M] per x row, or null for 1
+    float act_clamp;        // clamp value; inactive at or below 1e-6
 };
 
 // ---------------------------------------------------------------- dtypes ---
@@ -308,8 +316,9 @@ __device__ __forceinline__ void stage_x(const Params& p, const char* Xb, float4*
 }
 
 // Per-unit scales of chunk c for R rows (affine: scale + bias of the unit's
-// group; MX: one block scale; NV: two block scales per unit).
-template <int FAM, class T, int R, int U>
+// group; MX: one block scale; NV: two block scales per unit).  PAIR: row r is
+// virtual row rowc[r] of the interleaved gate / up pair (odd rows: up).
+template <int FAM, class T, int R, int U, bool PAIR = false>
 __device__ __forceinline__ void load_scales(const Params& p, const int (&rowc)[R], int c, long long sb,
                                             float (&sc)[R][U][2], float (&bi)[R][U]) {
     constexpr int C = 32 * U;
@@ -320,11 +329,18 @@ __device__ __forceinline__ void load_scales(const Params& p, const int (&rowc)[R
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const long long k0 = (long long)c * C + u * 32;
-            const long long rb = (long long)rowc[r] * KG;
+            long long row = rowc[r];
+            const void* sp = p.scales;
+            const void* bp = p.biases;
+            if constexpr (PAIR) {
+                if (row & 1) { sp = p.scales2; bp = p.biases2; }
+                row >>= 1;
+            }
+            const long long rb = row * KG;
             if constexpr (FAM == FAM_AFFINE) {
                 const long long gi = sb + rb + k0 / G;
-                sc[r][u][0] = DT<T>::ld(p.scales, gi);
-                bi[r][u] = DT<T>::ld(p.biases, gi);
+                sc[r][u][0] = DT<T>::ld(sp, gi);
+                bi[r][u] = DT<T>::ld(bp, gi);
             } else if constexpr (FAM == FAM_NVFP4) {
                 const uint8_t* s8 = reinterpret_cast<const uint8_t*>(p.scales) + sb + rb + k0 / 16;
                 sc[r][u][0] = e4m3_value(__ldg(s8));
@@ -415,6 +431,18 @@ __device__ __forceinline__ void compute_chunk(const uint32_t (&wv)[R][B * U], co
     }
 }
 
+// SwiGLU of one output (DS4 moe.metal, the routed-expert activation): with a
+// clamp c above 1e-6 the gate is limited to <= c and up to [-c, c]; then
+// silu(g) * u = g / (1 + exp(-g)) * u, in fp32.  The caller multiplies by the
+// route weight.
+__device__ __forceinline__ float swiglu_act(float g, float u, float c) {
+    if (c > 1.0e-6f) {
+        g = fminf(g, c);
+        u = fminf(fmaxf(u, -c), c);
+    }
+    return __fdiv_rn(g, 1.0f + expf(-g)) * u;
+}
+
 template <int R, int MAXM>
 __device__ __forceinline__ void warp_allreduce(float (&acc)[R][MAXM]) {
 #pragma unroll
@@ -434,8 +462,14 @@ __device__ __forceinline__ void warp_allreduce(float (&acc)[R][MAXM]) {
 //   sx : [MAXM][tile_iters][U][KT]            affine: sum(x) per unit
 //   red: [wk][wr*R*MAXM]                       cross-warp partials
 // KT = 32*wk.  Chunk c of the tile belongs to k-thread c % KT, iteration c / KT.
-template <int FAM, int BITS, class T, int MAXM, int R, bool WIDE>
+//
+// PAIR (affine only, R even): the fused gate + up projection with SwiGLU.
+// The rows are the 2N virtual rows of the interleaved pair (virtual row 2n =
+// gate row n, 2n + 1 = up row n), so each warp holds both sums of its R / 2
+// outputs and writes y[m, n] = swiglu_act(gate, up) * route_w[m].
+template <int FAM, int BITS, class T, int MAXM, int R, bool WIDE, bool PAIR = false>
 __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
+    static_assert(!PAIR || (FAM == FAM_AFFINE && R % 2 == 0), "pair rows come in twos");
     using F = Fmt<FAM, BITS>;
     constexpr int B = F::kBits;
     constexpr int U = WIDE ? F::kWideUnits : 1;
@@ -479,9 +513,10 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
     const char* Xb = reinterpret_cast<const char*>(p.x) + bz * p.x_bs * (long long)sizeof(T);
     const long long sb = be * p.s_bs;
 
+    const int NV = PAIR ? 2 * p.N : p.N;           // rows of the (virtual) matrix
     int rowc[R];
 #pragma unroll
-    for (int r = 0; r < R; ++r) rowc[r] = min(row0 + r, p.N - 1);
+    for (int r = 0; r < R; ++r) rowc[r] = min(row0 + r, NV - 1);
 
     float acc[R][MAXM];
 #pragma unroll
@@ -494,7 +529,13 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
     auto load_chunk = [&](int c) {
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            const uint8_t* src = W + (long long)rowc[r] * p.w_row + (long long)c * (C * B / 8);
+            const uint8_t* base = W;
+            long long prow = rowc[r];
+            if constexpr (PAIR) {
+                base = (prow & 1) ? p.w2 : W;
+                prow >>= 1;
+            }
+            const uint8_t* src = base + prow * p.w_row + (long long)c * (C * B / 8);
             if constexpr (WIDE) {
 #pragma unroll
                 for (int q = 0; q < CW / 4; ++q) {
@@ -506,7 +547,7 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
                 for (int q = 0; q < CW; ++q) wv[r][q] = __ldg(reinterpret_cast<const uint32_t*>(src) + q);
             }
         }
-        load_scales<FAM, T, R, U>(p, rowc, c, sb, sc, bi);
+        load_scales<FAM, T, R, U, PAIR>(p, rowc, c, sb, sc, bi);
     };
 
     const uint32_t kf32 = p.kf32;
@@ -547,6 +588,43 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
     if constexpr (FAM == FAM_NVFP4) gs = __ldg(p.gscale + be);
     T* Y = reinterpret_cast<T*>(p.y) + bz * p.y_bs;
     const int RM = R * MAXM;
+    if constexpr (PAIR) {
+        // output n = virtual rows (2n, 2n + 1); row0 is even
+        const float c = p.act_clamp;
+        if (p.wk == 1) {
+#pragma unroll
+            for (int j = 0; j < R / 2; ++j)
+#pragma unroll
+                for (int m = 0; m < MAXM; ++m)
+                    if (lane == j * MAXM + m && row0 + 2 * j < NV && m < p.M) {
+                        const float rw = p.route_w ? __ldg(p.route_w + m) : 1.0f;
+                        DT<T>::st(Y, (long long)m * p.N + (row0 >> 1) + j,
+                                  swiglu_act(acc[2 * j][m], acc[2 * j + 1][m], c) * rw);
+                    }
+        } else {
+            if (lane == 0) {
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+#pragma unroll
+                    for (int m = 0; m < MAXM; ++m) red[(wkid * p.wr + wrid) * RM + r * MAXM + m] = acc[r][m];
+            }
+            __syncthreads();
+            const int tot = p.wr * RM;
+            const int outs = p.wr * (R / 2) * MAXM;
+            for (int t = threadIdx.x; t < outs; t += blockDim.x) {
+                const int wr_ = t / ((R / 2) * MAXM), jm = t % ((R / 2) * MAXM), j = jm / MAXM, m = jm % MAXM;
+                const int ig = wr_ * RM + (2 * j) * MAXM + m, iu = ig + MAXM;
+                float g = 0.f, u = 0.f;
+                for (int k = 0; k < p.wk; ++k) { g += red[k * tot + ig]; u += red[k * tot + iu]; }
+                const int row = (blockIdx.x * p.wr + wr_) * R + 2 * j;
+                if (row < NV && m < p.M) {
+                    const float rw = p.route_w ? __ldg(p.route_w + m) : 1.0f;
+                    DT<T>::st(Y, (long long)m * p.N + (row >> 1), swiglu_act(g, u, c) * rw);
+                }
+            }
+        }
+        return;
+    }
     if (p.wk == 1) {
 #pragma unroll
         for (int r = 0; r < R; ++r)

@@ -1,0 +1,13 @@
+// qmv_inst_pair_b8.cu -- fused gate + up SwiGLU kernels, affine 8-bit (all
+// dtypes and pair launch shapes).
+#include "qmv_launch.cuh"
+
+namespace qmv {
+
+cudaError_t launch_affine_pair_b8(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L) {
+#define BITS_ 8
+    QMV_PAIR_DISPATCH_DTYPE()
+#undef BITS_
+}
+
+}  // namespace qmv

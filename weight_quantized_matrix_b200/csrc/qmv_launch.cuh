@@ -95,6 +95,16 @@ cudaError_t launch_dequant(int fam, int bits, int dtype, const uint8_t* w, const
                            const void* biases, const float* gscale, float* out, int N, int K, int G,
                            long long w_row, cudaStream_t s);
 
+// Fused gate + up with SwiGLU (qmv_kernel<..., PAIR = true>, affine): R in
+// {2, 4} wide (4 only for maxm <= 2), R = 2 narrow.  Returns
+// cudaErrorInvalidValue for a shape that is not instantiated.
+cudaError_t launch_affine_pair(int bits, int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+inline bool pair_shape_instantiated(int maxm, int R, bool wide) {
+    if (!wide) return R == 2 && (maxm == 1 || maxm == 2 || maxm == 4 || maxm == 8);
+    if (maxm == 1 || maxm == 2) return R == 2 || R == 4;
+    return (maxm == 4 || maxm == 8) && R == 2;
+}
+
 // Which (maxm, R, wide) shapes exist.
 inline bool shape_instantiated(int maxm, int R, bool wide) {
     if (!wide) return R == 1 && (maxm == 1 || maxm == 2 || maxm == 4 || maxm == 8);
@@ -119,6 +129,25 @@ inline bool shape_instantiated(int maxm, int R, bool wide) {
     QMV_SHAPE(T_, 8, 1, true) QMV_SHAPE(T_, 8, 2, true)                                      \
     QMV_SHAPE(T_, 1, 1, false) QMV_SHAPE(T_, 2, 1, false) QMV_SHAPE(T_, 4, 1, false)         \
     QMV_SHAPE(T_, 8, 1, false)
+#define QMV_PAIR_SHAPE(T_, MAXM_, R_, WIDE_)                                                 \
+    if (maxm == MAXM_ && R == R_ && wide == WIDE_) {                                         \
+        static std::atomic<unsigned> cfg_{0};                                                \
+        return launch_kernel(qmv_kernel<FAM_AFFINE, BITS_, T_, MAXM_, R_, WIDE_, true>, cfg_, L, p); \
+    }
+#define QMV_PAIR_SHAPES(T_)                                                                  \
+    QMV_PAIR_SHAPE(T_, 1, 2, true) QMV_PAIR_SHAPE(T_, 1, 4, true)                            \
+    QMV_PAIR_SHAPE(T_, 2, 2, true) QMV_PAIR_SHAPE(T_, 2, 4, true)                            \
+    QMV_PAIR_SHAPE(T_, 4, 2, true) QMV_PAIR_SHAPE(T_, 8, 2, true)                            \
+    QMV_PAIR_SHAPE(T_, 1, 2, false) QMV_PAIR_SHAPE(T_, 2, 2, false)                          \
+    QMV_PAIR_SHAPE(T_, 4, 2, false) QMV_PAIR_SHAPE(T_, 8, 2, false)
+#define QMV_PAIR_DISPATCH_DTYPE()                                                            \
+    switch (dtype) {                                                                         \
+        case 0: { QMV_PAIR_SHAPES(float) break; }                                            \
+        case 1: { QMV_PAIR_SHAPES(__half) break; }                                           \
+        case 2: { QMV_PAIR_SHAPES(__nv_bfloat16) break; }                                    \
+        default: break;                                                                      \
+    }                                                                                        \
+    return cudaErrorInvalidValue;
 #define QMV_TC_SHAPE(T_, NPASS_)                                                             \
     if (npass == NPASS_) {                                                                   \
         static std::atomic<unsigned> cfg_{0};                                                \

@@ -9,6 +9,8 @@
 #define PY_SSIZE_T_CLEAN
 #include <Python.h>
 
+#include <limits.h>
+
 #include "qmv.h"
 
 static int as_ptr(PyObject* o, void** out) {
@@ -17,9 +19,15 @@ static int as_ptr(PyObject* o, void** out) {
     return (*out == NULL && PyErr_Occurred()) ? -1 : 0;
 }
 
+/* A Python int that fits a C int; anything larger raises OverflowError
+ * instead of being narrowed. */
 static int as_int(PyObject* o, int* out) {
     long v = PyLong_AsLong(o);
     if (v == -1 && PyErr_Occurred()) return -1;
+    if (v < INT_MIN || v > INT_MAX) {
+        PyErr_SetString(PyExc_OverflowError, "argument does not fit a C int");
+        return -1;
+    }
     *out = (int)v;
     return 0;
 }
