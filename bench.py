@@ -573,6 +573,131 @@ WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe, "quantize": Quant
              "quantize_fp": QuantizeFp}
 
 
+# ------------------------------------------- per format / bits / shape --
+DT_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
+FP_MODES = ("mxfp4", "nvfp4", "mxfp8")
+
+
+def fp_bytes(M, N, K, mode, batch=1, eb=2):
+    """Algorithmic bytes of one FP call: codes + block scales (+ the NVFP4
+    global) + x + y, times the batch."""
+    bits, blk = synth.FP_BITS[mode], synth.FP_BLOCK[mode]
+    per = N * K * bits // 8 + N * (K // blk) + (4 if mode == "nvfp4" else 0) + M * K * eb + M * N * eb
+    return per * batch
+
+
+def _copies(torch, dev, arrays, n):
+    """n device copies of the same host arrays (distinct addresses, so each
+    call of a rotation reads its weights from HBM after an L2 flush)."""
+    base = [torch.from_numpy(np.ascontiguousarray(a).view(np.uint8).reshape(-1)).to(dev) for a in arrays]
+    return [tuple(b) for b in [base]] + [tuple(b.clone() for b in base) for _ in range(n - 1)]
+
+
+def _rotation(wbytes, cap=64, least=1):
+    return int(max(least, min(cap, np.ceil(2 * L2_BYTES / max(wbytes, 1)))))
+
+
+def shape_lines(q, torch, dev, stream, flush, flush_rd, peak, sets=None):
+    """Throughput per format, bits and shape (the metric's breakdown), each
+    line from ONE CUDA graph of R calls back to back on R weight copies that
+    together exceed twice the L2 (or, for the chained FP shapes, 64 dependent
+    calls), replayed after an L2 flush between a pair of events on the
+    launching stream; us_per_call = median replay time / R.  Sets: c1 (the
+    small 4-bit config), probe (16384^2 4-bit, M = 1 and 8), layer (the 7B
+    projections, M = 1 and 8), fp_chain (MXFP4 / NVFP4 / MXFP8 chains of the
+    pages' shapes), fp_probe (16384^2 in each FP format, M = 1) and sweep
+    (2/3/5/6-bit x group 32/64/128 x f32/f16/bf16 x M = 1, 4 at N = K = 4096)."""
+    lines = []
+    sets = sets or ("c1", "probe", "layer", "fp_chain", "fp_probe", "sweep")
+
+    def timed(tag, label, R, launch, nbytes, plan, reps=5):
+        for r in range(R):                          # eager warm-up (kernel attributes)
+            launch(r)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for r in range(R):
+                launch(r)
+        g.replay(); g.replay()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for i in range(reps):
+            flush.fill_(i & 0xFF)
+            flush_rd.max()
+            ev[i][0].record(stream)
+            g.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        ms = float(np.median([a.elapsed_time(b) for a, b in ev]))
+        us = ms * 1e3 / R
+        gbs = nbytes / (us * 1e-6) / 1e9
+        lines.append({"set": tag, "shape": label, "us_per_call": round(us, 3), "GB_s": round(gbs, 1),
+                      "frac_of_hbm": round(gbs / peak, 4), "calls_per_graph": R, "plan": plan})
+        del g
+
+    def affine(tag, label, M, N, K, bits, G, dtype, least=1, cap=64):
+        c = synth.affine_case(M, N, K, bits, G, dtype, seed=7000 + N + K + 13 * bits + G + M)
+        wb = affine_bytes(M, N, K, bits, G, DT_BYTES[dtype]) - M * K * DT_BYTES[dtype] - M * N * DT_BYTES[dtype]
+        R = _rotation(wb, cap, least)
+        ws = _copies(torch, dev, (c["w"], c["scales"], c["biases"]), R)
+        x = torch.from_numpy(c["x"][0].view(np.uint8).reshape(-1).copy()).to(dev)
+        y = torch.empty(M * N * DT_BYTES[dtype], dtype=torch.uint8, device=dev)
+
+        def launch(r):
+            w, sc, bi = ws[r]
+            q.qmv_affine(x, w, sc, bi, y, M, N, K, bits, G, dtype)
+        timed(tag, label, R, launch, affine_bytes(M, N, K, bits, G, DT_BYTES[dtype]),
+              q.qmv_describe_plan("affine", M, N, K, bits, G, dtype))
+
+    with torch.cuda.stream(stream):
+        if "c1" in sets:
+            affine("c1", "affine b4 g64 bf16 M=1 N=256 K=512", 1, 256, 512, 4, 64, "bf16")
+        if "probe" in sets:
+            for M in (1, 8):
+                affine("probe", f"affine b4 g64 bf16 M={M} N=K=16384", M, 16384, 16384, 4, 64, "bf16", least=3)
+        if "layer" in sets:
+            for M in (1, 8):
+                for name, N, K in LAYER:
+                    affine("layer", f"{name} {N}x{K} b4 g64 bf16 M={M}", M, N, K, 4, 64, "bf16", least=3)
+        if "fp_chain" in sets:
+            for mode in FP_MODES:
+                for (N, K, B) in ((5, 1024, 2), (12, 4096, 1)):
+                    c = synth.fp_case(1, N, K, mode, "bf16", seed=7100 + N + K, batch=B)
+                    ws = _copies(torch, dev, (c["w"], c["scales"]), CHAIN_CALLS)
+                    gs = (torch.tensor(np.full(B, c["global"], dtype=np.float32), device=dev)
+                          if mode == "nvfp4" else None)
+                    bufs = [torch.zeros(B * K, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+                    x0 = torch.from_numpy(c["x"].view(np.int16).reshape(-1).copy()).view(torch.bfloat16).to(dev)
+
+                    def launch(t, ws=ws, gs=gs, bufs=bufs, x0=x0, N=N, K=K, B=B, mode=mode):
+                        xin = x0 if t == 0 else bufs[(t - 1) % 2]
+                        w, sc = ws[t]
+                        q.qmv_fp_batched(xin, w, sc, gs, bufs[t % 2], 1, N, K, mode, "bf16", B, True)
+                    timed("fp_chain", f"{mode} chain N={N} K={K} batch={B}", CHAIN_CALLS, launch,
+                          fp_bytes(1, N, K, mode, B), q.qmv_describe_plan(mode, 1, N, K, 0, 0, "bf16"))
+        if "fp_probe" in sets:
+            for mode in FP_MODES:
+                N = K = 16384
+                c = synth.fp_case(1, N, K, mode, "bf16", seed=7200)
+                R = 3
+                ws = _copies(torch, dev, (c["w"], c["scales"]), R)
+                gs = torch.tensor([c["global"]], dtype=torch.float32, device=dev) if mode == "nvfp4" else None
+                x = torch.from_numpy(c["x"][0].view(np.int16).reshape(-1).copy()).view(torch.bfloat16).to(dev)
+                y = torch.empty(N, dtype=torch.bfloat16, device=dev)
+
+                def launch(r, ws=ws, gs=gs, x=x, y=y, mode=mode):
+                    w, sc = ws[r]
+                    q.qmv_fp(x, w, sc, gs, y, 1, 16384, 16384, mode, "bf16")
+                timed("fp_probe", f"{mode} M=1 N=K=16384", R, launch, fp_bytes(1, N, K, mode),
+                      q.qmv_describe_plan(mode, 1, N, K, 0, 0, "bf16"))
+        if "sweep" in sets:
+            for bits in (2, 3, 5, 6):
+                for G in (32, 64, 128):
+                    for dtype in ("f32", "f16", "bf16"):
+                        for M in (1, 4):
+                            affine("sweep", f"affine b{bits} g{G} {dtype} M={M} N=K=4096", M, 4096, 4096, bits, G,
+                                   dtype)
+    return lines
+
+
 # ---------------------------------------------------------------- our arm --
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -691,7 +816,8 @@ def run_ours(args, rank, world, local_rank):
         plan = wl.group_plan(s)
         kern = " ".join(w for w in plan.split() if w.split("=")[0] in ("path", "chunk", "maxm", "rows_per_warp"))
         gbs = b / (ms * 1e-3) / 1e9
-        shapes.append({"shape": label, "us_per_call": round(ms * 1e3 / n, 3), "GB_s": round(gbs, 1),
+        shapes.append({"set": args.workload, "shape": label, "us_per_call": round(ms * 1e3 / n, 3),
+                       "GB_s": round(gbs, 1),
                        "frac_of_hbm": round(gbs / peak, 4), "plan": plan})
         k = by_kernel.setdefault(kern, {"ms": 0.0, "launches": 0, "bytes": 0})
         k["ms"] += ms; k["launches"] += n; k["bytes"] += b
@@ -714,6 +840,9 @@ def run_ours(args, rank, world, local_rank):
                      "avg_launch_us": round(dom["ms"] * 1e3 / max(1, dom["launches"]), 3)},
         "clocks": clocks, "shapes": shapes, "wall_s_timed": round(wall, 3),
     }
+    if args.workload == "chain8" and not args.no_shapes:
+        # the metric's breakdown per format / bits / shape; not part of `value`
+        out["shapes"] += shape_lines(q, torch, dev, stream, flush, flush_rd, peak)
     if rank == 0:
         out["cpu_baseline"] = cpu_baseline(args.workload)
         print(json.dumps(out), flush=True)
@@ -866,6 +995,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="chain8")
+    ap.add_argument("--no-shapes", action="store_true",
+                    help="chain8 only: skip the per format / bits / shape lines")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -17,7 +17,9 @@
 // would not fit are rejected before any launch.  In host code the array's
 // name is only a host-side stand-in, so its device address is looked up with
 // cudaGetSymbolAddress, once per device, with that device current, on the
-// first call made on it.
+// first call made on it.  The address is cached for the life of the process;
+// a cudaDeviceReset() reloads the module and may move the array, so calls
+// after a reset of that device are not supported.
 #include <mutex>
 
 #include <cuda_runtime.h>
