@@ -16,6 +16,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include <cudaTypedefs.h>
@@ -23,6 +24,7 @@
 #include "../../include/qmv.h"
 #include "qmv_launch.cuh"
 #include "qmv_tc_plan.cuh"
+#include "qmv_umma.cuh"
 
 namespace {
 
@@ -94,6 +96,8 @@ struct Plan {
     int sps = 0, pitch = 0, spb = 1, sring = 0, soff = 0, boff = 0, sbw = 0;
     size_t smem;
     dim3 grid, block;
+    qmv::UmmaParams um{};    // tc == 5: the tensor-memory kernel
+    int mld = 0;
 };
 
 // Rows per warp on the wide path (x reuse vs registers); measured on B200:
@@ -390,9 +394,110 @@ bool tcf_shape(int N, int K, int bits, int G, bool w16, bool s16, TcbShape* ts) 
     return ts->smem <= (size_t)qmv::kMaxSmem;
 }
 
+// ---- tensor-memory (tcgen05) launch shape (qmv_umma.cuh) ---------------------
+// Geometry per code width (mirrors qmv::UmGeom).
+struct UmGeomH { int uc, npu, slot_cols, stage_codes, stage_bytes; };
+template <int B> UmGeomH um_geom_t() {
+    using G = qmv::UmGeom<B>;
+    return {G::UC, G::NPU, G::SLOT_COLS, G::STAGE_CODES, G::STAGE_BYTES};
+}
+bool um_geom(int bits, UmGeomH* g) {
+    switch (bits) {
+        case 2: *g = um_geom_t<2>(); return true;
+        case 3: *g = um_geom_t<3>(); return true;
+        case 4: *g = um_geom_t<4>(); return true;
+        case 5: *g = um_geom_t<5>(); return true;
+        case 6: *g = um_geom_t<6>(); return true;
+        case 8: *g = um_geom_t<8>(); return true;
+        default: return false;
+    }
+}
+long long gcd_ll(long long a, long long b) { while (b) { long long t = a % b; a = b; b = t; } return a; }
+
+// Clusters of S CTAs (one per SM) that fit at once, per device (queried once).
+int um_clusters(int bits, const qmv::UmmaParams& u, size_t smem) {
+    static int cache[64][9] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) { cudaGetLastError(); return 1; }
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    int& c = cache[dev][u.S];
+    if (!c) {
+        int n = 0;
+        if (qmv::umma_max_clusters(bits, u, smem, &n) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = device_sms() / u.S;
+        }
+        c = n < 1 ? 1 : n;
+    }
+    return c;
+}
+
+// Affine, bf16 x, one weight matrix, M <= 64.  Rows: 128-row tiles over a
+// persistent grid of clusters; K split over the S CTAs of a cluster when the
+// tiles alone leave SMs idle, or when x of the whole K would not fit.
+bool umma_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s16, bool x16, int batch, Plan* pl) {
+    UmGeomH g;
+    if (!um_geom(bits, &g)) return false;
+    if (dtype != QMV_BF16 || batch != 1 || M < 1 || M > 64 || N < 1 || K < 64) return false;
+    if (!w16 || !s16 || !x16) return false;
+    if (G < g.uc || K % 64 != 0 || K % G != 0 || (K / G) % 8 != 0) return false;
+    if (((long long)K * bits / 8) % 16 != 0) return false;
+    const int BLK = G > 64 ? G : 64, NBG = BLK / G, NBS = BLK / 64;
+    int mld = 1;
+    while (mld < M) mld *= 2;
+    const int ncol = mld < 16 ? 16 : mld;                          // MMA N >= the accumulator read width
+    const int blk_cols = NBS * g.slot_cols + NBG * ncol;
+    int DB = 2 * (512 / (2 * blk_cols));
+    if (DB > 16) DB = 16;
+    if (DB < 2) return false;
+    const long long QC = (long long)g.stage_codes / gcd_ll(g.stage_codes, 8LL * G) * (8LL * G);
+    const int nq = (int)((K + QC - 1) / QC);
+    const int tiles = (N + 127) / 128;
+    const int ksg = 2 * g.npu * G / g.uc;                       // k-slots per group
+    const int SSL = G == 32 ? 8 : 4;                             // scale slots: 8 groups each
+    auto smem_of = [&](int S, int WST, unsigned* smem_b) {
+        const long long rng = std::min<long long>((long long)((nq + S - 1) / S) * QC, K);
+        const long long ngr = rng / G;
+        *smem_b = (unsigned)(ngr * ksg * M * 2 + 1024);
+        return (size_t)2048 + (size_t)WST * g.stage_bytes + (size_t)SSL * 4096 + *smem_b + (size_t)(M * ngr + 3) / 4 * 16 +
+               (size_t)DB * NBG * 128 * 8 + (size_t)128 * mld * 4;
+    };
+    const int smax = std::min(8, nq);
+    int S = 0, WST = 0;
+    unsigned sb = 0;
+    for (int s_ = 1; s_ <= smax && !S; ++s_)
+        for (int w = 4; w >= 2; --w)
+            if (smem_of(s_, w, &sb) <= (size_t)qmv::kMaxSmem) { S = s_; WST = w; break; }
+    if (!S) return false;
+    const int sms = device_sms();
+    if (tiles < sms) {
+        int so = sms / tiles;
+        if (so > smax) so = smax;
+        if (so > S) S = so;
+    }
+    if (g_forced.wk > 0 && g_forced.wk <= smax) S = g_forced.wk;       // test knob: the K split
+    WST = 0;
+    for (int w = 4; w >= 2; --w)
+        if (smem_of(S, w, &sb) <= (size_t)qmv::kMaxSmem) { WST = w; break; }
+    if (!WST) return false;
+    size_t smem = smem_of(S, WST, &sb);
+    if (smem < 120 * 1024) smem = 120 * 1024;                      // one CTA per SM
+    qmv::UmmaParams& u = pl->um;
+    u.S = S; u.DB = DB; u.WST = WST; u.SSL = SSL; u.nq = nq; u.QC = (int)QC; u.ncols = 512; u.ncol_mma = ncol;
+    u.tiles = tiles; u.smem_b = sb;
+    u.ngr_max = (int)(std::min<long long>((long long)((nq + S - 1) / S) * QC, K) / G);
+    int ncl = um_clusters(bits, u, smem);
+    if (ncl > tiles) ncl = tiles;
+    pl->maxm = M; pl->R = 1; pl->wide = 1; pl->tc = 5; pl->npass = 0; pl->wk = S; pl->wr = 1;
+    pl->tile_iters = DB; pl->C = BLK; pl->smem = smem; pl->mld = mld;
+    pl->grid = dim3((unsigned)S, (unsigned)ncl, 1);
+    pl->block = dim3(320, 1, 1);
+    return true;
+}
+
 // Choose the launch shape.  Returns QMV_OK or an error (sizes too large).
 int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, bool w16, int batch, Plan* pl,
-              bool s16 = true, bool gather = false, bool pair = false) {
+              bool s16 = true, bool gather = false, bool pair = false, bool x16 = true) {
     // pair (fused gate + up): N counts the 2N virtual rows; only the
     // row-tiled CUDA-core kernel has the pair epilogue
     if (pair) gather = true;
@@ -420,6 +525,11 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
         pl->block = dim3((unsigned)thr, 1, 1);
         return QMV_OK;
     }
+
+    // ---- tensor-memory kernel (tcgen05): forced only, until measured ---------
+    if (!gather && aff && K > 0 && g_forced.path == 7 &&
+        umma_shape(M, N, K, bits, G_of_plan, dtype, w16, s16, x16, batch, pl))
+        return QMV_OK;
 
     // ---- one bf16 x row: CUDA cores with the weight ring ----------------------
     // (measured on B200: the fastest path for one bf16 x row from about 10 MB
@@ -601,6 +711,20 @@ bool encode_rows_map(CUtensorMap* m, const void* base, long long row_bytes, int 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// As encode_rows_map with the 128-byte swizzle (box {16, rows, 1}: 128 bytes
+// a row), for the tensor-memory kernel's conflict-free row reads.
+bool encode_rows_map_sw128(CUtensorMap* m, const void* base, long long row_bytes, int N, int batch, int rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)(row_bytes / 8), (cuuint64_t)N, (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)row_bytes * (cuuint64_t)N};
+    const cuuint32_t box[3] = {16, (cuuint32_t)rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // [batch][N][K/G] scales (or biases) as a 3-D tensor map with box
 // {box0 groups, rows, 1}; out-of-range elements read as zero.
 bool encode_scale_map(CUtensorMap* m, const void* base, int dtype, long long KG, int N, int batch, int box0,
@@ -627,9 +751,19 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     Plan pl;
     const bool w16 = aligned(w, 16);
     const bool s16 = fam == qmv::FAM_AFFINE && aligned(scales, 16) && aligned(biases, 16);
-    int st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, s16, ids != nullptr);
+    const bool x16 = aligned(x, 16) && ((size_t)K * elem_bytes(dtype)) % 16 == 0;
+    int st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, s16, ids != nullptr, false, x16);
     if (st != QMV_OK) return st;
     qmv::Params p;
+    if (pl.tc == 5) {
+        // tensor-memory kernel: swizzled row boxes, scale / bias boxes of 8 groups
+        if (!encode_rows_map_sw128(&p.wmap, w, row_bytes, N, batch, 128) ||
+            !encode_scale_map(&p.smap, scales, dtype, K / G, N, batch, 8, 128) ||
+            !encode_scale_map(&p.bmap, biases, dtype, K / G, N, batch, 8, 128)) {
+            cudaGetLastError();
+            return QMV_ECUDA;
+        }
+    }
     const bool ring = pl.tc == 2 || pl.tc == 4;        // the weight-ring kernels
     if (ring && pl.sring) {
         const int box0 = pl.sbw / elem_bytes(dtype), rows = 16 * pl.wr;
@@ -675,6 +809,11 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
         p.fault = fault_word();
         if (!p.fault) return QMV_ECUDA;
         return finish(qmv::launch_tcf_affine(bits, pl.wk * pl.wr, p, L));
+    }
+    if (pl.tc == 5) {
+        p.fault = fault_word();
+        if (!p.fault) return QMV_ECUDA;
+        return finish(qmv::launch_umma_affine(bits, pl.mld, p, pl.um, L));
     }
     if (pl.tc == 3) return finish(qmv::launch_direct(fam, bits, dtype, pl.maxm, pl.wide != 0, p, L));
     if (pl.tc) return finish(qmv::launch_tc_affine(bits, dtype, pl.npass, p, L));
@@ -976,7 +1115,7 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
     snprintf(buf, (size_t)buflen,
              "path=%s chunk=%d maxm=%d rows_per_warp=%d warps_k=%d warps_rows=%d tile_iters=%d "
              "grid=%u block=%u smem=%zu stage_sb=%d batch_sb=%d scale_ring=%d",
-             pl.tc == 4 ? "tcf" : pl.tc == 3 ? "direct" : pl.tc == 2 ? "tcb" : pl.tc ? "tc" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr,
+             pl.tc == 5 ? "umma" : pl.tc == 4 ? "tcf" : pl.tc == 3 ? "direct" : pl.tc == 2 ? "tcb" : pl.tc ? "tc" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr,
              pl.tile_iters, pl.grid.x, pl.block.x, pl.smem, pl.sps, pl.spb, pl.sring);
     return QMV_OK;
 }

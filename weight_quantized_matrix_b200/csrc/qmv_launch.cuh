@@ -105,6 +105,13 @@ inline bool pair_shape_instantiated(int maxm, int R, bool wide) {
     return (maxm == 4 || maxm == 8) && R == 2;
 }
 
+// Tensor-memory (tcgen05) kernels (qmv_umma.cuh), bf16 x: mld = the power of
+// two >= M (1..64); the grid is (S, clusters), cluster (S, 1, 1).
+struct UmmaParams;
+cudaError_t launch_umma_affine(int bits, int mld, const Params& p, const UmmaParams& u, const Launch& L);
+// Clusters of the tensor-memory kernel that fit on the device at once.
+cudaError_t umma_max_clusters(int bits, const UmmaParams& u, size_t smem, int* out);
+
 // Which (maxm, R, wide) shapes exist.
 inline bool shape_instantiated(int maxm, int R, bool wide) {
     if (!wide) return R == 1 && (maxm == 1 || maxm == 2 || maxm == 4 || maxm == 8);
