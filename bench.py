@@ -415,7 +415,7 @@ class Qmm(Layer):
         return 1
 
     def group_plan(self, s):
-        return "path=qmm " + self.q.qmv_describe_plan("affine", 8, s["N"], s["K"], 4, 64, "bf16")
+        return self.q.qmv_describe_plan("affine", s["M"], s["N"], s["K"], 4, 64, "bf16")
 
     def config(self):
         return {"workload": self.name, "bits": 4, "group": 64, "dtype": "bf16", "M": self.M,

@@ -204,10 +204,17 @@ int qmv_affine_swiglu(const void* x, const void* w_gate, const void* s_gate, con
  * qmv_qmm_affine -- small-M quantized matmul, y = x * dequant(W)^T for up to
  * QMV_QMM_MAX_M x rows (the qmm family of MLX quantized_nax.h and of the
  * wh-iron audit, M-batched prefill).  Arguments and layouts as qmv_affine,
- * with 1 <= M <= 64 (0 allowed as a no-op).  The rows run as chunks of
- * QMV_MAX_M through the qmv_affine kernels, back to back on `stream` (a weight
- * matrix that fits in L2 is read from HBM once); every argument is checked
- * before the first launch.  Same accumulation and rounding as qmv_affine.
+ * with 1 <= M <= 64 (0 allowed as a no-op).  M <= 8 is qmv_affine.  More
+ * rows: for N <= 5120 with bf16 x, 16-byte aligned x, weights, scales and
+ * biases, K a multiple of 64 and K / group_size a multiple of 8, ONE launch of
+ * the tensor-memory kernel (tcgen05: each weight decoded once for all rows,
+ * the rows are the MMA's N, K split over a thread-block cluster) when x fits
+ * its shared memory; otherwise chunks of 32 or 16 rows through the
+ * tensor-core ring kernel where it takes that many (x rows times groups of a
+ * 128-code super-block at most 32, N > 64, 16-byte aligned weights), else
+ * chunks of QMV_MAX_M, back to back on `stream` (a weight matrix that fits in
+ * L2 is read from HBM once).  Every argument is checked before the first
+ * launch.  Same accumulation and rounding as qmv_affine.
  */
 #define QMV_QMM_MAX_M 64
 int qmv_qmm_affine(const void* x, const void* w_packed, const void* scales, const void* biases,
@@ -329,8 +336,10 @@ int qmv_last_cuda_error(void);
 /*
  * qmv_describe_plan -- the launch the picker would choose for these sizes,
  * written as text into buf (at most buflen bytes, NUL-terminated).  `family`
- * is 0 for affine (bits, group_size used) or 1 + qmv_fp_mode.  Host-only; no
- * CUDA call except a cached device-property query.  Returns QMV_OK or an
+ * is 0 for affine (bits, group_size used) or 1 + qmv_fp_mode.  M up to 8 is
+ * qmv's plan; 9..64 (affine) is qmv_qmm_affine's ("path=umma ...", or
+ * "path=chunked<rows> chunks=<n>" and the plan of one chunk).  Host-only; no CUDA call except
+ * cached device-property and occupancy queries.  Returns QMV_OK or an
  * argument error.
  */
 int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size, int dtype,

@@ -1,7 +1,8 @@
-"""GPU parity of the small-M qmm (qmv_qmm_affine: up to 64 x rows, run as
-8-row chunks through the qmv kernels) against the oracle, element by element,
-within the qmv output tolerance.  Row counts cover one chunk plus a ragged
-remainder, several full chunks and the maximum of 64."""
+"""GPU parity of the small-M qmm (qmv_qmm_affine: up to 64 x rows, as chunks of
+32, 16 or 8 rows through the qmv kernels; forced, one launch of the
+tensor-memory kernel) against the oracle, element by element, within the qmv
+output tolerance.  Row counts cover one chunk plus a ragged remainder, several
+full chunks and the maximum of 64."""
 from __future__ import annotations
 
 import pytest
@@ -48,6 +49,44 @@ def test_qmm_layer_shape(q):
     ref, ad = oracle.qmv_affine(c["x"][0], c["w"][0], c["scales"][0], c["biases"][0], M, N, K, 4, 64, "bf16",
                                 rows=rows, threads=THREADS)
     assert_close(y[:, rows], ref[:, rows], ad[:, rows], "bf16", what="qmm 4096x14336 M=32")
+
+
+@pytest.mark.parametrize("M", [9, 16, 33, 64])
+@pytest.mark.parametrize("shape", [(28672, 4096), (4096, 14336)])
+@pytest.mark.parametrize("forced", [-1, 7])
+def test_qmm_layer_shapes(q, M, shape, forced):
+    """qmm beyond 8 rows on the 7B gate+up and down shapes (4-bit g64 bf16),
+    sampled rows: by default chunks of up to 32 rows through the tensor-core
+    ring kernel for the tall gate+up, one launch of the tensor-memory kernel
+    for the down projection (few row tiles) and whenever forced (path 7),
+    where x fits its shared memory."""
+    N, K = shape
+    q.qmv_force_config(forced, -1, -1, -1)
+    try:
+        plan = q.qmv_describe_plan("affine", M, N, K, 4, 64, "bf16")
+        fits = M * K <= 33 * 14336          # 64 x rows over K = 14336: x needs more than 16 CTAs
+        if forced == 7 or N <= 5120:
+            assert plan.startswith("path=umma") == fits, plan
+        else:
+            assert plan.startswith("path=chunked16 ") and "path=tcb" in plan, plan
+        c = synth.affine_case(M, N, K, 4, 64, "bf16", seed=M * 100 + K)
+        y = _run(q, c, M, N, K)
+    finally:
+        q.qmv_force_config()
+    rows = list(range(0, N, N // 40)) + [N - 1]
+    ref, ad = oracle.qmv_affine(c["x"][0], c["w"][0], c["scales"][0], c["biases"][0], M, N, K, 4, 64, "bf16",
+                                rows=rows, threads=THREADS)
+    assert_close(y[:, rows], ref[:, rows], ad[:, rows], "bf16", what=f"qmm {plan.split()[0]} {N}x{K} M={M}")
+
+
+def test_qmm_plans(q):
+    """Tall matrices: 32 rows a chunk where a super-block holds one group
+    (4-bit g128), 16 where it holds two (g64); f16 likewise through the ring
+    kernel.  Few row tiles, bf16: one tensor-memory launch."""
+    assert q.qmv_describe_plan("affine", 64, 8000, 1024, 4, 128, "bf16").startswith("path=chunked32 chunks=2 ")
+    assert q.qmv_describe_plan("affine", 33, 8000, 1024, 4, 64, "bf16").startswith("path=chunked16 chunks=3 ")
+    assert q.qmv_describe_plan("affine", 12, 8000, 1024, 4, 64, "f16").startswith("path=chunked16 chunks=1 ")
+    assert q.qmv_describe_plan("affine", 33, 1000, 1024, 4, 64, "bf16").startswith("path=umma ")
 
 
 def test_qmm_rejects_more_than_64_rows(q):

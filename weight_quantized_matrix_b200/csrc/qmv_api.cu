@@ -416,7 +416,7 @@ long long gcd_ll(long long a, long long b) { while (b) { long long t = a % b; a 
 
 // Clusters of S CTAs (one per SM) that fit at once, per device (queried once).
 int um_clusters(int bits, const qmv::UmmaParams& u, size_t smem) {
-    static int cache[64][9] = {};
+    static int cache[64][17] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) { cudaGetLastError(); return 1; }
     std::lock_guard<std::mutex> lk(g_dev_mu);
@@ -462,7 +462,7 @@ bool umma_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool 
         return (size_t)2048 + (size_t)WST * g.stage_bytes + (size_t)SSL * 4096 + *smem_b + (size_t)(M * ngr + 3) / 4 * 16 +
                (size_t)DB * NBG * 128 * 8 + (size_t)128 * mld * 4;
     };
-    const int smax = std::min(8, nq);
+    const int smax = std::min(16, nq);       // clusters beyond 8 are non-portable; B200 takes 16
     int S = 0, WST = 0;
     unsigned sb = 0;
     for (int s_ = 1; s_ <= smax && !S; ++s_)
@@ -497,7 +497,7 @@ bool umma_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool 
 
 // Choose the launch shape.  Returns QMV_OK or an error (sizes too large).
 int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, bool w16, int batch, Plan* pl,
-              bool s16 = true, bool gather = false, bool pair = false, bool x16 = true) {
+              bool s16 = true, bool gather = false, bool pair = false, bool x16 = true, bool qmm = false) {
     // pair (fused gate + up): N counts the 2N virtual rows; only the
     // row-tiled CUDA-core kernel has the pair epilogue
     if (pair) gather = true;
@@ -526,8 +526,14 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
         return QMV_OK;
     }
 
-    // ---- tensor-memory kernel (tcgen05): forced only, until measured ---------
-    if (!gather && aff && K > 0 && g_forced.path == 7 &&
+    // ---- tensor-memory kernel (tcgen05) ---------------------------------------
+    // Measured on B200: one tcgen05.mma kind::f16 (M = 128, K = 16) takes about
+    // 191 cycles whatever N is (16..256), so the tensor cores take in at most
+    // 128 * 16 / 191 = 10.7 weights per cycle per SM (about 1.6 TB/s of 4-bit
+    // weights): below the other kernels for M <= 8.  For x rows beyond 8 (qmm)
+    // it decodes every weight once where chunks decode it once per chunk; qmm
+    // takes it for matrices of few row tiles (qmm_prefers_umma).
+    if (!gather && aff && K > 0 && (g_forced.path == 7 || qmm) &&
         umma_shape(M, N, K, bits, G_of_plan, dtype, w16, s16, x16, batch, pl))
         return QMV_OK;
 
@@ -746,14 +752,16 @@ bool encode_scale_map(CUtensorMap* m, const void* base, int dtype, long long KG,
 
 int run(int fam, const void* x, const void* w, const void* scales, const void* biases,
         const float* gscale, void* y, int M, int N, int K, int bits, int G, int dtype, int batch,
-        int x_batched, void* stream, const int* ids = nullptr, int n_experts = 0) {
+        int x_batched, void* stream, const int* ids = nullptr, int n_experts = 0, bool qmm = false) {
     const long long row_bytes = (long long)K * (fam == qmv::FAM_AFFINE ? bits : (fam == qmv::FAM_MXFP8 ? 8 : 4)) / 8;
     Plan pl;
     const bool w16 = aligned(w, 16);
     const bool s16 = fam == qmv::FAM_AFFINE && aligned(scales, 16) && aligned(biases, 16);
     const bool x16 = aligned(x, 16) && ((size_t)K * elem_bytes(dtype)) % 16 == 0;
-    int st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, s16, ids != nullptr, false, x16);
+    int st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, s16, ids != nullptr, false, x16, qmm);
     if (st != QMV_OK) return st;
+    // M > 8 (qmm): only the tensor-memory kernel and the tensor-core ring take it
+    if (M > QMV_MAX_M && pl.tc != 5 && pl.tc != 2) return QMV_EUNSUPPORTED;
     qmv::Params p;
     if (pl.tc == 5) {
         // tensor-memory kernel: swizzled row boxes, scale / bias boxes of 8 groups
@@ -859,6 +867,27 @@ int run_pair(const void* x, const void* wg, const void* sg, const void* bg, cons
     p.kbf16 = 0x43004300u;
     qmv::Launch L{pl.grid, pl.block, pl.smem, static_cast<cudaStream_t>(stream), pdl_enabled()};
     return finish(qmv::launch_affine_pair(bits, dtype, pl.maxm, pl.R, pl.wide != 0, p, L));
+}
+
+// qmm beyond QMV_MAX_M rows: the tensor-memory kernel (one launch, each
+// weight decoded once) where the matrix has few 128-row tiles -- its K split
+// over a cluster keeps the SMs busy; measured on B200 (4-bit g64 bf16, M 16 /
+// 32 / 64): 4096 x 4096 27.6 / 37.2 / 101 us against 38.6 / 72.0 / 139 us in
+// 16-row chunks, 4096 x 14336 67 / 127 us against 104 / 199 us; for 28672 x
+// 4096 the chunks win (96 / 189 / 375 against 140 / 274 / 473 us).
+bool qmm_prefers_umma(int N) { return g_forced.path == 7 || (g_forced.path < 0 && N <= 5120); }
+
+// x rows per launch of qmv_qmm_affine beyond QMV_MAX_M rows: 32 or 16 when
+// the tensor-core ring kernel takes that many (x rows x groups of a
+// super-block <= 32 slot columns; more than 64 output rows), else QMV_MAX_M.
+int qmm_chunk(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s16) {
+    if (M <= QMV_MAX_M || N <= 64 || K <= 0) return QMV_MAX_M;
+    for (int c : {32, 16}) {
+        if (c >= M + QMV_MAX_M) continue;
+        TcbShape ts;
+        if (tcb_shape(c, N, K, bits, G, dtype, w16, s16, &ts)) return c;
+    }
+    return QMV_MAX_M;
 }
 
 int check_affine(int bits, int group) {
@@ -1028,10 +1057,25 @@ int qmv_qmm_affine(const void* x, const void* w_packed, const void* scales, cons
     if (K > 0 && !biases) return QMV_EINVAL;
     const size_t eb = elem_bytes(dtype);
     if (K > 0 && (!aligned(scales, eb) || !aligned(biases, eb))) return QMV_EALIGN;
-    // chunks of QMV_MAX_M x rows, back to back on the stream: a weight matrix
-    // that fits in L2 is read from HBM by the first chunk only
-    for (int m0 = 0; m0 < M; m0 += QMV_MAX_M) {
-        const int mc = M - m0 < QMV_MAX_M ? M - m0 : QMV_MAX_M;
+    // more than QMV_MAX_M rows: the tensor-memory kernel takes them all in one
+    // launch for matrices of few row tiles (qmm_prefers_umma, when its layout
+    // rules hold); otherwise the tensor-core ring kernel takes up to 32 rows a
+    // launch (its 32 slot columns: x rows x groups of a super-block), and the
+    // rest go in chunks of QMV_MAX_M
+    int chunk = QMV_MAX_M;
+    if (M > QMV_MAX_M) {
+        if (qmm_prefers_umma(N)) {
+            st = run(qmv::FAM_AFFINE, x, w_packed, scales, biases, nullptr, y, M, N, K, bits, group_size, dtype, 1, 1,
+                     stream, nullptr, 0, true);
+            if (st != QMV_EUNSUPPORTED) return st;
+        }
+        chunk = qmm_chunk(M, N, K, bits, group_size, dtype, aligned(w_packed, 16),
+                          aligned(scales, 16) && aligned(biases, 16));
+    }
+    // chunks, back to back on the stream: a weight matrix that fits in L2 is
+    // read from HBM by the first chunk only
+    for (int m0 = 0; m0 < M; m0 += chunk) {
+        const int mc = M - m0 < chunk ? M - m0 : chunk;
         const void* xc = x ? static_cast<const char*>(x) + (size_t)m0 * K * eb : nullptr;
         void* yc = static_cast<char*>(y) + (size_t)m0 * N * eb;
         st = run(qmv::FAM_AFFINE, xc, w_packed, scales, biases, nullptr, yc, mc, N, K, bits, group_size, dtype, 1,
@@ -1099,7 +1143,7 @@ int qmv_last_cuda_error(void) { return g_last_cuda; }
 int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size, int dtype, int w_align16,
                       char* buf, int buflen) {
     if (!buf || buflen <= 0) return QMV_EINVAL;
-    if (M < 1 || M > QMV_MAX_M || N < 1 || K < 0) return QMV_EINVAL;
+    if (M < 1 || M > QMV_QMM_MAX_M || N < 1 || K < 0) return QMV_EINVAL;
     int fam;
     if (family == 0) {
         if (check_affine(bits, group_size) != QMV_OK) return QMV_EUNSUPPORTED;
@@ -1110,8 +1154,22 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
         bits = 0;
     }
     Plan pl;
-    int st = make_plan(fam, M, N, K, bits, fam == qmv::FAM_AFFINE ? group_size : (family == 2 ? 16 : 32), dtype, w_align16 != 0, 1, &pl);
+    const bool qmm = M > QMV_MAX_M;
+    if (qmm && fam != qmv::FAM_AFFINE) return QMV_EINVAL;
+    int st = make_plan(fam, M, N, K, bits, fam == qmv::FAM_AFFINE ? group_size : (family == 2 ? 16 : 32), dtype,
+                       w_align16 != 0, 1, &pl, true, false, false, true, qmm && qmm_prefers_umma(N));
     if (st != QMV_OK) return st;
+    if (qmm && pl.tc != 5) {
+        // qmm: chunks of x rows, each through the qmv plan of its size
+        const int c = qmm_chunk(M, N, K, bits, group_size, dtype, w_align16 != 0, true);
+        st = make_plan(fam, c, N, K, bits, group_size, dtype, w_align16 != 0, 1, &pl);
+        if (st != QMV_OK) return st;
+        snprintf(buf, (size_t)buflen, "path=chunked%d chunks=%d ", c, (M + c - 1) / c);
+        const size_t n0 = strlen(buf);
+        if ((int)n0 >= buflen) return QMV_OK;
+        buf += n0;
+        buflen -= (int)n0;
+    }
     snprintf(buf, (size_t)buflen,
              "path=%s chunk=%d maxm=%d rows_per_warp=%d warps_k=%d warps_rows=%d tile_iters=%d "
              "grid=%u block=%u smem=%zu stage_sb=%d batch_sb=%d scale_ring=%d",

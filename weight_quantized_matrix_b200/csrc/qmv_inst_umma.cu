@@ -17,6 +17,7 @@ cudaError_t launch_umma_t(const Params& p, const UmmaParams& u, const Launch& L)
     const unsigned bit = 1u << (dev & 31);
     if (!(configured.load(std::memory_order_acquire) & bit)) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
@@ -46,6 +47,7 @@ template <int B, int MLD>
 cudaError_t clusters_t(const UmmaParams& u, size_t smem, int* out) {
     auto kern = qmv_umma_kernel<B, MLD>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)u.S, 1, 1);

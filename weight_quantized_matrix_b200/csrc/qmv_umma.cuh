@@ -36,7 +36,7 @@
 // ((t / 8) * M + m) * 16 + (t % 8) * 2 bytes, so the descriptor's stride
 // between 8-row groups is 128 bytes and between K halves 16 * M bytes.  Rows
 // m >= M of the MMA read the next rows of that buffer (never-read columns).
-// K split: the CTAs of a thread-block cluster (S <= 8) take contiguous K
+// K split: the CTAs of a thread-block cluster (S <= 16) take contiguous K
 // ranges of the same row tiles; their fp32 partials meet through distributed
 // shared memory (each CTA sums a slice of the rows in rank order), so nothing
 // outside the caller's buffers is written.
@@ -158,6 +158,32 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank
     asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
     return v;
 }
+// Waits that suspend: try_wait with a suspend-time hint parks the thread in
+// hardware until the phase completes (or the hint runs out), so waiting warps
+// take no issue slots from the decoders and the MMA thread.  (A plain
+// try_wait loop returned at once and spun: measured on B200 it starved the
+// SM's other warps, about 0.9 us per block of codes.)  Bounded by about one
+// second, as every wait here.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(1000000u)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool um_wait(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    }
+}
+
 // Arrive (release at cluster scope) on the mbarrier at the same shared
 // address in the CTA of the given cluster rank.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t local_bar, uint32_t rank) {
@@ -169,10 +195,10 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(1000000u)
         : "memory");
     return ok != 0;
 }
@@ -228,7 +254,7 @@ template <int B> __host__ __device__ constexpr UmXTab<B> um_make_xtab() {
 
 // Launch parameters of the tensor-memory kernel beyond Params.
 struct UmmaParams {
-    int S;            // K split = cluster size (1..8)
+    int S;            // K split = cluster size (1..16; beyond 8 non-portable)
     int DB;           // blocks in flight (even)
     int WST, SSL;     // weight stages, scale slots (<= 8 each)
     int nq, QC;       // K in quanta of QC codes (a range boundary)
@@ -353,7 +379,7 @@ __global__ void __launch_bounds__(320, 1) qmv_umma_kernel(const __grid_constant_
                 const int glast = min(ngr, (st + 1) * STAGE_CODES / G) - 1;
                 for (; snext <= glast / 8 && snext < nsslot; ++snext, ++ss) {
                     const int slot = ss % SSL, f = ss / SSL;
-                    if (ok && f > 0 && !mbar_wait(sempty(slot), (uint32_t)((f - 1) & 1))) ok = false;
+                    if (ok && f > 0 && !um_wait(sempty(slot), (uint32_t)((f - 1) & 1))) ok = false;
                     if (ok && lane == 0) {
                         mbar_arrive_expect_tx(sfull(slot), 4096u);
                         const int gx = k0 / G + 8 * snext;
@@ -363,7 +389,7 @@ __global__ void __launch_bounds__(320, 1) qmv_umma_kernel(const __grid_constant_
                     __syncwarp();
                 }
                 const int slot = ws % WST, f = ws / WST;
-                if (ok && f > 0 && !mbar_wait(wempty(slot), (uint32_t)((f - 1) & 1))) ok = false;
+                if (ok && f > 0 && !um_wait(wempty(slot), (uint32_t)((f - 1) & 1))) ok = false;
                 if (ok && lane == 0) {
                     mbar_arrive_expect_tx(wfull(slot), (uint32_t)STAGE_BYTES);
                     const int xe = (int)((long long)(k0 + st * STAGE_CODES) * B / 64);     // u64 elements
@@ -379,11 +405,11 @@ __global__ void __launch_bounds__(320, 1) qmv_umma_kernel(const __grid_constant_
         unsigned code = ok ? 0u : 2u;
         for (int s = 0; s < WST && s < ws; ++s) {
             const int g_ = ws - 1 - s;
-            if (!mbar_wait(wfull(g_ % WST), (uint32_t)((g_ / WST) & 1))) code |= 4u;
+            if (!um_wait(wfull(g_ % WST), (uint32_t)((g_ / WST) & 1))) code |= 4u;
         }
         for (int s = 0; s < SSL && s < ss; ++s) {
             const int g_ = ss - 1 - s;
-            if (!mbar_wait(sfull(g_ % SSL), (uint32_t)((g_ / SSL) & 1))) code |= 4u;
+            if (!um_wait(sfull(g_ % SSL), (uint32_t)((g_ / SSL) & 1))) code |= 4u;
         }
         if (code && lane == 0) atomicOr(p.fault, code);
     } else {
@@ -451,7 +477,7 @@ __global__ void __launch_bounds__(320, 1) qmv_umma_kernel(const __grid_constant_
             for (int i = 0; i < ntile_mine; ++i) {
                 for (int b = 0; b < nblk; ++b, ++gb) {
                     const int bs = gb % DB;
-                    if (ok && !mbar_wait(afull(bs), (uint32_t)((gb / DB) & 1))) {
+                    if (ok && !um_wait(afull(bs), (uint32_t)((gb / DB) & 1))) {
                         ok = false;
                         if (lane == 0) atomicOr(p.fault, 8u);
                     }
@@ -478,7 +504,7 @@ __global__ void __launch_bounds__(320, 1) qmv_umma_kernel(const __grid_constant_
             // the last commits complete before tensor memory is released
             for (int s = 0; s < DB && s < gb; ++s) {
                 const int g_ = gb - 1 - s;
-                if (!mbar_wait(dfull(g_ % DB), (uint32_t)((g_ / DB) & 1))) break;
+                if (!um_wait(dfull(g_ % DB), (uint32_t)((g_ / DB) & 1))) break;
             }
         } else {
             // ===================== decoders (warps 2..9) ===================
@@ -499,7 +525,7 @@ __global__ void __launch_bounds__(320, 1) qmv_umma_kernel(const __grid_constant_
                 const int gbt = gb;
                 auto epi = [&](int b) {
                     const int g = gbt + b, bs = g % DB;
-                    if (ok && !mbar_wait(dfull(bs), (uint32_t)((g / DB) & 1))) {
+                    if (ok && !um_wait(dfull(bs), (uint32_t)((g / DB) & 1))) {
                         ok = false;
                         if (lane == 0) atomicOr(p.fault, 16u);
                     }
@@ -524,11 +550,11 @@ __global__ void __launch_bounds__(320, 1) qmv_umma_kernel(const __grid_constant_
                         if (lane == 0) mbar_arrive(sempty(ss_cur % SSL));
                         ++ss_cur;
                     }
-                    if (ok && !mbar_wait(wfull(ws_cur % WST), (uint32_t)((ws_cur / WST) & 1))) {
+                    if (ok && !um_wait(wfull(ws_cur % WST), (uint32_t)((ws_cur / WST) & 1))) {
                         ok = false;
                         if (lane == 0) atomicOr(p.fault, 1u);
                     }
-                    if (ok && !mbar_wait(sfull(ss_cur % SSL), (uint32_t)((ss_cur / SSL) & 1))) {
+                    if (ok && !um_wait(sfull(ss_cur % SSL), (uint32_t)((ss_cur / SSL) & 1))) {
                         ok = false;
                         if (lane == 0) atomicOr(p.fault, 1u);
                     }
