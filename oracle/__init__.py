@@ -81,6 +81,8 @@ def lib():
         L.oracle_nearest_e2m1.argtypes = [d]; L.oracle_nearest_e2m1.restype = u
         L.oracle_nearest_e4m3.argtypes = [d]; L.oracle_nearest_e4m3.restype = u
         L.oracle_quantize_affine.restype = None
+        L.oracle_dequant_affine_f64.argtypes = [p, p, p, p, ll, ll, i, i, i, ll, ll]
+        L.oracle_dequant_affine_f64.restype = None
         _lib = L
     return _lib
 
@@ -252,6 +254,63 @@ def quantize_fp(w, N, K, mode, dtype, global_scale=1.0, rows=None, threads=1):
                                            DTYPE_CODES[dtype], a, b)
     _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
     return wq, sc
+
+
+def dequant_affine_f64(w, scales, biases, N, K, bits, group, dtype, rows=None, threads=1):
+    """Dequantized affine weights [N, K] in fp64 (rows outside `rows` stay 0)."""
+    out = np.zeros((N, K), dtype=np.float64)
+    L = lib()
+    w = np.ascontiguousarray(w); scales = np.ascontiguousarray(scales); biases = np.ascontiguousarray(biases)
+    fn = lambda a, b: L.oracle_dequant_affine_f64(_ptr(w), _ptr(scales), _ptr(biases), _ptr(out),
+                                                  N, K, bits, group, DTYPE_CODES[dtype], a, b)
+    _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
+    return out
+
+
+def _widen(a, dtype):
+    """Stored elements of `dtype` (float32, or uint16 bit patterns) as exact fp64."""
+    a = np.asarray(a)
+    if dtype == "f32":
+        return a.astype(np.float64)
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(
+        torch.float16 if dtype == "f16" else torch.bfloat16)
+    return t.to(torch.float64).numpy()
+
+
+# ---- batched Q / K / V projection --------------------------------------------
+def qmv_affine_qkv(x, q3, k3, v3, M, Nq, Nkv, K, bits, group, dtype, rows=None, threads=1):
+    """The three decode projections of one x in one call (wh-iron kernel-op
+    coverage audit, "batched_qkv_qgemv" row: Q / K / V qGEMV in one dispatch,
+    output concatenated [Q | K | V], K and V of the same size for grouped-query
+    attention).  q3, k3, v3 are (w_packed, scales, biases) triples with Nq,
+    Nkv, Nkv rows.  Returns (y, absdot), float64 [M, Nq + 2 Nkv]: each part is
+    qmv_affine of its matrix."""
+    parts = []
+    for (w, sc, bi), n, off in ((q3, Nq, 0), (k3, Nkv, Nq), (v3, Nkv, Nq + Nkv)):
+        r = None if rows is None else [t - off for t in rows if off <= t < off + n]
+        parts.append(qmv_affine(x, w, sc, bi, M, n, K, bits, group, dtype, rows=r, threads=threads))
+    y = np.concatenate([p_[0] for p_ in parts], axis=1)
+    a = np.concatenate([p_[1] for p_ in parts], axis=1)
+    return y, a
+
+
+# ---- RMSNorm fused into the qmv -----------------------------------------------
+def rms_norm(x, gamma, eps):
+    """x * gamma / sqrt(mean(x^2) + eps) per row, fp64 (x, gamma float64)."""
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return x * r * gamma
+
+
+def qmv_affine_rms_norm(x, gamma, eps, w, scales, biases, M, N, K, bits, group, dtype, rows=None, threads=1):
+    """RMSNorm of x fused into the affine qmv (wh-iron kernel-op coverage
+    audit, "rms_norm_qgemv" row): y[m, n] = sum_k xh[m, k] * w_hat[n, k] with
+    xh = rms_norm(x, gamma, eps) kept in full precision (it is not rounded to
+    the element type between the two steps), x and gamma stored in `dtype`.
+    fp64 throughout.  Returns (y, absdot) float64 [M, N]."""
+    xh = rms_norm(_widen(x, dtype).reshape(M, K), _widen(gamma, dtype).reshape(1, K), float(eps))
+    W = dequant_affine_f64(w, scales, biases, N, K, bits, group, dtype, rows=rows, threads=threads)
+    return xh @ W.T, np.abs(xh) @ np.abs(W).T
 
 
 # ---- fused gate + up with SwiGLU ---------------------------------------------

@@ -174,6 +174,28 @@ void oracle_dequant_affine_f32(const uint8_t* w, const void* scales, const void*
     }
 }
 
+/* Dequantized affine weights in fp64: w = scale * q + bias with the stored
+ * scale and bias widened exactly (MLX quantized_nax.h, dequantize).  The
+ * product is exact (at most 32 significant bits); the sum is exact whenever
+ * it fits 53 bits, which every f16 / bf16 scale and bias does (an f32 pair
+ * could exceed that only with exponents more than 29 apart, where the one
+ * fp64 rounding is far below any tolerance here).  Rows [n0, n1) of out
+ * [N, K]. */
+void oracle_dequant_affine_f64(const uint8_t* w, const void* scales, const void* biases,
+                               double* out, long long N, long long K, int bits, int group,
+                               int dtype, long long n0, long long n1) {
+    (void)N;
+    for (long long n = n0; n < n1; ++n) {
+        const uint8_t* row = w + n * oracle_row_bytes(K, bits);
+        for (long long k = 0; k < K; ++k) {
+            long long gi = n * (K / group) + k / group;
+            double s = load_elem(scales, (size_t)gi, dtype);
+            double b = load_elem(biases, (size_t)gi, dtype);
+            out[n * K + k] = s * (double)oracle_affine_code(row, k, bits) + b;
+        }
+    }
+}
+
 /* Block size along K and per-element width of each FP mode. */
 static int fp_block(int mode) { return mode == OR_NVFP4 ? 16 : 32; }
 static int fp_bits(int mode) { return mode == OR_MXFP8 ? 8 : 4; }

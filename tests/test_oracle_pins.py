@@ -765,3 +765,74 @@ def test_swiglu_clamp_route_weight_and_limits():
     assert np.allclose(mp, gp * up, rtol=1e-15)                               # silu(40) = 40 (1 - 4e-18)
     mn, _, _, _, _ = oracle.qmv_affine_swiglu(ones, zero_w, sg, neg, wu, su, bu, M, N, K, bits, group, "f32")
     assert (np.abs(mn) < 1e-15 * np.abs(up) + 1e-300).all()                   # silu(-40) = -40 e^-40
+
+
+# ------------------------------------------------ fp64 dequant, QKV, RMSNorm ----
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_dequant_f64_rounds_to_the_f32_check(bits, dtype):
+    """The fp64 weights round (once) to exactly the pinned fp32 check values."""
+    c = synth.affine_case(1, 5, 128, bits, 32, dtype, seed=bits)
+    w64 = oracle.dequant_affine_f64(c["w"][0], c["scales"][0], c["biases"][0], 5, 128, bits, 32, dtype)
+    w32 = oracle.dequant_affine_f32(c["w"][0], c["scales"][0], c["biases"][0], 5, 128, bits, 32, dtype)
+    assert np.array_equal(w64.astype(np.float32), w32)
+
+
+def test_dequant_f64_is_the_column_of_a_unit_x():
+    """x = e_k through the qmv oracle returns column k of the fp64 weights."""
+    N, K, bits, g = 7, 64, 5, 32
+    c = synth.affine_case(1, N, K, bits, g, "f32", seed=4)
+    W = oracle.dequant_affine_f64(c["w"][0], c["scales"][0], c["biases"][0], N, K, bits, g, "f32")
+    for k in (0, 31, 63):
+        x = np.zeros((1, K), dtype=np.float32); x[0, k] = 1.0
+        y, _ = oracle.qmv_affine(x, c["w"][0], c["scales"][0], c["biases"][0], 1, N, K, bits, g, "f32")
+        assert np.array_equal(y[0], W[:, k])
+
+
+def test_qkv_is_qmv_of_the_stacked_matrix():
+    """[Q | K | V] equals one qmv over the three matrices stacked along N, bit
+    for bit (the same fp64 sums)."""
+    M, Nq, Nkv, K, bits, g = 2, 24, 8, 128, 4, 64
+    cs = [synth.affine_case(M, n, K, bits, g, "bf16", seed=50 + i) for i, n in enumerate((Nq, Nkv, Nkv))]
+    x = cs[0]["x"][0]
+    t = [(c["w"][0], c["scales"][0], c["biases"][0]) for c in cs]
+    y, a = oracle.qmv_affine_qkv(x, *t, M, Nq, Nkv, K, bits, g, "bf16")
+    ws = np.concatenate([c["w"][0] for c in cs]); ss = np.concatenate([c["scales"][0] for c in cs])
+    bs = np.concatenate([c["biases"][0] for c in cs])
+    y2, a2 = oracle.qmv_affine(x, ws, ss, bs, M, Nq + 2 * Nkv, K, bits, g, "bf16")
+    assert np.array_equal(y, y2) and np.array_equal(a, a2)
+    rows = [0, Nq - 1, Nq, Nq + Nkv, Nq + 2 * Nkv - 1]
+    yr, _ = oracle.qmv_affine_qkv(x, *t, M, Nq, Nkv, K, bits, g, "bf16", rows=rows)
+    assert np.array_equal(yr[:, rows], y2[:, rows])
+
+
+def test_rms_norm_closed_forms():
+    """Constant rows: x = c gives gamma * c / sqrt(c^2 + eps); with eps = 0 and
+    gamma = 1 every row has unit RMS; scaling x leaves it unchanged (eps = 0)."""
+    K = 64
+    g = np.linspace(0.5, 2.0, K)
+    x = np.full((1, K), 3.0)
+    assert np.allclose(oracle.rms_norm(x, g, 1e-2), g * 3.0 / math.sqrt(9.0 + 1e-2), rtol=1e-15, atol=0)
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((3, K))
+    xh = oracle.rms_norm(x, np.ones(K), 0.0)
+    assert np.allclose(np.sqrt(np.mean(xh * xh, axis=1)), 1.0, rtol=1e-14)
+    assert np.allclose(oracle.rms_norm(7.5 * x, g, 0.0), oracle.rms_norm(x, g, 0.0), rtol=1e-14)
+
+
+def test_rms_norm_qmv_unit_x_and_scaling():
+    """x = 2 e_k (eps 0): xh = gamma_k sqrt(K) e_k, so y = gamma_k sqrt(K)
+    times column k of the weights; and y of alpha x equals y of x (eps 0)."""
+    N, K, bits, grp = 6, 64, 4, 32
+    c = synth.affine_case(1, N, K, bits, grp, "f32", seed=12)
+    gam = synth.to_storage(np.linspace(0.5, 1.5, K), "f32")
+    W = oracle.dequant_affine_f64(c["w"][0], c["scales"][0], c["biases"][0], N, K, bits, grp, "f32")
+    k = 17
+    x = np.zeros((1, K), dtype=np.float32); x[0, k] = 2.0
+    y, _ = oracle.qmv_affine_rms_norm(x, gam, 0.0, c["w"][0], c["scales"][0], c["biases"][0], 1, N, K, bits, grp, "f32")
+    assert np.allclose(y[0], float(gam[k]) * math.sqrt(K) * W[:, k], rtol=1e-14, atol=0)
+    xs = synth.to_storage(np.random.default_rng(1).standard_normal((1, K)), "f32")
+    y1, _ = oracle.qmv_affine_rms_norm(xs, gam, 0.0, c["w"][0], c["scales"][0], c["biases"][0], 1, N, K, bits, grp, "f32")
+    y2, _ = oracle.qmv_affine_rms_norm(xs * np.float32(4.0), gam, 0.0, c["w"][0], c["scales"][0], c["biases"][0], 1, N,
+                                       K, bits, grp, "f32")
+    assert np.allclose(y1, y2, rtol=1e-13, atol=1e-300)
