@@ -201,6 +201,42 @@ int qmv_affine_swiglu(const void* x, const void* w_gate, const void* s_gate, con
                       void* stream);
 
 /*
+ * qmv_affine_qkv -- the Q, K and V projections of one x in one launch
+ * (wh-iron kernel-op coverage audit, "batched_qkv_qgemv" row: Q / K / V
+ * 4-bit qGEMV in one dispatch, output concatenated [Q | K | V]; K and V have
+ * the same size, grouped-query attention).
+ *   w_q, s_q, b_q   [Nq, ...]  the Q matrix, as qmv_affine's w_packed, scales,
+ *   w_k, s_k, b_k   [Nkv, ...] biases (all three share K, bits, group_size)
+ *   w_v, s_v, b_v   [Nkv, ...]
+ *   y               [M, Nq + 2 Nkv] dtype: y[m, 0:Nq] = x W_q^T, then K, then V
+ * Each output as qmv_affine computes it; the row-tiled CUDA-core kernel reads
+ * each output row from its own matrix.  Nq, Nkv >= 0; a matrix with no rows
+ * may be NULL.  Other arguments, alignment and errors as qmv_affine.
+ */
+int qmv_affine_qkv(const void* x, const void* w_q, const void* s_q, const void* b_q, const void* w_k,
+                   const void* s_k, const void* b_k, const void* w_v, const void* s_v, const void* b_v,
+                   void* y, int M, int Nq, int Nkv, int K, int bits, int group_size, int dtype,
+                   void* stream);
+
+/*
+ * qmv_affine_rms_norm -- RMSNorm of x fused into the affine qmv (wh-iron
+ * kernel-op coverage audit, "rms_norm_qgemv" row):
+ *     y[m, n] = sum_k xh[m, k] * dequant(W)[n, k],
+ *     xh[m, k] = x[m, k] * gamma[k] / sqrt(mean_k x[m, k]^2 + eps),
+ * xh kept in fp32 (never rounded to dtype): the sum of squares and the
+ * products in fp32, then qmv_affine's accumulation and one rounding of y.
+ *   gamma   [K] dtype (device)
+ *   eps     >= 0 and finite (QMV_EINVAL otherwise)
+ * Other arguments, alignment and errors as qmv_affine (gamma aligned to its
+ * element).  Runs the row-tiled CUDA-core kernel: every block first reduces
+ * the sums of squares of the M x rows (read after the previous kernel in the
+ * stream completes), then stages xh instead of x.
+ */
+int qmv_affine_rms_norm(const void* x, const void* gamma, float eps, const void* w_packed,
+                        const void* scales, const void* biases, void* y, int M, int N, int K, int bits,
+                        int group_size, int dtype, void* stream);
+
+/*
  * qmv_qmm_affine -- small-M quantized matmul, y = x * dequant(W)^T for up to
  * QMV_QMM_MAX_M x rows (the qmm family of MLX quantized_nax.h and of the
  * wh-iron audit, M-batched prefill).  Arguments and layouts as qmv_affine,

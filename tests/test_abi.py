@@ -303,6 +303,24 @@ def test_swiglu_validation_before_any_launch():
     assert sw(M=0) == 0 and sw(N=0) == 0
 
 
+def test_qkv_and_rms_norm_validation_before_any_launch():
+    F = FAKE
+
+    def qkv(x=F, wq=F, wk=F, wv=F, y=F, M=1, Nq=64, Nkv=16, K=128, bits=4, gs=64, dt=2):
+        return L.qmv_affine_qkv(x, wq, F, F, wk, F, F, wv, F, F, y, M, Nq, Nkv, K, bits, gs, dt, None)
+
+    assert qkv(bits=7) == EUNSUP and qkv(K=100) == EINVAL and qkv(Nkv=-1) == EINVAL
+    assert qkv(wk=None) == EINVAL and qkv(wv=F + 2) == EALIGN
+    assert qkv(M=9) == EUNSUP and qkv(M=0) == 0 and qkv(Nq=0, Nkv=0) == 0
+
+    def rms(x=F, g=F, eps=1e-6, w=F, s=F, b=F, y=F, M=1, N=64, K=128, bits=4, gs=64, dt=2):
+        return L.qmv_affine_rms_norm(x, g, ctypes.c_float(eps), w, s, b, y, M, N, K, bits, gs, dt, None)
+
+    assert rms(eps=-1.0) == EINVAL and rms(eps=float("nan")) == EINVAL and rms(eps=float("inf")) == EINVAL
+    assert rms(g=None) == EINVAL and rms(g=F + 1) == EALIGN and rms(bits=1) == EUNSUP
+    assert rms(M=0) == 0
+
+
 @pytest.mark.parametrize("name", _declared())
 def test_python_binding_has_every_entry_point(name):
     """The binding exposes each C-ABI entry point under the same name."""

@@ -18,7 +18,7 @@ import os
 
 __all__ = [
     "QmvError", "qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
-    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_quantize_fp", "qmv_affine_gather", "qmv_affine_swiglu", "qmv_qmm_affine", "qmv_qvm_affine",
+    "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_quantize_fp", "qmv_affine_gather", "qmv_affine_swiglu", "qmv_affine_qkv", "qmv_affine_rms_norm", "qmv_qmm_affine", "qmv_qvm_affine",
     "qmv_qvm_workspace_bytes", "qmv_qvm_affine_noalloc", "qmv_status_string",
     "qmv_last_cuda_error",
     "qmv_describe_plan", "qmv_force_config", "DTYPES", "FP_MODES", "LIB_PATH", "lib",
@@ -63,6 +63,10 @@ _lib.qmv_quantize_fp.argtypes = [_p, _p, _p, _p, _i, _i, _i, _i, _p]
 _lib.qmv_quantize_fp.restype = _i
 _lib.qmv_affine_swiglu.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, ctypes.c_float, _p]
 _lib.qmv_affine_swiglu.restype = _i
+_lib.qmv_affine_qkv.argtypes = [_p] * 11 + [_i] * 7 + [_p]
+_lib.qmv_affine_qkv.restype = _i
+_lib.qmv_affine_rms_norm.argtypes = [_p, _p, ctypes.c_float, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p]
+_lib.qmv_affine_rms_norm.restype = _i
 _lib.qmv_affine_gather.restype = _i
 _lib.qmv_qmm_affine.restype = _i
 _lib.qmv_qvm_workspace_bytes.argtypes = [_i, _i]
@@ -253,6 +257,21 @@ def qmv_affine_swiglu(x, w_gate, s_gate, b_gate, w_up, s_up, b_up, route_weight,
     _check(_lib.qmv_affine_swiglu(_ptr(x), _ptr(w_gate), _ptr(s_gate), _ptr(b_gate), _ptr(w_up), _ptr(s_up),
                                   _ptr(b_up), _ptr(route_weight), _ptr(mid), M, N, K, bits, group_size,
                                   _dtype(dtype), ctypes.c_float(clamp), _stream(stream)), "qmv_affine_swiglu")
+
+
+def qmv_affine_qkv(x, q3, k3, v3, y, M, Nq, Nkv, K, bits, group_size, dtype, stream=None):
+    """Q, K and V projections in one launch; q3, k3, v3 are (w_packed, scales,
+    biases) and y is [M, Nq + 2 Nkv] = [Q | K | V]."""
+    _check(_lib.qmv_affine_qkv(_ptr(x), *(_ptr(t) for t in q3), *(_ptr(t) for t in k3), *(_ptr(t) for t in v3),
+                               _ptr(y), M, Nq, Nkv, K, bits, group_size, _dtype(dtype), _stream(stream)),
+           "qmv_affine_qkv")
+
+
+def qmv_affine_rms_norm(x, gamma, eps, w_packed, scales, biases, y, M, N, K, bits, group_size, dtype, stream=None):
+    """RMSNorm of x (gamma [K], eps) fused into the affine qmv."""
+    _check(_lib.qmv_affine_rms_norm(_ptr(x), _ptr(gamma), ctypes.c_float(eps), _ptr(w_packed), _ptr(scales),
+                                    _ptr(biases), _ptr(y), M, N, K, bits, group_size, _dtype(dtype), _stream(stream)),
+           "qmv_affine_rms_norm")
 
 
 def qmv_describe_plan(family, M, N, K, bits=4, group_size=64, dtype="bf16", w_align16=True) -> str:

@@ -497,10 +497,11 @@ bool umma_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool 
 
 // Choose the launch shape.  Returns QMV_OK or an error (sizes too large).
 int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, bool w16, int batch, Plan* pl,
-              bool s16 = true, bool gather = false, bool pair = false, bool x16 = true, bool qmm = false) {
-    // pair (fused gate + up): N counts the 2N virtual rows; only the
-    // row-tiled CUDA-core kernel has the pair epilogue
-    if (pair) gather = true;
+              bool s16 = true, bool gather = false, bool pair = false, bool x16 = true, bool qmm = false,
+              bool qkv = false, bool norm = false) {
+    // pair (fused gate + up): N counts the 2N virtual rows; pair, Q / K / V
+    // and the fused RMSNorm run on the row-tiled CUDA-core kernel only
+    if (pair || qkv || norm) gather = true;
     const FmtInfo fi = fmt_info(fam, bits);
     const bool aff = fam == qmv::FAM_AFFINE;
     int maxm = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
@@ -512,7 +513,8 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     // grid-dependency wait, one block per row) --------------------------------
     // (N <= 64 any M; up to 512 rows for one or two x rows: measured faster
     // than the row-tiled kernels on B200 up to about 1.3 MB of weights)
-    if (!pair && K > 0 && (g_forced.path == 5 || (g_forced.path < 0 && (N <= 64 || (N <= 512 && M <= 2))))) {
+    if (!pair && !qkv && !norm && K > 0 &&
+        (g_forced.path == 5 || (g_forced.path < 0 && (N <= 64 || (N <= 512 && M <= 2))))) {
         const int units = K / 32;
         int thr = ((units + 31) / 32) * 32;
         if (thr > 256) thr = 256;
@@ -622,6 +624,8 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     if (pair) {
         if (R < 2) R = 2;
         if (!qmv::pair_shape_instantiated(maxm, R, wide)) R = 2;
+    } else if (qkv) {
+        if (!qmv::qkv_shape_instantiated(maxm, R, wide)) R = wide ? (maxm <= 2 ? 4 : 2) : 1;
     } else if (!qmv::shape_instantiated(maxm, R, wide)) {
         R = 1;
     }
@@ -645,7 +649,7 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     long long ti = (long long)((budget > red ? budget - red : 0) / per_iter);
     if (ti < 1) ti = 1;
     if (ti > iters_needed) ti = iters_needed;
-    const size_t smem = per_iter * ti + red;
+    const size_t smem = per_iter * ti + red + (norm ? 512 : 0);     // + the RMSNorm partial sums
     if (smem > (size_t)qmv::kMaxSmem) return QMV_EUNSUPPORTED;
 
     const long long rows_per_block = (long long)wr * R;
@@ -762,7 +766,7 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     if (st != QMV_OK) return st;
     // M > 8 (qmm): only the tensor-memory kernel and the tensor-core ring take it
     if (M > QMV_MAX_M && pl.tc != 5 && pl.tc != 2) return QMV_EUNSUPPORTED;
-    qmv::Params p;
+    qmv::Params p{};
     if (pl.tc == 5) {
         // tensor-memory kernel: swizzled row boxes, scale / bias boxes of 8 groups
         if (!encode_rows_map_sw128(&p.wmap, w, row_bytes, N, batch, 128) ||
@@ -803,6 +807,7 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     qmv::Launch L{pl.grid, pl.block, pl.smem, static_cast<cudaStream_t>(stream), pdl_enabled() && !ids};
     p.ids = ids;
     p.n_experts = n_experts;
+    p.gamma = nullptr; p.eps = 0.f;
     cudaError_t e;
     p.sps = pl.sps; p.pitch = pl.pitch; p.fault = nullptr;
     p.sring = pl.sring; p.soff = pl.soff; p.boff = pl.boff; p.sbw = pl.sbw;
@@ -851,10 +856,12 @@ int run_pair(const void* x, const void* wg, const void* sg, const void* bg, cons
     const bool w16 = aligned(wg, 16) && aligned(wu, 16);
     int st = make_plan(qmv::FAM_AFFINE, M, 2 * N, K, bits, G, dtype, w16, 1, &pl, false, true, true);
     if (st != QMV_OK) return st;
-    qmv::Params p;
+    if (pl.tc != 0) return QMV_EUNSUPPORTED;       // the row-tiled kernel's launch shape only
+    qmv::Params p{};
     p.x = x; p.w = static_cast<const uint8_t*>(wg); p.scales = sg; p.biases = bg; p.gscale = nullptr; p.y = y;
     p.w2 = static_cast<const uint8_t*>(wu); p.scales2 = su; p.biases2 = bu;
     p.route_w = route_w; p.act_clamp = clamp;
+    p.gamma = nullptr; p.eps = 0.f;
     p.M = M; p.N = N; p.K = K; p.G = G;
     p.wk = pl.wk; p.wr = pl.wr; p.tile_iters = pl.tile_iters;
     const size_t eb = elem_bytes(dtype);
@@ -888,6 +895,66 @@ int qmm_chunk(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s1
         if (tcb_shape(c, N, K, bits, G, dtype, w16, s16, &ts)) return c;
     }
     return QMV_MAX_M;
+}
+
+// Fills the Params fields every row-tiled launch takes.
+void base_params(qmv::Params* p, const Plan& pl, const void* x, const void* w, const void* s, const void* b, void* y,
+                 int M, int N, int K, int bits, int G, int dtype) {
+    p->x = x; p->w = static_cast<const uint8_t*>(w); p->scales = s; p->biases = b; p->gscale = nullptr; p->y = y;
+    p->M = M; p->N = N; p->K = K; p->G = G;
+    p->wk = pl.wk; p->wr = pl.wr; p->tile_iters = pl.tile_iters;
+    const size_t eb = elem_bytes(dtype);
+    p->x_vec = (aligned(x, 16) && ((size_t)K * eb) % 16 == 0) ? 1 : 0;
+    p->x_bs = 0; p->w_bs = 0; p->s_bs = 0; p->y_bs = 0;
+    p->w_row = (long long)K * bits / 8;
+    p->ids = nullptr; p->n_experts = 0;
+    p->sps = 0; p->pitch = 0; p->fault = nullptr; p->sring = 0; p->soff = 0; p->boff = 0; p->sbw = 0;
+    p->kf32 = 0x4B000000u;
+    p->kbf16 = 0x43004300u;
+}
+
+// Q / K / V in one call: the row-tiled CUDA-core kernel over the Nq + 2 Nkv
+// output rows, each row reading its own matrix.
+int run_qkv(const void* x, const void* const (&w)[3], const void* const (&s)[3], const void* const (&b)[3], void* y,
+            int M, int Nq, int Nkv, int K, int bits, int G, int dtype, void* stream) {
+    const int N = Nq + 2 * Nkv;
+    Plan pl;
+    const bool w16 = aligned(w[0], 16) && aligned(w[1], 16) && aligned(w[2], 16);
+    int st = make_plan(qmv::FAM_AFFINE, M, N, K, bits, G, dtype, w16, 1, &pl, false, true, false, true, false, true);
+    if (st != QMV_OK) return st;
+    if (pl.tc != 0) return QMV_EUNSUPPORTED;       // the row-tiled kernel's launch shape only
+    qmv::Params p{};
+    base_params(&p, pl, x, w[0], s[0], b[0], y, M, N, K, bits, G, dtype);
+    p.w2 = static_cast<const uint8_t*>(w[1]); p.scales2 = s[1]; p.biases2 = b[1];
+    p.w3 = static_cast<const uint8_t*>(w[2]); p.scales3 = s[2]; p.biases3 = b[2];
+    p.n1 = Nq; p.n2 = Nq + Nkv;
+    qmv::Launch L{pl.grid, pl.block, pl.smem, static_cast<cudaStream_t>(stream), pdl_enabled()};
+    return finish(qmv::launch_affine_qkv(bits, dtype, pl.maxm, pl.R, pl.wide != 0, p, L));
+}
+
+// RMSNorm fused into the row-tiled CUDA-core kernel's x staging.
+int run_rms_norm(const void* x, const void* gamma, float eps, const void* w, const void* s, const void* b, void* y,
+                 int M, int N, int K, int bits, int G, int dtype, void* stream) {
+    Plan pl;
+    int st = make_plan(qmv::FAM_AFFINE, M, N, K, bits, G, dtype, aligned(w, 16), 1, &pl, false, true, false, true,
+                       false, false, true);
+    if (st != QMV_OK) return st;
+    if (pl.tc != 0) return QMV_EUNSUPPORTED;       // the row-tiled kernel's launch shape only
+    qmv::Params p{};
+    base_params(&p, pl, x, w, s, b, y, M, N, K, bits, G, dtype);
+    p.gamma = gamma; p.eps = eps;
+    qmv::Launch L{pl.grid, pl.block, pl.smem, static_cast<cudaStream_t>(stream), pdl_enabled()};
+    cudaError_t e;
+    switch (bits) {
+        case 2: e = qmv::launch_affine_b2(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
+        case 3: e = qmv::launch_affine_b3(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
+        case 4: e = qmv::launch_affine_b4(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
+        case 5: e = qmv::launch_affine_b5(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
+        case 6: e = qmv::launch_affine_b6(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
+        case 8: e = qmv::launch_affine_b8(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
+        default: return QMV_EUNSUPPORTED;
+    }
+    return finish(e);
 }
 
 int check_affine(int bits, int group) {
@@ -1103,6 +1170,46 @@ int qmv_affine_swiglu(const void* x, const void* w_gate, const void* s_gate, con
     if ((long long)N * 2 > 0x7FFFFFFFLL) return QMV_EINVAL;
     return run_pair(x, w_gate, s_gate, b_gate, w_up, s_up, b_up, route_weight, mid, M, N, K, bits, group_size,
                     dtype, clamp, stream);
+}
+
+int qmv_affine_qkv(const void* x, const void* w_q, const void* s_q, const void* b_q, const void* w_k,
+                   const void* s_k, const void* b_k, const void* w_v, const void* s_v, const void* b_v, void* y,
+                   int M, int Nq, int Nkv, int K, int bits, int group_size, int dtype, void* stream) {
+    int st = check_affine(bits, group_size);
+    if (st != QMV_OK) return st;
+    if (Nq < 0 || Nkv < 0 || K % group_size != 0) return QMV_EINVAL;
+    if ((long long)Nq + 2LL * Nkv > 0x7FFFFFFFLL) return QMV_EINVAL;
+    const int N = Nq + 2 * Nkv;
+    st = check_common(x, w_q, s_q, y, M, N, K, dtype);
+    if (st != QMV_OK || M == 0 || N == 0) return st;
+    const void* w[3] = {w_q, w_k, w_v};
+    const void* s[3] = {s_q, s_k, s_v};
+    const void* b[3] = {b_q, b_k, b_v};
+    const size_t eb = elem_bytes(dtype);
+    if (K > 0) {
+        for (int i = 0; i < 3; ++i) {
+            const int n = i == 0 ? Nq : Nkv;
+            if (n == 0) continue;
+            if (!w[i] || !s[i] || !b[i]) return QMV_EINVAL;
+            if (!aligned(w[i], 4) || !aligned(s[i], eb) || !aligned(b[i], eb)) return QMV_EALIGN;
+        }
+    }
+    return run_qkv(x, w, s, b, y, M, Nq, Nkv, K, bits, group_size, dtype, stream);
+}
+
+int qmv_affine_rms_norm(const void* x, const void* gamma, float eps, const void* w_packed, const void* scales,
+                        const void* biases, void* y, int M, int N, int K, int bits, int group_size, int dtype,
+                        void* stream) {
+    int st = check_affine(bits, group_size);
+    if (st != QMV_OK) return st;
+    if (K % group_size != 0) return QMV_EINVAL;
+    if (!(eps >= 0.0f) || !(eps < 3.0e38f)) return QMV_EINVAL;        // negative, NaN or infinite
+    st = check_common(x, w_packed, scales, y, M, N, K, dtype);
+    if (st != QMV_OK || M == 0 || N == 0) return st;
+    if (K > 0 && (!biases || !gamma)) return QMV_EINVAL;
+    const size_t eb = elem_bytes(dtype);
+    if (K > 0 && (!aligned(scales, eb) || !aligned(biases, eb) || !aligned(gamma, eb))) return QMV_EALIGN;
+    return run_rms_norm(x, gamma, eps, w_packed, scales, biases, y, M, N, K, bits, group_size, dtype, stream);
 }
 
 int qmv_qvm_affine(const void* x, const void* w_packed, const void* scales, const void* biases, void* y,

@@ -95,7 +95,22 @@ struct Params {
     const void* biases2;
     const float* route_w;   // [M] per x row, or null for 1
     float act_clamp;        // clamp value; inactive at or below 1e-6
+    // Q / K / V in one call (RMODE_QKV kernels): output rows [0, n1) read
+    // w / scales / biases, [n1, n2) w2 / scales2 / biases2, [n2, N) w3 /
+    // scales3 / biases3; y is [M, N] with the three parts side by side.
+    const uint8_t* w3;
+    const void* scales3;
+    const void* biases3;
+    int n1, n2;
+    // RMSNorm of x fused in (row-tiled kernel): non-null gamma [K] (dtype)
+    // scales x staged for the products by gamma[k] / sqrt(mean(x[m]^2) + eps).
+    const void* gamma;
+    float eps;
 };
+
+// Row mapping of the row-tiled kernel: plain, the interleaved gate / up
+// pair (SwiGLU), or the three Q / K / V matrices.
+enum RowMode { RMODE_PLAIN = 0, RMODE_PAIR = 1, RMODE_QKV = 2 };
 
 // ---------------------------------------------------------------- dtypes ---
 template <class T> struct DT;
@@ -260,7 +275,7 @@ template <int FAM, int BITS> struct Fmt {
 // k-thread cc % KT at iteration cc / KT.
 template <int FAM, int B, class T, int MAXM, int U>
 __device__ __forceinline__ void stage_x(const Params& p, const char* Xb, float4* xs, float* sx, int t0,
-                                        int tcn, int KT, int TI) {
+                                        int tcn, int KT, int TI, const float* rnorm = nullptr) {
     constexpr int C = 32 * U;
     constexpr bool AFF = (FAM == FAM_AFFINE);
     const int items = MAXM * tcn * U;
@@ -300,6 +315,13 @@ __device__ __forceinline__ void stage_x(const Params& p, const char* Xb, float4*
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.f;
         }
+        if (rnorm && m < p.M) {
+            // RMSNorm: x * r_m * gamma[k], in fp32 (kept unrounded)
+            const long long k0 = (long long)(t0 + cc) * C + u * 32;
+            const float r = rnorm[m];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(__fmul_rn(v[j], r), DT<T>::ld(p.gamma, k0 + j));
+        }
         if constexpr (AFF) {
             float s = 0.f;                      // sum(x), widened per element
 #pragma unroll
@@ -318,7 +340,7 @@ __device__ __forceinline__ void stage_x(const Params& p, const char* Xb, float4*
 // Per-unit scales of chunk c for R rows (affine: scale + bias of the unit's
 // group; MX: one block scale; NV: two block scales per unit).  PAIR: row r is
 // virtual row rowc[r] of the interleaved gate / up pair (odd rows: up).
-template <int FAM, class T, int R, int U, bool PAIR = false>
+template <int FAM, class T, int R, int U, int RMODE = RMODE_PLAIN>
 __device__ __forceinline__ void load_scales(const Params& p, const int (&rowc)[R], int c, long long sb,
                                             float (&sc)[R][U][2], float (&bi)[R][U]) {
     constexpr int C = 32 * U;
@@ -332,9 +354,12 @@ __device__ __forceinline__ void load_scales(const Params& p, const int (&rowc)[R
             long long row = rowc[r];
             const void* sp = p.scales;
             const void* bp = p.biases;
-            if constexpr (PAIR) {
+            if constexpr (RMODE == RMODE_PAIR) {
                 if (row & 1) { sp = p.scales2; bp = p.biases2; }
                 row >>= 1;
+            } else if constexpr (RMODE == RMODE_QKV) {
+                if (row >= p.n2) { sp = p.scales3; bp = p.biases3; row -= p.n2; }
+                else if (row >= p.n1) { sp = p.scales2; bp = p.biases2; row -= p.n1; }
             }
             const long long rb = row * KG;
             if constexpr (FAM == FAM_AFFINE) {
@@ -467,9 +492,11 @@ __device__ __forceinline__ void warp_allreduce(float (&acc)[R][MAXM]) {
 // The rows are the 2N virtual rows of the interleaved pair (virtual row 2n =
 // gate row n, 2n + 1 = up row n), so each warp holds both sums of its R / 2
 // outputs and writes y[m, n] = swiglu_act(gate, up) * route_w[m].
-template <int FAM, int BITS, class T, int MAXM, int R, bool WIDE, bool PAIR = false>
+template <int FAM, int BITS, class T, int MAXM, int R, bool WIDE, int RMODE = RMODE_PLAIN>
 __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
+    constexpr bool PAIR = RMODE == RMODE_PAIR;
     static_assert(!PAIR || (FAM == FAM_AFFINE && R % 2 == 0), "pair rows come in twos");
+    static_assert(RMODE != RMODE_QKV || FAM == FAM_AFFINE, "Q / K / V are affine");
     using F = Fmt<FAM, BITS>;
     constexpr int B = F::kBits;
     constexpr int U = WIDE ? F::kWideUnits : 1;
@@ -534,6 +561,9 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
             if constexpr (PAIR) {
                 base = (prow & 1) ? p.w2 : W;
                 prow >>= 1;
+            } else if constexpr (RMODE == RMODE_QKV) {
+                if (prow >= p.n2) { base = p.w3; prow -= p.n2; }
+                else if (prow >= p.n1) { base = p.w2; prow -= p.n1; }
             }
             const uint8_t* src = base + prow * p.w_row + (long long)c * (C * B / 8);
             if constexpr (WIDE) {
@@ -547,7 +577,7 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
                 for (int q = 0; q < CW; ++q) wv[r][q] = __ldg(reinterpret_cast<const uint32_t*>(src) + q);
             }
         }
-        load_scales<FAM, T, R, U, PAIR>(p, rowc, c, sb, sc, bi);
+        load_scales<FAM, T, R, U, RMODE>(p, rowc, c, sb, sc, bi);
     };
 
     const uint32_t kf32 = p.kf32;
@@ -561,6 +591,36 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
     grid_launch_dependents();
     grid_wait();
 
+    // RMSNorm: r_m = 1 / sqrt(mean_k x[m,k]^2 + eps) for every x row, by the
+    // whole block (fp32 sums of squares, warp shuffles, then one shared pass)
+    float* rnorm = nullptr;
+    if (p.gamma) {
+        float* part = red + (size_t)p.wk * p.wr * R * MAXM;      // [warps][MAXM], then r[MAXM]
+        const int nw = blockDim.x >> 5;
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) {
+            float q = 0.f;
+            if (m < p.M) {
+                const T* xr = reinterpret_cast<const T*>(Xb) + (long long)m * p.K;
+                for (int k = threadIdx.x; k < p.K; k += blockDim.x) {
+                    const float v = DT<T>::ld(xr, k);
+                    q = fmaf(v, v, q);
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xFFFFFFFFu, q, o);
+            if (lane == 0) part[warp * MAXM + m] = q;
+        }
+        __syncthreads();
+        if (threadIdx.x < MAXM) {
+            float q = 0.f;
+            for (int w = 0; w < nw; ++w) q += part[w * MAXM + threadIdx.x];
+            part[nw * MAXM + threadIdx.x] = 1.0f / sqrtf(q / (float)p.K + p.eps);
+        }
+        __syncthreads();
+        rnorm = part + nw * MAXM;
+    }
+
     for (int t0 = 0; t0 < NC; t0 += TC) {
         const int tcn = min(TC, NC - t0);          // chunks in this tile
         __syncthreads();
@@ -570,7 +630,7 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
             have = kt < tcn;
             if (have) load_chunk(t0 + kt);
         }
-        stage_x<FAM, B, T, MAXM, U>(p, Xb, xs, sx, t0, tcn, KT, TI);
+        stage_x<FAM, B, T, MAXM, U>(p, Xb, xs, sx, t0, tcn, KT, TI, rnorm);
         __syncthreads();
         for (int i = 0; have;) {
             compute_chunk<FAM, B, MAXM, R, U>(wv, sc, bi, xs + (size_t)i * (C / 4) * KT + kt,

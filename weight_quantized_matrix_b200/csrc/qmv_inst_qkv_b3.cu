@@ -1,0 +1,13 @@
+// qmv_inst_qkv_b3.cu -- Q / K / V in one call, affine 3-bit (all dtypes and
+// the row-tiled shapes of large N).
+#include "qmv_launch.cuh"
+
+namespace qmv {
+
+cudaError_t launch_affine_qkv_b3(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L) {
+#define BITS_ 3
+    QMV_QKV_DISPATCH_DTYPE()
+#undef BITS_
+}
+
+}  // namespace qmv

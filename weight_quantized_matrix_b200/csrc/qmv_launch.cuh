@@ -112,6 +112,15 @@ cudaError_t launch_umma_affine(int bits, int mld, const Params& p, const UmmaPar
 // Clusters of the tensor-memory kernel that fit on the device at once.
 cudaError_t umma_max_clusters(int bits, const UmmaParams& u, size_t smem, int* out);
 
+// Q / K / V in one call (qmv_kernel<..., RMODE_QKV>, affine): the shapes the
+// row-tiled picker takes for large N (R = 4 wide at maxm <= 2, R = 2 wide
+// above; R = 1 on the 4-byte path).
+cudaError_t launch_affine_qkv(int bits, int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+inline bool qkv_shape_instantiated(int maxm, int R, bool wide) {
+    if (!wide) return R == 1 && (maxm == 1 || maxm == 2 || maxm == 4 || maxm == 8);
+    return (maxm <= 2 && R == 4) || ((maxm == 4 || maxm == 8) && R == 2);
+}
+
 // Which (maxm, R, wide) shapes exist.
 inline bool shape_instantiated(int maxm, int R, bool wide) {
     if (!wide) return R == 1 && (maxm == 1 || maxm == 2 || maxm == 4 || maxm == 8);
@@ -139,7 +148,7 @@ inline bool shape_instantiated(int maxm, int R, bool wide) {
 #define QMV_PAIR_SHAPE(T_, MAXM_, R_, WIDE_)                                                 \
     if (maxm == MAXM_ && R == R_ && wide == WIDE_) {                                         \
         static std::atomic<unsigned> cfg_{0};                                                \
-        return launch_kernel(qmv_kernel<FAM_AFFINE, BITS_, T_, MAXM_, R_, WIDE_, true>, cfg_, L, p); \
+        return launch_kernel(qmv_kernel<FAM_AFFINE, BITS_, T_, MAXM_, R_, WIDE_, RMODE_PAIR>, cfg_, L, p); \
     }
 #define QMV_PAIR_SHAPES(T_)                                                                  \
     QMV_PAIR_SHAPE(T_, 1, 2, true) QMV_PAIR_SHAPE(T_, 1, 4, true)                            \
@@ -152,6 +161,24 @@ inline bool shape_instantiated(int maxm, int R, bool wide) {
         case 0: { QMV_PAIR_SHAPES(float) break; }                                            \
         case 1: { QMV_PAIR_SHAPES(__half) break; }                                           \
         case 2: { QMV_PAIR_SHAPES(__nv_bfloat16) break; }                                    \
+        default: break;                                                                      \
+    }                                                                                        \
+    return cudaErrorInvalidValue;
+#define QMV_QKV_SHAPE(T_, MAXM_, R_, WIDE_)                                                  \
+    if (maxm == MAXM_ && R == R_ && wide == WIDE_) {                                         \
+        static std::atomic<unsigned> cfg_{0};                                                \
+        return launch_kernel(qmv_kernel<FAM_AFFINE, BITS_, T_, MAXM_, R_, WIDE_, RMODE_QKV>, cfg_, L, p); \
+    }
+#define QMV_QKV_SHAPES(T_)                                                                   \
+    QMV_QKV_SHAPE(T_, 1, 4, true) QMV_QKV_SHAPE(T_, 2, 4, true)                              \
+    QMV_QKV_SHAPE(T_, 4, 2, true) QMV_QKV_SHAPE(T_, 8, 2, true)                              \
+    QMV_QKV_SHAPE(T_, 1, 1, false) QMV_QKV_SHAPE(T_, 2, 1, false)                            \
+    QMV_QKV_SHAPE(T_, 4, 1, false) QMV_QKV_SHAPE(T_, 8, 1, false)
+#define QMV_QKV_DISPATCH_DTYPE()                                                             \
+    switch (dtype) {                                                                         \
+        case 0: { QMV_QKV_SHAPES(float) break; }                                             \
+        case 1: { QMV_QKV_SHAPES(__half) break; }                                            \
+        case 2: { QMV_QKV_SHAPES(__nv_bfloat16) break; }                                     \
         default: break;                                                                      \
     }                                                                                        \
     return cudaErrorInvalidValue;
