@@ -11,8 +11,9 @@ the GIL, so a thread pool over row ranges runs them in parallel
 
 Page citations for each function are in the C file: the MLX
 ``quantized_nax.h`` source page (pack geometry, LSB-first codes,
-``w = scale * q + bias``), the wh-iron kernel-op coverage audit (Track 1 formats:
-E2M1, E4M3, E8M0, MXFP4, NVFP4, MXFP8) and the MLX pull request adding
+``w = scale * q + bias``), the wh-iron kernel-op coverage audit (the 30 Track 1
+formats: E2M1 / E4M3 / E5M2 / signed-int elements with E8M0, E4M3, FP32 or
+FP16 block scales) and the MLX pull request adding
 ``affine_qmv_fast_rows`` (fp32-widened sum(x)).
 """
 from __future__ import annotations
@@ -32,6 +33,32 @@ F32, F16, BF16 = 0, 1, 2
 MXFP4, NVFP4, MXFP8 = 0, 1, 2
 DTYPE_CODES = {"f32": F32, "f16": F16, "bf16": BF16}
 FP_MODES = {"mxfp4": MXFP4, "nvfp4": NVFP4, "mxfp8": MXFP8}
+
+# Track-1 symmetric block-scaled formats (wh-iron kernel-op coverage audit,
+# "Quantization precision coverage", Track 1 table): name -> (element, element
+# bits, block along K, block-scale type, FP32 global).  The integer rows: int2..8
+# with an FP32 scale per group of 64, mxint2..8 with an E8M0 scale per 32; every
+# FP32-scaled format has an FP16-scale twin "<name>_f16" (same element and
+# block).  30 formats.
+_ELEM_CODES = {"e2m1": 0, "e4m3": 1, "e5m2": 2, "int": 3}
+_SCALE_CODES = {"e8m0": 0, "e4m3": 1, "f32": 2, "f16": 3}
+TRACK1 = {
+    "nvfp4": ("e2m1", 4, 16, "e4m3", True),
+    "mxfp4": ("e2m1", 4, 32, "e8m0", False),
+    "mxfp8_e4m3": ("e4m3", 8, 32, "e8m0", False),
+    "mxfp8_e5m2": ("e5m2", 8, 32, "e8m0", False),
+    "nvfp8": ("e4m3", 8, 16, "f32", False),
+    "fp4": ("e2m1", 4, 32, "f32", False),
+    "fp8_e4m3": ("e4m3", 8, 32, "f32", False),
+    "fp8_e5m2": ("e5m2", 8, 32, "f32", False),
+}
+for _b in (2, 3, 4, 5, 6, 8):
+    TRACK1[f"int{_b}"] = ("int", _b, 64, "f32", False)
+for _b in (2, 3, 4, 5, 6, 8):
+    TRACK1[f"mxint{_b}"] = ("int", _b, 32, "e8m0", False)
+for _name in [n for n, v in TRACK1.items() if v[3] == "f32"]:
+    _e, _bb, _blk, _, _g = TRACK1[_name]
+    TRACK1[_name + "_f16"] = (_e, _bb, _blk, "f16", _g)
 
 
 def build(force: bool = False) -> str:
@@ -83,6 +110,13 @@ def lib():
         L.oracle_quantize_affine.restype = None
         L.oracle_dequant_affine_f64.argtypes = [p, p, p, p, ll, ll, i, i, i, ll, ll]
         L.oracle_dequant_affine_f64.restype = None
+        L.oracle_e5m2.argtypes = [u]; L.oracle_e5m2.restype = d
+        L.oracle_sint.argtypes = [u, i]; L.oracle_sint.restype = d
+        L.oracle_block_scale.argtypes = [p, ll, i]; L.oracle_block_scale.restype = d
+        L.oracle_dequant_block_scaled_f32.argtypes = [p, p, i, f, p, ll, ll, i, i, i, i, ll, ll]
+        L.oracle_dequant_block_scaled_f32.restype = None
+        L.oracle_qmv_block_scaled.argtypes = [p, p, p, i, f, p, p, ll, ll, ll, i, i, i, i, i, ll, ll]
+        L.oracle_qmv_block_scaled.restype = None
         _lib = L
     return _lib
 
@@ -132,6 +166,8 @@ def row_bytes(K, bits): return lib().oracle_row_bytes(K, bits)
 def e2m1(c): return lib().oracle_e2m1(int(c))
 def e4m3(c): return lib().oracle_e4m3(int(c))
 def e8m0(e): return lib().oracle_e8m0(int(e))
+def e5m2(c): return lib().oracle_e5m2(int(c))
+def sint(q, bits): return lib().oracle_sint(int(q), int(bits))
 def round_f32_sum(a, b): return lib().oracle_round_f32_sum(float(a), float(b))
 def f32_to_bf16(v): return lib().oracle_f32_to_bf16(float(v))
 def f32_to_f16(v): return lib().oracle_f32_to_f16(float(v))
@@ -162,6 +198,45 @@ def dequant_fp_f32(w, scales, global_scale, N, K, mode, rows=None, threads=1):
                                               FP_MODES[mode], a, b)
     _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
     return out
+
+
+def block_scales(scales, count, kind):
+    """The first ``count`` block scales of a raw scale array, widened exactly
+    (kind: "e8m0", "e4m3", "f32" or "f16")."""
+    a = np.ascontiguousarray(scales)
+    L = lib()
+    return np.array([L.oracle_block_scale(_ptr(a), i, _SCALE_CODES[kind]) for i in range(count)])
+
+
+def _track1(fmt):
+    e, b, blk, sk, g = TRACK1[fmt]
+    return _ELEM_CODES[e], b, blk, _SCALE_CODES[sk], g
+
+
+def dequant_block_scaled_f32(w, scales, global_scale, N, K, fmt, rows=None, threads=1):
+    """fp32 dequantized weights of a Track-1 format (the exact value rounded
+    once); ``global_scale`` only for NVFP4."""
+    out = np.zeros((N, K), dtype=np.float32)
+    el, b, blk, sk, ug = _track1(fmt)
+    g = float(global_scale) if ug else 1.0
+    L = lib()
+    fn = lambda a, c: L.oracle_dequant_block_scaled_f32(_ptr(w), _ptr(scales), int(ug), g, _ptr(out), N, K,
+                                                        el, b, blk, sk, a, c)
+    _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
+    return out
+
+
+def qmv_block_scaled(x, w, scales, global_scale, M, N, K, fmt, dtype, rows=None, threads=1):
+    """y = x . w_hat^T for a Track-1 format, fp64: returns (y, absdot), both
+    float64 [M, N]; rows not requested stay NaN."""
+    y = np.full((M, N), np.nan); a = np.full((M, N), np.nan)
+    el, b, blk, sk, ug = _track1(fmt)
+    g = float(global_scale) if ug else 1.0
+    L = lib()
+    fn = lambda r0, r1: L.oracle_qmv_block_scaled(_ptr(x), _ptr(w), _ptr(scales), int(ug), g, _ptr(y), _ptr(a),
+                                                  M, N, K, el, b, blk, sk, DTYPE_CODES[dtype], r0, r1)
+    _run(fn, _ranges(range(N) if rows is None else rows, threads), threads)
+    return y, a
 
 
 # ---- the product --------------------------------------------------------------

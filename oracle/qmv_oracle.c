@@ -16,7 +16,9 @@
  *    coverage", Track 1 table and the E2M1 / E4M3 / E8M0 codec notes:
  *    MXFP4 = E2M1 x E8M0 per 32, NVFP4 = E2M1 x E4M3 per 16 x FP32 global,
  *    MXFP8 = E4M3 x E8M0 per 32; E4M3 has 3 mantissa bits, exponent bias 7,
- *    max 448 and an explicit NaN code.
+ *    max 448 and an explicit NaN code; the rest of the Track 1 table (E5M2,
+ *    NVFP8, the FP32-scale legacy formats, the symmetric int / mxint
+ *    family and the FP16-scale twins) in oracle_qmv_block_scaled.
  *  - MLX pull request "affine_qmv_fast_rows / fp_qmv_fast_rows", description:
  *    the sum(x) bias term is formed from values widened before accumulation.
  *    The oracle has no such issue: it evaluates every product and sum in fp64.
@@ -284,6 +286,106 @@ void oracle_qmv_fp(const void* x, const uint8_t* w, const uint8_t* scales, float
             for (long long k = 0; k < K; ++k) {
                 double t = load_elem(x, (size_t)(m * K + k), dtype) *
                            fp_w(w, scales, (double)global, n, k, K, mode);
+                acc += t;
+                aacc += fabs(t);
+            }
+            y[m * N + n] = acc;
+            if (absdot) absdot[m * N + n] = aacc;
+        }
+}
+
+/* ---------------------------------------------------------------------------
+ * The Track-1 symmetric block-scaled formats (wh-iron kernel-op coverage
+ * audit, "Quantization precision coverage": the three axes element / scale /
+ * zero point, the Track 1 table, and the paragraph under it).  A weight
+ * [N, K] is cut along K into contiguous blocks; every element is a code,
+ * every block has one scale, there is no zero point, and the weight is
+ *     w_hat[n, k] = element(code[n, k]) * scale[n, k / block]  (* global),
+ * the tensor-wide FP32 global only for NVFP4.
+ *   element: E2M1, E4M3, E5M2, or a signed integer of 2..8 bits (the
+ *            audit's "signed integer ... float sign-extend": two's
+ *            complement, range -2^(b-1) .. 2^(b-1) - 1);
+ *   codes:   per row an LSB-first bit stream of b-bit codes, b the element
+ *            width (the audit: "tight-bit-pack LSB-first into u32 words", a
+ *            4-bit stream byte-identical to the nibble layout, 8-bit one byte
+ *            per code), read with oracle_affine_code;
+ *   scale:   E8M0 or E4M3 bytes, FP32 (4 B) or FP16 (2 B, the "*_f16"
+ *            twins), stored [N, K / block] row-major.
+ * ------------------------------------------------------------------------- */
+enum { OR_EL_E2M1 = 0, OR_EL_E4M3 = 1, OR_EL_E5M2 = 2, OR_EL_INT = 3 };
+enum { OR_SC_E8M0 = 0, OR_SC_E4M3 = 1, OR_SC_F32 = 2, OR_SC_F16 = 3 };
+
+/* E5M2: sign, 5 exponent bits (bias 15), 2 mantissa bits, with IEEE
+ * semantics: exponent field 0 is subnormal, 31 is infinity (mantissa 0) or
+ * NaN.  The audit's KV-cache row gives its largest finite value, 57344. */
+double oracle_e5m2(uint32_t c) {
+    c &= 0xFFu;
+    const double s = (c & 0x80u) ? -1.0 : 1.0;
+    const int e = (int)((c >> 2) & 31u), m = (int)(c & 3u);
+    if (e == 31) return m ? NAN : s * INFINITY;
+    if (e == 0) return s * ((double)m / 4.0) * ldexp(1.0, -14);
+    return s * (1.0 + (double)m / 4.0) * ldexp(1.0, e - 15);
+}
+
+/* Signed integer element of `bits` bits (2..8) from its raw field: two's
+ * complement, so a field with the top bit set is field - 2^bits. */
+double oracle_sint(uint32_t q, int bits) {
+    q &= (1u << bits) - 1u;
+    return (q >> (bits - 1)) ? (double)q - ldexp(1.0, bits) : (double)q;
+}
+
+/* Element k of a row. */
+static double bs_elem(const uint8_t* row, long long k, int elem, int bits) {
+    const uint32_t c = oracle_affine_code(row, k, bits);
+    switch (elem) {
+        case OR_EL_E2M1: return oracle_e2m1(c);
+        case OR_EL_E4M3: return oracle_e4m3(c);
+        case OR_EL_E5M2: return oracle_e5m2(c);
+        default: return oracle_sint(c, bits);
+    }
+}
+
+/* Block scale i of the scale array, widened exactly. */
+double oracle_block_scale(const void* s, long long i, int kind) {
+    switch (kind) {
+        case OR_SC_E8M0: return oracle_e8m0(((const uint8_t*)s)[i]);
+        case OR_SC_E4M3: return oracle_e4m3(((const uint8_t*)s)[i]);
+        case OR_SC_F32: { float f; memcpy(&f, (const char*)s + 4 * i, 4); return (double)f; }
+        default: { uint16_t h; memcpy(&h, (const char*)s + 2 * i, 2); return oracle_f16_value(h); }
+    }
+}
+
+/* Exact dequantized weight (fp64) of element (n, k).  Every product is exact:
+ * an element has at most 8 significant bits, an E8M0 / E4M3 / FP16 / FP32
+ * scale at most 24, and the NVFP4 global (24) meets an E2M1 x E4M3 product
+ * of at most 6. */
+static double bs_w(const uint8_t* w, const void* scales, int use_global, double global, long long n,
+                   long long k, long long K, int elem, int bits, int block, int kind) {
+    const uint8_t* row = w + n * (K * bits / 8);
+    const double v = bs_elem(row, k, elem, bits) * oracle_block_scale(scales, n * (K / block) + k / block, kind);
+    return use_global ? v * global : v;
+}
+
+/* fp32 dequantized Track-1 weights (the exact value, one rounding). */
+void oracle_dequant_block_scaled_f32(const uint8_t* w, const void* scales, int use_global, float global,
+                                     float* out, long long N, long long K, int elem, int bits, int block,
+                                     int kind, long long n0, long long n1) {
+    (void)N;
+    for (long long n = n0; n < n1; ++n)
+        for (long long k = 0; k < K; ++k)
+            out[n * K + k] = (float)bs_w(w, scales, use_global, (double)global, n, k, K, elem, bits, block, kind);
+}
+
+/* y[m, n] = sum_k x[m, k] * w_hat[n, k] in fp64 (and absdot), rows [n0, n1). */
+void oracle_qmv_block_scaled(const void* x, const uint8_t* w, const void* scales, int use_global, float global,
+                             double* y, double* absdot, long long M, long long N, long long K, int elem,
+                             int bits, int block, int kind, int dtype, long long n0, long long n1) {
+    for (long long n = n0; n < n1; ++n)
+        for (long long m = 0; m < M; ++m) {
+            double acc = 0.0, aacc = 0.0;
+            for (long long k = 0; k < K; ++k) {
+                double t = load_elem(x, (size_t)(m * K + k), dtype) *
+                           bs_w(w, scales, use_global, (double)global, n, k, K, elem, bits, block, kind);
                 acc += t;
                 aacc += fabs(t);
             }

@@ -15,6 +15,12 @@ Distributions (from the workload descriptions the tests and bench cover):
            min/max quantizer gives for zero-mean weights.
   FP:      E8M0 block exponents ~ U{118..130}; NVFP4 block scales are positive,
            non-zero, non-NaN E4M3 bytes (0x01..0x7E); NVFP4 global ~ U(0.5, 2).
+  Track-1 block-scaled (bs_case): codes are uniform random bytes for E2M1 and
+           the signed integers, uniform over the 254 non-NaN bytes for E4M3
+           and over the 248 finite bytes for E5M2 (exponent field not all
+           ones); E8M0 and E4M3 scales as above; FP32 / FP16 scales ~
+           U(0.005, 0.02) (rounded to f16 for the FP16 twins), or a caller's
+           range.
 """
 from __future__ import annotations
 
@@ -118,4 +124,44 @@ def fp_case(M, N, K, mode, dtype, seed, batch=1, precision=False):
     return {
         "x": to_storage(x, dtype), "w": np.ascontiguousarray(w, dtype=np.uint8), "scales": sc,
         "global": glob, "M": M, "N": N, "K": K, "mode": mode, "dtype": dtype, "batch": batch,
+    }
+
+
+# E5M2 bytes whose exponent field (bits 2..6) is not all ones: the finite codes
+_E5M2_FINITE = np.array([c for c in range(256) if (c & 0x7C) != 0x7C], dtype=np.uint8)
+_SCALE_BYTES = {"e8m0": 1, "e4m3": 1, "f32": 4, "f16": 2}
+
+
+def bs_case(M, N, K, elem, bits, block, scale, use_global, dtype, seed, batch=1, precision=False,
+            scale_range=(0.005, 0.02)):
+    """One Track-1 block-scaled problem, described by its layout: ``elem`` in
+    {"e2m1", "e4m3", "e5m2", "int"}, ``bits`` per code, ``block`` codes per
+    scale along K, ``scale`` in {"e8m0", "e4m3", "f32", "f16"}.  Returns w
+    [batch, N, K*bits/8] u8, scales [batch, N, K/block] as raw storage (u8,
+    float32 or uint16 f16 patterns), x raw storage of ``dtype``, and the
+    global (a float32 scalar when ``use_global``)."""
+    g = rng(seed)
+    x = g.uniform(1e-4, 1e-3, size=(batch, M, K)) if precision else g.standard_normal(size=(batch, M, K))
+    rb = K * bits // 8
+    if elem == "e4m3":
+        w = _E4M3_NON_NAN[g.integers(0, len(_E4M3_NON_NAN), size=(batch, N, rb))]
+    elif elem == "e5m2":
+        w = _E5M2_FINITE[g.integers(0, len(_E5M2_FINITE), size=(batch, N, rb))]
+    else:
+        w = random_bytes(g, (batch, N, rb))
+    shape = (batch, N, K // block)
+    if scale == "e8m0":
+        sc = g.integers(118, 131, size=shape, dtype=np.uint8)
+    elif scale == "e4m3":
+        sc = g.integers(0x01, 0x7F, size=shape, dtype=np.uint8)
+    elif scale == "f32":
+        sc = g.uniform(*scale_range, size=shape).astype(np.float32)
+    else:
+        sc = to_storage(g.uniform(*scale_range, size=shape), "f16")
+    glob = np.float32(g.uniform(0.5, 2.0)) if use_global else None
+    return {
+        "x": to_storage(x, dtype), "w": np.ascontiguousarray(w, dtype=np.uint8), "scales": np.ascontiguousarray(sc),
+        "global": glob, "M": M, "N": N, "K": K, "dtype": dtype, "batch": batch,
+        "elem": elem, "bits": bits, "block": block, "scale": scale, "use_global": use_global,
+        "scale_bytes": _SCALE_BYTES[scale],
     }
