@@ -58,6 +58,28 @@ typedef enum { QMV_F32 = 0, QMV_F16 = 1, QMV_BF16 = 2 } qmv_dtype;
 
 typedef enum { QMV_MXFP4 = 0, QMV_NVFP4 = 1, QMV_MXFP8_E4M3 = 2 } qmv_fp_mode;
 
+/* The symmetric block-scaled formats of the wh-iron kernel-op coverage audit,
+ * section "Quantization precision coverage", Track 1 table (30 formats):
+ * element / block along K / block-scale type (/ global).
+ *   NVFP4  E2M1 / 16 / E4M3 / FP32 global    MXFP4  E2M1 / 32 / E8M0
+ *   MXFP8_E4M3  E4M3 / 32 / E8M0            MXFP8_E5M2  E5M2 / 32 / E8M0
+ *   NVFP8  E4M3 / 16 / FP32                 FP4 (legacy) E2M1 / 32 / FP32
+ *   FP8_E4M3 (legacy) E4M3 / 32 / FP32      FP8_E5M2 (legacy) E5M2 / 32 / FP32
+ *   INTb   signed b-bit / 64 / FP32         MXINTb signed b-bit / 32 / E8M0
+ *   *_F16  the FP32-scaled formats above with an IEEE binary16 scale. */
+typedef enum {
+    QMV_FMT_NVFP4 = 0, QMV_FMT_MXFP4 = 1, QMV_FMT_MXFP8_E4M3 = 2, QMV_FMT_MXFP8_E5M2 = 3,
+    QMV_FMT_NVFP8 = 4, QMV_FMT_FP4 = 5, QMV_FMT_FP8_E4M3 = 6, QMV_FMT_FP8_E5M2 = 7,
+    QMV_FMT_INT2 = 8, QMV_FMT_INT3 = 9, QMV_FMT_INT4 = 10, QMV_FMT_INT5 = 11, QMV_FMT_INT6 = 12,
+    QMV_FMT_INT8 = 13,
+    QMV_FMT_MXINT2 = 14, QMV_FMT_MXINT3 = 15, QMV_FMT_MXINT4 = 16, QMV_FMT_MXINT5 = 17,
+    QMV_FMT_MXINT6 = 18, QMV_FMT_MXINT8 = 19,
+    QMV_FMT_NVFP8_F16 = 20, QMV_FMT_FP4_F16 = 21, QMV_FMT_FP8_E4M3_F16 = 22, QMV_FMT_FP8_E5M2_F16 = 23,
+    QMV_FMT_INT2_F16 = 24, QMV_FMT_INT3_F16 = 25, QMV_FMT_INT4_F16 = 26, QMV_FMT_INT5_F16 = 27,
+    QMV_FMT_INT6_F16 = 28, QMV_FMT_INT8_F16 = 29,
+    QMV_FMT_COUNT = 30
+} qmv_format;
+
 typedef enum {
     QMV_OK = 0,
     QMV_EINVAL = -1,        /* bad size, null pointer, K not a multiple of the group/block */
@@ -103,7 +125,7 @@ int qmv_affine_batched(const void* x, const void* w_packed, const void* scales,
  *                        scales [N, K/32] E8M0 bytes; K % 32 == 0
  *   mode QMV_NVFP4:      w_packed [N, K/2] E2M1 codes, scales [N, K/16] E4M3 bytes,
  *                        global_scale: DEVICE pointer to one float (required);
- *                        K % 16 == 0 (K % 32 == 0 for this implementation)
+ *                        K % 16 == 0 (a 16-code tail block when K % 32 == 16)
  *   mode QMV_MXFP8_E4M3: w_packed [N, K] E4M3 codes, scales [N, K/32] E8M0 bytes;
  *                        K % 32 == 0
  *   global_scale must be NULL for the MX modes.
@@ -119,6 +141,48 @@ int qmv_fp(const void* x, const void* w_packed, const void* scales, const float*
 int qmv_fp_batched(const void* x, const void* w_packed, const void* scales,
                    const float* global_scale, void* y, int M, int N, int K, int mode,
                    int dtype, int batch, int x_batched, void* stream);
+
+/*
+ * qmv_block_scaled -- qmv for any Track-1 format (qmv_format above; wh-iron
+ * kernel-op coverage audit, "Quantization precision coverage").
+ *   w_packed  [N, K*b/8] bytes, b = 4 (E2M1), 8 (E4M3 / E5M2) or the int width;
+ *             each row an LSB-first stream of b-bit codes (4-bit: low nibble =
+ *             even k; 8-bit: one byte per code; signed ints two's complement);
+ *             4-byte alignment required, 16 enables 16-byte loads
+ *   scales    [N, K/block] of the format's scale type: E8M0 / E4M3 bytes,
+ *             float (4-byte aligned) or IEEE half (2-byte aligned)
+ *   global_scale  NVFP4 only: DEVICE pointer to one float (required); NULL for
+ *             every other format
+ *   K % block == 0 (so K % 32 == 16 is valid for the 16-blocks: NVFP4, NVFP8);
+ *   1 <= M <= 8 (0 a no-op); x and y dtype elements as in qmv_affine.
+ * Output: sum over blocks of  scale_blk * sum_{k in blk} x[m,k] * elem[n,k]
+ * (times the global for NVFP4), fp32 accumulation, one rounding to dtype.
+ * Signed ints are read as offset binary q + 2^(b-1) with the bias term
+ * -2^(b-1) * scale * sum(x) (sum(x) widened per element).  NaN and infinite
+ * codes (E4M3 0x7F/0xFF, E5M2 exponent 31, E8M0 0xFF) propagate.
+ * Errors: format outside qmv_format -> QMV_EUNSUPPORTED; K % block, a missing
+ * or extra global_scale, null pointers -> QMV_EINVAL; misaligned w_packed or
+ * scales -> QMV_EALIGN.
+ */
+int qmv_block_scaled(const void* x, const void* w_packed, const void* scales, const float* global_scale,
+                     void* y, int M, int N, int K, int format, int dtype, void* stream);
+
+/* qmv_block_scaled_batched -- batched form; layouts as in qmv_affine_batched
+ * (for NVFP4 global_scale points to `batch` floats). */
+int qmv_block_scaled_batched(const void* x, const void* w_packed, const void* scales,
+                             const float* global_scale, void* y, int M, int N, int K, int format,
+                             int dtype, int batch, int x_batched, void* stream);
+
+/* qmv_dequant_block_scaled_f32 -- check kernel: w_out [N, K] fp32 (16-byte
+ * aligned) = element * scale rounded once (NVFP4: (element * E4M3) * global). */
+int qmv_dequant_block_scaled_f32(const void* w_packed, const void* scales, const float* global_scale,
+                                 float* w_out, int N, int K, int format, void* stream);
+
+/* qmv_format_info -- layout facts of a qmv_format, for sizing buffers: bits
+ * per code, codes per block scale, bytes per block scale, and whether a
+ * global scale is taken.  Any output pointer may be NULL.  Returns QMV_OK or
+ * QMV_EUNSUPPORTED. */
+int qmv_format_info(int format, int* element_bits, int* block, int* scale_bytes, int* has_global);
 
 /*
  * qmv_quantize_affine -- affine quantizer (wh-iron kernel-op coverage audit,
@@ -372,7 +436,8 @@ int qmv_last_cuda_error(void);
 /*
  * qmv_describe_plan -- the launch the picker would choose for these sizes,
  * written as text into buf (at most buflen bytes, NUL-terminated).  `family`
- * is 0 for affine (bits, group_size used) or 1 + qmv_fp_mode.  M up to 8 is
+ * is 0 for affine (bits, group_size used), 1 + qmv_fp_mode, or 100 + a
+ * qmv_format (bits and group_size ignored).  M up to 8 is
  * qmv's plan; 9..64 (affine) is qmv_qmm_affine's ("path=umma ...", or
  * "path=chunked<rows> chunks=<n>" and the plan of one chunk).  Host-only; no CUDA call except
  * cached device-property and occupancy queries.  Returns QMV_OK or an

@@ -18,7 +18,8 @@ Distributions (from the workload descriptions the tests and bench cover):
   Track-1 block-scaled (bs_case): codes are uniform random bytes for E2M1 and
            the signed integers, uniform over the 254 non-NaN bytes for E4M3
            and over the 248 finite bytes for E5M2 (exponent field not all
-           ones); E8M0 and E4M3 scales as above; FP32 / FP16 scales ~
+           ones); E8M0 and E4M3 scales as above (E8M0 ~ U{111..123} for E5M2
+           elements, whose range is 2^7 wider); FP32 / FP16 scales ~
            U(0.005, 0.02) (rounded to f16 for the FP16 twins), or a caller's
            range.
 """
@@ -151,7 +152,10 @@ def bs_case(M, N, K, elem, bits, block, scale, use_global, dtype, seed, batch=1,
         w = random_bytes(g, (batch, N, rb))
     shape = (batch, N, K // block)
     if scale == "e8m0":
-        sc = g.integers(118, 131, size=shape, dtype=np.uint8)
+        # E5M2 reaches 2^7 further than E4M3 (57344 vs 448): its exponents sit
+        # 7 lower so the weights span the same magnitudes as MXFP8-E4M3's
+        lo = 111 if elem == "e5m2" else 118
+        sc = g.integers(lo, lo + 13, size=shape, dtype=np.uint8)
     elif scale == "e4m3":
         sc = g.integers(0x01, 0x7F, size=shape, dtype=np.uint8)
     elif scale == "f32":

@@ -109,8 +109,65 @@ def test_fp_validation():
     assert fp(mode=0, K=48) == EINVAL
     assert fp(mode=2, K=40) == EINVAL
     assert fp(mode=1, gs=FAKE, K=40) == EINVAL     # not a multiple of the 16 block
-    assert fp(mode=1, gs=FAKE, K=48) == EUNSUP     # 16-code tail block not implemented
     assert fp(mode=1, gs=FAKE + 2) == EALIGN
+    # (K = 48 is a valid NVFP4 shape, with a 16-code tail block: the GPU tests run it)
+
+
+def bs(**kw):
+    a = dict(x=FAKE, w=FAKE, s=FAKE, gs=None, y=FAKE, M=1, N=8, K=128, fmt=4, dt=2, st=None)
+    a.update(kw)
+    return L.qmv_block_scaled(a["x"], a["w"], a["s"], a["gs"], a["y"], a["M"], a["N"], a["K"], a["fmt"], a["dt"],
+                              a["st"])
+
+
+def test_block_scaled_validation_before_any_launch():
+    F = q.FORMATS
+    assert bs(fmt=-1) == EUNSUP and bs(fmt=30) == EUNSUP
+    assert bs(fmt=F["nvfp4"]) == EINVAL                  # NVFP4 needs its global
+    assert bs(fmt=F["nvfp4"], gs=FAKE + 2) == EALIGN
+    assert bs(fmt=F["nvfp8"], gs=FAKE) == EINVAL         # no global for the rest
+    assert bs(fmt=F["nvfp8"], K=40) == EINVAL            # not a multiple of the 16 block
+    assert bs(fmt=F["fp4"], K=48) == EINVAL              # blocks of 32
+    assert bs(fmt=F["int4"], K=96) == EINVAL             # groups of 64
+    assert bs(fmt=F["nvfp8"], s=FAKE + 2) == EALIGN      # FP32 scales
+    assert bs(fmt=F["int4_f16"], s=FAKE + 1) == EALIGN   # FP16 scales
+    assert bs(fmt=F["int8"], w=FAKE + 2) == EALIGN
+    assert bs(fmt=F["int3"], M=9) == EUNSUP
+    assert bs(fmt=F["mxint5"], x=None) == EINVAL
+    assert bs(fmt=F["fp8_e5m2"], M=0) == 0 and bs(fmt=F["fp8_e5m2"], N=0) == 0
+    assert L.qmv_block_scaled_batched(FAKE, FAKE, FAKE, None, FAKE, 1, 8, 128, 4, 2, 0, 1, None) == EINVAL
+    out = FAKE
+    assert L.qmv_dequant_block_scaled_f32(FAKE, FAKE, None, out + 4, 8, 128, 4, None) == EALIGN
+    assert L.qmv_dequant_block_scaled_f32(FAKE, FAKE, None, out, 8, 128, 31, None) == EUNSUP
+    assert L.qmv_dequant_block_scaled_f32(FAKE, FAKE, None, out, 0, 128, 4, None) == 0
+
+
+def test_format_info_of_every_format():
+    """The C table against the pages' Track-1 layout: bits per code, block,
+    scale bytes, global."""
+    want = {"nvfp4": (4, 16, 1, True), "mxfp4": (4, 32, 1, False), "mxfp8_e4m3": (8, 32, 1, False),
+            "mxfp8_e5m2": (8, 32, 1, False), "nvfp8": (8, 16, 4, False), "fp4": (4, 32, 4, False),
+            "fp8_e4m3": (8, 32, 4, False), "fp8_e5m2": (8, 32, 4, False), "nvfp8_f16": (8, 16, 2, False),
+            "fp4_f16": (4, 32, 2, False), "fp8_e4m3_f16": (8, 32, 2, False), "fp8_e5m2_f16": (8, 32, 2, False)}
+    for b in (2, 3, 4, 5, 6, 8):
+        want[f"int{b}"] = (b, 64, 4, False)
+        want[f"mxint{b}"] = (b, 32, 1, False)
+        want[f"int{b}_f16"] = (b, 64, 2, False)
+    assert set(want) == set(q.FORMATS) and len(want) == 30
+    for name, (bits, blk, sb, g) in want.items():
+        assert q.qmv_format_info(name) == {"element_bits": bits, "block": blk, "scale_bytes": sb,
+                                          "has_global": g}, name
+    with pytest.raises(q.QmvError):
+        q.qmv_format_info(30)
+
+
+def test_block_scaled_plans():
+    """Every format plans on the few-rows or the row-tiled kernel, never on
+    the affine-only kernels."""
+    for name in q.FORMATS:
+        for (M, N, K) in [(1, 4, 1024), (1, 4096, 4096), (8, 14336, 4096)]:
+            plan = q.qmv_describe_plan(name, M, N, K, dtype="bf16")
+            assert plan.split()[0] in ("path=direct", "path=wide", "path=narrow"), (name, plan)
 
 
 def test_batched_validation():

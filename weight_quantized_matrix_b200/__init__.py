@@ -22,6 +22,8 @@ __all__ = [
     "qmv_qvm_workspace_bytes", "qmv_qvm_affine_noalloc", "qmv_status_string",
     "qmv_last_cuda_error",
     "qmv_describe_plan", "qmv_force_config", "DTYPES", "FP_MODES", "LIB_PATH", "lib",
+    "qmv_block_scaled", "qmv_block_scaled_batched", "qmv_dequant_block_scaled_f32", "qmv_format_info",
+    "FORMATS",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,6 +31,12 @@ LIB_PATH = os.path.join(_HERE, "lib", "libqmv.so")
 
 DTYPES = {"f32": 0, "f16": 1, "bf16": 2}
 FP_MODES = {"mxfp4": 0, "nvfp4": 1, "mxfp8": 2}
+# qmv_format of include/qmv.h: the Track-1 formats by the names of the wh-iron
+# audit's table ("Quantization precision coverage")
+FORMATS = {name: i for i, name in enumerate(
+    ["nvfp4", "mxfp4", "mxfp8_e4m3", "mxfp8_e5m2", "nvfp8", "fp4", "fp8_e4m3", "fp8_e5m2"]
+    + [f"int{b}" for b in (2, 3, 4, 5, 6, 8)] + [f"mxint{b}" for b in (2, 3, 4, 5, 6, 8)]
+    + ["nvfp8_f16", "fp4_f16", "fp8_e4m3_f16", "fp8_e5m2_f16"] + [f"int{b}_f16" for b in (2, 3, 4, 5, 6, 8)])}
 STATUS = {0: "QMV_OK", -1: "QMV_EINVAL", -2: "QMV_EUNSUPPORTED", -3: "QMV_EALIGN", -4: "QMV_ECUDA"}
 
 if not os.path.exists(LIB_PATH):
@@ -75,6 +83,10 @@ _lib.qmv_status_string.argtypes = [_i]
 _lib.qmv_status_string.restype = ctypes.c_char_p
 _lib.qmv_last_cuda_error.argtypes = []
 _lib.qmv_describe_plan.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, ctypes.c_char_p, _i]
+_lib.qmv_block_scaled.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p]
+_lib.qmv_block_scaled_batched.argtypes = [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p]
+_lib.qmv_dequant_block_scaled_f32.argtypes = [_p, _p, _p, _p, _i, _i, _i, _p]
+_lib.qmv_format_info.argtypes = [_i] + [ctypes.POINTER(ctypes.c_int)] * 4
 _lib.qmv_device_fault.argtypes = [ctypes.POINTER(ctypes.c_uint), _i]
 _lib.qmv_force_config.argtypes = [_i, _i, _i, _i]
 _lib.qmv_force_config.restype = None
@@ -118,6 +130,10 @@ def _dtype(d):
 
 def _mode(m):
     return m if isinstance(m, int) else FP_MODES[m]
+
+
+def _format(f):
+    return f if isinstance(f, int) else FORMATS[f]
 
 
 _raw_stream = None
@@ -169,6 +185,36 @@ def qmv_fp_batched(x, w_packed, scales, global_scale, y, M, N, K, mode, dtype, b
                    stream=None):
     _check(_fast.fp(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(global_scale), _ptr(y), M, N, K, _mode(mode),
                     _dtype(dtype), batch, int(bool(x_batched)), _stream(stream)), "qmv_fp_batched")
+
+
+def qmv_block_scaled(x, w_packed, scales, global_scale, y, M, N, K, fmt, dtype, stream=None):
+    """qmv for a Track-1 block-scaled format (name in FORMATS or a qmv_format
+    value); global_scale: a device float tensor for NVFP4, else None."""
+    st = _fast.block_scaled(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(global_scale), _ptr(y), M, N, K,
+                            _format(fmt), _dtype(dtype), 1, 1, _stream(stream))
+    if st:
+        raise QmvError(st, "qmv_block_scaled")
+
+
+def qmv_block_scaled_batched(x, w_packed, scales, global_scale, y, M, N, K, fmt, dtype, batch, x_batched=True,
+                             stream=None):
+    _check(_fast.block_scaled(_ptr(x), _ptr(w_packed), _ptr(scales), _ptr(global_scale), _ptr(y), M, N, K,
+                              _format(fmt), _dtype(dtype), batch, int(bool(x_batched)), _stream(stream)),
+           "qmv_block_scaled_batched")
+
+
+def qmv_dequant_block_scaled_f32(w_packed, scales, global_scale, w_out, N, K, fmt, stream=None):
+    _check(_lib.qmv_dequant_block_scaled_f32(_ptr(w_packed), _ptr(scales), _ptr(global_scale), _ptr(w_out), N, K,
+                                             _format(fmt), _stream(stream)), "qmv_dequant_block_scaled_f32")
+
+
+def qmv_format_info(fmt) -> dict:
+    """Layout of a Track-1 format: bits per code, block, bytes per scale, and
+    whether it takes a global scale."""
+    v = [ctypes.c_int(0) for _ in range(4)]
+    _check(_lib.qmv_format_info(_format(fmt), *[ctypes.byref(a) for a in v]), "qmv_format_info")
+    return {"element_bits": v[0].value, "block": v[1].value, "scale_bytes": v[2].value,
+            "has_global": bool(v[3].value)}
 
 
 def qmv_dequant_affine_f32(w_packed, scales, biases, w_out, N, K, bits, group_size, dtype, stream=None):
@@ -275,8 +321,14 @@ def qmv_affine_rms_norm(x, gamma, eps, w_packed, scales, biases, y, M, N, K, bit
 
 
 def qmv_describe_plan(family, M, N, K, bits=4, group_size=64, dtype="bf16", w_align16=True) -> str:
-    """Text of the launch the picker chooses; family 'affine' or an FP mode name."""
-    fam = 0 if family == "affine" else 1 + _mode(family)
+    """Text of the launch the picker chooses; family 'affine', an FP mode name
+    (qmv_fp) or a Track-1 format name (qmv_block_scaled)."""
+    if family == "affine":
+        fam = 0
+    elif family in FP_MODES:
+        fam = 1 + FP_MODES[family]
+    else:
+        fam = 100 + _format(family)
     buf = ctypes.create_string_buffer(256)
     _check(_lib.qmv_describe_plan(fam, M, N, K, bits, group_size, _dtype(dtype), int(w_align16), buf, 256),
            "qmv_describe_plan")

@@ -86,7 +86,8 @@ struct FmtInfo {
 };
 
 FmtInfo fmt_info(int fam, int bits) {
-    int b = fam == qmv::FAM_AFFINE ? bits : (fam == qmv::FAM_MXFP8 ? 8 : 4);
+    int b = (fam == qmv::FAM_AFFINE || fam == qmv::FAM_SINT) ? bits
+          : (fam == qmv::FAM_MXFP8 || fam == qmv::FAM_E4M3 || fam == qmv::FAM_E5M2) ? 8 : 4;
     int wu = b == 2 ? 4 : b == 3 ? 4 : b == 4 ? 2 : b == 5 ? 4 : b == 6 ? 2 : 1;
     return {fam, b, wu};
 }
@@ -503,7 +504,8 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     // and the fused RMSNorm run on the row-tiled CUDA-core kernel only
     if (pair || qkv || norm) gather = true;
     const FmtInfo fi = fmt_info(fam, bits);
-    const bool aff = fam == qmv::FAM_AFFINE;
+    const bool aff = fam == qmv::FAM_AFFINE;                 // the affine-only kernels
+    const bool affl = aff || fam == qmv::FAM_SINT;           // sum(x) staged with x
     int maxm = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
     const int c_wide = 32 * fi.wide_units;
     bool wide = w16 && (K % c_wide == 0);
@@ -638,7 +640,7 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     // x tile: shrink the k-warps until one iteration of x fits the budget
     const size_t budget = 96 * 1024;
     auto per_iter_of = [&](int wk_) {
-        return (size_t)maxm * C * 32 * wk_ * 4 + (aff ? (size_t)maxm * U * 32 * wk_ * 4 : 0);
+        return (size_t)maxm * C * 32 * wk_ * 4 + (affl ? (size_t)maxm * U * 32 * wk_ * 4 : 0);
     };
     while (wk > 1 && per_iter_of(wk) > budget) --wk;
     const int KT = 32 * wk;
@@ -756,8 +758,9 @@ bool encode_scale_map(CUtensorMap* m, const void* base, int dtype, long long KG,
 
 int run(int fam, const void* x, const void* w, const void* scales, const void* biases,
         const float* gscale, void* y, int M, int N, int K, int bits, int G, int dtype, int batch,
-        int x_batched, void* stream, const int* ids = nullptr, int n_experts = 0, bool qmm = false) {
-    const long long row_bytes = (long long)K * (fam == qmv::FAM_AFFINE ? bits : (fam == qmv::FAM_MXFP8 ? 8 : 4)) / 8;
+        int x_batched, void* stream, const int* ids = nullptr, int n_experts = 0, bool qmm = false,
+        int skind = 0) {
+    const long long row_bytes = (long long)K * fmt_info(fam, bits).bits / 8;
     Plan pl;
     const bool w16 = aligned(w, 16);
     const bool s16 = fam == qmv::FAM_AFFINE && aligned(scales, 16) && aligned(biases, 16);
@@ -808,6 +811,7 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     p.ids = ids;
     p.n_experts = n_experts;
     p.gamma = nullptr; p.eps = 0.f;
+    p.skind = skind;
     cudaError_t e;
     p.sps = pl.sps; p.pitch = pl.pitch; p.fault = nullptr;
     p.sring = pl.sring; p.soff = pl.soff; p.boff = pl.boff; p.sbw = pl.sbw;
@@ -840,6 +844,8 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
             case 8: e = qmv::launch_affine_b8(dtype, pl.maxm, pl.R, pl.wide, p, L); break;
             default: return QMV_EUNSUPPORTED;
         }
+    } else if (fam == qmv::FAM_SINT) {
+        e = qmv::launch_sint(bits, dtype, pl.maxm, pl.R, pl.wide, p, L);
     } else {
         e = qmv::launch_fp(fam, dtype, pl.maxm, pl.R, pl.wide, p, L);
     }
@@ -973,13 +979,53 @@ int check_fp(int mode, int K, const float* gscale) {
     if (fam < 0) return QMV_EUNSUPPORTED;
     if (mode == QMV_NVFP4) {
         if (K % 16 != 0) return QMV_EINVAL;
-        if (K % 32 != 0) return QMV_EUNSUPPORTED;   // 16-code tail blocks not implemented
         if (!gscale) return QMV_EINVAL;
         if (!aligned(gscale, 4)) return QMV_EALIGN;
     } else {
         if (K % 32 != 0) return QMV_EINVAL;
         if (gscale) return QMV_EINVAL;
     }
+    return QMV_OK;
+}
+
+// The Track-1 formats (qmv_format): kernel family, bits per code, block,
+// scale type, global scale.  The three formats of qmv_fp keep their own
+// families; the rest run on the run-time-scaled E2M1 / E4M3 / E5M2 families
+// or on the signed-integer family.
+struct BsFmt {
+    int fam, bits, block, skind, global;
+};
+constexpr int kSF32 = qmv::SK_F32, kSF16 = qmv::SK_F16, kSE8 = qmv::SK_E8M0, kSE4 = qmv::SK_E4M3;
+const BsFmt kBsFmt[QMV_FMT_COUNT] = {
+    {qmv::FAM_NVFP4, 4, 16, kSE4, 1}, {qmv::FAM_MXFP4, 4, 32, kSE8, 0},
+    {qmv::FAM_MXFP8, 8, 32, kSE8, 0}, {qmv::FAM_E5M2, 8, 32, kSE8, 0},
+    {qmv::FAM_E4M3, 8, 16, kSF32, 0}, {qmv::FAM_E2M1, 4, 32, kSF32, 0},
+    {qmv::FAM_E4M3, 8, 32, kSF32, 0}, {qmv::FAM_E5M2, 8, 32, kSF32, 0},
+    {qmv::FAM_SINT, 2, 64, kSF32, 0}, {qmv::FAM_SINT, 3, 64, kSF32, 0}, {qmv::FAM_SINT, 4, 64, kSF32, 0},
+    {qmv::FAM_SINT, 5, 64, kSF32, 0}, {qmv::FAM_SINT, 6, 64, kSF32, 0}, {qmv::FAM_SINT, 8, 64, kSF32, 0},
+    {qmv::FAM_SINT, 2, 32, kSE8, 0}, {qmv::FAM_SINT, 3, 32, kSE8, 0}, {qmv::FAM_SINT, 4, 32, kSE8, 0},
+    {qmv::FAM_SINT, 5, 32, kSE8, 0}, {qmv::FAM_SINT, 6, 32, kSE8, 0}, {qmv::FAM_SINT, 8, 32, kSE8, 0},
+    {qmv::FAM_E4M3, 8, 16, kSF16, 0}, {qmv::FAM_E2M1, 4, 32, kSF16, 0},
+    {qmv::FAM_E4M3, 8, 32, kSF16, 0}, {qmv::FAM_E5M2, 8, 32, kSF16, 0},
+    {qmv::FAM_SINT, 2, 64, kSF16, 0}, {qmv::FAM_SINT, 3, 64, kSF16, 0}, {qmv::FAM_SINT, 4, 64, kSF16, 0},
+    {qmv::FAM_SINT, 5, 64, kSF16, 0}, {qmv::FAM_SINT, 6, 64, kSF16, 0}, {qmv::FAM_SINT, 8, 64, kSF16, 0},
+};
+
+int scale_bytes_of(int skind) { return skind == qmv::SK_F32 ? 4 : skind == qmv::SK_F16 ? 2 : 1; }
+
+// Argument checks shared by the block-scaled entries (format, K, global, scales).
+int check_bs(int format, int K, const void* scales, const float* gscale, const BsFmt** out) {
+    if (format < 0 || format >= QMV_FMT_COUNT) return QMV_EUNSUPPORTED;
+    const BsFmt& f = kBsFmt[format];
+    if (K % f.block != 0) return QMV_EINVAL;
+    if (f.global) {
+        if (!gscale) return QMV_EINVAL;
+        if (!aligned(gscale, 4)) return QMV_EALIGN;
+    } else if (gscale) {
+        return QMV_EINVAL;
+    }
+    if (scales && !aligned(scales, scale_bytes_of(f.skind))) return QMV_EALIGN;
+    *out = &f;
     return QMV_OK;
 }
 
@@ -1026,6 +1072,48 @@ int qmv_fp_batched(const void* x, const void* w_packed, const void* scales, cons
 int qmv_fp(const void* x, const void* w_packed, const void* scales, const float* global_scale, void* y,
            int M, int N, int K, int mode, int dtype, void* stream) {
     return qmv_fp_batched(x, w_packed, scales, global_scale, y, M, N, K, mode, dtype, 1, 1, stream);
+}
+
+int qmv_block_scaled_batched(const void* x, const void* w_packed, const void* scales, const float* global_scale,
+                             void* y, int M, int N, int K, int format, int dtype, int batch, int x_batched,
+                             void* stream) {
+    const BsFmt* f = nullptr;
+    int st = check_bs(format, K, scales, global_scale, &f);
+    if (st != QMV_OK) return st;
+    if (batch < 1 || batch > 65535 || (x_batched != 0 && x_batched != 1)) return QMV_EINVAL;
+    st = check_common(x, w_packed, scales, y, M, N, K, dtype);
+    if (st != QMV_OK || M == 0 || N == 0) return st;
+    return run(f->fam, x, w_packed, scales, nullptr, global_scale, y, M, N, K, f->bits, f->block, dtype, batch,
+               x_batched, stream, nullptr, 0, false, f->skind);
+}
+
+int qmv_block_scaled(const void* x, const void* w_packed, const void* scales, const float* global_scale, void* y,
+                     int M, int N, int K, int format, int dtype, void* stream) {
+    return qmv_block_scaled_batched(x, w_packed, scales, global_scale, y, M, N, K, format, dtype, 1, 1, stream);
+}
+
+int qmv_dequant_block_scaled_f32(const void* w_packed, const void* scales, const float* global_scale,
+                                 float* w_out, int N, int K, int format, void* stream) {
+    const BsFmt* f = nullptr;
+    int st = check_bs(format, K, scales, global_scale, &f);
+    if (st != QMV_OK) return st;
+    if (N < 0 || K < 0) return QMV_EINVAL;
+    if (N == 0 || K == 0) return QMV_OK;
+    if (!w_packed || !scales || !w_out) return QMV_EINVAL;
+    if (!aligned(w_packed, 4) || !aligned(w_out, 16)) return QMV_EALIGN;
+    return finish(qmv::launch_dequant(f->fam, f->bits, 0, static_cast<const uint8_t*>(w_packed), scales, nullptr,
+                                      global_scale, w_out, N, K, f->block, (long long)K * f->bits / 8,
+                                      static_cast<cudaStream_t>(stream), f->skind));
+}
+
+int qmv_format_info(int format, int* element_bits, int* block, int* scale_bytes, int* has_global) {
+    if (format < 0 || format >= QMV_FMT_COUNT) return QMV_EUNSUPPORTED;
+    const BsFmt& f = kBsFmt[format];
+    if (element_bits) *element_bits = f.bits;
+    if (block) *block = f.block;
+    if (scale_bytes) *scale_bytes = scale_bytes_of(f.skind);
+    if (has_global) *has_global = f.global;
+    return QMV_OK;
 }
 
 int qmv_dequant_affine_f32(const void* w_packed, const void* scales, const void* biases, float* w_out,
@@ -1251,20 +1339,26 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
                       char* buf, int buflen) {
     if (!buf || buflen <= 0) return QMV_EINVAL;
     if (M < 1 || M > QMV_QMM_MAX_M || N < 1 || K < 0) return QMV_EINVAL;
-    int fam;
+    int fam, G;
     if (family == 0) {
         if (check_affine(bits, group_size) != QMV_OK) return QMV_EUNSUPPORTED;
         fam = qmv::FAM_AFFINE;
+        G = group_size;
+    } else if (family >= 100) {
+        if (family - 100 >= QMV_FMT_COUNT) return QMV_EUNSUPPORTED;
+        const BsFmt& f = kBsFmt[family - 100];
+        fam = f.fam; bits = f.bits; G = f.block;
     } else {
         fam = fp_family(family - 1);
         if (fam < 0) return QMV_EUNSUPPORTED;
         bits = 0;
+        G = family == 2 ? 16 : 32;
     }
     Plan pl;
     const bool qmm = M > QMV_MAX_M;
     if (qmm && fam != qmv::FAM_AFFINE) return QMV_EINVAL;
-    int st = make_plan(fam, M, N, K, bits, fam == qmv::FAM_AFFINE ? group_size : (family == 2 ? 16 : 32), dtype,
-                       w_align16 != 0, 1, &pl, true, false, false, true, qmm && qmm_prefers_umma(N));
+    int st = make_plan(fam, M, N, K, bits, G, dtype, w_align16 != 0, 1, &pl, true, false, false, true,
+                       qmm && qmm_prefers_umma(N));
     if (st != QMV_OK) return st;
     if (qmm && pl.tc != 5) {
         // qmm: chunks of x rows, each through the qmv plan of its size

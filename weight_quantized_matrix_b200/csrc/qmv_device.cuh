@@ -7,7 +7,14 @@
 //           quantized_nax.h, get_pack_factor / get_bytes_per_pack, qdot),
 //           w = scale * q + bias per group of G codes;
 //   MXFP4 / NVFP4 / MXFP8: E2M1 or E4M3 elements with E8M0 (per 32) or E4M3
-//           (per 16, times an FP32 global) block scales (wh-iron audit, Track 1).
+//           (per 16, times an FP32 global) block scales (wh-iron audit, Track 1);
+//   the rest of the audit's Track 1 table: E2M1 / E4M3 / E5M2 elements with a
+//           block scale whose type (E8M0, E4M3, FP32 or FP16) and block (16 or
+//           32) are run-time parameters (FAM_E2M1 / FAM_E4M3 / FAM_E5M2), and
+//           the symmetric signed integers int2..int8 / mxint2..mxint8
+//           (FAM_SINT): two's-complement codes in the affine bit stream, read
+//           through the affine machinery after flipping every field's sign bit
+//           (offset binary, field + 2^(b-1)) with bias = -2^(b-1) * scale.
 //
 // Work decomposition (B200-first, not the pages' Metal layout):
 //   * The K axis of a row is cut into CHUNKS of C codes (C a multiple of 32).
@@ -51,7 +58,22 @@
 
 namespace qmv {
 
-enum Family { FAM_AFFINE = 0, FAM_MXFP4 = 1, FAM_NVFP4 = 2, FAM_MXFP8 = 3 };
+enum Family {
+    FAM_AFFINE = 0, FAM_MXFP4 = 1, FAM_NVFP4 = 2, FAM_MXFP8 = 3,
+    FAM_E2M1 = 4, FAM_E4M3 = 5, FAM_E5M2 = 6,     // block and scale type at run time
+    FAM_SINT = 7                                  // symmetric signed integers
+};
+// Block-scale storage of the run-time-scaled families (Params::skind).
+enum ScaleKind { SK_E8M0 = 0, SK_E4M3 = 1, SK_F32 = 2, SK_F16 = 3 };
+
+// Families read through the affine machinery (codes in the LSB-first bit
+// stream, fp32 sum(x) per unit, scale * partial + bias * sum(x)).
+template <int FAM> __host__ __device__ constexpr bool affine_like() { return FAM == FAM_AFFINE || FAM == FAM_SINT; }
+// Families with one scale per 16 codes possible: a 32-code unit keeps two
+// partial sums, one per half.
+template <int FAM> __host__ __device__ constexpr bool half_units() {
+    return FAM == FAM_NVFP4 || FAM == FAM_E2M1 || FAM == FAM_E4M3 || FAM == FAM_E5M2;
+}
 
 struct Params {
     const void* x;          // [batch?][M][K] dtype
@@ -106,6 +128,8 @@ struct Params {
     // scales x staged for the products by gamma[k] / sqrt(mean(x[m]^2) + eps).
     const void* gamma;
     float eps;
+    // Block-scale type of FAM_E2M1 / FAM_E4M3 / FAM_E5M2 / FAM_SINT (ScaleKind).
+    int skind;
 };
 
 // Row mapping of the row-tiled kernel: plain, the interleaved gate / up
@@ -256,9 +280,45 @@ __device__ __forceinline__ float e8m0_value(uint32_t e) {
          : e == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(e << 23);
 }
 
+// E5M2 byte -> float: exponent+mantissa bits at fp32 bits 21..27 form the
+// value times 2^-112 (subnormals included), restored by one exact multiply;
+// exponent field 31 is infinity (mantissa 0) or NaN.
+__device__ __forceinline__ float e5m2_value(uint32_t c) {
+    c &= 0xFFu;
+    const float v = __uint_as_float(((c & 0x7Fu) << 21) | ((c & 0x80u) << 24)) * 0x1p112f;
+    return ((c & 0x7Cu) == 0x7Cu)
+               ? __uint_as_float((c & 3u) ? 0x7FC00000u : (((c & 0x80u) << 24) | 0x7F800000u))
+               : v;
+}
+// 8-bit element of a family (E5M2 for FAM_E5M2, E4M3 otherwise).
+template <int FAM> __device__ __forceinline__ float fp8_value(uint32_t c) {
+    if constexpr (FAM == FAM_E5M2) return e5m2_value(c);
+    else return e4m3_value(c);
+}
+// Block scale i of a run-time-typed scale array.
+__device__ __forceinline__ float block_scale(const void* s, long long i, int kind) {
+    switch (kind) {
+        case SK_E8M0: return e8m0_value(__ldg(reinterpret_cast<const uint8_t*>(s) + i));
+        case SK_E4M3: return e4m3_value(__ldg(reinterpret_cast<const uint8_t*>(s) + i));
+        case SK_F32: return __ldg(reinterpret_cast<const float*>(s) + i);
+        default: return __half2float(__ldg(reinterpret_cast<const __half*>(s) + i));
+    }
+}
+// Signed-int codes: the bits of word wi of a B-word unit that are a field's
+// top (sign) bit.  XOR-ing them maps a two's-complement field q to the offset
+// binary q + 2^(B-1), a plain unsigned code.
+template <int B> __host__ __device__ constexpr uint32_t sint_sign_mask(int wi) {
+    uint32_t m = 0;
+    for (int j = 0; j < 32; ++j) {
+        const int b = B * j + B - 1;
+        if (b / 32 == wi) m |= 1u << (b % 32);
+    }
+    return m;
+}
+
 // ----------------------------------------------------------- format traits --
 template <int FAM, int BITS> struct Fmt {
-    static constexpr int kBits = (FAM == FAM_AFFINE) ? BITS : (FAM == FAM_MXFP8 ? 8 : 4);
+    static constexpr int kBits = affine_like<FAM>() ? BITS : ((FAM == FAM_MXFP8 || FAM == FAM_E4M3 || FAM == FAM_E5M2) ? 8 : 4);
     static constexpr int kUnitWords = kBits;                 // words per 32 codes
     // Units per chunk on the wide path: the smallest whole number of units
     // whose byte size is a multiple of 16 (and at least 32 bytes for 2/4-bit).
@@ -277,7 +337,7 @@ template <int FAM, int B, class T, int MAXM, int U>
 __device__ __forceinline__ void stage_x(const Params& p, const char* Xb, float4* xs, float* sx, int t0,
                                         int tcn, int KT, int TI, const float* rnorm = nullptr) {
     constexpr int C = 32 * U;
-    constexpr bool AFF = (FAM == FAM_AFFINE);
+    constexpr bool AFF = affine_like<FAM>();
     const int items = MAXM * tcn * U;
     for (int it = threadIdx.x; it < items; it += blockDim.x) {
         const int u = it % U;
@@ -340,7 +400,7 @@ __device__ __forceinline__ void stage_x(const Params& p, const char* Xb, float4*
 // Per-unit scales of chunk c for R rows (affine: scale + bias of the unit's
 // group; MX: one block scale; NV: two block scales per unit).  PAIR: row r is
 // virtual row rowc[r] of the interleaved gate / up pair (odd rows: up).
-template <int FAM, class T, int R, int U, int RMODE = RMODE_PLAIN>
+template <int FAM, int B, class T, int R, int U, int RMODE = RMODE_PLAIN>
 __device__ __forceinline__ void load_scales(const Params& p, const int (&rowc)[R], int c, long long sb,
                                             float (&sc)[R][U][2], float (&bi)[R][U]) {
     constexpr int C = 32 * U;
@@ -366,6 +426,17 @@ __device__ __forceinline__ void load_scales(const Params& p, const int (&rowc)[R
                 const long long gi = sb + rb + k0 / G;
                 sc[r][u][0] = DT<T>::ld(sp, gi);
                 bi[r][u] = DT<T>::ld(bp, gi);
+            } else if constexpr (FAM == FAM_SINT) {
+                // offset-binary codes: w = s * (q' - 2^(B-1)) = s * q' + bias
+                const float sv = block_scale(p.scales, sb + rb + k0 / G, p.skind);
+                sc[r][u][0] = sv;
+                sc[r][u][1] = 0.f;
+                bi[r][u] = -sv * (float)(1 << (B - 1));
+            } else if constexpr (FAM == FAM_E2M1 || FAM == FAM_E4M3 || FAM == FAM_E5M2) {
+                const long long si = sb + rb + k0 / G;
+                sc[r][u][0] = block_scale(p.scales, si, p.skind);
+                sc[r][u][1] = G == 16 ? block_scale(p.scales, si + 1, p.skind) : sc[r][u][0];
+                bi[r][u] = 0.f;
             } else if constexpr (FAM == FAM_NVFP4) {
                 const uint8_t* s8 = reinterpret_cast<const uint8_t*>(p.scales) + sb + rb + k0 / 16;
                 sc[r][u][0] = e4m3_value(__ldg(s8));
@@ -390,7 +461,7 @@ __device__ __forceinline__ void compute_chunk(const uint32_t (&wv)[R][B * U], co
                                               const float* sxb, size_t sxm, int KT, float (&acc)[R][MAXM],
                                               uint32_t kf32) {
     constexpr int UW = B;
-    constexpr bool AFF = (FAM == FAM_AFFINE);
+    constexpr bool AFF = affine_like<FAM>();
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         float2 part[R][MAXM][2];                  // NV: one per 16-code block
@@ -425,10 +496,10 @@ __device__ __forceinline__ void compute_chunk(const uint32_t (&wv)[R][B * U], co
                     d1 = mul2(make_float2(__uint_as_float(e2m1_pattern(wd >> 8)), __uint_as_float(e2m1_pattern(wd >> 12))), s126);
                 } else {
                     const uint32_t wd = wu[q];
-                    d0 = make_float2(e4m3_value(wd), e4m3_value(wd >> 8));
-                    d1 = make_float2(e4m3_value(wd >> 16), e4m3_value(wd >> 24));
+                    d0 = make_float2(fp8_value<FAM>(wd), fp8_value<FAM>(wd >> 8));
+                    d1 = make_float2(fp8_value<FAM>(wd >> 16), fp8_value<FAM>(wd >> 24));
                 }
-                const int h = (FAM == FAM_NVFP4) ? (q >> 2) : 0;   // 16-code block within the unit
+                const int h = half_units<FAM>() ? (q >> 2) : 0;    // 16-code half of the unit
 #pragma unroll
                 for (int m = 0; m < MAXM; ++m) {
                     float2 a = part[r][m][h];
@@ -446,7 +517,7 @@ __device__ __forceinline__ void compute_chunk(const uint32_t (&wv)[R][B * U], co
                     const float s = sxb[(size_t)m * sxm + (size_t)u * KT];
                     const float pr = part[r][m][0].x + part[r][m][0].y;
                     acc[r][m] = fmaf(sc[r][u][0], pr, fmaf(bi[r][u], s, acc[r][m]));
-                } else if constexpr (FAM == FAM_NVFP4) {
+                } else if constexpr (half_units<FAM>()) {
                     acc[r][m] = fmaf(sc[r][u][0], part[r][m][0].x + part[r][m][0].y, acc[r][m]);
                     acc[r][m] = fmaf(sc[r][u][1], part[r][m][1].x + part[r][m][1].y, acc[r][m]);
                 } else {
@@ -502,7 +573,7 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
     constexpr int U = WIDE ? F::kWideUnits : 1;
     constexpr int C = 32 * U;
     constexpr int CW = B * U;
-    constexpr bool AFF = (FAM == FAM_AFFINE);
+    constexpr bool AFF = affine_like<FAM>();
 
     extern __shared__ float4 smem4[];
     const int KT = 32 * p.wk;
@@ -576,8 +647,12 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
 #pragma unroll
                 for (int q = 0; q < CW; ++q) wv[r][q] = __ldg(reinterpret_cast<const uint32_t*>(src) + q);
             }
+            if constexpr (FAM == FAM_SINT) {
+#pragma unroll
+                for (int q = 0; q < CW; ++q) wv[r][q] ^= sint_sign_mask<B>(q % B);
+            }
         }
-        load_scales<FAM, T, R, U, RMODE>(p, rowc, c, sb, sc, bi);
+        load_scales<FAM, B, T, R, U, RMODE>(p, rowc, c, sb, sc, bi);
     };
 
     const uint32_t kf32 = p.kf32;
@@ -643,6 +718,28 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
         }
     }
 
+    if constexpr (half_units<FAM>()) {
+        // K % 32 == 16 (blocks of 16): the row's last 16 codes lie outside
+        // the 32-code units; the first k-warp's lanes 0..15 take one each
+        if ((p.K & 31) && wkid == 0 && lane < 16) {
+            const long long k = (long long)p.K - 16 + lane;
+            const T* Xt = reinterpret_cast<const T*>(Xb);
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const uint8_t* rp = W + (long long)rowc[r] * p.w_row;
+                float e;
+                if constexpr (B == 4) e = e2m1_value(__ldg(rp + (k >> 1)) >> (4 * (int)(k & 1)));
+                else e = fp8_value<FAM>(__ldg(rp + k));
+                const long long si = sb + (long long)rowc[r] * (p.K / p.G) + k / p.G;
+                const float sv = FAM == FAM_NVFP4 ? e4m3_value(__ldg(reinterpret_cast<const uint8_t*>(p.scales) + si))
+                                                  : block_scale(p.scales, si, p.skind);
+                const float ws = __fmul_rn(e, sv);
+#pragma unroll
+                for (int m = 0; m < MAXM; ++m)
+                    if (m < p.M) acc[r][m] = fmaf(DT<T>::ld(Xt, (long long)m * p.K + k), ws, acc[r][m]);
+            }
+        }
+    }
     warp_allreduce<R, MAXM>(acc);
     float gs = 1.f;
     if constexpr (FAM == FAM_NVFP4) gs = __ldg(p.gscale + be);
@@ -714,13 +811,32 @@ __global__ void __launch_bounds__(256) qmv_kernel(const Params p) {
 // ------------------------------------------------- dequantization check ----
 // One thread per 32-code unit of one row; writes 32 fp32 weights.
 //   affine: fmaf(scale, c, bias) with c = (c * 2^p) * 2^-p (exact)
+//   signed int: the same on the offset-binary codes with bias = -2^(b-1) *
+//           scale, i.e. the one rounding of scale * q
 //   MX:     elem * e8m0 (exact in fp32)
 //   NV:     (elem * e4m3) * global (the first product exact, one rounding)
+//   E2M1 / E4M3 / E5M2 with a typed block scale: elem * scale, one rounding
+// With K % 32 == 16 (blocks of 16) the last 16 codes of each row follow, one
+// thread each.
+template <int FAM, int B>
+__device__ __forceinline__ float fp_elem_at(const uint32_t* wv, int j) {
+    if constexpr (B == 4) return e2m1_value(wv[j / 8] >> (4 * (j % 8)));
+    else return fp8_value<FAM>(wv[j / 4] >> (8 * (j % 4)));
+}
+
+template <int FAM>
+__device__ __forceinline__ float fp_scale_at(const void* scales, const float* gscale, long long si, int skind) {
+    const uint8_t* s8 = reinterpret_cast<const uint8_t*>(scales);
+    if constexpr (FAM == FAM_NVFP4) return e4m3_value(__ldg(s8 + si));
+    else if constexpr (FAM == FAM_MXFP4 || FAM == FAM_MXFP8) return e8m0_value(__ldg(s8 + si));
+    else return block_scale(scales, si, skind);
+}
+
 template <int FAM, int BITS, class T>
 __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict__ w,
                                                       const void* scales, const void* biases,
                                                       const float* gscale, float* __restrict__ out,
-                                                      int N, int K, int G, long long w_row) {
+                                                      int N, int K, int G, long long w_row, int skind) {
     using F = Fmt<FAM, BITS>;
     constexpr int B = F::kBits;
     const long long units = (long long)N * (K / 32);
@@ -735,9 +851,18 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
         for (int q = 0; q < B; ++q) wv[q] = __ldg(src + q);
         float o[32];
         const long long k0 = (long long)u * 32;
-        if constexpr (FAM == FAM_AFFINE) {
+        if constexpr (affine_like<FAM>()) {
             const long long gi = n * (K / G) + k0 / G;
-            const float s = DT<T>::ld(scales, gi), b = DT<T>::ld(biases, gi);
+            float s, b;
+            if constexpr (FAM == FAM_SINT) {
+#pragma unroll
+                for (int q = 0; q < B; ++q) wv[q] ^= sint_sign_mask<B>(q);
+                s = block_scale(scales, gi, skind);
+                b = -s * (float)(1 << (B - 1));
+            } else {
+                s = DT<T>::ld(scales, gi);
+                b = DT<T>::ld(biases, gi);
+            }
 #define QMV_D4(QQ) { float2 d0 = magic_pair(field_bits<B, 4 * QQ>(wv), field_bits<B, 4 * QQ + 1>(wv)); \
                      float2 d1 = magic_pair(field_bits<B, 4 * QQ + 2>(wv), field_bits<B, 4 * QQ + 3>(wv)); \
                      float c[4] = {d0.x, d0.y, d1.x, d1.y}; \
@@ -746,26 +871,32 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
                          o[4 * QQ + e] = fmaf(s, q_, b); } }
             QMV_D4(0) QMV_D4(1) QMV_D4(2) QMV_D4(3) QMV_D4(4) QMV_D4(5) QMV_D4(6) QMV_D4(7)
 #undef QMV_D4
-        } else if constexpr (B == 4) {
-            const uint8_t* s8 = reinterpret_cast<const uint8_t*>(scales) + n * (K / G);
+        } else {
+            const long long sr = n * (K / G);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const float e = e2m1_value(wv[j / 8] >> (4 * (j % 8)));
-                if constexpr (FAM == FAM_NVFP4) {
-                    o[j] = __fmul_rn(__fmul_rn(e, e4m3_value(__ldg(s8 + (k0 + j) / 16))), __ldg(gscale));
-                } else {
-                    o[j] = __fmul_rn(e, e8m0_value(__ldg(s8 + (k0 + j) / 32)));
-                }
+                const float v = __fmul_rn(fp_elem_at<FAM, B>(wv, j), fp_scale_at<FAM>(scales, gscale, sr + (k0 + j) / G, skind));
+                o[j] = FAM == FAM_NVFP4 ? __fmul_rn(v, __ldg(gscale)) : v;
             }
-        } else {
-            const uint8_t* s8 = reinterpret_cast<const uint8_t*>(scales) + n * (K / G);
-            const float s = e8m0_value(__ldg(s8 + k0 / 32));
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __fmul_rn(e4m3_value(wv[j / 4] >> (8 * (j % 4))), s);
         }
         float4* dst = reinterpret_cast<float4*>(out + n * (long long)K + k0);
 #pragma unroll
         for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    }
+    if constexpr (half_units<FAM>()) {
+        if (K & 31) {
+            const long long tails = (long long)N * 16;
+            for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < tails;
+                 t += (long long)gridDim.x * blockDim.x) {
+                const long long n = t / 16, k = (long long)K - 16 + (t % 16);
+                const uint8_t* rp = w + n * w_row;
+                float e;
+                if constexpr (B == 4) e = e2m1_value(__ldg(rp + (k >> 1)) >> (4 * (int)(k & 1)));
+                else e = fp8_value<FAM>(__ldg(rp + k));
+                const float v = __fmul_rn(e, fp_scale_at<FAM>(scales, gscale, n * (K / G) + k / G, skind));
+                out[n * (long long)K + k] = FAM == FAM_NVFP4 ? __fmul_rn(v, __ldg(gscale)) : v;
+            }
+        }
     }
 }
 

@@ -11,6 +11,10 @@
 //   MXFP4/8: w = element * E8M0 scale   (exact)
 //   NVFP4:   w = element * E4M3 scale   (exact; the FP32 global scale is
 //            applied once to the row's sum)
+//   E2M1 / E4M3 / E5M2 with a typed block scale: w = element * scale
+//   signed int: the affine form on offset-binary codes, bias = -2^(b-1) * scale
+// With K % 32 == 16 (blocks of 16) lanes 0..15 also take the row's last 16
+// codes after the wait.
 // After the wait only x is read: y[m, n] = sum_k x[m, k] * w[n, k], fp32
 // products and sums (warp butterfly, then one shared-memory step across
 // warps), rounded once to the output dtype.  Units past the first UPRE per
@@ -27,14 +31,24 @@ template <int FAM, int B, class T>
 __device__ __forceinline__ void direct_dequant(const Params& p, const uint32_t (&wv)[B], long long srow, int u,
                                                uint32_t kf32, float (&o)[32]) {
     const long long k0 = (long long)u * 32;
-    if constexpr (FAM == FAM_AFFINE) {
+    if constexpr (affine_like<FAM>()) {
         const long long gi = srow + k0 / p.G;
-        const float s = DT<T>::ld(p.scales, gi), b = DT<T>::ld(p.biases, gi);
+        float s, b;
+        uint32_t wx[B];
+#pragma unroll
+        for (int q = 0; q < B; ++q) wx[q] = FAM == FAM_SINT ? wv[q] ^ sint_sign_mask<B>(q) : wv[q];
+        if constexpr (FAM == FAM_SINT) {
+            s = block_scale(p.scales, gi, p.skind);
+            b = -s * (float)(1 << (B - 1));
+        } else {
+            s = DT<T>::ld(p.scales, gi);
+            b = DT<T>::ld(p.biases, gi);
+        }
 #define QMV_DD4(QQ)                                                                                            \
     {                                                                                                          \
-        const float2 d0 = magic_pair_ored(field_magic<B, 4 * QQ>(wv, kf32), field_magic<B, 4 * QQ + 1>(wv, kf32)); \
+        const float2 d0 = magic_pair_ored(field_magic<B, 4 * QQ>(wx, kf32), field_magic<B, 4 * QQ + 1>(wx, kf32)); \
         const float2 d1 =                                                                                      \
-            magic_pair_ored(field_magic<B, 4 * QQ + 2>(wv, kf32), field_magic<B, 4 * QQ + 3>(wv, kf32));       \
+            magic_pair_ored(field_magic<B, 4 * QQ + 2>(wx, kf32), field_magic<B, 4 * QQ + 3>(wx, kf32));       \
         const float c[4] = {d0.x, d0.y, d1.x, d1.y};                                                           \
         _Pragma("unroll") for (int e = 0; e < 4; ++e) {                                                        \
             const float q_ = __fmul_rn(c[e], __uint_as_float((127u - field_p(B, 4 * QQ + e)) << 23));         \
@@ -43,6 +57,14 @@ __device__ __forceinline__ void direct_dequant(const Params& p, const uint32_t (
     }
         QMV_DD4(0) QMV_DD4(1) QMV_DD4(2) QMV_DD4(3) QMV_DD4(4) QMV_DD4(5) QMV_DD4(6) QMV_DD4(7)
 #undef QMV_DD4
+    } else if constexpr (FAM == FAM_E2M1 || FAM == FAM_E4M3 || FAM == FAM_E5M2) {
+        const float s0 = block_scale(p.scales, srow + k0 / p.G, p.skind);
+        const float s1 = p.G == 16 ? block_scale(p.scales, srow + k0 / p.G + 1, p.skind) : s0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const float e = B == 4 ? e2m1_value(wv[j / 8] >> (4 * (j % 8))) : fp8_value<FAM>(wv[j / 4] >> (8 * (j % 4)));
+            o[j] = __fmul_rn(e, j < 16 ? s0 : s1);
+        }
     } else if constexpr (B == 4) {
         const uint8_t* s8 = reinterpret_cast<const uint8_t*>(p.scales) + srow;
         if constexpr (FAM == FAM_NVFP4) {
@@ -174,6 +196,22 @@ __global__ void __launch_bounds__(256) qmv_direct_kernel(const Params p) {
         direct_load<B, WIDE>(row, u, wv);
         direct_dequant<FAM, B, T>(p, wv, srow, u, kf32, wu);
         direct_fma<T, MAXM>(p, X, u, wu, acc);
+    }
+    if constexpr (half_units<FAM>()) {
+        // K % 32 == 16: the row's last 16 codes, one per lane of warp 0
+        if ((p.K & 31) && threadIdx.x < 16) {
+            const long long k = (long long)p.K - 16 + threadIdx.x;
+            float e;
+            if constexpr (B == 4) e = e2m1_value(__ldg(row + (k >> 1)) >> (4 * (int)(k & 1)));
+            else e = fp8_value<FAM>(__ldg(row + k));
+            const long long si = srow + k / p.G;
+            const float sv = FAM == FAM_NVFP4 ? e4m3_value(__ldg(reinterpret_cast<const uint8_t*>(p.scales) + si))
+                                              : block_scale(p.scales, si, p.skind);
+            const float ws = __fmul_rn(e, sv);
+#pragma unroll
+            for (int m = 0; m < MAXM; ++m)
+                if (m < p.M) acc[m] = fmaf(DT<T>::ld(X, (long long)m * p.K + k), ws, acc[m]);
+        }
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll

@@ -48,14 +48,19 @@ cudaError_t launch_direct_fp(int fam, int dtype, int maxm, bool wide, const Para
         case FAM_MXFP4: return direct_fb<FAM_MXFP4, 4>(dtype, maxm, wide, p, L);
         case FAM_NVFP4: return direct_fb<FAM_NVFP4, 4>(dtype, maxm, wide, p, L);
         case FAM_MXFP8: return direct_fb<FAM_MXFP8, 8>(dtype, maxm, wide, p, L);
+        case FAM_E2M1: return direct_fb<FAM_E2M1, 4>(dtype, maxm, wide, p, L);
+        case FAM_E4M3: return direct_fb<FAM_E4M3, 8>(dtype, maxm, wide, p, L);
+        case FAM_E5M2: return direct_fb<FAM_E5M2, 8>(dtype, maxm, wide, p, L);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_direct_affine(int bits, int dtype, int maxm, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_direct_sint(int bits, int dtype, int maxm, bool wide, const Params& p, const Launch& L);
 
 cudaError_t launch_direct(int fam, int bits, int dtype, int maxm, bool wide, const Params& p, const Launch& L) {
     return fam == FAM_AFFINE ? launch_direct_affine(bits, dtype, maxm, wide, p, L)
+         : fam == FAM_SINT   ? launch_direct_sint(bits, dtype, maxm, wide, p, L)
                              : launch_direct_fp(fam, dtype, maxm, wide, p, L);
 }
 

@@ -57,6 +57,18 @@ cudaError_t launch_affine_b5(int dtype, int maxm, int R, bool wide, const Params
 cudaError_t launch_affine_b6(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
 cudaError_t launch_affine_b8(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
 cudaError_t launch_fp(int fam, int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+// Run-time-scaled FP elements (qmv_inst_bs_*.cu) and the signed integers
+// (qmv_inst_sint_b*.cu); launch_fp dispatches the former, launch_sint the latter.
+cudaError_t launch_bs_e2m1(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_bs_e4m3(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_bs_e5m2(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_sint_b2(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_sint_b3(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_sint_b4(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_sint_b5(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_sint_b6(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_sint_b8(int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
+cudaError_t launch_sint(int bits, int dtype, int maxm, int R, bool wide, const Params& p, const Launch& L);
 
 // Tensor-core kernels (qmv_tc_kernel): npass in {1, 2, 4}.
 cudaError_t launch_tc_affine(int bits, int dtype, int npass, const Params& p, const Launch& L);
@@ -91,9 +103,10 @@ cudaError_t launch_quantize_fp(int mode, int dtype, const void* w, void* wq, voi
 cudaError_t launch_quantize_affine(int bits, int dtype, const void* w, void* wq, void* scales, void* biases,
                                    int N, int K, int G, int vec, cudaStream_t st);
 
+// skind: the block-scale type of FAM_E2M1 / FAM_E4M3 / FAM_E5M2 / FAM_SINT.
 cudaError_t launch_dequant(int fam, int bits, int dtype, const uint8_t* w, const void* scales,
                            const void* biases, const float* gscale, float* out, int N, int K, int G,
-                           long long w_row, cudaStream_t s);
+                           long long w_row, cudaStream_t s, int skind = 0);
 
 // Fused gate + up with SwiGLU (qmv_kernel<..., PAIR = true>, affine): R in
 // {2, 4} wide (4 only for maxm <= 2), R = 2 narrow.  Returns

@@ -66,9 +66,28 @@ static PyObject* py_fp(PyObject* self, PyObject* const* a, Py_ssize_t n) {
     return PyLong_FromLong(r);
 }
 
+/* block_scaled(x, w, scales, global_scale, y, M, N, K, format, dtype, batch, x_batched, stream) -> status */
+static PyObject* py_block_scaled(PyObject* self, PyObject* const* a, Py_ssize_t n) {
+    (void)self;
+    if (n != 13) { PyErr_SetString(PyExc_TypeError, "block_scaled() takes 13 arguments"); return NULL; }
+    void* p[5];
+    int v[7];
+    void* st;
+    for (int i = 0; i < 5; ++i) if (as_ptr(a[i], &p[i])) return NULL;
+    for (int i = 0; i < 7; ++i) if (as_int(a[5 + i], &v[i])) return NULL;
+    if (as_ptr(a[12], &st)) return NULL;
+    int r;
+    Py_BEGIN_ALLOW_THREADS
+    r = qmv_block_scaled_batched(p[0], p[1], p[2], (const float*)p[3], p[4], v[0], v[1], v[2], v[3], v[4], v[5],
+                                 v[6], st);
+    Py_END_ALLOW_THREADS
+    return PyLong_FromLong(r);
+}
+
 static PyMethodDef methods[] = {
     {"affine", (PyCFunction)(void (*)(void))py_affine, METH_FASTCALL, "qmv_affine_batched"},
     {"fp", (PyCFunction)(void (*)(void))py_fp, METH_FASTCALL, "qmv_fp_batched"},
+    {"block_scaled", (PyCFunction)(void (*)(void))py_block_scaled, METH_FASTCALL, "qmv_block_scaled_batched"},
     {NULL, NULL, 0, NULL},
 };
 
