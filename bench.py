@@ -597,6 +597,9 @@ def _rotation(wbytes, cap=64, least=1):
     return int(max(least, min(cap, np.ceil(2 * L2_BYTES / max(wbytes, 1)))))
 
 
+SHAPE_SETS = ("c1", "probe", "layer", "fp_chain", "fp_probe", "formats", "sweep")
+
+
 def shape_lines(q, torch, dev, stream, flush, flush_rd, peak, sets=None):
     """Throughput per format, bits and shape (the metric's breakdown), each
     line from ONE CUDA graph of R calls back to back on R weight copies that
@@ -605,10 +608,12 @@ def shape_lines(q, torch, dev, stream, flush, flush_rd, peak, sets=None):
     launching stream; us_per_call = median replay time / R.  Sets: c1 (the
     small 4-bit config), probe (16384^2 4-bit, M = 1 and 8), layer (the 7B
     projections, M = 1 and 8), fp_chain (MXFP4 / NVFP4 / MXFP8 chains of the
-    pages' shapes), fp_probe (16384^2 in each FP format, M = 1) and sweep
-    (2/3/5/6-bit x group 32/64/128 x f32/f16/bf16 x M = 1, 4 at N = K = 4096)."""
+    pages' shapes), fp_probe (16384^2 in each FP format, M = 1), sweep
+    (2/3/5/6-bit x group 32/64/128 x f32/f16/bf16 x M = 1, 4 at N = K = 4096)
+    and formats (every Track-1 block-scaled format at N = K = 8192, M = 1
+    bf16, through qmv_block_scaled)."""
     lines = []
-    sets = sets or ("c1", "probe", "layer", "fp_chain", "fp_probe", "sweep")
+    sets = sets or SHAPE_SETS
 
     def timed(tag, label, R, launch, nbytes, plan, reps=5):
         for r in range(R):                          # eager warm-up (kernel attributes)
@@ -688,6 +693,27 @@ def shape_lines(q, torch, dev, stream, flush, flush_rd, peak, sets=None):
                     q.qmv_fp(x, w, sc, gs, y, 1, 16384, 16384, mode, "bf16")
                 timed("fp_probe", f"{mode} M=1 N=K=16384", R, launch, fp_bytes(1, N, K, mode),
                       q.qmv_describe_plan(mode, 1, N, K, 0, 0, "bf16"))
+        if "formats" in sets:
+            for fmt in q.FORMATS:
+                N = K = 8192
+                info = q.qmv_format_info(fmt)
+                e = ("int" if fmt.startswith(("int", "mxint")) else "e5m2" if "e5m2" in fmt
+                     else "e2m1" if info["element_bits"] == 4 else "e4m3")
+                sk = {1: "e4m3" if info["has_global"] else "e8m0", 2: "f16", 4: "f32"}[info["scale_bytes"]]
+                c = synth.bs_case(1, N, K, e, info["element_bits"], info["block"], sk, info["has_global"], "bf16",
+                                  seed=7300 + q.FORMATS[fmt])
+                wb = N * K * info["element_bits"] // 8 + N * (K // info["block"]) * info["scale_bytes"]
+                R = _rotation(wb, 64, 3)
+                ws = _copies(torch, dev, (c["w"], c["scales"]), R)
+                gs = torch.tensor([c["global"]], dtype=torch.float32, device=dev) if info["has_global"] else None
+                x = torch.from_numpy(c["x"][0].view(np.int16).reshape(-1).copy()).view(torch.bfloat16).to(dev)
+                y = torch.empty(N, dtype=torch.bfloat16, device=dev)
+
+                def launch(r, ws=ws, gs=gs, x=x, y=y, fmt=fmt):
+                    w, sc = ws[r]
+                    q.qmv_block_scaled(x, w, sc, gs, y, 1, 8192, 8192, fmt, "bf16")
+                timed("formats", f"{fmt} M=1 N=K=8192 bf16", R, launch, wb + (4 if gs is not None else 0) + 2 * K + 2 * N,
+                      q.qmv_describe_plan(fmt, 1, N, K, dtype="bf16"))
         if "sweep" in sets:
             for bits in (2, 3, 5, 6):
                 for G in (32, 64, 128):
@@ -842,7 +868,7 @@ def run_ours(args, rank, world, local_rank):
     }
     if args.workload == "chain8" and not args.no_shapes:
         # the metric's breakdown per format / bits / shape; not part of `value`
-        out["shapes"] += shape_lines(q, torch, dev, stream, flush, flush_rd, peak)
+        out["shapes"] += shape_lines(q, torch, dev, stream, flush, flush_rd, peak, args.sets)
     if rank == 0:
         out["cpu_baseline"] = cpu_baseline(args.workload)
         print(json.dumps(out), flush=True)
@@ -997,6 +1023,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="chain8")
     ap.add_argument("--no-shapes", action="store_true",
                     help="chain8 only: skip the per format / bits / shape lines")
+    ap.add_argument("--sets", type=lambda v: tuple(v.split(",")), default=None,
+                    help="chain8: comma-separated subset of the shape sets " + ",".join(SHAPE_SETS))
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

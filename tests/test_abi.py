@@ -163,11 +163,20 @@ def test_format_info_of_every_format():
 
 def test_block_scaled_plans():
     """Every format plans on the few-rows or the row-tiled kernel, never on
-    the affine-only kernels."""
+    the affine-only kernels; the FP formats reach the weight ring only when
+    forced (path 6), for one bf16 x row."""
     for name in q.FORMATS:
-        for (M, N, K) in [(1, 4, 1024), (1, 4096, 4096), (8, 14336, 4096)]:
+        fp = not name.startswith(("int", "mxint"))
+        for (M, N, K) in [(1, 4, 1024), (1, 4096, 4096), (8, 14336, 4096), (1, 14336, 4096)]:
             plan = q.qmv_describe_plan(name, M, N, K, dtype="bf16")
             assert plan.split()[0] in ("path=direct", "path=wide", "path=narrow"), (name, plan)
+        q.qmv_force_config(6, -1, -1, -1)
+        try:
+            ring = q.qmv_describe_plan(name, 1, 14336, 4096, dtype="bf16")
+            assert ("path=tcf" in ring) == fp, (name, ring)
+            assert "path=tcf" not in q.qmv_describe_plan(name, 1, 14336, 4096, dtype="f16"), name
+        finally:
+            q.qmv_force_config()
 
 
 def test_batched_validation():

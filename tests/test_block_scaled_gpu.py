@@ -190,6 +190,47 @@ def test_bs_forced_paths(q, fmt, path):
         compare(y, ref, ad, "bf16", what=f"{fmt} path{path} M{M}")
 
 
+RING_FORMATS = [f for f in FORMATS if not f.startswith(("int", "mxint"))]
+
+
+@pytest.mark.parametrize("fmt", RING_FORMATS)
+def test_bs_weight_ring_path(q, fmt):
+    """One bf16 x row through the weight ring (forced path 6): ragged row
+    blocks, several stages per row block, more row blocks than the grid."""
+    q.qmv_force_config(6, -1, -1, -1)
+    for (N, K) in [(333, 4096), (148 * 128 * 2 + 45, 1024)]:
+        plan = q.qmv_describe_plan(fmt, 1, N, K, dtype="bf16")
+        assert "path=tcf" in plan, plan
+        c = _case(fmt, 1, N, K, "bf16", _seed("ring", fmt, N, K))
+        y = _run(q, c, fmt)[0]
+        rows = sample_rows(N, 64) + list(range(N - 70, N))
+        rows = sorted(set(rows))
+        ref, ad = _oracle(c, fmt, rows=rows)
+        compare(y, ref, ad, "bf16", rows=rows, what=f"ring {fmt} {N}x{K}")
+    assert q.qmv_device_fault(clear=True) == 0
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4", "mxfp8_e4m3", "fp8_e5m2_f16", "nvfp8"])
+def test_bs_weight_ring_precision_and_batch(q, fmt):
+    """The precision case and a batch of 2 (NVFP4: one global per entry)
+    through the weight ring (forced)."""
+    N, K = 2048, 6144
+    q.qmv_force_config(6, -1, -1, -1)
+    assert "path=tcf" in q.qmv_describe_plan(fmt, 1, N, K, dtype="bf16")
+    c = _case(fmt, 1, N, K, "bf16", _seed("ringprec", fmt), precision=True)
+    y = _run(q, c, fmt)[0]
+    ref, ad = _oracle(c, fmt)
+    compare(y, ref, ad, "bf16", what=f"ring precision {fmt}", max_floor_frac=0.25)
+    c = _case(fmt, 1, 300, 2048, "bf16", _seed("ringbatch", fmt), batch=2)
+    if c["global"] is not None:
+        c["global"] = np.float32(1.5)
+    y = _run(q, c, fmt)
+    for b in range(2):
+        ref, ad = _oracle(c, fmt, b=b)
+        compare(y[b], ref, ad, "bf16", what=f"ring batch {fmt} {b}")
+    assert q.qmv_device_fault(clear=True) == 0
+
+
 @pytest.mark.parametrize("fmt", ["int2", "int3", "int4", "int5", "int6", "int8", "mxint4", "int4_f16"])
 @pytest.mark.parametrize("M", [1, 8])
 def test_bs_signed_int_precision_case(q, fmt, M):

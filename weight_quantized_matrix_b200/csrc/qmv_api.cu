@@ -312,16 +312,19 @@ bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s
 // ---- CUDA-core ring launch shape (one bf16 x row, qmv_tcf.cuh) ---------------
 // Same ring and stage layout as the tensor-core ring; a warp takes two
 // super-blocks per step, so a stage is a multiple of 2 * wk super-blocks.  The
-// x tile holds (NP + 4) words of x~ pairs and two sums per unit.
-bool tcf_shape(int N, int K, int bits, int G, bool w16, bool s16, TcbShape* ts) {
+// x tile holds (NP + 4) words of x~ pairs and two sums per unit (affine), or
+// UC + 4 fp32 x values per unit (fp: the block-scaled FP formats, whose
+// scales stay in global memory).
+bool tcf_shape(int N, int K, int bits, int G, bool w16, bool s16, TcbShape* ts, bool fp = false) {
     const int ub = tc_unit_bytes(bits);
     const int uc = ub * 8 / bits;
     const int SB = 4 * uc;
     if (K % SB != 0 || !w16) return false;
     if (((long long)K * bits / 8) % 16 != 0) return false;     // tensor copies: 16-byte rows
-    if (G < uc) return false;                                   // a unit lies in one group
+    if (!fp && G < uc) return false;                            // a unit lies in one group
+    if (fp) s16 = false;
     const int es = 2;
-    const int nps = tc_np_of(bits) + 4;
+    const int nps = fp ? uc + 4 : tc_np_of(bits) + 4;
     const int nsbk = K / SB;
     const int sms = device_sms();
     // Block shape (measured on B200): the fewest rows on the busiest SM
@@ -372,7 +375,7 @@ bool tcf_shape(int N, int K, int bits, int G, bool w16, bool s16, TcbShape* ts) 
         return pitch;
     };
     const size_t red = (size_t)(qmv::kTcbStages + 1) * ncw * 16 * 4;
-    const size_t per_sb = (size_t)4 * (nps * 4 + 8);
+    const size_t per_sb = (size_t)4 * (nps * 4 + (fp ? 0 : 8));
     long long tsb = 0;
     int sring = 0, sbw = 0, stage = 0, pitch = 0;
     for (;;) {
@@ -545,16 +548,23 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     // (measured on B200: the fastest path for one bf16 x row from about 10 MB
     // of 2/3/4/5/6-bit weights; 8-bit codes take two fields each, and there
     // the register-streaming CUDA-core kernel is as fast)
-    const bool fma_ring_pick = M == 1 && dtype == QMV_BF16 && bits >= 2 && bits <= 6 &&
-                               (double)N * K * bits / 8.0 >= 10.0 * 1024 * 1024;
-    if (!gather && aff && K > 0 && M == 1 && dtype == QMV_BF16 &&
+    // The block-scaled FP formats run on the same ring when forced (path 6):
+    // with their block scales read from global memory in every step, 8
+    // compute warps per SM hide that latency worse than the row-tiled
+    // kernel's 16 (measured on B200, MXFP4 16384^2: 150 us on the ring, 53 us
+    // row-tiled), so the picker keeps them on the row-tiled kernel.
+    const bool fp_fam = fam == qmv::FAM_MXFP4 || fam == qmv::FAM_NVFP4 || fam == qmv::FAM_MXFP8 ||
+                        fam == qmv::FAM_E2M1 || fam == qmv::FAM_E4M3 || fam == qmv::FAM_E5M2;
+    const bool big = (double)N * K * fi.bits / 8.0 >= 10.0 * 1024 * 1024;
+    const bool fma_ring_pick = M == 1 && dtype == QMV_BF16 && aff && bits >= 2 && bits <= 6 && big;
+    if (!gather && (aff || fp_fam) && K > 0 && M == 1 && dtype == QMV_BF16 &&
         (g_forced.path == 6 || (g_forced.path < 0 && fma_ring_pick))) {
         TcbShape ts;
-        if (tcf_shape(N, K, bits, G_of_plan, w16, s16, &ts)) {
+        if (tcf_shape(N, K, fi.bits, G_of_plan, w16, aff && s16, &ts, !aff)) {
             pl->maxm = 1; pl->R = 1; pl->wide = 1; pl->tc = 4; pl->npass = 0;
             pl->wk = ts.wk; pl->wr = ts.wr; pl->tile_iters = ts.tsb; pl->sps = ts.sps; pl->pitch = ts.pitch;
             pl->spb = 1; pl->sring = ts.sring; pl->soff = ts.soff; pl->boff = ts.boff; pl->sbw = ts.sbw;
-            pl->C = 4 * tc_unit_bytes(bits) * 8 / bits; pl->smem = ts.smem;
+            pl->C = 4 * tc_unit_bytes(fi.bits) * 8 / fi.bits; pl->smem = ts.smem;
             pl->grid = dim3((unsigned)ts.gx, 1, (unsigned)batch);
             pl->block = dim3(32 * (ts.wk * ts.wr + 1), 1, 1);
             return QMV_OK;
@@ -615,10 +625,12 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
         // k-warps: at least 2 for long rows (>= 256 chunks: more loads in
         // flight per row; not for 6-bit, whose 12-word chunks already fill
         // the registers), more while the GPU holds fewer than ~8 warps per SM
-        wk = (NC >= 256 && fi.bits != 6) ? 2 : 1;
+        // (the block-scaled and signed-int families: one k-warp and 8 row
+        // warps, measured best on B200 for 4- and 8-bit codes at 16384^2)
+        wk = (aff && NC >= 256 && fi.bits != 6) ? 2 : 1;
         while (wk < 8 && warps * wk < (long long)sms * 8 && NC >= 64 * wk) wk *= 2;
         wr = wk >= 8 ? 1 : 8 / wk;
-        if (wr > 4 && wk == 1) wr = 4;
+        if (aff && wr > 4 && wk == 1) wr = 4;
     }
     if (g_forced.R > 0) R = g_forced.R;
     if (g_forced.wk > 0) wk = g_forced.wk;
@@ -825,7 +837,8 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     if (pl.tc == 4) {
         p.fault = fault_word();
         if (!p.fault) return QMV_ECUDA;
-        return finish(qmv::launch_tcf_affine(bits, pl.wk * pl.wr, p, L));
+        return finish(fam == qmv::FAM_AFFINE ? qmv::launch_tcf_affine(bits, pl.wk * pl.wr, p, L)
+                                             : qmv::launch_tcf_fp(fam, pl.wk * pl.wr, p, L));
     }
     if (pl.tc == 5) {
         p.fault = fault_word();

@@ -55,6 +55,7 @@
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <string.h>
 
 namespace qmv {
 
@@ -295,6 +296,31 @@ template <int FAM> __device__ __forceinline__ float fp8_value(uint32_t c) {
     if constexpr (FAM == FAM_E5M2) return e5m2_value(c);
     else return e4m3_value(c);
 }
+// Hardware element decode for the inner loops: two E2M1 codes (one byte, low
+// nibble first) or two E4M3 / E5M2 codes (two bytes, low byte first) -> f16x2
+// (low half first).  Exact: every value of these element types is a binary16
+// value (E4M3 NaN and E5M2 infinities / NaN included); widening to fp32 is
+// exact too.  The bit-pattern decoders above serve the check kernel.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(uint32_t v) {
+    uint32_t d;
+    asm("{.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;}" : "=r"(d) : "r"(v));
+    return d;
+}
+template <int FAM>
+__device__ __forceinline__ uint32_t cvt_fp8x2(uint32_t v) {
+    uint32_t d;
+    if constexpr (FAM == FAM_E5M2)
+        asm("{.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e5m2x2 %0, t;}" : "=r"(d) : "r"(v));
+    else
+        asm("{.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;}" : "=r"(d) : "r"(v));
+    return d;
+}
+__device__ __forceinline__ float2 half2_bits_to_float2(uint32_t h) {
+    __half2 v;
+    memcpy(&v, &h, 4);
+    return __half22float2(v);
+}
+
 // Block scale i of a run-time-typed scale array.
 __device__ __forceinline__ float block_scale(const void* s, long long i, int kind) {
     switch (kind) {
@@ -491,13 +517,12 @@ __device__ __forceinline__ void compute_chunk(const uint32_t (&wv)[R][B * U], co
                     d1 = magic_pair_ored(f2, f3);
                 } else if constexpr (B == 4) {
                     const uint32_t wd = wu[q >> 1] >> (16 * (q & 1));
-                    const float2 s126 = make_float2(0x1p126f, 0x1p126f);
-                    d0 = mul2(make_float2(__uint_as_float(e2m1_pattern(wd)), __uint_as_float(e2m1_pattern(wd >> 4))), s126);
-                    d1 = mul2(make_float2(__uint_as_float(e2m1_pattern(wd >> 8)), __uint_as_float(e2m1_pattern(wd >> 12))), s126);
+                    d0 = half2_bits_to_float2(cvt_e2m1x2(wd));
+                    d1 = half2_bits_to_float2(cvt_e2m1x2(wd >> 8));
                 } else {
                     const uint32_t wd = wu[q];
-                    d0 = make_float2(fp8_value<FAM>(wd), fp8_value<FAM>(wd >> 8));
-                    d1 = make_float2(fp8_value<FAM>(wd >> 16), fp8_value<FAM>(wd >> 24));
+                    d0 = half2_bits_to_float2(cvt_fp8x2<FAM>(wd));
+                    d1 = half2_bits_to_float2(cvt_fp8x2<FAM>(wd >> 16));
                 }
                 const int h = half_units<FAM>() ? (q >> 2) : 0;    // 16-code half of the unit
 #pragma unroll

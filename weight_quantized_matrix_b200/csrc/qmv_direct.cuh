@@ -61,26 +61,36 @@ __device__ __forceinline__ void direct_dequant(const Params& p, const uint32_t (
         const float s0 = block_scale(p.scales, srow + k0 / p.G, p.skind);
         const float s1 = p.G == 16 ? block_scale(p.scales, srow + k0 / p.G + 1, p.skind) : s0;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const float e = B == 4 ? e2m1_value(wv[j / 8] >> (4 * (j % 8))) : fp8_value<FAM>(wv[j / 4] >> (8 * (j % 4)));
-            o[j] = __fmul_rn(e, j < 16 ? s0 : s1);
+        for (int j = 0; j < 32; j += 2) {
+            const float2 e = B == 4 ? half2_bits_to_float2(cvt_e2m1x2(wv[j / 8] >> (4 * (j % 8))))
+                                    : half2_bits_to_float2(cvt_fp8x2<FAM>(wv[j / 4] >> (8 * (j % 4))));
+            o[j] = __fmul_rn(e.x, j < 16 ? s0 : s1);
+            o[j + 1] = __fmul_rn(e.y, j < 16 ? s0 : s1);
         }
     } else if constexpr (B == 4) {
         const uint8_t* s8 = reinterpret_cast<const uint8_t*>(p.scales) + srow;
+        float s0, s1;
         if constexpr (FAM == FAM_NVFP4) {
-            const float s0 = e4m3_value(__ldg(s8 + k0 / 16)), s1 = e4m3_value(__ldg(s8 + k0 / 16 + 1));
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __fmul_rn(e2m1_value(wv[j / 8] >> (4 * (j % 8))), j < 16 ? s0 : s1);
+            s0 = e4m3_value(__ldg(s8 + k0 / 16));
+            s1 = e4m3_value(__ldg(s8 + k0 / 16 + 1));
         } else {
-            const float s = e8m0_value(__ldg(s8 + k0 / 32));
+            s0 = s1 = e8m0_value(__ldg(s8 + k0 / 32));
+        }
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __fmul_rn(e2m1_value(wv[j / 8] >> (4 * (j % 8))), s);
+        for (int j = 0; j < 32; j += 2) {
+            const float2 e = half2_bits_to_float2(cvt_e2m1x2(wv[j / 8] >> (4 * (j % 8))));
+            o[j] = __fmul_rn(e.x, j < 16 ? s0 : s1);
+            o[j + 1] = __fmul_rn(e.y, j < 16 ? s0 : s1);
         }
     } else {
         const uint8_t* s8 = reinterpret_cast<const uint8_t*>(p.scales) + srow;
         const float s = e8m0_value(__ldg(s8 + k0 / 32));
 #pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] = __fmul_rn(e4m3_value(wv[j / 4] >> (8 * (j % 4))), s);
+        for (int j = 0; j < 32; j += 2) {
+            const float2 e = half2_bits_to_float2(cvt_fp8x2<FAM>(wv[j / 4] >> (8 * (j % 4))));
+            o[j] = __fmul_rn(e.x, s);
+            o[j + 1] = __fmul_rn(e.y, s);
+        }
     }
 }
 

@@ -11,11 +11,11 @@ template <int B>
 cudaError_t tcf_b(int ncw, const Params& p, const Launch& L) {
     if (ncw == 8) {
         static std::atomic<unsigned> cfg_{0};
-        return launch_kernel(qmv_tcf_kernel<B, kTcbStages, 288>, cfg_, L, p);
+        return launch_kernel(qmv_tcf_kernel<FAM_AFFINE, B, kTcbStages, 288>, cfg_, L, p);
     }
     if (ncw == 12) {
         static std::atomic<unsigned> cfg_{0};
-        return launch_kernel(qmv_tcf_kernel<B, kTcbStages, 416>, cfg_, L, p);
+        return launch_kernel(qmv_tcf_kernel<FAM_AFFINE, B, kTcbStages, 416>, cfg_, L, p);
     }
     return cudaErrorInvalidValue;
 }

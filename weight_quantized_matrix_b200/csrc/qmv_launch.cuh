@@ -80,6 +80,9 @@ constexpr int kTcbStages = 4;
 // CUDA-core kernels with the weight ring, one bf16 x row (qmv_tcf_kernel):
 // ncw = compute warps per block in {8, 12} (plus the producer warp).
 cudaError_t launch_tcf_affine(int bits, int ncw, const Params& p, const Launch& L);
+// The same ring for the block-scaled FP families (qmv_inst_tcf_fp.cu): fam one
+// of FAM_MXFP4 / NVFP4 / E2M1 / MXFP8 / E4M3 / E5M2.
+cudaError_t launch_tcf_fp(int fam, int ncw, const Params& p, const Launch& L);
 
 
 

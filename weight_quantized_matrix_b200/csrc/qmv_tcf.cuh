@@ -25,6 +25,15 @@
 // units sit 80 bytes apart (unit stride NP + 4 words), so neither load has
 // bank conflicts.  Warp (wrid, wkid) takes the steps wkid, wkid + wk, ... of
 // every stage; a stage holds a multiple of 2 * wk super-blocks.
+//
+// The block-scaled FP formats (FAM != FAM_AFFINE; E2M1 codes B = 4, E4M3 /
+// E5M2 codes B = 8) stream through the same ring and lane layout: a 16-byte
+// unit holds 32 E2M1 or 16 8-bit codes, decoded two at a time by the hardware
+// conversion to f16x2 and widened to fp32 (exact), against x staged as plain
+// fp32 rows of UC + 4 floats per unit (the pad keeps the 8 lanes of a
+// shared-memory phase on distinct banks); the unit's one or two block scales
+// (blocks of 16 or 32 codes, any scale type) come from global memory, and
+// NVFP4's global scale multiplies the stored row sum.
 #pragma once
 
 #include "qmv_tcb.cuh"
@@ -63,17 +72,58 @@ __device__ __forceinline__ void tcf_unit(std::integer_sequence<int, Q...>, const
 //   ring  STAGES stages (128-byte aligned): ROWS packed rows (pitch bytes
 //         each), then (p.sring) the scale tile at p.soff and the bias tile at
 //         p.boff, ROWS x p.sbw bytes each
-//   xs    TU * (NP + 4) u32     x~ pairs of the tile's units (bf16x2, plan order)
-//   us    TU * 2 floats         {sum(x), sum(x~)} per unit
+//   xs    TU * (NP + 4) u32     x~ pairs of the tile's units (bf16x2, plan order);
+//                               FP: TU * (UC + 4) fp32 x values
+//   us    TU * 2 floats         {sum(x), sum(x~)} per unit (affine only)
 //   red   (STAGES + 1) * NCW * 16 floats   per-warp row sums, by row block
 // MAXT = 32 * (NCW + 1): NCW = wk * wr in {8, 12} compute warps + the producer.
-template <int B, int STAGES, int MAXT>
+// FP unit: Y[i] += (block scale) * sum of x * element over the unit, with the
+// unit's codes w (16 bytes) and its x row xf (UC fp32 values).
+template <int FAM, int B>
+__device__ __forceinline__ void fpr_unit(const uint32_t (&w)[4], const float* xf, float2& p0, float2& p1) {
+    if constexpr (B == 4) {
+        // 32 E2M1 codes: codes 0..15 (words 0, 1) into p0, 16..31 into p1
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const float2 e = half2_bits_to_float2(cvt_e2m1x2(w[wi] >> (8 * b)));
+                const float2 xv = *reinterpret_cast<const float2*>(xf + 8 * wi + 2 * b);
+                if (wi < 2) p0 = fma2(xv, e, p0);
+                else p1 = fma2(xv, e, p1);
+            }
+    } else {
+        // 16 8-bit codes, one block
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float2 e = half2_bits_to_float2(cvt_fp8x2<FAM>(w[wi] >> (16 * h)));
+                const float2 xv = *reinterpret_cast<const float2*>(xf + 4 * wi + 2 * h);
+                p0 = fma2(xv, e, p0);
+            }
+    }
+}
+
+// Block scale of an FP family at element index i of the scale array.
+template <int FAM>
+__device__ __forceinline__ float fpr_scale(const Params& p, long long i) {
+    if constexpr (FAM == FAM_NVFP4) return e4m3_value(__ldg(reinterpret_cast<const uint8_t*>(p.scales) + i));
+    else if constexpr (FAM == FAM_MXFP4 || FAM == FAM_MXFP8) return e8m0_value(__ldg(reinterpret_cast<const uint8_t*>(p.scales) + i));
+    else return block_scale(p.scales, i, p.skind);
+}
+
+template <int FAM, int B, int STAGES, int MAXT>
 __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant__ Params p) {
     using T = __nv_bfloat16;
     using Gm = TcGeom<B>;
+    constexpr bool AFF = FAM == FAM_AFFINE;
     constexpr TcPlanData P = tc_make_plan<B, false>();
-    constexpr int NP = P.np, NPS = NP + 4;
     constexpr int NW = Gm::NW, UB = Gm::UNIT_BYTES, UC = Gm::UNIT_CODES, SB = Gm::SB;
+    // x words per unit in shared memory: bf16 pairs in plan order (affine) or
+    // fp32 values (FP), plus a 4-word pad
+    constexpr int NP = P.np, NPS = AFF ? NP + 4 : UC + 4;
+    static_assert(AFF || ((B == 4 || B == 8) && UB == 16), "FP units are 16 bytes");
     static_assert(2 * STAGES * 8 <= 96 && 4 * (STAGES + 1) <= 32, "barrier area");
 
     extern __shared__ float4 smem4[];
@@ -91,7 +141,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
     const int TSB = p.tile_iters;
     const int TU = TSB * 4;
     const int G = p.G;
-    const int segsz = min(G, SB);
+    const int segsz = AFF ? min(G, SB) : SB;
     const long long KG = p.K / G;
     const int bz = blockIdx.z;
     const int gmul = G < SB ? __ffs(SB / G) - 1 : 0;
@@ -101,8 +151,8 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
     unsigned* rdone = reinterpret_cast<unsigned*>(smem + 96);
     unsigned char* ring = smem + 128 + ((128u - (smem_addr(smem) & 127u)) & 127u);
     uint32_t* xs = reinterpret_cast<uint32_t*>(ring + (size_t)STAGES * stage_bytes);
-    float2* us = reinterpret_cast<float2*>(xs + (size_t)TU * NPS);
-    float* red = reinterpret_cast<float*>(us + TU);
+    float2* us = reinterpret_cast<float2*>(xs + (size_t)TU * NPS);       // affine only
+    float* red = AFF ? reinterpret_cast<float*>(us + TU) : reinterpret_cast<float*>(us);
     const uint32_t bar0 = smem_addr(bars);
     auto full = [&](int s) { return bar0 + 8u * (uint32_t)s; };
     auto empty = [&](int s) { return bar0 + 8u * (uint32_t)(STAGES + s); };
@@ -156,7 +206,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
     const int nthr = NCW * 32;
     const int r4 = lane >> 3, u8 = lane & 7;
     const int half = u8 >> 2, t = u8 & 3;          // super-block of the step, unit in it
-    const int useg = (t * UC) / segsz;              // scale group of the unit within its super-block
+    const int useg = AFF ? (t * UC) / segsz : 0;    // scale group of the unit within its super-block
     const int wkid = warp % wk, wrid = warp / wk;
     const T* X = reinterpret_cast<const T*>(p.x) + bz * p.x_bs;
     const uint32_t kbf16 = p.kbf16;
@@ -194,6 +244,13 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
                     } else {
 #pragma unroll
                         for (int c = 0; c < UC; ++c) xv[c] = DT<T>::ld(xr, c);
+                    }
+                    if constexpr (!AFF) {
+                        float4* dst = reinterpret_cast<float4*>(xs + (size_t)u * NPS);
+#pragma unroll
+                        for (int c = 0; c < UC / 4; ++c)
+                            dst[c] = make_float4(xv[4 * c], xv[4 * c + 1], xv[4 * c + 2], xv[4 * c + 3]);
+                        continue;
                     }
                     float usum = 0.f, tsum = 0.f;
 #pragma unroll
@@ -241,6 +298,27 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
                         const int sb = sbase + sbl;
                         const bool valid = sb < send;
                         const int ut = valid ? (sb - t0) * 4 + t : 0;   // unit within the x tile
+                        if constexpr (!AFF) {
+                            const float* xf = reinterpret_cast<const float*>(xs + (size_t)ut * NPS);
+                            const unsigned char* src0 = rows0 + (8 * j + u8) * UB;
+                            const long long k0 = (long long)sb * SB + t * UC;           // the unit's first code
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const uint4 a = *reinterpret_cast<const uint4*>(src0 + (size_t)(4 * i) * pitch);
+                                const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+                                float2 p0 = make_float2(0.f, 0.f), p1 = make_float2(0.f, 0.f);
+                                fpr_unit<FAM, B>(w, xf, p0, p1);
+                                const long long si = valid ? srow[i] + k0 / G : srow[i];
+                                const float s0 = fpr_scale<FAM>(p, si);
+                                float yn = fmaf(s0, p0.x + p0.y, Y[i]);
+                                if constexpr (B == 4) {
+                                    const float s1 = G == 16 ? fpr_scale<FAM>(p, si + 1) : s0;
+                                    yn = fmaf(s1, p1.x + p1.y, yn);
+                                }
+                                Y[i] = valid ? yn : Y[i];
+                            }
+                            return;
+                        }
                         uint32_t xq[NP];
 #pragma unroll
                         for (int q = 0; q < NP / 4; ++q) {
@@ -276,7 +354,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
                             Y[i] = valid ? yn : Y[i];
                         }
                     };
-                    if (sring) {
+                    if (AFF && sring) {
                         for (int j = wkid; j < nsteps; j += wk) step(std::true_type{}, j);
                     } else {
                         for (int j = wkid; j < nsteps; j += wk) step(std::false_type{}, j);
@@ -317,6 +395,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
                     float v = 0.f;
                     for (int k = 0; k < wk; ++k) v += rred[(w_ * wk + k) * 16 + r];
                     const int row = rb * ROWS + i;
+                    if constexpr (FAM == FAM_NVFP4) v *= __ldg(p.gscale + bz);
                     if (row < p.N) DT<T>::st(Yo, row, v);
                 }
             }
