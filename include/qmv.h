@@ -479,6 +479,19 @@ int qmv_device_fault(unsigned int* code, int clear);
  */
 void qmv_force_config(int path, int rows_per_warp, int warps_k, int warps_rows);
 
+/*
+ * qmv_test_skip_last_copy -- NOT FOR PRODUCTION USE (tests of the bounded
+ * waits).  While enabled (nonzero), every launch of a weight-ring kernel
+ * (paths "tcb" and "tcf") has the producer warp of block (0, 0) skip its final
+ * ring stage: no expected-bytes arrival and no tensor copy.  That block's
+ * consumer warps then give up their bounded wait on the stage (about 1 s) and
+ * OR code 1 into the fault word, the producer gives up its wait for its own
+ * copies on it and ORs code 4, and the kernel returns normally with undefined
+ * output; no copy is left in flight, and the context stays usable.  Process
+ * global, not thread-safe; 0 restores normal launches.
+ */
+void qmv_test_skip_last_copy(int enable);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,7 +23,7 @@ __all__ = [
     "qmv_last_cuda_error",
     "qmv_describe_plan", "qmv_force_config", "DTYPES", "FP_MODES", "LIB_PATH", "lib",
     "qmv_block_scaled", "qmv_block_scaled_batched", "qmv_dequant_block_scaled_f32", "qmv_format_info",
-    "FORMATS",
+    "FORMATS", "qmv_test_skip_last_copy",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -89,6 +89,7 @@ _lib.qmv_dequant_block_scaled_f32.argtypes = [_p, _p, _p, _p, _i, _i, _i, _p]
 _lib.qmv_format_info.argtypes = [_i] + [ctypes.POINTER(ctypes.c_int)] * 4
 _lib.qmv_device_fault.argtypes = [ctypes.POINTER(ctypes.c_uint), _i]
 _lib.qmv_force_config.argtypes = [_i, _i, _i, _i]
+_lib.qmv_test_skip_last_copy.argtypes = [_i]
 _lib.qmv_force_config.restype = None
 for _f in ("qmv_affine", "qmv_affine_batched", "qmv_fp", "qmv_fp_batched",
            "qmv_dequant_affine_f32", "qmv_dequant_fp_f32", "qmv_quantize_affine", "qmv_qvm_affine",
@@ -341,6 +342,12 @@ def qmv_device_fault(clear=False) -> int:
     code = ctypes.c_uint(0)
     _check(_lib.qmv_device_fault(ctypes.byref(code), int(bool(clear))), "qmv_device_fault")
     return code.value
+
+
+def qmv_test_skip_last_copy(enable=True):
+    """NOT FOR PRODUCTION USE: make the weight-ring kernels' block (0, 0) skip
+    its final stage so the bounded waits run out (see include/qmv.h)."""
+    _lib.qmv_test_skip_last_copy(int(bool(enable)))
 
 
 def qmv_force_config(path=-1, rows_per_warp=-1, warps_k=-1, warps_rows=-1):

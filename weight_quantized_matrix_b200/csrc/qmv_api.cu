@@ -17,6 +17,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include <cudaTypedefs.h>
@@ -32,6 +33,7 @@ thread_local int g_last_cuda = 0;
 
 struct Forced { int path = -1, R = -1, wk = -1, wr = -1; };
 Forced g_forced;
+std::atomic<int> g_test_skip{0};     // qmv_test_skip_last_copy
 
 struct DevInfo { int sms = 0; int ok = 0; unsigned* fault = nullptr; };
 DevInfo g_dev[64];
@@ -824,6 +826,7 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     p.n_experts = n_experts;
     p.gamma = nullptr; p.eps = 0.f;
     p.skind = skind;
+    p.test_skip = g_test_skip.load(std::memory_order_relaxed);
     cudaError_t e;
     p.sps = pl.sps; p.pitch = pl.pitch; p.fault = nullptr;
     p.sring = pl.sring; p.soff = pl.soff; p.boff = pl.boff; p.sbw = pl.sbw;
@@ -1403,6 +1406,8 @@ int qmv_device_fault(unsigned int* code, int clear) {
     }
     return finish(e);
 }
+
+void qmv_test_skip_last_copy(int enable) { g_test_skip.store(enable ? 1 : 0, std::memory_order_relaxed); }
 
 void qmv_force_config(int path, int rows_per_warp, int warps_k, int warps_rows) {
     g_forced.path = path;

@@ -131,6 +131,10 @@ struct Params {
     float eps;
     // Block-scale type of FAM_E2M1 / FAM_E4M3 / FAM_E5M2 / FAM_SINT (ScaleKind).
     int skind;
+    // Weight-ring kernels, tests only (qmv_test_skip_last_copy): nonzero makes
+    // block (0, 0)'s producer skip its final stage, so the bounded waits on it
+    // run out.
+    int test_skip;
 };
 
 // Row mapping of the row-tiled kernel: plain, the interleaved gate / up

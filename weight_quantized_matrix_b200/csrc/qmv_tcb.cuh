@@ -208,7 +208,13 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcb_kernel(const __grid_constant_
                 const int slot = it % STAGES, f = it / STAGES;
                 if (f > 0 && !mbar_wait(empty(slot), (uint32_t)((f - 1) & 1))) { ok = false; break; }
                 const uint32_t st0 = ring0 + (uint32_t)(slot * stage_bytes);
-                if (lane == 0) {
+                // test hook (qmv_test_skip_last_copy): block (0, 0)'s final stage
+                // gets neither its expected-bytes arrival nor its copies, so the
+                // bounded waits on it run out (codes 1 and 4); no copy is left
+                // in flight
+                const bool skip = p.test_skip && blockIdx.x == 0 && blockIdx.z == 0 &&
+                                  rb + (int)gridDim.x >= nrb && ks == nks - 1;
+                if (lane == 0 && !skip) {
                     // one tensor copy each: the stage's packed rows (ROWS x pitch
                     // bytes), scale tile and bias tile (ROWS x sbw bytes); rows
                     // past N and columns past the row end are zero-filled and
