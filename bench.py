@@ -2,7 +2,8 @@
 """Benchmark of the weight-quantized matrix-vector product on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload chain8|layer|probe|quantize|quantize_fp|qvm|qmm|moe]
+                    [--workload chain8|layer|probe|quantize|quantize_fp|qvm|qmm|moe|fmt_probe]
+                    [--format FMT] [--sets SET,...] [--no-shapes]
 
 Prints ONE JSON line (rank 0).  Metric: qmv microseconds per call and achieved
 HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
@@ -29,6 +30,8 @@ HBM GB/s.  Workloads (synthetic, seeded inputs from synth/):
   qvm               x times W stored [K, N] (qmv_qvm_affine), affine 4-bit g64
                     bf16, N=K=16384, M=1, with the K-split workspace: three
                     back-to-back calls per step, each on its own weight copy.
+  fmt_probe         the probe in one Track-1 block-scaled format (--format,
+                    default mxfp4) through qmv_block_scaled, bf16, N=K=16384.
 
 Timing: W untimed warm-up steps, then K steps.  A step is ONE CUDA graph
 holding every call of the workload (dependent calls linked by programmatic
@@ -336,6 +339,69 @@ class Probe(Layer):
                       "its own 151 MB weight copy"}
 
 
+def bs_layout(q, fmt):
+    """synth.bs_case layout arguments (element, bits, block, scale type,
+    global) of a Track-1 format, from the library's qmv_format_info."""
+    info = q.qmv_format_info(fmt)
+    e = ("int" if fmt.startswith(("int", "mxint")) else "e5m2" if "e5m2" in fmt
+         else "e2m1" if info["element_bits"] == 4 else "e4m3")
+    sk = {1: "e4m3" if info["has_global"] else "e8m0", 2: "f16", 4: "f32"}[info["scale_bytes"]]
+    return e, info["element_bits"], info["block"], sk, info["has_global"]
+
+
+def bs_bytes(q, fmt, M, N, K, eb=2):
+    """Algorithmic bytes of one Track-1 call: codes + block scales (+ the NVFP4
+    global) + x + y."""
+    info = q.qmv_format_info(fmt)
+    return (N * K * info["element_bits"] // 8 + N * (K // info["block"]) * info["scale_bytes"]
+            + (4 if info["has_global"] else 0) + M * K * eb + M * N * eb)
+
+
+class FmtProbe(Probe):
+    """The bandwidth probe in one Track-1 block-scaled format (--format): each
+    step makes CALLS calls of qmv_block_scaled, one on each of CALLS distinct
+    N = K = 16384 weight copies, M = 1, bf16 x and y."""
+    FMT = "mxfp4"
+    name = "bandwidth probe, mxfp4 bf16, N=K=16384, M=1"
+
+    def __init__(self, q, torch, dev):
+        self.q, self.torch = q, torch
+        self.fmt = fmt = self.FMT
+        N = K = 16384
+        lay = bs_layout(q, fmt)
+        c = synth.bs_case(1, N, K, *lay, "bf16", seed=3200)
+        ws = [tuple(torch.from_numpy(np.ascontiguousarray(a).view(np.uint8).reshape(-1)).to(dev)
+                    for a in (c["w"], c["scales"])) for _ in range(self.CALLS)]
+        self.g = torch.tensor([c["global"]], dtype=torch.float32, device=dev) if lay[4] else None
+        x_host = torch.from_numpy(c["x"][0].view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+        self.sets = [dict(name=f"{fmt} probe", M=1, N=N, K=K, ws=ws, x=x_host.to(dev), x_host=x_host,
+                          y=torch.empty((1, N), dtype=torch.bfloat16, device=dev),
+                          y_host=torch.empty((1, N), dtype=torch.bfloat16).pin_memory(), it=0)]
+        self.calls_per_step = self.CALLS
+
+    def run_group(self, s, e2e=False, v=0):
+        if e2e:
+            s["x"].copy_(s["x_host"], non_blocking=True)
+        for c in range(self.CALLS):
+            w, sc = s["ws"][c]
+            self.q.qmv_block_scaled(s["x"], w, sc, self.g, s["y"], 1, s["N"], s["K"], self.fmt, "bf16")
+        if e2e:
+            s["y_host"].copy_(s["y"], non_blocking=True)
+        return self.CALLS
+
+    def group_bytes(self, s):
+        return bs_bytes(self.q, self.fmt, 1, s["N"], s["K"]) * self.CALLS
+
+    def group_plan(self, s):
+        return self.q.qmv_describe_plan(self.fmt, 1, s["N"], s["K"], dtype="bf16")
+
+    def config(self):
+        return {"workload": self.name, "format": self.fmt, "dtype": "bf16", "M": 1, "N": 16384, "K": 16384,
+                "calls_per_step": self.CALLS,
+                "l2": "flushed before every step (512 MB write + 256 MB read); each of the step's 3 calls reads "
+                      "its own weight copy"}
+
+
 class Quantize(Layer):
     """The affine quantizer on the bandwidth-probe matrix: bf16 w [16384,
     16384] -> 4-bit g64 codes, scales, biases; two weight copies (537 MB each,
@@ -570,7 +636,7 @@ class Qvm(Layer):
 
 
 WORKLOADS = {"chain8": Chain8, "layer": Layer, "probe": Probe, "quantize": Quantize, "qvm": Qvm, "qmm": Qmm, "moe": Moe,
-             "quantize_fp": QuantizeFp}
+             "quantize_fp": QuantizeFp, "fmt_probe": FmtProbe}
 
 
 # ------------------------------------------- per format / bits / shape --
@@ -696,23 +762,19 @@ def shape_lines(q, torch, dev, stream, flush, flush_rd, peak, sets=None):
         if "formats" in sets:
             for fmt in q.FORMATS:
                 N = K = 8192
-                info = q.qmv_format_info(fmt)
-                e = ("int" if fmt.startswith(("int", "mxint")) else "e5m2" if "e5m2" in fmt
-                     else "e2m1" if info["element_bits"] == 4 else "e4m3")
-                sk = {1: "e4m3" if info["has_global"] else "e8m0", 2: "f16", 4: "f32"}[info["scale_bytes"]]
-                c = synth.bs_case(1, N, K, e, info["element_bits"], info["block"], sk, info["has_global"], "bf16",
-                                  seed=7300 + q.FORMATS[fmt])
-                wb = N * K * info["element_bits"] // 8 + N * (K // info["block"]) * info["scale_bytes"]
+                lay = bs_layout(q, fmt)
+                c = synth.bs_case(1, N, K, *lay, "bf16", seed=7300 + q.FORMATS[fmt])
+                wb = bs_bytes(q, fmt, 0, N, K)                     # codes + scales (M = 0: no x, y)
                 R = _rotation(wb, 64, 3)
                 ws = _copies(torch, dev, (c["w"], c["scales"]), R)
-                gs = torch.tensor([c["global"]], dtype=torch.float32, device=dev) if info["has_global"] else None
+                gs = torch.tensor([c["global"]], dtype=torch.float32, device=dev) if lay[4] else None
                 x = torch.from_numpy(c["x"][0].view(np.int16).reshape(-1).copy()).view(torch.bfloat16).to(dev)
                 y = torch.empty(N, dtype=torch.bfloat16, device=dev)
 
                 def launch(r, ws=ws, gs=gs, x=x, y=y, fmt=fmt):
                     w, sc = ws[r]
                     q.qmv_block_scaled(x, w, sc, gs, y, 1, 8192, 8192, fmt, "bf16")
-                timed("formats", f"{fmt} M=1 N=K=8192 bf16", R, launch, wb + (4 if gs is not None else 0) + 2 * K + 2 * N,
+                timed("formats", f"{fmt} M=1 N=K=8192 bf16", R, launch, bs_bytes(q, fmt, 1, N, K),
                       q.qmv_describe_plan(fmt, 1, N, K, dtype="bf16"))
         if "sweep" in sets:
             for bits in (2, 3, 5, 6):
@@ -887,6 +949,8 @@ def _oracle_sample(workload, budget_s=12.0, threads=None):
         return _oracle_qvm_sample(budget_s, threads)
     if workload == "quantize_fp":
         return _oracle_quantize_fp_sample(budget_s, threads)
+    if workload == "fmt_probe":
+        return _oracle_fmt_probe_sample(budget_s, threads)
     if workload == "chain8":
         spec = [(1, N, CHAIN_K, CHAIN_BITS, CHAIN_G, CHAIN_CALLS) for N in CHAIN_NS]
     elif workload == "layer":
@@ -919,6 +983,25 @@ def _oracle_sample(workload, budget_s=12.0, threads=None):
         sample.append(f"M={M} N={N} K={K}: {nrows}/{N} rows, {dt:.3f}s")
     ncalls = 1 if workload == "moe" else sum(s[-1] for s in spec)     # moe: one call = all its tokens
     return total_us / ncalls, threads, "; ".join(sample)
+
+
+def _oracle_fmt_probe_sample(budget_s, threads):
+    """The oracle's Track-1 qmv (oracle.qmv_block_scaled) on a growing row
+    sample of the format probe's 16384 x 16384 matrix, scaled to one call."""
+    import oracle
+    fmt = FmtProbe.FMT
+    N = K = 16384
+    c = synth.bs_case(1, N, K, *oracle.TRACK1[fmt], "bf16", seed=3200)
+    args = (c["x"][0], c["w"][0], c["scales"][0], c["global"], 1, N, K, fmt, "bf16")
+    nrows = 16
+    while True:
+        t0 = time.perf_counter()
+        oracle.qmv_block_scaled(*args, rows=range(nrows), threads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s / 4 or nrows >= N:
+            break
+        nrows = min(N, nrows * 4)
+    return dt * 1e6 * (N / nrows), threads, f"{fmt} N={N} K={K} bf16: {nrows}/{N} rows, {dt:.3f}s"
 
 
 def _oracle_quantize_fp_sample(budget_s, threads):
@@ -1023,9 +1106,13 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="chain8")
     ap.add_argument("--no-shapes", action="store_true",
                     help="chain8 only: skip the per format / bits / shape lines")
+    ap.add_argument("--format", default="mxfp4",
+                    help="fmt_probe: the Track-1 format (a qmv_block_scaled name, e.g. mxfp4, nvfp8, int4)")
     ap.add_argument("--sets", type=lambda v: tuple(v.split(",")), default=None,
                     help="chain8: comma-separated subset of the shape sets " + ",".join(SHAPE_SETS))
     args = ap.parse_args()
+    FmtProbe.FMT = args.format
+    FmtProbe.name = f"bandwidth probe, {args.format} bf16, N=K=16384, M=1"
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
