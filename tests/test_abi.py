@@ -163,13 +163,20 @@ def test_format_info_of_every_format():
 
 def test_block_scaled_plans():
     """Every format plans on the few-rows or the row-tiled kernel, never on
-    the affine-only kernels; the FP formats reach the weight ring only when
-    forced (path 6), for one bf16 x row."""
+    the affine-only kernels; the FP formats with FP32 / FP16 block scales also
+    on the weight ring for one large bf16 x row (scales in the ring), the
+    others reach it only when forced (path 6)."""
     for name in q.FORMATS:
         fp = not name.startswith(("int", "mxint"))
+        wide_scales = q.qmv_format_info(name)["scale_bytes"] >= 2
         for (M, N, K) in [(1, 4, 1024), (1, 4096, 4096), (8, 14336, 4096), (1, 14336, 4096)]:
             plan = q.qmv_describe_plan(name, M, N, K, dtype="bf16")
-            assert plan.split()[0] in ("path=direct", "path=wide", "path=narrow"), (name, plan)
+            bits = q.qmv_format_info(name)["element_bits"]
+            ring_ok = fp and wide_scales and M == 1 and N * K * bits / 8 >= 10 * 1024 * 1024
+            assert plan.split()[0] in ("path=direct", "path=wide", "path=narrow") + (("path=tcf",) if ring_ok else ()), \
+                (name, plan)
+            if ring_ok:
+                assert "path=tcf" in plan and "scale_ring=1" in plan, (name, plan)
         q.qmv_force_config(6, -1, -1, -1)
         try:
             ring = q.qmv_describe_plan(name, 1, 14336, 4096, dtype="bf16")

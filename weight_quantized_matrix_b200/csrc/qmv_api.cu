@@ -317,15 +317,17 @@ bool tcb_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s
 // x tile holds (NP + 4) words of x~ pairs and two sums per unit (affine), or
 // UC + 4 fp32 x values per unit (fp: the block-scaled FP formats, whose
 // scales stay in global memory).
-bool tcf_shape(int N, int K, int bits, int G, bool w16, bool s16, TcbShape* ts, bool fp = false) {
+bool tcf_shape(int N, int K, int bits, int G, bool w16, bool s16, TcbShape* ts, bool fp = false, int fp_es = 1) {
     const int ub = tc_unit_bytes(bits);
     const int uc = ub * 8 / bits;
     const int SB = 4 * uc;
     if (K % SB != 0 || !w16) return false;
     if (((long long)K * bits / 8) % 16 != 0) return false;     // tensor copies: 16-byte rows
     if (!fp && G < uc) return false;                            // a unit lies in one group
-    if (fp) s16 = false;
-    const int es = 2;
+    // scale elements: affine 2 bytes (the ring serves bf16 x); FP: the
+    // format's block-scale bytes, one tile per stage (no biases)
+    const int es = fp ? fp_es : 2;
+    const int ntiles = fp ? 1 : 2;
     const int nps = fp ? uc + 4 : tc_np_of(bits) + 4;
     const int nsbk = K / SB;
     const int sms = device_sms();
@@ -373,7 +375,7 @@ bool tcf_shape(int N, int K, int bits, int G, bool w16, bool s16, TcbShape* ts, 
         *sbw = box0 * es;
         *sring = (s16 && ((long long)(K / G) * es) % 16 == 0 && *sbw % 16 == 0 && box0 <= 256 && rows <= 256) ? 1 : 0;
         const int pitch = s * 4 * ub;
-        *stage = rows * pitch + (*sring ? 2 * rows * *sbw : 0);
+        *stage = rows * pitch + (*sring ? ntiles * rows * *sbw : 0);
         return pitch;
     };
     const size_t red = (size_t)(qmv::kTcbStages + 1) * ncw * 16 * 4;
@@ -504,7 +506,7 @@ bool umma_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool 
 // Choose the launch shape.  Returns QMV_OK or an error (sizes too large).
 int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, bool w16, int batch, Plan* pl,
               bool s16 = true, bool gather = false, bool pair = false, bool x16 = true, bool qmm = false,
-              bool qkv = false, bool norm = false) {
+              bool qkv = false, bool norm = false, int fp_es = 1) {
     // pair (fused gate + up): N counts the 2N virtual rows; pair, Q / K / V
     // and the fused RMSNorm run on the row-tiled CUDA-core kernel only
     if (pair || qkv || norm) gather = true;
@@ -550,19 +552,22 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
     // (measured on B200: the fastest path for one bf16 x row from about 10 MB
     // of 2/3/4/5/6-bit weights; 8-bit codes take two fields each, and there
     // the register-streaming CUDA-core kernel is as fast)
-    // The block-scaled FP formats run on the same ring when forced (path 6):
-    // with their block scales read from global memory in every step, 8
-    // compute warps per SM hide that latency worse than the row-tiled
-    // kernel's 16 (measured on B200, MXFP4 16384^2: 150 us on the ring, 53 us
-    // row-tiled), so the picker keeps them on the row-tiled kernel.
+    // The block-scaled FP formats take the same ring, their block scales
+    // copied into each stage next to the codes.  Measured on B200 (M = 1,
+    // bf16, 8192^2 .. 16384^2 and the layer shapes): the ring wins for
+    // FP32- and FP16-scaled formats (NVFP8 16384^2 110 -> 95 us, 28672 x
+    // 4096 63 -> 44 us; FP4_F16 80 -> 63 us), where the row-tiled kernel's
+    // per-chunk scale loads weigh most, and loses a little for the
+    // byte-scaled ones (MXFP8-E4M3 16384^2 63 -> 66 us), which stay row-tiled.
     const bool fp_fam = fam == qmv::FAM_MXFP4 || fam == qmv::FAM_NVFP4 || fam == qmv::FAM_MXFP8 ||
                         fam == qmv::FAM_E2M1 || fam == qmv::FAM_E4M3 || fam == qmv::FAM_E5M2;
     const bool big = (double)N * K * fi.bits / 8.0 >= 10.0 * 1024 * 1024;
-    const bool fma_ring_pick = M == 1 && dtype == QMV_BF16 && aff && bits >= 2 && bits <= 6 && big;
+    const bool fma_ring_pick = M == 1 && dtype == QMV_BF16 && big &&
+                               (aff ? (bits >= 2 && bits <= 6) : (fp_fam && fp_es >= 2));
     if (!gather && (aff || fp_fam) && K > 0 && M == 1 && dtype == QMV_BF16 &&
         (g_forced.path == 6 || (g_forced.path < 0 && fma_ring_pick))) {
         TcbShape ts;
-        if (tcf_shape(N, K, fi.bits, G_of_plan, w16, aff && s16, &ts, !aff)) {
+        if (tcf_shape(N, K, fi.bits, G_of_plan, w16, s16, &ts, !aff, fp_es)) {
             pl->maxm = 1; pl->R = 1; pl->wide = 1; pl->tc = 4; pl->npass = 0;
             pl->wk = ts.wk; pl->wr = ts.wr; pl->tile_iters = ts.tsb; pl->sps = ts.sps; pl->pitch = ts.pitch;
             pl->spb = 1; pl->sring = ts.sring; pl->soff = ts.soff; pl->boff = ts.boff; pl->sbw = ts.sbw;
@@ -770,6 +775,30 @@ bool encode_scale_map(CUtensorMap* m, const void* base, int dtype, long long KG,
            CUDA_SUCCESS;
 }
 
+// The same for block scales of 1, 2 or 4 bytes (the FP formats' E8M0 / E4M3
+// bytes, FP16 or FP32), copied as raw elements.
+bool encode_scale_map_es(CUtensorMap* m, const void* base, int es, long long KG, int N, int batch, int box0, int rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const CUtensorMapDataType dt = es == 4 ? CU_TENSOR_MAP_DATA_TYPE_UINT32
+                                 : es == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16
+                                           : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const cuuint64_t dims[3] = {(cuuint64_t)KG, (cuuint64_t)N, (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)KG * es, (cuuint64_t)KG * es * (cuuint64_t)N};
+    const cuuint32_t box[3] = {(cuuint32_t)box0, (cuuint32_t)rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// Bytes of one block scale of an FP family (skind for the run-time-scaled ones).
+int fp_scale_bytes(int fam, int skind) {
+    if (fam == qmv::FAM_E2M1 || fam == qmv::FAM_E4M3 || fam == qmv::FAM_E5M2 || fam == qmv::FAM_SINT)
+        return skind == qmv::SK_F32 ? 4 : skind == qmv::SK_F16 ? 2 : 1;
+    return 1;
+}
+
 int run(int fam, const void* x, const void* w, const void* scales, const void* biases,
         const float* gscale, void* y, int M, int N, int K, int bits, int G, int dtype, int batch,
         int x_batched, void* stream, const int* ids = nullptr, int n_experts = 0, bool qmm = false,
@@ -777,9 +806,12 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     const long long row_bytes = (long long)K * fmt_info(fam, bits).bits / 8;
     Plan pl;
     const bool w16 = aligned(w, 16);
-    const bool s16 = fam == qmv::FAM_AFFINE && aligned(scales, 16) && aligned(biases, 16);
+    const bool aff = fam == qmv::FAM_AFFINE;
+    const bool s16 = aligned(scales, 16) && (!aff || aligned(biases, 16));
     const bool x16 = aligned(x, 16) && ((size_t)K * elem_bytes(dtype)) % 16 == 0;
-    int st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, s16, ids != nullptr, false, x16, qmm);
+    const int fes = fp_scale_bytes(fam, skind);
+    int st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, s16, ids != nullptr, false, x16, qmm, false,
+                       false, fes);
     if (st != QMV_OK) return st;
     // M > 8 (qmm): only the tensor-memory kernel and the tensor-core ring take it
     if (M > QMV_MAX_M && pl.tc != 5 && pl.tc != 2) return QMV_EUNSUPPORTED;
@@ -795,11 +827,19 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     }
     const bool ring = pl.tc == 2 || pl.tc == 4;        // the weight-ring kernels
     if (ring && pl.sring) {
-        const int box0 = pl.sbw / elem_bytes(dtype), rows = 16 * pl.wr;
-        if (!encode_scale_map(&p.smap, scales, dtype, K / G, N, batch, box0, rows) ||
-            !encode_scale_map(&p.bmap, biases, dtype, K / G, N, batch, box0, rows)) {
+        const int rows = 16 * pl.wr;
+        bool okm;
+        if (aff) {
+            const int box0 = pl.sbw / elem_bytes(dtype);
+            okm = encode_scale_map(&p.smap, scales, dtype, K / G, N, batch, box0, rows) &&
+                  encode_scale_map(&p.bmap, biases, dtype, K / G, N, batch, box0, rows);
+        } else {
+            okm = encode_scale_map_es(&p.smap, scales, fes, K / G, N, batch, pl.sbw / fes, rows);
+        }
+        if (!okm) {
             cudaGetLastError();
-            st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, false);   // scales from global memory
+            st = make_plan(fam, M, N, K, bits, G, dtype, w16, batch, &pl, false, false, false, x16, qmm, false, false,
+                           fes);                                          // scales from global memory
             if (st != QMV_OK) return st;
         }
     }
@@ -1355,7 +1395,7 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
                       char* buf, int buflen) {
     if (!buf || buflen <= 0) return QMV_EINVAL;
     if (M < 1 || M > QMV_QMM_MAX_M || N < 1 || K < 0) return QMV_EINVAL;
-    int fam, G;
+    int fam, G, fes = 1;
     if (family == 0) {
         if (check_affine(bits, group_size) != QMV_OK) return QMV_EUNSUPPORTED;
         fam = qmv::FAM_AFFINE;
@@ -1364,6 +1404,7 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
         if (family - 100 >= QMV_FMT_COUNT) return QMV_EUNSUPPORTED;
         const BsFmt& f = kBsFmt[family - 100];
         fam = f.fam; bits = f.bits; G = f.block;
+        fes = scale_bytes_of(f.skind);
     } else {
         fam = fp_family(family - 1);
         if (fam < 0) return QMV_EUNSUPPORTED;
@@ -1374,7 +1415,7 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
     const bool qmm = M > QMV_MAX_M;
     if (qmm && fam != qmv::FAM_AFFINE) return QMV_EINVAL;
     int st = make_plan(fam, M, N, K, bits, G, dtype, w_align16 != 0, 1, &pl, true, false, false, true,
-                       qmm && qmm_prefers_umma(N));
+                       qmm && qmm_prefers_umma(N), false, false, fes);
     if (st != QMV_OK) return st;
     if (qmm && pl.tc != 5) {
         // qmm: chunks of x rows, each through the qmv plan of its size

@@ -32,8 +32,9 @@
 // conversion to f16x2 and widened to fp32 (exact), against x staged as plain
 // fp32 rows of UC + 4 floats per unit (the pad keeps the 8 lanes of a
 // shared-memory phase on distinct banks); the unit's one or two block scales
-// (blocks of 16 or 32 codes, any scale type) come from global memory, and
-// NVFP4's global scale multiplies the stored row sum.
+// (blocks of 16 or 32 codes, any scale type) travel in the ring as one more
+// tensor-copy tile per stage (p.sring; else from global memory), and NVFP4's
+// global scale multiplies the stored row sum.
 #pragma once
 
 #include "qmv_tcb.cuh"
@@ -105,6 +106,21 @@ __device__ __forceinline__ void fpr_unit(const uint32_t (&w)[4], const float* xf
     }
 }
 
+// Block scale of an FP family at element index i of a ring scale tile row.
+template <int FAM>
+__device__ __forceinline__ float fpr_ring_scale(const unsigned char* row, int i, int skind) {
+    if constexpr (FAM == FAM_NVFP4) return e4m3_value(row[i]);
+    else if constexpr (FAM == FAM_MXFP4 || FAM == FAM_MXFP8) return e8m0_value(row[i]);
+    else {
+        switch (skind) {
+            case SK_E8M0: return e8m0_value(row[i]);
+            case SK_E4M3: return e4m3_value(row[i]);
+            case SK_F32: return reinterpret_cast<const float*>(row)[i];
+            default: return __half2float(reinterpret_cast<const __half*>(row)[i]);
+        }
+    }
+}
+
 // Block scale of an FP family at element index i of the scale array.
 template <int FAM>
 __device__ __forceinline__ float fpr_scale(const Params& p, long long i) {
@@ -137,7 +153,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
     const int pitch = p.pitch;
     const int sbw = p.sbw;
     const bool sring = p.sring != 0;
-    const int stage_bytes = ROWS * pitch + (sring ? 2 * ROWS * sbw : 0);
+    const int stage_bytes = ROWS * pitch + (sring ? (AFF ? 2 : 1) * ROWS * sbw : 0);   // FP: no bias tile
     const int TSB = p.tile_iters;
     const int TU = TSB * 4;
     const int G = p.G;
@@ -172,7 +188,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
     if (warp == NCW) {                               // the producer warp
         grid_launch_dependents();
         const uint32_t ring0 = smem_addr(ring);
-        const uint32_t stage_tx = (uint32_t)ROWS * ((uint32_t)pitch + (sring ? 2u * (uint32_t)sbw : 0u));
+        const uint32_t stage_tx = (uint32_t)ROWS * ((uint32_t)pitch + (sring ? (AFF ? 2u : 1u) * (uint32_t)sbw : 0u));
         int it = 0;
         bool ok = true;
         for (int rb = blockIdx.x; rb < nrb && ok; rb += gridDim.x) {
@@ -192,7 +208,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
                     if (sring) {
                         const int g0 = ((ks * S) << gmul) >> gdiv;
                         tensor_copy_3d(st0 + (uint32_t)p.soff, &p.smap, g0, rb * ROWS, bz, full(slot));
-                        tensor_copy_3d(st0 + (uint32_t)p.boff, &p.bmap, g0, rb * ROWS, bz, full(slot));
+                        if (AFF) tensor_copy_3d(st0 + (uint32_t)p.boff, &p.bmap, g0, rb * ROWS, bz, full(slot));
                     }
                 }
                 __syncwarp();
@@ -314,13 +330,20 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
                                 const uint32_t w[4] = {a.x, a.y, a.z, a.w};
                                 float2 p0 = make_float2(0.f, 0.f), p1 = make_float2(0.f, 0.f);
                                 fpr_unit<FAM, B>(w, xf, p0, p1);
-                                const long long si = valid ? srow[i] + k0 / G : srow[i];
-                                const float s0 = fpr_scale<FAM>(p, si);
-                                float yn = fmaf(s0, p0.x + p0.y, Y[i]);
-                                if constexpr (B == 4) {
-                                    const float s1 = G == 16 ? fpr_scale<FAM>(p, si + 1) : s0;
-                                    yn = fmaf(s1, p1.x + p1.y, yn);
+                                float s0, s1;
+                                if constexpr (RING) {
+                                    // the unit's scale(s) in this stage's tile
+                                    const unsigned char* sr = srow0 + (size_t)(4 * i) * sbw;
+                                    const int sidx = (sbl * SB + t * UC) / G;
+                                    s0 = fpr_ring_scale<FAM>(sr, sidx, p.skind);
+                                    s1 = (B == 4 && G == 16) ? fpr_ring_scale<FAM>(sr, sidx + 1, p.skind) : s0;
+                                } else {
+                                    const long long si = valid ? srow[i] + k0 / G : srow[i];
+                                    s0 = fpr_scale<FAM>(p, si);
+                                    s1 = (B == 4 && G == 16) ? fpr_scale<FAM>(p, si + 1) : s0;
                                 }
+                                float yn = fmaf(s0, p0.x + p0.y, Y[i]);
+                                if constexpr (B == 4) yn = fmaf(s1, p1.x + p1.y, yn);
                                 Y[i] = valid ? yn : Y[i];
                             }
                             return;
@@ -360,7 +383,7 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
                             Y[i] = valid ? yn : Y[i];
                         }
                     };
-                    if (AFF && sring) {
+                    if (sring) {
                         for (int j = wkid; j < nsteps; j += wk) step(std::true_type{}, j);
                     } else {
                         for (int j = wkid; j < nsteps; j += wk) step(std::false_type{}, j);
