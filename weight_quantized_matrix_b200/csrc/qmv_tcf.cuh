@@ -78,10 +78,12 @@ __device__ __forceinline__ void tcf_unit(std::integer_sequence<int, Q...>, const
 //   us    TU * 2 floats         {sum(x), sum(x~)} per unit (affine only)
 //   red   (STAGES + 1) * NCW * 16 floats   per-warp row sums, by row block
 // MAXT = 32 * (NCW + 1): NCW = wk * wr in {8, 12} compute warps + the producer.
-// FP unit: Y[i] += (block scale) * sum of x * element over the unit, with the
-// unit's codes w (16 bytes) and its x row xf (UC fp32 values).
+// FP unit: the sums of x * element over the unit's halves (p1 only for 32
+// E2M1 codes), with the unit's codes w (16 bytes) and its x values xf (UC
+// fp32 values, held in registers for the lane's 4 rows).
 template <int FAM, int B>
-__device__ __forceinline__ void fpr_unit(const uint32_t (&w)[4], const float* xf, float2& p0, float2& p1) {
+__device__ __forceinline__ void fpr_unit(const uint32_t (&w)[4], const float (&xf)[B == 4 ? 32 : 16], float2& p0,
+                                         float2& p1) {
     if constexpr (B == 4) {
         // 32 E2M1 codes: codes 0..15 (words 0, 1) into p0, 16..31 into p1
 #pragma unroll
@@ -89,7 +91,7 @@ __device__ __forceinline__ void fpr_unit(const uint32_t (&w)[4], const float* xf
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
                 const float2 e = half2_bits_to_float2(cvt_e2m1x2(w[wi] >> (8 * b)));
-                const float2 xv = *reinterpret_cast<const float2*>(xf + 8 * wi + 2 * b);
+                const float2 xv = make_float2(xf[8 * wi + 2 * b], xf[8 * wi + 2 * b + 1]);
                 if (wi < 2) p0 = fma2(xv, e, p0);
                 else p1 = fma2(xv, e, p1);
             }
@@ -100,7 +102,7 @@ __device__ __forceinline__ void fpr_unit(const uint32_t (&w)[4], const float* xf
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const float2 e = half2_bits_to_float2(cvt_fp8x2<FAM>(w[wi] >> (16 * h)));
-                const float2 xv = *reinterpret_cast<const float2*>(xf + 4 * wi + 2 * h);
+                const float2 xv = make_float2(xf[4 * wi + 2 * h], xf[4 * wi + 2 * h + 1]);
                 p0 = fma2(xv, e, p0);
             }
     }
@@ -321,7 +323,15 @@ __global__ void __launch_bounds__(MAXT, 1) qmv_tcf_kernel(const __grid_constant_
                         const bool valid = sb < send;
                         const int ut = valid ? (sb - t0) * 4 + t : 0;   // unit within the x tile
                         if constexpr (!AFF) {
-                            const float* xf = reinterpret_cast<const float*>(xs + (size_t)ut * NPS);
+                            float xf[UC];                 // the unit's x, once for the 4 rows
+                            {
+                                const float4* xp = reinterpret_cast<const float4*>(xs + (size_t)ut * NPS);
+#pragma unroll
+                                for (int c = 0; c < UC / 4; ++c) {
+                                    const float4 v = xp[c];
+                                    xf[4 * c] = v.x; xf[4 * c + 1] = v.y; xf[4 * c + 2] = v.z; xf[4 * c + 3] = v.w;
+                                }
+                            }
                             const unsigned char* src0 = rows0 + (8 * j + u8) * UB;
                             const long long k0 = (long long)sb * SB + t * UC;           // the unit's first code
 #pragma unroll
