@@ -932,7 +932,9 @@ def run_ours(args, rank, world, local_rank):
         # the metric's breakdown per format / bits / shape; not part of `value`
         out["shapes"] += shape_lines(q, torch, dev, stream, flush, flush_rd, peak, args.sets)
     if rank == 0:
-        out["cpu_baseline"] = cpu_baseline(args.workload)
+        out["cpu_baseline"] = (cpu_baseline(args.workload) if not args.no_cpu_baseline
+                               else {"value": None, "unit": "us/call", "kind": "oracle",
+                                     "sample": "skipped (--no-cpu-baseline)"})
         print(json.dumps(out), flush=True)
 
 
@@ -1106,6 +1108,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="chain8")
     ap.add_argument("--no-shapes", action="store_true",
                     help="chain8 only: skip the per format / bits / shape lines")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip timing the oracle on the host cores (profiling runs)")
     ap.add_argument("--format", default="mxfp4",
                     help="fmt_probe: the Track-1 format (a qmv_block_scaled name, e.g. mxfp4, nvfp8, int4)")
     ap.add_argument("--sets", type=lambda v: tuple(v.split(",")), default=None,
