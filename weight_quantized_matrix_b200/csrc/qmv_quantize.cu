@@ -26,9 +26,18 @@
 // |Q|.  When t is
 // farther than that from every half-integer, t and d round (and clamp) to the
 // same code.  The kernels test the clamped t against the conservative margin
-// (2^B - 1) * 2^-21 and redo a weight with the division when it is closer, or
-// when the reciprocal is not a normal number (a scale beyond 2^125 or below
-// 2^-125): the codes are those of the division, bit for bit.
+// (2^B - 1) * 2^-21 and decide a weight that is closer exactly (near_code):
+// with h the half-integer next to t, the residual diff - h * scale_T from one
+// FMA has the sign (and zeroness) of the exact residual, since the FMA rounds
+// the exact value once.  Zero means the quotient IS h, which rounds to the
+// even neighbour; a residual larger than scale_T * 2^(B-23) puts the quotient
+// more than half an ulp of h away, on the side its sign gives, so its
+// correctly rounded value rounds the same way; anything closer, a scale
+// outside [2^-100, 2^100] (where the residual could underflow) or a
+// reciprocal that is not a normal number takes the IEEE division.  Exact
+// half-integer quotients are common with bf16 / f16 weights (few mantissa
+// bits), so the FMA test keeps them off the division.  The codes are those of
+// the division, bit for bit.
 //
 // Two forms: quantize_affine_tiles (aligned buffers: a warp double-buffers 32
 // groups at a time through shared memory for coalesced loads and stores) and
@@ -64,25 +73,28 @@ template <> struct QT<__nv_bfloat16> {
 // Codes of v[0..E): (v - bias_T) * inv clamped to [0, QMAX], then rounded to
 // the nearest integer, ties to even, by adding 2^23: an fp32 in [2^23, 2^24)
 // has unit spacing, so the sum is 2^23 plus the rounded value and its low bits
-// are the code.  Two values per packed fp32x2 op.  Returns true when some
-// clamped product lies within QMAX * 2^-21 of a half-integer, where it might
-// round differently from the quotient (the caller redoes those with
-// exact_code).
+// are the code.  Two values per packed fp32x2 op.  Returns the mask of the
+// values whose clamped product lies within QMAX * 2^-21 of a half-integer,
+// where it might round differently from the quotient (the caller decides
+// those with near_code), and leaves the clamped products in c.
 template <int QMAX, int E>
-__device__ __forceinline__ bool quantize_codes(const float* v, float bT, float inv, uint32_t* q) {
-    static_assert(E % 2 == 0, "pairs");
+__device__ __forceinline__ uint32_t quantize_codes(const float* v, float bT, float inv, uint32_t* q, float* c) {
+    static_assert(E % 2 == 0 && E <= 32, "pairs");
     constexpr float EDGE = 0.5f - (float)QMAX * 4.76837158203125e-07f;      // 0.5 - QMAX * 2^-21
-    bool near = false;
+    uint32_t near = 0;
 #pragma unroll
     for (int e = 0; e < E; e += 2) {
         const float2 d = mul2(add2(make_float2(v[e], v[e + 1]), make_float2(-bT, -bT)), make_float2(inv, inv));
-        const float2 c = make_float2(fminf(fmaxf(d.x, 0.0f), (float)QMAX), fminf(fmaxf(d.y, 0.0f), (float)QMAX));
-        const float2 r = add2(c, make_float2(8388608.0f, 8388608.0f));
+        const float2 cc = make_float2(fminf(fmaxf(d.x, 0.0f), (float)QMAX), fminf(fmaxf(d.y, 0.0f), (float)QMAX));
+        const float2 r = add2(cc, make_float2(8388608.0f, 8388608.0f));
         q[e] = __float_as_uint(r.x) & (uint32_t)QMAX;
         q[e + 1] = __float_as_uint(r.y) & (uint32_t)QMAX;
-        // c minus its rounded value (both exact): in [-0.5, 0.5]
-        const float2 f = add2(c, add2(make_float2(-r.x, -r.y), make_float2(8388608.0f, 8388608.0f)));
-        near |= (fabsf(f.x) >= EDGE) | (fabsf(f.y) >= EDGE);
+        c[e] = cc.x;
+        c[e + 1] = cc.y;
+        // cc minus its rounded value (both exact): in [-0.5, 0.5]
+        const float2 f = add2(cc, add2(make_float2(-r.x, -r.y), make_float2(8388608.0f, 8388608.0f)));
+        near |= (fabsf(f.x) >= EDGE ? 1u : 0u) << e;
+        near |= (fabsf(f.y) >= EDGE ? 1u : 0u) << (e + 1);
     }
     return near;
 }
@@ -94,6 +106,23 @@ __device__ __forceinline__ uint32_t exact_code(float v, float bT, float sT) {
     if (sT == 0.0f) return 0u;
     const float r = rintf(__fdiv_rn(__fsub_rn(v, bT), sT));
     return !(r > 0.0f) ? 0u : r >= (float)QMAX ? (uint32_t)QMAX : (uint32_t)r;
+}
+
+// The code of a weight whose product t (unclamped: a clamped product is never
+// near a half-integer) lies near the half-integer h = floor(t) + 1/2, decided
+// by the sign of the exact residual diff - h * sT (see the header).
+template <int QMAX>
+__device__ __forceinline__ uint32_t near_code(float v, float bT, float sT, float t) {
+    constexpr float ULP_MAX = (float)(QMAX + 1) * 1.1920928955078125e-07f;  // 2^(B-23) >= ulp(h)
+    if (sT >= 7.888609052210118e-31f && sT <= 1.2676506002282294e+30f) {   // 2^-100 .. 2^100
+        const float diff = __fsub_rn(v, bT);
+        const float k = floorf(t);
+        const float e = fmaf(-(k + 0.5f), sT, diff);
+        const uint32_t ki = (uint32_t)k;
+        if (e == 0.0f) return (ki & 1u) ? ki + 1u : ki;                    // the quotient is h: even
+        if (fabsf(e) > sT * ULP_MAX) return e > 0.0f ? ki + 1u : ki;
+    }
+    return exact_code<QMAX>(v, bT, sT);
 }
 
 // Whether the reciprocal fast path applies to a group: a zero scale (every
@@ -162,8 +191,9 @@ __global__ void __launch_bounds__(256) quantize_affine_kernel(const T* __restric
     auto put = [&](float v) {
         const float two[2] = {v, v};
         uint32_t qq[2];
-        const bool near = quantize_codes<QMAX, 2>(two, bT, inv, qq);
-        const uint32_t q = (near || !fast) ? exact_code<QMAX>(v, bT, sT) : qq[0];
+        float cc[2];
+        const uint32_t near = quantize_codes<QMAX, 2>(two, bT, inv, qq, cc);
+        const uint32_t q = !fast ? exact_code<QMAX>(v, bT, sT) : near ? near_code<QMAX>(v, bT, sT, cc[0]) : qq[0];
         acc |= (uint64_t)q << nb;
         nb += B;
         if (nb >= 32) {
@@ -328,10 +358,26 @@ __global__ void __launch_bounds__(32) quantize_affine_tiles(const T* __restrict_
                     float v[E];
                     widen16<T>(my[blk * (32 / E) + cc], v);
                     uint32_t q[E];
-                    const bool near = quantize_codes<QMAX, E>(v, bT, inv, q);
-                    if (near || !fast) {
-#pragma unroll 1
+                    float cv[E];
+                    uint32_t near = quantize_codes<QMAX, E>(v, bT, inv, q, cv);
+                    if (!fast) {
+                        // (fully unrolled: a run-time index would move v[] and
+                        // q[] to local memory for the whole loop)
+#pragma unroll
                         for (int e = 0; e < E; ++e) q[e] = exact_code<QMAX>(v[e], bT, sT);
+                    } else {
+                        while (near) {                       // the few values near a half-integer
+                            const int e = __ffs(near) - 1;
+                            near &= near - 1u;
+                            float ve = v[0], ce = cv[0];
+#pragma unroll
+                            for (int j = 1; j < E; ++j)
+                                if (j == e) { ve = v[j]; ce = cv[j]; }
+                            const uint32_t qe = near_code<QMAX>(ve, bT, sT, ce);
+#pragma unroll
+                            for (int j = 0; j < E; ++j)
+                                if (j == e) q[j] = qe;
+                        }
                     }
 #pragma unroll
                     for (int e = 0; e < E; ++e) {
