@@ -97,7 +97,14 @@ def source_hash():
     return h.hexdigest()[:16]
 
 
-def traffic_for(kernel_key):
+def traffic_key(workload, fmt, kernel_key):
+    """The traffic.json key of one workload's dominant kernel: the same kernel
+    key moves different bytes in different workloads (and formats)."""
+    w = f"{workload}:{fmt}" if workload == "fmt_probe" else workload
+    return f"{w} | {kernel_key}"
+
+
+def traffic_for(key):
     """dram bytes per launch from the committed ncu summary, only while the
     kernel sources are unchanged since the capture."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -107,7 +114,7 @@ def traffic_for(kernel_key):
         d = json.load(open(p))
     except ValueError:
         return None
-    e = d.get(kernel_key)
+    e = d.get(key)
     if not e or e.get("src_sha") != source_hash():
         return None
     return e.get("dram_bytes_per_launch")
@@ -911,7 +918,7 @@ def run_ours(args, rank, world, local_rank):
         k["ms"] += ms; k["launches"] += n; k["bytes"] += b
     dom_plan, dom = max(by_kernel.items(), key=lambda kv: kv[1]["ms"])
     achieved = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
-    traffic = traffic_for(dom_plan)
+    traffic = traffic_for(traffic_key(args.workload, args.format, dom_plan))
     h2d, d2h = wl.h2d_d2h()
     out = {
         "metric": METRIC, "value": round(us_per_call, 4), "unit": "us/call", "n_gpus": world,
