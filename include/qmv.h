@@ -460,16 +460,19 @@ int qmv_device_fault(unsigned int* code, int clear);
 
 /*
  * qmv_force_config -- benchmarking / testing knob: pin the launch shape used
- * by every later call in this process.  path: 6 = CUDA-core kernel with the
- * weight ring (affine, one bf16 x row), 5 = few-rows latency kernel, 4 =
+ * by every later call in this process.  path: 8 = per-group tensor-core
+ * kernel with the weight ring (affine 4-bit, f16 / bf16 x, up to 32 x rows,
+ * K a multiple of 8 groups), 7 = tensor-memory (tcgen05) kernel (qmm), 6 =
+ * CUDA-core kernel with the weight ring (one bf16 x row), 5 = few-rows
+ * latency kernel, 4 =
  * tensor-core kernel with the weight ring, 3 = tensor-core kernel (4 and 3 for
  * affine formats; paths fall back to automatic where their size rules do not
  * hold), 1 = CUDA-core kernel with wide (16-byte) chunk loads, 0 = CUDA-core
  * kernel with 4-byte chunks, -1 = automatic; rows_per_warp in {1,2,4} or -1
  * (CUDA-core kernel); warps_k (warps that split K inside a block) and
  * warps_rows (16-row tiles per block) up to 12 each, or -1; the weight-ring
- * kernels run warps_k * warps_rows in {8, 12} compute warps and a producer
- * warp.
+ * kernels run warps_k * warps_rows in {8, 12} compute warps (path 8: 8 or 16,
+ * warps_k in {1, 2, 4, 8}) and a producer warp.
  * Unsupported combinations fall back to automatic for that field.
  * NOT FOR PRODUCTION USE: this is process-wide state for the parity tests and
  * the benchmark's sweeps; it is not thread-safe with concurrent calls and

@@ -6,9 +6,9 @@ copy).  Nothing ever completes that stage's barrier, so the block's consumer
 warps give up their bounded wait (about one second) and OR code 1 into the
 device fault word, and the producer gives up waiting for its own copies on that
 stage and ORs code 4.  The kernel returns normally, nothing is left in flight,
-and the next call on the same context is correct again.  Covered for both
-weight-ring kernels: the CUDA-core ring (one bf16 x row) and the tensor-core
-ring (several x rows).
+and the next call on the same context is correct again.  Covered for the
+three weight-ring kernels: the CUDA-core ring (one bf16 x row), the
+tensor-core ring and the per-group tensor-core ring (several x rows).
 """
 from __future__ import annotations
 
@@ -40,7 +40,7 @@ def _clean(q):
     q.qmv_device_fault(clear=True)
 
 
-@pytest.mark.parametrize("path,M,want", [(6, 1, "path=tcf"), (4, 4, "path=tcb")])
+@pytest.mark.parametrize("path,M,want", [(6, 1, "path=tcf"), (4, 4, "path=tcb"), (8, 4, "path=tcg")])
 def test_ring_wait_runs_out_and_reports(q, path, M, want):
     N, K, bits, group = 333, 4096, 4, 64
     q.qmv_force_config(path, -1, -1, -1)

@@ -25,7 +25,7 @@ from gpu_util import compare, oracle_affine, oracle_fp, require_cuda, run_affine
 pytestmark = pytest.mark.gpu
 
 N, K = 16384, 2560
-PATHS = {0: "narrow", 1: "wide", 3: "tc", 4: "tcb", 5: "direct", 6: "tcf"}
+PATHS = {0: "narrow", 1: "wide", 3: "tc", 4: "tcb", 5: "direct", 6: "tcf", 8: "tcg"}
 PREC_FLOOR_FRAC = 0.25
 
 
@@ -56,6 +56,9 @@ def _cases():
                     out.append((path, M, bits, dtype))
     for bits in (2, 3, 4, 5, 6):
         out.append((6, 1, bits, "bf16"))       # the CUDA-core ring: one bf16 x row
+    for M in (1, 8):
+        for dtype in ("bf16", "f16"):
+            out.append((8, M, 4, dtype))       # the per-group tensor-core ring: 4-bit, 16-bit x
     return out
 
 

@@ -1,6 +1,7 @@
 """GPU parity of the small-M qmm (qmv_qmm_affine: up to 64 x rows, as chunks of
-32, 16 or 8 rows through the qmv kernels; forced, one launch of the
-tensor-memory kernel) against the oracle, element by element, within the qmv
+32, 16 or 8 rows through the qmv kernels -- the per-group tensor-core ring for
+4-bit codes; forced or for few row tiles, one launch of the tensor-memory
+kernel) against the oracle, element by element, within the qmv
 output tolerance.  Row counts cover one chunk plus a ragged remainder, several
 full chunks and the maximum of 64."""
 from __future__ import annotations
@@ -56,19 +57,18 @@ def test_qmm_layer_shape(q):
 @pytest.mark.parametrize("forced", [-1, 7])
 def test_qmm_layer_shapes(q, M, shape, forced):
     """qmm beyond 8 rows on the 7B gate+up and down shapes (4-bit g64 bf16),
-    sampled rows: by default chunks of up to 32 rows through the tensor-core
-    ring kernel for the tall gate+up, one launch of the tensor-memory kernel
-    for the down projection (few row tiles) and whenever forced (path 7),
-    where x fits its shared memory."""
+    sampled rows: by default chunks of up to 32 rows through the per-group
+    tensor-core ring kernel; forced (path 7), one launch of the tensor-memory
+    kernel where x fits its shared memory."""
     N, K = shape
     q.qmv_force_config(forced, -1, -1, -1)
     try:
         plan = q.qmv_describe_plan("affine", M, N, K, 4, 64, "bf16")
         fits = M * K <= 33 * 14336          # 64 x rows over K = 14336: x needs more than 16 CTAs
-        if forced == 7 or N <= 5120:
+        if forced == 7:
             assert plan.startswith("path=umma") == fits, plan
         else:
-            assert plan.startswith("path=chunked16 ") and "path=tcb" in plan, plan
+            assert plan.startswith(f"path=chunked{16 if M <= 16 else 32} ") and "path=tcg" in plan, plan
         c = synth.affine_case(M, N, K, 4, 64, "bf16", seed=M * 100 + K)
         y = _run(q, c, M, N, K)
     finally:
@@ -80,13 +80,20 @@ def test_qmm_layer_shapes(q, M, shape, forced):
 
 
 def test_qmm_plans(q):
-    """Tall matrices: 32 rows a chunk where a super-block holds one group
-    (4-bit g128), 16 where it holds two (g64); f16 likewise through the ring
-    kernel.  Few row tiles, bf16: one tensor-memory launch."""
-    assert q.qmv_describe_plan("affine", 64, 8000, 1024, 4, 128, "bf16").startswith("path=chunked32 chunks=2 ")
-    assert q.qmv_describe_plan("affine", 33, 8000, 1024, 4, 64, "bf16").startswith("path=chunked16 chunks=3 ")
-    assert q.qmv_describe_plan("affine", 12, 8000, 1024, 4, 64, "f16").startswith("path=chunked16 chunks=1 ")
-    assert q.qmv_describe_plan("affine", 33, 1000, 1024, 4, 64, "bf16").startswith("path=umma ")
+    """4-bit codes with bf16 / f16 x: 16 or 32 rows a launch through the
+    per-group tensor-core ring.  Other widths, tall matrices: 32 rows a chunk
+    through the tensor-core ring where a super-block holds one group (g128),
+    16 where it holds two (g64).  Few row tiles, bf16: one tensor-memory
+    launch."""
+    plan = lambda M, N, K, b, g, dt: q.qmv_describe_plan("affine", M, N, K, b, g, dt)
+    for args, want in [((64, 8000, 1024, 4, 128, "bf16"), "path=chunked32 chunks=2 path=tcg "),
+                       ((33, 8000, 1024, 4, 64, "bf16"), "path=chunked32 chunks=2 path=tcg "),
+                       ((12, 8000, 1024, 4, 64, "f16"), "path=chunked16 chunks=1 path=tcg "),
+                       ((33, 1000, 1024, 4, 64, "bf16"), "path=chunked32 chunks=2 path=tcg "),
+                       ((64, 8000, 1024, 3, 128, "bf16"), "path=chunked32 chunks=2 path=tcb "),
+                       ((33, 8000, 1024, 3, 64, "bf16"), "path=chunked16 chunks=3 path=tcb "),
+                       ((33, 1000, 1024, 8, 64, "bf16"), "path=umma ")]:
+        assert plan(*args).startswith(want), (args, plan(*args))
 
 
 def test_qmm_rejects_more_than_64_rows(q):

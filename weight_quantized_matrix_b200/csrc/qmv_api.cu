@@ -182,6 +182,79 @@ bool tc_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, TcShape
     return ts->gx <= 0x7FFFFFFFLL && ts->smem <= (size_t)qmv::kMaxSmem;
 }
 
+// ---- per-group tensor-core ring launch shape (qmv_tcg.cuh) ----------------------
+// 4-bit codes, bf16 / f16 x, G in {32, 64, 128}, K a multiple of 8 groups (a
+// ring stage is 8 groups; the scale tiles' tensor maps need 16-byte row
+// strides), up to 32 x rows (nt n-tiles of 8).  Row blocks of 16 * wr rows over
+// a persistent grid, wk in {1, 2, 4, 8} k-warps, 8 to 16 consumer warps.  Shared
+// memory: a ring of about 72 KB (2..8 stages), x staged for the whole K when it
+// fits beside a ring of at least 3 stages, else in tiles of whole stages.
+// The shape minimises, measured on B200 (M = 8, the 7B layer's projections):
+//   rounds of row blocks over the SMs x rows per block
+//   x (1 + log2(wk) / 4)     (a k-warp's fixed cost per stage: fewer, longer
+//                              k-ranges win once the SMs are busy)
+//   x 1.25 below 12 consumer warps (more warps hide more latency)
+//   x rounds again when x is tiled (staged anew for every row block)
+struct TcgShape { int nt, wk, wr, nst, sby, xt; long long gx; size_t smem; };
+
+bool tcg_plan_smem(int nt, int wk, int wr, int K, int G, TcgShape* ts) {
+    const int nc = 8 * nt;
+    const int rows = 16 * wr;
+    const int sby = ((rows * (4 * G + 32) + 1023) / 1024) * 1024;      // codes + scale and bias tiles
+    int nst = (72 * 1024) / sby;
+    nst = nst < 2 ? 2 : (nst > 8 ? 8 : nst);
+    const long long nks = K / (8 * G);
+    const size_t red = (size_t)(wr * wk) * 16 * nc * 4;
+    const size_t per_stage_x = (size_t)(G / 2) * nt * 32 * 8 + (size_t)8 * nc * 4;
+    const size_t lim = (size_t)qmv::kMaxSmem;
+    const size_t whole = 2048 + red + (size_t)nks * per_stage_x;
+    long long xt;
+    if (whole + 3 * (size_t)sby <= lim) {
+        const long long fit = (long long)((lim - whole) / sby);
+        if (fit < nst) nst = (int)fit;
+        xt = nks;
+    } else {
+        const size_t fixed = 2048 + red + (size_t)nst * sby;
+        if (fixed + per_stage_x > lim) return false;
+        xt = (long long)((lim - fixed) / per_stage_x);
+        if (xt > nks) xt = nks;
+    }
+    ts->nt = nt; ts->wk = wk; ts->wr = wr; ts->nst = nst; ts->sby = sby; ts->xt = (int)xt;
+    ts->smem = 2048 + (size_t)nst * sby + (size_t)xt * per_stage_x + red;
+    return ts->smem <= lim;
+}
+
+bool tcg_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s16, TcgShape* ts) {
+    if (bits != 4 || (dtype != QMV_BF16 && dtype != QMV_F16)) return false;
+    if (G != 32 && G != 64 && G != 128) return false;
+    if (M < 1 || M > 32 || N < 1 || K <= 0 || K % (8 * G) != 0 || !w16 || !s16) return false;
+    const int nt = M <= 8 ? 1 : M <= 16 ? 2 : 4;
+    const int sms = device_sms();
+    const long long nks = K / (8 * G);
+    double best = -1.0;
+    for (int wk = 1; wk <= 8; wk *= 2) {
+        for (int wr = 1; wr * wk <= 16; ++wr) {
+            const int ncw = wr * wk;
+            if (ncw < 8) continue;
+            if (g_forced.wr > 0 && wr != g_forced.wr) continue;
+            if (g_forced.wk > 0 && wk != g_forced.wk) continue;
+            TcgShape t;
+            if (!tcg_plan_smem(nt, wk, wr, K, G, &t)) continue;
+            const long long nrb = ((long long)N + 16 * wr - 1) / (16 * wr);
+            const long long rounds = (nrb + sms - 1) / sms;
+            const int lg = wk == 1 ? 0 : wk == 2 ? 1 : wk == 4 ? 2 : 3;
+            double cost = (double)rounds * wr * (1.0 + 0.25 * lg) * (ncw < 12 ? 1.25 : 1.0);
+            if (t.xt < nks) cost *= (double)rounds;
+            if (best < 0 || cost < best) {
+                best = cost;
+                *ts = t;
+                ts->gx = nrb < sms ? nrb : sms;
+            }
+        }
+    }
+    return best >= 0;
+}
+
 // ---- bulk-ring tensor-core launch shape ----------------------------------------
 // Row blocks of 16*wr rows are spread over a persistent grid of one block per
 // SM, wk = 8 / wr consumer warps split K.  A ring stage holds about 32 KB;
@@ -503,6 +576,17 @@ bool umma_shape(int M, int N, int K, int bits, int G, int dtype, bool w16, bool 
     return true;
 }
 
+// The per-group tensor-core ring for automatic plans: from 8 x rows (qmm
+// chunks up to 32), and from 4 for tall matrices.  Measured on B200 (4-bit g64
+// bf16, the 7B layer's projections, back-to-back calls): at M = 8 against the
+// tensor-core ring QKV 10.7 / 13.3 us, O 9.5 / 11.3, gate+up 26.3 / 44.1, down
+// 29.8 / 30.9; qmm M = 16..64 1.6-3x faster than the tensor-memory kernel or
+// the ring's chunks; at M = 4 gate+up 25.3 / 32.6 us, but the smaller shapes
+// stay faster on the ring below 8 rows (x is staged as 8 rows whatever M).
+bool tcg_preferred(int M, int N, int bits) {
+    return bits == 4 && M <= 32 && (M >= 8 || (M >= 4 && N >= 20000));
+}
+
 // Choose the launch shape.  Returns QMV_OK or an error (sizes too large).
 int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, bool w16, int batch, Plan* pl,
               bool s16 = true, bool gather = false, bool pair = false, bool x16 = true, bool qmm = false,
@@ -574,6 +658,20 @@ int make_plan(int fam, int M, int N, int K, int bits, int G_of_plan, int dtype, 
             pl->C = 4 * tc_unit_bytes(fi.bits) * 8 / fi.bits; pl->smem = ts.smem;
             pl->grid = dim3((unsigned)ts.gx, 1, (unsigned)batch);
             pl->block = dim3(32 * (ts.wk * ts.wr + 1), 1, 1);
+            return QMV_OK;
+        }
+    }
+
+    // ---- per-group tensor-core ring kernel (4-bit, bf16 / f16, M <= 32) --------
+    if (!gather && aff && K > 0 && (g_forced.path == 8 || (g_forced.path < 0 && tcg_preferred(M, N, bits)))) {
+        TcgShape ts;
+        if (tcg_shape(M, N, K, bits, G_of_plan, dtype, w16, s16, &ts)) {
+            pl->maxm = 8 * ts.nt; pl->R = 1; pl->wide = 1; pl->tc = 6; pl->npass = ts.nt;
+            pl->wk = ts.wk; pl->wr = ts.wr; pl->tile_iters = ts.xt; pl->sps = ts.nst; pl->pitch = ts.sby;
+            pl->spb = 1; pl->sring = 1; pl->soff = 0; pl->boff = 0; pl->sbw = 16;
+            pl->C = G_of_plan; pl->smem = ts.smem;
+            pl->grid = dim3((unsigned)ts.gx, 1, (unsigned)batch);
+            pl->block = dim3(32 * (ts.wk * ts.wr + 1), 1, 1);       // + the producer warp
             return QMV_OK;
         }
     }
@@ -814,13 +912,23 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
                        false, fes);
     if (st != QMV_OK) return st;
     // M > 8 (qmm): only the tensor-memory kernel and the tensor-core ring take it
-    if (M > QMV_MAX_M && pl.tc != 5 && pl.tc != 2) return QMV_EUNSUPPORTED;
+    if (M > QMV_MAX_M && pl.tc != 5 && pl.tc != 2 && pl.tc != 6) return QMV_EUNSUPPORTED;
     qmv::Params p{};
     if (pl.tc == 5) {
         // tensor-memory kernel: swizzled row boxes, scale / bias boxes of 8 groups
         if (!encode_rows_map_sw128(&p.wmap, w, row_bytes, N, batch, 128) ||
             !encode_scale_map(&p.smap, scales, dtype, K / G, N, batch, 8, 128) ||
             !encode_scale_map(&p.bmap, biases, dtype, K / G, N, batch, 8, 128)) {
+            cudaGetLastError();
+            return QMV_ECUDA;
+        }
+    }
+    if (pl.tc == 6) {
+        // per-group ring: swizzled 128-byte row boxes, scale / bias tiles of 8 groups
+        const int rows = 16 * pl.wr;
+        if (!encode_rows_map_sw128(&p.wmap, w, row_bytes, N, batch, rows) ||
+            !encode_scale_map(&p.smap, scales, dtype, K / G, N, batch, 8, rows) ||
+            !encode_scale_map(&p.bmap, biases, dtype, K / G, N, batch, 8, rows)) {
             cudaGetLastError();
             return QMV_ECUDA;
         }
@@ -872,6 +980,11 @@ int run(int fam, const void* x, const void* w, const void* scales, const void* b
     p.sring = pl.sring; p.soff = pl.soff; p.boff = pl.boff; p.sbw = pl.sbw;
     p.kf32 = 0x4B000000u;
     p.kbf16 = 0x43004300u;
+    if (pl.tc == 6) {
+        p.fault = fault_word();
+        if (!p.fault) return QMV_ECUDA;
+        return finish(qmv::launch_tcg_affine(dtype, G, pl.npass, p, L));
+    }
     if (pl.tc == 2) {
         p.fault = fault_word();
         if (!p.fault) return QMV_ECUDA;
@@ -944,13 +1057,24 @@ int run_pair(const void* x, const void* wg, const void* sg, const void* bg, cons
 // 32 / 64): 4096 x 4096 27.6 / 37.2 / 101 us against 38.6 / 72.0 / 139 us in
 // 16-row chunks, 4096 x 14336 67 / 127 us against 104 / 199 us; for 28672 x
 // 4096 the chunks win (96 / 189 / 375 against 140 / 274 / 473 us).
-bool qmm_prefers_umma(int N) { return g_forced.path == 7 || (g_forced.path < 0 && N <= 5120); }
+bool qmm_prefers_umma(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s16) {
+    if (g_forced.path == 7) return true;
+    if (g_forced.path >= 0 || N > 5120) return false;
+    TcgShape tg;      // the per-group tensor-core ring, where it applies, measured faster
+    return !(tcg_preferred(M > 32 ? 32 : M, N, bits) && tcg_shape(M > 32 ? 32 : M, N, K, bits, G, dtype, w16, s16, &tg));
+}
 
 // x rows per launch of qmv_qmm_affine beyond QMV_MAX_M rows: 32 or 16 when
 // the tensor-core ring kernel takes that many (x rows x groups of a
 // super-block <= 32 slot columns; more than 64 output rows), else QMV_MAX_M.
 int qmm_chunk(int M, int N, int K, int bits, int G, int dtype, bool w16, bool s16) {
     if (M <= QMV_MAX_M || N <= 64 || K <= 0) return QMV_MAX_M;
+    // the per-group tensor-core ring takes up to 32 rows a launch
+    const int c0 = M > 16 ? 32 : 16;
+    if (g_forced.path == 8 || (g_forced.path < 0 && tcg_preferred(c0, N, bits))) {
+        TcgShape tg;
+        if (tcg_shape(c0, N, K, bits, G, dtype, w16, s16, &tg)) return c0;
+    }
     for (int c : {32, 16}) {
         if (c >= M + QMV_MAX_M) continue;
         TcbShape ts;
@@ -1275,7 +1399,8 @@ int qmv_qmm_affine(const void* x, const void* w_packed, const void* scales, cons
     // rest go in chunks of QMV_MAX_M
     int chunk = QMV_MAX_M;
     if (M > QMV_MAX_M) {
-        if (qmm_prefers_umma(N)) {
+        if (qmm_prefers_umma(M, N, K, bits, group_size, dtype, aligned(w_packed, 16),
+                             aligned(scales, 16) && aligned(biases, 16))) {
             st = run(qmv::FAM_AFFINE, x, w_packed, scales, biases, nullptr, y, M, N, K, bits, group_size, dtype, 1, 1,
                      stream, nullptr, 0, true);
             if (st != QMV_EUNSUPPORTED) return st;
@@ -1415,7 +1540,7 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
     const bool qmm = M > QMV_MAX_M;
     if (qmm && fam != qmv::FAM_AFFINE) return QMV_EINVAL;
     int st = make_plan(fam, M, N, K, bits, G, dtype, w_align16 != 0, 1, &pl, true, false, false, true,
-                       qmm && qmm_prefers_umma(N), false, false, fes);
+                       qmm && qmm_prefers_umma(M, N, K, bits, G, dtype, w_align16 != 0, true), false, false, fes);
     if (st != QMV_OK) return st;
     if (qmm && pl.tc != 5) {
         // qmm: chunks of x rows, each through the qmv plan of its size
@@ -1431,7 +1556,7 @@ int qmv_describe_plan(int family, int M, int N, int K, int bits, int group_size,
     snprintf(buf, (size_t)buflen,
              "path=%s chunk=%d maxm=%d rows_per_warp=%d warps_k=%d warps_rows=%d tile_iters=%d "
              "grid=%u block=%u smem=%zu stage_sb=%d batch_sb=%d scale_ring=%d",
-             pl.tc == 5 ? "umma" : pl.tc == 4 ? "tcf" : pl.tc == 3 ? "direct" : pl.tc == 2 ? "tcb" : pl.tc ? "tc" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr,
+             pl.tc == 6 ? "tcg" : pl.tc == 5 ? "umma" : pl.tc == 4 ? "tcf" : pl.tc == 3 ? "direct" : pl.tc == 2 ? "tcb" : pl.tc ? "tc" : pl.wide ? "wide" : "narrow", pl.C, pl.maxm, pl.R, pl.wk, pl.wr,
              pl.tile_iters, pl.grid.x, pl.block.x, pl.smem, pl.sps, pl.spb, pl.sring);
     return QMV_OK;
 }

@@ -80,6 +80,12 @@ constexpr int kTcbStages = 4;
 // CUDA-core kernels with the weight ring, one bf16 x row (qmv_tcf_kernel):
 // ncw = compute warps per block in {8, 12} (plus the producer warp).
 cudaError_t launch_tcf_affine(int bits, int ncw, const Params& p, const Launch& L);
+// Per-group tensor-core ring kernels (qmv_tcg.cuh): 4-bit codes, dtype 1 (f16)
+// or 2 (bf16), G in {32, 64, 128}, nt n-tiles of 8 x rows in {1, 2, 4}
+// (qmv_inst_tcg_{f16,bf16}.cu); p.wk * p.wr consumer warps, at most 16.
+cudaError_t launch_tcg_affine(int dtype, int G, int nt, const Params& p, const Launch& L);
+cudaError_t launch_tcg_f16(int G, int nt, const Params& p, const Launch& L);
+cudaError_t launch_tcg_bf16(int G, int nt, const Params& p, const Launch& L);
 // The same ring for the block-scaled FP families (qmv_inst_tcf_fp.cu): fam one
 // of FAM_MXFP4 / NVFP4 / E2M1 / MXFP8 / E4M3 / E5M2.
 cudaError_t launch_tcf_fp(int fam, int ncw, const Params& p, const Launch& L);
