@@ -305,16 +305,20 @@ int qmv_affine_rms_norm(const void* x, const void* gamma, float eps, const void*
  * QMV_QMM_MAX_M x rows (the qmm family of MLX quantized_nax.h and of the
  * wh-iron audit, M-batched prefill).  Arguments and layouts as qmv_affine,
  * with 1 <= M <= 64 (0 allowed as a no-op).  M <= 8 is qmv_affine.  More
- * rows: for N <= 5120 with bf16 x, 16-byte aligned x, weights, scales and
- * biases, K a multiple of 64 and K / group_size a multiple of 8, ONE launch of
- * the tensor-memory kernel (tcgen05: each weight decoded once for all rows,
- * the rows are the MMA's N, K split over a thread-block cluster) when x fits
- * its shared memory; otherwise chunks of 32 or 16 rows through the
- * tensor-core ring kernel where it takes that many (x rows times groups of a
- * 128-code super-block at most 32, N > 64, 16-byte aligned weights), else
- * chunks of QMV_MAX_M, back to back on `stream` (a weight matrix that fits in
- * L2 is read from HBM once).  Every argument is checked before the first
- * launch.  Same accumulation and rounding as qmv_affine.
+ * rows, 4-bit codes with bf16 / f16 x, K a multiple of 8 groups, 16-byte
+ * aligned weights, scales and biases: chunks of 16 or 32 rows through the
+ * per-group tensor-core ring kernel (every decoded weight feeds all rows of
+ * the chunk).  Otherwise, for N <= 5120 with bf16 x, 16-byte aligned x,
+ * weights, scales and biases, K a multiple of 64 and K / group_size a
+ * multiple of 8, ONE launch of the tensor-memory kernel (tcgen05: each weight
+ * decoded once for all rows, the rows are the MMA's N, K split over a
+ * thread-block cluster) when x fits its shared memory; otherwise chunks of 32
+ * or 16 rows through the tensor-core ring kernel where it takes that many (x
+ * rows times groups of a 128-code super-block at most 32, N > 64, 16-byte
+ * aligned weights), else chunks of QMV_MAX_M.  Chunks run back to back on
+ * `stream` (a weight matrix that fits in L2 is read from HBM once).  Every
+ * argument is checked before the first launch.  Same accumulation and
+ * rounding as qmv_affine.
  */
 #define QMV_QMM_MAX_M 64
 int qmv_qmm_affine(const void* x, const void* w_packed, const void* scales, const void* biases,

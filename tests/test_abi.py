@@ -186,6 +186,50 @@ def test_block_scaled_plans():
             q.qmv_force_config()
 
 
+def _tcg_fields(plan):
+    """The per-group ring's launch fields from a plan (after any qmm chunk prefix)."""
+    tail = plan[plan.index("path=tcg "):]
+    return {k: v for k, v in (kv.split("=", 1) for kv in tail.split() if "=" in kv)}
+
+
+def test_per_group_ring_plans():
+    """4-bit affine with bf16 / f16 x takes the per-group tensor-core ring from
+    8 x rows (from 4 at N >= 20000), and qmm in chunks of 16 / 32 rows; other
+    widths, f32 x, K not a multiple of 8 groups and unaligned weights go
+    elsewhere.  Its shapes: wk in {1, 2, 4, 8}, 8..16 consumer warps plus the
+    producer, one persistent block per row block up to one per SM, shared
+    memory within the limit."""
+    plan = lambda M, N, K, **kw: q.qmv_describe_plan("affine", M, N, K, bits=kw.pop("bits", 4),
+                                                     group_size=kw.pop("g", 64), **kw)
+    for dt in ("bf16", "f16"):
+        for g in (32, 64, 128):
+            assert "path=tcg " in plan(8, 4096, 4096, g=g, dtype=dt)
+    assert "path=tcg " in plan(4, 28672, 4096)
+    assert "path=tcg " not in plan(4, 4096, 4096)
+    assert "path=tcg " not in plan(2, 28672, 4096)
+    for bits in (2, 3, 5, 6, 8):
+        assert "path=tcg " not in plan(8, 4096, 4096, bits=bits)
+    assert "path=tcg " not in plan(8, 4096, 4096, dtype="f32")
+    assert "path=tcg " not in plan(8, 4096, 1088)                  # 17 groups
+    assert "path=tcg " not in plan(8, 4096, 4096, w_align16=False)
+    assert plan(16, 4096, 4096).startswith("path=chunked16 chunks=1 path=tcg ")
+    assert plan(33, 4096, 4096).startswith("path=chunked32 chunks=2 path=tcg ")
+    assert plan(64, 28672, 4096).startswith("path=chunked32 chunks=2 path=tcg ")
+    sms = 148
+    for N, K in [(6144, 4096), (4096, 4096), (28672, 4096), (4096, 14336), (16384, 16384), (100, 1024), (2500, 14336)]:
+        for M in (8, 16, 32):
+            f = _tcg_fields(plan(M, N, K))
+            wk, wr = int(f["warps_k"]), int(f["warps_rows"])
+            assert wk in (1, 2, 4, 8) and 8 <= wk * wr <= 16, (N, K, M, f)
+            assert int(f["block"]) == 32 * (wk * wr + 1), (N, K, M, f)
+            assert int(f["grid"]) == min(-(-N // (16 * wr)), sms), (N, K, M, f)
+            assert int(f["smem"]) <= 227 * 1024, (N, K, M, f)
+            assert int(f["maxm"]) == (8 if M <= 8 else 16 if M <= 16 else 32), (N, K, M, f)
+    # the tall layer shape: one row block per SM, 13 row tiles of 16 on 138 SMs
+    f = _tcg_fields(plan(8, 28672, 4096))
+    assert (f["warps_k"], f["warps_rows"], f["grid"]) == ("1", "13", "138"), f
+
+
 def test_batched_validation():
     assert L.qmv_affine_batched(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 128, 4, 64, 2, 0, 1, None) == EINVAL
     assert L.qmv_affine_batched(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 128, 4, 64, 2, 70000, 1, None) == EINVAL
