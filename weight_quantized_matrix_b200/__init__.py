@@ -351,4 +351,9 @@ def qmv_test_skip_last_copy(enable=True):
 
 
 def qmv_force_config(path=-1, rows_per_warp=-1, warps_k=-1, warps_rows=-1):
+    """Test / benchmark knob (process-wide, not for production): pin the
+    picker's path (8 per-group tensor-core ring, 7 tcgen05, 6 CUDA-core ring,
+    5 few-rows, 4 tensor-core ring, 3 tensor cores, 1 / 0 CUDA-core wide /
+    4-byte, -1 automatic) and launch-shape fields; no arguments restores
+    automatic plans."""
     _lib.qmv_force_config(path, rows_per_warp, warps_k, warps_rows)
