@@ -673,7 +673,25 @@ def _rotation(wbytes, cap=64, least=1):
 SHAPE_SETS = ("c1", "probe", "layer", "fp_chain", "fp_probe", "formats", "sweep")
 
 
-def shape_lines(q, torch, dev, stream, flush, flush_rd, peak, sets=None):
+def alu_peak_tflops(torch, dev, sm_max_mhz):
+    """FP32 CUDA-core roof of this GPU: SMs x 128 FP32 lanes x 2 flops (FMA) x
+    the highest SM clock seen (B200: 148 x 128 x 2 x 1965 MHz = 74.4 TFLOP/s)."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = sm_max_mhz or 1965.0
+    return sms * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def alu_roof(flops, us, alu_peak):
+    """The FP32-ALU roof fields of a per-shape line (M >= 4 only): the dot
+    products' 2*M*N*K flops at the measured time, against alu_peak.  Context:
+    the tensor-core kernels do not run the products on that pipe."""
+    if not flops or not alu_peak:
+        return {}
+    tf = flops / (us * 1e-6) / 1e12
+    return {"alu_tflops": round(tf, 2), "alu_frac": round(tf / alu_peak, 4)}
+
+
+def shape_lines(q, torch, dev, stream, flush, flush_rd, peak, sets=None, alu_peak=None):
     """Throughput per format, bits and shape (the metric's breakdown), each
     line from ONE CUDA graph of R calls back to back on R weight copies that
     together exceed twice the L2 (or, for the chained FP shapes, 64 dependent
@@ -684,11 +702,13 @@ def shape_lines(q, torch, dev, stream, flush, flush_rd, peak, sets=None):
     pages' shapes), fp_probe (16384^2 in each FP format, M = 1), sweep
     (2/3/5/6-bit x group 32/64/128 x f32/f16/bf16 x M = 1, 4 at N = K = 4096)
     and formats (every Track-1 block-scaled format at N = K = 8192, M = 1
-    bf16, through qmv_block_scaled)."""
+    bf16, through qmv_block_scaled).  Each line also carries the 5th / 95th
+    percentile of its replays, and lines with M >= 4 the FP32-ALU roof: 2*M*N*K
+    flops per call against alu_peak (TFLOP/s)."""
     lines = []
     sets = sets or SHAPE_SETS
 
-    def timed(tag, label, R, launch, nbytes, plan, reps=5):
+    def timed(tag, label, R, launch, nbytes, plan, reps=7, flops=None):
         for r in range(R):                          # eager warm-up (kernel attributes)
             launch(r)
         g = torch.cuda.CUDAGraph()
@@ -704,11 +724,14 @@ def shape_lines(q, torch, dev, stream, flush, flush_rd, peak, sets=None):
             g.replay()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
-        ms = float(np.median([a.elapsed_time(b) for a, b in ev]))
-        us = ms * 1e3 / R
+        per = np.array([a.elapsed_time(b) for a, b in ev]) * 1e3 / R      # us per call, each replay
+        us = float(np.median(per))
         gbs = nbytes / (us * 1e-6) / 1e9
-        lines.append({"set": tag, "shape": label, "us_per_call": round(us, 3), "GB_s": round(gbs, 1),
-                      "frac_of_hbm": round(gbs / peak, 4), "calls_per_graph": R, "plan": plan})
+        line = {"set": tag, "shape": label, "us_per_call": round(us, 3), "us_p5": round(float(np.percentile(per, 5)), 3),
+                "us_p95": round(float(np.percentile(per, 95)), 3), "GB_s": round(gbs, 1),
+                "frac_of_hbm": round(gbs / peak, 4), "calls_per_graph": R, "plan": plan}
+        line.update(alu_roof(flops, us, alu_peak))
+        lines.append(line)
         del g
 
     def affine(tag, label, M, N, K, bits, G, dtype, least=1, cap=64):
@@ -723,7 +746,7 @@ def shape_lines(q, torch, dev, stream, flush, flush_rd, peak, sets=None):
             w, sc, bi = ws[r]
             q.qmv_affine(x, w, sc, bi, y, M, N, K, bits, G, dtype)
         timed(tag, label, R, launch, affine_bytes(M, N, K, bits, G, DT_BYTES[dtype]),
-              q.qmv_describe_plan("affine", M, N, K, bits, G, dtype))
+              q.qmv_describe_plan("affine", M, N, K, bits, G, dtype), flops=2 * M * N * K if M >= 4 else None)
 
     with torch.cuda.stream(stream):
         if "c1" in sets:
@@ -893,7 +916,7 @@ def run_ours(args, rank, world, local_rank):
                 gs[r % len(gs)].replay()
                 ev[r][1].record(stream)
             torch.cuda.synchronize()
-            per_group.append(float(np.mean([a.elapsed_time(b) for a, b in ev])))   # ms per group replay
+            per_group.append(np.array([a.elapsed_time(b) for a, b in ev]))   # ms per group replay
         del step_graphs, group_graphs
 
     tot_ms, tot_ms_e2e = max_over_ranks([float(step_ms.sum()), float(step_ms_e2e.sum())], world, dev)
@@ -904,16 +927,21 @@ def run_ours(args, rank, world, local_rank):
     # per-shape results and the dominant kernel (largest share of device time)
     shapes, by_kernel = [], {}
     peak, peak_kind = peaks()
+    alu_peak = alu_peak_tflops(torch, dev, (clocks or {}).get("sm_max_mhz"))
     for gi, (label, s) in enumerate(groups):
-        ms = float(per_group[gi])
+        ms = float(np.mean(per_group[gi]))
         n = wl.calls_per_step // len(groups)        # calls per group replay
         b = wl.group_bytes(s)
         plan = wl.group_plan(s)
         kern = " ".join(w for w in plan.split() if w.split("=")[0] in ("path", "chunk", "maxm", "rows_per_warp"))
         gbs = b / (ms * 1e-3) / 1e9
-        shapes.append({"set": args.workload, "shape": label, "us_per_call": round(ms * 1e3 / n, 3),
-                       "GB_s": round(gbs, 1),
-                       "frac_of_hbm": round(gbs / peak, 4), "plan": plan})
+        line = {"set": args.workload, "shape": label, "us_per_call": round(ms * 1e3 / n, 3),
+                "us_p5": round(float(np.percentile(per_group[gi], 5)) * 1e3 / n, 3),
+                "us_p95": round(float(np.percentile(per_group[gi], 95)) * 1e3 / n, 3),
+                "GB_s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4), "plan": plan}
+        if isinstance(s, dict) and s.get("M", 0) >= 4 and "N" in s and "K" in s:
+            line.update(alu_roof(2 * s["M"] * s["N"] * s["K"] * n, ms * 1e3, alu_peak))
+        shapes.append(line)
         k = by_kernel.setdefault(kern, {"ms": 0.0, "launches": 0, "bytes": 0})
         k["ms"] += ms; k["launches"] += n; k["bytes"] += b
     dom_plan, dom = max(by_kernel.items(), key=lambda kv: kv[1]["ms"])
@@ -933,11 +961,15 @@ def run_ours(args, rank, world, local_rank):
                      "kernel": dom_plan, "kernel_share": round(dom["ms"] / sum(v["ms"] for v in by_kernel.values()), 3),
                      "bytes_per_launch": dom["bytes"] // max(1, dom["launches"]),
                      "avg_launch_us": round(dom["ms"] * 1e3 / max(1, dom["launches"]), 3)},
+        "spread": {"unit": "us/call", "over": f"{args.steps} timed steps, this rank",
+                   "p5": round(float(np.percentile(step_ms, 5)) * 1e3 / wl.calls_per_step, 4),
+                   "p50": round(float(np.percentile(step_ms, 50)) * 1e3 / wl.calls_per_step, 4),
+                   "p95": round(float(np.percentile(step_ms, 95)) * 1e3 / wl.calls_per_step, 4)},
         "clocks": clocks, "shapes": shapes, "wall_s_timed": round(wall, 3),
     }
     if args.workload == "chain8" and not args.no_shapes:
         # the metric's breakdown per format / bits / shape; not part of `value`
-        out["shapes"] += shape_lines(q, torch, dev, stream, flush, flush_rd, peak, args.sets)
+        out["shapes"] += shape_lines(q, torch, dev, stream, flush, flush_rd, peak, args.sets, alu_peak)
     if rank == 0:
         out["cpu_baseline"] = (cpu_baseline(args.workload) if not args.no_cpu_baseline
                                else {"value": None, "unit": "us/call", "kind": "oracle",

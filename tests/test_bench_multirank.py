@@ -57,3 +57,18 @@ def test_max_over_ranks_single_rank_is_identity():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks([1.5, 2], 1, "cpu") == [1.5, 2.0]
+
+
+def test_alu_roof_fields():
+    """The FP32-ALU roof of the per-shape lines: SMs x 128 lanes x 2 flops x
+    the SM clock; a line's fraction is its 2*M*N*K flops over its time."""
+    import types
+    import bench
+    fake = types.SimpleNamespace(cuda=types.SimpleNamespace(
+        get_device_properties=lambda dev: types.SimpleNamespace(multi_processor_count=148)))
+    peak = bench.alu_peak_tflops(fake, 0, 1965.0)
+    assert abs(peak - 148 * 128 * 2 * 1965e6 / 1e12) < 1e-9
+    assert abs(bench.alu_peak_tflops(fake, 0, None) - peak) < 1e-9      # no clock sample: the boost clock
+    r = bench.alu_roof(2 * 8 * 4096 * 4096, 10.0, peak)                   # 268 Mflop in 10 us
+    assert abs(r["alu_tflops"] - 26.84) < 0.01 and abs(r["alu_frac"] - 26.8435 / peak) < 1e-3
+    assert bench.alu_roof(None, 10.0, peak) == {} and bench.alu_roof(1e9, 10.0, None) == {}
